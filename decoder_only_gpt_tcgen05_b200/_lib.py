@@ -1,0 +1,61 @@
+"""ctypes loader for libgpt_b200.so: argument marshalling only.
+
+Every call goes straight to the C ABI declared in include/gpt.h and
+include/gpt_ops.h; there is no Python or CPU fallback.  If the library has not
+been built, importing the binding raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgpt_b200.so")
+
+_lib = None
+
+
+class GptError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"gpt status {code}: {msg}")
+        self.code = code
+
+
+_P = C.c_void_p
+_I = C.c_int
+_LL = C.c_longlong
+_F = C.c_float
+
+# name -> argument types (restype is int for all but gpt_last_error)
+SIGNATURES = {
+    "gpt_op_gemm": [_I, _I, _P, _LL, _I, _P, _LL, _I, _I, _I, _I, _P, _LL, _P, _I, _P],
+    "gpt_op_attention_fwd": [_P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P],
+    "gpt_op_attention_bwd": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P],
+}
+
+
+def lib():
+    """The loaded library (loaded on first use)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m decoder_only_gpt_tcgen05_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        L.gpt_last_error.restype = C.c_char_p
+        L.gpt_last_error.argtypes = []
+        for name, args in SIGNATURES.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def check(rc: int) -> None:
+    if rc != 0:
+        raise GptError(rc, lib().gpt_last_error().decode())
+
+
+def call(name: str, *args) -> None:
+    check(getattr(lib(), name)(*args))

@@ -1,0 +1,840 @@
+// Causal flash attention for sm_100a: forward and backward on tcgen05 tensor cores.
+//
+// softmax(Q K^T / sqrt(hd) + causal mask) V  ("nanoGPT" wiki page, CausalSelfAttention:
+// the explicit mask blocks attention to future tokens), computed tile by tile with an
+// online softmax so the T x T score matrix never leaves the SM.
+//
+// Layout: q, k, v live in one bf16 buffer [B*T, 3, H, hdp] (hdp = head dim padded to 64 or
+// 128, padding zero); each (b, h) slice is read with 3-D TMA boxes {64 features, rows, 1}
+// under 128-byte swizzle, so rows past the end of a sequence arrive as zeros.
+//
+// Forward (one CTA per 128-query tile of one (b, h); heaviest causal tiles launched first):
+//   warp 0      TMA: Q once, then K_j and V_j through a 2-deep ring
+//   warp 1      one thread issues S_j = Q K_j^T into a double-buffered TMEM tile, then
+//               O += P_{j-1} V_{j-1} (P from shared memory, O accumulating in TMEM)
+//   warps 2..5  softmax, one query row per thread: row max and sum in registers, P = exp2(...)
+//               written to shared memory in the MMA operand layout; O is rescaled in TMEM
+//               only when the running max grows by more than 2^8 (otherwise the stale max
+//               stays exact because O and l use the same one)
+// Backward: delta = rowsum(dO * O) (kernels.cu), then
+//   dK/dV kernel: one CTA per 128-key tile, stepping over 64-query tiles:
+//               S^T = K Q^T, dP^T = V dO^T (TMEM, double buffered), P^T and dS^T to shared
+//               memory, dV += P^T dO, dK += dS^T Q (accumulating in TMEM)
+//   dQ kernel:  one CTA per 128-query tile, stepping over 64-key tiles:
+//               S = Q K^T, dP = dO V^T, dS to shared memory, dQ += dS K
+// Both are deterministic (no atomics).  Every wait is bounded (see ptx.cuh).
+#include <cmath>
+
+#include "host.cuh"
+#include "kernels.cuh"
+
+namespace gptk {
+
+static constexpr float kLog2e = 1.4426950408889634f;
+
+// Row r, columns [c0, c0 + 8) of a K-major, 128-byte-swizzled bf16 tile whose rows are 128 bytes:
+// byte offset of the 16-byte unit holding them.
+__device__ __forceinline__ uint32_t sw128_off(int r, int unit) { return r * 128 + ((unit ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// ====================================================================== forward
+
+template <int HD>
+struct FwdSmem {
+  static constexpr int TILE = HD * 256;  // 128 rows x HD bf16
+  static constexpr int Q = 0;
+  static constexpr int K0 = Q + TILE;
+  static constexpr int V0 = K0 + 2 * TILE;
+  static constexpr int P = V0 + 2 * TILE;
+  static constexpr int BAR = P + 32768;
+  static constexpr int BYTES = BAR + 256 + 1024;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnShape s, __nv_bfloat16* __restrict__ o,
+                    long long ldo, float* __restrict__ lse_out, float scale_log2, DevCtl ctl) {
+  using L = FwdSmem<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+  uint64_t* bar_q = bars + 0;
+  uint64_t* k_full = bars + 1;   // [2]
+  uint64_t* k_empty = bars + 3;  // [2]
+  uint64_t* v_full = bars + 5;   // [2]
+  uint64_t* v_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;   // [2]
+  uint64_t* s_free = bars + 11;  // [2]
+  uint64_t* p_full = bars + 13;
+  uint64_t* p_empty = bars + 14;
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = gridDim.x;
+  const int qt = n_qt - 1 - blockIdx.x;  // heaviest first
+  const int bh = blockIdx.y;
+  const int b = bh / s.H, h = bh % s.H;
+  const int q0 = qt * 128;
+  const int n_kv = qt + 1;
+  constexpr int NCH = HD / 64;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(p_empty, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_qkv);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tS = tbase;        // 2 x 128 columns
+  const uint32_t tO = tbase + 256;  // HD columns
+
+  const int colq = h * s.hdp;
+  const int colk = s.H * s.hdp + h * s.hdp;
+  const int colv = 2 * s.H * s.hdp + h * s.hdp;
+
+  if (warp == 0 && lane == 0) {
+    bool ok = true;
+    mbar_expect_tx(bar_q, L::TILE);
+    for (int c = 0; c < NCH; ++c) tma_load_3d(sm + L::Q + c * 16384, &tm_qkv, bar_q, colq + 64 * c, q0, b);
+    int issued_k = -1, issued_v = -1;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int st = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      if (!mbar_wait(&k_empty[st], ph ^ 1u, ctl, abort_flag, 20)) { ok = false; break; }
+      mbar_expect_tx(&k_full[st], L::TILE);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_3d(sm + L::K0 + st * L::TILE + c * 16384, &tm_qkv, &k_full[st], colk + 64 * c, j * 128, b);
+      issued_k = j;
+      if (!mbar_wait(&v_empty[st], ph ^ 1u, ctl, abort_flag, 21)) { ok = false; break; }
+      mbar_expect_tx(&v_full[st], L::TILE);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_3d(sm + L::V0 + st * L::TILE + c * 16384, &tm_qkv, &v_full[st], colv + 64 * c, j * 128, b);
+      issued_v = j;
+    }
+    if (!ok) {
+      // wait (bounded) for the copies still in flight
+      volatile int never = 0;
+      mbar_wait(bar_q, 0, ctl, &never, 22);
+      for (int j = (issued_k > 0 ? issued_k - 1 : 0); j <= issued_k; ++j)
+        mbar_wait(&k_full[j & 1], (j >> 1) & 1, ctl, &never, 22);
+      for (int j = (issued_v > 0 ? issued_v - 1 : 0); j <= issued_v && issued_v >= 0; ++j)
+        mbar_wait(&v_full[j & 1], (j >> 1) & 1, ctl, &never, 22);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t idesc_o = idesc_bf16(128, HD, 0, 1);
+    bool ok = mbar_wait(bar_q, 0, ctl, abort_flag, 23);
+    bool issued = false;
+    const uint32_t sQ = smem_u32(sm + L::Q);
+    const uint32_t sP = smem_u32(sm + L::P);
+    for (int j = 0; j <= n_kv && ok; ++j) {
+      if (j < n_kv) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&k_full[st], ph, ctl, abort_flag, 24)) { ok = false; break; }
+        if (!mbar_wait(&s_free[st], ph ^ 1u, ctl, abort_flag, 25)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + L::K0 + st * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tS + st * 128, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), idesc_s,
+                    kk > 0);
+        }
+        umma_commit(&s_full[st]);
+        umma_commit(&k_empty[st]);
+        issued = true;
+      }
+      if (j >= 1) {
+        const int jj = j - 1;
+        const int st = jj & 1;
+        if (!mbar_wait(p_full, jj & 1, ctl, abort_flag, 26)) { ok = false; break; }
+        if (!mbar_wait(&v_full[st], (jj >> 1) & 1, ctl, abort_flag, 27)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sV = smem_u32(sm + L::V0 + st * L::TILE);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          umma_bf16(tO, sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    sdesc_sw128(sV + kk * 2048, 16384, 1024), idesc_o, (jj | kk) != 0);
+        }
+        umma_commit(p_empty);
+        umma_commit(&v_empty[st]);
+        issued = true;
+      }
+    }
+    if (!ok && issued) {
+      volatile int never = 0;
+      umma_commit(drain);
+      mbar_wait(drain, 0, ctl, &never, 28);
+    }
+  } else if (warp >= 2) {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qi = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sP = smem_u32(sm + L::P);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&s_full[st], (j >> 1) & 1, ctl, abort_flag, 29)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tSrow = tS + st * 128 + lane_off;
+      const int kbase = j * 128;
+      const bool diag = (j == n_kv - 1);
+      // pass 1: row max of the (masked) scores
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(tSrow + c * 32, sv);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int key = kbase + c * 32 + e;
+          if (!diag || (key <= qi && key < s.T)) mx = fmaxf(mx, sv[e]);
+        }
+      }
+      mx *= scale_log2;
+      const float m_new = fmaxf(m, mx);
+      float alpha = 1.f;
+      if (m_new > m + 8.f) {
+        alpha = ex2_approx(m - m_new);
+        m = m_new;
+      }
+      if (j > 0) {
+        // O and the P buffer are still in use by the previous P V product
+        if (!mbar_wait(p_empty, (j - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < HD / 32; ++c) {
+            float ov[32];
+            tmem_ld32(tO + lane_off + c * 32, ov);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(tO + lane_off + c * 32, ov);
+          }
+        }
+      }
+      // pass 2: P = exp2(s * scale - m) -> shared memory (K-major, 128-byte swizzle;
+      // keys 0..63 in chunk 0, 64..127 in chunk 1), row sum in registers
+      float rs = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float sv[32];
+        tmem_ld32(tSrow + c * 32, sv);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int key = kbase + c * 32 + e;
+          const bool valid = !diag || (key <= qi && key < s.T);
+          sv[e] = valid ? ex2_approx(fmaf(sv[e], scale_log2, -m)) : 0.f;
+          rs += sv[e];
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int gg = c * 4 + g;
+          uint4 w;
+          w.x = pack_bf16x2(sv[8 * g + 0], sv[8 * g + 1]);
+          w.y = pack_bf16x2(sv[8 * g + 2], sv[8 * g + 3]);
+          w.z = pack_bf16x2(sv[8 * g + 4], sv[8 * g + 5]);
+          w.w = pack_bf16x2(sv[8 * g + 6], sv[8 * g + 7]);
+          st_shared_v4(sP + (gg >> 3) * 16384 + sw128_off(r, gg & 7), w);
+        }
+      }
+      l = l * alpha + rs;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && mbar_wait(p_empty, (n_kv - 1) & 1, ctl, abort_flag, 31)) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool row_ok = qi < s.T;
+      __nv_bfloat16* orow = o + ((long long)b * s.T + qi) * ldo + (long long)h * s.hd;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float ov[32];
+        tmem_ld32(tO + lane_off + c * 32, ov);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] *= inv_l;
+        if (row_ok) {
+          if (s.hd == HD) {
+            uint4* d = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int g = 0; g < 4; ++g)
+              d[g] = make_uint4(pack_bf16x2(ov[8 * g], ov[8 * g + 1]), pack_bf16x2(ov[8 * g + 2], ov[8 * g + 3]),
+                                pack_bf16x2(ov[8 * g + 4], ov[8 * g + 5]), pack_bf16x2(ov[8 * g + 6], ov[8 * g + 7]));
+          } else {
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e < s.hd) orow[c * 32 + e] = __float2bfloat16_rn(ov[e]);
+          }
+        }
+      }
+      if (row_ok) lse_out[(long long)bh * s.T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ====================================================================== backward: dK, dV
+
+template <int HD>
+struct DkvSmem {
+  static constexpr int KV_TILE = HD * 256;  // 128 rows
+  static constexpr int Q_TILE = HD * 128;   // 64 rows
+  static constexpr int K = 0;
+  static constexpr int V = K + KV_TILE;
+  static constexpr int Q0 = V + KV_TILE;          // [2]
+  static constexpr int DO0 = Q0 + 2 * Q_TILE;     // [2]
+  static constexpr int P = DO0 + 2 * Q_TILE;      // 128 keys x 64 queries bf16 = 16 KB
+  static constexpr int DS = P + 16384;
+  static constexpr int BAR = DS + 16384;
+  static constexpr int BYTES = BAR + 256 + 1024;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q64,
+                        const __grid_constant__ CUtensorMap tm_do64, const AttnShape s, const float* __restrict__ lse,
+                        const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, float scale_log2,
+                        float scale, DevCtl ctl) {
+  using L = DkvSmem<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;    // [2]
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* pd_full = bars + 9;
+  uint64_t* pd_empty = bars + 10;
+  uint64_t* acc_full = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / s.H, h = bh % s.H;
+  const int k0 = kt * 128;
+  const int n_q64 = (s.T + 63) / 64;
+  const int i0 = 2 * kt;
+  const int n_it = n_q64 - i0;
+  constexpr int NCH = HD / 64;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+    }
+    mbar_init(pd_full, 4);
+    mbar_init(pd_empty, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tS = tbase;         // [2] x 64
+  const uint32_t tdP = tbase + 128;  // [2] x 64
+  const uint32_t tdV = tbase + 256;
+  const uint32_t tdK = tbase + 384;
+
+  const int colq = h * s.hdp;
+  const int colk = s.H * s.hdp + h * s.hdp;
+  const int colv = 2 * s.H * s.hdp + h * s.hdp;
+  const int cold = h * s.hdp;
+
+  if (warp == 0 && lane == 0) {
+    bool ok = true;
+    mbar_expect_tx(kv_full, 2 * L::KV_TILE);
+    for (int c = 0; c < NCH; ++c) {
+      tma_load_3d(sm + L::K + c * 16384, &tm_kv128, kv_full, colk + 64 * c, k0, b);
+      tma_load_3d(sm + L::V + c * 16384, &tm_kv128, kv_full, colv + 64 * c, k0, b);
+    }
+    int issued = -1;
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int st = it & 1;
+      if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
+      const int qb = (i0 + it) * 64;
+      mbar_expect_tx(&q_full[st], 2 * L::Q_TILE);
+      for (int c = 0; c < NCH; ++c) {
+        tma_load_3d(sm + L::Q0 + st * L::Q_TILE + c * 8192, &tm_q64, &q_full[st], colq + 64 * c, qb, b);
+        tma_load_3d(sm + L::DO0 + st * L::Q_TILE + c * 8192, &tm_do64, &q_full[st], cold + 64 * c, qb, b);
+      }
+      issued = it;
+    }
+    if (!ok) {
+      volatile int never = 0;
+      mbar_wait(kv_full, 0, ctl, &never, 41);
+      for (int it = (issued > 0 ? issued - 1 : 0); it <= issued && issued >= 0; ++it)
+        mbar_wait(&q_full[it & 1], (it >> 1) & 1, ctl, &never, 41);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
+    constexpr uint32_t idesc_acc = idesc_bf16(128, HD, 0, 1);
+    bool ok = mbar_wait(kv_full, 0, ctl, abort_flag, 42);
+    bool issued = false;
+    const uint32_t sK = smem_u32(sm + L::K), sV = smem_u32(sm + L::V);
+    const uint32_t sP = smem_u32(sm + L::P), sDS = smem_u32(sm + L::DS);
+    for (int it = 0; it <= n_it && ok; ++it) {
+      if (it < n_it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        if (!mbar_wait(&q_full[st], ph, ctl, abort_flag, 43)) { ok = false; break; }
+        if (!mbar_wait(&s_free[st], ph ^ 1u, ctl, abort_flag, 44)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(sm + L::Q0 + st * L::Q_TILE);
+        const uint32_t sD = smem_u32(sm + L::DO0 + st * L::Q_TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_bf16(tS + st * 64, sdesc_sw128(sK + offa, 16, 1024), sdesc_sw128(sQ + offb, 16, 1024), idesc_s, kk > 0);
+          umma_bf16(tdP + st * 64, sdesc_sw128(sV + offa, 16, 1024), sdesc_sw128(sD + offb, 16, 1024), idesc_s,
+                    kk > 0);
+        }
+        umma_commit(&s_full[st]);
+        issued = true;
+      }
+      if (it >= 1) {
+        const int jt = it - 1;
+        const int st = jt & 1;
+        if (!mbar_wait(pd_full, jt & 1, ctl, abort_flag, 45)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(sm + L::Q0 + st * L::Q_TILE);
+        const uint32_t sD = smem_u32(sm + L::DO0 + st * L::Q_TILE);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_bf16(tdV, sdesc_sw128(sP + kk * 32, 16, 1024), sdesc_sw128(sD + kk * 2048, 8192, 1024), idesc_acc,
+                    (jt | kk) != 0);
+          umma_bf16(tdK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc,
+                    (jt | kk) != 0);
+        }
+        umma_commit(pd_empty);
+        umma_commit(&q_empty[st]);
+        issued = true;
+      }
+    }
+    if (ok) {
+      umma_commit(acc_full);
+    } else if (issued) {
+      volatile int never = 0;
+      umma_commit(drain);
+      mbar_wait(drain, 0, ctl, &never, 46);
+    }
+  } else if (warp >= 2) {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // key row within the tile
+    const int key = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sP = smem_u32(sm + L::P), sDS = smem_u32(sm + L::DS);
+    const float* lse_bh = lse + (long long)bh * s.T;
+    const float* del_bh = delta + (long long)bh * s.T;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int st = it & 1;
+      const int qb = (i0 + it) * 64;
+      if (!mbar_wait(&s_full[st], (it >> 1) & 1, ctl, abort_flag, 47)) { ok = false; break; }
+      if (it > 0 && !mbar_wait(pd_empty, (it - 1) & 1, ctl, abort_flag, 48)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float sv[32], dp[32];
+        tmem_ld32(tS + st * 64 + lane_off + c * 32, sv);
+        tmem_ld32(tdP + st * 64 + lane_off + c * 32, dp);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          // per-query statistics: every lane reads the same address (a broadcast load)
+          const int q = qb + 32 * c + e;
+          const bool valid = (q >= key) && (q < s.T);
+          const float l2 = valid ? __ldg(lse_bh + q) * kLog2e : 0.f;
+          const float dl = valid ? __ldg(del_bh + q) : 0.f;
+          const float p = valid ? ex2_approx(fmaf(sv[e], scale_log2, -l2)) : 0.f;
+          sv[e] = p;
+          dp[e] = p * (dp[e] - dl);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int unit = 4 * c + g;
+          uint4 w = make_uint4(pack_bf16x2(sv[8 * g], sv[8 * g + 1]), pack_bf16x2(sv[8 * g + 2], sv[8 * g + 3]),
+                               pack_bf16x2(sv[8 * g + 4], sv[8 * g + 5]), pack_bf16x2(sv[8 * g + 6], sv[8 * g + 7]));
+          st_shared_v4(sP + sw128_off(r, unit), w);
+          uint4 x = make_uint4(pack_bf16x2(dp[8 * g], dp[8 * g + 1]), pack_bf16x2(dp[8 * g + 2], dp[8 * g + 3]),
+                               pack_bf16x2(dp[8 * g + 4], dp[8 * g + 5]), pack_bf16x2(dp[8 * g + 6], dp[8 * g + 7]));
+          st_shared_v4(sDS + sw128_off(r, unit), x);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[st]);
+        mbar_arrive(pd_full);
+      }
+    }
+    if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 49)) {
+      tc_fence_after();
+      const bool row_ok = key < s.T;
+      const long long m = (long long)b * s.T + key;
+      __nv_bfloat16* dk = dqkv + m * s.ld_qkv + (long long)s.H * s.hdp + (long long)h * s.hdp;
+      __nv_bfloat16* dv = dqkv + m * s.ld_qkv + 2LL * s.H * s.hdp + (long long)h * s.hdp;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float a[32], bb[32];
+        tmem_ld32(tdK + lane_off + c * 32, a);
+        tmem_ld32(tdV + lane_off + c * 32, bb);
+        if (row_ok) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            reinterpret_cast<uint4*>(dk + c * 32)[g] =
+                make_uint4(pack_bf16x2(a[8 * g] * scale, a[8 * g + 1] * scale),
+                           pack_bf16x2(a[8 * g + 2] * scale, a[8 * g + 3] * scale),
+                           pack_bf16x2(a[8 * g + 4] * scale, a[8 * g + 5] * scale),
+                           pack_bf16x2(a[8 * g + 6] * scale, a[8 * g + 7] * scale));
+            reinterpret_cast<uint4*>(dv + c * 32)[g] =
+                make_uint4(pack_bf16x2(bb[8 * g], bb[8 * g + 1]), pack_bf16x2(bb[8 * g + 2], bb[8 * g + 3]),
+                           pack_bf16x2(bb[8 * g + 4], bb[8 * g + 5]), pack_bf16x2(bb[8 * g + 6], bb[8 * g + 7]));
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ====================================================================== backward: dQ
+
+template <int HD>
+struct DqSmem {
+  static constexpr int Q_TILE = HD * 256;   // 128 rows
+  static constexpr int KV_TILE = HD * 128;  // 64 rows
+  static constexpr int Q = 0;
+  static constexpr int DO = Q + Q_TILE;
+  static constexpr int K0 = DO + Q_TILE;         // [2]
+  static constexpr int V0 = K0 + 2 * KV_TILE;    // [2]
+  static constexpr int DS = V0 + 2 * KV_TILE;    // 128 queries x 64 keys bf16 = 16 KB
+  static constexpr int BAR = DS + 16384;
+  static constexpr int BYTES = BAR + 256 + 1024;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
+                       const __grid_constant__ CUtensorMap tm_kv64, const AttnShape s, const float* __restrict__ lse,
+                       const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, float scale_log2,
+                       float scale, DevCtl ctl) {
+  using L = DqSmem<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [2]
+  uint64_t* kv_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* ds_full = bars + 9;
+  uint64_t* ds_empty = bars + 10;
+  uint64_t* acc_full = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = gridDim.x;
+  const int qt = n_qt - 1 - blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / s.H, h = bh % s.H;
+  const int q0 = qt * 128;
+  const int kend = min(q0 + 128, s.T);
+  const int n_kv = (kend + 63) / 64;
+  constexpr int NCH = HD / 64;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+    }
+    mbar_init(ds_full, 4);
+    mbar_init(ds_empty, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t tS = tbase;         // [2] x 64
+  const uint32_t tdP = tbase + 128;  // [2] x 64
+  const uint32_t tdQ = tbase + 256;
+
+  const int colq = h * s.hdp;
+  const int colk = s.H * s.hdp + h * s.hdp;
+  const int colv = 2 * s.H * s.hdp + h * s.hdp;
+  const int cold = h * s.hdp;
+
+  if (warp == 0 && lane == 0) {
+    bool ok = true;
+    mbar_expect_tx(q_full, 2 * L::Q_TILE);
+    for (int c = 0; c < NCH; ++c) {
+      tma_load_3d(sm + L::Q + c * 16384, &tm_q128, q_full, colq + 64 * c, q0, b);
+      tma_load_3d(sm + L::DO + c * 16384, &tm_do128, q_full, cold + 64 * c, q0, b);
+    }
+    int issued = -1;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
+      mbar_expect_tx(&kv_full[st], 2 * L::KV_TILE);
+      for (int c = 0; c < NCH; ++c) {
+        tma_load_3d(sm + L::K0 + st * L::KV_TILE + c * 8192, &tm_kv64, &kv_full[st], colk + 64 * c, j * 64, b);
+        tma_load_3d(sm + L::V0 + st * L::KV_TILE + c * 8192, &tm_kv64, &kv_full[st], colv + 64 * c, j * 64, b);
+      }
+      issued = j;
+    }
+    if (!ok) {
+      volatile int never = 0;
+      mbar_wait(q_full, 0, ctl, &never, 61);
+      for (int j = (issued > 0 ? issued - 1 : 0); j <= issued && issued >= 0; ++j)
+        mbar_wait(&kv_full[j & 1], (j >> 1) & 1, ctl, &never, 61);
+    }
+  } else if (warp == 1 && lane == 0) {
+    constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
+    constexpr uint32_t idesc_acc = idesc_bf16(128, HD, 0, 1);
+    bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 62);
+    bool issued = false;
+    const uint32_t sQ = smem_u32(sm + L::Q), sD = smem_u32(sm + L::DO), sDS = smem_u32(sm + L::DS);
+    for (int j = 0; j <= n_kv && ok; ++j) {
+      if (j < n_kv) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&kv_full[st], ph, ctl, abort_flag, 63)) { ok = false; break; }
+        if (!mbar_wait(&s_free[st], ph ^ 1u, ctl, abort_flag, 64)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + L::K0 + st * L::KV_TILE);
+        const uint32_t sV = smem_u32(sm + L::V0 + st * L::KV_TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_bf16(tS + st * 64, sdesc_sw128(sQ + offa, 16, 1024), sdesc_sw128(sK + offb, 16, 1024), idesc_s, kk > 0);
+          umma_bf16(tdP + st * 64, sdesc_sw128(sD + offa, 16, 1024), sdesc_sw128(sV + offb, 16, 1024), idesc_s,
+                    kk > 0);
+        }
+        umma_commit(&s_full[st]);
+        issued = true;
+      }
+      if (j >= 1) {
+        const int jj = j - 1;
+        const int st = jj & 1;
+        if (!mbar_wait(ds_full, jj & 1, ctl, abort_flag, 65)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + L::K0 + st * L::KV_TILE);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tdQ, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sK + kk * 2048, 8192, 1024), idesc_acc,
+                    (jj | kk) != 0);
+        umma_commit(ds_empty);
+        umma_commit(&kv_empty[st]);
+        issued = true;
+      }
+    }
+    if (ok) {
+      umma_commit(acc_full);
+    } else if (issued) {
+      volatile int never = 0;
+      umma_commit(drain);
+      mbar_wait(drain, 0, ctl, &never, 66);
+    }
+  } else if (warp >= 2) {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qi = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t sDS = smem_u32(sm + L::DS);
+    const bool row_ok = qi < s.T;
+    const float lse2 = row_ok ? lse[(long long)bh * s.T + qi] * kLog2e : 0.f;
+    const float dl = row_ok ? delta[(long long)bh * s.T + qi] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(&s_full[st], (j >> 1) & 1, ctl, abort_flag, 67)) { ok = false; break; }
+      if (j > 0 && !mbar_wait(ds_empty, (j - 1) & 1, ctl, abort_flag, 68)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        float sv[32], dp[32];
+        tmem_ld32(tS + st * 64 + lane_off + c * 32, sv);
+        tmem_ld32(tdP + st * 64 + lane_off + c * 32, dp);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int key = j * 64 + 32 * c + e;
+          const bool valid = row_ok && key <= qi && key < s.T;
+          const float p = valid ? ex2_approx(fmaf(sv[e], scale_log2, -lse2)) : 0.f;
+          dp[e] = p * (dp[e] - dl);
+        }
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 x = make_uint4(pack_bf16x2(dp[8 * g], dp[8 * g + 1]), pack_bf16x2(dp[8 * g + 2], dp[8 * g + 3]),
+                               pack_bf16x2(dp[8 * g + 4], dp[8 * g + 5]), pack_bf16x2(dp[8 * g + 6], dp[8 * g + 7]));
+          st_shared_v4(sDS + sw128_off(r, 4 * c + g), x);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[st]);
+        mbar_arrive(ds_full);
+      }
+    }
+    if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 69)) {
+      tc_fence_after();
+      __nv_bfloat16* dq = dqkv + ((long long)b * s.T + qi) * s.ld_qkv + (long long)h * s.hdp;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float a[32];
+        tmem_ld32(tdQ + lane_off + c * 32, a);
+        if (row_ok) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            reinterpret_cast<uint4*>(dq + c * 32)[g] = make_uint4(
+                pack_bf16x2(a[8 * g] * scale, a[8 * g + 1] * scale), pack_bf16x2(a[8 * g + 2] * scale, a[8 * g + 3] * scale),
+                pack_bf16x2(a[8 * g + 4] * scale, a[8 * g + 5] * scale),
+                pack_bf16x2(a[8 * g + 6] * scale, a[8 * g + 7] * scale));
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ====================================================================== launchers
+
+template <int HD>
+static int attn_fwd_t(const __nv_bfloat16* qkv, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
+                      cudaStream_t st) {
+  using L = FwdSmem<HD>;
+  CUtensorMap tm;
+  GPTK_TRY(make_tmap_3d(&tm, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
+  GPTK_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
+  const float scale_log2 = kLog2e / sqrtf((float)s.hd);
+  dim3 grid((s.T + 127) / 128, s.B * s.H);
+  attn_fwd_kernel<HD><<<grid, 192, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+int launch_attn_fwd(const __nv_bfloat16* qkv_pad, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
+                    cudaStream_t st) {
+  if (s.B < 1 || s.T < 1 || s.H < 1) return set_error(ST_INVALID_ARG, "attention: empty shape");
+  if (s.B * s.H > 65535) return set_error(ST_UNSUPPORTED, "attention: B*H above 65535");
+  if (s.hdp == 64) return attn_fwd_t<64>(qkv_pad, s, o, ldo, lse, st);
+  if (s.hdp == 128) return attn_fwd_t<128>(qkv_pad, s, o, ldo, lse, st);
+  return set_error(ST_UNSUPPORTED, "attention: padded head dim must be 64 or 128");
+}
+
+template <int HD>
+static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const float* lse, const float* delta,
+                      const AttnShape& s, __nv_bfloat16* dqkv, cudaStream_t st) {
+  const uint64_t ldd = (uint64_t)s.H * s.hdp;
+  CUtensorMap kv128, q64, do64, q128, do128, kv64;
+  GPTK_TRY(make_tmap_3d(&kv128, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
+  GPTK_TRY(make_tmap_3d(&q64, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 64, 1));
+  GPTK_TRY(make_tmap_3d(&do64, dop, ldd, s.T, s.B, ldd, (uint64_t)s.T * ldd, 64, 64, 1));
+  GPTK_TRY(make_tmap_3d(&q128, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
+  GPTK_TRY(make_tmap_3d(&do128, dop, ldd, s.T, s.B, ldd, (uint64_t)s.T * ldd, 64, 128, 1));
+  GPTK_TRY(make_tmap_3d(&kv64, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 64, 1));
+  const float scale = 1.f / sqrtf((float)s.hd);
+  const float scale_log2 = kLog2e * scale;
+  const DevCtl ctl = device_ctl();
+  {
+    using L = DkvSmem<HD>;
+    GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
+    dim3 grid((s.T + 127) / 128, s.B * s.H);
+    attn_bwd_dkv_kernel<HD><<<grid, 192, L::BYTES, st>>>(kv128, q64, do64, s, lse, delta, dqkv, scale_log2, scale, ctl);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    using L = DqSmem<HD>;
+    GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
+    dim3 grid((s.T + 127) / 128, s.B * s.H);
+    attn_bwd_dq_kernel<HD><<<grid, 192, L::BYTES, st>>>(q128, do128, kv64, s, lse, delta, dqkv, scale_log2, scale, ctl);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  return ST_OK;
+}
+
+int launch_attn_bwd(const __nv_bfloat16* qkv_pad, const __nv_bfloat16* do_pad, const float* lse,
+                    const float* delta, const AttnShape& s, __nv_bfloat16* dqkv_pad, cudaStream_t st) {
+  if (s.B < 1 || s.T < 1 || s.H < 1) return set_error(ST_INVALID_ARG, "attention: empty shape");
+  if (s.B * s.H > 65535) return set_error(ST_UNSUPPORTED, "attention: B*H above 65535");
+  if (s.hdp == 64) return attn_bwd_t<64>(qkv_pad, do_pad, lse, delta, s, dqkv_pad, st);
+  if (s.hdp == 128) return attn_bwd_t<128>(qkv_pad, do_pad, lse, delta, s, dqkv_pad, st);
+  return set_error(ST_UNSUPPORTED, "attention: padded head dim must be 64 or 128");
+}
+
+}  // namespace gptk

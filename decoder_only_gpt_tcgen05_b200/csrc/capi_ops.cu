@@ -1,0 +1,85 @@
+// C ABI of the op-level entry points (include/gpt_ops.h).
+#include <string>
+
+#include "gemm.cuh"
+#include "gpt_ops.h"
+#include "host.cuh"
+#include "kernels.cuh"
+
+using namespace gptk;
+
+extern "C" {
+
+GPT_API const char* gpt_last_error(void) { return last_error(); }
+
+GPT_API int gpt_op_gemm(int epilogue, int bn, const void* a, long long lda, int a_mn, const void* b, long long ldb,
+                        int b_mn, int M, int N, int K, void* out, long long ldo, const float* bias, int accumulate,
+                        void* stream) {
+  set_error(ST_OK, "");
+  if (!a || !b || !out) return set_error(ST_INVALID_ARG, "gpt_op_gemm: null pointer");
+  if (M < 1 || N < 1 || K < 1) return set_error(ST_INVALID_ARG, "gpt_op_gemm: M, N, K must be >= 1");
+  if (epilogue != EPI_BF16 && epilogue != EPI_F32) return set_error(ST_INVALID_ARG, "gpt_op_gemm: bad epilogue");
+  if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "gpt_op_gemm: bn must be 128 or 256");
+  const long long need_a = a_mn ? M : K, need_b = b_mn ? N : K;
+  if (lda < need_a || ldb < need_b || ldo < N) return set_error(ST_INVALID_ARG, "gpt_op_gemm: pitch too small");
+  GemmParams p = {};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.out = out;
+  p.ldo = ldo;
+  p.bias = bias;
+  p.accumulate = accumulate;
+  p.hd = p.hdp = 1;
+  Operand A{a, lda, a_mn ? 1 : 0};
+  Operand B{b, ldb, b_mn ? 1 : 0};
+  return run_gemm(epilogue, bn, A, B, p, static_cast<cudaStream_t>(stream));
+}
+
+static int check_attn_shape(int B, int T, int H, int hd) {
+  if (B < 1 || T < 1 || H < 1) return set_error(ST_INVALID_ARG, "attention: B, T, H must be >= 1");
+  if (hd != 64 && hd != 128) return set_error(ST_UNSUPPORTED, "attention: head dim must be 64 or 128");
+  return ST_OK;
+}
+
+GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, int rope, int qk_norm, float rope_base,
+                                 float eps, void* qkv_norm, float* rstd_q, float* rstd_k, float* rope_cs, void* o,
+                                 float* lse, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(check_attn_shape(B, T, H, hd));
+  if (!qkv || !qkv_norm || !o || !lse) return set_error(ST_INVALID_ARG, "attention: null pointer");
+  if (rope && !rope_cs) return set_error(ST_INVALID_ARG, "attention: rope needs rope_cs");
+  if (qk_norm && (!rstd_q || !rstd_k)) return set_error(ST_INVALID_ARG, "attention: qk_norm needs rstd_q, rstd_k");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int M = B * T;
+  float2* cs = reinterpret_cast<float2*>(rope_cs);
+  if (rope) GPTK_TRY(launch_rope_table(cs, T, hd / 2, rope_base, st));
+  GPTK_TRY(launch_qk_fwd(static_cast<const __nv_bfloat16*>(qkv), cs, M, T, H, hd, hd, rope, qk_norm, eps,
+                         static_cast<__nv_bfloat16*>(qkv_norm), rstd_q, rstd_k, st));
+  AttnShape s{B, T, H, hd, hd, 3LL * H * hd};
+  return launch_attn_fwd(static_cast<const __nv_bfloat16*>(qkv_norm), s, static_cast<__nv_bfloat16*>(o),
+                         (long long)H * hd, lse, st);
+}
+
+GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, const float* rstd_k, const float* rope_cs,
+                                 const void* o, const float* lse, const void* dout, int B, int T, int H, int hd,
+                                 int rope, int qk_norm, float* delta, void* dqkv, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(check_attn_shape(B, T, H, hd));
+  if (!qkv_norm || !o || !lse || !dout || !delta || !dqkv) return set_error(ST_INVALID_ARG, "attention: null pointer");
+  if (rope && !rope_cs) return set_error(ST_INVALID_ARG, "attention: rope needs rope_cs");
+  if (qk_norm && (!rstd_q || !rstd_k)) return set_error(ST_INVALID_ARG, "attention: qk_norm needs rstd_q, rstd_k");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int M = B * T;
+  const __nv_bfloat16* qn = static_cast<const __nv_bfloat16*>(qkv_norm);
+  const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(dout);
+  __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(dqkv);
+  GPTK_TRY(launch_attn_delta(static_cast<const __nv_bfloat16*>(o), dO, B, T, H, hd, hd, delta, st));
+  AttnShape s{B, T, H, hd, hd, 3LL * H * hd};
+  GPTK_TRY(launch_attn_bwd(qn, dO, lse, delta, s, dq, st));
+  // gradient w.r.t. the normalised q, k, v -> through QK-norm and RoPE, in place
+  return launch_qk_bwd(dq, qn, rstd_q, rstd_k, reinterpret_cast<const float2*>(rope_cs), M, T, H, hd, hd, rope,
+                       qk_norm, dq, st);
+}
+
+}  // extern "C"

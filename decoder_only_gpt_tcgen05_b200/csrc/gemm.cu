@@ -1,0 +1,167 @@
+// Host launcher of the tcgen05 GEMM family and the tensor-map / status helpers.
+#include <mutex>
+#include <string>
+
+#include "gemm.cuh"
+#include "host.cuh"
+
+namespace gptk {
+
+// ------------------------------------------------------------ error string
+
+static thread_local std::string g_last_error;
+
+int set_error(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+const char* last_error() { return g_last_error.c_str(); }
+
+// ------------------------------------------------------------ device status word
+
+// One status word per device, in a __device__ variable: the library allocates nothing.
+__device__ unsigned int g_dev_status[4];
+static unsigned int* g_status[64];
+static std::once_flag g_status_once[64];
+static unsigned long long g_timeout_ns = 2000000000ull;  // 2 s per wait
+
+DevCtl device_ctl() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(g_status_once[dev & 63], [dev]() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_status) == cudaSuccess) g_status[dev & 63] = static_cast<unsigned int*>(p);
+  });
+  DevCtl c;
+  c.status = g_status[dev & 63];
+  c.timeout_ns = g_timeout_ns;
+  return c;
+}
+
+void set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns; }
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (cached[dev & 63] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev & 63] = n > 0 ? n : 148;
+  }
+  return cached[dev & 63];
+}
+
+// ------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+                 uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(ST_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15))
+    return set_error(ST_INVALID_ARG, "tensor base must be 16-byte aligned and its pitch a multiple of 16 bytes");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(ST_CUDA, "cuTensorMapEncodeTiled (2d) failed: " + std::to_string((int)r));
+  return ST_OK;
+}
+
+int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                 uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return set_error(ST_CUDA, "cuTensorMapEncodeTiled is not available");
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((s1 * 2) & 15) || ((s2 * 2) & 15))
+    return set_error(ST_INVALID_ARG, "tensor base must be 16-byte aligned and its pitches multiples of 16 bytes");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1 * 2, s2 * 2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(ST_CUDA, "cuTensorMapEncodeTiled (3d) failed: " + std::to_string((int)r));
+  return ST_OK;
+}
+
+// ------------------------------------------------------------ GEMM launcher
+
+template <int BN, int EPI>
+static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
+  using C = GemmCfg<BN>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set[dev & 63]) {
+    GPTK_CUDA(cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    attr_set[dev & 63] = true;
+  }
+  const int tiles = p.tiles_m * p.tiles_n;
+  int grid = num_sms();
+  if (grid > tiles) grid = tiles;
+  gemm_kernel<BN, EPI><<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, p);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+template <int BN>
+static int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                        cudaStream_t st) {
+  switch (epi) {
+    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16>(ta, tb, p, st);
+    case EPI_F32: return launch_gemm_t<BN, EPI_F32>(ta, tb, p, st);
+    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID>(ta, tb, p, st);
+    case EPI_QKV: return launch_gemm_t<BN, EPI_QKV>(ta, tb, p, st);
+    case EPI_UP: return launch_gemm_t<BN, EPI_UP>(ta, tb, p, st);
+    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD>(ta, tb, p, st);
+    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD>(ta, tb, p, st);
+    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD>(ta, tb, p, st);
+  }
+  return set_error(ST_INVALID_ARG, "unknown GEMM epilogue");
+}
+
+int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st) {
+  if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0) return set_error(ST_INVALID_ARG, "GEMM with an empty dimension");
+  CUtensorMap ta, tb;
+  if (!A.mn_major) {
+    GPTK_TRY(make_tmap_2d(&ta, A.ptr, p.K, p.M, A.ld, 64, 128));
+  } else {
+    GPTK_TRY(make_tmap_2d(&ta, A.ptr, p.M, p.K, A.ld, 64, 64));
+  }
+  if (!B.mn_major) {
+    GPTK_TRY(make_tmap_2d(&tb, B.ptr, p.K, p.N, B.ld, 64, bn));
+  } else {
+    GPTK_TRY(make_tmap_2d(&tb, B.ptr, p.N, p.K, B.ld, 64, 64));
+  }
+  p.a_mn = A.mn_major;
+  p.b_mn = B.mn_major;
+  p.tiles_m = (p.M + 127) / 128;
+  p.tiles_n = (p.N + bn - 1) / bn;
+  p.ctl = device_ctl();
+  if (p.ctl.status == nullptr) return set_error(ST_CUDA, "could not allocate the device status word");
+  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, p, st) : dispatch_epi<128>(epi, ta, tb, p, st);
+}
+
+}  // namespace gptk

@@ -1,0 +1,68 @@
+// Host-side helpers shared by the launchers: error plumbing, tensor-map
+// encoding, device properties.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+
+#include "ptx.cuh"
+
+namespace gptk {
+
+// status codes of the C ABI (mirrored in include/gpt.h)
+enum : int {
+  ST_OK = 0,
+  ST_INVALID_ARG = 1,
+  ST_UNSUPPORTED = 2,
+  ST_WORKSPACE_TOO_SMALL = 3,
+  ST_CUDA = 4,
+  ST_DEVICE_TIMEOUT = 5,
+};
+
+// Records a message for gpt_last_error() (thread-local) and returns the code.
+int set_error(int code, const std::string& msg);
+const char* last_error();
+
+// CUDA runtime check: records the call site and returns ST_CUDA on failure.
+#define GPTK_CUDA(call)                                                                        \
+  do {                                                                                         \
+    cudaError_t e_ = (call);                                                                   \
+    if (e_ != cudaSuccess)                                                                     \
+      return ::gptk::set_error(::gptk::ST_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+#define GPTK_TRY(expr)        \
+  do {                        \
+    int rc_ = (expr);         \
+    if (rc_ != 0) return rc_; \
+  } while (0)
+
+// The device status word and wait limit used by every kernel launched on this device.
+DevCtl device_ctl();
+int num_sms();
+
+// 2-D bf16 tensor map with 128-byte swizzle: inner extent `inner` (contiguous),
+// outer extent `outer`, row pitch `ld` elements, box {box_inner, box_outer}.
+int make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+                 uint32_t box_inner, uint32_t box_outer);
+// 3-D bf16 tensor map: dims {d0 (contiguous), d1, d2}, pitches (elements) s1, s2, box {b0, b1, b2}.
+int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                 uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
+
+// One GEMM operand in global memory.  For a K-major operand `ld` is the pitch
+// between consecutive M (or N) rows; for an MN-major operand it is the pitch
+// between consecutive K rows.
+struct Operand {
+  const void* ptr;
+  long long ld;
+  int mn_major;
+};
+
+struct GemmParams;
+// C[M,N] = A[M,K] B[N,K]^T with the fused epilogue `epi`; bn = 128 or 256.
+int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st);
+
+}  // namespace gptk

@@ -1,0 +1,697 @@
+// Memory-bound kernels of the hot path: parameter cast, RoPE table, embedding,
+// norms (forward / backward), column reductions, cross-entropy combine, loss and
+// bits-per-byte reduction, QK-norm + RoPE (forward / backward), attention delta,
+// and the counter-based initialiser.  Every reduction runs in a fixed order so
+// results are bitwise reproducible run to run.
+#include <cmath>
+#include <string>
+
+#include "host.cuh"
+#include "kernels.cuh"
+
+namespace gptk {
+
+static inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// ------------------------------------------------------------------ cast
+
+__global__ void cast_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, long long n4) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    float4 v = src[i];
+    dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
+int launch_cast_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t st) {
+  if (n % 4) return set_error(ST_INVALID_ARG, "cast: n must be a multiple of 4");
+  long long n4 = n / 4;
+  int grid = num_sms() * 8;
+  if (n4 < (long long)grid * 256) grid = cdiv(n4, 256);
+  if (grid < 1) return ST_OK;
+  cast_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst), n4);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ RoPE table
+
+__global__ void rope_table_kernel(float2* cs, int T, int half, double base) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T * half) return;
+  int t = i / half, j = i % half;
+  double inv = pow(base, -static_cast<double>(j) / static_cast<double>(half));
+  double s, c;
+  sincos(static_cast<double>(t) * inv, &s, &c);
+  cs[i] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+int launch_rope_table(float2* cs, int T, int half, double base, cudaStream_t st) {
+  rope_table_kernel<<<cdiv((long long)T * half, 256), 256, 0, st>>>(cs, T, half, base);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ embedding
+
+__global__ void embed_fwd_kernel(const int* __restrict__ idx, const float* __restrict__ wte,
+                                 const float* __restrict__ wpe, float* __restrict__ x, int M, int T, int D, int V,
+                                 DevCtl ctl) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (int m = blockIdx.x * warps + (threadIdx.x >> 5); m < M; m += gridDim.x * warps) {
+    int id = idx[m];
+    if (id < 0 || id >= V) {
+      if (lane == 0) dev_report(ctl, DEV_ERR_BAD_TOKEN, 0);
+      id = 0;
+    }
+    const float4* e = reinterpret_cast<const float4*>(wte + (long long)id * D);
+    const float4* p = wpe ? reinterpret_cast<const float4*>(wpe + (long long)(m % T) * D) : nullptr;
+    float4* o = reinterpret_cast<float4*>(x + (long long)m * D);
+    for (int c = lane; c < D / 4; c += 32) {
+      float4 v = __ldg(e + c);
+      if (p) {
+        float4 q = __ldg(p + c);
+        v.x += q.x; v.y += q.y; v.z += q.z; v.w += q.w;
+      }
+      o[c] = v;
+    }
+  }
+}
+
+int launch_embed_fwd(const int* idx, const float* wte, const float* wpe, float* x, int M, int T, int D, int V,
+                     cudaStream_t st) {
+  int grid = cdiv(M, 8);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  embed_fwd_kernel<<<grid, 256, 0, st>>>(idx, wte, wpe, x, M, T, D, V, device_ctl());
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ norms
+// One warp per row.  A row of D <= 128*NV floats lives in registers (NV float4 per lane).
+
+template <int NV>
+__global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const float* __restrict__ g,
+                                const float* __restrict__ b, int ln, float eps, __nv_bfloat16* __restrict__ y,
+                                long long ldy, float* __restrict__ mean_out, float* __restrict__ rstd_out) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int D4 = D / 4;
+  for (int m = blockIdx.x * warps + (threadIdx.x >> 5); m < M; m += gridDim.x * warps) {
+    const float4* xr = reinterpret_cast<const float4*>(x + (long long)m * D);
+    float4 v[NV];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      int c = i * 32 + lane;
+      v[i] = c < D4 ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      s += v[i].x + v[i].y + v[i].z + v[i].w;
+    }
+    float mu = 0.f;
+    if (ln) mu = warp_sum(s) / D;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      int c = i * 32 + lane;
+      if (c < D4) {
+        float a = v[i].x - mu, bb = v[i].y - mu, cc = v[i].z - mu, d = v[i].w - mu;
+        ss += a * a + bb * bb + cc * cc + d * d;
+      }
+    }
+    const float r = rsqrtf(warp_sum(ss) / D + eps);
+    if (lane == 0) {
+      rstd_out[m] = r;
+      if (ln) mean_out[m] = mu;
+    }
+    uint2* yr = reinterpret_cast<uint2*>(y + (long long)m * ldy);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      int c = i * 32 + lane;
+      if (c < D4) {
+        float4 o = make_float4((v[i].x - mu) * r, (v[i].y - mu) * r, (v[i].z - mu) * r, (v[i].w - mu) * r);
+        if (ln) {
+          float4 gg = __ldg(reinterpret_cast<const float4*>(g) + c);
+          o.x *= gg.x; o.y *= gg.y; o.z *= gg.z; o.w *= gg.w;
+          if (b) {
+            float4 bb = __ldg(reinterpret_cast<const float4*>(b) + c);
+            o.x += bb.x; o.y += bb.y; o.z += bb.z; o.w += bb.w;
+          }
+        }
+        yr[c] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+      }
+    }
+  }
+}
+
+template <int NV>
+__global__ void norm_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
+                                const float* __restrict__ mean, const float* __restrict__ rstd,
+                                const float* __restrict__ g, int ln, int M, int D, float* __restrict__ dres,
+                                int dres_init, __nv_bfloat16* __restrict__ dres_bf, float* __restrict__ dg_part,
+                                float* __restrict__ db_part) {
+  extern __shared__ float red[];  // [warps][2][D] when ln
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int D4 = D / 4;
+  float4 dg[NV], db[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) dg[i] = db[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int m = blockIdx.x * warps + w; m < M; m += gridDim.x * warps) {
+    const float4* xr = reinterpret_cast<const float4*>(x + (long long)m * D);
+    const float4* gr = reinterpret_cast<const float4*>(dy + (long long)m * D);
+    const float mu = ln ? mean[m] : 0.f;
+    const float r = rstd[m];
+    float4 xh[NV], gh[NV];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      int c = i * 32 + lane;
+      if (c < D4) {
+        float4 xv = xr[c], gv = gr[c];
+        xh[i] = make_float4((xv.x - mu) * r, (xv.y - mu) * r, (xv.z - mu) * r, (xv.w - mu) * r);
+        if (ln) {
+          db[i].x += gv.x; db[i].y += gv.y; db[i].z += gv.z; db[i].w += gv.w;
+          dg[i].x += gv.x * xh[i].x; dg[i].y += gv.y * xh[i].y; dg[i].z += gv.z * xh[i].z; dg[i].w += gv.w * xh[i].w;
+          float4 gg = __ldg(reinterpret_cast<const float4*>(g) + c);
+          gv.x *= gg.x; gv.y *= gg.y; gv.z *= gg.z; gv.w *= gg.w;
+        }
+        gh[i] = gv;
+        s1 += gv.x + gv.y + gv.z + gv.w;
+        s2 += gv.x * xh[i].x + gv.y * xh[i].y + gv.z * xh[i].z + gv.w * xh[i].w;
+      } else {
+        xh[i] = gh[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    const float m1 = ln ? warp_sum(s1) / D : 0.f;
+    const float m2 = warp_sum(s2) / D;
+    float4* dr = reinterpret_cast<float4*>(dres + (long long)m * D);
+    uint2* db16 = reinterpret_cast<uint2*>(dres_bf + (long long)m * D);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      int c = i * 32 + lane;
+      if (c < D4) {
+        float4 o = make_float4(r * (gh[i].x - m1 - xh[i].x * m2), r * (gh[i].y - m1 - xh[i].y * m2),
+                               r * (gh[i].z - m1 - xh[i].z * m2), r * (gh[i].w - m1 - xh[i].w * m2));
+        if (!dres_init) {
+          float4 prev = dr[c];
+          o.x += prev.x; o.y += prev.y; o.z += prev.z; o.w += prev.w;
+        }
+        dr[c] = o;
+        db16[c] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+      }
+    }
+  }
+  if (!ln) return;
+  // block-level reduction of the gain / bias partials in warp order
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    int c = i * 32 + lane;
+    if (c < D4) {
+      reinterpret_cast<float4*>(red + (size_t)w * 2 * D)[c] = dg[i];
+      reinterpret_cast<float4*>(red + (size_t)w * 2 * D + D)[c] = db[i];
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    float a = 0.f, bsum = 0.f;
+    for (int k = 0; k < warps; ++k) {
+      a += red[(size_t)k * 2 * D + c];
+      bsum += red[(size_t)k * 2 * D + D + c];
+    }
+    dg_part[(size_t)blockIdx.x * D + c] = a;
+    db_part[(size_t)blockIdx.x * D + c] = bsum;
+  }
+}
+
+template <typename F>
+static int norm_dispatch(int D, F&& f) {
+  if (D % 4) return set_error(ST_UNSUPPORTED, "norm: n_embd must be a multiple of 4");
+  if (D <= 512) return f(std::integral_constant<int, 4>());
+  if (D <= 1024) return f(std::integral_constant<int, 8>());
+  if (D <= 2048) return f(std::integral_constant<int, 16>());
+  if (D <= 4096) return f(std::integral_constant<int, 32>());
+  return set_error(ST_UNSUPPORTED, "norm: n_embd above 4096");
+}
+
+int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b, int ln, float eps,
+                    __nv_bfloat16* y, long long ldy, float* mean, float* rstd, cudaStream_t st) {
+  return norm_dispatch(D, [&](auto nv) {
+    constexpr int NV = decltype(nv)::value;
+    int grid = cdiv(M, 8);
+    if (grid > num_sms() * 8) grid = num_sms() * 8;
+    norm_fwd_kernel<NV><<<grid, 256, 0, st>>>(x, M, D, g, b, ln, eps, y, ldy, mean, rstd);
+    GPTK_CUDA(cudaGetLastError());
+    return (int)ST_OK;
+  });
+}
+
+static const int kNormBwdBlocks = 296;
+
+int launch_norm_bwd(const float* dy, const float* x, const float* mean, const float* rstd, const float* g, int ln,
+                    int M, int D, float* dres, int dres_init, __nv_bfloat16* dres_bf, float* dg_part,
+                    float* db_part, int* nblk_out, cudaStream_t st) {
+  return norm_dispatch(D, [&](auto nv) {
+    constexpr int NV = decltype(nv)::value;
+    int grid = cdiv(M, 8);
+    if (grid > kNormBwdBlocks) grid = kNormBwdBlocks;
+    size_t smem = ln ? (size_t)8 * 2 * D * sizeof(float) : 0;
+    if (smem > 48 * 1024) {
+      GPTK_CUDA(cudaFuncSetAttribute(norm_bwd_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    }
+    norm_bwd_kernel<NV><<<grid, 256, smem, st>>>(dy, x, mean, rstd, g, ln, M, D, dres, dres_init, dres_bf, dg_part,
+                                                 db_part);
+    GPTK_CUDA(cudaGetLastError());
+    if (nblk_out) *nblk_out = grid;
+    return (int)ST_OK;
+  });
+}
+
+int norm_bwd_max_blocks() { return kNormBwdBlocks; }
+
+// ------------------------------------------------------------------ column reductions
+
+__global__ void colreduce_kernel(const float* __restrict__ part, int R, int N, float* __restrict__ out,
+                                 int accumulate) {
+  int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= N) return;
+  float s = 0.f;
+  for (int r = 0; r < R; ++r) s += part[(size_t)r * N + c];
+  out[c] = accumulate ? out[c] + s : s;
+}
+
+int launch_colreduce(const float* part, int R, int N, float* out, int accumulate, cudaStream_t st) {
+  colreduce_kernel<<<cdiv(N, 256), 256, 0, st>>>(part, R, N, out, accumulate);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+static const int kColsumChunks = 128;
+int colsum_max_chunks() { return kColsumChunks; }
+
+template <typename T>
+__global__ void colsum_kernel(const T* __restrict__ a, long long lda, int M, int N, int rows_per, float* part) {
+  int c = blockIdx.x * blockDim.x + threadIdx.x;
+  int r0 = blockIdx.y * rows_per;
+  if (c >= N) return;
+  int r1 = min(M, r0 + rows_per);
+  float s = 0.f;
+  for (int r = r0; r < r1; ++r) s += static_cast<float>(a[(long long)r * lda + c]);
+  part[(size_t)blockIdx.y * N + c] = s;
+}
+
+template <typename T>
+static int colsum_t(const T* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st) {
+  int rows_per = cdiv(M, kColsumChunks);
+  int chunks = cdiv(M, rows_per);
+  dim3 grid(cdiv(N, 128), chunks);
+  colsum_kernel<T><<<grid, 128, 0, st>>>(a, lda, M, N, rows_per, part);
+  GPTK_CUDA(cudaGetLastError());
+  *R = chunks;
+  return ST_OK;
+}
+
+int launch_colsum_f32(const float* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st) {
+  return colsum_t(a, lda, M, N, part, R, st);
+}
+int launch_colsum_bf16(const __nv_bfloat16* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st) {
+  return colsum_t(a, lda, M, N, part, R, st);
+}
+
+// ------------------------------------------------------------------ cross-entropy combine
+
+__global__ void ce_combine_kernel(const float2* __restrict__ part, int ntiles, const float* __restrict__ zy, int M,
+                                  float* __restrict__ ell, float* __restrict__ lse) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  for (int m = blockIdx.x * warps + (threadIdx.x >> 5); m < M; m += gridDim.x * warps) {
+    const float2* p = part + (long long)m * ntiles;
+    float mx = -INFINITY;
+    for (int t = lane; t < ntiles; t += 32) mx = fmaxf(mx, p[t].x);
+    mx = warp_max(mx);
+    float s = 0.f;
+    for (int t = lane; t < ntiles; t += 32) {
+      float2 q = p[t];
+      if (q.x != -INFINITY) s += q.y * ex2_approx(q.x - mx);
+    }
+    s = warp_sum(s);
+    if (lane == 0) {
+      float l = (mx + log2f(s)) * 0.6931471805599453f;
+      lse[m] = l;
+      ell[m] = l - zy[m];
+    }
+  }
+}
+
+int launch_ce_combine(const float2* part, int ntiles, const float* zy, int M, float* ell, float* lse,
+                      cudaStream_t st) {
+  int grid = cdiv(M, 8);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  ce_combine_kernel<<<grid, 256, 0, st>>>(part, ntiles, zy, M, ell, lse);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ loss / bpb reduction
+
+static const int kLossBlocks = 256;
+int loss_reduce_blocks() { return kLossBlocks; }
+
+// part_d: [blocks][2] (sum of loss, sum of loss over byte-bearing targets); part_i: [blocks][2] (bytes, count)
+__global__ void loss_partial_kernel(const float* __restrict__ ell, const int* __restrict__ targets,
+                                    const int* __restrict__ tb, int M, double* part_d, long long* part_i) {
+  __shared__ double sd[2][8];
+  __shared__ long long si[2][8];
+  int per = (M + gridDim.x - 1) / gridDim.x;
+  int r0 = blockIdx.x * per, r1 = min(M, r0 + per);
+  double a = 0.0, b = 0.0;
+  long long nb = 0, cnt = 0;
+  for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+    double l = ell[r];
+    a += l;
+    if (tb) {
+      int bytes = tb[targets[r]];
+      if (bytes > 0) {
+        b += l;
+        nb += bytes;
+        cnt += 1;
+      }
+    }
+  }
+  a = warp_sum_d(a);
+  b = warp_sum_d(b);
+  nb = warp_sum_ll(nb);
+  cnt = warp_sum_ll(cnt);
+  int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    sd[0][w] = a; sd[1][w] = b; si[0][w] = nb; si[1][w] = cnt;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double A = 0, Bs = 0;
+    long long NB = 0, C = 0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+      A += sd[0][k]; Bs += sd[1][k]; NB += si[0][k]; C += si[1][k];
+    }
+    part_d[2 * blockIdx.x] = A;
+    part_d[2 * blockIdx.x + 1] = Bs;
+    part_i[2 * blockIdx.x] = NB;
+    part_i[2 * blockIdx.x + 1] = C;
+  }
+}
+
+__global__ void loss_final_kernel(const double* part_d, const long long* part_i, int nblk, int M, float* loss,
+                                  double* sum_nats, long long* sum_bytes, float* bpb) {
+  if (threadIdx.x != 0) return;
+  double A = 0, Bs = 0;
+  long long NB = 0;
+  for (int k = 0; k < nblk; ++k) {
+    A += part_d[2 * k];
+    Bs += part_d[2 * k + 1];
+    NB += part_i[2 * k];
+  }
+  if (loss) *loss = static_cast<float>(A / M);
+  if (sum_nats) *sum_nats = Bs;
+  if (sum_bytes) *sum_bytes = NB;
+  if (bpb) *bpb = NB > 0 ? static_cast<float>(Bs / (0.6931471805599453 * (double)NB)) : NAN;
+}
+
+int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int M, double* part_d,
+                       long long* part_i, float* loss, double* sum_nats, long long* sum_bytes, float* bpb,
+                       cudaStream_t st) {
+  loss_partial_kernel<<<kLossBlocks, 256, 0, st>>>(ell, targets, token_bytes, M, part_d, part_i);
+  GPTK_CUDA(cudaGetLastError());
+  loss_final_kernel<<<1, 32, 0, st>>>(part_d, part_i, kLossBlocks, M, loss, sum_nats, sum_bytes, bpb);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ QK-norm + RoPE
+// One warp per (token, head).  Lane l handles pair indices i = l + 32 j (i < hd/2) and their
+// partners i + hd/2, so a RoPE pair never crosses lanes.
+
+template <int PAIRS>
+__global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ qkv, const float2* __restrict__ cs, int M, int T,
+                              int H, int hd, int hdp, int rope, int qk_norm, float eps,
+                              __nv_bfloat16* __restrict__ out, float* __restrict__ rq, float* __restrict__ rk) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int half = hd / 2;
+  const long long D = (long long)H * hd;
+  for (long long wid = blockIdx.x * (long long)warps + (threadIdx.x >> 5); wid < (long long)M * H;
+       wid += (long long)gridDim.x * warps) {
+    const int m = static_cast<int>(wid / H), h = static_cast<int>(wid % H);
+    const int t = m % T;
+    for (int sct = 0; sct < 3; ++sct) {
+      const __nv_bfloat16* src = qkv + (long long)m * 3 * D + sct * D + (long long)h * hd;
+      __nv_bfloat16* dst = out + (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
+      float a[PAIRS], b[PAIRS];
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < PAIRS; ++j) {
+        int i = lane + 32 * j;
+        a[j] = i < half ? __bfloat162float(src[i]) : 0.f;
+        b[j] = i < half ? __bfloat162float(src[i + half]) : 0.f;
+        ss += a[j] * a[j] + b[j] * b[j];
+      }
+      float r = 1.f;
+      if (sct < 2) {
+        if (qk_norm) {
+          r = rsqrtf(warp_sum(ss) / hd + eps);
+          if (lane == 0) (sct == 0 ? rq : rk)[(long long)m * H + h] = r;
+        }
+#pragma unroll
+        for (int j = 0; j < PAIRS; ++j) {
+          int i = lane + 32 * j;
+          if (rope && i < half) {
+            float2 e = cs[(long long)t * half + i];
+            float x1 = a[j], x2 = b[j];
+            a[j] = x1 * e.x - x2 * e.y;
+            b[j] = x1 * e.y + x2 * e.x;
+          }
+          a[j] *= r;
+          b[j] *= r;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < PAIRS; ++j) {
+        int i = lane + 32 * j;
+        if (i < half) {
+          dst[i] = __float2bfloat16_rn(a[j]);
+          dst[i + half] = __float2bfloat16_rn(b[j]);
+        }
+      }
+    }
+  }
+}
+
+template <int PAIRS>
+__global__ void qk_bwd_kernel(const __nv_bfloat16* __restrict__ dpad, const __nv_bfloat16* __restrict__ qpad,
+                              const float* __restrict__ rq, const float* __restrict__ rk,
+                              const float2* __restrict__ cs, int M, int T, int H, int hd, int hdp, int rope,
+                              int qk_norm, __nv_bfloat16* __restrict__ dqkv) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int half = hd / 2;
+  const long long D = (long long)H * hd;
+  for (long long wid = blockIdx.x * (long long)warps + (threadIdx.x >> 5); wid < (long long)M * H;
+       wid += (long long)gridDim.x * warps) {
+    const int m = static_cast<int>(wid / H), h = static_cast<int>(wid % H);
+    const int t = m % T;
+    for (int sct = 0; sct < 3; ++sct) {
+      const long long po = (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
+      const __nv_bfloat16* dsrc = dpad + po;
+      __nv_bfloat16* dst = dqkv + (long long)m * 3 * D + sct * D + (long long)h * hd;
+      float a[PAIRS], b[PAIRS];
+#pragma unroll
+      for (int j = 0; j < PAIRS; ++j) {
+        int i = lane + 32 * j;
+        a[j] = i < half ? __bfloat162float(dsrc[i]) : 0.f;
+        b[j] = i < half ? __bfloat162float(dsrc[i + half]) : 0.f;
+      }
+      if (sct < 2) {
+        if (qk_norm) {
+          // dx = r (dy - y mean(dy y)), y the normalised output that the forward saved
+          const __nv_bfloat16* ysrc = qpad + po;
+          float ya[PAIRS], yb[PAIRS];
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j) {
+            int i = lane + 32 * j;
+            ya[j] = i < half ? __bfloat162float(ysrc[i]) : 0.f;
+            yb[j] = i < half ? __bfloat162float(ysrc[i + half]) : 0.f;
+            s += a[j] * ya[j] + b[j] * yb[j];
+          }
+          const float mdy = warp_sum(s) / hd;
+          const float r = (sct == 0 ? rq : rk)[(long long)m * H + h];
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j) {
+            a[j] = r * (a[j] - ya[j] * mdy);
+            b[j] = r * (b[j] - yb[j] * mdy);
+          }
+        }
+        if (rope) {
+          // the rotation is orthogonal: its reverse rotates by -phi
+#pragma unroll
+          for (int j = 0; j < PAIRS; ++j) {
+            int i = lane + 32 * j;
+            if (i < half) {
+              float2 e = cs[(long long)t * half + i];
+              float x1 = a[j], x2 = b[j];
+              a[j] = x1 * e.x + x2 * e.y;
+              b[j] = -x1 * e.y + x2 * e.x;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < PAIRS; ++j) {
+        int i = lane + 32 * j;
+        if (i < half) {
+          dst[i] = __float2bfloat16_rn(a[j]);
+          dst[i + half] = __float2bfloat16_rn(b[j]);
+        }
+      }
+    }
+  }
+}
+
+int launch_qk_fwd(const __nv_bfloat16* qkv, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
+                  int qk_norm, float eps, __nv_bfloat16* qkv_pad, float* rstd_q, float* rstd_k, cudaStream_t st) {
+  if (hd % 2) return set_error(ST_UNSUPPORTED, "head_dim must be even");
+  long long work = (long long)M * H;
+  int grid = cdiv(work, 8);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  if (hd <= 64)
+    qk_fwd_kernel<1><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k);
+  else if (hd <= 128)
+    qk_fwd_kernel<2><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k);
+  else
+    return set_error(ST_UNSUPPORTED, "head_dim above 128");
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, const float* rstd_q,
+                  const float* rstd_k, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
+                  int qk_norm, __nv_bfloat16* dqkv, cudaStream_t st) {
+  if (hd % 2) return set_error(ST_UNSUPPORTED, "head_dim must be even");
+  long long work = (long long)M * H;
+  int grid = cdiv(work, 8);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  if (hd <= 64)
+    qk_bwd_kernel<1><<<grid, 256, 0, st>>>(dqkv_pad, qkv_pad, rstd_q, rstd_k, rope_cs, M, T, H, hd, hdp, rope, qk_norm,
+                                           dqkv);
+  else if (hd <= 128)
+    qk_bwd_kernel<2><<<grid, 256, 0, st>>>(dqkv_pad, qkv_pad, rstd_q, rstd_k, rope_cs, M, T, H, hd, hdp, rope, qk_norm,
+                                           dqkv);
+  else
+    return set_error(ST_UNSUPPORTED, "head_dim above 128");
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ attention delta
+
+__global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dpad, int B,
+                                  int T, int H, int hd, int hdp, float* __restrict__ delta) {
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long M = (long long)B * T;
+  for (long long wid = blockIdx.x * (long long)warps + (threadIdx.x >> 5); wid < M * H;
+       wid += (long long)gridDim.x * warps) {
+    const long long m = wid / H;
+    const int h = static_cast<int>(wid % H);
+    const __nv_bfloat16* orow = o + m * H * hd + (long long)h * hd;
+    const __nv_bfloat16* drow = dpad + m * H * hdp + (long long)h * hdp;
+    float s = 0.f;
+    for (int d = lane; d < hd; d += 32) s += __bfloat162float(orow[d]) * __bfloat162float(drow[d]);
+    s = warp_sum(s);
+    if (lane == 0) {
+      const long long b = m / T, t = m % T;
+      delta[(b * H + h) * T + t] = s;
+    }
+  }
+}
+
+int launch_attn_delta(const __nv_bfloat16* o, const __nv_bfloat16* do_pad, int B, int T, int H, int hd, int hdp,
+                      float* delta, cudaStream_t st) {
+  long long work = (long long)B * T * H;
+  int grid = cdiv(work, 8);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  attn_delta_kernel<<<grid, 256, 0, st>>>(o, do_pad, B, T, H, hd, hdp, delta);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ initialisation
+// SplitMix64 (Steele, Lea, Flood 2014): output n of the stream seeded with s is
+// mix(s + (n+1) * golden_gamma).  Element i takes outputs 2i and 2i+1, turns their top
+// 24 bits into u1 in (0,1] and u2 in [0,1), and Box-Muller gives sqrt(-2 ln u1) cos(2 pi u2).
+
+__device__ __forceinline__ unsigned long long splitmix64_at(unsigned long long seed, unsigned long long n) {
+  unsigned long long z = seed + (n + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__global__ void init_normal_kernel(float* __restrict__ p, long long off, long long n, unsigned long long seed,
+                                   float stdv) {
+  for (long long k = blockIdx.x * (long long)blockDim.x + threadIdx.x; k < n; k += (long long)gridDim.x * blockDim.x) {
+    const unsigned long long i = static_cast<unsigned long long>(off + k);
+    const unsigned long long r0 = splitmix64_at(seed, 2ull * i);
+    const unsigned long long r1 = splitmix64_at(seed, 2ull * i + 1ull);
+    const double u1 = (static_cast<double>(r0 >> 40) + 1.0) * (1.0 / 16777216.0);
+    const double u2 = static_cast<double>(r1 >> 40) * (1.0 / 16777216.0);
+    const double z = sqrt(-2.0 * log(u1)) * cospi(2.0 * u2);
+    p[off + k] = static_cast<float>(static_cast<double>(stdv) * z);
+  }
+}
+
+__global__ void fill_kernel(float* p, long long n, float v) {
+  for (long long k = blockIdx.x * (long long)blockDim.x + threadIdx.x; k < n; k += (long long)gridDim.x * blockDim.x)
+    p[k] = v;
+}
+
+int launch_init_normal(float* params, long long off, long long n, unsigned long long seed, float stdv,
+                       cudaStream_t st) {
+  if (n <= 0) return ST_OK;
+  int grid = cdiv(n, 256);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  init_normal_kernel<<<grid, 256, 0, st>>>(params, off, n, seed, stdv);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+int launch_fill(float* p, long long n, float value, cudaStream_t st) {
+  if (n <= 0) return ST_OK;
+  int grid = cdiv(n, 256);
+  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  fill_kernel<<<grid, 256, 0, st>>>(p, n, value);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+}  // namespace gptk

@@ -1,0 +1,79 @@
+// Declarations of the launchers for the memory-bound kernels (kernels.cu,
+// embed_bwd.cu) and the attention kernels (attention.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace gptk {
+
+enum : unsigned int { DEV_ERR_BAD_TOKEN = 2u };
+
+// fp32 -> bf16, n elements (n % 4 == 0, 16-byte aligned)
+int launch_cast_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStream_t st);
+// cs[t][i] = (cos, sin)(t * base^(-i/half)), computed in double
+int launch_rope_table(float2* cs, int T, int half, double base, cudaStream_t st);
+// x[m] = wte[idx[m]] (+ wpe[m % T])   (fp32 [M, D])
+int launch_embed_fwd(const int* idx, const float* wte, const float* wpe, float* x, int M, int T, int D, int V,
+                     cudaStream_t st);
+// y = norm(x) as bf16 [M, ldy]; saves mean (LayerNorm only) and rstd per row
+int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b, int ln, float eps,
+                    __nv_bfloat16* y, long long ldy, float* mean, float* rstd, cudaStream_t st);
+// dres (+)= norm'(x)^T dy ; also writes a bf16 copy of the result; LayerNorm gain/bias
+// gradients go to per-block partials (dg_part, db_part: [nblk][D]) for launch_colreduce
+int launch_norm_bwd(const float* dy, const float* x, const float* mean, const float* rstd, const float* g, int ln,
+                    int M, int D, float* dres, int dres_init, __nv_bfloat16* dres_bf, float* dg_part,
+                    float* db_part, int* nblk_out, cudaStream_t st);
+// out[c] (+)= sum_r part[r][c]  (fixed order)
+int launch_colreduce(const float* part, int R, int N, float* out, int accumulate, cudaStream_t st);
+// column sums of an [M, N] matrix into per-chunk partials (returns the number of chunks)
+int launch_colsum_f32(const float* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st);
+int launch_colsum_bf16(const __nv_bfloat16* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st);
+int colsum_max_chunks();
+// per-row cross-entropy from the vocab-tile partials: ell = lse - z_y
+int launch_ce_combine(const float2* part, int ntiles, const float* zy, int M, float* ell, float* lse,
+                      cudaStream_t st);
+// deterministic reduction of per-token losses: loss = sum/M, and bpb sums over targets with bytes > 0
+int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int M, double* part_d,
+                       long long* part_i, float* loss, double* sum_nats, long long* sum_bytes, float* bpb,
+                       cudaStream_t st);
+int loss_reduce_blocks();
+// q,k,v (head padded) -> per-head RMSNorm / RoPE reverse -> dqkv [M, 3D] (unpadded)
+int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, const float* rstd_q,
+                  const float* rstd_k, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
+                  int qk_norm, __nv_bfloat16* dqkv, cudaStream_t st);
+// raw qkv [M, 3D] -> RoPE, per-head RMSNorm -> padded q,k,v
+int launch_qk_fwd(const __nv_bfloat16* qkv, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
+                  int qk_norm, float eps, __nv_bfloat16* qkv_pad, float* rstd_q, float* rstd_k, cudaStream_t st);
+// delta[b,h,t] = sum_d o[m, h*hd + d] * do[m, h, d]
+int launch_attn_delta(const __nv_bfloat16* o, const __nv_bfloat16* do_pad, int B, int T, int H, int hd, int hdp,
+                      float* delta, cudaStream_t st);
+// params[off, off+n) = std * N(0,1) from the counter-based generator, or = value
+int launch_init_normal(float* params, long long off, long long n, unsigned long long seed, float std,
+                       cudaStream_t st);
+int launch_fill(float* p, long long n, float value, cudaStream_t st);
+
+// ---- embedding backward (embed_bwd.cu)
+// scratch layout sizes for M tokens over V ids
+long long embed_bwd_scratch_bytes(int M, int V);
+// dwte[v] += sum over tokens m with idx[m] == v of dx[m]  (deterministic order: ascending m)
+int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float* dwte, void* scratch,
+                     cudaStream_t st);
+// dwpe[t] (+)= sum_b dx[b*T + t]
+int launch_pos_bwd(const float* dx, int B, int T, int D, float* dwpe, int accumulate, cudaStream_t st);
+
+// ---- attention (attention.cu)
+struct AttnShape {
+  int B, T, H, hd, hdp;
+  long long ld_qkv;  // pitch (elements) between tokens in the padded q|k|v buffer: 3*H*hdp
+};
+int launch_attn_fwd(const __nv_bfloat16* qkv_pad, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
+                    cudaStream_t st);
+int launch_attn_bwd(const __nv_bfloat16* qkv_pad, const __nv_bfloat16* do_pad, const float* lse,
+                    const float* delta, const AttnShape& s, __nv_bfloat16* dqkv_pad, cudaStream_t st);
+
+}  // namespace gptk

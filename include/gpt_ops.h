@@ -1,0 +1,81 @@
+/* Op-level entry points of the B200 GPT library: the individual steps of the
+ * hot path, callable one at a time for unit tests and for the attention-only
+ * and lm_head-only measurements.  The model-level calls are in gpt.h.
+ *
+ * Conventions (shared with gpt.h):
+ *   - every pointer argument is DEVICE memory owned by the caller, unless a
+ *     comment says otherwise; the library allocates nothing and frees nothing;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream); every call only enqueues work and returns;
+ *   - bf16 tensors are passed as `const void*` holding IEEE bfloat16 values;
+ *   - matrices are row-major with an explicit pitch `ld*` in elements, which
+ *     must make every row start on a 16-byte boundary (ld multiple of 8 for
+ *     bf16, of 4 for fp32); base pointers must be 16-byte aligned;
+ *   - return value: 0 (GPT_OK) or a gpt_status code from gpt.h, with a
+ *     message in gpt_last_error(); argument errors are detected on the host
+ *     before anything is launched.
+ */
+#ifndef GPT_OPS_H
+#define GPT_OPS_H
+
+#include "gpt.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogues of gpt_op_gemm. */
+#define GPT_GEMM_OUT_BF16 0 /* out (bf16) = A B^T (+ bias)                          */
+#define GPT_GEMM_OUT_F32 1  /* out (fp32) = A B^T (+ bias), or out += A B^T          */
+
+/* The tensor-core matrix product used by every linear layer of the model
+ * ("nanoGPT" wiki page, model.py walkthrough: c_attn, c_proj, c_fc and
+ * lm_head are nn.Linear layers, y = x W^T + b):
+ *
+ *   out[M,N] = A[M,K] * B[N,K]^T
+ *
+ * A is given K-major (a_mn = 0: element (m,k) at a[m*lda + k]) or MN-major
+ * (a_mn = 1: element (m,k) at a[k*lda + m]); likewise B (b_mn = 0: (n,k) at
+ * b[n*ldb + k]; b_mn = 1: (n,k) at b[k*ldb + n]).  A and B are bf16; the
+ * product accumulates in fp32.  `bias` (fp32 [N], may be NULL) is added to
+ * every row.  With GPT_GEMM_OUT_F32 and accumulate != 0 the product is added
+ * to the existing contents of `out`.  bn selects the tile width (128 or 256).
+ * Any M, N, K >= 1 is accepted; ragged edges are handled in the kernel. */
+GPT_API int gpt_op_gemm(int epilogue, int bn, const void* a, long long lda, int a_mn, const void* b,
+                        long long ldb, int b_mn, int M, int N, int K, void* out, long long ldo,
+                        const float* bias, int accumulate, void* stream);
+
+/* Causal self-attention of one layer with RoPE and QK-norm, forward
+ * ("nanoGPT" wiki page, CausalSelfAttention: q, k, v split from one fused
+ * projection, reshaped to (B, n_head, T, head_dim), causal mask;
+ * "nanochat-d20-chat" card, Architecture: RoPE + QK-norm).
+ *
+ *   qkv      in  bf16 [B*T, 3*H*hd]  raw q|k|v rows (token-major; head h of q
+ *                 at columns h*hd .. h*hd+hd-1, k after all q heads, v after k)
+ *   qkv_norm out bf16 [B*T, 3*H*hd]  q, k after RoPE (if rope) and per-head
+ *                 RMSNorm (if qk_norm); v copied
+ *   rstd_q, rstd_k out fp32 [B*T, H]  per-head 1/rms of q and k (qk_norm only;
+ *                 may be NULL otherwise)
+ *   rope_cs  out fp32 [T, hd/2, 2]   (cos, sin) of t * base^(-2i/hd) (rope
+ *                 only; may be NULL otherwise); kept for the backward
+ *   o        out bf16 [B*T, H*hd]    softmax(q k^T / sqrt(hd) + mask) v
+ *   lse      out fp32 [B, H, T]      natural-log logsumexp of each score row
+ * hd must be 64 or 128.  RoPE rotates the pairs (i, i + hd/2). */
+GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, int rope, int qk_norm,
+                                 float rope_base, float eps, void* qkv_norm, float* rstd_q, float* rstd_k,
+                                 float* rope_cs, void* o, float* lse, void* stream);
+
+/* Backward of gpt_op_attention_fwd: given dout = dL/do (bf16 [B*T, H*hd]) and
+ * the forward's outputs, writes dqkv = dL/dqkv (bf16 [B*T, 3*H*hd], the
+ * gradient w.r.t. the RAW projection output, through QK-norm and RoPE).
+ * delta is caller scratch, fp32 [B, H, T].  Deterministic. */
+GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, const float* rstd_k,
+                                 const float* rope_cs, const void* o, const float* lse, const void* dout, int B,
+                                 int T, int H, int hd, int rope, int qk_norm, float* delta, void* dqkv,
+                                 void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT_OPS_H */
