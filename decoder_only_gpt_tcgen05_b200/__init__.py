@@ -7,3 +7,5 @@ pointers and the current CUDA stream to the library and does nothing else.
 """
 from ._lib import GptError, LIB_PATH, lib  # noqa: F401
 from . import ops  # noqa: F401
+from . import model  # noqa: F401
+from .model import GPT, GPTConfig, PRESETS, preset  # noqa: F401

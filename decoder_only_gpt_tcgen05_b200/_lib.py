@@ -31,6 +31,16 @@ SIGNATURES = {
     "gpt_op_gemm": [_I, _I, _P, _LL, _I, _P, _LL, _I, _I, _I, _I, _P, _LL, _P, _I, _P],
     "gpt_op_attention_fwd": [_P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P],
     "gpt_op_attention_bwd": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P],
+    "gpt_param_count": [_P, _P],
+    "gpt_param_tensor_count": [_P, _P],
+    "gpt_param_tensor": [_P, _I, _P, _I, _P, _P, _P],
+    "gpt_workspace_size": [_P, _I, _I, _P],
+    "gpt_init_weights": [_P, C.c_uint64, _P, _P],
+    "gpt_forward_loss": [_P, _P, _P, _P, _I, _I, _P, C.c_size_t, _P, _P],
+    "gpt_backward": [_P, _P, _I, _I, _P, C.c_size_t, _P, _I, _P],
+    "gpt_eval_bpb": [_P, _P, _P, _P, _P, _I, _I, _P, C.c_size_t, _P, _P, _P, _P],
+    "gpt_sync_status": [_P],
+    "gpt_set_wait_timeout_ns": [C.c_uint64],
 }
 
 

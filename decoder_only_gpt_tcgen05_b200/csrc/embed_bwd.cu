@@ -1,0 +1,185 @@
+// Deterministic backward of the token and position embeddings.
+//
+//   dwte[v] += sum over tokens m with idx[m] == v of dx[m]        (ascending m)
+//   dwpe[t] += sum over b of dx[b*T + t]                          (ascending b)
+//
+// Token ids follow a Zipf law, so one id can own thousands of rows; floating-point
+// atomics would make the sum order (and the result) vary run to run.  Instead the
+// tokens are counting-sorted by id with a stable order:
+//   1. chunks of 256 tokens: each token's rank among equal ids earlier in its chunk,
+//      and the per-chunk count of every id
+//   2. per id, an exclusive scan of the chunk counts over chunks (column scan)
+//   3. an exclusive scan of the per-id totals (bucket offsets)
+//   4. scatter: position = offset[id] + earlier chunks' count + rank in chunk
+//   5. one block per id sums its bucket's rows in ascending token order
+#include "host.cuh"
+#include "kernels.cuh"
+
+namespace gptk {
+
+static constexpr int kChunk = 256;
+
+static inline long long align256(long long x) { return (x + 255) & ~255LL; }
+
+struct EmbedScratch {
+  int* cnt;     // [G][V]
+  int* total;   // [V]
+  int* offs;    // [V]
+  int* rank;    // [M]
+  int* sorted;  // [M]
+};
+
+static EmbedScratch carve(void* base, int M, int V) {
+  const int G = (M + kChunk - 1) / kChunk;
+  char* p = static_cast<char*>(base);
+  EmbedScratch s;
+  s.cnt = reinterpret_cast<int*>(p);
+  p += align256((long long)G * V * 4);
+  s.total = reinterpret_cast<int*>(p);
+  p += align256((long long)V * 4);
+  s.offs = reinterpret_cast<int*>(p);
+  p += align256((long long)V * 4);
+  s.rank = reinterpret_cast<int*>(p);
+  p += align256((long long)M * 4);
+  s.sorted = reinterpret_cast<int*>(p);
+  return s;
+}
+
+long long embed_bwd_scratch_bytes(int M, int V) {
+  const long long G = (M + kChunk - 1) / kChunk;
+  return align256(G * V * 4) + 2 * align256((long long)V * 4) + 2 * align256((long long)M * 4);
+}
+
+__global__ void chunk_rank_kernel(const int* __restrict__ idx, int M, int V, int* __restrict__ cnt,
+                                  int* __restrict__ rank) {
+  __shared__ int ids[kChunk];
+  const int g = blockIdx.x;
+  const int t = threadIdx.x;
+  const int m = g * kChunk + t;
+  int id = -1;
+  if (m < M) {
+    id = idx[m];
+    if (id < 0 || id >= V) id = 0;  // out-of-range ids were reported by the forward embedding
+  }
+  ids[t] = id;
+  __syncthreads();
+  if (m >= M) return;
+  int r = 0;
+  bool last = true;
+  for (int u = 0; u < kChunk; ++u) {
+    const int o = ids[u];
+    if (o == id) {
+      if (u < t) ++r;
+      if (u > t) last = false;
+    }
+  }
+  rank[m] = r;
+  if (last) cnt[(long long)g * V + id] = r + 1;
+}
+
+__global__ void col_scan_kernel(int* __restrict__ cnt, int G, int V, int* __restrict__ total) {
+  const int v = blockIdx.x * blockDim.x + threadIdx.x;
+  if (v >= V) return;
+  int run = 0;
+  for (int g = 0; g < G; ++g) {
+    const long long i = (long long)g * V + v;
+    const int c = cnt[i];
+    cnt[i] = run;
+    run += c;
+  }
+  total[v] = run;
+}
+
+// single block, 1024 threads: exclusive scan of total[0..V)
+__global__ void offsets_kernel(const int* __restrict__ total, int V, int* __restrict__ offs) {
+  __shared__ int part[1024];
+  const int t = threadIdx.x;
+  const int per = (V + 1023) / 1024;
+  const int v0 = t * per, v1 = min(V, v0 + per);
+  int s = 0;
+  for (int v = v0; v < v1; ++v) s += total[v];
+  part[t] = s;
+  __syncthreads();
+  // Hillis-Steele inclusive scan over the 1024 partial sums
+  for (int o = 1; o < 1024; o <<= 1) {
+    int x = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += x;
+    __syncthreads();
+  }
+  int run = t > 0 ? part[t - 1] : 0;
+  for (int v = v0; v < v1; ++v) {
+    offs[v] = run;
+    run += total[v];
+  }
+}
+
+__global__ void scatter_kernel(const int* __restrict__ idx, int M, int V, const int* __restrict__ cnt,
+                               const int* __restrict__ offs, const int* __restrict__ rank, int* __restrict__ sorted) {
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= M) return;
+  int id = idx[m];
+  if (id < 0 || id >= V) id = 0;
+  const int g = m / kChunk;
+  sorted[offs[id] + cnt[(long long)g * V + id] + rank[m]] = m;
+}
+
+__global__ void segsum_kernel(const float* __restrict__ dx, int D, const int* __restrict__ total,
+                              const int* __restrict__ offs, const int* __restrict__ sorted, float* __restrict__ dwte) {
+  const int v = blockIdx.x;
+  const int n = total[v];
+  if (n == 0) return;
+  const int o = offs[v];
+  const int D4 = D / 4;
+  for (int c = threadIdx.x; c < D4; c += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < n; ++i) {
+      const int m = sorted[o + i];
+      const float4 x = reinterpret_cast<const float4*>(dx + (long long)m * D)[c];
+      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    }
+    float4* w = reinterpret_cast<float4*>(dwte + (long long)v * D) + c;
+    float4 cur = *w;
+    cur.x += acc.x; cur.y += acc.y; cur.z += acc.z; cur.w += acc.w;
+    *w = cur;
+  }
+}
+
+int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float* dwte, void* scratch,
+                     cudaStream_t st) {
+  if (D % 4) return set_error(ST_UNSUPPORTED, "embedding backward: n_embd must be a multiple of 4");
+  const int G = (M + kChunk - 1) / kChunk;
+  EmbedScratch s = carve(scratch, M, V);
+  GPTK_CUDA(cudaMemsetAsync(s.cnt, 0, (size_t)G * V * sizeof(int), st));
+  chunk_rank_kernel<<<G, kChunk, 0, st>>>(idx, M, V, s.cnt, s.rank);
+  GPTK_CUDA(cudaGetLastError());
+  col_scan_kernel<<<(V + 255) / 256, 256, 0, st>>>(s.cnt, G, V, s.total);
+  GPTK_CUDA(cudaGetLastError());
+  offsets_kernel<<<1, 1024, 0, st>>>(s.total, V, s.offs);
+  GPTK_CUDA(cudaGetLastError());
+  scatter_kernel<<<(M + 255) / 256, 256, 0, st>>>(idx, M, V, s.cnt, s.offs, s.rank, s.sorted);
+  GPTK_CUDA(cudaGetLastError());
+  int threads = D / 4 < 256 ? ((D / 4 + 31) / 32) * 32 : 256;
+  segsum_kernel<<<V, threads, 0, st>>>(dx, D, s.total, s.offs, s.sorted, dwte);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+__global__ void pos_bwd_kernel(const float* __restrict__ dx, int B, int T, int D, float* __restrict__ dwpe,
+                               int accumulate) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= (long long)T * D) return;
+  const int t = static_cast<int>(i / D), d = static_cast<int>(i % D);
+  float s = 0.f;
+  for (int b = 0; b < B; ++b) s += dx[((long long)b * T + t) * D + d];
+  dwpe[i] = accumulate ? dwpe[i] + s : s;
+}
+
+int launch_pos_bwd(const float* dx, int B, int T, int D, float* dwpe, int accumulate, cudaStream_t st) {
+  const long long n = (long long)T * D;
+  pos_bwd_kernel<<<(int)((n + 255) / 256), 256, 0, st>>>(dx, B, T, D, dwpe, accumulate);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+}  // namespace gptk

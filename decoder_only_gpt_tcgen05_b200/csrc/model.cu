@@ -1,0 +1,676 @@
+// Model-level C ABI (include/gpt.h): parameter layout, workspace planner, and the
+// stream-ordered launch sequences of the forward loss, the backward and the bpb
+// evaluation.
+//
+// Forward (per layer): norm -> QKV GEMM (+bias, RoPE, QK-norm in the epilogue) ->
+// flash attention -> out-proj GEMM (+bias, residual add in the epilogue) -> norm ->
+// MLP-up GEMM (+bias, activation in the epilogue) -> MLP-down GEMM (+bias, residual).
+// Then the final norm and the lm_head GEMM whose epilogue keeps an online logsumexp
+// per row over each vocab tile, so the logits never reach memory.
+//
+// Backward: cross-entropy gradient tiles (recomputed logits, softmax - onehot) in
+// row chunks feed the lm_head data- and weight-gradient GEMMs; each layer then runs
+// its GEMM gradients (MN-major operands, no transposes), the activation gradient in
+// the data-gradient epilogue, the flash-attention backward, the QK-norm/RoPE
+// reverse, the norm backward with the residual add, and finally the deterministic
+// embedding scatter.
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "gemm.cuh"
+#include "gpt.h"
+#include "host.cuh"
+#include "kernels.cuh"
+
+namespace gptk {
+
+void set_wait_timeout_ns(unsigned long long ns);
+int norm_bwd_max_blocks();
+
+// ------------------------------------------------------------------ parameter layout
+
+struct ParamInfo {
+  std::string name;
+  long long off, rows, cols;
+};
+
+struct LayerOff {
+  long long ln1_g = -1, ln1_b = -1, w_qkv = -1, b_qkv = -1, w_o = -1, b_o = -1;
+  long long ln2_g = -1, ln2_b = -1, w_up = -1, b_up = -1, w_down = -1, b_down = -1;
+};
+
+struct Layout {
+  std::vector<ParamInfo> list;
+  long long wte = -1, wpe = -1, lnf_g = -1, lnf_b = -1, lm_head = -1;
+  std::vector<LayerOff> layer;
+  long long total = 0;
+};
+
+static long long add_param(Layout& L, const std::string& name, long long rows, long long cols) {
+  ParamInfo p{name, L.total, rows, cols};
+  L.list.push_back(p);
+  L.total += rows * cols;
+  return p.off;
+}
+
+static Layout make_layout(const gpt_config& c) {
+  Layout L;
+  const long long D = c.n_embd, V = c.vocab_size, F = 4LL * c.n_embd;
+  const bool ln = c.norm == 1, bias = c.linear_bias != 0;
+  L.wte = add_param(L, "wte", V, D);
+  if (c.pos == 0) L.wpe = add_param(L, "wpe", c.block_size, D);
+  for (int l = 0; l < c.n_layer; ++l) {
+    LayerOff o;
+    const std::string p = "h" + std::to_string(l) + ".";
+    if (ln) {
+      o.ln1_g = add_param(L, p + "ln1_g", D, 1);
+      if (bias) o.ln1_b = add_param(L, p + "ln1_b", D, 1);
+    }
+    o.w_qkv = add_param(L, p + "w_qkv", 3 * D, D);
+    if (bias) o.b_qkv = add_param(L, p + "b_qkv", 3 * D, 1);
+    o.w_o = add_param(L, p + "w_o", D, D);
+    if (bias) o.b_o = add_param(L, p + "b_o", D, 1);
+    if (ln) {
+      o.ln2_g = add_param(L, p + "ln2_g", D, 1);
+      if (bias) o.ln2_b = add_param(L, p + "ln2_b", D, 1);
+    }
+    o.w_up = add_param(L, p + "w_up", F, D);
+    if (bias) o.b_up = add_param(L, p + "b_up", F, 1);
+    o.w_down = add_param(L, p + "w_down", D, F);
+    if (bias) o.b_down = add_param(L, p + "b_down", D, 1);
+    L.layer.push_back(o);
+  }
+  if (ln) {
+    L.lnf_g = add_param(L, "lnf_g", D, 1);
+    if (bias) L.lnf_b = add_param(L, "lnf_b", D, 1);
+  }
+  if (!c.tie_embed) L.lm_head = add_param(L, "lm_head", V, D);
+  return L;
+}
+
+static int validate(const gpt_config* c) {
+  if (!c) return set_error(ST_INVALID_ARG, "null config");
+  if (c->n_layer < 1 || c->n_embd < 1 || c->n_head < 1 || c->vocab_size < 1 || c->block_size < 1)
+    return set_error(ST_INVALID_ARG, "config: every size must be >= 1");
+  if (c->norm < 0 || c->norm > 1 || c->pos < 0 || c->pos > 1 || c->act < 0 || c->act > 1)
+    return set_error(ST_INVALID_ARG, "config: norm, pos and act must be 0 or 1");
+  if (!(c->norm_eps > 0.f)) return set_error(ST_INVALID_ARG, "config: norm_eps must be > 0");
+  if (c->pos == 1 && !(c->rope_base > 1.f)) return set_error(ST_INVALID_ARG, "config: rope_base must be > 1");
+  if (c->n_embd % 16) return set_error(ST_UNSUPPORTED, "config: n_embd must be a multiple of 16");
+  if (c->n_embd > 4096) return set_error(ST_UNSUPPORTED, "config: n_embd above 4096");
+  if (c->n_embd % c->n_head) return set_error(ST_INVALID_ARG, "config: n_embd must be divisible by n_head");
+  const int hd = c->n_embd / c->n_head;
+  if (hd % 2 || hd > 128) return set_error(ST_UNSUPPORTED, "config: head dim must be even and at most 128");
+  if ((c->pos == 1 || c->qk_norm) && hd != 64 && hd != 128)
+    return set_error(ST_UNSUPPORTED, "config: RoPE / QK-norm need a head dim of 64 or 128");
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ workspace plan
+
+static inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Plan {
+  int B, T, M, D, H, hd, hdp, F, L, V, Vp, ntn, Mc;
+  long long P;
+  // byte offsets into the workspace
+  size_t wbf, rope_cs, idx, tgt, xs, a1, st1, qkv, rq, rk, o, lse, a2, st2, u, h, af, stf;
+  size_t ce_part, zy, ell, lse_ce, loss_d, loss_i, loss_f;
+  size_t dlog, da, dres, dres_bf, du, do_pad, delta, dqkv_pad, dqkv, part_a, part_b, embed;
+  size_t total;
+  long long partN;
+};
+
+static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
+  Plan p;
+  p.B = B;
+  p.T = T;
+  p.M = B * T;
+  p.D = c.n_embd;
+  p.H = c.n_head;
+  p.hd = c.n_embd / c.n_head;
+  p.hdp = p.hd <= 64 ? 64 : 128;
+  p.F = 4 * c.n_embd;
+  p.L = c.n_layer;
+  p.V = c.vocab_size;
+  p.Vp = (c.vocab_size + 7) / 8 * 8;
+  p.ntn = (c.vocab_size + 255) / 256;
+  p.Mc = p.M < 4096 ? p.M : 4096;
+  p.P = P;
+  const size_t M = p.M, D = p.D, F = p.F, L = p.L, H = p.H, hdp = p.hdp;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t r = off;
+    off += al(bytes);
+    return r;
+  };
+  p.wbf = take((size_t)P * 2);
+  p.rope_cs = take((size_t)T * (p.hd / 2) * 8);
+  p.idx = take(M * 4);
+  p.tgt = take(M * 4);
+  p.xs = take((2 * L + 1) * M * D * 4);
+  p.a1 = take(L * M * D * 2);
+  p.st1 = take(L * 2 * M * 4);
+  p.qkv = take(L * M * 3 * H * hdp * 2);
+  p.rq = take(L * M * H * 4);
+  p.rk = take(L * M * H * 4);
+  p.o = take(L * M * D * 2);
+  p.lse = take(L * M * H * 4);
+  p.a2 = take(L * M * D * 2);
+  p.st2 = take(L * 2 * M * 4);
+  p.u = take(L * M * F * 2);
+  p.h = take(L * M * F * 2);
+  p.af = take(M * D * 2);
+  p.stf = take(2 * M * 4);
+  p.ce_part = take(M * p.ntn * 8);
+  p.zy = take(M * 4);
+  p.ell = take(M * 4);
+  p.lse_ce = take(M * 4);
+  p.loss_d = take(loss_reduce_blocks() * 2 * 8);
+  p.loss_i = take(loss_reduce_blocks() * 2 * 8);
+  p.loss_f = take(64);
+  p.dlog = take((size_t)p.Mc * p.Vp * 2);
+  p.da = take(M * D * 4);
+  p.dres = take(M * D * 4);
+  p.dres_bf = take(M * D * 2);
+  p.du = take(M * F * 2);
+  p.do_pad = take(M * H * hdp * 2);
+  p.delta = take(M * H * 4);
+  p.dqkv_pad = take(M * 3 * H * hdp * 2);
+  p.dqkv = take(M * 3 * D * 2);
+  long long maxN = F > 3 * D ? F : 3 * D;
+  long long rows = norm_bwd_max_blocks() > colsum_max_chunks() ? norm_bwd_max_blocks() : colsum_max_chunks();
+  p.partN = maxN;
+  p.part_a = take((size_t)rows * maxN * 4);
+  p.part_b = take((size_t)rows * maxN * 4);
+  p.embed = take((size_t)embed_bwd_scratch_bytes(p.M, p.V));
+  p.total = off;
+  return p;
+}
+
+static int check_batch(const gpt_config* c, int B, int T) {
+  if (B < 1 || T < 1) return set_error(ST_INVALID_ARG, "B and T must be >= 1");
+  if (c->pos == 0 && T > c->block_size) return set_error(ST_INVALID_ARG, "T exceeds block_size");
+  if ((long long)B * T > (1LL << 30)) return set_error(ST_UNSUPPORTED, "B*T too large");
+  if ((long long)B * c->n_head > 65535) return set_error(ST_UNSUPPORTED, "B * n_head above 65535");
+  return ST_OK;
+}
+
+template <typename T>
+static T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ------------------------------------------------------------------ GEMM helper
+
+static GemmParams gp(int M, int N, int K) {
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.hd = p.hdp = 1;
+  return p;
+}
+
+// tile width: 256 unless that leaves most SMs idle
+static int pick_bn(int M, int N) {
+  const long long t256 = (long long)((M + 127) / 128) * ((N + 255) / 256);
+  return (N <= 128 || t256 < num_sms()) ? 128 : 256;
+}
+
+static int gemm(int epi, const Operand& A, const Operand& Bm, GemmParams p, cudaStream_t st, int bn = 0) {
+  if (bn == 0) bn = pick_bn(p.M, p.N);
+  return run_gemm(epi, bn, A, Bm, p, st);
+}
+
+// ------------------------------------------------------------------ forward
+
+static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, const float* params, const int* idx,
+                        const int* targets, const int* token_bytes, void* ws, float* loss, double* sum_nats,
+                        long long* sum_bytes, float* bpb, cudaStream_t st) {
+  const int M = pl.M, D = pl.D, H = pl.H, hd = pl.hd, hdp = pl.hdp, F = pl.F, T = pl.T, B = pl.B, V = pl.V;
+  const int ln = c.norm == 1;
+  __nv_bfloat16* wbf = at<__nv_bfloat16>(ws, pl.wbf);
+  float2* cs = at<float2>(ws, pl.rope_cs);
+  int* idx_ws = at<int>(ws, pl.idx);
+  int* tgt_ws = at<int>(ws, pl.tgt);
+  GPTK_CUDA(cudaMemcpyAsync(idx_ws, idx, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
+  GPTK_CUDA(cudaMemcpyAsync(tgt_ws, targets, (size_t)M * 4, cudaMemcpyDeviceToDevice, st));
+  GPTK_TRY(launch_cast_bf16(params, wbf, pl.P, st));
+  if (c.pos == 1) GPTK_TRY(launch_rope_table(cs, T, hd / 2, (double)c.rope_base, st));
+
+  float* xs = at<float>(ws, pl.xs);
+  const size_t MD = (size_t)M * D;
+  GPTK_TRY(launch_embed_fwd(idx_ws, params + Lo.wte, Lo.wpe >= 0 ? params + Lo.wpe : nullptr, xs, M, T, D, V, st));
+
+  for (int l = 0; l < pl.L; ++l) {
+    const LayerOff& o = Lo.layer[l];
+    float* x_in = xs + (size_t)(2 * l) * MD;
+    float* x_mid = xs + (size_t)(2 * l + 1) * MD;
+    float* x_out = xs + (size_t)(2 * l + 2) * MD;
+    __nv_bfloat16* a1 = at<__nv_bfloat16>(ws, pl.a1) + (size_t)l * MD;
+    float* st1 = at<float>(ws, pl.st1) + (size_t)l * 2 * M;
+    __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, pl.qkv) + (size_t)l * M * 3 * H * hdp;
+    float* rq = at<float>(ws, pl.rq) + (size_t)l * M * H;
+    float* rk = at<float>(ws, pl.rk) + (size_t)l * M * H;
+    __nv_bfloat16* ob = at<__nv_bfloat16>(ws, pl.o) + (size_t)l * MD;
+    float* lse = at<float>(ws, pl.lse) + (size_t)l * M * H;
+    __nv_bfloat16* a2 = at<__nv_bfloat16>(ws, pl.a2) + (size_t)l * MD;
+    float* st2 = at<float>(ws, pl.st2) + (size_t)l * 2 * M;
+    __nv_bfloat16* u = at<__nv_bfloat16>(ws, pl.u) + (size_t)l * M * F;
+    __nv_bfloat16* h = at<__nv_bfloat16>(ws, pl.h) + (size_t)l * M * F;
+
+    // attention sublayer
+    GPTK_TRY(launch_norm_fwd(x_in, M, D, ln ? params + o.ln1_g : nullptr, o.ln1_b >= 0 ? params + o.ln1_b : nullptr, ln,
+                             c.norm_eps, a1, D, st1, st1 + M, st));
+    if (hdp != hd) GPTK_CUDA(cudaMemsetAsync(qkv, 0, (size_t)M * 3 * H * hdp * 2, st));
+    {
+      GemmParams p = gp(M, 3 * D, D);
+      p.out = qkv;
+      p.ldo = 3LL * H * hdp;
+      p.bias = o.b_qkv >= 0 ? params + o.b_qkv : nullptr;
+      p.hd = hd;
+      p.hdp = hdp;
+      p.d_model = D;
+      p.n_head = H;
+      p.T = T;
+      p.rope = c.pos == 1;
+      p.qk_norm = c.qk_norm;
+      p.eps = c.norm_eps;
+      p.rope_cs = cs;
+      p.rstd_q = rq;
+      p.rstd_k = rk;
+      GPTK_TRY(gemm(EPI_QKV, Operand{a1, D, 0}, Operand{wbf + o.w_qkv, D, 0}, p, st, 256));
+    }
+    AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp};
+    GPTK_TRY(launch_attn_fwd(qkv, as, ob, D, lse, st));
+    {
+      GemmParams p = gp(M, D, D);
+      p.out = x_mid;
+      p.ldo = D;
+      p.resid = x_in;
+      p.ldr = D;
+      p.bias = o.b_o >= 0 ? params + o.b_o : nullptr;
+      GPTK_TRY(gemm(EPI_RESID, Operand{ob, D, 0}, Operand{wbf + o.w_o, D, 0}, p, st));
+    }
+    // MLP sublayer
+    GPTK_TRY(launch_norm_fwd(x_mid, M, D, ln ? params + o.ln2_g : nullptr, o.ln2_b >= 0 ? params + o.ln2_b : nullptr,
+                             ln, c.norm_eps, a2, D, st2, st2 + M, st));
+    {
+      GemmParams p = gp(M, F, D);
+      p.out = u;
+      p.out2 = h;
+      p.ldo = F;
+      p.act = c.act;
+      p.bias = o.b_up >= 0 ? params + o.b_up : nullptr;
+      GPTK_TRY(gemm(EPI_UP, Operand{a2, D, 0}, Operand{wbf + o.w_up, D, 0}, p, st));
+    }
+    {
+      GemmParams p = gp(M, D, F);
+      p.out = x_out;
+      p.ldo = D;
+      p.resid = x_mid;
+      p.ldr = D;
+      p.bias = o.b_down >= 0 ? params + o.b_down : nullptr;
+      GPTK_TRY(gemm(EPI_RESID, Operand{h, F, 0}, Operand{wbf + o.w_down, F, 0}, p, st));
+    }
+  }
+  // final norm + lm_head + cross-entropy
+  __nv_bfloat16* af = at<__nv_bfloat16>(ws, pl.af);
+  float* stf = at<float>(ws, pl.stf);
+  GPTK_TRY(launch_norm_fwd(xs + (size_t)(2 * pl.L) * MD, M, D, ln ? params + Lo.lnf_g : nullptr,
+                           Lo.lnf_b >= 0 ? params + Lo.lnf_b : nullptr, ln, c.norm_eps, af, D, stf, stf + M, st));
+  const long long wlm = c.tie_embed ? Lo.wte : Lo.lm_head;
+  float2* part = at<float2>(ws, pl.ce_part);
+  float* zy = at<float>(ws, pl.zy);
+  {
+    GemmParams p = gp(M, V, D);
+    p.targets = tgt_ws;
+    p.ce_part = part;
+    p.ce_zy = zy;
+    GPTK_TRY(gemm(EPI_CE_FWD, Operand{af, D, 0}, Operand{wbf + wlm, D, 0}, p, st, 256));
+  }
+  float* ell = at<float>(ws, pl.ell);
+  float* lse_ce = at<float>(ws, pl.lse_ce);
+  GPTK_TRY(launch_ce_combine(part, pl.ntn, zy, M, ell, lse_ce, st));
+  GPTK_TRY(launch_loss_reduce(ell, tgt_ws, token_bytes, M, at<double>(ws, pl.loss_d), at<long long>(ws, pl.loss_i),
+                              loss ? loss : at<float>(ws, pl.loss_f), sum_nats, sum_bytes, bpb, st));
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ backward
+
+static int bias_grad_f32(const float* a, int M, int N, float* part, float* dst, cudaStream_t st) {
+  int R = 0;
+  GPTK_TRY(launch_colsum_f32(a, N, M, N, part, &R, st));
+  return launch_colreduce(part, R, N, dst, 1, st);
+}
+
+static int bias_grad_bf16(const __nv_bfloat16* a, int M, int N, float* part, float* dst, cudaStream_t st) {
+  int R = 0;
+  GPTK_TRY(launch_colsum_bf16(a, N, M, N, part, &R, st));
+  return launch_colreduce(part, R, N, dst, 1, st);
+}
+
+static int norm_backward(const gpt_config& c, const Plan& pl, const float* dy, const float* x, const float* stats,
+                         const float* params, long long g_off, long long b_off, float* grads, float* dres,
+                         int dres_init, __nv_bfloat16* dres_bf, float* pa, float* pb, cudaStream_t st) {
+  const int ln = c.norm == 1;
+  const int M = pl.M, D = pl.D;
+  int nblk = 0;
+  GPTK_TRY(launch_norm_bwd(dy, x, stats, stats + M, ln ? params + g_off : nullptr, ln, M, D, dres, dres_init, dres_bf,
+                           pa, pb, &nblk, st));
+  if (ln) {
+    GPTK_TRY(launch_colreduce(pa, nblk, D, grads + g_off, 1, st));
+    if (b_off >= 0) GPTK_TRY(launch_colreduce(pb, nblk, D, grads + b_off, 1, st));
+  }
+  return ST_OK;
+}
+
+static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, const float* params, void* ws,
+                         float* grads, int accumulate, cudaStream_t st) {
+  const int M = pl.M, D = pl.D, H = pl.H, hd = pl.hd, hdp = pl.hdp, F = pl.F, T = pl.T, B = pl.B, V = pl.V;
+  const size_t MD = (size_t)M * D;
+  __nv_bfloat16* wbf = at<__nv_bfloat16>(ws, pl.wbf);
+  const float2* cs = at<float2>(ws, pl.rope_cs);
+  const int* idx_ws = at<int>(ws, pl.idx);
+  const int* tgt_ws = at<int>(ws, pl.tgt);
+  float* xs = at<float>(ws, pl.xs);
+  __nv_bfloat16* af = at<__nv_bfloat16>(ws, pl.af);
+  float* stf = at<float>(ws, pl.stf);
+  float* lse_ce = at<float>(ws, pl.lse_ce);
+  __nv_bfloat16* dlog = at<__nv_bfloat16>(ws, pl.dlog);
+  float* da = at<float>(ws, pl.da);
+  float* dres = at<float>(ws, pl.dres);
+  __nv_bfloat16* dres_bf = at<__nv_bfloat16>(ws, pl.dres_bf);
+  __nv_bfloat16* du = at<__nv_bfloat16>(ws, pl.du);
+  __nv_bfloat16* do_pad = at<__nv_bfloat16>(ws, pl.do_pad);
+  float* delta = at<float>(ws, pl.delta);
+  __nv_bfloat16* dqkv_pad = at<__nv_bfloat16>(ws, pl.dqkv_pad);
+  __nv_bfloat16* dqkv = hdp == hd ? dqkv_pad : at<__nv_bfloat16>(ws, pl.dqkv);
+  float* pa = at<float>(ws, pl.part_a);
+  float* pb = at<float>(ws, pl.part_b);
+
+  if (!accumulate) GPTK_CUDA(cudaMemsetAsync(grads, 0, (size_t)pl.P * 4, st));
+
+  // ---- lm_head + cross-entropy, in row chunks: dlogits never exist for all rows at once
+  const long long wlm = c.tie_embed ? Lo.wte : Lo.lm_head;
+  for (int r0 = 0; r0 < M; r0 += pl.Mc) {
+    const int mc = (M - r0) < pl.Mc ? (M - r0) : pl.Mc;
+    {
+      GemmParams p = gp(mc, V, D);
+      p.out = dlog;
+      p.ldo = pl.Vp;
+      p.targets = tgt_ws + r0;
+      p.ce_lse = lse_ce + r0;
+      p.ce_scale = 1.f / (float)M;
+      GPTK_TRY(gemm(EPI_CE_BWD, Operand{af + (size_t)r0 * D, D, 0}, Operand{wbf + wlm, D, 0}, p, st, 256));
+    }
+    {  // d af = dlogits W_lm
+      GemmParams p = gp(mc, D, V);
+      p.out = da + (size_t)r0 * D;
+      p.ldo = D;
+      GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 0}, Operand{wbf + wlm, D, 1}, p, st));
+    }
+    {  // d W_lm += dlogits^T af
+      GemmParams p = gp(V, D, mc);
+      p.out = grads + wlm;
+      p.ldo = D;
+      p.accumulate = 1;
+      GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 1}, Operand{af + (size_t)r0 * D, D, 1}, p, st));
+    }
+  }
+  GPTK_TRY(norm_backward(c, pl, da, xs + (size_t)(2 * pl.L) * MD, stf, params, Lo.lnf_g, Lo.lnf_b, grads, dres, 1,
+                         dres_bf, pa, pb, st));
+
+  for (int l = pl.L - 1; l >= 0; --l) {
+    const LayerOff& o = Lo.layer[l];
+    const float* x_in = xs + (size_t)(2 * l) * MD;
+    const float* x_mid = xs + (size_t)(2 * l + 1) * MD;
+    const __nv_bfloat16* a1 = at<__nv_bfloat16>(ws, pl.a1) + (size_t)l * MD;
+    const float* st1 = at<float>(ws, pl.st1) + (size_t)l * 2 * M;
+    const __nv_bfloat16* qkv = at<__nv_bfloat16>(ws, pl.qkv) + (size_t)l * M * 3 * H * hdp;
+    const float* rq = at<float>(ws, pl.rq) + (size_t)l * M * H;
+    const float* rk = at<float>(ws, pl.rk) + (size_t)l * M * H;
+    const __nv_bfloat16* ob = at<__nv_bfloat16>(ws, pl.o) + (size_t)l * MD;
+    const float* lse = at<float>(ws, pl.lse) + (size_t)l * M * H;
+    const __nv_bfloat16* a2 = at<__nv_bfloat16>(ws, pl.a2) + (size_t)l * MD;
+    const float* st2 = at<float>(ws, pl.st2) + (size_t)l * 2 * M;
+    const __nv_bfloat16* u = at<__nv_bfloat16>(ws, pl.u) + (size_t)l * M * F;
+    const __nv_bfloat16* h = at<__nv_bfloat16>(ws, pl.h) + (size_t)l * M * F;
+
+    // ---- MLP: x_out = x_mid + act(N(x_mid) W_up^T + b_up) W_down^T + b_down
+    {  // du = (dres W_down) * act'(u)
+      GemmParams p = gp(M, F, D);
+      p.out = du;
+      p.ldo = F;
+      p.aux = u;
+      p.ld_aux = F;
+      p.act = c.act;
+      GPTK_TRY(gemm(EPI_ACTBWD, Operand{dres_bf, D, 0}, Operand{wbf + o.w_down, F, 1}, p, st));
+    }
+    {  // dW_down += dres^T h
+      GemmParams p = gp(D, F, M);
+      p.out = grads + o.w_down;
+      p.ldo = F;
+      p.accumulate = 1;
+      GPTK_TRY(gemm(EPI_F32, Operand{dres_bf, D, 1}, Operand{h, F, 1}, p, st));
+    }
+    if (o.b_down >= 0) GPTK_TRY(bias_grad_f32(dres, M, D, pa, grads + o.b_down, st));
+    {  // da = du W_up
+      GemmParams p = gp(M, D, F);
+      p.out = da;
+      p.ldo = D;
+      GPTK_TRY(gemm(EPI_F32, Operand{du, F, 0}, Operand{wbf + o.w_up, D, 1}, p, st));
+    }
+    {  // dW_up += du^T a2
+      GemmParams p = gp(F, D, M);
+      p.out = grads + o.w_up;
+      p.ldo = D;
+      p.accumulate = 1;
+      GPTK_TRY(gemm(EPI_F32, Operand{du, F, 1}, Operand{a2, D, 1}, p, st));
+    }
+    if (o.b_up >= 0) GPTK_TRY(bias_grad_bf16(du, M, F, pa, grads + o.b_up, st));
+    GPTK_TRY(norm_backward(c, pl, da, x_mid, st2, params, o.ln2_g, o.ln2_b, grads, dres, 0, dres_bf, pa, pb, st));
+
+    // ---- attention: x_mid = x_in + attn(N(x_in)) W_o^T + b_o
+    if (hdp != hd) GPTK_CUDA(cudaMemsetAsync(do_pad, 0, (size_t)M * H * hdp * 2, st));
+    {  // do = dres W_o  (written in the head-padded layout the attention kernels read)
+      GemmParams p = gp(M, D, D);
+      p.out = do_pad;
+      p.ldo = (long long)H * hdp;
+      p.hd = hd;
+      p.hdp = hdp;
+      GPTK_TRY(gemm(EPI_BF16, Operand{dres_bf, D, 0}, Operand{wbf + o.w_o, D, 1}, p, st));
+    }
+    {  // dW_o += dres^T o
+      GemmParams p = gp(D, D, M);
+      p.out = grads + o.w_o;
+      p.ldo = D;
+      p.accumulate = 1;
+      GPTK_TRY(gemm(EPI_F32, Operand{dres_bf, D, 1}, Operand{ob, D, 1}, p, st));
+    }
+    if (o.b_o >= 0) GPTK_TRY(bias_grad_f32(dres, M, D, pa, grads + o.b_o, st));
+    GPTK_TRY(launch_attn_delta(ob, do_pad, B, T, H, hd, hdp, delta, st));
+    AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp};
+    GPTK_TRY(launch_attn_bwd(qkv, do_pad, lse, delta, as, dqkv_pad, st));
+    GPTK_TRY(launch_qk_bwd(dqkv_pad, qkv, rq, rk, cs, M, T, H, hd, hdp, c.pos == 1, c.qk_norm, dqkv, st));
+    {  // da = dqkv W_qkv
+      GemmParams p = gp(M, D, 3 * D);
+      p.out = da;
+      p.ldo = D;
+      GPTK_TRY(gemm(EPI_F32, Operand{dqkv, 3LL * D, 0}, Operand{wbf + o.w_qkv, D, 1}, p, st));
+    }
+    {  // dW_qkv += dqkv^T a1
+      GemmParams p = gp(3 * D, D, M);
+      p.out = grads + o.w_qkv;
+      p.ldo = D;
+      p.accumulate = 1;
+      GPTK_TRY(gemm(EPI_F32, Operand{dqkv, 3LL * D, 1}, Operand{a1, D, 1}, p, st));
+    }
+    if (o.b_qkv >= 0) GPTK_TRY(bias_grad_bf16(dqkv, M, 3 * D, pa, grads + o.b_qkv, st));
+    GPTK_TRY(norm_backward(c, pl, da, x_in, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0, dres_bf, pa, pb, st));
+  }
+  // ---- embeddings
+  GPTK_TRY(launch_embed_bwd(idx_ws, dres, M, D, V, grads + Lo.wte, at<void>(ws, pl.embed), st));
+  if (Lo.wpe >= 0) GPTK_TRY(launch_pos_bwd(dres, B, T, D, grads + Lo.wpe, 1, st));
+  return ST_OK;
+}
+
+// ------------------------------------------------------------------ init
+
+static int init_impl(const gpt_config& c, const Layout& Lo, unsigned long long seed, float* params, cudaStream_t st) {
+  for (const ParamInfo& p : Lo.list) {
+    const std::string& n = p.name;
+    const long long size = p.rows * p.cols;
+    const std::string base = n.substr(n.find('.') == std::string::npos ? 0 : n.find('.') + 1);
+    if (base == "ln1_g" || base == "ln2_g" || base == "lnf_g") {
+      GPTK_TRY(launch_fill(params + p.off, size, 1.f, st));
+    } else if (base.rfind("b_", 0) == 0 || base == "ln1_b" || base == "ln2_b" || base == "lnf_b") {
+      GPTK_TRY(launch_fill(params + p.off, size, 0.f, st));
+    } else {
+      float stdv = 0.02f;
+      if (c.scale_resid_init && (base == "w_o" || base == "w_down"))
+        stdv = (float)(0.02 / std::sqrt(2.0 * c.n_layer));
+      GPTK_TRY(launch_init_normal(params, p.off, size, seed, stdv, st));
+    }
+  }
+  return ST_OK;
+}
+
+}  // namespace gptk
+
+using namespace gptk;
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+GPT_API int gpt_param_count(const gpt_config* cfg, int64_t* n_out) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!n_out) return set_error(ST_INVALID_ARG, "null output");
+  *n_out = make_layout(*cfg).total;
+  return ST_OK;
+}
+
+GPT_API int gpt_param_tensor_count(const gpt_config* cfg, int32_t* n_out) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!n_out) return set_error(ST_INVALID_ARG, "null output");
+  *n_out = (int32_t)make_layout(*cfg).list.size();
+  return ST_OK;
+}
+
+GPT_API int gpt_param_tensor(const gpt_config* cfg, int32_t i, char* name, int32_t name_len, int64_t* offset,
+                             int64_t* rows, int64_t* cols) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  Layout L = make_layout(*cfg);
+  if (i < 0 || i >= (int32_t)L.list.size()) return set_error(ST_INVALID_ARG, "tensor index out of range");
+  const ParamInfo& p = L.list[i];
+  if (name && name_len > 0) {
+    std::strncpy(name, p.name.c_str(), (size_t)name_len - 1);
+    name[name_len - 1] = '\0';
+  }
+  if (offset) *offset = p.off;
+  if (rows) *rows = p.rows;
+  if (cols) *cols = p.cols;
+  return ST_OK;
+}
+
+GPT_API int gpt_workspace_size(const gpt_config* cfg, int32_t B, int32_t T, size_t* bytes) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  if (!bytes) return set_error(ST_INVALID_ARG, "null output");
+  Layout L = make_layout(*cfg);
+  *bytes = make_plan(*cfg, B, T, L.total).total;
+  return ST_OK;
+}
+
+GPT_API int gpt_init_weights(const gpt_config* cfg, uint64_t seed, float* params, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!params) return set_error(ST_INVALID_ARG, "null params");
+  return init_impl(*cfg, make_layout(*cfg), seed, params, static_cast<cudaStream_t>(stream));
+}
+
+static int check_ws(void* ws, size_t have, size_t need) {
+  if (!ws) return set_error(ST_INVALID_ARG, "null workspace");
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return set_error(ST_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (have < need)
+    return set_error(ST_WORKSPACE_TOO_SMALL,
+                     "workspace has " + std::to_string(have) + " bytes, needs " + std::to_string(need));
+  return ST_OK;
+}
+
+GPT_API int gpt_forward_loss(const gpt_config* cfg, const float* params, const int32_t* idx, const int32_t* targets,
+                             int32_t B, int32_t T, void* workspace, size_t workspace_bytes, float* loss,
+                             void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  if (!params || !idx || !targets || !loss) return set_error(ST_INVALID_ARG, "null pointer");
+  Layout L = make_layout(*cfg);
+  Plan pl = make_plan(*cfg, B, T, L.total);
+  GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
+  return forward_impl(*cfg, L, pl, params, idx, targets, nullptr, workspace, loss, nullptr, nullptr, nullptr,
+                      static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_backward(const gpt_config* cfg, const float* params, int32_t B, int32_t T, void* workspace,
+                         size_t workspace_bytes, float* grads, int32_t accumulate, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  if (!params || !grads) return set_error(ST_INVALID_ARG, "null pointer");
+  Layout L = make_layout(*cfg);
+  Plan pl = make_plan(*cfg, B, T, L.total);
+  GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
+  return backward_impl(*cfg, L, pl, params, workspace, grads, accumulate, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_eval_bpb(const gpt_config* cfg, const float* params, const int32_t* idx, const int32_t* targets,
+                         const int32_t* token_bytes, int32_t B, int32_t T, void* workspace, size_t workspace_bytes,
+                         double* sum_nats, int64_t* sum_bytes, float* bpb, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  if (!params || !idx || !targets || !token_bytes) return set_error(ST_INVALID_ARG, "null pointer");
+  Layout L = make_layout(*cfg);
+  Plan pl = make_plan(*cfg, B, T, L.total);
+  GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
+  return forward_impl(*cfg, L, pl, params, idx, targets, token_bytes, workspace, nullptr, sum_nats,
+                      reinterpret_cast<long long*>(sum_bytes), bpb, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_sync_status(void* stream) {
+  set_error(ST_OK, "");
+  GPTK_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  DevCtl c = device_ctl();
+  if (!c.status) return set_error(ST_CUDA, "device status word unavailable");
+  unsigned int v = 0;
+  GPTK_CUDA(cudaMemcpy(&v, c.status, sizeof(v), cudaMemcpyDeviceToHost));
+  if (v == 0) return ST_OK;
+  const unsigned int zero = 0;
+  GPTK_CUDA(cudaMemcpy(c.status, &zero, sizeof(zero), cudaMemcpyHostToDevice));
+  const unsigned int code = v >> 24, site = (v >> 16) & 0xff, blk = v & 0xffff;
+  if (code == DEV_ERR_TIMEOUT)
+    return set_error(ST_DEVICE_TIMEOUT, "a kernel gave up a bounded wait (site " + std::to_string(site) + ", block " +
+                                            std::to_string(blk) + ")");
+  if (code == DEV_ERR_BAD_TOKEN) return set_error(ST_INVALID_ARG, "a token id was outside [0, vocab_size)");
+  return set_error(ST_CUDA, "device status word " + std::to_string(v));
+}
+
+GPT_API int gpt_set_wait_timeout_ns(uint64_t ns) {
+  set_error(ST_OK, "");
+  if (ns == 0) return set_error(ST_INVALID_ARG, "timeout must be > 0");
+  set_wait_timeout_ns(ns);
+  return ST_OK;
+}
+
+}  // extern "C"

@@ -44,6 +44,99 @@ typedef enum gpt_status {
   GPT_ERR_DEVICE_TIMEOUT = 5        /* a kernel gave up a bounded wait (see gpt_sync_status)   */
 } gpt_status;
 
+/* Model shape (GPTConfig of the "nanoGPT" wiki page, model.py walkthrough,
+ * plus the nanochat switches of the d20 card).
+ *
+ * Supported shapes (else GPT_ERR_UNSUPPORTED): n_embd a multiple of 16 and at
+ * most 4096; n_embd divisible by n_head with an even head dim of at most 128;
+ * with RoPE or QK-norm the head dim must be 64 or 128. */
+typedef struct gpt_config {
+  int32_t n_layer;          /* number of blocks                                         */
+  int32_t n_embd;           /* width D                                                  */
+  int32_t n_head;           /* heads H; head dim hd = D / H                             */
+  int32_t block_size;       /* maximum context (rows of the learned position table)     */
+  int32_t vocab_size;       /* V                                                        */
+  int32_t norm;             /* 0: parameter-free RMSNorm, 1: LayerNorm (gain, + bias if linear_bias) */
+  int32_t pos;              /* 0: learned absolute position embedding, 1: RoPE          */
+  int32_t act;              /* MLP activation: 0 GELU (erf form), 1 ReLU^2              */
+  int32_t tie_embed;        /* 1: lm_head shares the token embedding ("weight tying")   */
+  int32_t qk_norm;          /* 1: per-head RMSNorm of q and k after RoPE                */
+  int32_t linear_bias;      /* 1: biases on every Linear and LayerNorm (GPT-2 shape)    */
+  int32_t scale_resid_init; /* 1: init std of attn/MLP output projections 0.02/sqrt(2 n_layer) */
+  float rope_base;          /* RoPE base (10000)                                        */
+  float norm_eps;           /* epsilon of every norm (1e-5)                             */
+} gpt_config;
+
+/* Parameters: ONE flat fp32 buffer, tensors back to back in this order:
+ *   wte [V, D]; wpe [block_size, D] (pos == 0); then per layer l:
+ *   ln1_g [D], ln1_b [D] (LayerNorm; _b only with linear_bias),
+ *   w_qkv [3D, D], b_qkv [3D], w_o [D, D], b_o [D], ln2_g, ln2_b,
+ *   w_up [4D, D], b_up [4D], w_down [D, 4D], b_down [D]   (b_* only with linear_bias);
+ *   then lnf_g, lnf_b (LayerNorm); lm_head [V, D] (untied only).
+ * Linear weights are [out, in] row-major (y = x W^T + b).  Gradients use the
+ * same layout.  Every tensor starts at a multiple of 16 elements. */
+GPT_API int gpt_param_count(const gpt_config* cfg, int64_t* n_out);
+GPT_API int gpt_param_tensor_count(const gpt_config* cfg, int32_t* n_out);
+/* Name (NUL-terminated, truncated to name_len), element offset and shape of
+ * tensor i (cols = 1 for vectors). */
+GPT_API int gpt_param_tensor(const gpt_config* cfg, int32_t i, char* name, int32_t name_len, int64_t* offset,
+                             int64_t* rows, int64_t* cols);
+
+/* Bytes of device workspace that gpt_forward_loss / gpt_backward /
+ * gpt_eval_bpb need for a batch of B sequences of T tokens.  The workspace
+ * holds the bf16 weight copies, the activations the backward reuses, and the
+ * scratch of every kernel.  It must be 256-byte aligned. */
+GPT_API int gpt_workspace_size(const gpt_config* cfg, int32_t B, int32_t T, size_t* bytes);
+
+/* Initial weights into `params` (fp32 [gpt_param_count]): every matrix and
+ * embedding N(0, 0.02^2) (0.02/sqrt(2 n_layer) for w_o and w_down when
+ * scale_resid_init), biases 0, LayerNorm gains 1.  Element i draws
+ * SplitMix64 outputs 2i and 2i+1 of the stream seeded with `seed` and turns
+ * them into one normal by Box-Muller, so the result does not depend on the
+ * launch configuration. */
+GPT_API int gpt_init_weights(const gpt_config* cfg, uint64_t seed, float* params, void* stream);
+
+/* Forward pass and mean next-token cross-entropy of one batch.
+ *   params   fp32 [gpt_param_count]
+ *   idx      int32 [B, T] input token ids in [0, V)
+ *   targets  int32 [B, T] next-token ids (the inputs shifted by one)
+ *   loss     fp32 [1] out: mean over the B*T targets of logsumexp(z) - z[y]
+ * The logits are never written to memory: the lm_head product streams vocab
+ * tiles through an online logsumexp.  The activations the backward needs
+ * stay in `workspace` (copies of idx and targets included).  T <= block_size
+ * when pos == 0.  An id outside [0, V) is reported by gpt_sync_status. */
+GPT_API int gpt_forward_loss(const gpt_config* cfg, const float* params, const int32_t* idx, const int32_t* targets,
+                             int32_t B, int32_t T, void* workspace, size_t workspace_bytes, float* loss,
+                             void* stream);
+
+/* Gradient of that mean loss w.r.t. every parameter, into `grads` (fp32,
+ * parameter layout): written when accumulate == 0, added when != 0.
+ * Requires that the last call on this workspace was gpt_forward_loss with the
+ * same cfg, params, B and T (the parameters must not have changed since).
+ * Deterministic: the same inputs give bitwise the same gradients. */
+GPT_API int gpt_backward(const gpt_config* cfg, const float* params, int32_t B, int32_t T, void* workspace,
+                         size_t workspace_bytes, float* grads, int32_t accumulate, void* stream);
+
+/* Bits per byte of one batch ("Train your own ChatGPT", read the source
+ * loss_eval.py): sum_nats = sum of the per-token loss over targets whose
+ * byte length token_bytes[y] > 0; sum_bytes = sum of token_bytes[y] over all
+ * targets; bpb = sum_nats / (ln 2 * sum_bytes) (NaN when sum_bytes == 0).
+ *   token_bytes int32 [V]; sum_nats fp64 [1]; sum_bytes int64 [1]; bpb fp32 [1]
+ *   (any of the three outputs may be NULL).
+ * The sums are reduced in a fixed order (bitwise reproducible). */
+GPT_API int gpt_eval_bpb(const gpt_config* cfg, const float* params, const int32_t* idx, const int32_t* targets,
+                         const int32_t* token_bytes, int32_t B, int32_t T, void* workspace, size_t workspace_bytes,
+                         double* sum_nats, int64_t* sum_bytes, float* bpb, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait runs out (GPT_ERR_DEVICE_TIMEOUT) or an
+ * input id is out of range (GPT_ERR_INVALID_ARG). */
+GPT_API int gpt_sync_status(void* stream);
+
+/* Wall-time limit of every bounded wait inside the kernels, in nanoseconds
+ * (default 2e9).  For tests of the timeout path. */
+GPT_API int gpt_set_wait_timeout_ns(uint64_t ns);
+
 /* Last error message of the calling thread ("" after success). */
 GPT_API const char* gpt_last_error(void);
 

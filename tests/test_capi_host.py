@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI: no GPU needed, no compute launched.
+
+The library must load, export every symbol the headers declare, lay out the
+parameters exactly as the oracle does, and reject bad arguments on the host
+with the documented status codes."""
+import ctypes as C
+import dataclasses
+import glob
+import os
+import re
+
+import pytest
+
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pkg():
+    import decoder_only_gpt_tcgen05_b200 as g
+    g.lib()
+    return g
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        names |= set(re.findall(r"GPT_API\s+[\w\s\*]+?\b(gpt_\w+)\s*\(", open(h).read()))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol(pkg):
+    syms = _declared_symbols()
+    assert len(syms) >= 14
+    L = pkg.lib()
+    for s in syms:
+        assert hasattr(L, s), s
+
+
+CONFIGS = ["tiny", "gpt2", "d20", "d26"]
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+def test_presets_match_oracle(pkg, name):
+    assert dataclasses.asdict(pkg.PRESETS[name]) == dataclasses.asdict(O.PRESETS[name])
+
+
+@pytest.mark.parametrize("name,over", [(n, {}) for n in CONFIGS] + [
+    ("tiny", {"tie_embed": 0}), ("gpt2", {"n_layer": 2, "linear_bias": 0}), ("gpt2", {"norm": 0})])
+def test_param_layout_matches_oracle(pkg, name, over):
+    cfg = pkg.preset(name, **over)
+    ocfg = O.Config(**dataclasses.asdict(cfg))
+    assert pkg.model.param_count(cfg) == O.param_count(ocfg)
+    lay = pkg.model.param_tensors(cfg)
+    ref = O.param_offsets(ocfg)
+    assert [t[0] for t in lay] == list(ref)
+    for nm, off, rows, cols in lay:
+        o, shape = ref[nm]
+        assert off == o and off % 16 == 0
+        assert (rows, cols) == (shape if len(shape) == 2 else (shape[0], 1))
+
+
+def test_workspace_size_grows_with_batch(pkg):
+    cfg = pkg.preset("d20")
+    a = pkg.model.workspace_size(cfg, 1, 2048)
+    b = pkg.model.workspace_size(cfg, 16, 2048)
+    assert 0 < a < b < 80 * 2 ** 30
+
+
+def _status(pkg, fn, *args):
+    return getattr(pkg.lib(), fn)(*args)
+
+
+def test_bad_arguments_are_rejected_on_the_host(pkg):
+    L = pkg.lib()
+    n = C.c_int64()
+    assert L.gpt_param_count(None, C.byref(n)) == 1
+    bad = pkg.preset("tiny", n_embd=24, n_head=4).c()
+    assert L.gpt_param_count(C.byref(bad), C.byref(n)) == 2
+    bad = pkg.preset("d20", n_head=20).c()   # head dim 64 is fine ...
+    assert L.gpt_param_count(C.byref(bad), C.byref(n)) == 0
+    bad = pkg.preset("d20", n_head=40).c()   # ... head dim 32 with RoPE is not
+    assert L.gpt_param_count(C.byref(bad), C.byref(n)) == 2
+    assert b"RoPE" in L.gpt_last_error()
+    cfg = pkg.preset("gpt2").c()
+    sz = C.c_size_t()
+    assert L.gpt_workspace_size(C.byref(cfg), 1, 1025, C.byref(sz)) == 1   # T > block_size
+    assert L.gpt_workspace_size(C.byref(cfg), 0, 16, C.byref(sz)) == 1
+    assert L.gpt_workspace_size(C.byref(cfg), 2, 1024, C.byref(sz)) == 0
+    # null pointers and a too-small workspace: caught before any launch
+    fake = C.c_void_p(1 << 20)
+    assert L.gpt_forward_loss(C.byref(cfg), None, fake, fake, 2, 1024, fake, sz.value, fake, None) == 1
+    assert L.gpt_forward_loss(C.byref(cfg), fake, fake, fake, 2, 1024, fake, sz.value - 1, fake, None) == 3
+    assert b"workspace" in L.gpt_last_error()
+    mis = C.c_void_p((1 << 20) + 16)
+    assert L.gpt_forward_loss(C.byref(cfg), fake, fake, fake, 2, 1024, mis, sz.value, fake, None) == 1
+    assert L.gpt_backward(C.byref(cfg), fake, 2, 1024, fake, sz.value, None, 0, None) == 1
+    assert L.gpt_eval_bpb(C.byref(cfg), fake, fake, fake, None, 2, 1024, fake, sz.value, None, None, None,
+                          None) == 1
+    assert L.gpt_set_wait_timeout_ns(0) == 1
+    assert L.gpt_op_gemm(0, 192, fake, 64, 0, fake, 64, 0, 8, 8, 8, fake, 8, None, 0, None) == 1
+    assert L.gpt_op_attention_fwd(fake, 1, 16, 1, 32, 1, 1, C.c_float(1e4), C.c_float(1e-5), fake, fake, fake, fake,
+                                  fake, fake, None) == 2

@@ -1,0 +1,131 @@
+"""End-to-end parity of the model-level C ABI against the oracle.
+
+Same seeded tokens and the same parameters on both sides (the GPU-initialised
+buffer is copied to the oracle).  Bar: token and byte counts bit-exact; loss
+and bpb within 2e-3 relative; every parameter gradient at cosine >= 0.999 and
+relative L2 <= 3e-2."""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda:0")
+
+
+def _pkg():
+    import decoder_only_gpt_tcgen05_b200 as g
+    return g
+
+
+CASES = {
+    # name: (config overrides on a preset, B, T, byte table range)
+    "tiny": (("tiny", {}), 4, 16, (1, 1)),
+    "gpt2_small": (("gpt2", dict(n_layer=2, n_embd=128, n_head=2, vocab_size=1000, block_size=256)), 2, 128, (1, 12)),
+    "gpt2_ragged": (("gpt2", dict(n_layer=1, n_embd=64, n_head=1, vocab_size=300, block_size=256)), 3, 200, (1, 12)),
+    "d20_small": (("d20", dict(n_layer=2, n_embd=256, n_head=2, vocab_size=2048, block_size=512)), 2, 256, (1, 16)),
+    "d20_ragged": (("d20", dict(n_layer=1, n_embd=128, n_head=1, vocab_size=777, block_size=512)), 2, 300, (1, 16)),
+}
+
+
+def _setup(name, params="init"):
+    g = _pkg()
+    (base, over), B, T, (blo, bhi) = CASES[name]
+    cfg = g.preset(base, **over)
+    ocfg = O.Config(**dataclasses.asdict(cfg))
+    model = g.GPT(cfg, B, T, device=DEV, seed=0)
+    if params == "wide":
+        # larger weights so that every nonlinearity matters; LayerNorm gains near 1
+        p = synth.normal(O.param_count(ocfg), 11, std=0.1).astype(np.float64)
+        for nm, v in O.unflatten(ocfg, p).items():
+            if nm.endswith("_g"):
+                v += 1.0
+        model.params.copy_(torch.from_numpy(p.astype(np.float32)))
+    dist = "uniform" if base == "tiny" else "zipf"
+    idx, tgt = synth.next_token_batch(B, T, cfg.vocab_size, dist=dist, seed=1)
+    tb = synth.byte_table(cfg.vocab_size, blo, bhi, seed=2, n_zero=0 if base == "tiny" else 3)
+    return g, cfg, ocfg, model, idx, tgt, tb
+
+
+def test_init_weights_match_oracle():
+    g = _pkg()
+    for name in ("tiny", "gpt2_small", "d20_small"):
+        (base, over), B, T, _ = CASES[name]
+        cfg = g.preset(base, **over)
+        m = g.GPT(cfg, 1, 16, device=DEV, seed=1234)
+        torch.cuda.synchronize()
+        ref = O.init_params(O.Config(**dataclasses.asdict(cfg)), 1234)
+        got = m.params.double().cpu().numpy()
+        assert np.allclose(got, ref, rtol=1e-6, atol=1e-9), np.abs(got - ref).max()
+
+
+@pytest.mark.parametrize("params", ["init", "wide"])
+@pytest.mark.parametrize("name", list(CASES))
+def test_forward_backward_bpb_match_oracle(name, params):
+    g, cfg, ocfg, model, idx, tgt, tb = _setup(name, params)
+    idx_d = torch.from_numpy(idx).to(DEV)
+    tgt_d = torch.from_numpy(tgt).to(DEV)
+    tb_d = torch.from_numpy(tb).to(DEV)
+    loss = model.forward_loss(idx_d, tgt_d).item()
+    grads = model.backward().double().cpu().numpy()
+    sum_nats, sum_bytes, bpb = (t.item() for t in model.eval_bpb(idx_d, tgt_d, tb_d))
+    g.model.sync_status()
+    p = model.params.double().cpu().numpy()
+    f = O.forward(ocfg, p, idx, tgt)
+    ref_g = O.backward(ocfg, p, f)
+    rs, rb, rn, rbpb = O.bits_per_byte(f["ell"], tgt, tb)
+    assert abs(loss - f["loss"]) / f["loss"] <= 2e-3, (loss, f["loss"])
+    assert sum_bytes == rb
+    assert abs(sum_nats - rs) / abs(rs) <= 2e-3
+    assert abs(bpb - rbpb) / rbpb <= 2e-3
+    for nm, (off, shape) in O.param_offsets(ocfg).items():
+        n = int(np.prod(shape))
+        a, b = grads[off:off + n], ref_g[off:off + n]
+        nb = np.linalg.norm(b)
+        if nb < 1e-30:
+            assert np.linalg.norm(a) < 1e-12, nm
+            continue
+        cos = float(a @ b / (np.linalg.norm(a) * nb))
+        rel = float(np.linalg.norm(a - b) / nb)
+        assert cos >= 0.999 and rel <= 3e-2, (nm, cos, rel)
+
+
+def test_backward_is_deterministic_and_accumulates():
+    g, cfg, ocfg, model, idx, tgt, tb = _setup("d20_small", "wide")
+    idx_d = torch.from_numpy(idx).to(DEV)
+    tgt_d = torch.from_numpy(tgt).to(DEV)
+    model.forward_loss(idx_d, tgt_d)
+    g1 = model.backward().clone()
+    model.forward_loss(idx_d, tgt_d)
+    g2 = model.backward().clone()
+    assert torch.equal(g1, g2)
+    model.forward_loss(idx_d, tgt_d)
+    model.backward()
+    g3 = model.backward(accumulate=True)
+    assert torch.equal(g3, 2 * g1)
+
+
+def test_loss_is_batch_row_independent():
+    """Each sequence's losses depend only on that sequence: the mean loss of a
+    batch equals the mean of its single-sequence losses (within rounding)."""
+    g, cfg, ocfg, model, idx, tgt, tb = _setup("d20_small", "wide")
+    B, T = idx.shape
+    full = model.forward_loss(torch.from_numpy(idx).to(DEV), torch.from_numpy(tgt).to(DEV)).item()
+    one = g.GPT(cfg, 1, T, device=DEV, params=model.params)
+    parts = [one.forward_loss(torch.from_numpy(idx[b:b + 1].copy()).to(DEV),
+                              torch.from_numpy(tgt[b:b + 1].copy()).to(DEV)).item() for b in range(B)]
+    assert abs(full - sum(parts) / B) <= 1e-5 * full
+
+
+def test_uniform_logits_loss_is_ln_v():
+    g, cfg, ocfg, model, idx, tgt, tb = _setup("d20_small", "wide")
+    off = [t for t in g.model.param_tensors(cfg) if t[0] == "lm_head"][0][1]
+    model.params[off:off + cfg.vocab_size * cfg.n_embd] = 0
+    loss = model.forward_loss(torch.from_numpy(idx).to(DEV), torch.from_numpy(tgt).to(DEV)).item()
+    assert abs(loss - math.log(cfg.vocab_size)) <= 1e-5 * math.log(cfg.vocab_size)
