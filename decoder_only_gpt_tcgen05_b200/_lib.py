@@ -31,6 +31,9 @@ SIGNATURES = {
     "gpt_op_gemm": [_I, _I, _P, _LL, _I, _P, _LL, _I, _I, _I, _I, _P, _LL, _P, _I, _P],
     "gpt_op_attention_fwd": [_P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P],
     "gpt_op_attention_bwd": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P],
+    "gpt_op_lmhead_ce_fwd": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P],
+    "gpt_profile_start": [],
+    "gpt_profile_stop": [_I, _P, _P, _P, _P],
     "gpt_param_count": [_P, _P],
     "gpt_param_tensor_count": [_P, _P],
     "gpt_param_tensor": [_P, _I, _P, _I, _P, _P, _P],
@@ -54,6 +57,10 @@ def lib():
         L = C.CDLL(LIB_PATH)
         L.gpt_last_error.restype = C.c_char_p
         L.gpt_last_error.argtypes = []
+        L.gpt_launch_count.restype = C.c_ulonglong
+        L.gpt_launch_count.argtypes = []
+        L.gpt_op_lmhead_ce_scratch_bytes.restype = C.c_size_t
+        L.gpt_op_lmhead_ce_scratch_bytes.argtypes = [_I, _I]
         for name, args in SIGNATURES.items():
             f = getattr(L, name)
             f.argtypes = args

@@ -783,6 +783,8 @@ static int attn_fwd_t(const __nv_bfloat16* qkv, const AttnShape& s, __nv_bfloat1
   GPTK_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
   const float scale_log2 = kLog2e / sqrtf((float)s.hd);
   dim3 grid((s.T + 127) / 128, s.B * s.H);
+  const double causal = (double)s.B * s.H * ((double)s.T * (s.T + 1) / 2);
+  Prof prof(PK_ATTN_FWD, 4.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 4, st);
   attn_fwd_kernel<HD><<<grid, 192, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -811,10 +813,12 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
   const float scale = 1.f / sqrtf((float)s.hd);
   const float scale_log2 = kLog2e * scale;
   const DevCtl ctl = device_ctl();
+  const double causal = (double)s.B * s.H * ((double)s.T * (s.T + 1) / 2);
   {
     using L = DkvSmem<HD>;
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
+    Prof prof(PK_ATTN_BWD_DKV, 8.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 6, st);
     attn_bwd_dkv_kernel<HD><<<grid, 192, L::BYTES, st>>>(kv128, q64, do64, s, lse, delta, dqkv, scale_log2, scale, ctl);
     GPTK_CUDA(cudaGetLastError());
   }
@@ -822,6 +826,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     using L = DqSmem<HD>;
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
+    Prof prof(PK_ATTN_BWD_DQ, 6.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 5, st);
     attn_bwd_dq_kernel<HD><<<grid, 192, L::BYTES, st>>>(q128, do128, kv64, s, lse, delta, dqkv, scale_log2, scale, ctl);
     GPTK_CUDA(cudaGetLastError());
   }

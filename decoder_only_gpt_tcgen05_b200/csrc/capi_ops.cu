@@ -82,4 +82,33 @@ GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, cons
                        qk_norm, dq, st);
 }
 
+GPT_API size_t gpt_op_lmhead_ce_scratch_bytes(int M, int V) {
+  if (M < 1 || V < 1) return 0;
+  const size_t ntn = (size_t)(V + 255) / 256;
+  return ((size_t)M * ntn * 8 + 255) / 256 * 256 + ((size_t)M * 4 + 255) / 256 * 256;
+}
+
+GPT_API int gpt_op_lmhead_ce_fwd(const void* x, const void* w, const int32_t* targets, int M, int D, int V, float* ell,
+                                 float* lse, void* scratch, void* stream) {
+  set_error(ST_OK, "");
+  if (!x || !w || !targets || !ell || !lse || !scratch) return set_error(ST_INVALID_ARG, "lmhead_ce: null pointer");
+  if (M < 1 || D < 1 || V < 1) return set_error(ST_INVALID_ARG, "lmhead_ce: M, D, V must be >= 1");
+  if (D % 8) return set_error(ST_UNSUPPORTED, "lmhead_ce: D must be a multiple of 8");
+  if (reinterpret_cast<uintptr_t>(scratch) & 255) return set_error(ST_INVALID_ARG, "lmhead_ce: scratch alignment");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int ntn = (V + 255) / 256;
+  float2* part = static_cast<float2*>(scratch);
+  float* zy = reinterpret_cast<float*>(static_cast<char*>(scratch) + ((size_t)M * ntn * 8 + 255) / 256 * 256);
+  GemmParams p = {};
+  p.M = M;
+  p.N = V;
+  p.K = D;
+  p.hd = p.hdp = 1;
+  p.targets = targets;
+  p.ce_part = part;
+  p.ce_zy = zy;
+  GPTK_TRY(run_gemm(EPI_CE_FWD, 256, Operand{x, D, 0}, Operand{w, D, 0}, p, st));
+  return launch_ce_combine(part, ntn, zy, M, ell, lse, st);
+}
+
 }  // extern "C"

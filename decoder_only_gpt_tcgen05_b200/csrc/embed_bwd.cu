@@ -151,17 +151,32 @@ int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float
   const int G = (M + kChunk - 1) / kChunk;
   EmbedScratch s = carve(scratch, M, V);
   GPTK_CUDA(cudaMemsetAsync(s.cnt, 0, (size_t)G * V * sizeof(int), st));
-  chunk_rank_kernel<<<G, kChunk, 0, st>>>(idx, M, V, s.cnt, s.rank);
-  GPTK_CUDA(cudaGetLastError());
-  col_scan_kernel<<<(V + 255) / 256, 256, 0, st>>>(s.cnt, G, V, s.total);
-  GPTK_CUDA(cudaGetLastError());
-  offsets_kernel<<<1, 1024, 0, st>>>(s.total, V, s.offs);
-  GPTK_CUDA(cudaGetLastError());
-  scatter_kernel<<<(M + 255) / 256, 256, 0, st>>>(idx, M, V, s.cnt, s.offs, s.rank, s.sorted);
-  GPTK_CUDA(cudaGetLastError());
-  int threads = D / 4 < 256 ? ((D / 4 + 31) / 32) * 32 : 256;
-  segsum_kernel<<<V, threads, 0, st>>>(dx, D, s.total, s.offs, s.sorted, dwte);
-  GPTK_CUDA(cudaGetLastError());
+  {
+    Prof prof(PK_EMBED_BWD, 0, M * 8.0, st);
+    chunk_rank_kernel<<<G, kChunk, 0, st>>>(idx, M, V, s.cnt, s.rank);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    Prof prof(PK_EMBED_BWD, 0, (double)G * V * 8, st);
+    col_scan_kernel<<<(V + 255) / 256, 256, 0, st>>>(s.cnt, G, V, s.total);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    Prof prof(PK_EMBED_BWD, 0, V * 8.0, st);
+    offsets_kernel<<<1, 1024, 0, st>>>(s.total, V, s.offs);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    Prof prof(PK_EMBED_BWD, 0, M * 20.0, st);
+    scatter_kernel<<<(M + 255) / 256, 256, 0, st>>>(idx, M, V, s.cnt, s.offs, s.rank, s.sorted);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    int threads = D / 4 < 256 ? ((D / 4 + 31) / 32) * 32 : 256;
+    Prof prof(PK_EMBED_BWD, 0, (double)M * D * 4 + M * 4.0, st);
+    segsum_kernel<<<V, threads, 0, st>>>(dx, D, s.total, s.offs, s.sorted, dwte);
+    GPTK_CUDA(cudaGetLastError());
+  }
   return ST_OK;
 }
 
@@ -177,6 +192,7 @@ __global__ void pos_bwd_kernel(const float* __restrict__ dx, int B, int T, int D
 
 int launch_pos_bwd(const float* dx, int B, int T, int D, float* dwpe, int accumulate, cudaStream_t st) {
   const long long n = (long long)T * D;
+  Prof prof(PK_EMBED_BWD, 0, (double)B * T * D * 4 + (double)T * D * 8, st);
   pos_bwd_kernel<<<(int)((n + 255) / 256), 256, 0, st>>>(dx, B, T, D, dwpe, accumulate);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;

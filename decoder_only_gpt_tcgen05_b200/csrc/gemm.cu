@@ -120,6 +120,13 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   const int tiles = p.tiles_m * p.tiles_n;
   int grid = num_sms();
   if (grid > tiles) grid = tiles;
+  const double M = p.M, N = p.N, K = p.K;
+  double out_bytes = M * N * 2;
+  if (EPI == EPI_F32 || EPI == EPI_RESID) out_bytes = M * N * 4 * (1 + (p.accumulate || EPI == EPI_RESID));
+  if (EPI == EPI_UP) out_bytes = M * N * 4;
+  if (EPI == EPI_ACTBWD) out_bytes = M * N * 4;
+  if (EPI == EPI_CE_FWD) out_bytes = M * p.tiles_n * 8;
+  Prof prof(PK_GEMM, 2.0 * M * N * K, (M * K + N * K) * 2 + out_bytes, st);
   gemm_kernel<BN, EPI><<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, p);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;

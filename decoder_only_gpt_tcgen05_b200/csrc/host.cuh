@@ -61,6 +61,23 @@ struct Operand {
   int mn_major;
 };
 
+// ---- launch accounting and optional per-launch timing
+// Every kernel launch site constructs a Prof scope: it counts the launch and, while
+// profiling is on, brackets it with CUDA events on the launching stream together with
+// the launch's algorithmic FLOPs and bytes.
+enum ProfKind : int {
+  PK_GEMM = 0, PK_ATTN_FWD, PK_ATTN_BWD_DKV, PK_ATTN_BWD_DQ, PK_NORM_FWD, PK_NORM_BWD, PK_EMBED_FWD,
+  PK_EMBED_BWD, PK_CAST, PK_CE_COMBINE, PK_LOSS, PK_QK, PK_DELTA, PK_COLSUM, PK_MISC, PK_COUNT
+};
+class Prof {
+ public:
+  Prof(int kind, double flops, double bytes, cudaStream_t st);
+  ~Prof();
+ private:
+  int idx_;
+  cudaStream_t st_;
+};
+
 struct GemmParams;
 // C[M,N] = A[M,K] B[N,K]^T with the fused epilogue `epi`; bn = 128 or 256.
 int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st);

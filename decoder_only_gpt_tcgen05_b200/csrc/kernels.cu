@@ -49,6 +49,7 @@ int launch_cast_bf16(const float* src, __nv_bfloat16* dst, long long n, cudaStre
   int grid = num_sms() * 8;
   if (n4 < (long long)grid * 256) grid = cdiv(n4, 256);
   if (grid < 1) return ST_OK;
+  Prof prof(PK_CAST, 0, n * 6.0, st);
   cast_bf16_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst), n4);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -67,6 +68,7 @@ __global__ void rope_table_kernel(float2* cs, int T, int half, double base) {
 }
 
 int launch_rope_table(float2* cs, int T, int half, double base, cudaStream_t st) {
+  Prof prof(PK_MISC, 0, (double)T * half * 8, st);
   rope_table_kernel<<<cdiv((long long)T * half, 256), 256, 0, st>>>(cs, T, half, base);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -103,6 +105,7 @@ int launch_embed_fwd(const int* idx, const float* wte, const float* wpe, float* 
                      cudaStream_t st) {
   int grid = cdiv(M, 8);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_EMBED_FWD, 0, (double)M * D * (wpe ? 12 : 8) + M * 4.0, st);
   embed_fwd_kernel<<<grid, 256, 0, st>>>(idx, wte, wpe, x, M, T, D, V, device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -261,6 +264,7 @@ int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b
     constexpr int NV = decltype(nv)::value;
     int grid = cdiv(M, 8);
     if (grid > num_sms() * 8) grid = num_sms() * 8;
+    Prof prof(PK_NORM_FWD, 0, (double)M * D * 6 + M * 8.0, st);
     norm_fwd_kernel<NV><<<grid, 256, 0, st>>>(x, M, D, g, b, ln, eps, y, ldy, mean, rstd);
     GPTK_CUDA(cudaGetLastError());
     return (int)ST_OK;
@@ -280,6 +284,7 @@ int launch_norm_bwd(const float* dy, const float* x, const float* mean, const fl
     if (smem > 48 * 1024) {
       GPTK_CUDA(cudaFuncSetAttribute(norm_bwd_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
     }
+    Prof prof(PK_NORM_BWD, 0, (double)M * D * (dres_init ? 14 : 18), st);
     norm_bwd_kernel<NV><<<grid, 256, smem, st>>>(dy, x, mean, rstd, g, ln, M, D, dres, dres_init, dres_bf, dg_part,
                                                  db_part);
     GPTK_CUDA(cudaGetLastError());
@@ -302,6 +307,7 @@ __global__ void colreduce_kernel(const float* __restrict__ part, int R, int N, f
 }
 
 int launch_colreduce(const float* part, int R, int N, float* out, int accumulate, cudaStream_t st) {
+  Prof prof(PK_COLSUM, 0, (double)R * N * 4, st);
   colreduce_kernel<<<cdiv(N, 256), 256, 0, st>>>(part, R, N, out, accumulate);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -326,6 +332,7 @@ static int colsum_t(const T* a, long long lda, int M, int N, float* part, int* R
   int rows_per = cdiv(M, kColsumChunks);
   int chunks = cdiv(M, rows_per);
   dim3 grid(cdiv(N, 128), chunks);
+  Prof prof(PK_COLSUM, 0, (double)M * N * sizeof(T), st);
   colsum_kernel<T><<<grid, 128, 0, st>>>(a, lda, M, N, rows_per, part);
   GPTK_CUDA(cudaGetLastError());
   *R = chunks;
@@ -368,6 +375,7 @@ int launch_ce_combine(const float2* part, int ntiles, const float* zy, int M, fl
                       cudaStream_t st) {
   int grid = cdiv(M, 8);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_CE_COMBINE, 0, (double)M * ntiles * 8 + M * 12.0, st);
   ce_combine_kernel<<<grid, 256, 0, st>>>(part, ntiles, zy, M, ell, lse);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -440,10 +448,16 @@ __global__ void loss_final_kernel(const double* part_d, const long long* part_i,
 int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int M, double* part_d,
                        long long* part_i, float* loss, double* sum_nats, long long* sum_bytes, float* bpb,
                        cudaStream_t st) {
-  loss_partial_kernel<<<kLossBlocks, 256, 0, st>>>(ell, targets, token_bytes, M, part_d, part_i);
-  GPTK_CUDA(cudaGetLastError());
-  loss_final_kernel<<<1, 32, 0, st>>>(part_d, part_i, kLossBlocks, M, loss, sum_nats, sum_bytes, bpb);
-  GPTK_CUDA(cudaGetLastError());
+  {
+    Prof prof(PK_LOSS, 0, M * 12.0, st);
+    loss_partial_kernel<<<kLossBlocks, 256, 0, st>>>(ell, targets, token_bytes, M, part_d, part_i);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    Prof prof(PK_LOSS, 0, kLossBlocks * 32.0, st);
+    loss_final_kernel<<<1, 32, 0, st>>>(part_d, part_i, kLossBlocks, M, loss, sum_nats, sum_bytes, bpb);
+    GPTK_CUDA(cudaGetLastError());
+  }
   return ST_OK;
 }
 
@@ -583,6 +597,7 @@ int launch_qk_fwd(const __nv_bfloat16* qkv, const float2* rope_cs, int M, int T,
   long long work = (long long)M * H;
   int grid = cdiv(work, 8);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_QK, 0, (double)M * 3 * H * hd * 4, st);
   if (hd <= 64)
     qk_fwd_kernel<1><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k);
   else if (hd <= 128)
@@ -600,6 +615,7 @@ int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, c
   long long work = (long long)M * H;
   int grid = cdiv(work, 8);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_QK, 0, (double)M * 3 * H * hd * 4 + (qk_norm ? (double)M * 2 * H * hd * 2 : 0), st);
   if (hd <= 64)
     qk_bwd_kernel<1><<<grid, 256, 0, st>>>(dqkv_pad, qkv_pad, rstd_q, rstd_k, rope_cs, M, T, H, hd, hdp, rope, qk_norm,
                                            dqkv);
@@ -640,6 +656,7 @@ int launch_attn_delta(const __nv_bfloat16* o, const __nv_bfloat16* do_pad, int B
   long long work = (long long)B * T * H;
   int grid = cdiv(work, 8);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_DELTA, 0, (double)B * T * H * (hd * 2 + hdp * 2 + 4), st);
   attn_delta_kernel<<<grid, 256, 0, st>>>(o, do_pad, B, T, H, hd, hdp, delta);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -680,6 +697,7 @@ int launch_init_normal(float* params, long long off, long long n, unsigned long 
   if (n <= 0) return ST_OK;
   int grid = cdiv(n, 256);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_MISC, 0, n * 4.0, st);
   init_normal_kernel<<<grid, 256, 0, st>>>(params, off, n, seed, stdv);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
@@ -689,6 +707,7 @@ int launch_fill(float* p, long long n, float value, cudaStream_t st) {
   if (n <= 0) return ST_OK;
   int grid = cdiv(n, 256);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
+  Prof prof(PK_MISC, 0, n * 4.0, st);
   fill_kernel<<<grid, 256, 0, st>>>(p, n, value);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;

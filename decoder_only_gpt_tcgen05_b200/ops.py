@@ -65,3 +65,45 @@ def attention_bwd(fwd: dict, dout: torch.Tensor, B: int, T: int, H: int, hd: int
          _ptr(fwd["rope_cs"]), fwd["o"].data_ptr(), fwd["lse"].data_ptr(), dout.data_ptr(), B, T, H, hd, int(rope),
          int(qk_norm), delta.data_ptr(), dqkv.data_ptr(), _stream(dout))
     return dqkv
+
+
+def lmhead_ce_fwd(x: torch.Tensor, w: torch.Tensor, targets: torch.Tensor):
+    """Per-row (loss, logsumexp) of logits x w^T without storing them.
+    x bf16 [M, D], w bf16 [V, D], targets int32 [M]."""
+    from ._lib import lib
+    M, D = x.shape
+    V = w.shape[0]
+    ell = torch.empty(M, dtype=torch.float32, device=x.device)
+    lse = torch.empty(M, dtype=torch.float32, device=x.device)
+    scratch = torch.empty(lib().gpt_op_lmhead_ce_scratch_bytes(M, V), dtype=torch.uint8, device=x.device)
+    call("gpt_op_lmhead_ce_fwd", x.data_ptr(), w.data_ptr(), targets.data_ptr(), M, D, V, ell.data_ptr(),
+         lse.data_ptr(), scratch.data_ptr(), _stream(x))
+    return ell, lse
+
+
+PROFILE_FAMILIES = ["gemm", "attn_fwd", "attn_bwd_dkv", "attn_bwd_dq", "norm_fwd", "norm_bwd", "embed_fwd",
+                    "embed_bwd", "cast", "ce_combine", "loss", "qk", "delta", "colsum", "misc"]
+
+
+def launch_count() -> int:
+    from ._lib import lib
+    return int(lib().gpt_launch_count())
+
+
+def profile_start() -> None:
+    call("gpt_profile_start")
+
+
+def profile_stop() -> dict:
+    """{family: (ms, launches, flops, bytes)} summed over the launches since profile_start()."""
+    import ctypes as C
+    from ._lib import lib
+    n = len(PROFILE_FAMILIES)
+    ms = (C.c_double * n)()
+    cnt = (C.c_longlong * n)()
+    fl = (C.c_double * n)()
+    by = (C.c_double * n)()
+    rc = lib().gpt_profile_stop(n, ms, cnt, fl, by)
+    if rc != n:
+        raise RuntimeError(lib().gpt_last_error().decode())
+    return {f: (ms[i], cnt[i], fl[i], by[i]) for i, f in enumerate(PROFILE_FAMILIES)}

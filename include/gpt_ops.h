@@ -74,6 +74,35 @@ GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, cons
                                  int T, int H, int hd, int rope, int qk_norm, float* delta, void* dqkv,
                                  void* stream);
 
+/* Fused lm_head + cross-entropy, forward ("nanoGPT" wiki page, model.py
+ * walkthrough: final norm -> lm_head linear to vocab logits; next-token loss
+ * l_m = logsumexp(z_m) - z_m[y_m]).  z = x W^T is produced tile by tile on
+ * the tensor cores and folded into a per-row online logsumexp over each
+ * 256-wide vocab tile; the M x V logits are never written.
+ *   x        bf16 [M, D] (normalised final hidden states), w bf16 [V, D]
+ *   targets  int32 [M]; ell, lse out fp32 [M] (loss and logsumexp per row)
+ *   scratch  caller memory of gpt_op_lmhead_ce_scratch_bytes(M, V) bytes
+ *            (per-row partials of each vocab tile), 256-byte aligned
+ * D must be a multiple of 8. */
+GPT_API size_t gpt_op_lmhead_ce_scratch_bytes(int M, int V);
+GPT_API int gpt_op_lmhead_ce_fwd(const void* x, const void* w, const int32_t* targets, int M, int D, int V,
+                                 float* ell, float* lse, void* scratch, void* stream);
+
+/* Measurement hooks (no counterpart on the pages).
+ * gpt_launch_count: kernels this process has launched through the library.
+ * gpt_profile_start: from now on, bracket every launch with CUDA events on its
+ *   stream (adds a few microseconds per launch).
+ * gpt_profile_stop: synchronise those events and add up, per kernel family
+ *   k < max_kinds, the elapsed milliseconds, launches, algorithmic FLOPs and
+ *   algorithmic bytes (host arrays of max_kinds entries, any may be NULL).
+ *   Returns the number of families, or GPT_ERR_CUDA (with gpt_last_error) if
+ *   an event could not be read.  Families, in order: gemm, attn_fwd,
+ *   attn_bwd_dkv, attn_bwd_dq, norm_fwd, norm_bwd, embed_fwd, embed_bwd,
+ *   cast, ce_combine, loss, qk, delta, colsum, misc. */
+GPT_API unsigned long long gpt_launch_count(void);
+GPT_API int gpt_profile_start(void);
+GPT_API int gpt_profile_stop(int max_kinds, double* ms, long long* count, double* flops, double* bytes);
+
 #ifdef __cplusplus
 }
 #endif
