@@ -32,6 +32,7 @@ SIGNATURES = {
     "gpt_op_attention_fwd": [_P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P],
     "gpt_op_attention_bwd": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P],
     "gpt_op_lmhead_ce_fwd": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P],
+    "gpt_op_lmhead_ce_fwd_noalloc": [_P, _P, _P, _I, _I, _I, _P, _P, _P],
     "gpt_profile_start": [],
     "gpt_profile_stop": [_I, _P, _P, _P, _P],
     "gpt_param_count": [_P, _P],
@@ -61,6 +62,8 @@ def lib():
         L.gpt_launch_count.argtypes = []
         L.gpt_op_lmhead_ce_scratch_bytes.restype = C.c_size_t
         L.gpt_op_lmhead_ce_scratch_bytes.argtypes = [_I, _I]
+        L.gpt_op_lmhead_ce_noalloc_max_scratch_bytes.restype = C.c_size_t
+        L.gpt_op_lmhead_ce_noalloc_max_scratch_bytes.argtypes = []
         for name, args in SIGNATURES.items():
             f = getattr(L, name)
             f.argtypes = args

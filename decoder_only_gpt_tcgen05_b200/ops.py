@@ -81,6 +81,20 @@ def lmhead_ce_fwd(x: torch.Tensor, w: torch.Tensor, targets: torch.Tensor):
     return ell, lse
 
 
+def lmhead_ce_fwd_noalloc(x: torch.Tensor, w: torch.Tensor, targets: torch.Tensor,
+                          ell: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """lmhead_ce_fwd without caller scratch: the library keeps its scratch in a
+    fixed device array, so only the outputs are passed (pre-allocate them to
+    make the call itself allocation-free)."""
+    M, D = x.shape
+    V = w.shape[0]
+    ell = torch.empty(M, dtype=torch.float32, device=x.device) if ell is None else ell
+    lse = torch.empty(M, dtype=torch.float32, device=x.device) if lse is None else lse
+    call("gpt_op_lmhead_ce_fwd_noalloc", x.data_ptr(), w.data_ptr(), targets.data_ptr(), M, D, V, ell.data_ptr(),
+         lse.data_ptr(), _stream(x))
+    return ell, lse
+
+
 PROFILE_FAMILIES = ["gemm", "attn_fwd", "attn_bwd_dkv", "attn_bwd_dq", "norm_fwd", "norm_bwd", "embed_fwd",
                     "embed_bwd", "cast", "ce_combine", "loss", "qk", "delta", "colsum", "misc"]
 

@@ -88,6 +88,25 @@ GPT_API size_t gpt_op_lmhead_ce_scratch_bytes(int M, int V);
 GPT_API int gpt_op_lmhead_ce_fwd(const void* x, const void* w, const int32_t* targets, int M, int D, int V,
                                  float* ell, float* lse, void* scratch, void* stream);
 
+/* The same lm_head + cross-entropy forward for callers that cannot allocate
+ * device memory (the pages have no counterpart: this is a deployment
+ * variant).  A serving or training loop whose device memory is all reserved
+ * up front by its own pool cannot hand out scratch, and a cudaMalloc there
+ * would fail or fragment the pool (and may synchronise the device mid-step).
+ * This entry point takes no scratch argument: it uses a fixed file-scope
+ * device array of gpt_op_lmhead_ce_noalloc_max_scratch_bytes() bytes
+ * (16 MiB) that every GPU loading the library holds until exit, and it calls
+ * no allocator.  It needs gpt_op_lmhead_ce_scratch_bytes(M, V) <= that size
+ * (else GPT_ERR_INVALID_ARG, nothing launched).  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it;
+ * make that first call before any stream capture.  All calls share the one
+ * array, which keeps the last call's contents (the call clears what must
+ * start at zero); calls that overlap on the GPU race on it, so order them on
+ * one stream or with events.  Arguments as gpt_op_lmhead_ce_fwd. */
+GPT_API size_t gpt_op_lmhead_ce_noalloc_max_scratch_bytes(void);
+GPT_API int gpt_op_lmhead_ce_fwd_noalloc(const void* x, const void* w, const int32_t* targets, int M, int D,
+                                         int V, float* ell, float* lse, void* stream);
+
 /* Measurement hooks (no counterpart on the pages).
  * gpt_launch_count: kernels this process has launched through the library.
  * gpt_profile_start: from now on, bracket every launch with CUDA events on its
