@@ -11,7 +11,11 @@
 //   2. per id, an exclusive scan of the chunk counts over chunks (column scan)
 //   3. an exclusive scan of the per-id totals (bucket offsets)
 //   4. scatter: position = offset[id] + earlier chunks' count + rank in chunk
-//   5. one block per id sums its bucket's rows in ascending token order
+//   5. the sorted positions are cut into chunks of 256; each chunk sums the rows of
+//      every id segment inside it in ascending token order and adds complete
+//      buckets straight into dwte; a bucket that crosses chunk edges leaves one
+//      partial per chunk, and the chunk where it starts adds them up in chunk
+//      order (a fixed order, so the result is reproducible)
 #include "host.cuh"
 #include "kernels.cuh"
 
@@ -22,14 +26,16 @@ static constexpr int kChunk = 256;
 static inline long long align256(long long x) { return (x + 255) & ~255LL; }
 
 struct EmbedScratch {
-  int* cnt;     // [G][V]
-  int* total;   // [V]
-  int* offs;    // [V]
-  int* rank;    // [M]
-  int* sorted;  // [M]
+  int* cnt;      // [G][V]
+  int* total;    // [V]
+  int* offs;     // [V]
+  int* rank;     // [M]
+  int* sorted;   // [M]
+  float* head;   // [G][D]  sum of a chunk's first segment when its bucket began in an earlier chunk
+  float* tail;   // [G][D]  sum of a chunk's last segment when its bucket begins here and goes on
 };
 
-static EmbedScratch carve(void* base, int M, int V) {
+static EmbedScratch carve(void* base, int M, int V, int D) {
   const int G = (M + kChunk - 1) / kChunk;
   char* p = static_cast<char*>(base);
   EmbedScratch s;
@@ -42,12 +48,17 @@ static EmbedScratch carve(void* base, int M, int V) {
   s.rank = reinterpret_cast<int*>(p);
   p += align256((long long)M * 4);
   s.sorted = reinterpret_cast<int*>(p);
+  p += align256((long long)M * 4);
+  s.head = reinterpret_cast<float*>(p);
+  p += align256((long long)G * D * 4);
+  s.tail = reinterpret_cast<float*>(p);
   return s;
 }
 
-long long embed_bwd_scratch_bytes(int M, int V) {
+long long embed_bwd_scratch_bytes(int M, int V, int D) {
   const long long G = (M + kChunk - 1) / kChunk;
-  return align256(G * V * 4) + 2 * align256((long long)V * 4) + 2 * align256((long long)M * 4);
+  return align256(G * V * 4) + 2 * align256((long long)V * 4) + 2 * align256((long long)M * 4) +
+         2 * align256(G * D * 4);
 }
 
 __global__ void chunk_rank_kernel(const int* __restrict__ idx, int M, int V, int* __restrict__ cnt,
@@ -124,21 +135,60 @@ __global__ void scatter_kernel(const int* __restrict__ idx, int M, int V, const 
   sorted[offs[id] + cnt[(long long)g * V + id] + rank[m]] = m;
 }
 
-__global__ void segsum_kernel(const float* __restrict__ dx, int D, const int* __restrict__ total,
-                              const int* __restrict__ offs, const int* __restrict__ sorted, float* __restrict__ dwte) {
-  const int v = blockIdx.x;
-  const int n = total[v];
-  if (n == 0) return;
-  const int o = offs[v];
+__device__ __forceinline__ int clamp_id(int id, int V) { return (id < 0 || id >= V) ? 0 : id; }
+
+// One block per chunk of 256 sorted positions; threads stride over float4 columns.
+__global__ void segsum_chunk_kernel(const int* __restrict__ idx, const float* __restrict__ dx, int M, int D, int V,
+                                    const int* __restrict__ total, const int* __restrict__ offs,
+                                    const int* __restrict__ sorted, float* __restrict__ dwte,
+                                    float* __restrict__ head, float* __restrict__ tail) {
+  const int c = blockIdx.x;
+  const int p0 = c * kChunk, p1 = min(M, p0 + kChunk);
   const int D4 = D / 4;
-  for (int c = threadIdx.x; c < D4; c += blockDim.x) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < n; ++i) {
-      const int m = sorted[o + i];
-      const float4 x = reinterpret_cast<const float4*>(dx + (long long)m * D)[c];
-      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+  for (int col = threadIdx.x; col < D4; col += blockDim.x) {
+    int pos = p0;
+    while (pos < p1) {
+      const int id = clamp_id(idx[sorted[pos]], V);
+      const int bstart = offs[id], bend = bstart + total[id];
+      const int send = min(bend, p1);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = pos; q < send; ++q) {
+        const float4 x = reinterpret_cast<const float4*>(dx + (long long)sorted[q] * D)[col];
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+      }
+      if (bstart < p0) {
+        reinterpret_cast<float4*>(head + (long long)c * D)[col] = acc;
+      } else if (bend > p1) {
+        reinterpret_cast<float4*>(tail + (long long)c * D)[col] = acc;
+      } else {
+        float4* w = reinterpret_cast<float4*>(dwte + (long long)id * D) + col;
+        float4 cur = *w;
+        cur.x += acc.x; cur.y += acc.y; cur.z += acc.z; cur.w += acc.w;
+        *w = cur;
+      }
+      pos = send;
     }
-    float4* w = reinterpret_cast<float4*>(dwte + (long long)v * D) + c;
+  }
+}
+
+// Buckets that start in chunk c and run past its end: tail[c] + head[c+1] + ... in chunk order.
+__global__ void segsum_fixup_kernel(const int* __restrict__ idx, int M, int D, int V, const int* __restrict__ total,
+                                    const int* __restrict__ offs, const int* __restrict__ sorted,
+                                    float* __restrict__ dwte, const float* __restrict__ head,
+                                    const float* __restrict__ tail) {
+  const int c = blockIdx.x;
+  const int p0 = c * kChunk, p1 = min(M, p0 + kChunk);
+  const int id = clamp_id(idx[sorted[p1 - 1]], V);
+  const int bstart = offs[id], bend = bstart + total[id];
+  if (bstart < p0 || bend <= p1) return;
+  const int D4 = D / 4;
+  for (int col = threadIdx.x; col < D4; col += blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(tail + (long long)c * D)[col];
+    for (int cc = c + 1; cc * kChunk < bend; ++cc) {
+      const float4 h = reinterpret_cast<const float4*>(head + (long long)cc * D)[col];
+      acc.x += h.x; acc.y += h.y; acc.z += h.z; acc.w += h.w;
+    }
+    float4* w = reinterpret_cast<float4*>(dwte + (long long)id * D) + col;
     float4 cur = *w;
     cur.x += acc.x; cur.y += acc.y; cur.z += acc.z; cur.w += acc.w;
     *w = cur;
@@ -149,7 +199,7 @@ int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float
                      cudaStream_t st) {
   if (D % 4) return set_error(ST_UNSUPPORTED, "embedding backward: n_embd must be a multiple of 4");
   const int G = (M + kChunk - 1) / kChunk;
-  EmbedScratch s = carve(scratch, M, V);
+  EmbedScratch s = carve(scratch, M, V, D);
   GPTK_CUDA(cudaMemsetAsync(s.cnt, 0, (size_t)G * V * sizeof(int), st));
   {
     Prof prof(PK_EMBED_BWD, 0, M * 8.0, st);
@@ -171,10 +221,15 @@ int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float
     scatter_kernel<<<(M + 255) / 256, 256, 0, st>>>(idx, M, V, s.cnt, s.offs, s.rank, s.sorted);
     GPTK_CUDA(cudaGetLastError());
   }
+  const int threads = D / 4 < 256 ? ((D / 4 + 31) / 32) * 32 : 256;
   {
-    int threads = D / 4 < 256 ? ((D / 4 + 31) / 32) * 32 : 256;
-    Prof prof(PK_EMBED_BWD, 0, (double)M * D * 4 + M * 4.0, st);
-    segsum_kernel<<<V, threads, 0, st>>>(dx, D, s.total, s.offs, s.sorted, dwte);
+    Prof prof(PK_EMBED_BWD, 0, (double)M * D * 4 + M * 8.0, st);
+    segsum_chunk_kernel<<<G, threads, 0, st>>>(idx, dx, M, D, V, s.total, s.offs, s.sorted, dwte, s.head, s.tail);
+    GPTK_CUDA(cudaGetLastError());
+  }
+  {
+    Prof prof(PK_EMBED_BWD, 0, (double)G * D * 8, st);
+    segsum_fixup_kernel<<<G, threads, 0, st>>>(idx, M, D, V, s.total, s.offs, s.sorted, dwte, s.head, s.tail);
     GPTK_CUDA(cudaGetLastError());
   }
   return ST_OK;

@@ -1,4 +1,6 @@
 // Host launcher of the tcgen05 GEMM family and the tensor-map / status helpers.
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <string>
 
@@ -72,16 +74,16 @@ static EncodeTiledFn encode_fn() {
 }
 
 int make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-                 uint32_t box_inner, uint32_t box_outer) {
+                 uint32_t box_inner, uint32_t box_outer, int esize) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return set_error(ST_CUDA, "cuTensorMapEncodeTiled is not available");
-  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15))
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * esize) & 15))
     return set_error(ST_INVALID_ARG, "tensor base must be 16-byte aligned and its pitch a multiple of 16 bytes");
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
+  cuuint64_t strides[1] = {ld * (uint64_t)esize};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  CUresult r = fn(map, esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(ST_CUDA, "cuTensorMapEncodeTiled (2d) failed: " + std::to_string((int)r));
@@ -107,14 +109,15 @@ int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, u
 
 // ------------------------------------------------------------ GEMM launcher
 
-template <int BN, int EPI>
-static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p, cudaStream_t st) {
-  using C = GemmCfg<BN>;
+template <int BN, int EPI, bool LONGK>
+static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
+                         const CUtensorMap& tr, const GemmParams& p, cudaStream_t st) {
+  using C = GemmCfg<BN, LONGK>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 63]) {
-    GPTK_CUDA(cudaFuncSetAttribute(gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    GPTK_CUDA(cudaFuncSetAttribute(gemm_kernel<BN, EPI, LONGK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     attr_set[dev & 63] = true;
   }
   const int tiles = p.tiles_m * p.tiles_n;
@@ -123,35 +126,43 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const Gem
   const double M = p.M, N = p.N, K = p.K;
   double out_bytes = M * N * 2;
   if (EPI == EPI_F32 || EPI == EPI_RESID) out_bytes = M * N * 4 * (1 + (p.accumulate || EPI == EPI_RESID));
-  if (EPI == EPI_UP) out_bytes = M * N * 4;
+  if (EPI == EPI_UP) out_bytes = M * N * (p.out ? 4 : 2);
   if (EPI == EPI_ACTBWD) out_bytes = M * N * 4;
   if (EPI == EPI_CE_FWD) out_bytes = M * p.tiles_n * 8;
-  Prof prof(PK_GEMM, 2.0 * M * N * K, (M * K + N * K) * 2 + out_bytes, st);
-  gemm_kernel<BN, EPI><<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, p);
+  Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, 2.0 * M * N * K, (M * K + N * K) * 2 + out_bytes, st);
+  gemm_kernel<BN, EPI, LONGK><<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, tc, tc2, tr, p);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
 
 template <int BN>
-static int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                        cudaStream_t st) {
+static int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                        const CUtensorMap& tc2, const CUtensorMap& tr, const GemmParams& p, cudaStream_t st) {
+  // reductions over all tokens (weight gradients) and over the vocabulary take the deep ring
+  if (epi == EPI_F32 && p.K >= 8192) return launch_gemm_t<BN, EPI_F32, true>(ta, tb, tc, tc2, tr, p, st);
   switch (epi) {
-    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16>(ta, tb, p, st);
-    case EPI_F32: return launch_gemm_t<BN, EPI_F32>(ta, tb, p, st);
-    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID>(ta, tb, p, st);
-    case EPI_QKV: return launch_gemm_t<BN, EPI_QKV>(ta, tb, p, st);
-    case EPI_UP: return launch_gemm_t<BN, EPI_UP>(ta, tb, p, st);
-    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD>(ta, tb, p, st);
-    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD>(ta, tb, p, st);
-    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD>(ta, tb, p, st);
+    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_F32: return launch_gemm_t<BN, EPI_F32, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_UP: return launch_gemm_t<BN, EPI_UP, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD, false>(ta, tb, tc, tc2, tr, p, st);
   }
   return set_error(ST_INVALID_ARG, "unknown GEMM epilogue");
+}
+
+static bool aligned16(const void* ptr, long long ld, int esize) {
+  return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0 && ((ld * esize) & 15) == 0;
 }
 
 int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st) {
   if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return set_error(ST_INVALID_ARG, "GEMM with an empty dimension");
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc, tc2, tr;
+  std::memset(&tc, 0, sizeof(tc));
+  std::memset(&tc2, 0, sizeof(tc2));
+  std::memset(&tr, 0, sizeof(tr));
   if (!A.mn_major) {
     GPTK_TRY(make_tmap_2d(&ta, A.ptr, p.K, p.M, A.ld, 64, 128));
   } else {
@@ -162,13 +173,51 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   } else {
     GPTK_TRY(make_tmap_2d(&tb, B.ptr, p.N, p.K, B.ld, 64, 64));
   }
+  // output / input tensor maps of the TMA epilogue, where the layout allows one
+  p.tma_out = 0;
+  const bool f32out = (epi == EPI_F32 || epi == EPI_RESID);
+  const int es = f32out ? 4 : 2;
+  const unsigned bw = f32out ? 32 : 64;
+  bool ok = epi != EPI_CE_FWD && (epi == EPI_UP ? (p.out == nullptr || aligned16(p.out, p.ldo, 2))
+                                                  : aligned16(p.out, p.ldo, es)) &&
+            (epi != EPI_BF16 || p.hd == p.hdp);
+  if (ok && epi == EPI_RESID) ok = aligned16(p.resid, p.ldr, 4);
+  if (ok && epi == EPI_UP) ok = aligned16(p.out2, p.ldo, 2);
+  if (ok && epi == EPI_ACTBWD) ok = aligned16(p.aux, p.ld_aux, 2);
+  if (ok) {
+    if (p.out) GPTK_TRY(make_tmap_2d(&tc, p.out, p.N, p.M, p.ldo, bw, 32, es));
+    if (epi == EPI_UP) GPTK_TRY(make_tmap_2d(&tc2, p.out2, p.N, p.M, p.ldo, 64, 32, 2));
+    if (epi == EPI_RESID) GPTK_TRY(make_tmap_2d(&tr, p.resid, p.N, p.M, p.ldr, 32, 32, 4));
+    if (epi == EPI_ACTBWD) GPTK_TRY(make_tmap_2d(&tr, p.aux, p.N, p.M, p.ld_aux, 64, 32, 2));
+    p.tma_out = 1;
+  }
   p.a_mn = A.mn_major;
   p.b_mn = B.mn_major;
   p.tiles_m = (p.M + 127) / 128;
   p.tiles_n = (p.N + bn - 1) / bn;
+  {
+    // band height: a few m-tiles whose A rows (128 x K bf16 each) stay within about 48 MB of L2
+    const long long a_band_row = 128LL * p.K * 2;
+    int gm = 8;  // measured best among 8, 16, 32 and the plain order on B200 (d20 shapes)
+    const int gm_l2 = (int)((48LL << 20) / (a_band_row > 0 ? a_band_row : 1));
+    if (gm > gm_l2) gm = gm_l2;
+    // very long K (weight gradients): bands would be too thin to help; keep the plain order,
+    // whose concurrent tiles share B columns while moving through K in step
+    if (gm < 8) gm = p.tiles_m;
+    // tuning override: GPT_GEMM_GROUP_M=<n> forces the band height (0 = plain order)
+    static const int forced = []() {
+      const char* e = std::getenv("GPT_GEMM_GROUP_M");
+      return e ? std::atoi(e) : -1;
+    }();
+    if (forced == 0) gm = p.tiles_m;
+    if (forced > 0) gm = forced < p.tiles_m ? forced : p.tiles_m;
+    if (gm > p.tiles_m) gm = p.tiles_m;
+    p.group_m = gm;
+  }
   p.ctl = device_ctl();
-  if (p.ctl.status == nullptr) return set_error(ST_CUDA, "could not allocate the device status word");
-  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, p, st) : dispatch_epi<128>(epi, ta, tb, p, st);
+  if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
+  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, tc, tc2, tr, p, st)
+                   : dispatch_epi<128>(epi, ta, tb, tc, tc2, tr, p, st);
 }
 
 }  // namespace gptk

@@ -3,11 +3,18 @@
 // One CTA per SM walks output tiles of 128 x BN.  Warp roles:
 //   warp 0      TMA producer: stages 128x64 A and BNx64 B tiles (128-byte swizzle) into a ring
 //   warp 1      one thread issues tcgen05.mma (M=128, N=BN, K=16 per instruction); owns TMEM
-//   warps 2..5  epilogue: tcgen05.ld the accumulator rows (one row per thread) and apply the
-//               fused epilogue of the call (norm scale, bias, RoPE, QK-norm, residual add,
-//               activation, activation gradient, cross-entropy partials or gradient)
+//   warps 2..9  epilogue: tcgen05.ld the accumulator rows (one row per thread; two warps per
+//               TMEM lane quadrant, each taking half of the tile's columns), apply the fused
+//               epilogue of the call (bias, residual add, activation, activation gradient,
+//               cross-entropy partials or gradient), and write through shared memory with TMA
 // The accumulator is double buffered in tensor memory (2 x BN columns) so the epilogue of one
 // tile overlaps the main loop of the next.
+//
+// Epilogue data path: each epilogue warp owns 32 rows x BN/2 columns and two 4 KB staging buffers.  A chunk of
+// 32 fp32 or 64 bf16 columns (128-byte rows) goes registers -> swizzled shared memory -> one TMA
+// tile store (or TMA reduce-add for accumulated gradients), so global writes are whole lines.
+// Epilogue inputs (the residual stream, the saved pre-activation) arrive the same way by TMA
+// load.  Rows and columns past M and N are clipped by the tensor maps.
 //
 // Either operand may be K-major (rows of K contiguous elements: the usual [out,in] weight and
 // [tokens,features] activation layouts) or MN-major (M or N contiguous: what the gradient GEMMs
@@ -20,12 +27,11 @@
 namespace gptk {
 
 enum EpiKind : int {
-  EPI_BF16 = 0,     // out bf16 = acc (+ bias), optional head-padded column map
+  EPI_BF16 = 0,     // out bf16 = acc (+ bias); optional head-padded column map (generic path)
   EPI_F32 = 1,      // out fp32 = acc (+ bias)  or  out += acc  (accumulate)
   EPI_RESID = 2,    // out fp32 = resid + acc (+ bias)
-  EPI_QKV = 3,      // q,k,v bf16 (head padded), + bias, RoPE, per-head RMSNorm of q and k
-  EPI_UP = 4,       // u = acc (+ bias) -> u bf16, h = act(u) bf16
-  EPI_ACTBWD = 5,   // out bf16 = acc * act'(u)
+  EPI_UP = 4,       // u = acc (+ bias) -> h = act(u) bf16 (out2), and u bf16 (out) unless out is null
+  EPI_ACTBWD = 5,   // out bf16 = acc * act'(u); aux is u, or h = relu(u)^2 when act is ReLU^2
   EPI_CE_FWD = 6,   // per-row (max, sum exp) partials over this tile's vocab columns + target logit
   EPI_CE_BWD = 7,   // out bf16 = (softmax - onehot) * scale
 };
@@ -34,6 +40,8 @@ struct GemmParams {
   int M, N, K;
   int a_mn, b_mn;             // 1 = operand stored MN-major
   int tiles_m, tiles_n;
+  int tma_out;                // 1 = epilogue writes through the output tensor maps (fast path)
+  int group_m;                // tile order: bands of group_m m-tiles sweep every n-tile
   DevCtl ctl;
   // generic output
   void* out;
@@ -46,35 +54,32 @@ struct GemmParams {
   const __nv_bfloat16* aux;   // EPI_ACTBWD: u
   long long ld_aux;
   int act;                    // 0 GELU(erf), 1 ReLU^2
-  // head-padded layout of q/k/v (and of attention-gradient inputs): column c of a D-wide
-  // block maps to (c / hd) * hdp + c % hd
+  // head-padded output layout (generic BF16 path): column c maps to (c / hd) * hdp + c % hd
   int hd, hdp;
-  // QKV epilogue
-  int d_model, n_head, T;
-  int rope, qk_norm;
-  float eps;
-  const float2* rope_cs;      // [T][hd/2] (cos, sin)
-  float* rstd_q;              // [M][H]
-  float* rstd_k;
   // cross-entropy
   const int* targets;         // [M]
   float2* ce_part;            // [M][tiles_n]  (max log2, sum exp2)
   float* ce_zy;               // [M] target logit
   const float* ce_lse;        // [M] natural-log logsumexp (backward)
   float ce_scale;             // 1/M_total (backward)
+  int prof_kind;              // host only: profiler family of this call (0 = generic GEMM)
 };
 
-template <int BN>
+// LONGK: the variant for very long reductions (weight gradients over all tokens), where the
+// epilogue is rare and a deeper TMA ring matters more than epilogue parallelism.
+template <int BN, bool LONGK = false>
 struct GemmCfg {
   static constexpr int BM = 128;
   static constexpr int BK = 64;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int STAGES = LONGK ? ((BN == 256) ? 4 : 6) : ((BN == 256) ? 3 : 5);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_WARPS = LONGK ? 4 : 8;             // one or two per TMEM lane quadrant
+  static constexpr int STAGING_BYTES = EPI_WARPS * 2 * 4096;  // 2 buffers of 32 rows x 128 B per warp
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-  static constexpr int THREADS = 192;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
 };
 
 // --------------------------------------------------------------- epilogue helpers
@@ -89,224 +94,165 @@ __device__ __forceinline__ float act_fwd(float u, int act) {
 
 __device__ __forceinline__ float act_grad(float u, int act) {
   if (act == 1) return 2.f * fmaxf(u, 0.f);
+  if (act == 2) return 2.f * sqrtf(fmaxf(u, 0.f));  // ReLU^2 given h = relu(u)^2: 2 relu(u) = 2 sqrt(h)
   // d/du of 0.5 u (1 + erf(u/sqrt2)) = 0.5 (1 + erf(u/sqrt2)) + u * exp(-u^2/2) / sqrt(2 pi)
   return 0.5f * (1.f + erff(u * 0.70710678118654752f)) + u * expf(-0.5f * u * u) * 0.3989422804014327f;
 }
 
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 w;
-    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    d[q] = w;
-  }
-}
-
-__device__ __forceinline__ void add_bias32(float (&v)[32], const float* bias, int col0, int N) {
+__device__ __forceinline__ void add_bias32(float* v, const float* bias, int col0, int N) {
   if (bias == nullptr) return;
 #pragma unroll
   for (int j = 0; j < 32; ++j)
     if (col0 + j < N) v[j] += __ldg(bias + col0 + j);
 }
 
-// Plain column-chunk epilogues: one 32-column chunk of one row.
+// 16-byte unit `u` of row r in a 128-byte-swizzled staging buffer
+__device__ __forceinline__ uint32_t stg_addr(uint32_t base, int r, int u) {
+  return base + r * 128 + ((u ^ (r & 7)) << 4);
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
+// row r of a staging buffer <- 32 fp32 values
+__device__ __forceinline__ void stage_f32(uint32_t buf, int r, const float* v) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    sts128(stg_addr(buf, r, u), __float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
+           __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3]));
+}
+// row r of a staging buffer <- 64 bf16 values
+__device__ __forceinline__ void stage_bf16(uint32_t buf, int r, const float* v) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    sts128(stg_addr(buf, r, u), pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+           pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+}
+__device__ __forceinline__ void unstage_f32(uint32_t buf, int r, float* v) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    uint4 x = lds128(stg_addr(buf, r, u));
+    v[4 * u] = __uint_as_float(x.x);
+    v[4 * u + 1] = __uint_as_float(x.y);
+    v[4 * u + 2] = __uint_as_float(x.z);
+    v[4 * u + 3] = __uint_as_float(x.w);
+  }
+}
+__device__ __forceinline__ void unstage_bf16(uint32_t buf, int r, float* v) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    uint4 x = lds128(stg_addr(buf, r, u));
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[8 * u + 2 * k] = __uint_as_float(w[k] << 16);
+      v[8 * u + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+  }
+}
+
+// Generic (per-thread store) epilogue for one 32-column chunk of one row; used where the
+// output is not a plain 2-D tile (head-padded layouts) or cannot be described by a tensor map.
 template <int EPI>
-__device__ __forceinline__ void epi_chunk(const GemmParams& p, float (&v)[32], int row, int col0, bool row_ok) {
-  const bool full = (col0 + 32 <= p.N);
+__device__ __forceinline__ void epi_chunk_generic(const GemmParams& p, float* v, int row, int col0, bool row_ok) {
   if (EPI == EPI_BF16) {
     add_bias32(v, p.bias, col0, p.N);
     if (!row_ok) return;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo;
-    if (p.hd == p.hdp && full && (p.ldo % 8) == 0) {
-      store_bf16x32(out + col0, v);
-    } else {
-      for (int j = 0; j < 32; ++j) {
-        int c = col0 + j;
-        if (c < p.N) out[(c / p.hd) * p.hdp + c % p.hd] = __float2bfloat16_rn(v[j]);
-      }
+    for (int j = 0; j < 32; ++j) {
+      int c = col0 + j;
+      if (c < p.N) out[(c / p.hd) * p.hdp + c % p.hd] = __float2bfloat16_rn(v[j]);
     }
   } else if (EPI == EPI_F32) {
     add_bias32(v, p.bias, col0, p.N);
     if (!row_ok) return;
     float* out = reinterpret_cast<float*>(p.out) + (long long)row * p.ldo;
-    if (full && (p.ldo % 4) == 0) {
-      float4* o4 = reinterpret_cast<float4*>(out + col0);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float4 w = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        if (p.accumulate) {
-          float4 o = o4[q];
-          w.x += o.x; w.y += o.y; w.z += o.z; w.w += o.w;
-        }
-        o4[q] = w;
-      }
-    } else {
-      for (int j = 0; j < 32; ++j) {
-        int c = col0 + j;
-        if (c < p.N) out[c] = p.accumulate ? out[c] + v[j] : v[j];
-      }
+    for (int j = 0; j < 32; ++j) {
+      int c = col0 + j;
+      if (c < p.N) out[c] = p.accumulate ? out[c] + v[j] : v[j];
     }
   } else if (EPI == EPI_RESID) {
     add_bias32(v, p.bias, col0, p.N);
     if (!row_ok) return;
     float* out = reinterpret_cast<float*>(p.out) + (long long)row * p.ldo;
     const float* res = p.resid + (long long)row * p.ldr;
-    if (full && (p.ldo % 4) == 0 && (p.ldr % 4) == 0) {
-      float4* o4 = reinterpret_cast<float4*>(out + col0);
-      const float4* r4 = reinterpret_cast<const float4*>(res + col0);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float4 r = r4[q];
-        o4[q] = make_float4(r.x + v[4 * q], r.y + v[4 * q + 1], r.z + v[4 * q + 2], r.w + v[4 * q + 3]);
-      }
-    } else {
-      for (int j = 0; j < 32; ++j) {
-        int c = col0 + j;
-        if (c < p.N) out[c] = res[c] + v[j];
-      }
+    for (int j = 0; j < 32; ++j) {
+      int c = col0 + j;
+      if (c < p.N) out[c] = res[c] + v[j];
     }
   } else if (EPI == EPI_UP) {
     add_bias32(v, p.bias, col0, p.N);
     if (!row_ok) return;
-    __nv_bfloat16* u = reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo;
+    __nv_bfloat16* u = p.out ? reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo : nullptr;
     __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(p.out2) + (long long)row * p.ldo;
-    float hv[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) hv[j] = act_fwd(v[j], p.act);
-    if (full && (p.ldo % 8) == 0) {
-      store_bf16x32(u + col0, v);
-      store_bf16x32(h + col0, hv);
-    } else {
-      for (int j = 0; j < 32; ++j) {
-        int c = col0 + j;
-        if (c < p.N) {
-          u[c] = __float2bfloat16_rn(v[j]);
-          h[c] = __float2bfloat16_rn(hv[j]);
-        }
+    for (int j = 0; j < 32; ++j) {
+      int c = col0 + j;
+      if (c < p.N) {
+        if (u) u[c] = __float2bfloat16_rn(v[j]);
+        h[c] = __float2bfloat16_rn(act_fwd(v[j], p.act));
       }
     }
   } else if (EPI == EPI_ACTBWD) {
     if (!row_ok) return;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo;
     const __nv_bfloat16* u = p.aux + (long long)row * p.ld_aux;
-    if (full && (p.ldo % 8) == 0 && (p.ld_aux % 8) == 0) {
-      const uint4* u4 = reinterpret_cast<const uint4*>(u + col0);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 w = u4[q];
-        const __nv_bfloat16* ub = reinterpret_cast<const __nv_bfloat16*>(&w);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[8 * q + e] *= act_grad(__bfloat162float(ub[e]), p.act);
-      }
-      store_bf16x32(out + col0, v);
-    } else {
-      for (int j = 0; j < 32; ++j) {
-        int c = col0 + j;
-        if (c < p.N) out[c] = __float2bfloat16_rn(v[j] * act_grad(__bfloat162float(u[c]), p.act));
-      }
+    for (int j = 0; j < 32; ++j) {
+      int c = col0 + j;
+      if (c < p.N) out[c] = __float2bfloat16_rn(v[j] * act_grad(__bfloat162float(u[c]), p.act));
     }
   } else if (EPI == EPI_CE_BWD) {
     if (!row_ok) return;
     const float lse2 = p.ce_lse[row] * 1.4426950408889634f;
     const int y = p.targets[row];
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo;
-#pragma unroll
     for (int j = 0; j < 32; ++j) {
       int c = col0 + j;
       float g = ex2_approx(fmaf(v[j], 1.4426950408889634f, -lse2));
       if (c == y) g -= 1.f;
-      v[j] = g * p.ce_scale;
-    }
-    if (full && (p.ldo % 8) == 0) {
-      store_bf16x32(out + col0, v);
-    } else {
-      for (int j = 0; j < 32; ++j)
-        if (col0 + j < p.N) out[col0 + j] = __float2bfloat16_rn(v[j]);
+      if (c < p.N) out[c] = __float2bfloat16_rn(g * p.ce_scale);
     }
   }
 }
 
-// QKV epilogue for one head of q or k: RoPE on pairs (i, i + hd/2), then per-head RMSNorm.
-// taddr points at this thread's row, column of the head's first element.
-__device__ __forceinline__ void epi_qk_head(const GemmParams& p, uint32_t taddr, int row, bool row_ok, int col,
-                                            int sect, int head) {
-  const int hd = p.hd;
-  const float* bias = p.bias ? p.bias + col : nullptr;
-  float rstd = 1.f;
-  if (p.qk_norm) {
-    float ss = 0.f;
-    for (int c = 0; c < hd; c += 32) {
-      float v[32];
-      tmem_ld32(taddr + c, v);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        float x = v[j] + (bias ? __ldg(bias + c + j) : 0.f);
-        ss = fmaf(x, x, ss);
-      }
-    }
-    rstd = rsqrtf(ss / (float)hd + p.eps);
-    if (row_ok) (sect == 0 ? p.rstd_q : p.rstd_k)[(long long)row * p.n_head + head] = rstd;
-  }
-  const int half = hd / 2;
-  const int t = row % p.T;
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo +
-                       (long long)sect * p.n_head * p.hdp + (long long)head * p.hdp;
-  for (int c = 0; c < half; c += 32) {
-    float x1[32], x2[32];
-    tmem_ld32(taddr + c, x1);
-    tmem_ld32(taddr + half + c, x2);
-    if (bias) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x1[j] += __ldg(bias + c + j);
-        x2[j] += __ldg(bias + half + c + j);
-      }
-    }
-    if (p.rope) {
-      const float2* cs = p.rope_cs + (long long)t * half + c;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        float2 e = __ldg(cs + j);
-        float a = x1[j], b = x2[j];
-        x1[j] = (a * e.x - b * e.y) * rstd;
-        x2[j] = (a * e.y + b * e.x) * rstd;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        x1[j] *= rstd;
-        x2[j] *= rstd;
-      }
-    }
-    if (row_ok) {
-      store_bf16x32(out + c, x1);
-      store_bf16x32(out + half + c, x2);
-    }
-  }
+// Tile t -> (tm, tn).  Tiles are taken in bands of group_m m-tiles; inside a band the m index
+// runs fastest, and the band sweeps every n-tile before the next band starts, so the A rows
+// of a band stay in L2 while all of B passes by.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& tm, int& tn) {
+  const int per_band = p.group_m * p.tiles_n;
+  const int band = tile / per_band;
+  const int first = band * p.group_m;
+  const int gm = min(p.group_m, p.tiles_m - first);
+  const int local = tile - band * per_band;
+  tm = first + local % gm;
+  tn = local / gm;
 }
 
 // --------------------------------------------------------------- the kernel
 
-template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, int EPI, bool LONGK>
+__global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<BN>;
+                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
+                const __grid_constant__ CUtensorMap tmR, const __grid_constant__ GemmParams p) {
+  using C = GemmCfg<BN, LONGK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
   uint64_t* tempty = bars + 2 * C::STAGES + 2;
   uint64_t* drain = bars + 2 * C::STAGES + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5);
+  uint64_t* inbar = bars + 2 * C::STAGES + 5;  // [EPI_WARPS][2 buffers]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5 + 2 * C::EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -319,9 +265,10 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], C::EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 2 * C::EPI_WARPS; ++i) mbar_init(&inbar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
@@ -346,8 +293,8 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t pending = 0;  // stages with a load in flight that the MMA has not yet released
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      const int tm = tile % p.tiles_m;
-      const int tn = tile / p.tiles_m;
+      int tm, tn;
+      tile_coords(p, tile, tm, tn);
       for (int kb = 0; kb < num_k; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctl, abort_flag, 1)) {
           ok = false;
@@ -361,7 +308,8 @@ __global__ void __launch_bounds__(192, 1)
           tma_load_2d(a, &tmA, &full[stage], kb * C::BK, tm * C::BM);
         } else {
 #pragma unroll
-          for (int c = 0; c < C::BM / 64; ++c) tma_load_2d(a + c * 8192, &tmA, &full[stage], tm * C::BM + c * 64, kb * C::BK);
+          for (int c = 0; c < C::BM / 64; ++c)
+            tma_load_2d(a + c * 8192, &tmA, &full[stage], tm * C::BM + c * 64, kb * C::BK);
         }
         if (!p.b_mn) {
           tma_load_2d(b, &tmB, &full[stage], kb * C::BK, tn * BN);
@@ -378,13 +326,12 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (!ok) {
       // drain the copies still in flight before the CTA goes away (bounded as well)
-      DevCtl c2 = p.ctl;
       volatile int never = 0;
       for (int s = 0; s < C::STAGES; ++s) {
         if (!(pending & (1u << s))) continue;
         // stage s was issued in the current or the previous lap of the ring
         uint32_t ph = (s < stage) ? phase : (phase ^ 1u);
-        mbar_wait(&full[s], ph, c2, &never, 2);
+        mbar_wait(&full[s], ph, p.ctl, &never, 2);
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -427,7 +374,6 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) break;
       umma_commit(&tfull[acc]);
-      issued = true;
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -442,78 +388,174 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue
     const int quad = warp & 3;
+    const int ew = warp - 2;
+    const int chalf = ew >> 2;  // which part of the tile's columns this warp writes
     const int r_in_tile = quad * 32 + lane;
+    uint8_t* stg_ptr = staging + ew * 8192;
+    const uint32_t stg = smem_u32(stg_ptr);
+    uint64_t* ibar = inbar + 2 * ew;
+    uint32_t in_uses = 0;  // bit b flips on every use of input buffer b (its mbarrier parity)
+    int chunk_ctr = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
+    constexpr bool F32OUT = (EPI == EPI_F32 || EPI == EPI_RESID);
+    constexpr int CW = F32OUT ? 32 : 64;
+    constexpr bool HAS_IN = (EPI == EPI_RESID || EPI == EPI_ACTBWD);
+    constexpr int HALF = BN * 4 / C::EPI_WARPS;  // columns per epilogue warp
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int tm = tile % p.tiles_m;
-      const int tn = tile / p.tiles_m;
+      int tm, tn;
+      tile_coords(p, tile, tm, tn);
+      const int row = tm * 128 + r_in_tile;
+      const int row0 = tm * 128 + quad * 32;
+      const bool row_ok = row < p.M;
+      const int c_begin = chalf * HALF;
+      const int n0 = tn * BN;
+      const bool tma = p.tma_out && EPI != EPI_CE_FWD;
+      // the first input chunk of the tile can load while the main loop still runs
+      if (HAS_IN && tma && n0 + c_begin < p.N && lane == 0) {
+        const int b = chunk_ctr & 1;
+        bulk_wait_read<1>();
+        mbar_expect_tx(&ibar[b], 4096);
+        tma_load_2d(stg_ptr + b * 4096, &tmR, &ibar[b], n0 + c_begin, row0);
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, p.ctl, abort_flag, 5)) break;
       tc_fence_after();
-      const int row = tm * 128 + r_in_tile;
-      const bool row_ok = row < p.M;
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
-      const int n0 = tn * BN;
-      if (EPI == EPI_QKV) {
-        const int D = p.d_model;
-        // a tile never straddles q/k/v sections when hd divides BN and D
-        for (int c = 0; c < BN; c += 32) {
-          const int col = n0 + c;
-          if (col >= p.N) break;
-          const int sect = col / D;
-          const int within = col - sect * D;
-          if (sect < 2 && (p.rope || p.qk_norm)) {
-            if (within % p.hd == 0 && c + p.hd <= BN) {
-              epi_qk_head(p, trow + c, row, row_ok, col, sect, within / p.hd);
-            }
-            continue;  // columns of a head are handled by the head's first chunk
-          }
-          float v[32];
-          tmem_ld32(trow + c, v);
-          add_bias32(v, p.bias, col, p.N);
-          if (row_ok) {
-            __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.out) + (long long)row * p.ldo;
+      bool ok = true;
+      if (EPI == EPI_CE_FWD) {
+        // both warps of a quadrant see the whole row; the lower-half warp reduces it
+        if (chalf == 0) {
+          const int y = row_ok ? p.targets[row] : -1;
+          float m2 = -INFINITY, s = 0.f;
+          for (int c = 0; c < BN; c += 32) {
+            float v[32];
+            tmem_ld32(trow + c, v);
+            const int col0 = n0 + c;
+            float cm = -INFINITY;
+#pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const int cc = col + j;
-              if (cc >= p.N) break;
-              const int s = cc / D, w = cc - s * D;
-              out[(long long)s * p.n_head * p.hdp + (w / p.hd) * p.hdp + (w % p.hd)] = __float2bfloat16_rn(v[j]);
+              v[j] = (col0 + j < p.N) ? v[j] * 1.4426950408889634f : -INFINITY;
+              cm = fmaxf(cm, v[j]);
+            }
+            if (y >= col0 && y < col0 + 32 && row_ok) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j == y) p.ce_zy[row] = v[j] * 0.6931471805599453f;
+            }
+            if (cm != -INFINITY) {
+              const float mn = fmaxf(m2, cm);
+              float cs = 0.f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) cs += ex2_approx(v[j] - mn);
+              s = s * ex2_approx(m2 - mn) + cs;
+              m2 = mn;
             }
           }
+          if (row_ok) p.ce_part[(long long)row * p.tiles_n + tn] = make_float2(m2, s);
         }
-      } else if (EPI == EPI_CE_FWD) {
-        const int y = row_ok ? p.targets[row] : -1;
-        float m2 = -INFINITY, s = 0.f;
-        for (int c = 0; c < BN; c += 32) {
+      } else if (!tma) {
+        for (int c = c_begin; c < c_begin + HALF; c += 32) {
           float v[32];
           tmem_ld32(trow + c, v);
-          const int col0 = n0 + c;
-          float cm = -INFINITY;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            v[j] = (col0 + j < p.N) ? v[j] * 1.4426950408889634f : -INFINITY;
-            cm = fmaxf(cm, v[j]);
-          }
-          if (y >= col0 && y < col0 + 32 && row_ok) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j == y) p.ce_zy[row] = v[j] * 0.6931471805599453f;
-          }
-          if (cm != -INFINITY) {
-            const float mn = fmaxf(m2, cm);
-            float cs = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) cs += ex2_approx(v[j] - mn);
-            s = s * ex2_approx(m2 - mn) + cs;
-            m2 = mn;
-          }
+          epi_chunk_generic<EPI>(p, v, row, n0 + c, row_ok);
         }
-        if (row_ok) p.ce_part[(long long)row * p.tiles_n + tn] = make_float2(m2, s);
       } else {
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          tmem_ld32(trow + c, v);
-          epi_chunk<EPI>(p, v, row, n0 + c, row_ok);
+        // TMA path: chunks of 32 fp32 or 64 bf16 columns (128-byte staging rows)
+        for (int c = c_begin; c < c_begin + HALF; c += CW) {
+          const int col0 = n0 + c;
+          if (col0 >= p.N) break;
+          const int b = chunk_ctr & 1;
+          const uint32_t buf = stg + b * 4096;
+          const bool two_out = (EPI == EPI_UP) && p.out != nullptr;
+          if (!HAS_IN) {
+            // the staging buffer must no longer be read by an earlier store
+            if (lane == 0) {
+              if (two_out) bulk_wait_read<0>();
+              else bulk_wait_read<1>();
+            }
+            __syncwarp();
+          }
+          float v[CW];
+          tmem_ld32(trow + c, *reinterpret_cast<float(*)[32]>(&v[0]));
+          if (CW == 64) tmem_ld32(trow + c + 32, *reinterpret_cast<float(*)[32]>(&v[32 % CW]));
+          if (EPI != EPI_ACTBWD && EPI != EPI_CE_BWD) {
+            add_bias32(v, p.bias, col0, p.N);
+            if (CW == 64) add_bias32(v + (32 % CW), p.bias, col0 + 32, p.N);
+          }
+          if (HAS_IN) {
+            if (!mbar_wait(&ibar[b], (in_uses >> b) & 1u, p.ctl, abort_flag, 7)) {
+              ok = false;
+              break;
+            }
+            in_uses ^= 1u << b;
+            float in[CW];
+            if (EPI == EPI_RESID) {
+              unstage_f32(buf, lane, in);
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] += in[j];
+            } else if (p.act == 2) {  // EPI_ACTBWD, ReLU^2 from h: 2 relu(u) = 2 sqrt(h)
+              unstage_bf16(buf, lane, in);
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] *= 2.f * sqrtf(fmaxf(in[j], 0.f));
+            } else if (p.act == 1) {  // ReLU^2 from u
+              unstage_bf16(buf, lane, in);
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] *= 2.f * fmaxf(in[j], 0.f);
+            } else {  // GELU from u
+              unstage_bf16(buf, lane, in);
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] *= act_grad(in[j], 0);
+            }
+          }
+          if (EPI == EPI_CE_BWD) {
+            const float lse2 = row_ok ? p.ce_lse[row] * 1.4426950408889634f : 0.f;
+            const int y = row_ok ? p.targets[row] : -1;
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+              float gv = ex2_approx(fmaf(v[j], 1.4426950408889634f, -lse2));
+              if (col0 + j == y) gv -= 1.f;
+              v[j] = gv * p.ce_scale;
+            }
+          }
+          if (EPI == EPI_UP) {
+            // h = act(u) to buffer b (tensor map tmC2); u itself to buffer b^1 when kept
+            if (two_out) stage_bf16(stg + (b ^ 1) * 4096, lane, v);
+            if (p.act == 1) {
+#pragma unroll
+              for (int j = 0; j < CW; ++j) {
+                const float r = fmaxf(v[j], 0.f);
+                v[j] = r * r;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] = act_fwd(v[j], 0);
+            }
+            stage_bf16(buf, lane, v);
+          } else if (F32OUT) {
+            stage_f32(buf, lane, v);
+          } else {
+            stage_bf16(buf, lane, v);
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (EPI == EPI_UP) {
+              tma_store_2d(&tmC2, stg_ptr + b * 4096, col0, row0);
+              if (two_out) tma_store_2d(&tmC, stg_ptr + (b ^ 1) * 4096, col0, row0);
+            } else if (EPI == EPI_F32 && p.accumulate) {
+              tma_reduce_add_2d(&tmC, stg_ptr + b * 4096, col0, row0);
+            } else {
+              tma_store_2d(&tmC, stg_ptr + b * 4096, col0, row0);
+            }
+            bulk_commit();
+            // prefetch the next input chunk into the other buffer once its last store has read it
+            if (HAS_IN && c + CW < c_begin + HALF && col0 + CW < p.N) {
+              bulk_wait_read<1>();
+              mbar_expect_tx(&ibar[b ^ 1], 4096);
+              tma_load_2d(stg_ptr + (b ^ 1) * 4096, &tmR, &ibar[b ^ 1], col0 + CW, row0);
+            }
+          }
+          ++chunk_ctr;
         }
       }
       tc_fence_before();
@@ -523,7 +565,9 @@ __global__ void __launch_bounds__(192, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+      if (!ok) break;
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   __syncthreads();

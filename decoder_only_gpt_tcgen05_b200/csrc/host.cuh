@@ -44,10 +44,11 @@ const char* last_error();
 DevCtl device_ctl();
 int num_sms();
 
-// 2-D bf16 tensor map with 128-byte swizzle: inner extent `inner` (contiguous),
-// outer extent `outer`, row pitch `ld` elements, box {box_inner, box_outer}.
+// 2-D tensor map with 128-byte swizzle: inner extent `inner` (contiguous), outer
+// extent `outer`, row pitch `ld` elements, box {box_inner, box_outer}; elements are
+// bf16 (esize 2) or fp32 (esize 4).
 int make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-                 uint32_t box_inner, uint32_t box_outer);
+                 uint32_t box_inner, uint32_t box_outer, int esize = 2);
 // 3-D bf16 tensor map: dims {d0 (contiguous), d1, d2}, pitches (elements) s1, s2, box {b0, b1, b2}.
 int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                  uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
@@ -67,7 +68,10 @@ struct Operand {
 // the launch's algorithmic FLOPs and bytes.
 enum ProfKind : int {
   PK_GEMM = 0, PK_ATTN_FWD, PK_ATTN_BWD_DKV, PK_ATTN_BWD_DQ, PK_NORM_FWD, PK_NORM_BWD, PK_EMBED_FWD,
-  PK_EMBED_BWD, PK_CAST, PK_CE_COMBINE, PK_LOSS, PK_QK, PK_DELTA, PK_COLSUM, PK_MISC, PK_COUNT
+  PK_EMBED_BWD, PK_CAST, PK_CE_COMBINE, PK_LOSS, PK_QK, PK_DELTA, PK_COLSUM, PK_MISC,
+  // GEMM roles (the model tags each GEMM call; untagged calls count as PK_GEMM)
+  PK_GEMM_QKV, PK_GEMM_O, PK_GEMM_UP, PK_GEMM_DOWN, PK_GEMM_LM_FWD, PK_GEMM_LM_BWD, PK_GEMM_DGRAD,
+  PK_GEMM_WGRAD, PK_COUNT
 };
 class Prof {
  public:

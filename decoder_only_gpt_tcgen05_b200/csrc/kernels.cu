@@ -114,9 +114,9 @@ int launch_embed_fwd(const int* idx, const float* wte, const float* wpe, float* 
 // ------------------------------------------------------------------ norms
 // One warp per row.  A row of D <= 128*NV floats lives in registers (NV float4 per lane).
 
-template <int NV>
+template <int NV, bool LN>
 __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const float* __restrict__ g,
-                                const float* __restrict__ b, int ln, float eps, __nv_bfloat16* __restrict__ y,
+                                const float* __restrict__ b, float eps, __nv_bfloat16* __restrict__ y,
                                 long long ldy, float* __restrict__ mean_out, float* __restrict__ rstd_out) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -132,7 +132,7 @@ __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const
       s += v[i].x + v[i].y + v[i].z + v[i].w;
     }
     float mu = 0.f;
-    if (ln) mu = warp_sum(s) / D;
+    if (LN) mu = warp_sum(s) / D;
     float ss = 0.f;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
@@ -145,7 +145,7 @@ __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const
     const float r = rsqrtf(warp_sum(ss) / D + eps);
     if (lane == 0) {
       rstd_out[m] = r;
-      if (ln) mean_out[m] = mu;
+      if (LN) mean_out[m] = mu;
     }
     uint2* yr = reinterpret_cast<uint2*>(y + (long long)m * ldy);
 #pragma unroll
@@ -153,7 +153,7 @@ __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const
       int c = i * 32 + lane;
       if (c < D4) {
         float4 o = make_float4((v[i].x - mu) * r, (v[i].y - mu) * r, (v[i].z - mu) * r, (v[i].w - mu) * r);
-        if (ln) {
+        if (LN) {
           float4 gg = __ldg(reinterpret_cast<const float4*>(g) + c);
           o.x *= gg.x; o.y *= gg.y; o.z *= gg.z; o.w *= gg.w;
           if (b) {
@@ -167,24 +167,26 @@ __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const
   }
 }
 
-template <int NV>
+template <int NV, bool LN>
 __global__ void norm_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
                                 const float* __restrict__ mean, const float* __restrict__ rstd,
-                                const float* __restrict__ g, int ln, int M, int D, float* __restrict__ dres,
-                                int dres_init, __nv_bfloat16* __restrict__ dres_bf, float* __restrict__ dg_part,
+                                const float* __restrict__ g, int M, int D, float* __restrict__ dres, int dres_init,
+                                __nv_bfloat16* __restrict__ dres_bf, float* __restrict__ dg_part,
                                 float* __restrict__ db_part) {
-  extern __shared__ float red[];  // [warps][2][D] when ln
+  extern __shared__ float red[];  // [warps][2][D] (LayerNorm only)
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int D4 = D / 4;
-  float4 dg[NV], db[NV];
+  float4 dg[LN ? NV : 1], db[LN ? NV : 1];
+  if (LN) {
 #pragma unroll
-  for (int i = 0; i < NV; ++i) dg[i] = db[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < NV; ++i) dg[i] = db[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   for (int m = blockIdx.x * warps + w; m < M; m += gridDim.x * warps) {
     const float4* xr = reinterpret_cast<const float4*>(x + (long long)m * D);
     const float4* gr = reinterpret_cast<const float4*>(dy + (long long)m * D);
-    const float mu = ln ? mean[m] : 0.f;
+    const float mu = LN ? mean[m] : 0.f;
     const float r = rstd[m];
     float4 xh[NV], gh[NV];
     float s1 = 0.f, s2 = 0.f;
@@ -194,20 +196,20 @@ __global__ void norm_bwd_kernel(const float* __restrict__ dy, const float* __res
       if (c < D4) {
         float4 xv = xr[c], gv = gr[c];
         xh[i] = make_float4((xv.x - mu) * r, (xv.y - mu) * r, (xv.z - mu) * r, (xv.w - mu) * r);
-        if (ln) {
+        if (LN) {
           db[i].x += gv.x; db[i].y += gv.y; db[i].z += gv.z; db[i].w += gv.w;
           dg[i].x += gv.x * xh[i].x; dg[i].y += gv.y * xh[i].y; dg[i].z += gv.z * xh[i].z; dg[i].w += gv.w * xh[i].w;
           float4 gg = __ldg(reinterpret_cast<const float4*>(g) + c);
           gv.x *= gg.x; gv.y *= gg.y; gv.z *= gg.z; gv.w *= gg.w;
+          s1 += gv.x + gv.y + gv.z + gv.w;
         }
         gh[i] = gv;
-        s1 += gv.x + gv.y + gv.z + gv.w;
         s2 += gv.x * xh[i].x + gv.y * xh[i].y + gv.z * xh[i].z + gv.w * xh[i].w;
       } else {
         xh[i] = gh[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    const float m1 = ln ? warp_sum(s1) / D : 0.f;
+    const float m1 = LN ? warp_sum(s1) / D : 0.f;
     const float m2 = warp_sum(s2) / D;
     float4* dr = reinterpret_cast<float4*>(dres + (long long)m * D);
     uint2* db16 = reinterpret_cast<uint2*>(dres_bf + (long long)m * D);
@@ -226,7 +228,7 @@ __global__ void norm_bwd_kernel(const float* __restrict__ dy, const float* __res
       }
     }
   }
-  if (!ln) return;
+  if (!LN) return;
   // block-level reduction of the gain / bias partials in warp order
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
@@ -248,13 +250,23 @@ __global__ void norm_bwd_kernel(const float* __restrict__ dy, const float* __res
   }
 }
 
+// NV = float4 per lane = ceil(D / 128): the row lives in registers without slack
 template <typename F>
 static int norm_dispatch(int D, F&& f) {
   if (D % 4) return set_error(ST_UNSUPPORTED, "norm: n_embd must be a multiple of 4");
-  if (D <= 512) return f(std::integral_constant<int, 4>());
-  if (D <= 1024) return f(std::integral_constant<int, 8>());
-  if (D <= 2048) return f(std::integral_constant<int, 16>());
-  if (D <= 4096) return f(std::integral_constant<int, 32>());
+  const int nv = (D + 127) / 128;
+  switch (nv) {
+    case 1: return f(std::integral_constant<int, 1>());
+    case 2: return f(std::integral_constant<int, 2>());
+    case 3: case 4: return f(std::integral_constant<int, 4>());
+    case 5: case 6: return f(std::integral_constant<int, 6>());
+    case 7: case 8: return f(std::integral_constant<int, 8>());
+    case 9: case 10: return f(std::integral_constant<int, 10>());
+    case 11: case 12: case 13: return f(std::integral_constant<int, 13>());
+    case 14: case 15: case 16: return f(std::integral_constant<int, 16>());
+  }
+  if (nv <= 24) return f(std::integral_constant<int, 24>());
+  if (nv <= 32) return f(std::integral_constant<int, 32>());
   return set_error(ST_UNSUPPORTED, "norm: n_embd above 4096");
 }
 
@@ -263,9 +275,12 @@ int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b
   return norm_dispatch(D, [&](auto nv) {
     constexpr int NV = decltype(nv)::value;
     int grid = cdiv(M, 8);
-    if (grid > num_sms() * 8) grid = num_sms() * 8;
+    if (grid > num_sms() * 16) grid = num_sms() * 16;
     Prof prof(PK_NORM_FWD, 0, (double)M * D * 6 + M * 8.0, st);
-    norm_fwd_kernel<NV><<<grid, 256, 0, st>>>(x, M, D, g, b, ln, eps, y, ldy, mean, rstd);
+    if (ln)
+      norm_fwd_kernel<NV, true><<<grid, 256, 0, st>>>(x, M, D, g, b, eps, y, ldy, mean, rstd);
+    else
+      norm_fwd_kernel<NV, false><<<grid, 256, 0, st>>>(x, M, D, g, b, eps, y, ldy, mean, rstd);
     GPTK_CUDA(cudaGetLastError());
     return (int)ST_OK;
   });
@@ -279,14 +294,21 @@ int launch_norm_bwd(const float* dy, const float* x, const float* mean, const fl
   return norm_dispatch(D, [&](auto nv) {
     constexpr int NV = decltype(nv)::value;
     int grid = cdiv(M, 8);
-    if (grid > kNormBwdBlocks) grid = kNormBwdBlocks;
-    size_t smem = ln ? (size_t)8 * 2 * D * sizeof(float) : 0;
-    if (smem > 48 * 1024) {
-      GPTK_CUDA(cudaFuncSetAttribute(norm_bwd_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    }
+    // LayerNorm keeps one gain/bias partial per block, so its grid is capped
+    const int cap = ln ? kNormBwdBlocks : num_sms() * 16;
+    if (grid > cap) grid = cap;
     Prof prof(PK_NORM_BWD, 0, (double)M * D * (dres_init ? 14 : 18), st);
-    norm_bwd_kernel<NV><<<grid, 256, smem, st>>>(dy, x, mean, rstd, g, ln, M, D, dres, dres_init, dres_bf, dg_part,
-                                                 db_part);
+    if (ln) {
+      size_t smem = (size_t)8 * 2 * D * sizeof(float);
+      if (smem > 48 * 1024)
+        GPTK_CUDA(cudaFuncSetAttribute(norm_bwd_kernel<NV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem));
+      norm_bwd_kernel<NV, true><<<grid, 256, smem, st>>>(dy, x, mean, rstd, g, M, D, dres, dres_init, dres_bf,
+                                                         dg_part, db_part);
+    } else {
+      norm_bwd_kernel<NV, false><<<grid, 256, 0, st>>>(dy, x, mean, rstd, g, M, D, dres, dres_init, dres_bf,
+                                                       dg_part, db_part);
+    }
     GPTK_CUDA(cudaGetLastError());
     if (nblk_out) *nblk_out = grid;
     return (int)ST_OK;
@@ -462,45 +484,73 @@ int launch_loss_reduce(const float* ell, const int* targets, const int* token_by
 }
 
 // ------------------------------------------------------------------ QK-norm + RoPE
-// One warp per (token, head).  Lane l handles pair indices i = l + 32 j (i < hd/2) and their
-// partners i + hd/2, so a RoPE pair never crosses lanes.
+// One warp per (token, head).  Lane l owns pair indices i = l*PPL .. l*PPL+PPL-1 (i < hd/2)
+// and their partners i + hd/2, so a RoPE pair never crosses lanes; with PPL = 2 the loads
+// and stores are bf16x2.  src is [M, 3, H, hd]; dst is [M, 3, H, hdp] (may be src itself
+// when hdp == hd, in which case v is left untouched).
 
-template <int PAIRS>
-__global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ qkv, const float2* __restrict__ cs, int M, int T,
-                              int H, int hd, int hdp, int rope, int qk_norm, float eps,
-                              __nv_bfloat16* __restrict__ out, float* __restrict__ rq, float* __restrict__ rk) {
+template <int PPL>
+__device__ __forceinline__ void ld_pairs(const __nv_bfloat16* p, int i, int half, float* a, float* b) {
+  if (PPL == 2) {
+    if (i < half) {
+      const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(p + i);
+      const __nv_bfloat162 y = *reinterpret_cast<const __nv_bfloat162*>(p + half + i);
+      a[0] = __low2float(x); a[1] = __high2float(x);
+      b[0] = __low2float(y); b[1] = __high2float(y);
+    } else {
+      a[0] = a[1] = b[0] = b[1] = 0.f;
+    }
+  } else {
+    a[0] = i < half ? __bfloat162float(p[i]) : 0.f;
+    b[0] = i < half ? __bfloat162float(p[half + i]) : 0.f;
+  }
+}
+
+template <int PPL>
+__device__ __forceinline__ void st_pairs(__nv_bfloat16* p, int i, int half, const float* a, const float* b) {
+  if (i >= half) return;
+  if (PPL == 2) {
+    *reinterpret_cast<__nv_bfloat162*>(p + i) = __floats2bfloat162_rn(a[0], a[1]);
+    *reinterpret_cast<__nv_bfloat162*>(p + half + i) = __floats2bfloat162_rn(b[0], b[1]);
+  } else {
+    p[i] = __float2bfloat16_rn(a[0]);
+    p[half + i] = __float2bfloat16_rn(b[0]);
+  }
+}
+
+template <int PPL>
+__global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ src, const float2* __restrict__ cs, int M, int T,
+                              int H, int hd, int hdp, int rope, int qk_norm, float eps, __nv_bfloat16* dst,
+                              float* __restrict__ rq, float* __restrict__ rk, int in_place) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int half = hd / 2;
+  const int i = lane * PPL;
   const long long D = (long long)H * hd;
-  for (long long wid = blockIdx.x * (long long)warps + (threadIdx.x >> 5); wid < (long long)M * H;
-       wid += (long long)gridDim.x * warps) {
-    const int m = static_cast<int>(wid / H), h = static_cast<int>(wid % H);
+  const int nsect = in_place ? 2 : 3;
+  const int total = M * H;
+  for (int wid = blockIdx.x * warps + (threadIdx.x >> 5); wid < total; wid += gridDim.x * warps) {
+    const int m = wid / H, h = wid - (wid / H) * H;
     const int t = m % T;
-    for (int sct = 0; sct < 3; ++sct) {
-      const __nv_bfloat16* src = qkv + (long long)m * 3 * D + sct * D + (long long)h * hd;
-      __nv_bfloat16* dst = out + (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
-      float a[PAIRS], b[PAIRS];
-      float ss = 0.f;
-#pragma unroll
-      for (int j = 0; j < PAIRS; ++j) {
-        int i = lane + 32 * j;
-        a[j] = i < half ? __bfloat162float(src[i]) : 0.f;
-        b[j] = i < half ? __bfloat162float(src[i + half]) : 0.f;
-        ss += a[j] * a[j] + b[j] * b[j];
-      }
-      float r = 1.f;
+    for (int sct = 0; sct < nsect; ++sct) {
+      const __nv_bfloat16* sp = src + (long long)m * 3 * D + sct * D + (long long)h * hd;
+      __nv_bfloat16* dp = dst + (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
+      float a[PPL], b[PPL];
+      ld_pairs<PPL>(sp, i, half, a, b);
       if (sct < 2) {
+        float r = 1.f;
         if (qk_norm) {
+          float ss = 0.f;
+#pragma unroll
+          for (int j = 0; j < PPL; ++j) ss += a[j] * a[j] + b[j] * b[j];
           r = rsqrtf(warp_sum(ss) / hd + eps);
           if (lane == 0) (sct == 0 ? rq : rk)[(long long)m * H + h] = r;
         }
 #pragma unroll
-        for (int j = 0; j < PAIRS; ++j) {
-          int i = lane + 32 * j;
-          if (rope && i < half) {
-            float2 e = cs[(long long)t * half + i];
-            float x1 = a[j], x2 = b[j];
+        for (int j = 0; j < PPL; ++j) {
+          if (rope && i + j < half) {
+            const float2 e = cs[(long long)t * half + i + j];
+            const float x1 = a[j], x2 = b[j];
             a[j] = x1 * e.x - x2 * e.y;
             b[j] = x1 * e.y + x2 * e.x;
           }
@@ -508,59 +558,44 @@ __global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ qkv, const float
           b[j] *= r;
         }
       }
-#pragma unroll
-      for (int j = 0; j < PAIRS; ++j) {
-        int i = lane + 32 * j;
-        if (i < half) {
-          dst[i] = __float2bfloat16_rn(a[j]);
-          dst[i + half] = __float2bfloat16_rn(b[j]);
-        }
-      }
+      st_pairs<PPL>(dp, i, half, a, b);
     }
   }
 }
 
-template <int PAIRS>
-__global__ void qk_bwd_kernel(const __nv_bfloat16* __restrict__ dpad, const __nv_bfloat16* __restrict__ qpad,
+template <int PPL>
+__global__ void qk_bwd_kernel(const __nv_bfloat16* dpad, const __nv_bfloat16* __restrict__ qpad,
                               const float* __restrict__ rq, const float* __restrict__ rk,
                               const float2* __restrict__ cs, int M, int T, int H, int hd, int hdp, int rope,
-                              int qk_norm, __nv_bfloat16* __restrict__ dqkv) {
+                              int qk_norm, __nv_bfloat16* dqkv) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int half = hd / 2;
+  const int i = lane * PPL;
   const long long D = (long long)H * hd;
-  for (long long wid = blockIdx.x * (long long)warps + (threadIdx.x >> 5); wid < (long long)M * H;
-       wid += (long long)gridDim.x * warps) {
-    const int m = static_cast<int>(wid / H), h = static_cast<int>(wid % H);
+  const bool in_place = (const void*)dpad == (const void*)dqkv;
+  const int total = M * H;
+  for (int wid = blockIdx.x * warps + (threadIdx.x >> 5); wid < total; wid += gridDim.x * warps) {
+    const int m = wid / H, h = wid - (wid / H) * H;
     const int t = m % T;
     for (int sct = 0; sct < 3; ++sct) {
+      if (in_place && sct == 2) break;  // dv is already in place
       const long long po = (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
-      const __nv_bfloat16* dsrc = dpad + po;
       __nv_bfloat16* dst = dqkv + (long long)m * 3 * D + sct * D + (long long)h * hd;
-      float a[PAIRS], b[PAIRS];
-#pragma unroll
-      for (int j = 0; j < PAIRS; ++j) {
-        int i = lane + 32 * j;
-        a[j] = i < half ? __bfloat162float(dsrc[i]) : 0.f;
-        b[j] = i < half ? __bfloat162float(dsrc[i + half]) : 0.f;
-      }
+      float a[PPL], b[PPL];
+      ld_pairs<PPL>(dpad + po, i, half, a, b);
       if (sct < 2) {
         if (qk_norm) {
           // dx = r (dy - y mean(dy y)), y the normalised output that the forward saved
-          const __nv_bfloat16* ysrc = qpad + po;
-          float ya[PAIRS], yb[PAIRS];
+          float ya[PPL], yb[PPL];
+          ld_pairs<PPL>(qpad + po, i, half, ya, yb);
           float s = 0.f;
 #pragma unroll
-          for (int j = 0; j < PAIRS; ++j) {
-            int i = lane + 32 * j;
-            ya[j] = i < half ? __bfloat162float(ysrc[i]) : 0.f;
-            yb[j] = i < half ? __bfloat162float(ysrc[i + half]) : 0.f;
-            s += a[j] * ya[j] + b[j] * yb[j];
-          }
+          for (int j = 0; j < PPL; ++j) s += a[j] * ya[j] + b[j] * yb[j];
           const float mdy = warp_sum(s) / hd;
           const float r = (sct == 0 ? rq : rk)[(long long)m * H + h];
 #pragma unroll
-          for (int j = 0; j < PAIRS; ++j) {
+          for (int j = 0; j < PPL; ++j) {
             a[j] = r * (a[j] - ya[j] * mdy);
             b[j] = r * (b[j] - yb[j] * mdy);
           }
@@ -568,25 +603,17 @@ __global__ void qk_bwd_kernel(const __nv_bfloat16* __restrict__ dpad, const __nv
         if (rope) {
           // the rotation is orthogonal: its reverse rotates by -phi
 #pragma unroll
-          for (int j = 0; j < PAIRS; ++j) {
-            int i = lane + 32 * j;
-            if (i < half) {
-              float2 e = cs[(long long)t * half + i];
-              float x1 = a[j], x2 = b[j];
+          for (int j = 0; j < PPL; ++j) {
+            if (i + j < half) {
+              const float2 e = cs[(long long)t * half + i + j];
+              const float x1 = a[j], x2 = b[j];
               a[j] = x1 * e.x + x2 * e.y;
               b[j] = -x1 * e.y + x2 * e.x;
             }
           }
         }
       }
-#pragma unroll
-      for (int j = 0; j < PAIRS; ++j) {
-        int i = lane + 32 * j;
-        if (i < half) {
-          dst[i] = __float2bfloat16_rn(a[j]);
-          dst[i + half] = __float2bfloat16_rn(b[j]);
-        }
-      }
+      st_pairs<PPL>(dst, i, half, a, b);
     }
   }
 }
@@ -594,14 +621,18 @@ __global__ void qk_bwd_kernel(const __nv_bfloat16* __restrict__ dpad, const __nv
 int launch_qk_fwd(const __nv_bfloat16* qkv, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
                   int qk_norm, float eps, __nv_bfloat16* qkv_pad, float* rstd_q, float* rstd_k, cudaStream_t st) {
   if (hd % 2) return set_error(ST_UNSUPPORTED, "head_dim must be even");
+  const int in_place = (const void*)qkv == (const void*)qkv_pad;
+  if (in_place && hdp != hd) return set_error(ST_INVALID_ARG, "qk_fwd: in place needs an unpadded layout");
   long long work = (long long)M * H;
   int grid = cdiv(work, 8);
-  if (grid > num_sms() * 16) grid = num_sms() * 16;
-  Prof prof(PK_QK, 0, (double)M * 3 * H * hd * 4, st);
+  if (grid > num_sms() * 32) grid = num_sms() * 32;
+  Prof prof(PK_QK, 0, (double)M * (in_place ? 2 : 3) * H * hd * 4, st);
   if (hd <= 64)
-    qk_fwd_kernel<1><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k);
+    qk_fwd_kernel<1><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k,
+                                           in_place);
   else if (hd <= 128)
-    qk_fwd_kernel<2><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k);
+    qk_fwd_kernel<2><<<grid, 256, 0, st>>>(qkv, rope_cs, M, T, H, hd, hdp, rope, qk_norm, eps, qkv_pad, rstd_q, rstd_k,
+                                           in_place);
   else
     return set_error(ST_UNSUPPORTED, "head_dim above 128");
   GPTK_CUDA(cudaGetLastError());
@@ -612,9 +643,11 @@ int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, c
                   const float* rstd_k, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
                   int qk_norm, __nv_bfloat16* dqkv, cudaStream_t st) {
   if (hd % 2) return set_error(ST_UNSUPPORTED, "head_dim must be even");
+  if ((const void*)dqkv_pad == (const void*)dqkv && hdp != hd)
+    return set_error(ST_INVALID_ARG, "qk_bwd: in place needs an unpadded layout");
   long long work = (long long)M * H;
   int grid = cdiv(work, 8);
-  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  if (grid > num_sms() * 32) grid = num_sms() * 32;
   Prof prof(PK_QK, 0, (double)M * 3 * H * hd * 4 + (qk_norm ? (double)M * 2 * H * hd * 2 : 0), st);
   if (hd <= 64)
     qk_bwd_kernel<1><<<grid, 256, 0, st>>>(dqkv_pad, qkv_pad, rstd_q, rstd_k, rope_cs, M, T, H, hd, hdp, rope, qk_norm,
@@ -634,11 +667,10 @@ __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __n
                                   int T, int H, int hd, int hdp, float* __restrict__ delta) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long M = (long long)B * T;
-  for (long long wid = blockIdx.x * (long long)warps + (threadIdx.x >> 5); wid < M * H;
-       wid += (long long)gridDim.x * warps) {
+  const int total = B * T * H;
+  for (int wid = blockIdx.x * warps + (threadIdx.x >> 5); wid < total; wid += gridDim.x * warps) {
     const long long m = wid / H;
-    const int h = static_cast<int>(wid % H);
+    const int h = wid - (wid / H) * H;
     const __nv_bfloat16* orow = o + m * H * hd + (long long)h * hd;
     const __nv_bfloat16* drow = dpad + m * H * hdp + (long long)h * hdp;
     float s = 0.f;

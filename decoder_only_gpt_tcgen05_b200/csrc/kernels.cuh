@@ -59,7 +59,7 @@ int launch_fill(float* p, long long n, float value, cudaStream_t st);
 
 // ---- embedding backward (embed_bwd.cu)
 // scratch layout sizes for M tokens over V ids
-long long embed_bwd_scratch_bytes(int M, int V);
+long long embed_bwd_scratch_bytes(int M, int V, int D);
 // dwte[v] += sum over tokens m with idx[m] == v of dx[m]  (deterministic order: ascending m)
 int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float* dwte, void* scratch,
                      cudaStream_t st);

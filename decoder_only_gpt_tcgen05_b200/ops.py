@@ -96,7 +96,10 @@ def lmhead_ce_fwd_noalloc(x: torch.Tensor, w: torch.Tensor, targets: torch.Tenso
 
 
 PROFILE_FAMILIES = ["gemm", "attn_fwd", "attn_bwd_dkv", "attn_bwd_dq", "norm_fwd", "norm_bwd", "embed_fwd",
-                    "embed_bwd", "cast", "ce_combine", "loss", "qk", "delta", "colsum", "misc"]
+                    "embed_bwd", "cast", "ce_combine", "loss", "qk", "delta", "colsum", "misc",
+                    "gemm_qkv", "gemm_o", "gemm_up", "gemm_down", "gemm_lm_fwd", "gemm_lm_bwd", "gemm_dgrad",
+                    "gemm_wgrad"]
+GEMM_FAMILIES = [f for f in PROFILE_FAMILIES if f.startswith("gemm")]
 
 
 def launch_count() -> int:

@@ -117,7 +117,9 @@ GPT_API int gpt_op_lmhead_ce_fwd_noalloc(const void* x, const void* w, const int
  *   Returns the number of families, or GPT_ERR_CUDA (with gpt_last_error) if
  *   an event could not be read.  Families, in order: gemm, attn_fwd,
  *   attn_bwd_dkv, attn_bwd_dq, norm_fwd, norm_bwd, embed_fwd, embed_bwd,
- *   cast, ce_combine, loss, qk, delta, colsum, misc. */
+ *   cast, ce_combine, loss, qk, delta, colsum, misc, then the model's GEMMs by
+ *   role: gemm_qkv, gemm_o, gemm_up, gemm_down, gemm_lm_fwd, gemm_lm_bwd,
+ *   gemm_dgrad, gemm_wgrad (op-level GEMMs count as gemm). */
 GPT_API unsigned long long gpt_launch_count(void);
 GPT_API int gpt_profile_start(void);
 GPT_API int gpt_profile_stop(int max_kinds, double* ms, long long* count, double* flops, double* bytes);
