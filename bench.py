@@ -231,11 +231,13 @@ def main():
     tb_d = torch.from_numpy(tb).to(dev)
     stream = torch.cuda.current_stream(dev)
 
+    from decoder_only_gpt_tcgen05_b200 import dist as gdist
+
     def step():
         model.forward_loss(idx_d, tgt_d)
         model.backward()
         if world > 1:
-            dist.all_reduce(model.grads)
+            gdist.allreduce_grads_(model.grads)
 
     def barrier():
         if world > 1:

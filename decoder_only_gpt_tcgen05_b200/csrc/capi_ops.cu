@@ -8,7 +8,36 @@
 
 using namespace gptk;
 
+namespace gptk {
+// Waits on an mbarrier that nothing arrives at, through the same bounded wait as every
+// pipeline kernel: after ctl.timeout_ns it records DEV_ERR_TIMEOUT and returns.
+__global__ void wait_probe_kernel(DevCtl ctl) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, ctl, &abort_flag, 99);
+}
+}  // namespace gptk
+
 extern "C" {
+
+GPT_API int gpt_op_wait_probe(unsigned long long timeout_ns, void* stream) {
+  set_error(ST_OK, "");
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull)
+    return set_error(ST_INVALID_ARG, "wait_probe: timeout must be in (0, 10 s]");
+  DevCtl ctl = device_ctl();
+  if (!ctl.status) return set_error(ST_CUDA, "device status word unavailable");
+  ctl.timeout_ns = timeout_ns;
+  Prof prof(PK_MISC, 0, 0, static_cast<cudaStream_t>(stream));
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ctl);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
 
 GPT_API const char* gpt_last_error(void) { return last_error(); }
 

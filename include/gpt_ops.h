@@ -107,6 +107,14 @@ GPT_API size_t gpt_op_lmhead_ce_noalloc_max_scratch_bytes(void);
 GPT_API int gpt_op_lmhead_ce_fwd_noalloc(const void* x, const void* w, const int32_t* targets, int M, int D,
                                          int V, float* ell, float* lse, void* stream);
 
+/* Failure-detection probe (no counterpart on the pages): launches one kernel
+ * that waits on an mbarrier nothing ever arrives at, through the same bounded
+ * wait every pipeline kernel uses.  After timeout_ns (at most 10 s) the kernel
+ * records a timeout in the device status word and returns, so the next
+ * gpt_sync_status() reports GPT_ERR_DEVICE_TIMEOUT and the context stays
+ * usable.  Nothing faults, traps or hangs. */
+GPT_API int gpt_op_wait_probe(unsigned long long timeout_ns, void* stream);
+
 /* Measurement hooks (no counterpart on the pages).
  * gpt_launch_count: kernels this process has launched through the library.
  * gpt_profile_start: from now on, bracket every launch with CUDA events on its
