@@ -42,60 +42,63 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 }
 
 // ====================================================================== forward
+// One CTA per (b, h, pair of 128-query tiles A = 2p, B = 2p+1): two softmax warpgroups, one
+// per query tile, and one MMA thread that alternates between them, so that the tensor core
+// computes one tile's S or PV while the other tile's softmax runs.  K and V tiles stream
+// through a 3-slot ring shared by both query tiles (K_0, V_0, K_1, V_1, ...).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,256+HD), O_B [384,384+HD).
 
 template <int HD>
 struct FwdSmem {
   static constexpr int TILE = HD * 256;  // 128 rows x HD bf16
-  static constexpr int Q = 0;
-  static constexpr int K0 = Q + TILE;
-  static constexpr int V0 = K0 + 2 * TILE;
-  static constexpr int P = V0 + 2 * TILE;
-  static constexpr int BAR = P + 32768;
+  static constexpr int Q0 = 0;           // Q_A, Q_B
+  static constexpr int KV = 2 * TILE;    // 3 ring slots
+  static constexpr int P = 5 * TILE;     // P_A, P_B: 128 x 128 bf16 each
+  static constexpr int BAR = P + 2 * 32768;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnShape s, __nv_bfloat16* __restrict__ o,
                     long long ldo, float* __restrict__ lse_out, float scale_log2, DevCtl ctl) {
   using L = FwdSmem<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
-  uint64_t* bar_q = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* s_free = bars + 11;  // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* p_empty = bars + 14;
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [3]
+  uint64_t* kv_empty = bars + 4;  // [3]
+  uint64_t* s_full = bars + 7;    // [2] (A, B)
+  uint64_t* p_full = bars + 9;    // [2]
+  uint64_t* o_done = bars + 11;   // [2]
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = gridDim.x;
-  const int qt = n_qt - 1 - blockIdx.x;  // heaviest first
+  const int n_pairs = gridDim.x;
+  const int pr = n_pairs - 1 - blockIdx.x;  // heaviest first
   const int bh = blockIdx.y;
   const int b = bh / s.H, h = bh % s.H;
-  const int q0 = qt * 128;
-  const int n_kv = qt + 1;
+  const int q0 = pr * 256;
+  // KV tiles each query tile needs (0 when the tile lies past the end of the sequence)
+  const int n_a = 2 * pr + 1;
+  const int n_b = (q0 + 128 < s.T) ? 2 * pr + 2 : 0;
+  const int n_kv = n_b > 0 ? n_b : n_a;
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1);
-      mbar_init(&k_empty[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
     }
-    mbar_init(p_full, 4);
-    mbar_init(p_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_done[i], 1);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -109,82 +112,88 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tS = tbase;        // 2 x 128 columns
-  const uint32_t tO = tbase + 256;  // HD columns
 
   const int colq = h * s.hdp;
   const int colk = s.H * s.hdp + h * s.hdp;
   const int colv = 2 * s.H * s.hdp + h * s.hdp;
 
   if (warp == 0 && lane == 0) {
+    // ---------------------------------------------- TMA producer
     bool ok = true;
-    mbar_expect_tx(bar_q, L::TILE);
-    for (int c = 0; c < NCH; ++c) tma_load_3d(sm + L::Q + c * 16384, &tm_qkv, bar_q, colq + 64 * c, q0, b);
-    int issued_k = -1, issued_v = -1;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int st = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      if (!mbar_wait(&k_empty[st], ph ^ 1u, ctl, abort_flag, 20)) { ok = false; break; }
-      mbar_expect_tx(&k_full[st], L::TILE);
+    mbar_expect_tx(q_full, 2 * L::TILE);
+    for (int t = 0; t < 2; ++t)
       for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::K0 + st * L::TILE + c * 16384, &tm_qkv, &k_full[st], colk + 64 * c, j * 128, b);
-      issued_k = j;
-      if (!mbar_wait(&v_empty[st], ph ^ 1u, ctl, abort_flag, 21)) { ok = false; break; }
-      mbar_expect_tx(&v_full[st], L::TILE);
+        tma_load_3d(sm + L::Q0 + t * L::TILE + c * 16384, &tm_qkv, q_full, colq + 64 * c, q0 + 128 * t, b);
+    int issued = -1;
+    for (int seq = 0; seq < 2 * n_kv && ok; ++seq) {
+      const int slot = seq % 3;
+      const uint32_t ph = (seq / 3) & 1;
+      if (!mbar_wait(&kv_empty[slot], ph ^ 1u, ctl, abort_flag, 20)) { ok = false; break; }
+      mbar_expect_tx(&kv_full[slot], L::TILE);
+      const int col = (seq & 1) ? colv : colk;
       for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::V0 + st * L::TILE + c * 16384, &tm_qkv, &v_full[st], colv + 64 * c, j * 128, b);
-      issued_v = j;
+        tma_load_3d(sm + L::KV + slot * L::TILE + c * 16384, &tm_qkv, &kv_full[slot], col + 64 * c, (seq >> 1) * 128, b);
+      issued = seq;
     }
     if (!ok) {
-      // wait (bounded) for the copies still in flight
       volatile int never = 0;
-      mbar_wait(bar_q, 0, ctl, &never, 22);
-      for (int j = (issued_k > 0 ? issued_k - 1 : 0); j <= issued_k; ++j)
-        mbar_wait(&k_full[j & 1], (j >> 1) & 1, ctl, &never, 22);
-      for (int j = (issued_v > 0 ? issued_v - 1 : 0); j <= issued_v && issued_v >= 0; ++j)
-        mbar_wait(&v_full[j & 1], (j >> 1) & 1, ctl, &never, 22);
+      mbar_wait(q_full, 0, ctl, &never, 22);
+      for (int seq = (issued > 1 ? issued - 2 : 0); seq <= issued && issued >= 0; ++seq)
+        mbar_wait(&kv_full[seq % 3], (seq / 3) & 1, ctl, &never, 22);
     }
   } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------- MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t idesc_o = idesc_bf16(128, HD, 0, 1);
-    bool ok = mbar_wait(bar_q, 0, ctl, abort_flag, 23);
+    bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 23);
     bool issued = false;
-    const uint32_t sQ = smem_u32(sm + L::Q);
-    const uint32_t sP = smem_u32(sm + L::P);
-    for (int j = 0; j <= n_kv && ok; ++j) {
-      if (j < n_kv) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&k_full[st], ph, ctl, abort_flag, 24)) { ok = false; break; }
-        if (!mbar_wait(&s_free[st], ph ^ 1u, ctl, abort_flag, 25)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::K0 + st * L::TILE);
+    const int n_t[2] = {n_a, n_b};
+    auto kv_wait = [&](int seq) -> bool {
+      return mbar_wait(&kv_full[seq % 3], (seq / 3) & 1, ctl, abort_flag, 24);
+    };
+    auto issue_s = [&](int t, int j) {
+      const uint32_t sQ = smem_u32(sm + L::Q0 + t * L::TILE);
+      const uint32_t sK = smem_u32(sm + L::KV + ((2 * j) % 3) * L::TILE);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tS + st * 128, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), idesc_s,
-                    kk > 0);
-        }
-        umma_commit(&s_full[st]);
-        umma_commit(&k_empty[st]);
-        issued = true;
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        umma_bf16(tbase + 128 * t, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), idesc_s, kk > 0);
       }
-      if (j >= 1) {
-        const int jj = j - 1;
-        const int st = jj & 1;
-        if (!mbar_wait(p_full, jj & 1, ctl, abort_flag, 26)) { ok = false; break; }
-        if (!mbar_wait(&v_full[st], (jj >> 1) & 1, ctl, abort_flag, 27)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sV = smem_u32(sm + L::V0 + st * L::TILE);
+      umma_commit(&s_full[t]);
+    };
+    auto issue_pv = [&](int t, int j) {
+      const uint32_t sP = smem_u32(sm + L::P + t * 32768);
+      const uint32_t sV = smem_u32(sm + L::KV + ((2 * j + 1) % 3) * L::TILE);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          umma_bf16(tO, sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                    sdesc_sw128(sV + kk * 2048, 16384, 1024), idesc_o, (jj | kk) != 0);
+      for (int kk = 0; kk < 8; ++kk)
+        umma_bf16(tbase + 256 + 128 * t, sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(sV + kk * 2048, 16384, 1024), idesc_o, (j | kk) != 0);
+      umma_commit(&o_done[t]);
+    };
+    if (ok && kv_wait(0)) {
+      tc_fence_after();
+      for (int t = 0; t < 2; ++t)
+        if (n_t[t] > 0) issue_s(t, 0);
+      umma_commit(&kv_empty[0]);
+      issued = true;
+    } else {
+      ok = false;
+    }
+    for (int j = 0; j < n_kv && ok; ++j) {
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (j >= n_t[t]) continue;
+        if (!mbar_wait(&p_full[t], j & 1, ctl, abort_flag, 26) || !kv_wait(2 * j + 1)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(t, j);
+        if (j + 1 < n_t[t]) {
+          if (!kv_wait(2 * j + 2)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(t, j + 1);
         }
-        umma_commit(p_empty);
-        umma_commit(&v_empty[st]);
-        issued = true;
       }
+      if (!ok) break;
+      umma_commit(&kv_empty[(2 * j + 1) % 3]);                   // V_j
+      if (j + 1 < n_kv) umma_commit(&kv_empty[(2 * j + 2) % 3]);  // K_{j+1}
     }
     if (!ok && issued) {
       volatile int never = 0;
@@ -192,32 +201,50 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain, 0, ctl, &never, 28);
     }
   } else if (warp >= 2) {
+    // ---------------------------------------------- softmax: warpgroup t handles query tile t
+    const int t = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    const int qi = q0 + r;
+    const int qi = q0 + 128 * t + r;
+    const int n = t == 0 ? n_a : n_b;
+    const int diag = 2 * pr + t;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t sP = smem_u32(sm + L::P);
+    const uint32_t tS = tbase + 128 * t + lane_off;
+    const uint32_t tO = tbase + 256 + 128 * t + lane_off;
+    const uint32_t sP = smem_u32(sm + L::P + t * 32768);
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, ctl, abort_flag, 29)) { ok = false; break; }
+    bool ok = n > 0;
+    for (int j = 0; j < n; ++j) {
+      if (!mbar_wait(&s_full[t], j & 1, ctl, abort_flag, 29)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tSrow = tS + st * 128 + lane_off;
+      // The row is handled as two halves of 64 scores (two TMEM loads in flight per half):
+      // ten warps leave at most 168 registers per thread, too few to hold all 128 scores.
       const int kbase = j * 128;
-      const bool diag = (j == n_kv - 1);
-      // pass 1: row max of the (masked) scores
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tSrow + c * 32, sv);
+      const bool dg = (j == diag);
+      uint32_t raw[64];
+      float* sv = reinterpret_cast<float*>(raw);
+      float mx8[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int key = kbase + c * 32 + e;
-          if (!diag || (key <= qi && key < s.T)) mx = fmaxf(mx, sv[e]);
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        tmem_ld32_nowait(tS + hf * 64, raw);
+        tmem_ld32_nowait(tS + hf * 64 + 32, raw + 32);
+        tmem_wait_ld();
+        tmem_fence_regs<64>(raw);
+        if (dg) {
+          // diagonal tile: keys after the query (or past the sequence) do not exist
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const int key = kbase + hf * 64 + e;
+            if (key > qi || key >= s.T) sv[e] = -INFINITY;
+          }
         }
+#pragma unroll
+        for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], sv[e]);
       }
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= scale_log2;
       const float m_new = fmaxf(m, mx);
       float alpha = 1.f;
@@ -226,55 +253,63 @@ __global__ void __launch_bounds__(192, 1)
         m = m_new;
       }
       if (j > 0) {
-        // O and the P buffer are still in use by the previous P V product
-        if (!mbar_wait(p_empty, (j - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
+        // O and P_t are still in use by the previous P V product of this tile
+        if (!mbar_wait(&o_done[t], (j - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
           for (int c = 0; c < HD / 32; ++c) {
             float ov[32];
-            tmem_ld32(tO + lane_off + c * 32, ov);
+            tmem_ld32(tO + c * 32, ov);
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-            tmem_st32(tO + lane_off + c * 32, ov);
+            tmem_st32(tO + c * 32, ov);
           }
         }
       }
-      // pass 2: P = exp2(s * scale - m) -> shared memory (K-major, 128-byte swizzle;
-      // keys 0..63 in chunk 0, 64..127 in chunk 1), row sum in registers
-      float rs = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float sv[32];
-        tmem_ld32(tSrow + c * 32, sv);
+      // P = exp2(s * scale - m) -> shared memory (K-major, 128-byte swizzle; masked scores are
+      // -inf and give 0).  The second half is still in registers; the first is read again.
+      float rs8[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int key = kbase + c * 32 + e;
-          const bool valid = !diag || (key <= qi && key < s.T);
-          sv[e] = valid ? ex2_approx(fmaf(sv[e], scale_log2, -m)) : 0.f;
-          rs += sv[e];
+      for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        const int hf = 1 - it;
+        if (it == 1) {
+          tmem_ld32_nowait(tS, raw);
+          tmem_ld32_nowait(tS + 32, raw + 32);
+          tmem_wait_ld();
+          tmem_fence_regs<64>(raw);
+          if (dg) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e) {
+              const int key = kbase + e;
+              if (key > qi || key >= s.T) sv[e] = -INFINITY;
+            }
+          }
         }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int gg = c * 4 + g;
-          uint4 w;
-          w.x = pack_bf16x2(sv[8 * g + 0], sv[8 * g + 1]);
-          w.y = pack_bf16x2(sv[8 * g + 2], sv[8 * g + 3]);
-          w.z = pack_bf16x2(sv[8 * g + 4], sv[8 * g + 5]);
-          w.w = pack_bf16x2(sv[8 * g + 6], sv[8 * g + 7]);
-          st_shared_v4(sP + (gg >> 3) * 16384 + sw128_off(r, gg & 7), w);
+        for (int g = 0; g < 8; ++g) {
+          float pv[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            pv[k] = ex2_approx(fmaf(sv[8 * g + k], scale_log2, -m));
+            rs8[k] += pv[k];
+          }
+          // 16-byte unit (hf*8 + g): chunk hf (keys 64*hf ..), unit g within the 128-byte row
+          st_shared_v4(sP + hf * 16384 + sw128_off(r, g),
+                       make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
+                                  pack_bf16x2(pv[6], pv[7])));
         }
       }
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l = l * alpha + rs;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[st]);
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    if (ok && mbar_wait(p_empty, (n_kv - 1) & 1, ctl, abort_flag, 31)) {
+    if (ok && mbar_wait(&o_done[t], (n - 1) & 1, ctl, abort_flag, 31)) {
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool row_ok = qi < s.T;
@@ -282,7 +317,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         float ov[32];
-        tmem_ld32(tO + lane_off + c * 32, ov);
+        tmem_ld32(tO + c * 32, ov);
 #pragma unroll
         for (int e = 0; e < 32; ++e) ov[e] *= inv_l;
         if (row_ok) {
@@ -782,10 +817,10 @@ static int attn_fwd_t(const __nv_bfloat16* qkv, const AttnShape& s, __nv_bfloat1
   GPTK_TRY(make_tmap_3d(&tm, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
   GPTK_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
   const float scale_log2 = kLog2e / sqrtf((float)s.hd);
-  dim3 grid((s.T + 127) / 128, s.B * s.H);
+  dim3 grid((s.T + 255) / 256, s.B * s.H);
   const double causal = (double)s.B * s.H * ((double)s.T * (s.T + 1) / 2);
   Prof prof(PK_ATTN_FWD, 4.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 4, st);
-  attn_fwd_kernel<HD><<<grid, 192, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
+  attn_fwd_kernel<HD><<<grid, 320, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
