@@ -345,6 +345,10 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ====================================================================== backward: dK, dV
+// One CTA per 128-key tile, stepping over 64-query tiles: S^T = K Q^T and dP^T = V dO^T into
+// double-buffered TMEM, P^T and dS^T = P^T (dP^T - delta) into double-buffered shared memory,
+// dV += P^T dO and dK += dS^T Q accumulating in TMEM.  The per-query statistics (lse, delta)
+// of a step are staged once in shared memory by the four softmax warps.
 
 template <int HD>
 struct DkvSmem {
@@ -352,16 +356,17 @@ struct DkvSmem {
   static constexpr int Q_TILE = HD * 128;   // 64 rows
   static constexpr int K = 0;
   static constexpr int V = K + KV_TILE;
-  static constexpr int Q0 = V + KV_TILE;          // [2]
-  static constexpr int DO0 = Q0 + 2 * Q_TILE;     // [2]
-  static constexpr int P = DO0 + 2 * Q_TILE;      // 128 keys x 64 queries bf16 = 16 KB
-  static constexpr int DS = P + 16384;
-  static constexpr int BAR = DS + 16384;
+  static constexpr int Q0 = V + KV_TILE;       // [2]
+  static constexpr int DO0 = Q0 + 2 * Q_TILE;  // [2]
+  static constexpr int P0 = DO0 + 2 * Q_TILE;  // [2] 128 keys x 64 queries bf16 = 16 KB
+  static constexpr int DS0 = P0 + 32768;       // [2]
+  static constexpr int STATS = DS0 + 32768;    // [2][lse2 x 64, delta x 64] fp32
+  static constexpr int BAR = STATS + 1024;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q64,
                         const __grid_constant__ CUtensorMap tm_do64, const AttnShape s, const float* __restrict__ lse,
                         const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, float scale_log2,
@@ -371,16 +376,18 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;    // [2]
-  uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* pd_full = bars + 9;
-  uint64_t* pd_empty = bars + 10;
-  uint64_t* acc_full = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* q_full = bars + 1;      // [2]
+  uint64_t* q_empty = bars + 3;     // [2]
+  uint64_t* s_full = bars + 5;      // [2]
+  uint64_t* s_free = bars + 7;      // [2]
+  uint64_t* pd_full = bars + 9;     // [2]
+  uint64_t* pd_empty = bars + 11;   // [2]
+  uint64_t* stats_bar = bars + 13;  // [2]
+  uint64_t* acc_full = bars + 15;
+  uint64_t* drain = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* stats = reinterpret_cast<float*>(sm + L::STATS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kt = blockIdx.x;
@@ -398,10 +405,11 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], 8);
+      mbar_init(&pd_full[i], 8);
+      mbar_init(&pd_empty[i], 1);
+      mbar_init(&stats_bar[i], 8);
     }
-    mbar_init(pd_full, 4);
-    mbar_init(pd_empty, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -456,7 +464,6 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = mbar_wait(kv_full, 0, ctl, abort_flag, 42);
     bool issued = false;
     const uint32_t sK = smem_u32(sm + L::K), sV = smem_u32(sm + L::V);
-    const uint32_t sP = smem_u32(sm + L::P), sDS = smem_u32(sm + L::DS);
     for (int it = 0; it <= n_it && ok; ++it) {
       if (it < n_it) {
         const int st = it & 1;
@@ -479,11 +486,13 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (it >= 1) {
         const int jt = it - 1;
-        const int st = jt & 1;
-        if (!mbar_wait(pd_full, jt & 1, ctl, abort_flag, 45)) { ok = false; break; }
+        const int bb = jt & 1;
+        if (!mbar_wait(&pd_full[bb], (jt >> 1) & 1, ctl, abort_flag, 45)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sQ = smem_u32(sm + L::Q0 + st * L::Q_TILE);
-        const uint32_t sD = smem_u32(sm + L::DO0 + st * L::Q_TILE);
+        const uint32_t sQ = smem_u32(sm + L::Q0 + bb * L::Q_TILE);
+        const uint32_t sD = smem_u32(sm + L::DO0 + bb * L::Q_TILE);
+        const uint32_t sP = smem_u32(sm + L::P0 + bb * 16384);
+        const uint32_t sDS = smem_u32(sm + L::DS0 + bb * 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           umma_bf16(tdV, sdesc_sw128(sP + kk * 32, 16, 1024), sdesc_sw128(sD + kk * 2048, 8192, 1024), idesc_acc,
@@ -491,8 +500,8 @@ __global__ void __launch_bounds__(192, 1)
           umma_bf16(tdK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc,
                     (jt | kk) != 0);
         }
-        umma_commit(pd_empty);
-        umma_commit(&q_empty[st]);
+        umma_commit(&pd_empty[bb]);
+        umma_commit(&q_empty[bb]);
         issued = true;
       }
     }
@@ -504,78 +513,99 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain, 0, ctl, &never, 46);
     }
   } else if (warp >= 2) {
+    // two warpgroups: group cg takes query columns [32 cg, 32 cg + 32) of every 64-query step
     const int quad = warp & 3;
+    const int cg = (warp - 2) >> 2;
+    const int sw = warp - 2;         // 0..7: which 8 queries' statistics this warp stages
     const int r = quad * 32 + lane;  // key row within the tile
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t sP = smem_u32(sm + L::P), sDS = smem_u32(sm + L::DS);
     const float* lse_bh = lse + (long long)bh * s.T;
     const float* del_bh = delta + (long long)bh * s.T;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
       const int qb = (i0 + it) * 64;
+      {  // per-query statistics of this step: lse in log2 units and delta
+        if (lane < 16) {
+          const int qq = 8 * sw + (lane & 7);
+          const int q = qb + qq;
+          float v = 0.f;
+          if (q < s.T) v = lane < 8 ? __ldg(lse_bh + q) * kLog2e : __ldg(del_bh + q);
+          stats[st * 128 + (lane < 8 ? 0 : 64) + qq] = v;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&stats_bar[st]);
+      }
+      if (!mbar_wait(&stats_bar[st], (it >> 1) & 1, ctl, abort_flag, 50)) { ok = false; break; }
       if (!mbar_wait(&s_full[st], (it >> 1) & 1, ctl, abort_flag, 47)) { ok = false; break; }
-      if (it > 0 && !mbar_wait(pd_empty, (it - 1) & 1, ctl, abort_flag, 48)) { ok = false; break; }
       tc_fence_after();
+      uint32_t rs[32], rd[32];
+      tmem_ld32_nowait(tS + st * 64 + lane_off + 32 * cg, rs);
+      tmem_ld32_nowait(tdP + st * 64 + lane_off + 32 * cg, rd);
+      tmem_wait_ld();
+      tmem_fence_regs<32>(rs);
+      tmem_fence_regs<32>(rd);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      // the P^T / dS^T buffer of this step is free once the dV/dK products two steps back are done
+      if (!mbar_wait(&pd_empty[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 48)) { ok = false; break; }
+      const bool masked = (qb < k0 + 128) || (qb + 64 > s.T);
+      const uint32_t sP = smem_u32(sm + L::P0 + st * 16384);
+      const uint32_t sDS = smem_u32(sm + L::DS0 + st * 16384);
+      const float* stl = stats + st * 128 + 32 * cg;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float sv[32], dp[32];
-        tmem_ld32(tS + st * 64 + lane_off + c * 32, sv);
-        tmem_ld32(tdP + st * 64 + lane_off + c * 32, dp);
+      for (int g = 0; g < 4; ++g) {
+        const float4 l0 = *reinterpret_cast<const float4*>(stl + 8 * g);
+        const float4 l1 = *reinterpret_cast<const float4*>(stl + 8 * g + 4);
+        const float4 d0 = *reinterpret_cast<const float4*>(stl + 64 + 8 * g);
+        const float4 d1 = *reinterpret_cast<const float4*>(stl + 64 + 8 * g + 4);
+        const float l2[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+        const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+        float p[8], ds[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          // per-query statistics: every lane reads the same address (a broadcast load)
-          const int q = qb + 32 * c + e;
-          const bool valid = (q >= key) && (q < s.T);
-          const float l2 = valid ? __ldg(lse_bh + q) * kLog2e : 0.f;
-          const float dl = valid ? __ldg(del_bh + q) : 0.f;
-          const float p = valid ? ex2_approx(fmaf(sv[e], scale_log2, -l2)) : 0.f;
-          sv[e] = p;
-          dp[e] = p * (dp[e] - dl);
+        for (int k = 0; k < 8; ++k) {
+          const int e = 8 * g + k;
+          float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
+          if (masked) {
+            const int q = qb + 32 * cg + e;
+            if (q < key || q >= s.T) pv = 0.f;
+          }
+          p[k] = pv;
+          ds[k] = pv * (__uint_as_float(rd[e]) - dl[k]);
         }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int unit = 4 * c + g;
-          uint4 w = make_uint4(pack_bf16x2(sv[8 * g], sv[8 * g + 1]), pack_bf16x2(sv[8 * g + 2], sv[8 * g + 3]),
-                               pack_bf16x2(sv[8 * g + 4], sv[8 * g + 5]), pack_bf16x2(sv[8 * g + 6], sv[8 * g + 7]));
-          st_shared_v4(sP + sw128_off(r, unit), w);
-          uint4 x = make_uint4(pack_bf16x2(dp[8 * g], dp[8 * g + 1]), pack_bf16x2(dp[8 * g + 2], dp[8 * g + 3]),
-                               pack_bf16x2(dp[8 * g + 4], dp[8 * g + 5]), pack_bf16x2(dp[8 * g + 6], dp[8 * g + 7]));
-          st_shared_v4(sDS + sw128_off(r, unit), x);
-        }
+        st_shared_v4(sP + sw128_off(r, 4 * cg + g), make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
+                                                               pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7])));
+        st_shared_v4(sDS + sw128_off(r, 4 * cg + g),
+                     make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
+                                pack_bf16x2(ds[6], ds[7])));
       }
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_free[st]);
-        mbar_arrive(pd_full);
-      }
+      if (lane == 0) mbar_arrive(&pd_full[st]);
     }
+    // the two warpgroups share the epilogue: group 0 writes dK, group 1 writes dV
     if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 49)) {
       tc_fence_after();
       const bool row_ok = key < s.T;
       const long long m = (long long)b * s.T + key;
-      __nv_bfloat16* dk = dqkv + m * s.ld_qkv + (long long)s.H * s.hdp + (long long)h * s.hdp;
-      __nv_bfloat16* dv = dqkv + m * s.ld_qkv + 2LL * s.H * s.hdp + (long long)h * s.hdp;
+      // group 0: dK (times the softmax scale), group 1: dV
+      __nv_bfloat16* dst = dqkv + m * s.ld_qkv + (long long)(1 + cg) * s.H * s.hdp + (long long)h * s.hdp;
+      const uint32_t tsrc = (cg == 0 ? tdK : tdV) + lane_off;
+      const float f = cg == 0 ? scale : 1.f;
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
-        float a[32], bb[32];
-        tmem_ld32(tdK + lane_off + c * 32, a);
-        tmem_ld32(tdV + lane_off + c * 32, bb);
+        float a[32];
+        tmem_ld32(tsrc + c * 32, a);
         if (row_ok) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            reinterpret_cast<uint4*>(dk + c * 32)[g] =
-                make_uint4(pack_bf16x2(a[8 * g] * scale, a[8 * g + 1] * scale),
-                           pack_bf16x2(a[8 * g + 2] * scale, a[8 * g + 3] * scale),
-                           pack_bf16x2(a[8 * g + 4] * scale, a[8 * g + 5] * scale),
-                           pack_bf16x2(a[8 * g + 6] * scale, a[8 * g + 7] * scale));
-            reinterpret_cast<uint4*>(dv + c * 32)[g] =
-                make_uint4(pack_bf16x2(bb[8 * g], bb[8 * g + 1]), pack_bf16x2(bb[8 * g + 2], bb[8 * g + 3]),
-                           pack_bf16x2(bb[8 * g + 4], bb[8 * g + 5]), pack_bf16x2(bb[8 * g + 6], bb[8 * g + 7]));
-          }
+          for (int g = 0; g < 4; ++g)
+            reinterpret_cast<uint4*>(dst + c * 32)[g] =
+                make_uint4(pack_bf16x2(a[8 * g] * f, a[8 * g + 1] * f), pack_bf16x2(a[8 * g + 2] * f, a[8 * g + 3] * f),
+                           pack_bf16x2(a[8 * g + 4] * f, a[8 * g + 5] * f),
+                           pack_bf16x2(a[8 * g + 6] * f, a[8 * g + 7] * f));
         }
       }
     }
@@ -589,6 +619,8 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ====================================================================== backward: dQ
+// One CTA per 128-query tile, stepping over 64-key tiles: S = Q K^T and dP = dO V^T into
+// double-buffered TMEM, dS = P (dP - delta) into double-buffered shared memory, dQ += dS K.
 
 template <int HD>
 struct DqSmem {
@@ -596,15 +628,15 @@ struct DqSmem {
   static constexpr int KV_TILE = HD * 128;  // 64 rows
   static constexpr int Q = 0;
   static constexpr int DO = Q + Q_TILE;
-  static constexpr int K0 = DO + Q_TILE;         // [2]
-  static constexpr int V0 = K0 + 2 * KV_TILE;    // [2]
-  static constexpr int DS = V0 + 2 * KV_TILE;    // 128 queries x 64 keys bf16 = 16 KB
-  static constexpr int BAR = DS + 16384;
+  static constexpr int K0 = DO + Q_TILE;       // [2]
+  static constexpr int V0 = K0 + 2 * KV_TILE;  // [2]
+  static constexpr int DS0 = V0 + 2 * KV_TILE; // [2] 128 queries x 64 keys bf16 = 16 KB
+  static constexpr int BAR = DS0 + 32768;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
                        const __grid_constant__ CUtensorMap tm_kv64, const AttnShape s, const float* __restrict__ lse,
                        const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, float scale_log2,
@@ -618,11 +650,11 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* kv_empty = bars + 3;  // [2]
   uint64_t* s_full = bars + 5;    // [2]
   uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* ds_full = bars + 9;
-  uint64_t* ds_empty = bars + 10;
-  uint64_t* acc_full = bars + 11;
-  uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* ds_full = bars + 9;   // [2]
+  uint64_t* ds_empty = bars + 11; // [2]
+  uint64_t* acc_full = bars + 13;
+  uint64_t* drain = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -641,10 +673,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
+      mbar_init(&s_free[i], 8);
+      mbar_init(&ds_full[i], 8);
+      mbar_init(&ds_empty[i], 1);
     }
-    mbar_init(ds_full, 4);
-    mbar_init(ds_empty, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -696,7 +728,7 @@ __global__ void __launch_bounds__(192, 1)
     constexpr uint32_t idesc_acc = idesc_bf16(128, HD, 0, 1);
     bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 62);
     bool issued = false;
-    const uint32_t sQ = smem_u32(sm + L::Q), sD = smem_u32(sm + L::DO), sDS = smem_u32(sm + L::DS);
+    const uint32_t sQ = smem_u32(sm + L::Q), sD = smem_u32(sm + L::DO);
     for (int j = 0; j <= n_kv && ok; ++j) {
       if (j < n_kv) {
         const int st = j & 1;
@@ -719,16 +751,17 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (j >= 1) {
         const int jj = j - 1;
-        const int st = jj & 1;
-        if (!mbar_wait(ds_full, jj & 1, ctl, abort_flag, 65)) { ok = false; break; }
+        const int bb = jj & 1;
+        if (!mbar_wait(&ds_full[bb], (jj >> 1) & 1, ctl, abort_flag, 65)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::K0 + st * L::KV_TILE);
+        const uint32_t sK = smem_u32(sm + L::K0 + bb * L::KV_TILE);
+        const uint32_t sDS = smem_u32(sm + L::DS0 + bb * 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_bf16(tdQ, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sK + kk * 2048, 8192, 1024), idesc_acc,
                     (jj | kk) != 0);
-        umma_commit(ds_empty);
-        umma_commit(&kv_empty[st]);
+        umma_commit(&ds_empty[bb]);
+        umma_commit(&kv_empty[bb]);
         issued = true;
       }
     }
@@ -740,11 +773,12 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(drain, 0, ctl, &never, 66);
     }
   } else if (warp >= 2) {
+    // two warpgroups: group cg takes key columns [32 cg, 32 cg + 32) of every 64-key step
     const int quad = warp & 3;
+    const int cg = (warp - 2) >> 2;
     const int r = quad * 32 + lane;
     const int qi = q0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t sDS = smem_u32(sm + L::DS);
     const bool row_ok = qi < s.T;
     const float lse2 = row_ok ? lse[(long long)bh * s.T + qi] * kLog2e : 0.f;
     const float dl = row_ok ? delta[(long long)bh * s.T + qi] : 0.f;
@@ -752,40 +786,48 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < n_kv; ++j) {
       const int st = j & 1;
       if (!mbar_wait(&s_full[st], (j >> 1) & 1, ctl, abort_flag, 67)) { ok = false; break; }
-      if (j > 0 && !mbar_wait(ds_empty, (j - 1) & 1, ctl, abort_flag, 68)) { ok = false; break; }
       tc_fence_after();
+      uint32_t rs[32], rd[32];
+      tmem_ld32_nowait(tS + st * 64 + lane_off + 32 * cg, rs);
+      tmem_ld32_nowait(tdP + st * 64 + lane_off + 32 * cg, rd);
+      tmem_wait_ld();
+      tmem_fence_regs<32>(rs);
+      tmem_fence_regs<32>(rd);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[st]);
+      if (!mbar_wait(&ds_empty[st], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 68)) { ok = false; break; }
+      const int kb = j * 64 + 32 * cg;
+      const bool masked = (kb + 31 > q0) || (kb + 32 > s.T) || !row_ok;
+      const uint32_t sDS = smem_u32(sm + L::DS0 + st * 16384);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float sv[32], dp[32];
-        tmem_ld32(tS + st * 64 + lane_off + c * 32, sv);
-        tmem_ld32(tdP + st * 64 + lane_off + c * 32, dp);
+      for (int g = 0; g < 4; ++g) {
+        float ds[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int key = j * 64 + 32 * c + e;
-          const bool valid = row_ok && key <= qi && key < s.T;
-          const float p = valid ? ex2_approx(fmaf(sv[e], scale_log2, -lse2)) : 0.f;
-          dp[e] = p * (dp[e] - dl);
+        for (int k = 0; k < 8; ++k) {
+          const int e = 8 * g + k;
+          float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -lse2));
+          if (masked) {
+            const int key = kb + e;
+            if (!row_ok || key > qi || key >= s.T) pv = 0.f;
+          }
+          ds[k] = pv * (__uint_as_float(rd[e]) - dl);
         }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint4 x = make_uint4(pack_bf16x2(dp[8 * g], dp[8 * g + 1]), pack_bf16x2(dp[8 * g + 2], dp[8 * g + 3]),
-                               pack_bf16x2(dp[8 * g + 4], dp[8 * g + 5]), pack_bf16x2(dp[8 * g + 6], dp[8 * g + 7]));
-          st_shared_v4(sDS + sw128_off(r, 4 * c + g), x);
-        }
+        st_shared_v4(sDS + sw128_off(r, 4 * cg + g),
+                     make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
+                                pack_bf16x2(ds[6], ds[7])));
       }
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_free[st]);
-        mbar_arrive(ds_full);
-      }
+      if (lane == 0) mbar_arrive(&ds_full[st]);
     }
     if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 69)) {
       tc_fence_after();
       __nv_bfloat16* dq = dqkv + ((long long)b * s.T + qi) * s.ld_qkv + (long long)h * s.hdp;
+      // the two groups split dQ's columns
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = cg * (HD / 64); c < (cg + 1) * (HD / 64); ++c) {
         float a[32];
         tmem_ld32(tdQ + lane_off + c * 32, a);
         if (row_ok) {
@@ -854,7 +896,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
     Prof prof(PK_ATTN_BWD_DKV, 8.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 6, st);
-    attn_bwd_dkv_kernel<HD><<<grid, 192, L::BYTES, st>>>(kv128, q64, do64, s, lse, delta, dqkv, scale_log2, scale, ctl);
+    attn_bwd_dkv_kernel<HD><<<grid, 320, L::BYTES, st>>>(kv128, q64, do64, s, lse, delta, dqkv, scale_log2, scale, ctl);
     GPTK_CUDA(cudaGetLastError());
   }
   {
@@ -862,7 +904,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
     Prof prof(PK_ATTN_BWD_DQ, 6.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 5, st);
-    attn_bwd_dq_kernel<HD><<<grid, 192, L::BYTES, st>>>(q128, do128, kv64, s, lse, delta, dqkv, scale_log2, scale, ctl);
+    attn_bwd_dq_kernel<HD><<<grid, 320, L::BYTES, st>>>(q128, do128, kv64, s, lse, delta, dqkv, scale_log2, scale, ctl);
     GPTK_CUDA(cudaGetLastError());
   }
   return ST_OK;

@@ -518,6 +518,9 @@ __device__ __forceinline__ void st_pairs(__nv_bfloat16* p, int i, int half, cons
   }
 }
 
+// Every load of a (token, head) item is issued before its reductions and stores, so a warp
+// keeps several independent loads in flight (the in-place form would otherwise stop the
+// compiler from hoisting them past the stores).
 template <int PPL>
 __global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ src, const float2* __restrict__ cs, int M, int T,
                               int H, int hd, int hdp, int rope, int qk_norm, float eps, __nv_bfloat16* dst,
@@ -527,39 +530,40 @@ __global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ src, const float
   const int half = hd / 2;
   const int i = lane * PPL;
   const long long D = (long long)H * hd;
-  const int nsect = in_place ? 2 : 3;
   const int total = M * H;
   for (int wid = blockIdx.x * warps + (threadIdx.x >> 5); wid < total; wid += gridDim.x * warps) {
     const int m = wid / H, h = wid - (wid / H) * H;
     const int t = m % T;
-    for (int sct = 0; sct < nsect; ++sct) {
-      const __nv_bfloat16* sp = src + (long long)m * 3 * D + sct * D + (long long)h * hd;
-      __nv_bfloat16* dp = dst + (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
-      float a[PPL], b[PPL];
-      ld_pairs<PPL>(sp, i, half, a, b);
-      if (sct < 2) {
-        float r = 1.f;
-        if (qk_norm) {
-          float ss = 0.f;
+    const __nv_bfloat16* sp = src + (long long)m * 3 * D + (long long)h * hd;
+    __nv_bfloat16* dp = dst + (long long)m * 3 * H * hdp + (long long)h * hdp;
+    float a[3][PPL], b[3][PPL];
+    ld_pairs<PPL>(sp, i, half, a[0], b[0]);
+    ld_pairs<PPL>(sp + D, i, half, a[1], b[1]);
+    if (!in_place) ld_pairs<PPL>(sp + 2 * D, i, half, a[2], b[2]);
+    float2 e[PPL];
 #pragma unroll
-          for (int j = 0; j < PPL; ++j) ss += a[j] * a[j] + b[j] * b[j];
-          r = rsqrtf(warp_sum(ss) / hd + eps);
-          if (lane == 0) (sct == 0 ? rq : rk)[(long long)m * H + h] = r;
-        }
+    for (int j = 0; j < PPL; ++j)
+      e[j] = (rope && i + j < half) ? cs[(long long)t * half + i + j] : make_float2(1.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < PPL; ++j) {
-          if (rope && i + j < half) {
-            const float2 e = cs[(long long)t * half + i + j];
-            const float x1 = a[j], x2 = b[j];
-            a[j] = x1 * e.x - x2 * e.y;
-            b[j] = x1 * e.y + x2 * e.x;
-          }
-          a[j] *= r;
-          b[j] *= r;
-        }
+    for (int sct = 0; sct < 2; ++sct) {
+      float r = 1.f;
+      if (qk_norm) {
+        float ss = 0.f;
+#pragma unroll
+        for (int j = 0; j < PPL; ++j) ss += a[sct][j] * a[sct][j] + b[sct][j] * b[sct][j];
+        r = rsqrtf(warp_sum(ss) / hd + eps);
+        if (lane == 0) (sct == 0 ? rq : rk)[(long long)m * H + h] = r;
       }
-      st_pairs<PPL>(dp, i, half, a, b);
+#pragma unroll
+      for (int j = 0; j < PPL; ++j) {
+        const float x1 = a[sct][j], x2 = b[sct][j];
+        a[sct][j] = (x1 * e[j].x - x2 * e[j].y) * r;
+        b[sct][j] = (x1 * e[j].y + x2 * e[j].x) * r;
+      }
     }
+    st_pairs<PPL>(dp, i, half, a[0], b[0]);
+    st_pairs<PPL>(dp + (long long)H * hdp, i, half, a[1], b[1]);
+    if (!in_place) st_pairs<PPL>(dp + 2LL * H * hdp, i, half, a[2], b[2]);
   }
 }
 
@@ -578,43 +582,51 @@ __global__ void qk_bwd_kernel(const __nv_bfloat16* dpad, const __nv_bfloat16* __
   for (int wid = blockIdx.x * warps + (threadIdx.x >> 5); wid < total; wid += gridDim.x * warps) {
     const int m = wid / H, h = wid - (wid / H) * H;
     const int t = m % T;
-    for (int sct = 0; sct < 3; ++sct) {
-      if (in_place && sct == 2) break;  // dv is already in place
-      const long long po = (long long)m * 3 * H * hdp + (long long)sct * H * hdp + (long long)h * hdp;
-      __nv_bfloat16* dst = dqkv + (long long)m * 3 * D + sct * D + (long long)h * hd;
-      float a[PPL], b[PPL];
-      ld_pairs<PPL>(dpad + po, i, half, a, b);
-      if (sct < 2) {
-        if (qk_norm) {
-          // dx = r (dy - y mean(dy y)), y the normalised output that the forward saved
-          float ya[PPL], yb[PPL];
-          ld_pairs<PPL>(qpad + po, i, half, ya, yb);
-          float s = 0.f;
+    const long long po = (long long)m * 3 * H * hdp + (long long)h * hdp;
+    const long long ps = (long long)H * hdp;  // section pitch in the padded layout
+    float a[3][PPL], b[3][PPL], ya[2][PPL], yb[2][PPL];
+    ld_pairs<PPL>(dpad + po, i, half, a[0], b[0]);
+    ld_pairs<PPL>(dpad + po + ps, i, half, a[1], b[1]);
+    if (!in_place) ld_pairs<PPL>(dpad + po + 2 * ps, i, half, a[2], b[2]);
+    if (qk_norm) {
+      ld_pairs<PPL>(qpad + po, i, half, ya[0], yb[0]);
+      ld_pairs<PPL>(qpad + po + ps, i, half, ya[1], yb[1]);
+    }
+    float r2[2] = {1.f, 1.f};
+    if (qk_norm) {
+      r2[0] = rq[(long long)m * H + h];
+      r2[1] = rk[(long long)m * H + h];
+    }
+    float2 e[PPL];
 #pragma unroll
-          for (int j = 0; j < PPL; ++j) s += a[j] * ya[j] + b[j] * yb[j];
-          const float mdy = warp_sum(s) / hd;
-          const float r = (sct == 0 ? rq : rk)[(long long)m * H + h];
+    for (int j = 0; j < PPL; ++j)
+      e[j] = (rope && i + j < half) ? cs[(long long)t * half + i + j] : make_float2(1.f, 0.f);
 #pragma unroll
-          for (int j = 0; j < PPL; ++j) {
-            a[j] = r * (a[j] - ya[j] * mdy);
-            b[j] = r * (b[j] - yb[j] * mdy);
-          }
-        }
-        if (rope) {
-          // the rotation is orthogonal: its reverse rotates by -phi
+    for (int sct = 0; sct < 2; ++sct) {
+      if (qk_norm) {
+        // dx = r (dy - y mean(dy y)), y the normalised output that the forward saved
+        float s = 0.f;
 #pragma unroll
-          for (int j = 0; j < PPL; ++j) {
-            if (i + j < half) {
-              const float2 e = cs[(long long)t * half + i + j];
-              const float x1 = a[j], x2 = b[j];
-              a[j] = x1 * e.x + x2 * e.y;
-              b[j] = -x1 * e.y + x2 * e.x;
-            }
-          }
+        for (int j = 0; j < PPL; ++j) s += a[sct][j] * ya[sct][j] + b[sct][j] * yb[sct][j];
+        const float mdy = warp_sum(s) / hd;
+#pragma unroll
+        for (int j = 0; j < PPL; ++j) {
+          a[sct][j] = r2[sct] * (a[sct][j] - ya[sct][j] * mdy);
+          b[sct][j] = r2[sct] * (b[sct][j] - yb[sct][j] * mdy);
         }
       }
-      st_pairs<PPL>(dst, i, half, a, b);
+      // the rotation is orthogonal: its reverse rotates by -phi
+#pragma unroll
+      for (int j = 0; j < PPL; ++j) {
+        const float x1 = a[sct][j], x2 = b[sct][j];
+        a[sct][j] = x1 * e[j].x + x2 * e[j].y;
+        b[sct][j] = -x1 * e[j].y + x2 * e[j].x;
+      }
     }
+    __nv_bfloat16* dst = dqkv + (long long)m * 3 * D + (long long)h * hd;
+    st_pairs<PPL>(dst, i, half, a[0], b[0]);
+    st_pairs<PPL>(dst + D, i, half, a[1], b[1]);
+    if (!in_place) st_pairs<PPL>(dst + 2 * D, i, half, a[2], b[2]);
   }
 }
 

@@ -1,0 +1,123 @@
+"""Parity at the full sizes of the measured workloads, on outputs the oracle can
+compute, using properties that hold at any size.
+
+- Sequences are independent, so a batch of B copies of one sequence has the mean
+  loss, the bits per byte and the gradients of that single sequence: the GPU runs
+  the full launch configuration (d20: B=16 x T=2048; GPT-2: B=8 x T=1024) and the
+  oracle runs one sequence.
+- Causality: the first P rows of a long sequence's attention equal the length-P
+  problem (and with the output gradient zeroed past P, so do the gradients).
+- Rows of the lm_head + cross-entropy are independent: sampled rows are checked
+  against fp64 dot products."""
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def _pkg():
+    import decoder_only_gpt_tcgen05_b200 as g
+    return g
+
+
+def _cos_rel(a, b):
+    a, b = a.reshape(-1), b.reshape(-1)
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b))), float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+@pytest.mark.parametrize("name,B,T,bytes_hi", [("d20", 16, 2048, 16), ("gpt2", 8, 1024, 12)])
+def test_full_size_replicated_batch_matches_one_sequence(name, B, T, bytes_hi):
+    g = _pkg()
+    cfg = g.preset(name)
+    ocfg = O.Config(**dataclasses.asdict(cfg))
+    model = g.GPT(cfg, B, T, device=DEV, seed=0)
+    idx1, tgt1 = synth.next_token_batch(1, T, cfg.vocab_size, seed=1)
+    tb = synth.byte_table(cfg.vocab_size, 1, bytes_hi, seed=2, n_zero=5)
+    idx = torch.from_numpy(np.repeat(idx1, B, axis=0)).to(DEV)
+    tgt = torch.from_numpy(np.repeat(tgt1, B, axis=0)).to(DEV)
+    loss = model.forward_loss(idx, tgt).item()
+    grads = model.backward().clone()
+    model.forward_loss(idx, tgt)
+    assert torch.equal(model.backward(), grads)          # bitwise deterministic at full size
+    sn, sb, bpb = (t.item() for t in model.eval_bpb(idx, tgt, torch.from_numpy(tb).to(DEV)))
+    g.model.sync_status(DEV)
+    p = model.params.double().cpu().numpy()
+    f = O.forward(ocfg, p, idx1, tgt1)
+    rs, rb, _, rbpb = O.bits_per_byte(f["ell"], tgt1, tb)
+    assert abs(loss - f["loss"]) / f["loss"] <= 2e-3, (loss, f["loss"])
+    assert sb == B * rb
+    assert abs(bpb - rbpb) / rbpb <= 2e-3
+    assert abs(sn - B * rs) / abs(B * rs) <= 2e-3
+    # sampled rows of the lm_head gradient: dW[v] = sum_m (softmax - onehot)[m, v] af[m] / T
+    c = f["cache"]
+    head = "wte" if cfg.tie_embed else "lm_head"
+    W = O.unflatten(ocfg, p)[head]
+    rows = np.concatenate([np.arange(8), np.random.default_rng(3).choice(cfg.vocab_size, 56, replace=False)])
+    dz = np.exp(c["af"] @ W[rows].T - f["lse"][:, None])
+    for k, v in enumerate(rows):
+        dz[tgt1.reshape(-1) == v, k] -= 1.0
+    ref = dz.T @ c["af"] / T
+    off = O.param_offsets(ocfg)[head][0]
+    got = grads.double().cpu().numpy()[off:off + cfg.vocab_size * cfg.n_embd].reshape(cfg.vocab_size, cfg.n_embd)[rows]
+    if cfg.tie_embed:
+        # the tied table also receives the embedding gradient of the rows that occur as inputs
+        keep = ~np.isin(rows, idx1)
+        got, ref = got[keep], ref[keep]
+    cos, rel = _cos_rel(got, ref)
+    assert cos >= 0.999 and rel <= 3e-2, (cos, rel)
+
+
+def test_attention_sweep_prefix_rows_match_oracle():
+    from test_gpu_attention import _oracle_attention
+    g = _pkg()
+    H, hd, P = 10, 128, 512
+    # numpy fills row-major, so the first P rows of every draw below are the same numbers:
+    # one oracle run on the length-P problem serves every T
+    qkv_p = torch.from_numpy(synth.normal((P, 3 * H * hd), 3)).bfloat16()
+    dout_p = torch.from_numpy(synth.normal((P, H * hd), 4)).bfloat16()
+    o_ref, lse_ref, dqkv_ref = _oracle_attention(qkv_p.double().numpy(), 1, P, H, hd, True, True,
+                                                 dout_p.double().numpy())
+    for T in (512, 1024, 2048, 4096, 8192):
+        B = 32768 // T
+        qkv = torch.from_numpy(synth.normal((B * T, 3 * H * hd), 3)).bfloat16()
+        dout = torch.from_numpy(synth.normal((B * T, H * hd), 4)).bfloat16()
+        assert torch.equal(qkv[:P], qkv_p) and torch.equal(dout[:P], dout_p)
+        dout.view(B, T, H * hd)[0, P:] = 0
+        f = g.ops.attention_fwd(qkv.to(DEV), B, T, H, hd)
+        dq = g.ops.attention_bwd(f, dout.to(DEV), B, T, H, hd)
+        torch.cuda.synchronize()
+        o = f["o"][:P].double().cpu().numpy()
+        cos, rel = _cos_rel(o, o_ref)
+        assert cos >= 0.9999 and rel <= 1e-2, (T, cos, rel)
+        assert np.abs(f["lse"][0, :, :P].double().cpu().numpy() - lse_ref[0]).max() < 2e-2
+        got = dq[:T].double().cpu().numpy()   # sequence 0
+        for i, nm in enumerate("qkv"):
+            sl = slice(i * H * hd, (i + 1) * H * hd)
+            cos, rel = _cos_rel(got[:P, sl], dqkv_ref[:, sl])
+            assert cos >= 0.999 and rel <= 3e-2, (T, nm, cos, rel)
+            if T > P:
+                assert np.abs(got[P:, sl]).max() == 0.0, (T, nm)
+
+
+def test_d26_lmhead_ce_full_size_sampled_rows():
+    g = _pkg()
+    M, D, V = 32768, 1664, 32768
+    x = torch.from_numpy(synth.normal((M, D), 41)).bfloat16()
+    w = torch.from_numpy(synth.normal((V, D), 42, std=0.05)).bfloat16()
+    tg = torch.from_numpy(synth.zipf_tokens(M, V, seed=43))
+    ell, lse = g.ops.lmhead_ce_fwd(x.to(DEV), w.to(DEV), tg.to(DEV))
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(44).choice(M, 64, replace=False)
+    z = x[rows].double().numpy() @ w.double().numpy().T
+    ref_ell, ref_lse = O.cross_entropy(z, tg.numpy()[rows])
+    assert np.allclose(ell.cpu().numpy()[rows], ref_ell, rtol=2e-3, atol=2e-3)
+    assert np.allclose(lse.cpu().numpy()[rows], ref_lse, rtol=1e-4, atol=1e-3)
+    assert math.isfinite(float(ell.sum().item()))
