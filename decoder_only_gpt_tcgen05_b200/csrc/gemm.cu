@@ -110,8 +110,7 @@ int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, u
 // ------------------------------------------------------------ GEMM launcher
 
 template <int BN, int EPI, bool LONGK>
-static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tc2,
-                         const CUtensorMap& tr, const GemmParams& p, cudaStream_t st) {
+static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
   using C = GemmCfg<BN, LONGK>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -120,34 +119,38 @@ static int launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
     GPTK_CUDA(cudaFuncSetAttribute(gemm_kernel<BN, EPI, LONGK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
     attr_set[dev & 63] = true;
   }
-  const int tiles = p.tiles_m * p.tiles_n;
+  const int tiles = p.tile_start[p.n_prob];
   int grid = num_sms();
   if (grid > tiles) grid = tiles;
-  const double M = p.M, N = p.N, K = p.K;
-  double out_bytes = M * N * 2;
-  if (EPI == EPI_F32 || EPI == EPI_RESID) out_bytes = M * N * 4 * (1 + (p.accumulate || EPI == EPI_RESID));
-  if (EPI == EPI_UP) out_bytes = M * N * (p.out ? 4 : 2);
-  if (EPI == EPI_ACTBWD) out_bytes = M * N * 4;
-  if (EPI == EPI_CE_FWD) out_bytes = M * p.tiles_n * 8;
-  Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, 2.0 * M * N * K, (M * K + N * K) * 2 + out_bytes, st);
-  gemm_kernel<BN, EPI, LONGK><<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, tc, tc2, tr, p);
+  double flops = 0, bytes = 0;
+  for (int q = 0; q < p.n_prob; ++q) {
+    const double M = p.pM[q], N = p.pN[q], K = p.K;
+    double out_bytes = M * N * 2;
+    if (EPI == EPI_F32 || EPI == EPI_RESID) out_bytes = M * N * 4 * (1 + (p.accumulate || EPI == EPI_RESID));
+    if (EPI == EPI_UP) out_bytes = M * N * (p.out ? 4 : 2);
+    if (EPI == EPI_ACTBWD) out_bytes = M * N * 4;
+    if (EPI == EPI_CE_FWD) out_bytes = M * p.tiles_n * 8;
+    flops += 2.0 * M * N * K;
+    bytes += (M * K + N * K) * 2 + out_bytes;
+  }
+  Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, flops, bytes, st);
+  gemm_kernel<BN, EPI, LONGK><<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
 
 template <int BN>
-static int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
-                        const CUtensorMap& tc2, const CUtensorMap& tr, const GemmParams& p, cudaStream_t st) {
+static int dispatch_epi(int epi, const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
   // reductions over all tokens (weight gradients) and over the vocabulary take the deep ring
-  if (epi == EPI_F32 && p.K >= 8192) return launch_gemm_t<BN, EPI_F32, true>(ta, tb, tc, tc2, tr, p, st);
+  if (epi == EPI_F32 && p.K >= 8192) return launch_gemm_t<BN, EPI_F32, true>(maps, p, st);
   switch (epi) {
-    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false>(ta, tb, tc, tc2, tr, p, st);
-    case EPI_F32: return launch_gemm_t<BN, EPI_F32, false>(ta, tb, tc, tc2, tr, p, st);
-    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false>(ta, tb, tc, tc2, tr, p, st);
-    case EPI_UP: return launch_gemm_t<BN, EPI_UP, false>(ta, tb, tc, tc2, tr, p, st);
-    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD, false>(ta, tb, tc, tc2, tr, p, st);
-    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD, false>(ta, tb, tc, tc2, tr, p, st);
-    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD, false>(ta, tb, tc, tc2, tr, p, st);
+    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false>(maps, p, st);
+    case EPI_F32: return launch_gemm_t<BN, EPI_F32, false>(maps, p, st);
+    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false>(maps, p, st);
+    case EPI_UP: return launch_gemm_t<BN, EPI_UP, false>(maps, p, st);
+    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD, false>(maps, p, st);
+    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD, false>(maps, p, st);
+    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD, false>(maps, p, st);
   }
   return set_error(ST_INVALID_ARG, "unknown GEMM epilogue");
 }
@@ -156,23 +159,47 @@ static bool aligned16(const void* ptr, long long ld, int esize) {
   return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0 && ((ld * esize) & 15) == 0;
 }
 
+static int operand_maps(const Operand& A, const Operand& B, int M, int N, int K, int bn, CUtensorMap* ta,
+                        CUtensorMap* tb) {
+  if (!A.mn_major) {
+    GPTK_TRY(make_tmap_2d(ta, A.ptr, K, M, A.ld, 64, 128));
+  } else {
+    GPTK_TRY(make_tmap_2d(ta, A.ptr, M, K, A.ld, 64, 64));
+  }
+  if (!B.mn_major) {
+    GPTK_TRY(make_tmap_2d(tb, B.ptr, K, N, B.ld, 64, bn));
+  } else {
+    GPTK_TRY(make_tmap_2d(tb, B.ptr, N, K, B.ld, 64, 64));
+  }
+  return ST_OK;
+}
+
+// band height: a few m-tiles whose A rows (128 x K bf16 each) stay within about 48 MB of L2
+static int band_height(int tiles_m, int K) {
+  const long long a_band_row = 128LL * K * 2;
+  int gm = 8;  // measured best among 8, 16, 32 and the plain order on B200 (d20 shapes)
+  const int gm_l2 = (int)((48LL << 20) / (a_band_row > 0 ? a_band_row : 1));
+  if (gm > gm_l2) gm = gm_l2;
+  // very long K (weight gradients): bands would be too thin to help; keep the plain order,
+  // whose concurrent tiles share B columns while moving through K in step
+  if (gm < 8) gm = tiles_m;
+  // tuning override: GPT_GEMM_GROUP_M=<n> forces the band height (0 = plain order)
+  static const int forced = []() {
+    const char* e = std::getenv("GPT_GEMM_GROUP_M");
+    return e ? std::atoi(e) : -1;
+  }();
+  if (forced == 0) gm = tiles_m;
+  if (forced > 0) gm = forced < tiles_m ? forced : tiles_m;
+  if (gm > tiles_m) gm = tiles_m;
+  return gm < 1 ? 1 : gm;
+}
+
 int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st) {
   if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return set_error(ST_INVALID_ARG, "GEMM with an empty dimension");
-  CUtensorMap ta, tb, tc, tc2, tr;
-  std::memset(&tc, 0, sizeof(tc));
-  std::memset(&tc2, 0, sizeof(tc2));
-  std::memset(&tr, 0, sizeof(tr));
-  if (!A.mn_major) {
-    GPTK_TRY(make_tmap_2d(&ta, A.ptr, p.K, p.M, A.ld, 64, 128));
-  } else {
-    GPTK_TRY(make_tmap_2d(&ta, A.ptr, p.M, p.K, A.ld, 64, 64));
-  }
-  if (!B.mn_major) {
-    GPTK_TRY(make_tmap_2d(&tb, B.ptr, p.K, p.N, B.ld, 64, bn));
-  } else {
-    GPTK_TRY(make_tmap_2d(&tb, B.ptr, p.N, p.K, B.ld, 64, 64));
-  }
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  GPTK_TRY(operand_maps(A, B, p.M, p.N, p.K, bn, &maps.a[0], &maps.b[0]));
   // output / input tensor maps of the TMA epilogue, where the layout allows one
   p.tma_out = 0;
   const bool f32out = (epi == EPI_F32 || epi == EPI_RESID);
@@ -185,39 +212,71 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   if (ok && epi == EPI_UP) ok = aligned16(p.out2, p.ldo, 2);
   if (ok && epi == EPI_ACTBWD) ok = aligned16(p.aux, p.ld_aux, 2);
   if (ok) {
-    if (p.out) GPTK_TRY(make_tmap_2d(&tc, p.out, p.N, p.M, p.ldo, bw, 32, es));
-    if (epi == EPI_UP) GPTK_TRY(make_tmap_2d(&tc2, p.out2, p.N, p.M, p.ldo, 64, 32, 2));
-    if (epi == EPI_RESID) GPTK_TRY(make_tmap_2d(&tr, p.resid, p.N, p.M, p.ldr, 32, 32, 4));
-    if (epi == EPI_ACTBWD) GPTK_TRY(make_tmap_2d(&tr, p.aux, p.N, p.M, p.ld_aux, 64, 32, 2));
+    if (p.out) GPTK_TRY(make_tmap_2d(&maps.c[0], p.out, p.N, p.M, p.ldo, bw, 32, es));
+    if (epi == EPI_UP) GPTK_TRY(make_tmap_2d(&maps.c2, p.out2, p.N, p.M, p.ldo, 64, 32, 2));
+    if (epi == EPI_RESID) GPTK_TRY(make_tmap_2d(&maps.r, p.resid, p.N, p.M, p.ldr, 32, 32, 4));
+    if (epi == EPI_ACTBWD) GPTK_TRY(make_tmap_2d(&maps.r, p.aux, p.N, p.M, p.ld_aux, 64, 32, 2));
     p.tma_out = 1;
   }
   p.a_mn = A.mn_major;
   p.b_mn = B.mn_major;
   p.tiles_m = (p.M + 127) / 128;
   p.tiles_n = (p.N + bn - 1) / bn;
-  {
-    // band height: a few m-tiles whose A rows (128 x K bf16 each) stay within about 48 MB of L2
-    const long long a_band_row = 128LL * p.K * 2;
-    int gm = 8;  // measured best among 8, 16, 32 and the plain order on B200 (d20 shapes)
-    const int gm_l2 = (int)((48LL << 20) / (a_band_row > 0 ? a_band_row : 1));
-    if (gm > gm_l2) gm = gm_l2;
-    // very long K (weight gradients): bands would be too thin to help; keep the plain order,
-    // whose concurrent tiles share B columns while moving through K in step
-    if (gm < 8) gm = p.tiles_m;
-    // tuning override: GPT_GEMM_GROUP_M=<n> forces the band height (0 = plain order)
-    static const int forced = []() {
-      const char* e = std::getenv("GPT_GEMM_GROUP_M");
-      return e ? std::atoi(e) : -1;
-    }();
-    if (forced == 0) gm = p.tiles_m;
-    if (forced > 0) gm = forced < p.tiles_m ? forced : p.tiles_m;
-    if (gm > p.tiles_m) gm = p.tiles_m;
-    p.group_m = gm;
-  }
+  p.group_m = band_height(p.tiles_m, p.K);
+  p.n_prob = 1;
+  p.tile_start[0] = 0;
+  p.tile_start[1] = p.tiles_m * p.tiles_n;
+  p.pM[0] = p.M;
+  p.pN[0] = p.N;
+  p.ptiles_m[0] = p.tiles_m;
+  p.ptiles_n[0] = p.tiles_n;
+  p.pgroup_m[0] = p.group_m;
   p.ctl = device_ctl();
   if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
-  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, tc, tc2, tr, p, st)
-                   : dispatch_epi<128>(epi, ta, tb, tc, tc2, tr, p, st);
+  return bn == 256 ? dispatch_epi<256>(epi, maps, p, st) : dispatch_epi<128>(epi, maps, p, st);
+}
+
+int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
+                   cudaStream_t st) {
+  if (n < 1 || n > kMaxProblems) return set_error(ST_INVALID_ARG, "grouped GEMM: 1 to 4 problems");
+  if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
+  GemmMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.K = K;
+  p.a_mn = a_mn;
+  p.b_mn = b_mn;
+  p.accumulate = 1;
+  p.hd = p.hdp = 1;
+  p.tma_out = 1;
+  p.prof_kind = prof_kind;
+  p.n_prob = n;
+  int start = 0;
+  for (int q = 0; q < n; ++q) {
+    const GroupProblem& g = probs[q];
+    if (g.M <= 0 || g.N <= 0 || !aligned16(g.out, g.ldo, 4))
+      return set_error(ST_INVALID_ARG, "grouped GEMM: bad problem");
+    GPTK_TRY(operand_maps(Operand{g.a, g.lda, a_mn}, Operand{g.b, g.ldb, b_mn}, g.M, g.N, K, bn, &maps.a[q],
+                          &maps.b[q]));
+    GPTK_TRY(make_tmap_2d(&maps.c[q], g.out, g.N, g.M, g.ldo, 32, 32, 4));
+    p.pM[q] = g.M;
+    p.pN[q] = g.N;
+    p.ptiles_m[q] = (g.M + 127) / 128;
+    p.ptiles_n[q] = (g.N + bn - 1) / bn;
+    p.pgroup_m[q] = band_height(p.ptiles_m[q], K);
+    p.tile_start[q] = start;
+    start += p.ptiles_m[q] * p.ptiles_n[q];
+  }
+  p.tile_start[n] = start;
+  p.M = p.pM[0];
+  p.N = p.pN[0];
+  p.tiles_m = p.ptiles_m[0];
+  p.tiles_n = p.ptiles_n[0];
+  p.group_m = p.pgroup_m[0];
+  p.ctl = device_ctl();
+  if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
+  return bn == 256 ? dispatch_epi<256>(EPI_F32, maps, p, st) : dispatch_epi<128>(EPI_F32, maps, p, st);
 }
 
 }  // namespace gptk

@@ -63,6 +63,20 @@ struct GemmParams {
   const float* ce_lse;        // [M] natural-log logsumexp (backward)
   float ce_scale;             // 1/M_total (backward)
   int prof_kind;              // host only: profiler family of this call (0 = generic GEMM)
+  // grouped launch: up to kMaxProblems products with the same K, operand layouts and epilogue
+  // share one persistent tile space; problem q owns tiles [tile_start[q], tile_start[q+1]).
+  int n_prob;
+  int tile_start[5];
+  int pM[4], pN[4], ptiles_m[4], ptiles_n[4], pgroup_m[4];
+};
+
+constexpr int kMaxProblems = 4;
+
+// Tensor maps of a launch: A and B (and the output C) per problem, plus the second output and
+// the epilogue input of single-problem launches.
+struct GemmMaps {
+  CUtensorMap a[kMaxProblems], b[kMaxProblems], c[kMaxProblems];
+  CUtensorMap c2, r;
 };
 
 // LONGK: the variant for very long reductions (weight gradients over all tokens), where the
@@ -219,26 +233,35 @@ __device__ __forceinline__ void epi_chunk_generic(const GemmParams& p, float* v,
   }
 }
 
-// Tile t -> (tm, tn).  Tiles are taken in bands of group_m m-tiles; inside a band the m index
-// runs fastest, and the band sweeps every n-tile before the next band starts, so the A rows
-// of a band stay in L2 while all of B passes by.
-__device__ __forceinline__ void tile_coords(const GemmParams& p, int tile, int& tm, int& tn) {
-  const int per_band = p.group_m * p.tiles_n;
-  const int band = tile / per_band;
-  const int first = band * p.group_m;
-  const int gm = min(p.group_m, p.tiles_m - first);
-  const int local = tile - band * per_band;
-  tm = first + local % gm;
-  tn = local / gm;
+// Tile t -> (problem, tm, tn).  Within a problem, tiles are taken in bands of group_m m-tiles;
+// inside a band the m index runs fastest, and the band sweeps every n-tile before the next
+// band starts, so the A rows of a band stay in L2 while all of B passes by.
+struct TileInfo {
+  int prob, tm, tn, M, N;
+};
+__device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int tile) {
+  TileInfo t;
+  int q = 0;
+  while (q + 1 < p.n_prob && tile >= p.tile_start[q + 1]) ++q;
+  t.prob = q;
+  t.M = p.pM[q];
+  t.N = p.pN[q];
+  const int local = tile - p.tile_start[q];
+  const int per_band = p.pgroup_m[q] * p.ptiles_n[q];
+  const int band = local / per_band;
+  const int first = band * p.pgroup_m[q];
+  const int gm = min(p.pgroup_m[q], p.ptiles_m[q] - first);
+  const int in_band = local - band * per_band;
+  t.tm = first + in_band % gm;
+  t.tn = in_band / gm;
+  return t;
 }
 
 // --------------------------------------------------------------- the kernel
 
 template <int BN, int EPI, bool LONGK>
 __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
-                const __grid_constant__ CUtensorMap tmR, const __grid_constant__ GemmParams p) {
+    gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using C = GemmCfg<BN, LONGK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -271,8 +294,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     for (int i = 0; i < 2 * C::EPI_WARPS; ++i) mbar_init(&inbar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
+    for (int q = 0; q < p.n_prob; ++q) {
+      prefetch_tmap(&maps.a[q]);
+      prefetch_tmap(&maps.b[q]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * BN);
@@ -283,7 +308,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = p.tiles_m * p.tiles_n;
+  const int num_tiles = p.tile_start[p.n_prob];
   const int num_k = (p.K + C::BK - 1) / C::BK;
 
   if (warp == 0 && lane == 0) {
@@ -293,8 +318,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     uint32_t pending = 0;  // stages with a load in flight that the MMA has not yet released
     bool ok = true;
     for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-      int tm, tn;
-      tile_coords(p, tile, tm, tn);
+      const TileInfo ti = tile_info(p, tile);
+      const int tm = ti.tm, tn = ti.tn;
+      const CUtensorMap* tmA = &maps.a[ti.prob];
+      const CUtensorMap* tmB = &maps.b[ti.prob];
       for (int kb = 0; kb < num_k; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctl, abort_flag, 1)) {
           ok = false;
@@ -305,17 +332,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
         uint8_t* a = sA + stage * C::A_BYTES;
         uint8_t* b = sB + stage * C::B_BYTES;
         if (!p.a_mn) {
-          tma_load_2d(a, &tmA, &full[stage], kb * C::BK, tm * C::BM);
+          tma_load_2d(a, tmA, &full[stage], kb * C::BK, tm * C::BM);
         } else {
 #pragma unroll
           for (int c = 0; c < C::BM / 64; ++c)
-            tma_load_2d(a + c * 8192, &tmA, &full[stage], tm * C::BM + c * 64, kb * C::BK);
+            tma_load_2d(a + c * 8192, tmA, &full[stage], tm * C::BM + c * 64, kb * C::BK);
         }
         if (!p.b_mn) {
-          tma_load_2d(b, &tmB, &full[stage], kb * C::BK, tn * BN);
+          tma_load_2d(b, tmB, &full[stage], kb * C::BK, tn * BN);
         } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tma_load_2d(b + c * 8192, &tmB, &full[stage], tn * BN + c * 64, kb * C::BK);
+          for (int c = 0; c < BN / 64; ++c) tma_load_2d(b + c * 8192, tmB, &full[stage], tn * BN + c * 64, kb * C::BK);
         }
         pending |= 1u << stage;
         if (++stage == C::STAGES) {
@@ -403,20 +430,24 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     constexpr bool HAS_IN = (EPI == EPI_RESID || EPI == EPI_ACTBWD);
     constexpr int HALF = BN * 4 / C::EPI_WARPS;  // columns per epilogue warp
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int tm, tn;
-      tile_coords(p, tile, tm, tn);
+      const TileInfo ti = tile_info(p, tile);
+      const int tm = ti.tm, tn = ti.tn;
+      const int pN = ti.N;
+      const CUtensorMap* tmC = &maps.c[ti.prob];
+      const CUtensorMap* tmC2 = &maps.c2;
+      const CUtensorMap* tmR = &maps.r;
       const int row = tm * 128 + r_in_tile;
       const int row0 = tm * 128 + quad * 32;
-      const bool row_ok = row < p.M;
+      const bool row_ok = row < ti.M;
       const int c_begin = chalf * HALF;
       const int n0 = tn * BN;
       const bool tma = p.tma_out && EPI != EPI_CE_FWD;
       // the first input chunk of the tile can load while the main loop still runs
-      if (HAS_IN && tma && n0 + c_begin < p.N && lane == 0) {
+      if (HAS_IN && tma && n0 + c_begin < pN && lane == 0) {
         const int b = chunk_ctr & 1;
         bulk_wait_read<1>();
         mbar_expect_tx(&ibar[b], 4096);
-        tma_load_2d(stg_ptr + b * 4096, &tmR, &ibar[b], n0 + c_begin, row0);
+        tma_load_2d(stg_ptr + b * 4096, tmR, &ibar[b], n0 + c_begin, row0);
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.ctl, abort_flag, 5)) break;
       tc_fence_after();
@@ -463,7 +494,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
         // TMA path: chunks of 32 fp32 or 64 bf16 columns (128-byte staging rows)
         for (int c = c_begin; c < c_begin + HALF; c += CW) {
           const int col0 = n0 + c;
-          if (col0 >= p.N) break;
+          if (col0 >= pN) break;
           const int b = chunk_ctr & 1;
           const uint32_t buf = stg + b * 4096;
           const bool two_out = (EPI == EPI_UP) && p.out != nullptr;
@@ -479,8 +510,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
           tmem_ld32(trow + c, *reinterpret_cast<float(*)[32]>(&v[0]));
           if (CW == 64) tmem_ld32(trow + c + 32, *reinterpret_cast<float(*)[32]>(&v[32 % CW]));
           if (EPI != EPI_ACTBWD && EPI != EPI_CE_BWD) {
-            add_bias32(v, p.bias, col0, p.N);
-            if (CW == 64) add_bias32(v + (32 % CW), p.bias, col0 + 32, p.N);
+            add_bias32(v, p.bias, col0, pN);
+            if (CW == 64) add_bias32(v + (32 % CW), p.bias, col0 + 32, pN);
           }
           if (HAS_IN) {
             if (!mbar_wait(&ibar[b], (in_uses >> b) & 1u, p.ctl, abort_flag, 7)) {
@@ -540,19 +571,19 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
           __syncwarp();
           if (lane == 0) {
             if (EPI == EPI_UP) {
-              tma_store_2d(&tmC2, stg_ptr + b * 4096, col0, row0);
-              if (two_out) tma_store_2d(&tmC, stg_ptr + (b ^ 1) * 4096, col0, row0);
+              tma_store_2d(tmC2, stg_ptr + b * 4096, col0, row0);
+              if (two_out) tma_store_2d(tmC, stg_ptr + (b ^ 1) * 4096, col0, row0);
             } else if (EPI == EPI_F32 && p.accumulate) {
-              tma_reduce_add_2d(&tmC, stg_ptr + b * 4096, col0, row0);
+              tma_reduce_add_2d(tmC, stg_ptr + b * 4096, col0, row0);
             } else {
-              tma_store_2d(&tmC, stg_ptr + b * 4096, col0, row0);
+              tma_store_2d(tmC, stg_ptr + b * 4096, col0, row0);
             }
             bulk_commit();
             // prefetch the next input chunk into the other buffer once its last store has read it
-            if (HAS_IN && c + CW < c_begin + HALF && col0 + CW < p.N) {
+            if (HAS_IN && c + CW < c_begin + HALF && col0 + CW < pN) {
               bulk_wait_read<1>();
               mbar_expect_tx(&ibar[b ^ 1], 4096);
-              tma_load_2d(stg_ptr + (b ^ 1) * 4096, &tmR, &ibar[b ^ 1], col0 + CW, row0);
+              tma_load_2d(stg_ptr + (b ^ 1) * 4096, tmR, &ibar[b ^ 1], col0 + CW, row0);
             }
           }
           ++chunk_ctr;

@@ -86,4 +86,19 @@ struct GemmParams;
 // C[M,N] = A[M,K] B[N,K]^T with the fused epilogue `epi`; bn = 128 or 256.
 int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st);
 
+// One product of a grouped launch: out[M,N] += A B^T in fp32 (accumulating).
+struct GroupProblem {
+  const void* a;
+  long long lda;
+  const void* b;
+  long long ldb;
+  int M, N;
+  float* out;
+  long long ldo;
+};
+// Up to 4 accumulating fp32 products with the same K and operand layouts in one persistent
+// launch (their tiles share one schedule, so small products do not leave SMs idle).
+int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
+                   cudaStream_t st);
+
 }  // namespace gptk

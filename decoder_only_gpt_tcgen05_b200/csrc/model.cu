@@ -16,7 +16,6 @@
 // embedding scatter.
 #include <cmath>
 #include <cstring>
-#include <mutex>
 #include <string>
 #include <vector>
 
@@ -172,15 +171,15 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   p.loss_d = take(loss_reduce_blocks() * 2 * 8);
   p.loss_i = take(loss_reduce_blocks() * 2 * 8);
   p.loss_f = take(64);
-  p.dlog = take(2 * (size_t)p.Mc * p.Vp * 2);  // two slots (see backward_impl)
+  p.dlog = take((size_t)p.Mc * p.Vp * 2);
   p.da = take(M * D * 4);
   p.dres = take(M * D * 4);
-  p.dres_bf = take(2 * M * D * 2);
-  p.du = take(2 * M * F * 2);
+  p.dres_bf = take(2 * M * D * 2);  // one per sublayer of a layer
+  p.du = take(M * F * 2);
   p.do_pad = take(M * H * hdp * 2);
   p.delta = take(M * H * 4);
-  p.dqkv_pad = take(2 * M * 3 * H * hdp * 2);
-  p.dqkv = take(2 * M * 3 * D * 2);
+  p.dqkv_pad = take(M * 3 * H * hdp * 2);
+  p.dqkv = take(M * 3 * D * 2);
   long long maxN = F > 3 * D ? F : 3 * D;
   long long rows = norm_bwd_max_blocks() > colsum_max_chunks() ? norm_bwd_max_blocks() : colsum_max_chunks();
   p.partN = maxN;
@@ -371,43 +370,6 @@ static int norm_backward(const gpt_config& c, const Plan& pl, const float* dy, c
   return ST_OK;
 }
 
-// The weight-gradient GEMMs only feed the final gradients, so they run on a side stream:
-// each forks from the main stream once its inputs exist and the main stream joins it at
-// the end.  Their inputs (dlogits chunks, the bf16 residual gradient, du, dqkv) live in
-// two-slot rings; before the main stream rewrites a slot it waits for the last
-// weight-gradient GEMM that read it.  Stream and events are created once per device.
-struct SideCtx {
-  cudaStream_t side = nullptr;
-  cudaEvent_t ev[64];
-  int next = 0;
-  bool ready = false;
-};
-
-static SideCtx g_side[64];
-static std::mutex g_side_mu;
-
-static int side_ctx(SideCtx** out) {
-  int dev = 0;
-  GPTK_CUDA(cudaGetDevice(&dev));
-  std::lock_guard<std::mutex> lk(g_side_mu);
-  SideCtx& s = g_side[dev & 63];
-  if (!s.ready) {
-    GPTK_CUDA(cudaStreamCreateWithFlags(&s.side, cudaStreamNonBlocking));
-    for (int i = 0; i < 64; ++i) GPTK_CUDA(cudaEventCreateWithFlags(&s.ev[i], cudaEventDisableTiming));
-    s.ready = true;
-  }
-  *out = &s;
-  return ST_OK;
-}
-
-static cudaEvent_t next_event(SideCtx* s) { return s->ev[(s->next++) & 63]; }
-
-static constexpr bool kUseSideStream = false;
-
-struct Slot {
-  cudaEvent_t reader = nullptr;  // last side-stream GEMM that read this slot
-};
-
 static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, const float* params, void* ws,
                          float* grads, int accumulate, cudaStream_t st) {
   const int M = pl.M, D = pl.D, H = pl.H, hd = pl.hd, hdp = pl.hdp, F = pl.F, T = pl.T, B = pl.B, V = pl.V;
@@ -426,49 +388,14 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
   float* delta = at<float>(ws, pl.delta);
   float* pa = at<float>(ws, pl.part_a);
   float* pb = at<float>(ws, pl.part_b);
-  // two-slot rings
-  __nv_bfloat16* dlog_s[2] = {at<__nv_bfloat16>(ws, pl.dlog), at<__nv_bfloat16>(ws, pl.dlog) + (size_t)pl.Mc * pl.Vp};
-  __nv_bfloat16* dres_bf_s[2] = {at<__nv_bfloat16>(ws, pl.dres_bf), at<__nv_bfloat16>(ws, pl.dres_bf) + MD};
-  __nv_bfloat16* du_s[2] = {at<__nv_bfloat16>(ws, pl.du), at<__nv_bfloat16>(ws, pl.du) + (size_t)M * F};
-  __nv_bfloat16* dqkvp_s[2] = {at<__nv_bfloat16>(ws, pl.dqkv_pad),
-                               at<__nv_bfloat16>(ws, pl.dqkv_pad) + (size_t)M * 3 * H * hdp};
-  __nv_bfloat16* dqkv_s[2] = {hdp == hd ? dqkvp_s[0] : at<__nv_bfloat16>(ws, pl.dqkv),
-                              hdp == hd ? dqkvp_s[1] : at<__nv_bfloat16>(ws, pl.dqkv) + (size_t)M * 3 * D};
-  Slot dlog_r[2], dres_r[2], du_r[2], dqkv_r[2];
-  int dlog_i = 0, dres_i = 0, du_i = 0, dqkv_i = 0;
-
-  // Weight-gradient GEMMs on a second stream were measured to give no gain (the persistent
-  // GEMMs already occupy every SM), so by default everything stays on the caller's stream and
-  // the fork / mark / claim steps below reduce to nothing.
-  SideCtx* sc = nullptr;
-  cudaStream_t side = st;
-  if (kUseSideStream) {
-    GPTK_TRY(side_ctx(&sc));
-    side = sc->side;
-  }
-  // main -> side: the side stream may start what is enqueued next on it
-  auto fork = [&]() -> int {
-    if (side == st) return ST_OK;
-    cudaEvent_t e = next_event(sc);
-    GPTK_CUDA(cudaEventRecord(e, st));
-    GPTK_CUDA(cudaStreamWaitEvent(side, e, 0));
-    return ST_OK;
-  };
-  // side -> event marking the completion of the side work enqueued so far
-  auto mark = [&](Slot& a, Slot* b2) -> int {
-    if (side == st) return ST_OK;
-    cudaEvent_t e = next_event(sc);
-    GPTK_CUDA(cudaEventRecord(e, side));
-    a.reader = e;
-    if (b2) b2->reader = e;
-    return ST_OK;
-  };
-  // before the main stream overwrites a slot: wait for its last reader
-  auto claim = [&](Slot& s) -> int {
-    if (s.reader) GPTK_CUDA(cudaStreamWaitEvent(st, s.reader, 0));
-    s.reader = nullptr;
-    return ST_OK;
-  };
+  __nv_bfloat16* dlog = at<__nv_bfloat16>(ws, pl.dlog);
+  // bf16 copies of the residual gradient: one for each sublayer of a layer, because the
+  // layer's weight gradients (launched together at the end of the layer) read both
+  __nv_bfloat16* dres_bf_mlp = at<__nv_bfloat16>(ws, pl.dres_bf);
+  __nv_bfloat16* dres_bf_att = at<__nv_bfloat16>(ws, pl.dres_bf) + MD;
+  __nv_bfloat16* du = at<__nv_bfloat16>(ws, pl.du);
+  __nv_bfloat16* dqkv_pad = at<__nv_bfloat16>(ws, pl.dqkv_pad);
+  __nv_bfloat16* dqkv = hdp == hd ? dqkv_pad : at<__nv_bfloat16>(ws, pl.dqkv);
 
   if (!accumulate) GPTK_CUDA(cudaMemsetAsync(grads, 0, (size_t)pl.P * 4, st));
 
@@ -476,8 +403,6 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
   const long long wlm = c.tie_embed ? Lo.wte : Lo.lm_head;
   for (int r0 = 0; r0 < M; r0 += pl.Mc) {
     const int mc = (M - r0) < pl.Mc ? (M - r0) : pl.Mc;
-    __nv_bfloat16* dlog = dlog_s[dlog_i];
-    GPTK_TRY(claim(dlog_r[dlog_i]));
     {
       GemmParams p = gp(mc, V, D);
       p.out = dlog;
@@ -488,15 +413,13 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       p.prof_kind = PK_GEMM_LM_BWD;
       GPTK_TRY(gemm(EPI_CE_BWD, Operand{af + (size_t)r0 * D, D, 0}, Operand{wbf + wlm, D, 0}, p, st, 256));
     }
-    GPTK_TRY(fork());
-    {  // d W_lm += dlogits^T af   (side stream)
+    {  // d W_lm += dlogits^T af
       GemmParams p = gp(V, D, mc);
       p.out = grads + wlm;
       p.ldo = D;
       p.accumulate = 1;
       p.prof_kind = PK_GEMM_WGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 1}, Operand{af + (size_t)r0 * D, D, 1}, p, side));
-      GPTK_TRY(mark(dlog_r[dlog_i], nullptr));
+      GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 1}, Operand{af + (size_t)r0 * D, D, 1}, p, st));
     }
     {  // d af = dlogits W_lm
       GemmParams p = gp(mc, D, V);
@@ -505,11 +428,9 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       p.prof_kind = PK_GEMM_LM_BWD;
       GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 0}, Operand{wbf + wlm, D, 1}, p, st));
     }
-    dlog_i ^= 1;
   }
-  GPTK_TRY(claim(dres_r[dres_i]));
   GPTK_TRY(norm_backward(c, pl, da, xs + (size_t)(2 * pl.L) * MD, stf, params, Lo.lnf_g, Lo.lnf_b, grads, dres, 1,
-                         dres_bf_s[dres_i], pa, pb, st));
+                         dres_bf_mlp, pa, pb, st));
 
   for (int l = pl.L - 1; l >= 0; --l) {
     const LayerOff& o = Lo.layer[l];
@@ -528,18 +449,6 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
     const __nv_bfloat16* h = at<__nv_bfloat16>(ws, pl.h) + (size_t)l * M * F;
 
     // ---- MLP: x_out = x_mid + act(N(x_mid) W_up^T + b_up) W_down^T + b_down
-    __nv_bfloat16* dres_bf = dres_bf_s[dres_i];
-    GPTK_TRY(fork());
-    {  // dW_down += dres^T h   (side stream)
-      GemmParams p = gp(D, F, M);
-      p.out = grads + o.w_down;
-      p.ldo = F;
-      p.accumulate = 1;
-      p.prof_kind = PK_GEMM_WGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{dres_bf, D, 1}, Operand{h, F, 1}, p, side));
-    }
-    __nv_bfloat16* du = du_s[du_i];
-    GPTK_TRY(claim(du_r[du_i]));
     {  // du = (dres W_down) * act'(u)
       GemmParams p = gp(M, F, D);
       p.out = du;
@@ -548,19 +457,9 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       p.ld_aux = F;
       p.act = c.act == 1 ? 2 : c.act;
       p.prof_kind = PK_GEMM_DGRAD;
-      GPTK_TRY(gemm(EPI_ACTBWD, Operand{dres_bf, D, 0}, Operand{wbf + o.w_down, F, 1}, p, st));
+      GPTK_TRY(gemm(EPI_ACTBWD, Operand{dres_bf_mlp, D, 0}, Operand{wbf + o.w_down, F, 1}, p, st));
     }
     if (o.b_down >= 0) GPTK_TRY(bias_grad_f32(dres, M, D, pa, grads + o.b_down, st));
-    GPTK_TRY(fork());
-    {  // dW_up += du^T a2   (side stream)
-      GemmParams p = gp(F, D, M);
-      p.out = grads + o.w_up;
-      p.ldo = D;
-      p.accumulate = 1;
-      p.prof_kind = PK_GEMM_WGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{du, F, 1}, Operand{a2, D, 1}, p, side));
-      GPTK_TRY(mark(du_r[du_i], &dres_r[dres_i]));
-    }
     {  // da = du W_up
       GemmParams p = gp(M, D, F);
       p.out = da;
@@ -569,23 +468,9 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       GPTK_TRY(gemm(EPI_F32, Operand{du, F, 0}, Operand{wbf + o.w_up, D, 1}, p, st));
     }
     if (o.b_up >= 0) GPTK_TRY(bias_grad_bf16(du, M, F, pa, grads + o.b_up, st));
-    du_i ^= 1;
-    dres_i ^= 1;
-    GPTK_TRY(claim(dres_r[dres_i]));
-    dres_bf = dres_bf_s[dres_i];
-    GPTK_TRY(norm_backward(c, pl, da, x_mid, st2, params, o.ln2_g, o.ln2_b, grads, dres, 0, dres_bf, pa, pb, st));
+    GPTK_TRY(norm_backward(c, pl, da, x_mid, st2, params, o.ln2_g, o.ln2_b, grads, dres, 0, dres_bf_att, pa, pb, st));
 
     // ---- attention: x_mid = x_in + attn(N(x_in)) W_o^T + b_o
-    GPTK_TRY(fork());
-    {  // dW_o += dres^T o   (side stream)
-      GemmParams p = gp(D, D, M);
-      p.out = grads + o.w_o;
-      p.ldo = D;
-      p.accumulate = 1;
-      p.prof_kind = PK_GEMM_WGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{dres_bf, D, 1}, Operand{ob, D, 1}, p, side));
-      GPTK_TRY(mark(dres_r[dres_i], nullptr));
-    }
     if (hdp != hd) GPTK_CUDA(cudaMemsetAsync(do_pad, 0, (size_t)M * H * hdp * 2, st));
     {  // do = dres W_o  (written in the head-padded layout the attention kernels read)
       GemmParams p = gp(M, D, D);
@@ -594,26 +479,13 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       p.hd = hd;
       p.hdp = hdp;
       p.prof_kind = PK_GEMM_DGRAD;
-      GPTK_TRY(gemm(EPI_BF16, Operand{dres_bf, D, 0}, Operand{wbf + o.w_o, D, 1}, p, st));
+      GPTK_TRY(gemm(EPI_BF16, Operand{dres_bf_att, D, 0}, Operand{wbf + o.w_o, D, 1}, p, st));
     }
     if (o.b_o >= 0) GPTK_TRY(bias_grad_f32(dres, M, D, pa, grads + o.b_o, st));
     GPTK_TRY(launch_attn_delta(ob, do_pad, B, T, H, hd, hdp, delta, st));
     AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp};
-    __nv_bfloat16* dqkv_pad = dqkvp_s[dqkv_i];
-    __nv_bfloat16* dqkv = dqkv_s[dqkv_i];
-    GPTK_TRY(claim(dqkv_r[dqkv_i]));
     GPTK_TRY(launch_attn_bwd(qkv, do_pad, lse, delta, as, dqkv_pad, st));
     GPTK_TRY(launch_qk_bwd(dqkv_pad, qkv, rq, rk, cs, M, T, H, hd, hdp, c.pos == 1, c.qk_norm, dqkv, st));
-    GPTK_TRY(fork());
-    {  // dW_qkv += dqkv^T a1   (side stream)
-      GemmParams p = gp(3 * D, D, M);
-      p.out = grads + o.w_qkv;
-      p.ldo = D;
-      p.accumulate = 1;
-      p.prof_kind = PK_GEMM_WGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{dqkv, 3LL * D, 1}, Operand{a1, D, 1}, p, side));
-      GPTK_TRY(mark(dqkv_r[dqkv_i], nullptr));
-    }
     {  // da = dqkv W_qkv
       GemmParams p = gp(M, D, 3 * D);
       p.out = da;
@@ -622,17 +494,17 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       GPTK_TRY(gemm(EPI_F32, Operand{dqkv, 3LL * D, 0}, Operand{wbf + o.w_qkv, D, 1}, p, st));
     }
     if (o.b_qkv >= 0) GPTK_TRY(bias_grad_bf16(dqkv, M, 3 * D, pa, grads + o.b_qkv, st));
-    dqkv_i ^= 1;
-    dres_i ^= 1;
-    GPTK_TRY(claim(dres_r[dres_i]));
-    GPTK_TRY(norm_backward(c, pl, da, x_in, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0, dres_bf_s[dres_i], pa, pb,
+    {  // the layer's four weight gradients in one launch: W += dY^T X over all tokens
+      const GroupProblem probs[4] = {
+          {dres_bf_mlp, D, h, F, D, F, grads + o.w_down, F},
+          {du, F, a2, D, F, D, grads + o.w_up, D},
+          {dres_bf_att, D, ob, D, D, D, grads + o.w_o, D},
+          {dqkv, 3LL * D, a1, D, 3 * D, D, grads + o.w_qkv, D},
+      };
+      GPTK_TRY(run_gemm_group(4, probs, M, 1, 1, 256, PK_GEMM_WGRAD, st));
+    }
+    GPTK_TRY(norm_backward(c, pl, da, x_in, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0, dres_bf_mlp, pa, pb,
                            st));
-  }
-  // ---- join the side stream (the tied lm_head gradient shares wte's rows with the scatter)
-  if (side != st) {
-    cudaEvent_t e = next_event(sc);
-    GPTK_CUDA(cudaEventRecord(e, side));
-    GPTK_CUDA(cudaStreamWaitEvent(st, e, 0));
   }
   // ---- embeddings
   GPTK_TRY(launch_embed_bwd(idx_ws, dres, M, D, V, grads + Lo.wte, at<void>(ws, pl.embed), st));
