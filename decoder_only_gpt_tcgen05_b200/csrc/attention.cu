@@ -352,13 +352,14 @@ __global__ void __launch_bounds__(320, 1)
 
 template <int HD>
 struct DkvSmem {
+  static constexpr int QS = 3;              // Q / dO ring depth
   static constexpr int KV_TILE = HD * 256;  // 128 rows
   static constexpr int Q_TILE = HD * 128;   // 64 rows
   static constexpr int K = 0;
   static constexpr int V = K + KV_TILE;
-  static constexpr int Q0 = V + KV_TILE;       // [2]
-  static constexpr int DO0 = Q0 + 2 * Q_TILE;  // [2]
-  static constexpr int P0 = DO0 + 2 * Q_TILE;  // [2] 128 keys x 64 queries bf16 = 16 KB
+  static constexpr int Q0 = V + KV_TILE;        // [QS]
+  static constexpr int DO0 = Q0 + QS * Q_TILE;  // [QS]
+  static constexpr int P0 = DO0 + QS * Q_TILE;  // [2] 128 keys x 64 queries bf16 = 16 KB
   static constexpr int DS0 = P0 + 32768;       // [2]
   static constexpr int STATS = DS0 + 32768;    // [2][lse2 x 64, delta x 64] fp32
   static constexpr int BAR = STATS + 1024;
@@ -375,17 +376,18 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+  constexpr int QS = L::QS;
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;      // [2]
-  uint64_t* q_empty = bars + 3;     // [2]
-  uint64_t* s_full = bars + 5;      // [2]
-  uint64_t* s_free = bars + 7;      // [2]
-  uint64_t* pd_full = bars + 9;     // [2]
-  uint64_t* pd_empty = bars + 11;   // [2]
-  uint64_t* stats_bar = bars + 13;  // [2]
-  uint64_t* acc_full = bars + 15;
-  uint64_t* drain = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* q_full = bars + 1;           // [QS]
+  uint64_t* q_empty = bars + 1 + QS;     // [QS]
+  uint64_t* s_full = bars + 1 + 2 * QS;  // [2]
+  uint64_t* s_free = s_full + 2;         // [2]
+  uint64_t* pd_full = s_full + 4;        // [2]
+  uint64_t* pd_empty = s_full + 6;       // [2]
+  uint64_t* stats_bar = s_full + 8;      // [2]
+  uint64_t* acc_full = s_full + 10;
+  uint64_t* drain = s_full + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 12);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* stats = reinterpret_cast<float*>(sm + L::STATS);
 
@@ -401,9 +403,11 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < QS; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 8);
       mbar_init(&pd_full[i], 8);
@@ -442,8 +446,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     int issued = -1;
     for (int it = 0; it < n_it && ok; ++it) {
-      const int st = it & 1;
-      if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
+      const int st = it % QS;
+      if (!mbar_wait(&q_empty[st], ((it / QS) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
       const int qb = (i0 + it) * 64;
       mbar_expect_tx(&q_full[st], 2 * L::Q_TILE);
       for (int c = 0; c < NCH; ++c) {
@@ -455,8 +459,8 @@ __global__ void __launch_bounds__(320, 1)
     if (!ok) {
       volatile int never = 0;
       mbar_wait(kv_full, 0, ctl, &never, 41);
-      for (int it = (issued > 0 ? issued - 1 : 0); it <= issued && issued >= 0; ++it)
-        mbar_wait(&q_full[it & 1], (it >> 1) & 1, ctl, &never, 41);
+      for (int it = (issued >= QS ? issued - QS + 1 : 0); it <= issued && issued >= 0; ++it)
+        mbar_wait(&q_full[it % QS], (it / QS) & 1, ctl, &never, 41);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
@@ -467,12 +471,12 @@ __global__ void __launch_bounds__(320, 1)
     for (int it = 0; it <= n_it && ok; ++it) {
       if (it < n_it) {
         const int st = it & 1;
-        const uint32_t ph = (it >> 1) & 1;
-        if (!mbar_wait(&q_full[st], ph, ctl, abort_flag, 43)) { ok = false; break; }
-        if (!mbar_wait(&s_free[st], ph ^ 1u, ctl, abort_flag, 44)) { ok = false; break; }
+        const int qs = it % QS;
+        if (!mbar_wait(&q_full[qs], (it / QS) & 1, ctl, abort_flag, 43)) { ok = false; break; }
+        if (!mbar_wait(&s_free[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 44)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sQ = smem_u32(sm + L::Q0 + st * L::Q_TILE);
-        const uint32_t sD = smem_u32(sm + L::DO0 + st * L::Q_TILE);
+        const uint32_t sQ = smem_u32(sm + L::Q0 + qs * L::Q_TILE);
+        const uint32_t sD = smem_u32(sm + L::DO0 + qs * L::Q_TILE);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -489,8 +493,9 @@ __global__ void __launch_bounds__(320, 1)
         const int bb = jt & 1;
         if (!mbar_wait(&pd_full[bb], (jt >> 1) & 1, ctl, abort_flag, 45)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sQ = smem_u32(sm + L::Q0 + bb * L::Q_TILE);
-        const uint32_t sD = smem_u32(sm + L::DO0 + bb * L::Q_TILE);
+        const int qs = jt % QS;
+        const uint32_t sQ = smem_u32(sm + L::Q0 + qs * L::Q_TILE);
+        const uint32_t sD = smem_u32(sm + L::DO0 + qs * L::Q_TILE);
         const uint32_t sP = smem_u32(sm + L::P0 + bb * 16384);
         const uint32_t sDS = smem_u32(sm + L::DS0 + bb * 16384);
 #pragma unroll
@@ -501,7 +506,7 @@ __global__ void __launch_bounds__(320, 1)
                     (jt | kk) != 0);
         }
         umma_commit(&pd_empty[bb]);
-        umma_commit(&q_empty[bb]);
+        umma_commit(&q_empty[qs]);
         issued = true;
       }
     }
@@ -624,13 +629,14 @@ __global__ void __launch_bounds__(320, 1)
 
 template <int HD>
 struct DqSmem {
+  static constexpr int KS = 4;              // K / V ring depth
   static constexpr int Q_TILE = HD * 256;   // 128 rows
   static constexpr int KV_TILE = HD * 128;  // 64 rows
   static constexpr int Q = 0;
   static constexpr int DO = Q + Q_TILE;
-  static constexpr int K0 = DO + Q_TILE;       // [2]
-  static constexpr int V0 = K0 + 2 * KV_TILE;  // [2]
-  static constexpr int DS0 = V0 + 2 * KV_TILE; // [2] 128 queries x 64 keys bf16 = 16 KB
+  static constexpr int K0 = DO + Q_TILE;        // [KS]
+  static constexpr int V0 = K0 + KS * KV_TILE;  // [KS]
+  static constexpr int DS0 = V0 + KS * KV_TILE; // [2] 128 queries x 64 keys bf16 = 16 KB
   static constexpr int BAR = DS0 + 32768;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
@@ -645,16 +651,17 @@ __global__ void __launch_bounds__(320, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+  constexpr int KS = L::KS;
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* ds_full = bars + 9;   // [2]
-  uint64_t* ds_empty = bars + 11; // [2]
-  uint64_t* acc_full = bars + 13;
-  uint64_t* drain = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* kv_full = bars + 1;          // [KS]
+  uint64_t* kv_empty = bars + 1 + KS;    // [KS]
+  uint64_t* s_full = bars + 1 + 2 * KS;  // [2]
+  uint64_t* s_free = s_full + 2;         // [2]
+  uint64_t* ds_full = s_full + 4;        // [2]
+  uint64_t* ds_empty = s_full + 6;       // [2]
+  uint64_t* acc_full = s_full + 8;
+  uint64_t* drain = s_full + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -669,9 +676,11 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 8);
       mbar_init(&ds_full[i], 8);
@@ -708,8 +717,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     int issued = -1;
     for (int j = 0; j < n_kv && ok; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
+      const int st = j % KS;
+      if (!mbar_wait(&kv_empty[st], ((j / KS) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
       mbar_expect_tx(&kv_full[st], 2 * L::KV_TILE);
       for (int c = 0; c < NCH; ++c) {
         tma_load_3d(sm + L::K0 + st * L::KV_TILE + c * 8192, &tm_kv64, &kv_full[st], colk + 64 * c, j * 64, b);
@@ -720,8 +729,8 @@ __global__ void __launch_bounds__(320, 1)
     if (!ok) {
       volatile int never = 0;
       mbar_wait(q_full, 0, ctl, &never, 61);
-      for (int j = (issued > 0 ? issued - 1 : 0); j <= issued && issued >= 0; ++j)
-        mbar_wait(&kv_full[j & 1], (j >> 1) & 1, ctl, &never, 61);
+      for (int j = (issued >= KS ? issued - KS + 1 : 0); j <= issued && issued >= 0; ++j)
+        mbar_wait(&kv_full[j % KS], (j / KS) & 1, ctl, &never, 61);
     }
   } else if (warp == 1 && lane == 0) {
     constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
@@ -732,12 +741,12 @@ __global__ void __launch_bounds__(320, 1)
     for (int j = 0; j <= n_kv && ok; ++j) {
       if (j < n_kv) {
         const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&kv_full[st], ph, ctl, abort_flag, 63)) { ok = false; break; }
-        if (!mbar_wait(&s_free[st], ph ^ 1u, ctl, abort_flag, 64)) { ok = false; break; }
+        const int ks = j % KS;
+        if (!mbar_wait(&kv_full[ks], (j / KS) & 1, ctl, abort_flag, 63)) { ok = false; break; }
+        if (!mbar_wait(&s_free[st], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 64)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::K0 + st * L::KV_TILE);
-        const uint32_t sV = smem_u32(sm + L::V0 + st * L::KV_TILE);
+        const uint32_t sK = smem_u32(sm + L::K0 + ks * L::KV_TILE);
+        const uint32_t sV = smem_u32(sm + L::V0 + ks * L::KV_TILE);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -754,14 +763,15 @@ __global__ void __launch_bounds__(320, 1)
         const int bb = jj & 1;
         if (!mbar_wait(&ds_full[bb], (jj >> 1) & 1, ctl, abort_flag, 65)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::K0 + bb * L::KV_TILE);
+        const int ks = jj % KS;
+        const uint32_t sK = smem_u32(sm + L::K0 + ks * L::KV_TILE);
         const uint32_t sDS = smem_u32(sm + L::DS0 + bb * 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_bf16(tdQ, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sK + kk * 2048, 8192, 1024), idesc_acc,
                     (jj | kk) != 0);
         umma_commit(&ds_empty[bb]);
-        umma_commit(&kv_empty[bb]);
+        umma_commit(&kv_empty[ks]);
         issued = true;
       }
     }
@@ -893,6 +903,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
   const double causal = (double)s.B * s.H * ((double)s.T * (s.T + 1) / 2);
   {
     using L = DkvSmem<HD>;
+    static_assert(L::BYTES <= 232448, "dK/dV shared memory above the per-block limit");
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
     Prof prof(PK_ATTN_BWD_DKV, 8.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 6, st);
@@ -901,6 +912,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
   }
   {
     using L = DqSmem<HD>;
+    static_assert(L::BYTES <= 232448, "dQ shared memory above the per-block limit");
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
     Prof prof(PK_ATTN_BWD_DQ, 6.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 5, st);
