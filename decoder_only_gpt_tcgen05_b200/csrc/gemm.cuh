@@ -108,7 +108,7 @@ __device__ __forceinline__ float act_fwd(float u, int act) {
 
 __device__ __forceinline__ float act_grad(float u, int act) {
   if (act == 1) return 2.f * fmaxf(u, 0.f);
-  if (act == 2) return 2.f * sqrtf(fmaxf(u, 0.f));  // ReLU^2 given h = relu(u)^2: 2 relu(u) = 2 sqrt(h)
+  if (act == 2) return 2.f * sqrt_approx(fmaxf(u, 0.f));  // ReLU^2 given h = relu(u)^2: 2 relu(u) = 2 sqrt(h)
   // d/du of 0.5 u (1 + erf(u/sqrt2)) = 0.5 (1 + erf(u/sqrt2)) + u * exp(-u^2/2) / sqrt(2 pi)
   return 0.5f * (1.f + erff(u * 0.70710678118654752f)) + u * expf(-0.5f * u * u) * 0.3989422804014327f;
 }
@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
             } else if (p.act == 2) {  // EPI_ACTBWD, ReLU^2 from h: 2 relu(u) = 2 sqrt(h)
               unstage_bf16(buf, lane, in);
 #pragma unroll
-              for (int j = 0; j < CW; ++j) v[j] *= 2.f * sqrtf(fmaxf(in[j], 0.f));
+              for (int j = 0; j < CW; ++j) v[j] *= 2.f * sqrt_approx(fmaxf(in[j], 0.f));
             } else if (p.act == 1) {  // ReLU^2 from u
               unstage_bf16(buf, lane, in);
 #pragma unroll

@@ -268,6 +268,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Hardware square root (sqrt.approx: +0 maps to +0; its error of a few ulp is far below bf16
+// rounding).  The IEEE sqrtf leaves its fast path for zero inputs, which ReLU^2 makes common.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
