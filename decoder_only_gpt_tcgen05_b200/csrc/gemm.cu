@@ -109,18 +109,38 @@ int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, u
 
 // ------------------------------------------------------------ GEMM launcher
 
-template <int BN, int EPI, bool LONGK>
+template <int BN, int EPI, bool LONGK, bool PAIR>
 static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
-  using C = GemmCfg<BN, LONGK>;
+  using C = GemmCfg<BN, LONGK, PAIR>;
+  auto kern = gemm_kernel<BN, EPI, LONGK, PAIR>;
   static bool attr_set[64] = {false};
+  static int max_pairs[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set[dev & 63]) {
-    GPTK_CUDA(cudaFuncSetAttribute(gemm_kernel<BN, EPI, LONGK>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    GPTK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM));
+    if (PAIR) {
+      // how many CTA pairs fit at once (an SM whose GPC has no free partner SM stays out)
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+      cfg.blockDim = dim3(C::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = C::SMEM;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      GPTK_CUDA(cudaOccupancyMaxActiveClusters(&n, kern, &cfg));
+      if (n < 1) return set_error(ST_UNSUPPORTED, "GEMM: no CTA pair fits on this device");
+      max_pairs[dev & 63] = n;
+    }
     attr_set[dev & 63] = true;
   }
   const int tiles = p.tile_start[p.n_prob];
-  int grid = num_sms();
+  int grid = PAIR ? max_pairs[dev & 63] : num_sms();
   if (grid > tiles) grid = tiles;
   double flops = 0, bytes = 0;
   for (int q = 0; q < p.n_prob; ++q) {
@@ -134,32 +154,66 @@ static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t
     bytes += (M * K + N * K) * 2 + out_bytes;
   }
   Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, flops, bytes, st);
-  gemm_kernel<BN, EPI, LONGK><<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
+  if (PAIR) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * grid, 1, 1);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    GPTK_CUDA(cudaLaunchKernelEx(&cfg, kern, maps, p));
+  } else {
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
+  }
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 static int dispatch_epi(int epi, const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
   // reductions over all tokens (weight gradients) and over the vocabulary take the deep ring
-  if (epi == EPI_F32 && p.K >= 8192) return launch_gemm_t<BN, EPI_F32, true>(maps, p, st);
+  if (epi == EPI_F32 && p.K >= 8192) return launch_gemm_t<BN, EPI_F32, true, PAIR>(maps, p, st);
   switch (epi) {
-    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false>(maps, p, st);
-    case EPI_F32: return launch_gemm_t<BN, EPI_F32, false>(maps, p, st);
-    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false>(maps, p, st);
-    case EPI_UP: return launch_gemm_t<BN, EPI_UP, false>(maps, p, st);
-    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD, false>(maps, p, st);
-    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD, false>(maps, p, st);
-    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD, false>(maps, p, st);
+    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false, PAIR>(maps, p, st);
+    case EPI_F32: return launch_gemm_t<BN, EPI_F32, false, PAIR>(maps, p, st);
+    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false, PAIR>(maps, p, st);
+    case EPI_UP: return launch_gemm_t<BN, EPI_UP, false, PAIR>(maps, p, st);
+    case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD, false, PAIR>(maps, p, st);
+    case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD, false, PAIR>(maps, p, st);
+    case EPI_CE_BWD: return launch_gemm_t<BN, EPI_CE_BWD, false, PAIR>(maps, p, st);
   }
   return set_error(ST_INVALID_ARG, "unknown GEMM epilogue");
+}
+
+static int dispatch(int epi, int bn, bool pair, const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
+  if (pair) return dispatch_epi<256, true>(epi, maps, p, st);
+  return bn == 256 ? dispatch_epi<256, false>(epi, maps, p, st) : dispatch_epi<128, false>(epi, maps, p, st);
+}
+
+// CTA pairs (256-row tiles) for N-256 tiles when the 256-row tiles still give every pair of SMs
+// at least one tile; GPT_GEMM_PAIR=0 / 1 forces the choice (tuning and comparison).
+static bool use_pair(int bn, long long tiles256) {
+  static const int forced = []() {
+    const char* e = std::getenv("GPT_GEMM_PAIR");
+    return e ? std::atoi(e) : -1;
+  }();
+  if (bn != 256 || forced == 0) return false;
+  if (forced == 1) return true;
+  return tiles256 >= num_sms() / 2;
 }
 
 static bool aligned16(const void* ptr, long long ld, int esize) {
   return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0 && ((ld * esize) & 15) == 0;
 }
 
-static int operand_maps(const Operand& A, const Operand& B, int M, int N, int K, int bn, CUtensorMap* ta,
+// b_rows: B rows one CTA stages per K step (the tile's N, or half of it for CTA pairs)
+static int operand_maps(const Operand& A, const Operand& B, int M, int N, int K, int b_rows, CUtensorMap* ta,
                         CUtensorMap* tb) {
   if (!A.mn_major) {
     GPTK_TRY(make_tmap_2d(ta, A.ptr, K, M, A.ld, 64, 128));
@@ -167,16 +221,16 @@ static int operand_maps(const Operand& A, const Operand& B, int M, int N, int K,
     GPTK_TRY(make_tmap_2d(ta, A.ptr, M, K, A.ld, 64, 64));
   }
   if (!B.mn_major) {
-    GPTK_TRY(make_tmap_2d(tb, B.ptr, K, N, B.ld, 64, bn));
+    GPTK_TRY(make_tmap_2d(tb, B.ptr, K, N, B.ld, 64, b_rows));
   } else {
     GPTK_TRY(make_tmap_2d(tb, B.ptr, N, K, B.ld, 64, 64));
   }
   return ST_OK;
 }
 
-// band height: a few m-tiles whose A rows (128 x K bf16 each) stay within about 48 MB of L2
-static int band_height(int tiles_m, int K) {
-  const long long a_band_row = 128LL * K * 2;
+// band height: a few m-tiles whose A rows (tile_m x K bf16 each) stay within about 48 MB of L2
+static int band_height(int tiles_m, int K, int tile_m) {
+  const long long a_band_row = (long long)tile_m * K * 2;
   int gm = 8;  // measured best among 8, 16, 32 and the plain order on B200 (d20 shapes)
   const int gm_l2 = (int)((48LL << 20) / (a_band_row > 0 ? a_band_row : 1));
   if (gm > gm_l2) gm = gm_l2;
@@ -199,7 +253,9 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return set_error(ST_INVALID_ARG, "GEMM with an empty dimension");
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
-  GPTK_TRY(operand_maps(A, B, p.M, p.N, p.K, bn, &maps.a[0], &maps.b[0]));
+  const bool pair = use_pair(bn, (long long)((p.M + 255) / 256) * ((p.N + 255) / 256));
+  const int tile_m = pair ? 256 : 128;
+  GPTK_TRY(operand_maps(A, B, p.M, p.N, p.K, pair ? bn / 2 : bn, &maps.a[0], &maps.b[0]));
   // output / input tensor maps of the TMA epilogue, where the layout allows one
   p.tma_out = 0;
   const bool f32out = (epi == EPI_F32 || epi == EPI_RESID);
@@ -220,9 +276,9 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   }
   p.a_mn = A.mn_major;
   p.b_mn = B.mn_major;
-  p.tiles_m = (p.M + 127) / 128;
+  p.tiles_m = (p.M + tile_m - 1) / tile_m;
   p.tiles_n = (p.N + bn - 1) / bn;
-  p.group_m = band_height(p.tiles_m, p.K);
+  p.group_m = band_height(p.tiles_m, p.K, tile_m);
   p.n_prob = 1;
   p.tile_start[0] = 0;
   p.tile_start[1] = p.tiles_m * p.tiles_n;
@@ -233,7 +289,7 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   p.pgroup_m[0] = p.group_m;
   p.ctl = device_ctl();
   if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
-  return bn == 256 ? dispatch_epi<256>(epi, maps, p, st) : dispatch_epi<128>(epi, maps, p, st);
+  return dispatch(epi, bn, pair, maps, p, st);
 }
 
 int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
@@ -252,19 +308,23 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
   p.tma_out = 1;
   p.prof_kind = prof_kind;
   p.n_prob = n;
+  long long tiles256 = 0;
+  for (int q = 0; q < n; ++q) tiles256 += (long long)((probs[q].M + 255) / 256) * ((probs[q].N + 255) / 256);
+  const bool pair = use_pair(bn, tiles256);
+  const int tile_m = pair ? 256 : 128;
   int start = 0;
   for (int q = 0; q < n; ++q) {
     const GroupProblem& g = probs[q];
     if (g.M <= 0 || g.N <= 0 || !aligned16(g.out, g.ldo, 4))
       return set_error(ST_INVALID_ARG, "grouped GEMM: bad problem");
-    GPTK_TRY(operand_maps(Operand{g.a, g.lda, a_mn}, Operand{g.b, g.ldb, b_mn}, g.M, g.N, K, bn, &maps.a[q],
+    GPTK_TRY(operand_maps(Operand{g.a, g.lda, a_mn}, Operand{g.b, g.ldb, b_mn}, g.M, g.N, K, pair ? bn / 2 : bn, &maps.a[q],
                           &maps.b[q]));
     GPTK_TRY(make_tmap_2d(&maps.c[q], g.out, g.N, g.M, g.ldo, 32, 32, 4));
     p.pM[q] = g.M;
     p.pN[q] = g.N;
-    p.ptiles_m[q] = (g.M + 127) / 128;
+    p.ptiles_m[q] = (g.M + tile_m - 1) / tile_m;
     p.ptiles_n[q] = (g.N + bn - 1) / bn;
-    p.pgroup_m[q] = band_height(p.ptiles_m[q], K);
+    p.pgroup_m[q] = band_height(p.ptiles_m[q], K, tile_m);
     p.tile_start[q] = start;
     start += p.ptiles_m[q] * p.ptiles_n[q];
   }
@@ -276,7 +336,7 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
   p.group_m = p.pgroup_m[0];
   p.ctl = device_ctl();
   if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
-  return bn == 256 ? dispatch_epi<256>(EPI_F32, maps, p, st) : dispatch_epi<128>(EPI_F32, maps, p, st);
+  return dispatch(EPI_F32, bn, pair, maps, p, st);
 }
 
 }  // namespace gptk

@@ -10,6 +10,15 @@
 // The accumulator is double buffered in tensor memory (2 x BN columns) so the epilogue of one
 // tile overlaps the main loop of the next.
 //
+// PAIR variant (cluster of two CTAs on two SMs): the pair walks 256 x BN tiles with one
+// tcgen05.mma.cta_group::2 (M = 256) per K step, issued by the even CTA.  Each CTA stages its
+// own 128 A rows and its own BN/2 B rows, so a K step moves half the B bytes per SM of the
+// single-CTA form and the same shared memory holds a deeper ring.  Both CTAs' TMA loads
+// complete on the even CTA's "full" barrier; its MMA commits release both CTAs' stages and
+// accumulators; both CTAs' epilogues (each on its own 128 accumulator rows) arrive on the even
+// CTA's "tempty" barrier.  Every cross-CTA arrival is waited for before the final cluster
+// barrier, so neither CTA leaves while its peer may still touch its shared memory.
+//
 // Epilogue data path: each epilogue warp owns 32 rows x BN/2 columns and two 4 KB staging buffers.  A chunk of
 // 32 fp32 or 64 bf16 columns (128-byte rows) goes registers -> swizzled shared memory -> one TMA
 // tile store (or TMA reduce-add for accumulated gradients), so global writes are whole lines.
@@ -81,17 +90,20 @@ struct GemmMaps {
 
 // LONGK: the variant for very long reductions (weight gradients over all tokens), where the
 // epilogue is rare and a deeper TMA ring matters more than epilogue parallelism.
-template <int BN, bool LONGK = false>
+template <int BN, bool LONGK = false, bool PAIR = false>
 struct GemmCfg {
-  static constexpr int BM = 128;
+  static constexpr int BM = 128;                    // accumulator rows per CTA
+  static constexpr int TILE_M = PAIR ? 256 : 128;   // output rows per tile
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN; // B rows staged per CTA
   static constexpr int BK = 64;
-  static constexpr int STAGES = LONGK ? ((BN == 256) ? 4 : 6) : ((BN == 256) ? 3 : 5);
+  static constexpr int STAGES = PAIR ? (LONGK ? 6 : 5) : (LONGK ? ((BN == 256) ? 4 : 6) : ((BN == 256) ? 3 : 5));
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int EPI_WARPS = LONGK ? 4 : 8;             // one or two per TMEM lane quadrant
   static constexpr int STAGING_BYTES = EPI_WARPS * 2 * 4096;  // 2 buffers of 32 rows x 128 B per warp
-  static constexpr int BAR_BYTES = 256;
+  static constexpr int BAR_BYTES = 512;
+  static_assert((2 * STAGES + 5 + 2 * EPI_WARPS) * 8 + 8 <= BAR_BYTES, "barrier block too small");
   static constexpr int SMEM = STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 1024;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
 };
@@ -259,10 +271,10 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int tile) {
 
 // --------------------------------------------------------------- the kernel
 
-template <int BN, int EPI, bool LONGK>
-__global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
+template <int BN, int EPI, bool LONGK, bool PAIR>
+__global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
     gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
-  using C = GemmCfg<BN, LONGK>;
+  using C = GemmCfg<BN, LONGK, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -280,6 +292,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // CTA pairs: rank within the pair, and the pair's place in the persistent tile walk
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile0 = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+  const int tile_step = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -288,7 +304,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::EPI_WARPS);
+      mbar_init(&tempty[b], C::EPI_WARPS * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
     for (int i = 0; i < 2 * C::EPI_WARPS; ++i) mbar_init(&inbar[i], 1);
@@ -299,7 +315,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
       prefetch_tmap(&maps.b[q]);
     }
   }
-  if (warp == 1) {
+  if (PAIR) {
+    // the peer's barriers must be initialised before anything is signalled across the pair
+    cluster_sync();
+    if (warp == 1) {
+      tmem_alloc_pair(tmem_slot, 2 * BN);
+      tmem_relinquish_pair();
+    }
+  } else if (warp == 1) {
     tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
@@ -317,32 +340,54 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     uint32_t phase = 0;
     uint32_t pending = 0;  // stages with a load in flight that the MMA has not yet released
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = tile0; tile < num_tiles && ok; tile += tile_step) {
       const TileInfo ti = tile_info(p, tile);
       const int tm = ti.tm, tn = ti.tn;
       const CUtensorMap* tmA = &maps.a[ti.prob];
       const CUtensorMap* tmB = &maps.b[ti.prob];
+      const int arow = tm * C::TILE_M + (int)rank * C::BM;     // this CTA's A rows
+      const int brow = tn * BN + (int)rank * C::B_ROWS;        // this CTA's B rows
       for (int kb = 0; kb < num_k; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctl, abort_flag, 1)) {
           ok = false;
           break;
         }
         pending &= ~(1u << stage);
-        mbar_expect_tx(&full[stage], C::STAGE_BYTES);
         uint8_t* a = sA + stage * C::A_BYTES;
         uint8_t* b = sB + stage * C::B_BYTES;
-        if (!p.a_mn) {
-          tma_load_2d(a, tmA, &full[stage], kb * C::BK, tm * C::BM);
-        } else {
+        if (PAIR) {
+          // both CTAs' bytes complete on the even CTA's barrier, which expects all of them
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          if (!p.a_mn) {
+            tma_load_2d_pair(a, tmA, fb, kb * C::BK, arow);
+          } else {
 #pragma unroll
-          for (int c = 0; c < C::BM / 64; ++c)
-            tma_load_2d(a + c * 8192, tmA, &full[stage], tm * C::BM + c * 64, kb * C::BK);
-        }
-        if (!p.b_mn) {
-          tma_load_2d(b, tmB, &full[stage], kb * C::BK, tn * BN);
-        } else {
+            for (int c = 0; c < C::BM / 64; ++c) tma_load_2d_pair(a + c * 8192, tmA, fb, arow + c * 64, kb * C::BK);
+          }
+          if (!p.b_mn) {
+            tma_load_2d_pair(b, tmB, fb, kb * C::BK, brow);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tma_load_2d(b + c * 8192, tmB, &full[stage], tn * BN + c * 64, kb * C::BK);
+            for (int c = 0; c < C::B_ROWS / 64; ++c)
+              tma_load_2d_pair(b + c * 8192, tmB, fb, brow + c * 64, kb * C::BK);
+          }
+        } else {
+          mbar_expect_tx(&full[stage], C::STAGE_BYTES);
+          if (!p.a_mn) {
+            tma_load_2d(a, tmA, &full[stage], kb * C::BK, arow);
+          } else {
+#pragma unroll
+            for (int c = 0; c < C::BM / 64; ++c)
+              tma_load_2d(a + c * 8192, tmA, &full[stage], arow + c * 64, kb * C::BK);
+          }
+          if (!p.b_mn) {
+            tma_load_2d(b, tmB, &full[stage], kb * C::BK, brow);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(b + c * 8192, tmB, &full[stage], brow + c * 64, kb * C::BK);
+          }
         }
         pending |= 1u << stage;
         if (++stage == C::STAGES) {
@@ -351,7 +396,18 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
         }
       }
     }
-    if (!ok) {
+    if (PAIR && ok) {
+      // wait until the MMAs have released every stage, i.e. until the even CTA's last commits
+      // to this CTA's "empty" barriers have landed
+      for (int i = 0; i < C::STAGES && ok; ++i) {
+        ok = mbar_wait(&empty[stage], phase ^ 1u, p.ctl, abort_flag, 8);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && (!PAIR || rank == 0)) {
       // drain the copies still in flight before the CTA goes away (bounded as well)
       volatile int never = 0;
       for (int s = 0; s < C::STAGES; ++s) {
@@ -361,9 +417,9 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
         mbar_wait(&full[s], ph, p.ctl, &never, 2);
       }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------ MMA issuer
-    constexpr uint32_t IDESC_KK = idesc_bf16(128, BN, 0, 0);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------ MMA issuer (the even CTA of a pair)
+    constexpr uint32_t IDESC_KK = idesc_bf16(C::TILE_M, BN, 0, 0);
     const uint32_t idesc = IDESC_KK | (static_cast<uint32_t>(p.a_mn) << 15) | (static_cast<uint32_t>(p.b_mn) << 16);
     int stage = 0;
     uint32_t phase = 0;
@@ -371,7 +427,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     bool issued = false;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int tile = tile0; tile < num_tiles && ok; tile += tile_step) {
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.ctl, abort_flag, 3)) {
         ok = false;
         break;
@@ -390,9 +446,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
         for (int kk = 0; kk < C::BK / 16; ++kk) {
           const uint64_t ad = p.a_mn ? sdesc_sw128(a0 + kk * 2048, 8192, 1024) : sdesc_sw128(a0 + kk * 32, 16, 1024);
           const uint64_t bd = p.b_mn ? sdesc_sw128(b0 + kk * 2048, 8192, 1024) : sdesc_sw128(b0 + kk * 32, 16, 1024);
-          umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
         }
-        umma_commit(&empty[stage]);
+        if (PAIR) {
+          // the stage is free in both CTAs once these MMAs have read it
+          const uint32_t eb = smem_u32(&empty[stage]);
+          umma_commit_pair(eb);
+          umma_commit_pair(mapa_shared(eb, 1));
+        } else {
+          umma_commit(&empty[stage]);
+        }
         issued = true;
         if (++stage == C::STAGES) {
           stage = 0;
@@ -400,16 +464,34 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
         }
       }
       if (!ok) break;
-      umma_commit(&tfull[acc]);
+      if (PAIR) {
+        const uint32_t tb = smem_u32(&tfull[acc]);
+        umma_commit_pair(tb);
+        umma_commit_pair(mapa_shared(tb, 1));
+      } else {
+        umma_commit(&tfull[acc]);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
       }
     }
+    if (PAIR && ok) {
+      // both CTAs' epilogues have finished with both accumulators: every arrival from the
+      // peer on this CTA's "tempty" barriers has landed
+      for (int i = 0; i < 2 && ok; ++i) {
+        ok = mbar_wait(&tempty[acc], acc_phase ^ 1u, p.ctl, abort_flag, 9);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+    }
     if (!ok && issued) {
       // let the MMAs already issued finish before tensor memory is released
       volatile int never = 0;
-      umma_commit(drain);
+      if (PAIR) umma_commit_pair(smem_u32(drain));
+      else umma_commit(drain);
       mbar_wait(drain, 0, p.ctl, &never, 6);
     }
   } else if (warp >= 2) {
@@ -417,7 +499,6 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     const int quad = warp & 3;
     const int ew = warp - 2;
     const int chalf = ew >> 2;  // which part of the tile's columns this warp writes
-    const int r_in_tile = quad * 32 + lane;
     uint8_t* stg_ptr = staging + ew * 8192;
     const uint32_t stg = smem_u32(stg_ptr);
     uint64_t* ibar = inbar + 2 * ew;
@@ -429,15 +510,15 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
     constexpr int CW = F32OUT ? 32 : 64;
     constexpr bool HAS_IN = (EPI == EPI_RESID || EPI == EPI_ACTBWD);
     constexpr int HALF = BN * 4 / C::EPI_WARPS;  // columns per epilogue warp
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = tile0; tile < num_tiles; tile += tile_step) {
       const TileInfo ti = tile_info(p, tile);
       const int tm = ti.tm, tn = ti.tn;
       const int pN = ti.N;
       const CUtensorMap* tmC = &maps.c[ti.prob];
       const CUtensorMap* tmC2 = &maps.c2;
       const CUtensorMap* tmR = &maps.r;
-      const int row = tm * 128 + r_in_tile;
-      const int row0 = tm * 128 + quad * 32;
+      const int row0 = tm * C::TILE_M + (int)rank * C::BM + quad * 32;
+      const int row = row0 + lane;
       const bool row_ok = row < ti.M;
       const int c_begin = chalf * HALF;
       const int n0 = tn * BN;
@@ -591,7 +672,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -602,7 +686,14 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK>::THREADS, 1)
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (PAIR) {
+    // neither CTA leaves while the other may still address its shared or tensor memory
+    cluster_sync();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc_pair(tmem_base, 2 * BN);
+    }
+  } else if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * BN);
   }
