@@ -345,49 +345,53 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ====================================================================== backward: dK, dV
-// One CTA per 128-key tile, stepping over 64-query tiles: S^T = K Q^T and dP^T = V dO^T into
-// double-buffered TMEM, P^T and dS^T = P^T (dP^T - delta) into double-buffered shared memory,
-// dV += P^T dO and dK += dS^T Q accumulating in TMEM.  The per-query statistics (lse, delta)
-// of a step are staged once in shared memory by the four softmax warps.
+// One CTA per 128-key tile, stepping over 128-query blocks from the diagonal block on.
+//   S^T = K Q^T and dP^T = V dO^T go into TMEM (M = 128 keys, N = 128 queries, full-rate MMAs).
+//   Sixteen elementwise warps turn them into P^T = exp2(S^T scale - lse) and
+//   dS^T = P^T (dP^T - delta) and write both back as bf16 over the fp32 columns each warp has
+//   just read (element (key, query) at lane key, column query/2 of its 16-query group), where
+//   they are the tensor-memory A operand of dV += P^T dO and dK += dS^T Q.
+//   The block's queries go in two halves: the dV/dK products of the first half run while the
+//   elementwise warps work on the second.
+// TMEM: S^T/P^T [0,128), dP^T/dS^T [128,256), dV [256, 256+HD), dK [384, 384+HD).
+// The per-query statistics (lse in log2 units, delta) of each block are staged in shared
+// memory by the elementwise warps, loaded from global memory one block ahead.
+
+constexpr int kBwdThreads = 576;  // TMA warp, MMA warp, 16 elementwise warps
+constexpr int kBwdEw = 16;        // elementwise warps: 4 per TMEM lane quadrant
 
 template <int HD>
 struct DkvSmem {
-  static constexpr int QS = 3;              // Q / dO ring depth
-  static constexpr int KV_TILE = HD * 256;  // 128 rows
-  static constexpr int Q_TILE = HD * 128;   // 64 rows
+  static constexpr int TILE = HD * 256;            // 128 rows x HD bf16 (64-column chunks of 16 KB)
   static constexpr int K = 0;
-  static constexpr int V = K + KV_TILE;
-  static constexpr int Q0 = V + KV_TILE;        // [QS]
-  static constexpr int DO0 = Q0 + QS * Q_TILE;  // [QS]
-  static constexpr int P0 = DO0 + QS * Q_TILE;  // [2] 128 keys x 64 queries bf16 = 16 KB
-  static constexpr int DS0 = P0 + 32768;       // [2]
-  static constexpr int STATS = DS0 + 32768;    // [2][lse2 x 64, delta x 64] fp32
-  static constexpr int BAR = STATS + 1024;
+  static constexpr int V = K + TILE;
+  static constexpr int Q0 = V + TILE;              // [2] query-block ring
+  static constexpr int DO0 = Q0 + 2 * TILE;        // [2]
+  static constexpr int STATS = DO0 + 2 * TILE;     // [2][lse2 x 128, delta x 128] fp32
+  static constexpr int BAR = STATS + 2048;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
 
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
-    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q64,
-                        const __grid_constant__ CUtensorMap tm_do64, const AttnShape s, const float* __restrict__ lse,
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_kv128, const __grid_constant__ CUtensorMap tm_q128,
+                        const __grid_constant__ CUtensorMap tm_do128, const AttnShape s, const float* __restrict__ lse,
                         const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, float scale_log2,
                         float scale, DevCtl ctl) {
   using L = DkvSmem<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
-  constexpr int QS = L::QS;
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;           // [QS]
-  uint64_t* q_empty = bars + 1 + QS;     // [QS]
-  uint64_t* s_full = bars + 1 + 2 * QS;  // [2]
-  uint64_t* s_free = s_full + 2;         // [2]
-  uint64_t* pd_full = s_full + 4;        // [2]
-  uint64_t* pd_empty = s_full + 6;       // [2]
-  uint64_t* stats_bar = s_full + 8;      // [2]
-  uint64_t* acc_full = s_full + 10;
-  uint64_t* drain = s_full + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 12);
+  uint64_t* q_full = bars + 1;     // [2]
+  uint64_t* q_empty = bars + 3;    // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* h_full = bars + 6;     // [2] one per half of the elementwise pass
+  uint64_t* d_done = bars + 8;
+  uint64_t* stats_bar = bars + 9;  // [2]
+  uint64_t* acc_full = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* stats = reinterpret_cast<float*>(sm + L::STATS);
 
@@ -396,24 +400,19 @@ __global__ void __launch_bounds__(320, 1)
   const int bh = blockIdx.y;
   const int b = bh / s.H, h = bh % s.H;
   const int k0 = kt * 128;
-  const int n_q64 = (s.T + 63) / 64;
-  const int i0 = 2 * kt;
-  const int n_it = n_q64 - i0;
+  const int n_it = (s.T + 127) / 128 - kt;  // query blocks from the diagonal one on
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < QS; ++i) {
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
+      mbar_init(&h_full[i], kBwdEw);
+      mbar_init(&stats_bar[i], kBwdEw);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 8);
-      mbar_init(&pd_full[i], 8);
-      mbar_init(&pd_empty[i], 1);
-      mbar_init(&stats_bar[i], 8);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(d_done, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -427,8 +426,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tS = tbase;         // [2] x 64
-  const uint32_t tdP = tbase + 128;  // [2] x 64
+  const uint32_t tS = tbase;
+  const uint32_t tdP = tbase + 128;
   const uint32_t tdV = tbase + 256;
   const uint32_t tdK = tbase + 384;
 
@@ -438,77 +437,79 @@ __global__ void __launch_bounds__(320, 1)
   const int cold = h * s.hdp;
 
   if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer
     bool ok = true;
-    mbar_expect_tx(kv_full, 2 * L::KV_TILE);
+    mbar_expect_tx(kv_full, 2 * L::TILE);
     for (int c = 0; c < NCH; ++c) {
       tma_load_3d(sm + L::K + c * 16384, &tm_kv128, kv_full, colk + 64 * c, k0, b);
       tma_load_3d(sm + L::V + c * 16384, &tm_kv128, kv_full, colv + 64 * c, k0, b);
     }
     int issued = -1;
     for (int it = 0; it < n_it && ok; ++it) {
-      const int st = it % QS;
-      if (!mbar_wait(&q_empty[st], ((it / QS) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
-      const int qb = (i0 + it) * 64;
-      mbar_expect_tx(&q_full[st], 2 * L::Q_TILE);
+      const int st = it & 1;
+      if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
+      const int qb = (kt + it) * 128;
+      mbar_expect_tx(&q_full[st], 2 * L::TILE);
       for (int c = 0; c < NCH; ++c) {
-        tma_load_3d(sm + L::Q0 + st * L::Q_TILE + c * 8192, &tm_q64, &q_full[st], colq + 64 * c, qb, b);
-        tma_load_3d(sm + L::DO0 + st * L::Q_TILE + c * 8192, &tm_do64, &q_full[st], cold + 64 * c, qb, b);
+        tma_load_3d(sm + L::Q0 + st * L::TILE + c * 16384, &tm_q128, &q_full[st], colq + 64 * c, qb, b);
+        tma_load_3d(sm + L::DO0 + st * L::TILE + c * 16384, &tm_do128, &q_full[st], cold + 64 * c, qb, b);
       }
       issued = it;
     }
     if (!ok) {
+      // wait (bounded) for the copies still in flight before the CTA goes away
       volatile int never = 0;
       mbar_wait(kv_full, 0, ctl, &never, 41);
-      for (int it = (issued >= QS ? issued - QS + 1 : 0); it <= issued && issued >= 0; ++it)
-        mbar_wait(&q_full[it % QS], (it / QS) & 1, ctl, &never, 41);
+      for (int it = (issued >= 2 ? issued - 1 : 0); it <= issued && issued >= 0; ++it)
+        mbar_wait(&q_full[it & 1], (it >> 1) & 1, ctl, &never, 41);
     }
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
-    constexpr uint32_t idesc_acc = idesc_bf16(128, HD, 0, 1);
+    // ------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t idesc_d = idesc_bf16(128, HD, 0, 1);
     bool ok = mbar_wait(kv_full, 0, ctl, abort_flag, 42);
     bool issued = false;
-    const uint32_t sK = smem_u32(sm + L::K), sV = smem_u32(sm + L::V);
-    for (int it = 0; it <= n_it && ok; ++it) {
-      if (it < n_it) {
-        const int st = it & 1;
-        const int qs = it % QS;
-        if (!mbar_wait(&q_full[qs], (it / QS) & 1, ctl, abort_flag, 43)) { ok = false; break; }
-        if (!mbar_wait(&s_free[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 44)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sQ = smem_u32(sm + L::Q0 + qs * L::Q_TILE);
-        const uint32_t sD = smem_u32(sm + L::DO0 + qs * L::Q_TILE);
+    // operand descriptors, computed once: K-major K, V, Q, dO; MN-major Q, dO for dK, dV
+    const uint64_t dK = sdesc_sw128(smem_u32(sm + L::K), 16, 1024);
+    const uint64_t dV = sdesc_sw128(smem_u32(sm + L::V), 16, 1024);
+    uint64_t dQk[2], dDk[2], dQm[2], dDm[2];
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * 8192 + (kk & 3) * 32;
-          umma_bf16(tS + st * 64, sdesc_sw128(sK + offa, 16, 1024), sdesc_sw128(sQ + offb, 16, 1024), idesc_s, kk > 0);
-          umma_bf16(tdP + st * 64, sdesc_sw128(sV + offa, 16, 1024), sdesc_sw128(sD + offb, 16, 1024), idesc_s,
-                    kk > 0);
-        }
-        umma_commit(&s_full[st]);
-        issued = true;
-      }
-      if (it >= 1) {
-        const int jt = it - 1;
-        const int bb = jt & 1;
-        if (!mbar_wait(&pd_full[bb], (jt >> 1) & 1, ctl, abort_flag, 45)) { ok = false; break; }
-        tc_fence_after();
-        const int qs = jt % QS;
-        const uint32_t sQ = smem_u32(sm + L::Q0 + qs * L::Q_TILE);
-        const uint32_t sD = smem_u32(sm + L::DO0 + qs * L::Q_TILE);
-        const uint32_t sP = smem_u32(sm + L::P0 + bb * 16384);
-        const uint32_t sDS = smem_u32(sm + L::DS0 + bb * 16384);
+    for (int i = 0; i < 2; ++i) {
+      dQk[i] = sdesc_sw128(smem_u32(sm + L::Q0 + i * L::TILE), 16, 1024);
+      dDk[i] = sdesc_sw128(smem_u32(sm + L::DO0 + i * L::TILE), 16, 1024);
+      dQm[i] = sdesc_sw128(smem_u32(sm + L::Q0 + i * L::TILE), 16384, 1024);
+      dDm[i] = sdesc_sw128(smem_u32(sm + L::DO0 + i * L::TILE), 16384, 1024);
+    }
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int st = it & 1;
+      if (!mbar_wait(&q_full[st], (it >> 1) & 1, ctl, abort_flag, 43)) { ok = false; break; }
+      // the S^T / dP^T columns still hold the previous block's P^T / dS^T until its products finish
+      if (it > 0 && !mbar_wait(d_done, (it - 1) & 1, ctl, abort_flag, 44)) { ok = false; break; }
+      tc_fence_after();
+      const uint64_t dQ = st ? dQk[1] : dQk[0], dD = st ? dDk[1] : dDk[0];
+      const uint64_t dQn = st ? dQm[1] : dQm[0], dDn = st ? dDm[1] : dDm[0];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          umma_bf16(tdV, sdesc_sw128(sP + kk * 32, 16, 1024), sdesc_sw128(sD + kk * 2048, 8192, 1024), idesc_acc,
-                    (jt | kk) != 0);
-          umma_bf16(tdK, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sQ + kk * 2048, 8192, 1024), idesc_acc,
-                    (jt | kk) != 0);
-        }
-        umma_commit(&pd_empty[bb]);
-        umma_commit(&q_empty[qs]);
-        issued = true;
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        umma_bf16(tS, sdesc_add(dK, off), sdesc_add(dQ, off), idesc_s, kk > 0);
+        umma_bf16(tdP, sdesc_add(dV, off), sdesc_add(dD, off), idesc_s, kk > 0);
       }
+      umma_commit(s_full);
+      issued = true;
+      for (int hh = 0; hh < 2 && ok; ++hh) {
+        if (!mbar_wait(&h_full[hh], it & 1, ctl, abort_flag, 45)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const int kk = 4 * hh + kq;  // 16 queries
+          const uint32_t acc = (it | kk) != 0;
+          umma_bf16_ts(tdV, tS + 16 * kk, sdesc_add(dDn, kk * 2048), idesc_d, acc);
+          umma_bf16_ts(tdK, tdP + 16 * kk, sdesc_add(dQn, kk * 2048), idesc_d, acc);
+        }
+      }
+      if (!ok) break;
+      umma_commit(d_done);
+      umma_commit(&q_empty[st]);
     }
     if (ok) {
       umma_commit(acc_full);
@@ -518,96 +519,103 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(drain, 0, ctl, &never, 46);
     }
   } else if (warp >= 2) {
-    // two warpgroups: group cg takes query columns [32 cg, 32 cg + 32) of every 64-query step
-    const int quad = warp & 3;
-    const int cg = (warp - 2) >> 2;
-    const int sw = warp - 2;         // 0..7: which 8 queries' statistics this warp stages
+    // ------------------------------------------------ elementwise warps
+    const int ew = warp - 2;         // 0..15
+    const int quad = warp & 3;       // TMEM lane quadrant: keys 32 quad .. 32 quad + 31
+    const int w = ew >> 2;           // 16-query group within each half
     const int r = quad * 32 + lane;  // key row within the tile
     const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const float* lse_bh = lse + (long long)bh * s.T;
     const float* del_bh = delta + (long long)bh * s.T;
+    // statistics staging: this warp owns 8 queries of each block (lanes 0-7 lse, 8-15 delta)
+    const int qq = 8 * ew + (lane & 7);
+    auto stat_of = [&](int qb) -> float {
+      const int q = qb + qq;
+      if (lane >= 16 || q >= s.T) return 0.f;
+      return lane < 8 ? __ldg(lse_bh + q) * kLog2e : __ldg(del_bh + q);
+    };
+    float v_next = stat_of(k0);
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int st = it & 1;
-      const int qb = (i0 + it) * 64;
-      {  // per-query statistics of this step: lse in log2 units and delta
-        if (lane < 16) {
-          const int qq = 8 * sw + (lane & 7);
-          const int q = qb + qq;
-          float v = 0.f;
-          if (q < s.T) v = lane < 8 ? __ldg(lse_bh + q) * kLog2e : __ldg(del_bh + q);
-          stats[st * 128 + (lane < 8 ? 0 : 64) + qq] = v;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&stats_bar[st]);
-      }
+      const int qb = (kt + it) * 128;
+      if (lane < 16) stats[st * 256 + (lane < 8 ? 0 : 128) + qq] = v_next;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&stats_bar[st]);
+      if (it + 1 < n_it) v_next = stat_of(qb + 128);  // one block ahead
       if (!mbar_wait(&stats_bar[st], (it >> 1) & 1, ctl, abort_flag, 50)) { ok = false; break; }
-      if (!mbar_wait(&s_full[st], (it >> 1) & 1, ctl, abort_flag, 47)) { ok = false; break; }
+      if (!mbar_wait(s_full, it & 1, ctl, abort_flag, 47)) { ok = false; break; }
       tc_fence_after();
-      uint32_t rs[32], rd[32];
-      tmem_ld32_nowait(tS + st * 64 + lane_off + 32 * cg, rs);
-      tmem_ld32_nowait(tdP + st * 64 + lane_off + 32 * cg, rd);
-      tmem_wait_ld();
-      tmem_fence_regs<32>(rs);
-      tmem_fence_regs<32>(rd);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[st]);
-      // the P^T / dS^T buffer of this step is free once the dV/dK products two steps back are done
-      if (!mbar_wait(&pd_empty[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 48)) { ok = false; break; }
-      const bool masked = (qb < k0 + 128) || (qb + 64 > s.T);
-      const uint32_t sP = smem_u32(sm + L::P0 + st * 16384);
-      const uint32_t sDS = smem_u32(sm + L::DS0 + st * 16384);
-      const float* stl = stats + st * 128 + 32 * cg;
+      const bool masked = (it == 0) || (qb + 128 > s.T);
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c = 4 * hh + w;  // queries qb + 16c .. qb + 16c + 15
+        uint32_t rs[16], rd[16];
+        tmem_ld16_nowait(tS + lane_off + 16 * c, rs);
+        tmem_ld16_nowait(tdP + lane_off + 16 * c, rd);
+        tmem_wait_ld();
+        tmem_fence_regs<16>(rs);
+        tmem_fence_regs<16>(rd);
+        const float* stl = stats + st * 256 + 16 * c;
+        uint32_t pw[8], dw[8];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float4 l0 = *reinterpret_cast<const float4*>(stl + 8 * g);
-        const float4 l1 = *reinterpret_cast<const float4*>(stl + 8 * g + 4);
-        const float4 d0 = *reinterpret_cast<const float4*>(stl + 64 + 8 * g);
-        const float4 d1 = *reinterpret_cast<const float4*>(stl + 64 + 8 * g + 4);
-        const float l2[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-        const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-        float p[8], ds[8];
+        for (int g = 0; g < 4; ++g) {
+          const float4 l4 = *reinterpret_cast<const float4*>(stl + 4 * g);
+          const float4 d4 = *reinterpret_cast<const float4*>(stl + 128 + 4 * g);
+          const float l2[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
+          float p[4], ds[4];
+          if (masked) {  // the diagonal block or the ragged end: causal / range mask
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int e = 8 * g + k;
-          float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
-          if (masked) {
-            const int q = qb + 32 * cg + e;
-            if (q < key || q >= s.T) pv = 0.f;
+            for (int k = 0; k < 4; ++k) {
+              const int e = 4 * g + k;
+              const int q = qb + 16 * c + e;
+              float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
+              if (q < key || q >= s.T) pv = 0.f;
+              p[k] = pv;
+              ds[k] = pv * (__uint_as_float(rd[e]) - dl[k]);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 4 * g + k;
+              p[k] = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
+              ds[k] = p[k] * (__uint_as_float(rd[e]) - dl[k]);
+            }
           }
-          p[k] = pv;
-          ds[k] = pv * (__uint_as_float(rd[e]) - dl[k]);
+          pw[2 * g] = pack_bf16x2(p[0], p[1]);
+          pw[2 * g + 1] = pack_bf16x2(p[2], p[3]);
+          dw[2 * g] = pack_bf16x2(ds[0], ds[1]);
+          dw[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        st_shared_v4(sP + sw128_off(r, 4 * cg + g), make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]),
-                                                               pack_bf16x2(p[4], p[5]), pack_bf16x2(p[6], p[7])));
-        st_shared_v4(sDS + sw128_off(r, 4 * cg + g),
-                     make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
-                                pack_bf16x2(ds[6], ds[7])));
+        // bf16 P^T and dS^T over the first 8 of the 16 columns this warp has just read
+        tmem_st8(tS + lane_off + 16 * c, pw);
+        tmem_st8(tdP + lane_off + 16 * c, dw);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&h_full[hh]);
       }
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&pd_full[st]);
     }
-    // the two warpgroups share the epilogue: group 0 writes dK, group 1 writes dV
+    // epilogue: the four warps of a quadrant split dK (times the softmax scale) and dV
     if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 49)) {
       tc_fence_after();
+      constexpr int CPW = HD / 2;  // columns per warp
       const bool row_ok = key < s.T;
       const long long m = (long long)b * s.T + key;
-      // group 0: dK (times the softmax scale), group 1: dV
-      __nv_bfloat16* dst = dqkv + m * s.ld_qkv + (long long)(1 + cg) * s.H * s.hdp + (long long)h * s.hdp;
-      const uint32_t tsrc = (cg == 0 ? tdK : tdV) + lane_off;
-      const float f = cg == 0 ? scale : 1.f;
+      const int which = w >> 1;  // 0: dK, 1: dV
+      const int cbase = (w & 1) * CPW;
+      __nv_bfloat16* dst = dqkv + m * s.ld_qkv + (long long)(1 + which) * s.H * s.hdp + (long long)h * s.hdp;
+      const uint32_t tsrc = (which == 0 ? tdK : tdV) + lane_off;
+      const float f = which == 0 ? scale : 1.f;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
+      for (int c = cbase; c < cbase + CPW; c += 32) {
         float a[32];
-        tmem_ld32(tsrc + c * 32, a);
+        tmem_ld32(tsrc + c, a);
         if (row_ok) {
 #pragma unroll
           for (int g = 0; g < 4; ++g)
-            reinterpret_cast<uint4*>(dst + c * 32)[g] =
+            reinterpret_cast<uint4*>(dst + c)[g] =
                 make_uint4(pack_bf16x2(a[8 * g] * f, a[8 * g + 1] * f), pack_bf16x2(a[8 * g + 2] * f, a[8 * g + 3] * f),
                            pack_bf16x2(a[8 * g + 4] * f, a[8 * g + 5] * f),
                            pack_bf16x2(a[8 * g + 6] * f, a[8 * g + 7] * f));
@@ -624,66 +632,74 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ====================================================================== backward: dQ
-// One CTA per 128-query tile, stepping over 64-key tiles: S = Q K^T and dP = dO V^T into
-// double-buffered TMEM, dS = P (dP - delta) into double-buffered shared memory, dQ += dS K.
+// One CTA per 128-query tile, stepping over 128-key blocks up to the diagonal one:
+//   S = Q K^T and dP = dO V^T into TMEM (N = 128, full rate); sixteen elementwise warps write
+//   dS = P (dP - delta) as bf16 into one of two TMEM buffers, from which dQ += dS K takes its
+//   A operand.  S and dP are free again as soon as the elementwise warps have loaded them, so
+//   the next block's S / dP products run while this block's dS is computed.
+// TMEM: S [0,128), dP [128,256), dQ [256, 256+HD), dS [2] at 384 and 448.
+// Shared memory: Q, dO, a 3-deep K ring (K is read by S and by dQ) and a 2-deep V ring.
 
 template <int HD>
 struct DqSmem {
-  static constexpr int KS = 4;              // K / V ring depth
-  static constexpr int Q_TILE = HD * 256;   // 128 rows
-  static constexpr int KV_TILE = HD * 128;  // 64 rows
+  static constexpr int TILE = HD * 256;
+  static constexpr int KS = 3, VS = 2;
   static constexpr int Q = 0;
-  static constexpr int DO = Q + Q_TILE;
-  static constexpr int K0 = DO + Q_TILE;        // [KS]
-  static constexpr int V0 = K0 + KS * KV_TILE;  // [KS]
-  static constexpr int DS0 = V0 + KS * KV_TILE; // [2] 128 queries x 64 keys bf16 = 16 KB
-  static constexpr int BAR = DS0 + 32768;
+  static constexpr int DO = Q + TILE;
+  static constexpr int K0 = DO + TILE;        // [KS]
+  static constexpr int V0 = K0 + KS * TILE;   // [VS]
+  static constexpr int BAR = V0 + VS * TILE;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
 
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q128, const __grid_constant__ CUtensorMap tm_do128,
-                       const __grid_constant__ CUtensorMap tm_kv64, const AttnShape s, const float* __restrict__ lse,
+                       const __grid_constant__ CUtensorMap tm_kv128, const AttnShape s, const float* __restrict__ lse,
                        const float* __restrict__ delta, __nv_bfloat16* __restrict__ dqkv, float scale_log2,
                        float scale, DevCtl ctl) {
   using L = DqSmem<HD>;
+  constexpr int KS = L::KS, VS = L::VS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
-  constexpr int KS = L::KS;
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;          // [KS]
-  uint64_t* kv_empty = bars + 1 + KS;    // [KS]
-  uint64_t* s_full = bars + 1 + 2 * KS;  // [2]
-  uint64_t* s_free = s_full + 2;         // [2]
-  uint64_t* ds_full = s_full + 4;        // [2]
-  uint64_t* ds_empty = s_full + 6;       // [2]
-  uint64_t* acc_full = s_full + 8;
-  uint64_t* drain = s_full + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
+  uint64_t* k_full = bars + 1;             // [KS]
+  uint64_t* k_empty = k_full + KS;         // [KS]
+  uint64_t* v_full = k_empty + KS;         // [VS]
+  uint64_t* v_empty = v_full + VS;         // [VS]
+  uint64_t* s_full = v_empty + VS;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* ds_full = s_full + 2;          // [2]
+  uint64_t* ds_empty = s_full + 4;         // [2]
+  uint64_t* acc_full = s_full + 6;
+  uint64_t* drain = s_full + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = gridDim.x;
-  const int qt = n_qt - 1 - blockIdx.x;
+  const int qt = n_qt - 1 - blockIdx.x;  // heaviest tiles first
   const int bh = blockIdx.y;
   const int b = bh / s.H, h = bh % s.H;
   const int q0 = qt * 128;
-  const int kend = min(q0 + 128, s.T);
-  const int n_kv = (kend + 63) / 64;
+  const int n_kv = qt + 1;  // 128-key blocks 0 .. qt (the last one is the diagonal block)
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < KS; ++i) {
-      mbar_init(&kv_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
     }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kBwdEw);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 8);
-      mbar_init(&ds_full[i], 8);
+      mbar_init(&ds_full[i], kBwdEw);
       mbar_init(&ds_empty[i], 1);
     }
     mbar_init(acc_full, 1);
@@ -699,9 +715,10 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t tS = tbase;         // [2] x 64
-  const uint32_t tdP = tbase + 128;  // [2] x 64
+  const uint32_t tS = tbase;
+  const uint32_t tdP = tbase + 128;
   const uint32_t tdQ = tbase + 256;
+  const uint32_t tdS = tbase + 384;  // [2] x 64 columns
 
   const int colq = h * s.hdp;
   const int colk = s.H * s.hdp + h * s.hdp;
@@ -709,69 +726,79 @@ __global__ void __launch_bounds__(320, 1)
   const int cold = h * s.hdp;
 
   if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer
     bool ok = true;
-    mbar_expect_tx(q_full, 2 * L::Q_TILE);
+    mbar_expect_tx(q_full, 2 * L::TILE);
     for (int c = 0; c < NCH; ++c) {
       tma_load_3d(sm + L::Q + c * 16384, &tm_q128, q_full, colq + 64 * c, q0, b);
       tma_load_3d(sm + L::DO + c * 16384, &tm_do128, q_full, cold + 64 * c, q0, b);
     }
-    int issued = -1;
+    int issued_k = -1, issued_v = -1;
     for (int j = 0; j < n_kv && ok; ++j) {
-      const int st = j % KS;
-      if (!mbar_wait(&kv_empty[st], ((j / KS) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
-      mbar_expect_tx(&kv_full[st], 2 * L::KV_TILE);
-      for (int c = 0; c < NCH; ++c) {
-        tma_load_3d(sm + L::K0 + st * L::KV_TILE + c * 8192, &tm_kv64, &kv_full[st], colk + 64 * c, j * 64, b);
-        tma_load_3d(sm + L::V0 + st * L::KV_TILE + c * 8192, &tm_kv64, &kv_full[st], colv + 64 * c, j * 64, b);
-      }
-      issued = j;
+      const int ks = j % KS;
+      if (!mbar_wait(&k_empty[ks], ((j / KS) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
+      mbar_expect_tx(&k_full[ks], L::TILE);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_3d(sm + L::K0 + ks * L::TILE + c * 16384, &tm_kv128, &k_full[ks], colk + 64 * c, j * 128, b);
+      issued_k = j;
+      const int vs = j % VS;
+      if (!mbar_wait(&v_empty[vs], ((j / VS) & 1) ^ 1u, ctl, abort_flag, 61)) { ok = false; break; }
+      mbar_expect_tx(&v_full[vs], L::TILE);
+      for (int c = 0; c < NCH; ++c)
+        tma_load_3d(sm + L::V0 + vs * L::TILE + c * 16384, &tm_kv128, &v_full[vs], colv + 64 * c, j * 128, b);
+      issued_v = j;
     }
     if (!ok) {
       volatile int never = 0;
-      mbar_wait(q_full, 0, ctl, &never, 61);
-      for (int j = (issued >= KS ? issued - KS + 1 : 0); j <= issued && issued >= 0; ++j)
-        mbar_wait(&kv_full[j % KS], (j / KS) & 1, ctl, &never, 61);
+      mbar_wait(q_full, 0, ctl, &never, 62);
+      for (int j = (issued_k >= KS ? issued_k - KS + 1 : 0); j <= issued_k && issued_k >= 0; ++j)
+        mbar_wait(&k_full[j % KS], (j / KS) & 1, ctl, &never, 62);
+      for (int j = (issued_v >= VS ? issued_v - VS + 1 : 0); j <= issued_v && issued_v >= 0; ++j)
+        mbar_wait(&v_full[j % VS], (j / VS) & 1, ctl, &never, 62);
     }
   } else if (warp == 1 && lane == 0) {
-    constexpr uint32_t idesc_s = idesc_bf16(128, 64, 0, 0);
-    constexpr uint32_t idesc_acc = idesc_bf16(128, HD, 0, 1);
-    bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 62);
+    // ------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
+    constexpr uint32_t idesc_d = idesc_bf16(128, HD, 0, 1);
+    bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 63);
     bool issued = false;
-    const uint32_t sQ = smem_u32(sm + L::Q), sD = smem_u32(sm + L::DO);
+    const uint64_t dQ = sdesc_sw128(smem_u32(sm + L::Q), 16, 1024);
+    const uint64_t dD = sdesc_sw128(smem_u32(sm + L::DO), 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::K0), 16, 1024);       // K-major, stage 0
+    const uint64_t dKm0 = sdesc_sw128(smem_u32(sm + L::K0), 16384, 1024);   // MN-major, stage 0
+    const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::V0), 16, 1024);
     for (int j = 0; j <= n_kv && ok; ++j) {
       if (j < n_kv) {
-        const int st = j & 1;
-        const int ks = j % KS;
-        if (!mbar_wait(&kv_full[ks], (j / KS) & 1, ctl, abort_flag, 63)) { ok = false; break; }
-        if (!mbar_wait(&s_free[st], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 64)) { ok = false; break; }
+        const int ks = j % KS, vs = j % VS;
+        if (!mbar_wait(&k_full[ks], (j / KS) & 1, ctl, abort_flag, 64)) { ok = false; break; }
+        if (!mbar_wait(&v_full[vs], (j / VS) & 1, ctl, abort_flag, 64)) { ok = false; break; }
+        // S / dP are free once the elementwise warps have loaded the previous block's
+        if (j > 0 && !mbar_wait(s_free, (j - 1) & 1, ctl, abort_flag, 65)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sK = smem_u32(sm + L::K0 + ks * L::KV_TILE);
-        const uint32_t sV = smem_u32(sm + L::V0 + ks * L::KV_TILE);
+        const uint64_t dK = sdesc_add(dK0, ks * L::TILE);
+        const uint64_t dV = sdesc_add(dV0, vs * L::TILE);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t offb = (kk >> 2) * 8192 + (kk & 3) * 32;
-          umma_bf16(tS + st * 64, sdesc_sw128(sQ + offa, 16, 1024), sdesc_sw128(sK + offb, 16, 1024), idesc_s, kk > 0);
-          umma_bf16(tdP + st * 64, sdesc_sw128(sD + offa, 16, 1024), sdesc_sw128(sV + offb, 16, 1024), idesc_s,
-                    kk > 0);
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tS, sdesc_add(dQ, off), sdesc_add(dK, off), idesc_s, kk > 0);
+          umma_bf16(tdP, sdesc_add(dD, off), sdesc_add(dV, off), idesc_s, kk > 0);
         }
-        umma_commit(&s_full[st]);
+        umma_commit(s_full);
+        umma_commit(&v_empty[vs]);
         issued = true;
       }
       if (j >= 1) {
         const int jj = j - 1;
         const int bb = jj & 1;
-        if (!mbar_wait(&ds_full[bb], (jj >> 1) & 1, ctl, abort_flag, 65)) { ok = false; break; }
+        if (!mbar_wait(&ds_full[bb], (jj >> 1) & 1, ctl, abort_flag, 66)) { ok = false; break; }
         tc_fence_after();
-        const int ks = jj % KS;
-        const uint32_t sK = smem_u32(sm + L::K0 + ks * L::KV_TILE);
-        const uint32_t sDS = smem_u32(sm + L::DS0 + bb * 16384);
+        const uint64_t dKm = sdesc_add(dKm0, (jj % KS) * L::TILE);
+        const uint32_t tA = tdS + 64 * bb;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tdQ, sdesc_sw128(sDS + kk * 32, 16, 1024), sdesc_sw128(sK + kk * 2048, 8192, 1024), idesc_acc,
-                    (jj | kk) != 0);
+        for (int kk = 0; kk < 8; ++kk)  // 16 keys each
+          umma_bf16_ts(tdQ, tA + 8 * kk, sdesc_add(dKm, kk * 2048), idesc_d, (jj | kk) != 0);
         umma_commit(&ds_empty[bb]);
-        umma_commit(&kv_empty[ks]);
+        umma_commit(&k_empty[jj % KS]);
         issued = true;
       }
     }
@@ -780,73 +807,93 @@ __global__ void __launch_bounds__(320, 1)
     } else if (issued) {
       volatile int never = 0;
       umma_commit(drain);
-      mbar_wait(drain, 0, ctl, &never, 66);
+      mbar_wait(drain, 0, ctl, &never, 67);
     }
   } else if (warp >= 2) {
-    // two warpgroups: group cg takes key columns [32 cg, 32 cg + 32) of every 64-key step
-    const int quad = warp & 3;
-    const int cg = (warp - 2) >> 2;
-    const int r = quad * 32 + lane;
-    const int qi = q0 + r;
+    // ------------------------------------------------ elementwise warps
+    const int ew = warp - 2;
+    const int quad = warp & 3;  // TMEM lane quadrant: queries 32 quad .. 32 quad + 31
+    const int cg = ew >> 2;     // key columns 32 cg .. 32 cg + 31 of each block
+    const int qi = q0 + quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const bool row_ok = qi < s.T;
     const float lse2 = row_ok ? lse[(long long)bh * s.T + qi] * kLog2e : 0.f;
     const float dl = row_ok ? delta[(long long)bh * s.T + qi] : 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&s_full[st], (j >> 1) & 1, ctl, abort_flag, 67)) { ok = false; break; }
+      if (!mbar_wait(s_full, j & 1, ctl, abort_flag, 68)) { ok = false; break; }
       tc_fence_after();
       uint32_t rs[32], rd[32];
-      tmem_ld32_nowait(tS + st * 64 + lane_off + 32 * cg, rs);
-      tmem_ld32_nowait(tdP + st * 64 + lane_off + 32 * cg, rd);
+      tmem_ld32_nowait(tS + lane_off + 32 * cg, rs);
+      tmem_ld32_nowait(tdP + lane_off + 32 * cg, rd);
       tmem_wait_ld();
       tmem_fence_regs<32>(rs);
       tmem_fence_regs<32>(rd);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[st]);
-      if (!mbar_wait(&ds_empty[st], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 68)) { ok = false; break; }
-      const int kb = j * 64 + 32 * cg;
-      const bool masked = (kb + 31 > q0) || (kb + 32 > s.T) || !row_ok;
-      const uint32_t sDS = smem_u32(sm + L::DS0 + st * 16384);
+      if (lane == 0) mbar_arrive(s_free);
+      const int bb = j & 1;
+      if (!mbar_wait(&ds_empty[bb], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 69)) { ok = false; break; }
+      const int kb = j * 128 + 32 * cg;
+      uint32_t dw[16];
+      if ((kb + 31 > q0) || (kb + 32 > s.T) || !row_ok) {
+        // diagonal block, ragged end or rows past T: causal / range mask
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float ds[8];
+        for (int e2 = 0; e2 < 16; ++e2) {
+          float d2[2];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int e = 8 * g + k;
-          float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -lse2));
-          if (masked) {
+          for (int k = 0; k < 2; ++k) {
+            const int e = 2 * e2 + k;
             const int key = kb + e;
+            float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -lse2));
             if (!row_ok || key > qi || key >= s.T) pv = 0.f;
+            d2[k] = pv * (__uint_as_float(rd[e]) - dl);
           }
-          ds[k] = pv * (__uint_as_float(rd[e]) - dl);
+          dw[e2] = pack_bf16x2(d2[0], d2[1]);
         }
-        st_shared_v4(sDS + sw128_off(r, 4 * cg + g),
-                     make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
-                                pack_bf16x2(ds[6], ds[7])));
+      } else {
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(rs[2 * e2]), scale_log2, -lse2));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(rs[2 * e2 + 1]), scale_log2, -lse2));
+          dw[e2] = pack_bf16x2(p0 * (__uint_as_float(rd[2 * e2]) - dl), p1 * (__uint_as_float(rd[2 * e2 + 1]) - dl));
+        }
       }
-      fence_async_smem();
+      tmem_st16(tdS + 64 * bb + lane_off + 16 * cg, dw);
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[st]);
+      if (lane == 0) mbar_arrive(&ds_full[bb]);
     }
-    if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 69)) {
+    if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 70)) {
       tc_fence_after();
-      __nv_bfloat16* dq = dqkv + ((long long)b * s.T + qi) * s.ld_qkv + (long long)h * s.hdp;
-      // the two groups split dQ's columns
-#pragma unroll 1
-      for (int c = cg * (HD / 64); c < (cg + 1) * (HD / 64); ++c) {
+      // the four warps of a quadrant split dQ's columns
+      constexpr int CPW = HD / 4;
+      __nv_bfloat16* dq = dqkv + ((long long)b * s.T + qi) * s.ld_qkv + (long long)h * s.hdp + cg * CPW;
+      if (CPW == 32) {
         float a[32];
-        tmem_ld32(tdQ + lane_off + c * 32, a);
+        tmem_ld32(tdQ + lane_off + cg * CPW, a);
         if (row_ok) {
 #pragma unroll
           for (int g = 0; g < 4; ++g)
-            reinterpret_cast<uint4*>(dq + c * 32)[g] = make_uint4(
+            reinterpret_cast<uint4*>(dq)[g] = make_uint4(
                 pack_bf16x2(a[8 * g] * scale, a[8 * g + 1] * scale), pack_bf16x2(a[8 * g + 2] * scale, a[8 * g + 3] * scale),
                 pack_bf16x2(a[8 * g + 4] * scale, a[8 * g + 5] * scale),
                 pack_bf16x2(a[8 * g + 6] * scale, a[8 * g + 7] * scale));
+        }
+      } else {
+        uint32_t a[16];
+        tmem_ld16_nowait(tdQ + lane_off + cg * CPW, a);
+        tmem_wait_ld();
+        tmem_fence_regs<16>(a);
+        if (row_ok) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+            reinterpret_cast<uint4*>(dq)[g] = make_uint4(
+                pack_bf16x2(__uint_as_float(a[8 * g]) * scale, __uint_as_float(a[8 * g + 1]) * scale),
+                pack_bf16x2(__uint_as_float(a[8 * g + 2]) * scale, __uint_as_float(a[8 * g + 3]) * scale),
+                pack_bf16x2(__uint_as_float(a[8 * g + 4]) * scale, __uint_as_float(a[8 * g + 5]) * scale),
+                pack_bf16x2(__uint_as_float(a[8 * g + 6]) * scale, __uint_as_float(a[8 * g + 7]) * scale));
         }
       }
     }
@@ -890,13 +937,10 @@ template <int HD>
 static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const float* lse, const float* delta,
                       const AttnShape& s, __nv_bfloat16* dqkv, cudaStream_t st) {
   const uint64_t ldd = (uint64_t)s.H * s.hdp;
-  CUtensorMap kv128, q64, do64, q128, do128, kv64;
-  GPTK_TRY(make_tmap_3d(&kv128, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
-  GPTK_TRY(make_tmap_3d(&q64, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 64, 1));
-  GPTK_TRY(make_tmap_3d(&do64, dop, ldd, s.T, s.B, ldd, (uint64_t)s.T * ldd, 64, 64, 1));
-  GPTK_TRY(make_tmap_3d(&q128, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
+  // 128-row boxes of one 64-column chunk of q, k, v (the padded q|k|v buffer) and of dO
+  CUtensorMap qkv128, do128;
+  GPTK_TRY(make_tmap_3d(&qkv128, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
   GPTK_TRY(make_tmap_3d(&do128, dop, ldd, s.T, s.B, ldd, (uint64_t)s.T * ldd, 64, 128, 1));
-  GPTK_TRY(make_tmap_3d(&kv64, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 64, 1));
   const float scale = 1.f / sqrtf((float)s.hd);
   const float scale_log2 = kLog2e * scale;
   const DevCtl ctl = device_ctl();
@@ -907,7 +951,8 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
     Prof prof(PK_ATTN_BWD_DKV, 8.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 6, st);
-    attn_bwd_dkv_kernel<HD><<<grid, 320, L::BYTES, st>>>(kv128, q64, do64, s, lse, delta, dqkv, scale_log2, scale, ctl);
+    attn_bwd_dkv_kernel<HD><<<grid, kBwdThreads, L::BYTES, st>>>(qkv128, qkv128, do128, s, lse, delta, dqkv, scale_log2,
+                                                                 scale, ctl);
     GPTK_CUDA(cudaGetLastError());
   }
   {
@@ -916,7 +961,8 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
     dim3 grid((s.T + 127) / 128, s.B * s.H);
     Prof prof(PK_ATTN_BWD_DQ, 6.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 5, st);
-    attn_bwd_dq_kernel<HD><<<grid, 320, L::BYTES, st>>>(q128, do128, kv64, s, lse, delta, dqkv, scale_log2, scale, ctl);
+    attn_bwd_dq_kernel<HD><<<grid, kBwdThreads, L::BYTES, st>>>(qkv128, do128, qkv128, s, lse, delta, dqkv, scale_log2,
+                                                                scale, ctl);
     GPTK_CUDA(cudaGetLastError());
   }
   return ST_OK;
