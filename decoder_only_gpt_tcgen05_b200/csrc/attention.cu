@@ -151,23 +151,46 @@ __global__ void __launch_bounds__(320, 1)
     auto kv_wait = [&](int seq) -> bool {
       return mbar_wait(&kv_full[seq % 3], (seq / 3) & 1, ctl, abort_flag, 24);
     };
+    // operand descriptors computed once; the MMAs of a product go out back to back (umma8_ss)
+    const uint64_t dQ0 = sdesc_sw128(smem_u32(sm + L::Q0), 16, 1024);
+    const uint64_t dKV0 = sdesc_sw128(smem_u32(sm + L::KV), 16, 1024);     // K-major (K for S)
+    const uint64_t dKVm0 = sdesc_sw128(smem_u32(sm + L::KV), 16384, 1024);  // MN-major (V for PV)
+    const uint64_t dP0 = sdesc_sw128(smem_u32(sm + L::P), 16, 1024);
     auto issue_s = [&](int t, int j) {
-      const uint32_t sQ = smem_u32(sm + L::Q0 + t * L::TILE);
-      const uint32_t sK = smem_u32(sm + L::KV + ((2 * j) % 3) * L::TILE);
+      const uint64_t dQ = sdesc_add(dQ0, t * L::TILE);
+      const uint64_t dK = sdesc_add(dKV0, ((2 * j) % 3) * L::TILE);
+      if (HD == 128) {
+        uint32_t dd[8];
+        uint64_t aa[8], bb[8];
 #pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        umma_bf16(tbase + 128 * t, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), idesc_s, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          dd[kk] = tbase + 128 * t;
+          aa[kk] = sdesc_add(dQ, off);
+          bb[kk] = sdesc_add(dK, off);
+        }
+        umma8_ss(dd, aa, bb, idesc_s, 0xfeu);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_bf16(tbase + 128 * t, sdesc_add(dQ, off), sdesc_add(dK, off), idesc_s, kk > 0);
+        }
       }
       umma_commit(&s_full[t]);
     };
     auto issue_pv = [&](int t, int j) {
-      const uint32_t sP = smem_u32(sm + L::P + t * 32768);
-      const uint32_t sV = smem_u32(sm + L::KV + ((2 * j + 1) % 3) * L::TILE);
+      const uint64_t dP = sdesc_add(dP0, t * 32768);
+      const uint64_t dV = sdesc_add(dKVm0, ((2 * j + 1) % 3) * L::TILE);
+      uint32_t dd[8];
+      uint64_t aa[8], bb[8];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        umma_bf16(tbase + 256 + 128 * t, sdesc_sw128(sP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(sV + kk * 2048, 16384, 1024), idesc_o, (j | kk) != 0);
+      for (int kk = 0; kk < 8; ++kk) {
+        dd[kk] = tbase + 256 + 128 * t;
+        aa[kk] = sdesc_add(dP, (kk >> 2) * 16384 + (kk & 3) * 32);
+        bb[kk] = sdesc_add(dV, kk * 2048);
+      }
+      umma8_ss(dd, aa, bb, idesc_o, j == 0 ? 0xfeu : 0xffu);
       umma_commit(&o_done[t]);
     };
     if (ok && kv_wait(0)) {
@@ -488,24 +511,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after();
       const uint64_t dQ = st ? dQk[1] : dQk[0], dD = st ? dDk[1] : dDk[0];
       const uint64_t dQn = st ? dQm[1] : dQm[0], dDn = st ? dDm[1] : dDm[0];
+      // S^T and dP^T, interleaved, in groups of four K steps issued back to back
 #pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        umma_bf16(tS, sdesc_add(dK, off), sdesc_add(dQ, off), idesc_s, kk > 0);
-        umma_bf16(tdP, sdesc_add(dV, off), sdesc_add(dD, off), idesc_s, kk > 0);
+      for (int g = 0; g < HD / 64; ++g) {
+        uint32_t dd[8];
+        uint64_t aa[8], bb[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t off = g * 16384 + i * 32;
+          dd[2 * i] = tS;
+          dd[2 * i + 1] = tdP;
+          aa[2 * i] = sdesc_add(dK, off);
+          aa[2 * i + 1] = sdesc_add(dV, off);
+          bb[2 * i] = sdesc_add(dQ, off);
+          bb[2 * i + 1] = sdesc_add(dD, off);
+        }
+        umma8_ss(dd, aa, bb, idesc_s, g == 0 ? 0xfcu : 0xffu);
       }
       umma_commit(s_full);
       issued = true;
       for (int hh = 0; hh < 2 && ok; ++hh) {
         if (!mbar_wait(&h_full[hh], it & 1, ctl, abort_flag, 45)) { ok = false; break; }
         tc_fence_after();
+        uint32_t dd[8], aa[8];
+        uint64_t bb[8];
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int kk = 4 * hh + kq;  // 16 queries
-          const uint32_t acc = (it | kk) != 0;
-          umma_bf16_ts(tdV, tS + 16 * kk, sdesc_add(dDn, kk * 2048), idesc_d, acc);
-          umma_bf16_ts(tdK, tdP + 16 * kk, sdesc_add(dQn, kk * 2048), idesc_d, acc);
+          dd[2 * kq] = tdV;
+          dd[2 * kq + 1] = tdK;
+          aa[2 * kq] = tS + 16 * kk;
+          aa[2 * kq + 1] = tdP + 16 * kk;
+          bb[2 * kq] = sdesc_add(dDn, kk * 2048);
+          bb[2 * kq + 1] = sdesc_add(dQn, kk * 2048);
         }
+        umma8_ts(dd, aa, bb, idesc_d, (hh == 0 && it == 0) ? 0xfcu : 0xffu);
       }
       if (!ok) break;
       umma_commit(d_done);
@@ -778,10 +818,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint64_t dK = sdesc_add(dK0, ks * L::TILE);
         const uint64_t dV = sdesc_add(dV0, vs * L::TILE);
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_bf16(tS, sdesc_add(dQ, off), sdesc_add(dK, off), idesc_s, kk > 0);
-          umma_bf16(tdP, sdesc_add(dD, off), sdesc_add(dV, off), idesc_s, kk > 0);
+        for (int g = 0; g < HD / 64; ++g) {
+          uint32_t dd[8];
+          uint64_t aa[8], bb[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t off = g * 16384 + i * 32;
+            dd[2 * i] = tS;
+            dd[2 * i + 1] = tdP;
+            aa[2 * i] = sdesc_add(dQ, off);
+            aa[2 * i + 1] = sdesc_add(dD, off);
+            bb[2 * i] = sdesc_add(dK, off);
+            bb[2 * i + 1] = sdesc_add(dV, off);
+          }
+          umma8_ss(dd, aa, bb, idesc_s, g == 0 ? 0xfcu : 0xffu);
         }
         umma_commit(s_full);
         umma_commit(&v_empty[vs]);
@@ -794,9 +844,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         const uint64_t dKm = sdesc_add(dKm0, (jj % KS) * L::TILE);
         const uint32_t tA = tdS + 64 * bb;
+        uint32_t dd[8], aa[8];
+        uint64_t bd[8];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 16 keys each
-          umma_bf16_ts(tdQ, tA + 8 * kk, sdesc_add(dKm, kk * 2048), idesc_d, (jj | kk) != 0);
+        for (int kk = 0; kk < 8; ++kk) {  // 16 keys each
+          dd[kk] = tdQ;
+          aa[kk] = tA + 8 * kk;
+          bd[kk] = sdesc_add(dKm, kk * 2048);
+        }
+        umma8_ts(dd, aa, bd, idesc_d, jj == 0 ? 0xfeu : 0xffu);
         umma_commit(&ds_empty[bb]);
         umma_commit(&k_empty[jj % KS]);
         issued = true;

@@ -427,6 +427,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
     uint32_t acc_phase = 0;
     bool ok = true;
     bool issued = false;
+    // stage-0 descriptors and the per-K-step advance, computed once: the four MMAs of a stage
+    // then go out back to back (umma4_ss*)
+    const uint64_t descA0 = p.a_mn ? sdesc_sw128(smem_u32(sA), 8192, 1024) : sdesc_sw128(smem_u32(sA), 16, 1024);
+    const uint64_t descB0 = p.b_mn ? sdesc_sw128(smem_u32(sB), 8192, 1024) : sdesc_sw128(smem_u32(sB), 16, 1024);
+    const uint32_t stepA = p.a_mn ? 2048u : 32u, stepB = p.b_mn ? 2048u : 32u;
     for (int tile = tile0; tile < num_tiles && ok; tile += tile_step) {
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.ctl, abort_flag, 3)) {
         ok = false;
@@ -440,15 +445,17 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
-        const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+        const uint64_t da = sdesc_add(descA0, stage * C::A_BYTES);
+        const uint64_t db = sdesc_add(descB0, stage * C::B_BYTES);
+        static_assert(C::BK == 64, "one stage is four K = 16 MMAs");
+        uint64_t aa[4], bb[4];
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk) {
-          const uint64_t ad = p.a_mn ? sdesc_sw128(a0 + kk * 2048, 8192, 1024) : sdesc_sw128(a0 + kk * 32, 16, 1024);
-          const uint64_t bd = p.b_mn ? sdesc_sw128(b0 + kk * 2048, 8192, 1024) : sdesc_sw128(b0 + kk * 32, 16, 1024);
-          if (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
-          else umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+        for (int kk = 0; kk < 4; ++kk) {
+          aa[kk] = sdesc_add(da, kk * stepA);
+          bb[kk] = sdesc_add(db, kk * stepB);
         }
+        if (PAIR) umma4_ss_pair(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
+        else umma4_ss(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
         if (PAIR) {
           // the stage is free in both CTAs once these MMAs have read it
           const uint32_t eb = smem_u32(&empty[stage]);

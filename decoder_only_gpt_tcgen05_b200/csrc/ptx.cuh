@@ -227,6 +227,102 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// Eight MMAs issued back to back from one asm block, every operand in a register beforehand and
+// the eight enable-accumulate predicates set up front (bit i of acc_mask for MMA i).  The issue
+// of tcgen05.mma is synchronous with the tensor pipe, so any instruction between two MMAs
+// lengthens the pipe's cycle; this form leaves none.
+__device__ __forceinline__ void umma8_ss(const uint32_t (&d)[8], const uint64_t (&a)[8], const uint64_t (&b)[8],
+                                         uint32_t idesc, uint32_t acc_mask) {
+  asm volatile(
+      "{\n\t.reg .pred p<8>;\n\t.reg .b32 t<8>;\n\t"
+      "and.b32 t0, %25, 1;\n\tsetp.ne.b32 p0, t0, 0;\n\t"
+      "and.b32 t1, %25, 2;\n\tsetp.ne.b32 p1, t1, 0;\n\t"
+      "and.b32 t2, %25, 4;\n\tsetp.ne.b32 p2, t2, 0;\n\t"
+      "and.b32 t3, %25, 8;\n\tsetp.ne.b32 p3, t3, 0;\n\t"
+      "and.b32 t4, %25, 16;\n\tsetp.ne.b32 p4, t4, 0;\n\t"
+      "and.b32 t5, %25, 32;\n\tsetp.ne.b32 p5, t5, 0;\n\t"
+      "and.b32 t6, %25, 64;\n\tsetp.ne.b32 p6, t6, 0;\n\t"
+      "and.b32 t7, %25, 128;\n\tsetp.ne.b32 p7, t7, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %24, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], %9, %17, %24, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], %10, %18, %24, p2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%3], %11, %19, %24, p3;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%4], %12, %20, %24, p4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%5], %13, %21, %24, p5;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%6], %14, %22, %24, p6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%7], %15, %23, %24, p7;\n\t"
+      "}"
+      ::"r"(d[0]), "r"(d[1]), "r"(d[2]), "r"(d[3]), "r"(d[4]), "r"(d[5]), "r"(d[6]), "r"(d[7]),
+      "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(a[4]), "l"(a[5]), "l"(a[6]), "l"(a[7]),
+      "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc),
+      "r"(acc_mask)
+      : "memory");
+}
+// Four MMAs into one accumulator, back to back (one K = 64 stage of a GEMM); bit i of acc_mask
+// enables accumulation for MMA i.  The pair form is the cta_group::2 MMA of a CTA pair.
+__device__ __forceinline__ void umma4_ss(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4], uint32_t idesc,
+                                         uint32_t acc_mask) {
+  asm volatile(
+      "{\n\t.reg .pred p<4>;\n\t.reg .b32 t<4>;\n\t"
+      "and.b32 t0, %10, 1;\n\tsetp.ne.b32 p0, t0, 0;\n\t"
+      "and.b32 t1, %10, 2;\n\tsetp.ne.b32 p1, t1, 0;\n\t"
+      "and.b32 t2, %10, 4;\n\tsetp.ne.b32 p2, t2, 0;\n\t"
+      "and.b32 t3, %10, 8;\n\tsetp.ne.b32 p3, t3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, p2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, p3;\n\t"
+      "}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc),
+      "r"(acc_mask)
+      : "memory");
+}
+__device__ __forceinline__ void umma4_ss_pair(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                              uint32_t idesc, uint32_t acc_mask) {
+  asm volatile(
+      "{\n\t.reg .pred p<4>;\n\t.reg .b32 t<4>;\n\t"
+      "and.b32 t0, %10, 1;\n\tsetp.ne.b32 p0, t0, 0;\n\t"
+      "and.b32 t1, %10, 2;\n\tsetp.ne.b32 p1, t1, 0;\n\t"
+      "and.b32 t2, %10, 4;\n\tsetp.ne.b32 p2, t2, 0;\n\t"
+      "and.b32 t3, %10, 8;\n\tsetp.ne.b32 p3, t3, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %5, %9, p0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %2, %6, %9, p1;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %3, %7, %9, p2;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %4, %8, %9, p3;\n\t"
+      "}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc),
+      "r"(acc_mask)
+      : "memory");
+}
+// the same with A (bf16 pairs) read from tensor memory
+__device__ __forceinline__ void umma8_ts(const uint32_t (&d)[8], const uint32_t (&a)[8], const uint64_t (&b)[8],
+                                         uint32_t idesc, uint32_t acc_mask) {
+  asm volatile(
+      "{\n\t.reg .pred p<8>;\n\t.reg .b32 t<8>;\n\t"
+      "and.b32 t0, %25, 1;\n\tsetp.ne.b32 p0, t0, 0;\n\t"
+      "and.b32 t1, %25, 2;\n\tsetp.ne.b32 p1, t1, 0;\n\t"
+      "and.b32 t2, %25, 4;\n\tsetp.ne.b32 p2, t2, 0;\n\t"
+      "and.b32 t3, %25, 8;\n\tsetp.ne.b32 p3, t3, 0;\n\t"
+      "and.b32 t4, %25, 16;\n\tsetp.ne.b32 p4, t4, 0;\n\t"
+      "and.b32 t5, %25, 32;\n\tsetp.ne.b32 p5, t5, 0;\n\t"
+      "and.b32 t6, %25, 64;\n\tsetp.ne.b32 p6, t6, 0;\n\t"
+      "and.b32 t7, %25, 128;\n\tsetp.ne.b32 p7, t7, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%8], %16, %24, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%9], %17, %24, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%2], [%10], %18, %24, p2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%3], [%11], %19, %24, p3;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%4], [%12], %20, %24, p4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%5], [%13], %21, %24, p5;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%6], [%14], %22, %24, p6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%7], [%15], %23, %24, p7;\n\t"
+      "}"
+      ::"r"(d[0]), "r"(d[1]), "r"(d[2]), "r"(d[3]), "r"(d[4]), "r"(d[5]), "r"(d[6]), "r"(d[7]),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+      "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]), "l"(b[6]), "l"(b[7]), "r"(idesc),
+      "r"(acc_mask)
+      : "memory");
+}
+
 // Pair form: D (M = 256 rows split over the two CTAs) (+)= A * B^T, issued by one thread of the
 // even CTA; the descriptors address both CTAs' shared memory at the same offsets.
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
