@@ -183,6 +183,10 @@ static int dispatch_epi(int epi, const GemmMaps& maps, const GemmParams& p, cuda
     case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false, PAIR>(maps, p, st);
     case EPI_F32: return launch_gemm_t<BN, EPI_F32, false, PAIR>(maps, p, st);
     case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false, PAIR>(maps, p, st);
+    case EPI_QKV:
+      if (BN != 256 || !p.tma_out || p.qk_D % 256 != 0)
+        return set_error(ST_UNSUPPORTED, "fused RoPE/QK-norm epilogue needs 256-column tiles over whole heads");
+      return launch_gemm_t<BN, EPI_QKV, false, PAIR>(maps, p, st);
     case EPI_UP: return launch_gemm_t<BN, EPI_UP, false, PAIR>(maps, p, st);
     case EPI_ACTBWD: return launch_gemm_t<BN, EPI_ACTBWD, false, PAIR>(maps, p, st);
     case EPI_CE_FWD: return launch_gemm_t<BN, EPI_CE_FWD, false, PAIR>(maps, p, st);

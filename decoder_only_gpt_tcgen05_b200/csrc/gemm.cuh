@@ -39,6 +39,7 @@ enum EpiKind : int {
   EPI_BF16 = 0,     // out bf16 = acc (+ bias); optional head-padded column map (generic path)
   EPI_F32 = 1,      // out fp32 = acc (+ bias)  or  out += acc  (accumulate)
   EPI_RESID = 2,    // out fp32 = resid + acc (+ bias)
+  EPI_QKV = 3,      // out bf16 = acc, with RoPE + per-head RMSNorm applied to the q and k heads
   EPI_UP = 4,       // u = acc (+ bias) -> h = act(u) bf16 (out2), and u bf16 (out) unless out is null
   EPI_ACTBWD = 5,   // out bf16 = acc * act'(u); aux is u, or h = relu(u)^2 when act is ReLU^2
   EPI_CE_FWD = 6,   // per-row (max, sum exp) partials over this tile's vocab columns + target logit
@@ -71,6 +72,16 @@ struct GemmParams {
   float* ce_zy;               // [M] target logit
   const float* ce_lse;        // [M] natural-log logsumexp (backward)
   float ce_scale;             // 1/M_total (backward)
+  // EPI_QKV (128-wide heads, 256-column tiles: one head per epilogue warp): columns [0, qk_D)
+  // are q and [qk_D, 2 qk_D) are k; each head row gets r = rsqrt(mean(x^2) + qk_eps) (when
+  // qk_norm; RoPE keeps the row norm, so the accumulator gives it) and the rotation of the pairs
+  // (i, i + 64) by rope_cs[t][i] (when qk_rope), t = row % rope_T; r goes to rstd_q / rstd_k
+  // [rows][qk_H].  Columns from 2 qk_D on (v) are stored as they are.
+  const float2* rope_cs;
+  int rope_T, qk_D, qk_H, qk_rope, qk_norm;
+  float qk_eps;
+  float* rstd_q;
+  float* rstd_k;
   int prof_kind;              // host only: profiler family of this call (0 = generic GEMM)
   // grouped launch: up to kMaxProblems products with the same K, operand layouts and epilogue
   // share one persistent tile space; problem q owns tiles [tile_start[q], tile_start[q+1]).
@@ -151,6 +162,13 @@ __device__ __forceinline__ void stage_f32(uint32_t buf, int r, const float* v) {
   for (int u = 0; u < 8; ++u)
     sts128(stg_addr(buf, r, u), __float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
            __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3]));
+}
+// units u0 .. u0+3 (32 bf16 columns) of row r of a staging buffer <- 32 values
+__device__ __forceinline__ void stage_bf16_half(uint32_t buf, int r, int u0, const float* v) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    sts128(stg_addr(buf, r, u0 + u), pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+           pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
 }
 // row r of a staging buffer <- 64 bf16 values
 __device__ __forceinline__ void stage_bf16(uint32_t buf, int r, const float* v) {
@@ -572,6 +590,57 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
           }
           if (row_ok) p.ce_part[(long long)row * p.tiles_n + tn] = make_float2(m2, s);
         }
+      } else if (EPI == EPI_QKV && tma && n0 + c_begin < 2 * p.qk_D) {
+        // one q or k head (128 columns) per warp: RMS of the row, then RoPE and the scale, both
+        // halves of the head staged (buffer 0: columns 0-63, buffer 1: 64-127) and stored
+        const int g0 = n0 + c_begin;
+        const int part = g0 >= p.qk_D;
+        const int hh = (g0 - part * p.qk_D) >> 7;
+        float r = 1.f;
+        if (p.qk_norm) {
+          float ss = 0.f;
+#pragma unroll 1
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float v[32];
+            tmem_ld32(trow + c_begin + 32 * q4, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+          }
+          r = rsqrtf(ss * (1.f / 128.f) + p.qk_eps);
+          if (row_ok) (part ? p.rstd_k : p.rstd_q)[(long long)row * p.qk_H + hh] = r;
+        }
+        if (lane == 0) bulk_wait_read<0>();  // both staging buffers free
+        __syncwarp();
+        const float4* csr = reinterpret_cast<const float4*>(p.rope_cs + (long long)(row_ok ? row % p.rope_T : 0) * 64);
+#pragma unroll 1
+        for (int rr = 0; rr < 2; ++rr) {
+          float x1[32], x2[32];
+          tmem_ld32(trow + c_begin + 32 * rr, x1);
+          tmem_ld32(trow + c_begin + 64 + 32 * rr, x2);
+#pragma unroll
+          for (int j2 = 0; j2 < 16; ++j2) {
+            const float4 e = p.qk_rope ? __ldg(csr + 16 * rr + j2) : make_float4(1.f, 0.f, 1.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int j = 2 * j2 + k;
+              const float c = k ? e.z : e.x, sn = k ? e.w : e.y;
+              const float a = x1[j], b = x2[j];
+              x1[j] = (a * c - b * sn) * r;
+              x2[j] = (a * sn + b * c) * r;
+            }
+          }
+          stage_bf16_half(stg, lane, 4 * rr, x1);
+          stage_bf16_half(stg + 4096, lane, 4 * rr, x2);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {  // one bulk group per buffer, so a later chunk waits only for its own
+          tma_store_2d(tmC, stg_ptr, g0, row0);
+          bulk_commit();
+          tma_store_2d(tmC, stg_ptr + 4096, g0 + 64, row0);
+          bulk_commit();
+        }
+        chunk_ctr += 2;
       } else if (!tma) {
         for (int c = c_begin; c < c_begin + HALF; c += 32) {
           float v[32];

@@ -267,19 +267,34 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
     GPTK_TRY(launch_norm_fwd(x_in, M, D, ln ? params + o.ln1_g : nullptr, o.ln1_b >= 0 ? params + o.ln1_b : nullptr, ln,
                              c.norm_eps, a1, D, st1, st1 + M, st));
     {
-      // q|k|v = a1 W_qkv^T (+ b): straight into the attention layout when it is unpadded,
-      // then RoPE and QK-norm in place on q and k
+      // q|k|v = a1 W_qkv^T (+ b): straight into the attention layout when it is unpadded.
+      // With 128-wide heads and no bias, RoPE and QK-norm run in the GEMM epilogue on the fp32
+      // accumulator; otherwise they follow as an in-place pass on q and k.
       const bool padded = hdp != hd;
+      const bool fused = !padded && hd == 128 && D % 256 == 0 && o.b_qkv < 0 && (c.pos == 1 || c.qk_norm);
       __nv_bfloat16* raw = padded ? at<__nv_bfloat16>(ws, pl.dqkv) : qkv;
       GemmParams p = gp(M, 3 * D, D);
       p.out = raw;
       p.ldo = 3LL * D;
       p.bias = o.b_qkv >= 0 ? params + o.b_qkv : nullptr;
       p.prof_kind = PK_GEMM_QKV;
-      GPTK_TRY(gemm(EPI_BF16, Operand{a1, D, 0}, Operand{wbf + o.w_qkv, D, 0}, p, st));
-      if (padded) GPTK_CUDA(cudaMemsetAsync(qkv, 0, (size_t)M * 3 * H * hdp * 2, st));
-      if (padded || c.pos == 1 || c.qk_norm)
-        GPTK_TRY(launch_qk_fwd(raw, cs, M, T, H, hd, hdp, c.pos == 1, c.qk_norm, c.norm_eps, qkv, rq, rk, st));
+      if (fused) {
+        p.rope_cs = cs;
+        p.rope_T = T;
+        p.qk_D = D;
+        p.qk_H = H;
+        p.qk_rope = c.pos == 1;
+        p.qk_norm = c.qk_norm;
+        p.qk_eps = c.norm_eps;
+        p.rstd_q = rq;
+        p.rstd_k = rk;
+        GPTK_TRY(gemm(EPI_QKV, Operand{a1, D, 0}, Operand{wbf + o.w_qkv, D, 0}, p, st, 256));
+      } else {
+        GPTK_TRY(gemm(EPI_BF16, Operand{a1, D, 0}, Operand{wbf + o.w_qkv, D, 0}, p, st));
+        if (padded) GPTK_CUDA(cudaMemsetAsync(qkv, 0, (size_t)M * 3 * H * hdp * 2, st));
+        if (padded || c.pos == 1 || c.qk_norm)
+          GPTK_TRY(launch_qk_fwd(raw, cs, M, T, H, hd, hdp, c.pos == 1, c.qk_norm, c.norm_eps, qkv, rq, rk, st));
+      }
     }
     AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp};
     GPTK_TRY(launch_attn_fwd(qkv, as, ob, D, lse, st));
