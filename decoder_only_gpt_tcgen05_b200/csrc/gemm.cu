@@ -298,7 +298,7 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
 
 int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
                    cudaStream_t st) {
-  if (n < 1 || n > kMaxProblems) return set_error(ST_INVALID_ARG, "grouped GEMM: 1 to 4 problems");
+  if (n < 1 || n > kMaxProblems) return set_error(ST_INVALID_ARG, "grouped GEMM: 1 to 8 problems");
   if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));

@@ -86,11 +86,11 @@ struct GemmParams {
   // grouped launch: up to kMaxProblems products with the same K, operand layouts and epilogue
   // share one persistent tile space; problem q owns tiles [tile_start[q], tile_start[q+1]).
   int n_prob;
-  int tile_start[5];
-  int pM[4], pN[4], ptiles_m[4], ptiles_n[4], pgroup_m[4];
+  int tile_start[9];
+  int pM[8], pN[8], ptiles_m[8], ptiles_n[8], pgroup_m[8];
 };
 
-constexpr int kMaxProblems = 4;
+constexpr int kMaxProblems = 8;
 
 // Tensor maps of a launch: A and B (and the output C) per problem, plus the second output and
 // the epilogue input of single-problem launches.

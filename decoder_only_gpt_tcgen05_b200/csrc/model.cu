@@ -174,12 +174,14 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   p.dlog = take((size_t)p.Mc * p.Vp * 2);
   p.da = take(M * D * 4);
   p.dres = take(M * D * 4);
-  p.dres_bf = take(2 * M * D * 2);  // one per sublayer of a layer
-  p.du = take(M * F * 2);
+  // the scratch gradients the weight-gradient GEMMs read have two slots (layer parity): a pair of
+  // layers' weight gradients is launched together
+  p.dres_bf = take(4 * M * D * 2);  // [slot][sublayer]
+  p.du = take(2 * M * F * 2);
   p.do_pad = take(M * H * hdp * 2);
   p.delta = take(M * H * 4);
-  p.dqkv_pad = take(M * 3 * H * hdp * 2);
-  p.dqkv = take(M * 3 * D * 2);
+  p.dqkv_pad = take((p.hdp == p.hd ? 2 : 1) * M * 3 * H * hdp * 2);  // [slot] when it is dqkv itself
+  p.dqkv = take(2 * M * 3 * D * 2);
   long long maxN = F > 3 * D ? F : 3 * D;
   long long rows = norm_bwd_max_blocks() > colsum_max_chunks() ? norm_bwd_max_blocks() : colsum_max_chunks();
   p.partN = maxN;
@@ -404,13 +406,21 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
   float* pa = at<float>(ws, pl.part_a);
   float* pb = at<float>(ws, pl.part_b);
   __nv_bfloat16* dlog = at<__nv_bfloat16>(ws, pl.dlog);
-  // bf16 copies of the residual gradient: one for each sublayer of a layer, because the
-  // layer's weight gradients (launched together at the end of the layer) read both
-  __nv_bfloat16* dres_bf_mlp = at<__nv_bfloat16>(ws, pl.dres_bf);
-  __nv_bfloat16* dres_bf_att = at<__nv_bfloat16>(ws, pl.dres_bf) + MD;
-  __nv_bfloat16* du = at<__nv_bfloat16>(ws, pl.du);
-  __nv_bfloat16* dqkv_pad = at<__nv_bfloat16>(ws, pl.dqkv_pad);
-  __nv_bfloat16* dqkv = hdp == hd ? dqkv_pad : at<__nv_bfloat16>(ws, pl.dqkv);
+  // Scratch gradients read by the weight-gradient GEMMs, in two slots by layer parity: the
+  // weight gradients of an odd layer wait and run in one grouped launch with those of the even
+  // layer below it (eight products: better-filled waves than four), so an odd layer's bf16
+  // residual gradients (one per sublayer), du and dqkv must outlive the next layer's backward.
+  auto dres_bf_mlp_of = [&](int l) { return at<__nv_bfloat16>(ws, pl.dres_bf) + (size_t)(2 * (l & 1)) * MD; };
+  auto dres_bf_att_of = [&](int l) { return at<__nv_bfloat16>(ws, pl.dres_bf) + (size_t)(2 * (l & 1) + 1) * MD; };
+  auto du_of = [&](int l) { return at<__nv_bfloat16>(ws, pl.du) + (size_t)(l & 1) * M * F; };
+  auto dqkv_pad_of = [&](int l) {
+    return at<__nv_bfloat16>(ws, pl.dqkv_pad) + (hdp == hd ? (size_t)(l & 1) * M * 3 * H * hdp : 0);
+  };
+  auto dqkv_of = [&](int l) {
+    return hdp == hd ? dqkv_pad_of(l) : at<__nv_bfloat16>(ws, pl.dqkv) + (size_t)(l & 1) * M * 3 * D;
+  };
+  GroupProblem pending[4];  // an odd layer's weight-gradient products, waiting for the next layer
+  int n_pending = 0;
 
   if (!accumulate) GPTK_CUDA(cudaMemsetAsync(grads, 0, (size_t)pl.P * 4, st));
 
@@ -445,10 +455,15 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
     }
   }
   GPTK_TRY(norm_backward(c, pl, da, xs + (size_t)(2 * pl.L) * MD, stf, params, Lo.lnf_g, Lo.lnf_b, grads, dres, 1,
-                         dres_bf_mlp, pa, pb, st));
+                         dres_bf_mlp_of(pl.L - 1), pa, pb, st));
 
   for (int l = pl.L - 1; l >= 0; --l) {
     const LayerOff& o = Lo.layer[l];
+    __nv_bfloat16* dres_bf_mlp = dres_bf_mlp_of(l);
+    __nv_bfloat16* dres_bf_att = dres_bf_att_of(l);
+    __nv_bfloat16* du = du_of(l);
+    __nv_bfloat16* dqkv_pad = dqkv_pad_of(l);
+    __nv_bfloat16* dqkv = dqkv_of(l);
     const float* x_in = xs + (size_t)(2 * l) * MD;
     const float* x_mid = xs + (size_t)(2 * l + 1) * MD;
     const __nv_bfloat16* a1 = at<__nv_bfloat16>(ws, pl.a1) + (size_t)l * MD;
@@ -509,17 +524,28 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       GPTK_TRY(gemm(EPI_F32, Operand{dqkv, 3LL * D, 0}, Operand{wbf + o.w_qkv, D, 1}, p, st));
     }
     if (o.b_qkv >= 0) GPTK_TRY(bias_grad_bf16(dqkv, M, 3 * D, pa, grads + o.b_qkv, st));
-    {  // the layer's four weight gradients in one launch: W += dY^T X over all tokens
+    {  // the layer's four weight gradients W += dY^T X over all tokens, launched together with the
+       // pending four of the layer above (odd layers wait for the even one below them)
       const GroupProblem probs[4] = {
           {dres_bf_mlp, D, h, F, D, F, grads + o.w_down, F},
           {du, F, a2, D, F, D, grads + o.w_up, D},
           {dres_bf_att, D, ob, D, D, D, grads + o.w_o, D},
           {dqkv, 3LL * D, a1, D, 3 * D, D, grads + o.w_qkv, D},
       };
-      GPTK_TRY(run_gemm_group(4, probs, M, 1, 1, 256, PK_GEMM_WGRAD, st));
+      if ((l & 1) && l > 0) {
+        for (int q = 0; q < 4; ++q) pending[q] = probs[q];
+        n_pending = 4;
+      } else {
+        GroupProblem all[8];
+        for (int q = 0; q < n_pending; ++q) all[q] = pending[q];
+        for (int q = 0; q < 4; ++q) all[n_pending + q] = probs[q];
+        GPTK_TRY(run_gemm_group(n_pending + 4, all, M, 1, 1, 256, PK_GEMM_WGRAD, st));
+        n_pending = 0;
+      }
     }
-    GPTK_TRY(norm_backward(c, pl, da, x_in, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0, dres_bf_mlp, pa, pb,
-                           st));
+    // the residual gradient of the layer below goes to that layer's slot
+    GPTK_TRY(norm_backward(c, pl, da, x_in, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0,
+                           l > 0 ? dres_bf_mlp_of(l - 1) : dres_bf_mlp_of(0), pa, pb, st));
   }
   // ---- embeddings
   GPTK_TRY(launch_embed_bwd(idx_ws, dres, M, D, V, grads + Lo.wte, at<void>(ws, pl.embed), st));
