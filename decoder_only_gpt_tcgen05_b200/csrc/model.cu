@@ -137,7 +137,16 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   p.V = c.vocab_size;
   p.Vp = (c.vocab_size + 7) / 8 * 8;
   p.ntn = (c.vocab_size + 255) / 256;
-  p.Mc = p.M < 4096 ? p.M : 4096;
+  // lm_head backward row chunk: every row at once when their bf16 dlogits fit in 4 GiB (then the
+  // three lm_head products fill their waves: with 4096-row chunks the logits-gradient product
+  // d af = dlogits W_lm had 80 tiles of 256 x 256 for 74 CTA pairs), else the largest multiple
+  // of 4096 rows that fits
+  {
+    const long long cap = (4LL << 30) / ((long long)p.Vp * 2);
+    long long mc = cap / 4096 * 4096;
+    if (mc < 4096) mc = 4096;
+    p.Mc = (int)(mc < p.M ? mc : p.M);
+  }
   p.P = P;
   const size_t M = p.M, D = p.D, F = p.F, L = p.L, H = p.H, hdp = p.hdp;
   size_t off = 0;
