@@ -651,6 +651,97 @@ int launch_qk_fwd(const __nv_bfloat16* qkv, const float2* rope_cs, int M, int T,
   return ST_OK;
 }
 
+// In-place QK-norm / RoPE backward for 64- or 128-wide unpadded heads: HD / 8 lanes per
+// (token, head) item, each lane four consecutive pairs (i .. i+3 with i + HD/2 ..), 8-byte loads
+// and stores, a segmented shuffle reduction; v is left as it is.
+template <int HD>
+__global__ void qk_bwd_vec_kernel(__nv_bfloat16* __restrict__ dqkv, const __nv_bfloat16* __restrict__ qpad,
+                                  const float* __restrict__ rq, const float* __restrict__ rk,
+                                  const float2* __restrict__ cs, int M, int T, int H, int rope, int qk_norm) {
+  constexpr int HALF = HD / 2;
+  constexpr int LPI = HD / 8;
+  constexpr int IPW = 32 / LPI;
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPI, l8 = lane % LPI;
+  const int i = 4 * l8;
+  const long long total = (long long)M * H;
+  const long long ps = (long long)H * HD;  // q -> k section pitch
+  for (long long base = ((long long)blockIdx.x * warps + (threadIdx.x >> 5)) * IPW; base < total;
+       base += (long long)gridDim.x * warps * IPW) {
+    const long long w = base + sub;
+    const bool live = w < total;
+    const long long m = live ? w / H : 0;
+    const int h = live ? (int)(w - m * H) : 0;
+    const long long po = m * 3 * ps + (long long)h * HD;
+    float a[2][4], b[2][4], ya[2][4], yb[2][4];
+    auto ld4 = [&](const __nv_bfloat16* p, float* v) {
+      const uint2 x = live ? __ldg(reinterpret_cast<const uint2*>(p)) : make_uint2(0u, 0u);
+      v[0] = __uint_as_float(x.x << 16);
+      v[1] = __uint_as_float(x.x & 0xffff0000u);
+      v[2] = __uint_as_float(x.y << 16);
+      v[3] = __uint_as_float(x.y & 0xffff0000u);
+    };
+#pragma unroll
+    for (int sct = 0; sct < 2; ++sct) {
+      ld4(dqkv + po + sct * ps + i, a[sct]);
+      ld4(dqkv + po + sct * ps + HALF + i, b[sct]);
+      if (qk_norm) {
+        ld4(qpad + po + sct * ps + i, ya[sct]);
+        ld4(qpad + po + sct * ps + HALF + i, yb[sct]);
+      }
+    }
+    float2 e[4];
+    if (rope && live) {
+      const float4* c4 = reinterpret_cast<const float4*>(cs + (long long)(m % T) * HALF + i);
+      const float4 c0 = __ldg(c4), c1 = __ldg(c4 + 1);
+      e[0] = make_float2(c0.x, c0.y);
+      e[1] = make_float2(c0.z, c0.w);
+      e[2] = make_float2(c1.x, c1.y);
+      e[3] = make_float2(c1.z, c1.w);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) e[k] = make_float2(1.f, 0.f);
+    }
+    const float r2[2] = {(qk_norm && live) ? rq[m * H + h] : 1.f, (qk_norm && live) ? rk[m * H + h] : 1.f};
+#pragma unroll
+    for (int sct = 0; sct < 2; ++sct) {
+      if (qk_norm) {
+        // dx = r (dy - y mean(dy y)), y the normalised output that the forward saved
+        float sm = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sm += a[sct][k] * ya[sct][k] + b[sct][k] * yb[sct][k];
+#pragma unroll
+        for (int off = LPI / 2; off > 0; off >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, off);
+        const float mdy = sm * (1.f / HD);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          a[sct][k] = r2[sct] * (a[sct][k] - ya[sct][k] * mdy);
+          b[sct][k] = r2[sct] * (b[sct][k] - yb[sct][k] * mdy);
+        }
+      }
+      // the rotation is orthogonal: its reverse rotates by -phi
+      uint32_t wa[2], wb[2];
+#pragma unroll
+      for (int k2 = 0; k2 < 2; ++k2) {
+        float oa[2], ob[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int k = 2 * k2 + q;
+          oa[q] = a[sct][k] * e[k].x + b[sct][k] * e[k].y;
+          ob[q] = -a[sct][k] * e[k].y + b[sct][k] * e[k].x;
+        }
+        wa[k2] = pack_bf16x2(oa[0], oa[1]);
+        wb[k2] = pack_bf16x2(ob[0], ob[1]);
+      }
+      if (live) {
+        *reinterpret_cast<uint2*>(dqkv + po + sct * ps + i) = make_uint2(wa[0], wa[1]);
+        *reinterpret_cast<uint2*>(dqkv + po + sct * ps + HALF + i) = make_uint2(wb[0], wb[1]);
+      }
+    }
+  }
+}
+
 int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, const float* rstd_q,
                   const float* rstd_k, const float2* rope_cs, int M, int T, int H, int hd, int hdp, int rope,
                   int qk_norm, __nv_bfloat16* dqkv, cudaStream_t st) {
@@ -658,6 +749,19 @@ int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, c
   if ((const void*)dqkv_pad == (const void*)dqkv && hdp != hd)
     return set_error(ST_INVALID_ARG, "qk_bwd: in place needs an unpadded layout");
   long long work = (long long)M * H;
+  if ((hd == 64 || hd == 128) && hdp == hd && (const void*)dqkv_pad == (const void*)dqkv) {
+    // in place, unpadded: the vectorised form (v needs nothing)
+    const int ipb = 8 * (32 / (hd / 8));  // items per 256-thread block and pass
+    long long grid = (work + ipb - 1) / ipb;
+    if (grid > (long long)num_sms() * 32) grid = num_sms() * 32;
+    Prof prof(PK_QK, 0, (double)M * 2 * H * hd * 4 + (qk_norm ? (double)M * 2 * H * hd * 2 : 0), st);
+    if (hd == 128)
+      qk_bwd_vec_kernel<128><<<(int)grid, 256, 0, st>>>(dqkv, qkv_pad, rstd_q, rstd_k, rope_cs, M, T, H, rope, qk_norm);
+    else
+      qk_bwd_vec_kernel<64><<<(int)grid, 256, 0, st>>>(dqkv, qkv_pad, rstd_q, rstd_k, rope_cs, M, T, H, rope, qk_norm);
+    GPTK_CUDA(cudaGetLastError());
+    return ST_OK;
+  }
   int grid = cdiv(work, 8);
   if (grid > num_sms() * 32) grid = num_sms() * 32;
   Prof prof(PK_QK, 0, (double)M * 3 * H * hd * 4 + (qk_norm ? (double)M * 2 * H * hd * 2 : 0), st);
@@ -675,8 +779,47 @@ int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, c
 
 // ------------------------------------------------------------------ attention delta
 
+// delta[b, h, t] = sum_d o[m, h hd + d] * dO[m, h hdp + d]: hd / 8 lanes per (token, head) item,
+// 16-byte loads, a segmented shuffle reduction; 32 / (hd / 8) items per warp and pass.
+template <int HD>
 __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dpad, int B,
-                                  int T, int H, int hd, int hdp, float* __restrict__ delta) {
+                                  int T, int H, int hdp, float* __restrict__ delta) {
+  constexpr int LPI = HD / 8;  // lanes per item
+  constexpr int IPW = 32 / LPI;
+  const int warps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPI, l8 = lane % LPI;
+  const long long total = (long long)B * T * H;
+  for (long long base = ((long long)blockIdx.x * warps + (threadIdx.x >> 5)) * IPW; base < total;
+       base += (long long)gridDim.x * warps * IPW) {
+    const long long w = base + sub;
+    float s = 0.f;
+    if (w < total) {
+      const long long m = w / H;
+      const int h = (int)(w - m * H);
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + m * H * HD + (long long)h * HD) + l8);
+      const uint4 d = __ldg(reinterpret_cast<const uint4*>(dpad + m * H * hdp + (long long)h * hdp) + l8);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, dv[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        s = fmaf(__uint_as_float(av[k] << 16), __uint_as_float(dv[k] << 16), s);
+        s = fmaf(__uint_as_float(av[k] & 0xffff0000u), __uint_as_float(dv[k] & 0xffff0000u), s);
+      }
+    }
+#pragma unroll
+    for (int off = LPI / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (l8 == 0 && w < total) {
+      const long long m = w / H;
+      const int h = (int)(w - m * H);
+      const long long b = m / T, t = m % T;
+      delta[(b * H + h) * T + t] = s;
+    }
+  }
+}
+
+// any even head dim: one warp per (token, head)
+__global__ void attn_delta_generic_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dpad,
+                                          int B, int T, int H, int hd, int hdp, float* __restrict__ delta) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total = B * T * H;
@@ -697,11 +840,22 @@ __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __n
 
 int launch_attn_delta(const __nv_bfloat16* o, const __nv_bfloat16* do_pad, int B, int T, int H, int hd, int hdp,
                       float* delta, cudaStream_t st) {
-  long long work = (long long)B * T * H;
-  int grid = cdiv(work, 8);
-  if (grid > num_sms() * 16) grid = num_sms() * 16;
+  if (hd != 64 && hd != 128) {
+    long long work = (long long)B * T * H;
+    int grid = cdiv(work, 8);
+    if (grid > num_sms() * 16) grid = num_sms() * 16;
+    Prof prof(PK_DELTA, 0, (double)B * T * H * (hd * 2 + hdp * 2 + 4), st);
+    attn_delta_generic_kernel<<<grid, 256, 0, st>>>(o, do_pad, B, T, H, hd, hdp, delta);
+    GPTK_CUDA(cudaGetLastError());
+    return ST_OK;
+  }
+  const long long items = (long long)B * T * H;
+  const int ipb = 8 * (hd == 128 ? 2 : 4);  // items per 256-thread block and pass
+  long long grid = (items + ipb - 1) / ipb;
+  if (grid > (long long)num_sms() * 16) grid = num_sms() * 16;
   Prof prof(PK_DELTA, 0, (double)B * T * H * (hd * 2 + hdp * 2 + 4), st);
-  attn_delta_kernel<<<grid, 256, 0, st>>>(o, do_pad, B, T, H, hd, hdp, delta);
+  if (hd == 128) attn_delta_kernel<128><<<(int)grid, 256, 0, st>>>(o, do_pad, B, T, H, hdp, delta);
+  else attn_delta_kernel<64><<<(int)grid, 256, 0, st>>>(o, do_pad, B, T, H, hdp, delta);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
