@@ -216,17 +216,6 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x 16, bf16, two per 32-bit column: element (m, k) at
-// lane m, column k/2) read from tensor memory, B from a shared-memory descriptor.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Eight MMAs issued back to back from one asm block, every operand in a register beforehand and
 // the eight enable-accumulate predicates set up front (bit i of acc_mask for MMA i).  The issue
 // of tcgen05.mma is synchronous with the tensor pipe, so any instruction between two MMAs
@@ -294,7 +283,8 @@ __device__ __forceinline__ void umma4_ss_pair(uint32_t d, const uint64_t (&a)[4]
       "r"(acc_mask)
       : "memory");
 }
-// the same with A (bf16 pairs) read from tensor memory
+// the same with A read from tensor memory: each A is an M x 16 bf16 block stored two per 32-bit
+// column (element (m, k) at lane m, column k / 2 from the given address)
 __device__ __forceinline__ void umma8_ts(const uint32_t (&d)[8], const uint32_t (&a)[8], const uint64_t (&b)[8],
                                          uint32_t idesc, uint32_t acc_mask) {
   asm volatile(
@@ -323,16 +313,6 @@ __device__ __forceinline__ void umma8_ts(const uint32_t (&d)[8], const uint32_t 
       : "memory");
 }
 
-// Pair form: D (M = 256 rows split over the two CTAs) (+)= A * B^T, issued by one thread of the
-// even CTA; the descriptors address both CTAs' shared memory at the same offsets.
-__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                               uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 // Arrive once on the mbarrier at `bar_cluster` (either CTA of the pair) when every pair MMA
 // issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
