@@ -14,6 +14,7 @@
 // the data-gradient epilogue, the flash-attention backward, the QK-norm/RoPE
 // reverse, the norm backward with the residual add, and finally the deterministic
 // embedding scatter.
+#include <cstdlib>
 #include <cmath>
 #include <cstring>
 #include <string>
@@ -145,6 +146,12 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
     const long long cap = (4LL << 30) / ((long long)p.Vp * 2);
     long long mc = cap / 4096 * 4096;
     if (mc < 4096) mc = 4096;
+    // GPT_LM_CHUNK_ROWS=<n> forces n-row blocks (tests of the blocked path on small batches)
+    static const long long forced = []() {
+      const char* e = std::getenv("GPT_LM_CHUNK_ROWS");
+      return e ? std::atoll(e) : 0LL;
+    }();
+    if (forced > 0) mc = forced;
     p.Mc = (int)(mc < p.M ? mc : p.M);
   }
   p.P = P;
