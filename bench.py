@@ -41,6 +41,33 @@ WORKLOADS = {
 }
 
 
+def metric_name(preset_name: str) -> str:
+    return METRIC if preset_name == "d20" else METRIC.replace("d20", preset_name)
+
+
+def matmul_params(cfg) -> int:
+    """Parameters that take part in a matmul for every token: the block matrices (q, k, v, output
+    projection, MLP up and down with width 4D) and the lm_head; embedding lookups are gathers."""
+    D = cfg.n_embd
+    return cfg.n_layer * (4 * D * D + 2 * D * 4 * D) + cfg.vocab_size * D
+
+
+def step_flops(cfg, B: int, T: int, causal: bool = True) -> float:
+    """Forward + backward FLOPs of one step: 6 per matmul parameter per token plus attention
+    ("Train your own ChatGPT", gpt.py estimate_flops: 6 FLOPs per parameter per token plus
+    attention terms).  causal=True counts only the unmasked half of the score matrix
+    (6 L D T per token), causal=False the full 12 L D T."""
+    att = (6 if causal else 12) * cfg.n_layer * cfg.n_embd * T
+    return float(B * T) * (6.0 * matmul_params(cfg) + att)
+
+
+def attention_flops(B: int, T: int, H: int, hd: int):
+    """Algorithmic FLOPs of causal attention: the forward's two products (q k^T and P v) over the
+    unmasked half of the T x T scores, 2 B H T^2 hd; the backward's four (dP, dV, dQ, dK) twice that."""
+    fwd = 2.0 * B * H * T * T * hd
+    return fwd, 2.0 * fwd
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -169,7 +196,7 @@ def run_reference(args, rank, world):
     ms = 1000.0 * sum(times) / len(times)
     value = T / (ms / 1000.0)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "impl": "reference", "metric": metric_name(preset_name), "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": desc, "sample": f"1 sequence x {T} tokens per step", "parallelism": "cpu"},
@@ -182,13 +209,110 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------- our arm
 
+# ---------------------------------------------------------------- attention alone
+
+ATTN_SWEEP_T = (512, 1024, 2048, 4096, 8192)
+
+
+def run_attn_sweep(args):
+    """RoPE + QK-norm + causal attention forward and backward through the op-level calls,
+    H = 10 heads of 128 (the d20 layer), B = 32768 / T sequences for each T of the sweep.
+    Inputs: raw q|k|v N(0, 1) (seed 3) and dL/do N(0, 1) (seed 4), bf16; the same 32768-token
+    arrays serve every T.  Each call is timed with CUDA events over `steps` back-to-back calls;
+    a second pass under the library's per-launch profiler splits out the attention kernels."""
+    import torch
+    import decoder_only_gpt_tcgen05_b200 as g
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])   # kernels timed alone: burst peak
+    H, hd, tokens = 10, 128, 32768
+    qkv = torch.from_numpy(synth.normal((tokens, 3 * H * hd), 3)).to(dev).to(torch.bfloat16)
+    dout = torch.from_numpy(synth.normal((tokens, H * hd), 4)).to(dev).to(torch.bfloat16)
+    dqkv = torch.empty_like(qkv)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, k):
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / k
+
+    rows = []
+    n0 = g.ops.launch_count()
+    n_calls = 0
+    with ClockSampler(0) as clk:
+        for T in ATTN_SWEEP_T:
+            B = tokens // T
+            fwd = g.ops.attention_fwd(qkv, B, T, H, hd)
+            delta = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+
+            def f():
+                g.ops.attention_fwd(qkv, B, T, H, hd, out=fwd)
+
+            def bwd():
+                g.ops.attention_bwd(fwd, dout, B, T, H, hd, delta=delta, dqkv=dqkv)
+            for _ in range(args.warmup):
+                f()
+                bwd()
+            ms_f = timed(f, args.steps)
+            ms_b = timed(bwd, args.steps)
+            n_calls += 2 * (args.warmup + args.steps)
+            g.ops.profile_start()
+            for _ in range(args.steps):
+                f()
+                bwd()
+            torch.cuda.synchronize(dev)
+            prof = g.ops.profile_stop()
+            n_calls += 2 * args.steps
+            fl_f, fl_b = attention_flops(B, T, H, hd)
+            k_f = prof["attn_fwd"][0] / args.steps
+            k_b = (prof["attn_bwd_dkv"][0] + prof["attn_bwd_dq"][0]) / args.steps
+            rows.append({
+                "T": T, "B": B, "fwd_ms": ms_f, "bwd_ms": ms_b,
+                "fwd_tflops": fl_f / ms_f / 1e9, "bwd_tflops": fl_b / ms_b / 1e9,
+                "fwd_bwd_tflops": (fl_f + fl_b) / (ms_f + ms_b) / 1e9,
+                "kernel_ms": {k: prof[k][0] / args.steps for k in ("attn_fwd", "attn_bwd_dkv", "attn_bwd_dq", "qk",
+                                                                    "delta", "misc")},
+                "kernel_fwd_tflops": fl_f / k_f / 1e9 if k_f > 0 else None,
+                "kernel_bwd_tflops": fl_b / k_b / 1e9 if k_b > 0 else None,
+            })
+            g.model.sync_status(dev)
+    launches = (g.ops.launch_count() - n0) / max(1, n_calls // 2)   # per forward + backward pair
+    head = next(r for r in rows if r["T"] == 2048)
+    kms = head["kernel_ms"]["attn_fwd"] + head["kernel_ms"]["attn_bwd_dkv"] + head["kernel_ms"]["attn_bwd_dq"]
+    ach = sum(attention_flops(head["B"], 2048, H, hd)) / kms / 1e9 if kms > 0 else None
+    line = {
+        "metric": "causal attention fwd+bwd TFLOP/s (algorithmic), RoPE + QK-norm, 10 heads x 128, 32768 tokens, T=2048",
+        "value": head["fwd_bwd_tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["fwd_ms"] + head["bwd_ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "attention sweep: H=10, hd=128, B*T=32768, T in " + ",".join(map(str, ATTN_SWEEP_T)),
+                   "l2": "q|k|v, o and dq|dk|dv 250 MB each, above the 126 MB L2; no flush"},
+        "roofline": {"kernel": "attn_fwd + attn_bwd_dkv + attn_bwd_dq at T=2048", "bound": "tensor", "achieved": ach,
+                     "peak": peak, "unit": "TFLOP/s", "frac": ach / peak if ach else None, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "sweep": rows,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default="d20")
+    ap.add_argument("--workload", choices=list(WORKLOADS) + ["attn_sweep"], default="d20",
+                    help="attn_sweep: the attention kernels alone over T = 512..8192 at 32768 tokens")
     ap.add_argument("--profile-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="also print the per-kernel-family table to stderr")
@@ -202,6 +326,11 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.workload == "attn_sweep":
+        if args.impl != "ours" or world != 1:
+            ap.error("attn_sweep times this library's attention kernels on one GPU")
+        run_attn_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
@@ -209,7 +338,6 @@ def main():
     import torch
     import torch.distributed as dist
     import decoder_only_gpt_tcgen05_b200 as g
-    import oracle  # noqa: F401  (FLOP accounting of the workload: the cpu_baseline leg)
     import synth
 
     torch.cuda.set_device(local)
@@ -314,13 +442,11 @@ def main():
             dist.destroy_process_group()
         return
 
-    import oracle as O
-    ocfg = O.preset(preset_name)
-    step_flops = O.step_flops(ocfg, B, T)            # per GPU, causal attention count
-    step_flops_nc = O.step_flops(ocfg, B, T, causal=False)
+    flops = step_flops(cfg, B, T)                    # per GPU, causal attention count
+    flops_nc = step_flops(cfg, B, T, causal=False)
     tokens = B * T * world
     value = tokens / (ms / 1000.0)
-    tflops = step_flops / (ms / 1000.0) / 1e12       # per GPU
+    tflops = flops / (ms / 1000.0) / 1e12            # per GPU
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     total_prof_ms = sum(v[0] for v in prof.values()) or 1.0
     # the dominant kernel: the GEMM kernel (all its roles) when it leads, else the leading family
@@ -350,7 +476,8 @@ def main():
         try:
             import hashlib
             t = json.load(open(traffic_file)).get(dom)
-            if t:
+            # counters taken on one workload and batch describe that launch mix only
+            if t and t.get("workload") == args.workload and t.get("batch") == B:
                 src = open(os.path.join(ROOT, t["source"]), "rb").read()
                 if hashlib.sha256(src).hexdigest() == t["source_sha256"]:
                     roof["traffic"] = t["bytes_per_launch"]
@@ -371,7 +498,7 @@ def main():
                   f"{(v['tflops'] or 0):8.1f} TF/s  {(v['gbs'] or 0):8.1f} GB/s", file=sys.stderr)
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": metric_name(preset_name), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": desc, "B": B, "T": T, "tokens_per_step": tokens,
@@ -380,7 +507,7 @@ def main():
         "mfu": {"tflops_per_gpu": tflops, "vs_measured_sustained": tflops / peak_sus,
                 "vs_measured_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
                 "vs_datasheet_2250": tflops / DATASHEET_BF16_TFLOPS,
-                "flops_per_step": step_flops, "flops_per_step_noncausal": step_flops_nc,
+                "flops_per_step": flops, "flops_per_step_noncausal": flops_nc,
                 "peak_source": peak_src},
         "eval": ({"metric": "val_bpb eval tokens/s", "value": tokens / (ms_eval / 1000.0), "ms_per_step": ms_eval}
                  if ms_eval else None),

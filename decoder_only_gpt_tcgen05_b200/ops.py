@@ -36,12 +36,14 @@ def _ptr(t):
 
 
 def attention_fwd(qkv: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: bool = True, qk_norm: bool = True,
-                  rope_base: float = 10000.0, eps: float = 1e-5):
+                  rope_base: float = 10000.0, eps: float = 1e-5, out: dict | None = None):
     """RoPE + QK-norm + causal attention.  qkv: bf16 [B*T, 3*H*hd] (raw).
-    Returns a dict with qkv_norm, rstd_q, rstd_k, rope_cs, o, lse."""
+    Returns a dict with qkv_norm, rstd_q, rstd_k, rope_cs, o, lse; ``out``, a
+    dict returned by an earlier call with the same sizes, is written again
+    instead of allocating."""
     dev = qkv.device
     M = B * T
-    r = {
+    r = out if out is not None else {
         "qkv_norm": torch.empty((M, 3 * H * hd), dtype=torch.bfloat16, device=dev),
         "rstd_q": torch.empty((M, H), dtype=torch.float32, device=dev) if qk_norm else None,
         "rstd_k": torch.empty((M, H), dtype=torch.float32, device=dev) if qk_norm else None,
@@ -49,6 +51,9 @@ def attention_fwd(qkv: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: b
         "o": torch.empty((M, H * hd), dtype=torch.bfloat16, device=dev),
         "lse": torch.empty((B, H, T), dtype=torch.float32, device=dev),
     }
+    assert r["qkv_norm"].numel() >= M * 3 * H * hd and r["o"].numel() >= M * H * hd and r["lse"].numel() >= M * H
+    assert not rope or r["rope_cs"].numel() >= T * hd
+    assert not qk_norm or (r["rstd_q"].numel() >= M * H and r["rstd_k"].numel() >= M * H)
     call("gpt_op_attention_fwd", qkv.data_ptr(), B, T, H, hd, int(rope), int(qk_norm), rope_base, eps,
          r["qkv_norm"].data_ptr(), _ptr(r["rstd_q"]), _ptr(r["rstd_k"]), _ptr(r["rope_cs"]), r["o"].data_ptr(),
          r["lse"].data_ptr(), _stream(qkv))
@@ -56,11 +61,17 @@ def attention_fwd(qkv: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: b
 
 
 def attention_bwd(fwd: dict, dout: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: bool = True,
-                  qk_norm: bool = True) -> torch.Tensor:
-    """dL/dqkv (bf16 [B*T, 3*H*hd]) from dout = dL/do (bf16 [B*T, H*hd])."""
+                  qk_norm: bool = True, delta: torch.Tensor | None = None,
+                  dqkv: torch.Tensor | None = None) -> torch.Tensor:
+    """dL/dqkv (bf16 [B*T, 3*H*hd]) from dout = dL/do (bf16 [B*T, H*hd]).
+    ``delta`` (fp32 [B, H, T] scratch) and ``dqkv`` may be passed in to avoid
+    allocating them."""
     dev = dout.device
-    delta = torch.empty((B, H, T), dtype=torch.float32, device=dev)
-    dqkv = torch.empty((B * T, 3 * H * hd), dtype=torch.bfloat16, device=dev)
+    if delta is None:
+        delta = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    if dqkv is None:
+        dqkv = torch.empty((B * T, 3 * H * hd), dtype=torch.bfloat16, device=dev)
+    assert delta.numel() >= B * H * T and dqkv.numel() >= B * T * 3 * H * hd
     call("gpt_op_attention_bwd", fwd["qkv_norm"].data_ptr(), _ptr(fwd["rstd_q"]), _ptr(fwd["rstd_k"]),
          _ptr(fwd["rope_cs"]), fwd["o"].data_ptr(), fwd["lse"].data_ptr(), dout.data_ptr(), B, T, H, hd, int(rope),
          int(qk_norm), delta.data_ptr(), dqkv.data_ptr(), _stream(dout))

@@ -102,3 +102,19 @@ def test_bad_arguments_are_rejected_on_the_host(pkg):
     assert L.gpt_op_gemm(0, 192, fake, 64, 0, fake, 64, 0, 8, 8, 8, fake, 8, None, 0, None) == 1
     assert L.gpt_op_attention_fwd(fake, 1, 16, 1, 32, 1, 1, C.c_float(1e4), C.c_float(1e-5), fake, fake, fake, fake,
                                   fake, fake, None) == 2
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+def test_bench_flop_accounting_matches_oracle(pkg, name):
+    """bench.py's MFU numerator is its own formula; it must agree with the oracle's pinned count."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    cfg, ocfg = pkg.preset(name), O.preset(name)
+    for B, T in ((16, 2048), (8, 1024), (1, 16)):
+        assert bench.step_flops(cfg, B, T) == O.step_flops(ocfg, B, T)
+        assert bench.step_flops(cfg, B, T, causal=False) == O.step_flops(ocfg, B, T, causal=False)
+    # attention alone: forward 2 B H T^2 hd, i.e. T x 83.9 MFLOP at 32768 tokens, 10 heads of 128
+    for T in (512, 2048, 8192):
+        f, b = bench.attention_flops(32768 // T, T, 10, 128)
+        assert f == T * 83_886_080 and b == 2 * f
