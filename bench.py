@@ -319,6 +319,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B (sequences per GPU), e.g. for profiling")
     ap.add_argument("--no-eval", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time replays of one step captured in a CUDA graph (one GPU)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -334,6 +336,8 @@ def main():
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
+    if args.graph and world != 1:
+        ap.error("--graph times one GPU (the step's all-reduce is not captured)")
 
     import torch
     import torch.distributed as dist
@@ -392,12 +396,30 @@ def main():
     for _ in range(args.warmup):
         step()
     g.model.sync_status(dev)
+    timed_step = step
+    graph_launches = None
+    if args.graph:
+        # one step captured once; each timed iteration replays it (kernel arguments, tensor maps
+        # and buffers are the eager step's, so the replay recomputes the same loss and gradients)
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        n_cap = g.ops.launch_count()
+        with torch.cuda.graph(graph):
+            step()
+        graph_launches = g.ops.launch_count() - n_cap
+        timed_step = graph.replay
+        for _ in range(args.warmup):
+            timed_step()
     n0 = g.ops.launch_count()
     with ClockSampler(local) as clk:
         torch.cuda.nvtx.range_push("timed")
-        ms = timed(step, args.steps)
+        ms = timed(timed_step, args.steps)
         torch.cuda.nvtx.range_pop()
-    launches = (g.ops.launch_count() - n0) // args.steps
+    launches = (g.ops.launch_count() - n0) // args.steps if graph_launches is None else graph_launches
     clocks = clk.summary()
     g.model.sync_status(dev)
 
@@ -503,6 +525,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": desc, "B": B, "T": T, "tokens_per_step": tokens,
                    "parallelism": f"dp{world}" if world > 1 else "single",
+                   "launch": "CUDA graph replay of one captured step" if args.graph else "eager stream launches",
                    "l2": "working set (~35 GB of weights and saved activations) far above the 126 MB L2; no flush"},
         "mfu": {"tflops_per_gpu": tflops, "vs_measured_sustained": tflops / peak_sus,
                 "vs_measured_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
