@@ -307,6 +307,43 @@ def test_dlogits_rows_sum_to_zero():
     assert np.allclose(O.unflatten(cfg, g)["lm_head"], dz.T @ f["cache"]["af"] / M, atol=1e-14)
 
 
+def test_embedding_gradient_rows_follow_the_inputs():
+    """x0[m] = wte[idx[m]] (+ wpe[t]): the embedding gradient scatters into the rows of the INPUT
+    ids and positions only.  Untied, the rows of ids absent from idx are exactly zero (ids that
+    occur only as targets included), and wpe rows at positions >= T are zero.  Tied, the absent
+    rows carry the lm_head part alone, which equals the untied model's lm_head gradient."""
+    B, T, V = 2, 6, 40
+    rng = np.random.default_rng(7)
+    idx = rng.integers(0, 10, size=(B, T)).astype(np.int32)        # inputs use ids 0..9 only
+    tgt = rng.integers(20, V, size=(B, T)).astype(np.int32)        # targets 20..39 only
+    absent = np.setdiff1d(np.arange(V), idx)
+    present = np.unique(idx)
+    grads = {}
+    for tie in (0, 1):
+        cfg = _cfg(vocab_size=V, tie_embed=tie, pos=O.POS_LEARNED, block_size=16)
+        p = _random_params(cfg, 43, std=0.3)
+        gr = O.unflatten(cfg, O.backward(cfg, p, O.forward(cfg, p, idx, tgt)))
+        grads[tie] = (cfg, p, gr)
+        assert not np.any(gr["wpe"][T:]) and np.all(np.abs(gr["wpe"][:T]).sum(-1) > 0)
+    cfg0, p0, g0 = grads[0]
+    assert not np.any(g0["wte"][absent])
+    assert np.all(np.abs(g0["wte"][present]).sum(-1) > 0)
+    # tied: same weights with lm_head := wte; the absent rows hold only the lm_head gradient
+    cfg1 = grads[1][0]
+    p1 = O.unflatten(cfg1, np.zeros(O.param_count(cfg1)))
+    for name, v in O.unflatten(cfg0, p0).items():
+        if name in p1:
+            p1[name][...] = v
+    pu = O.unflatten(cfg0, p0.copy())
+    pu["lm_head"][...] = pu["wte"]
+    flat_u = np.concatenate([pu[n].reshape(-1) for n, _ in O.param_shapes(cfg0)])
+    flat_t = np.concatenate([p1[n].reshape(-1) for n, _ in O.param_shapes(cfg1)])
+    gu = O.unflatten(cfg0, O.backward(cfg0, flat_u, O.forward(cfg0, flat_u, idx, tgt)))
+    gt = O.unflatten(cfg1, O.backward(cfg1, flat_t, O.forward(cfg1, flat_t, idx, tgt)))
+    assert np.allclose(gt["wte"][absent], gu["lm_head"][absent], rtol=0, atol=1e-15)
+    assert np.allclose(gt["wte"], gu["wte"] + gu["lm_head"], rtol=0, atol=1e-14)
+
+
 @pytest.mark.parametrize("name", list(SMALL_CONFIGS))
 def test_gradients_match_central_differences(name):
     """fp64 central differences, h = 1e-5 (about 1e-4 relative to the
