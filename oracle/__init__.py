@@ -6,3 +6,4 @@ by the benchmark's CPU-baseline leg, never by the library itself.
 from .gpt_oracle import *  # noqa: F401,F403
 from .gpt_oracle import Config  # noqa: F401
 from .presets import PRESETS, preset  # noqa: F401
+from . import optim_oracle as optim  # noqa: F401,E402
