@@ -319,6 +319,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B (sequences per GPU), e.g. for profiling")
     ap.add_argument("--no-eval", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--optimizer", action="store_true",
+                    help="add nanoGPT's AdamW step (clip_grad_norm_ at 1.0, decay on 2-D tensors) to every step")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured in a CUDA graph (one GPU)")
     args = ap.parse_args()
@@ -364,12 +366,15 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     from decoder_only_gpt_tcgen05_b200 import dist as gdist
+    opt = g.AdamW(model, lr=6e-4, betas=(0.9, 0.95), weight_decay=0.1, grad_clip=1.0) if args.optimizer else None
 
     def step():
         model.forward_loss(idx_d, tgt_d)
         model.backward()
         if world > 1:
             gdist.allreduce_grads_(model.grads)
+        if opt is not None:
+            opt.step()
 
     def barrier():
         if world > 1:
@@ -526,6 +531,8 @@ def main():
         "config": {"workload": desc, "B": B, "T": T, "tokens_per_step": tokens,
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "launch": "CUDA graph replay of one captured step" if args.graph else "eager stream launches",
+                   "optimizer": ("AdamW step inside every timed step (clip 1.0, decay on 2-D tensors)"
+                                 if args.optimizer else "none: forward + backward"),
                    "l2": "working set (~35 GB of weights and saved activations) far above the 126 MB L2; no flush"},
         "mfu": {"tflops_per_gpu": tflops, "vs_measured_sustained": tflops / peak_sus,
                 "vs_measured_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),

@@ -46,7 +46,17 @@ SIGNATURES = {
     "gpt_eval_bpb": [_P, _P, _P, _P, _P, _I, _I, _P, C.c_size_t, _P, _P, _P, _P],
     "gpt_sync_status": [_P],
     "gpt_set_wait_timeout_ns": [C.c_uint64],
+    "gpt_adamw_scratch_size": [_P],
+    "gpt_adamw_step": [_P, _P, _P, _P, _P, _LL, _P, _P, _P, _P],
+    "gpt_lr_schedule": [_LL, _LL, _LL, C.c_double, C.c_double, _P],
+    "gpt_op_adamw": [_P, _P, _P, _P, _LL, _P, _P, _I, _LL, _P, _P, _P, _P],
 }
+
+
+class AdamWParams(C.Structure):
+    """gpt_adamw of include/gpt.h."""
+    _fields_ = [("lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
+                ("weight_decay", C.c_float), ("grad_scale", C.c_float), ("grad_clip", C.c_float)]
 
 
 def lib():
@@ -65,6 +75,8 @@ def lib():
         L.gpt_op_lmhead_ce_scratch_bytes.argtypes = [_I, _I]
         L.gpt_op_lmhead_ce_noalloc_max_scratch_bytes.restype = C.c_size_t
         L.gpt_op_lmhead_ce_noalloc_max_scratch_bytes.argtypes = []
+        L.gpt_op_adamw_scratch_bytes.restype = C.c_size_t
+        L.gpt_op_adamw_scratch_bytes.argtypes = []
         for name, args in SIGNATURES.items():
             f = getattr(L, name)
             f.argtypes = args

@@ -71,7 +71,9 @@ enum ProfKind : int {
   PK_EMBED_BWD, PK_CAST, PK_CE_COMBINE, PK_LOSS, PK_QK, PK_DELTA, PK_COLSUM, PK_MISC,
   // GEMM roles (the model tags each GEMM call; untagged calls count as PK_GEMM)
   PK_GEMM_QKV, PK_GEMM_O, PK_GEMM_UP, PK_GEMM_DOWN, PK_GEMM_LM_FWD, PK_GEMM_LM_BWD, PK_GEMM_DGRAD,
-  PK_GEMM_WGRAD, PK_COUNT
+  PK_GEMM_WGRAD,
+  PK_OPTIM,  // gradient norm and AdamW update
+  PK_COUNT
 };
 class Prof {
  public:

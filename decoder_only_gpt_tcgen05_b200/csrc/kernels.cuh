@@ -2,6 +2,8 @@
 // embed_bwd.cu) and the attention kernels (attention.cu).
 #pragma once
 
+#include "gpt.h"
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -65,6 +67,15 @@ int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float
                      cudaStream_t st);
 // dwpe[t] (+)= sum_b dx[b*T + t]
 int launch_pos_bwd(const float* dx, int B, int T, int D, float* dwpe, int accumulate, cudaStream_t st);
+
+// ---- optimizer step (optim.cu)
+// fp64 partials of the gradient norm
+size_t adamw_scratch_bytes();
+// clip_grad_norm_ + AdamW over params[0, n): run r of the host table covers
+// [run_start[r], run_start[r + 1]) (the last one up to n) and is weight-decayed when run_decay[r]
+int launch_adamw(float* params, const float* grads, float* m, float* v, long long n, const long long* run_start,
+                 const unsigned char* run_decay, int n_runs, long long step, const gpt_adamw& h, void* scratch,
+                 double* grad_norm, cudaStream_t st);
 
 // ---- attention (attention.cu)
 struct AttnShape {

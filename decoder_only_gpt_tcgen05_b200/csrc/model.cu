@@ -631,6 +631,27 @@ GPT_API int gpt_param_tensor(const gpt_config* cfg, int32_t i, char* name, int32
   return ST_OK;
 }
 
+GPT_API int gpt_adamw_step(const gpt_config* cfg, float* params, const float* grads, float* m, float* v,
+                           int64_t step, const gpt_adamw* h, void* scratch, double* grad_norm, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!h) return set_error(ST_INVALID_ARG, "gpt_adamw_step: null hyperparameters");
+  // weight decay on the 2-D tensors (vectors are stored with cols == 1); adjacent tensors with
+  // the same flag merge into one run
+  Layout L = make_layout(*cfg);
+  std::vector<long long> start;
+  std::vector<unsigned char> decay;
+  for (const ParamInfo& p : L.list) {
+    const unsigned char d = p.cols > 1 ? 1 : 0;
+    if (decay.empty() || decay.back() != d) {
+      start.push_back(p.off);
+      decay.push_back(d);
+    }
+  }
+  return launch_adamw(params, grads, m, v, L.total, start.data(), decay.data(), (int)start.size(), step, *h, scratch,
+                      grad_norm, static_cast<cudaStream_t>(stream));
+}
+
 GPT_API int gpt_workspace_size(const gpt_config* cfg, int32_t B, int32_t T, size_t* bytes) {
   set_error(ST_OK, "");
   GPTK_TRY(validate(cfg));

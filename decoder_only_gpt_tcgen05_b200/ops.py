@@ -3,7 +3,7 @@ from __future__ import annotations
 
 import torch
 
-from ._lib import call
+from ._lib import AdamWParams, call
 
 GEMM_OUT_BF16 = 0
 GEMM_OUT_F32 = 1
@@ -109,7 +109,7 @@ def lmhead_ce_fwd_noalloc(x: torch.Tensor, w: torch.Tensor, targets: torch.Tenso
 PROFILE_FAMILIES = ["gemm", "attn_fwd", "attn_bwd_dkv", "attn_bwd_dq", "norm_fwd", "norm_bwd", "embed_fwd",
                     "embed_bwd", "cast", "ce_combine", "loss", "qk", "delta", "colsum", "misc",
                     "gemm_qkv", "gemm_o", "gemm_up", "gemm_down", "gemm_lm_fwd", "gemm_lm_bwd", "gemm_dgrad",
-                    "gemm_wgrad"]
+                    "gemm_wgrad", "optim"]
 GEMM_FAMILIES = [f for f in PROFILE_FAMILIES if f.startswith("gemm")]
 
 
@@ -135,3 +135,28 @@ def profile_stop() -> dict:
     if rc != n:
         raise RuntimeError(lib().gpt_last_error().decode())
     return {f: (ms[i], cnt[i], fl[i], by[i]) for i, f in enumerate(PROFILE_FAMILIES)}
+
+
+def adamw(params: torch.Tensor, grads: torch.Tensor, m: torch.Tensor, v: torch.Tensor, run_start, run_decay,
+          step: int, *, lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+          weight_decay: float = 0.0, grad_scale: float = 1.0, grad_clip: float = 0.0,
+          scratch: torch.Tensor | None = None, grad_norm: torch.Tensor | None = None) -> torch.Tensor:
+    """clip_grad_norm_ + AdamW over flat fp32 buffers (gpt_op_adamw).  run_start / run_decay: the
+    weight-decay table (run r covers [run_start[r], run_start[r+1]), decayed when run_decay[r]).
+    Returns the fp64 gradient norm (device scalar)."""
+    import ctypes as C
+    from ._lib import lib
+    n = params.numel()
+    for t in (params, grads, m, v):
+        assert t.dtype == torch.float32 and t.is_contiguous() and t.numel() == n and t.device == params.device
+    dev = params.device
+    if scratch is None:
+        scratch = torch.empty(int(lib().gpt_op_adamw_scratch_bytes()), dtype=torch.uint8, device=dev)
+    if grad_norm is None:
+        grad_norm = torch.empty((), dtype=torch.float64, device=dev)
+    rs = (C.c_int64 * len(run_start))(*[int(x) for x in run_start])
+    rd = (C.c_uint8 * len(run_decay))(*[1 if x else 0 for x in run_decay])
+    h = AdamWParams(lr, beta1, beta2, eps, weight_decay, grad_scale, grad_clip)
+    call("gpt_op_adamw", params.data_ptr(), grads.data_ptr(), m.data_ptr(), v.data_ptr(), n, rs, rd, len(run_start),
+         step, C.byref(h), scratch.data_ptr(), grad_norm.data_ptr(), _stream(params))
+    return grad_norm

@@ -128,6 +128,52 @@ GPT_API int gpt_eval_bpb(const gpt_config* cfg, const float* params, const int32
                          const int32_t* token_bytes, int32_t B, int32_t T, void* workspace, size_t workspace_bytes,
                          double* sum_nats, int64_t* sum_bytes, float* bpb, void* stream);
 
+/* Hyperparameters of one optimizer step ("nanoGPT - Karpathy's minimal GPT
+ * pretraining repo", How it works: configure_optimizers builds AdamW; train.py
+ * clips the gradient with clip_grad_norm_ and divides the loss by the number
+ * of accumulated micro-steps). */
+typedef struct gpt_adamw {
+  float lr;            /* learning rate of this step (see gpt_lr_schedule), >= 0                */
+  float beta1, beta2;  /* decay rates of the first and second moments, in [0, 1)                */
+  float eps;           /* > 0, added to the root of the bias-corrected second moment            */
+  float weight_decay;  /* >= 0: p <- p (1 - lr weight_decay) on decayed tensors; lr wd <= 1      */
+  float grad_scale;    /* > 0: multiplies the gradient first (1 / micro-steps, 1 / ranks)       */
+  float grad_clip;     /* >= 0: clip the scaled gradient to this global L2 norm; 0 = no clipping */
+} gpt_adamw;
+
+/* Bytes of device scratch (8-byte aligned) that gpt_adamw_step needs: the
+ * partial sums of the gradient-norm reduction.  Independent of the model. */
+GPT_API int gpt_adamw_scratch_size(size_t* bytes);
+
+/* One optimizer step of nanoGPT's training loop on the flat parameter buffer:
+ * global L2 norm of grad_scale * grads, clip_grad_norm_'s factor
+ * min(1, grad_clip / (norm + 1e-6)), then AdamW with decoupled weight decay:
+ *   g = grads * grad_scale * factor
+ *   m <- beta1 m + (1 - beta1) g;   v <- beta2 v + (1 - beta2) g^2
+ *   p <- p (1 - lr weight_decay)    (2-D tensors only: wte, wpe, lm_head and
+ *                                    the Linear weights; biases and LayerNorm
+ *                                    gains are not decayed)
+ *   p <- p - lr / (1 - beta1^step) * m / (sqrt(v) / sqrt(1 - beta2^step) + eps)
+ *   params    fp32 [gpt_param_count], updated in place
+ *   grads     fp32 [gpt_param_count], read only
+ *   m, v      fp32 [gpt_param_count]: the moments (zero before step 1), updated
+ *   step      1-based step number
+ *   scratch   gpt_adamw_scratch_size bytes
+ *   grad_norm fp64 [1] out: the norm before clipping (may be NULL)
+ * params, grads, m and v are distinct, 16-byte aligned buffers.  The norm is
+ * reduced over a fixed partition, so results are bitwise reproducible. */
+GPT_API int gpt_adamw_step(const gpt_config* cfg, float* params, const float* grads, float* m, float* v,
+                           int64_t step, const gpt_adamw* h, void* scratch, double* grad_norm, void* stream);
+
+/* Learning rate at iteration `it` (host arithmetic, nothing launched): linear
+ * warmup from 0 at it = 0 to learning_rate at it = warmup_iters, then cosine
+ * decay, lr = min_lr + 0.5 (1 + cos(pi r)) (learning_rate - min_lr) with
+ * r = (it - warmup_iters) / (lr_decay_iters - warmup_iters), and min_lr after
+ * lr_decay_iters ("nanoGPT" wiki page, train.py: LR schedule).  Needs
+ * 0 <= warmup_iters <= lr_decay_iters and it >= 0. */
+GPT_API int gpt_lr_schedule(int64_t it, int64_t warmup_iters, int64_t lr_decay_iters, double learning_rate,
+                            double min_lr, double* lr_out);
+
 /* Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait runs out (GPT_ERR_DEVICE_TIMEOUT) or an
  * input id is out of range (GPT_ERR_INVALID_ARG). */

@@ -132,6 +132,17 @@ GPT_API unsigned long long gpt_launch_count(void);
 GPT_API int gpt_profile_start(void);
 GPT_API int gpt_profile_stop(int max_kinds, double* ms, long long* count, double* flops, double* bytes);
 
+/* The optimizer step of gpt_adamw_step on any fp32 buffer of n elements, with
+ * an explicit weight-decay table in HOST memory: run r covers elements
+ * [run_start[r], run_start[r + 1]) (the last run up to n) and is decayed when
+ * run_decay[r] != 0.  run_start[0] == 0 and the starts increase strictly and
+ * stay below n.  scratch: gpt_op_adamw_scratch_bytes() bytes of device memory,
+ * 8-byte aligned.  n == 0 writes a zero grad_norm and launches nothing else. */
+GPT_API size_t gpt_op_adamw_scratch_bytes(void);
+GPT_API int gpt_op_adamw(float* params, const float* grads, float* m, float* v, int64_t n,
+                         const int64_t* run_start, const uint8_t* run_decay, int32_t n_runs, int64_t step,
+                         const gpt_adamw* h, void* scratch, double* grad_norm, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -118,3 +118,51 @@ def test_bench_flop_accounting_matches_oracle(pkg, name):
     for T in (512, 2048, 8192):
         f, b = bench.attention_flops(32768 // T, T, 10, 128)
         assert f == T * 83_886_080 and b == 2 * f
+
+
+def test_lr_schedule_matches_oracle(pkg):
+    for warm, decay in ((2000, 600_000), (0, 100), (10, 10), (1, 7)):
+        for it in sorted({0, 1, warm // 2, warm, warm + 1, (warm + decay) // 2, decay - 1, decay, decay + 5}):
+            if it < 0:
+                continue
+            got = pkg.lr_schedule(it, warm, decay, 6e-4, 6e-5)
+            assert got == pytest.approx(O.optim.lr_schedule(it, warm, decay, 6e-4, 6e-5), rel=1e-14, abs=0), (it, warm)
+
+
+def test_adamw_rejects_bad_arguments_on_the_host(pkg):
+    """Every case below is refused before anything is launched (the pointers are never touched)."""
+    from decoder_only_gpt_tcgen05_b200._lib import AdamWParams, lib
+    L = lib()
+    P = 1 << 20                                   # a 16-byte aligned address that is never dereferenced
+    ok = dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, grad_scale=1.0, grad_clip=1.0)
+
+    def op(params=P, grads=P + 4096, m=P + 8192, v=P + 12288, n=1000, starts=(0, 10), decay=(1, 0), step=1,
+           scratch=P + 16384, **over):
+        h = AdamWParams(**{**ok, **over})
+        rs = (C.c_int64 * max(1, len(starts)))(*starts)
+        rd = (C.c_uint8 * max(1, len(decay)))(*decay)
+        return L.gpt_op_adamw(params, grads, m, v, n, rs, rd, len(starts), step, C.byref(h), scratch, None, None)
+
+    assert op(params=None) == 1
+    assert op(grads=P + 4) == 1                   # misaligned
+    assert op(scratch=None) == 1
+    assert op(n=-1) == 1
+    assert op(step=0) == 1
+    assert op(beta1=1.0) == 1 and op(beta2=-0.1) == 1
+    assert op(eps=0.0) == 1 and op(lr=float("nan")) == 1 and op(lr=-1.0) == 1
+    assert op(grad_scale=0.0) == 1 and op(grad_clip=-1.0) == 1
+    assert op(lr=2.0, weight_decay=1.0) == 1      # lr * weight_decay > 1
+    assert op(starts=(1, 10)) == 1                # the first run must start at 0
+    assert op(starts=(0, 10, 10), decay=(1, 0, 1)) == 1
+    assert op(starts=(0, 1000), decay=(1, 0)) == 1
+    assert op(starts=(), decay=()) == 1
+    assert "adamw" in L.gpt_last_error().decode()
+    c = pkg.preset("tiny").c()
+    h = AdamWParams(**ok)
+    assert L.gpt_adamw_step(None, P, P + 4096, P + 8192, P + 12288, 1, C.byref(h), P + 16384, None, None) == 1
+    assert L.gpt_adamw_step(C.byref(c), P, P + 4096, P + 8192, P + 12288, 1, None, P + 16384, None, None) == 1
+    assert L.gpt_adamw_step(C.byref(c), P, P + 4096, P + 8192, P + 12288, 0, C.byref(h), P + 16384, None, None) == 1
+    assert L.gpt_adamw_step(C.byref(c), P + 8, P + 4096, P + 8192, P + 12288, 1, C.byref(h), P + 16384, None,
+                            None) == 1
+    n = C.c_size_t()
+    assert L.gpt_adamw_scratch_size(C.byref(n)) == 0 and n.value >= 8 and n.value % 8 == 0
