@@ -8,8 +8,9 @@
 // Then the final norm and the lm_head GEMM whose epilogue keeps an online logsumexp
 // per row over each vocab tile, so the logits never reach memory.
 //
-// Backward: cross-entropy gradient tiles (recomputed logits, softmax - onehot) in
-// row chunks feed the lm_head data- and weight-gradient GEMMs; each layer then runs
+// Backward: cross-entropy gradient tiles (recomputed logits, softmax - onehot, bf16
+// dlogits for a block of rows: all of them when they fit in 4 GiB) feed the lm_head
+// data- and weight-gradient GEMMs; each layer then runs
 // its GEMM gradients (MN-major operands, no transposes), the activation gradient in
 // the data-gradient epilogue, the flash-attention backward, the QK-norm/RoPE
 // reverse, the norm backward with the residual add, and finally the deterministic
@@ -440,7 +441,8 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
 
   if (!accumulate) GPTK_CUDA(cudaMemsetAsync(grads, 0, (size_t)pl.P * 4, st));
 
-  // ---- lm_head + cross-entropy, in row chunks: dlogits never exist for all rows at once
+  // ---- lm_head + cross-entropy backward, one block of pl.Mc rows at a time (one block for every
+  //      row when the bf16 dlogits fit in 4 GiB)
   const long long wlm = c.tie_embed ? Lo.wte : Lo.lm_head;
   for (int r0 = 0; r0 < M; r0 += pl.Mc) {
     const int mc = (M - r0) < pl.Mc ? (M - r0) : pl.Mc;
