@@ -8,20 +8,23 @@
 // 128, padding zero); each (b, h) slice is read with 3-D TMA boxes {64 features, rows, 1}
 // under 128-byte swizzle, so rows past the end of a sequence arrive as zeros.
 //
-// Forward (one CTA per 128-query tile of one (b, h); heaviest causal tiles launched first):
-//   warp 0      TMA: Q once, then K_j and V_j through a 2-deep ring
-//   warp 1      one thread issues S_j = Q K_j^T into a double-buffered TMEM tile, then
-//               O += P_{j-1} V_{j-1} (P from shared memory, O accumulating in TMEM)
-//   warps 2..5  softmax, one query row per thread: row max and sum in registers, P = exp2(...)
-//               written to shared memory in the MMA operand layout; O is rescaled in TMEM
-//               only when the running max grows by more than 2^8 (otherwise the stale max
-//               stays exact because O and l use the same one)
+// Forward (one CTA per pair of 128-query tiles of one (b, h); heaviest causal pairs first):
+//   warp 0      TMA: the two Q tiles once, then K_j and V_j through a 3-slot ring
+//   warp 1      one thread alternates between the two tiles: S_j = Q K_j^T into that tile's
+//               TMEM scores, then O += P_{j-1} V_{j-1} (P from shared memory, O in TMEM), so
+//               the tensor core works on one tile while the other tile's softmax runs
+//   warps 2..9  two softmax warpgroups, one per query tile, one query row per thread: row max
+//               and sum in registers, P = exp2(...) written to shared memory in the MMA operand
+//               layout; O is rescaled in TMEM only when the running max grows by more than 2^8
+//               (otherwise the stale max stays exact because O and l use the same one)
 // Backward: delta = rowsum(dO * O) (kernels.cu), then
-//   dK/dV kernel: one CTA per 128-key tile, stepping over 64-query tiles:
-//               S^T = K Q^T, dP^T = V dO^T (TMEM, double buffered), P^T and dS^T to shared
-//               memory, dV += P^T dO, dK += dS^T Q (accumulating in TMEM)
-//   dQ kernel:  one CTA per 128-query tile, stepping over 64-key tiles:
-//               S = Q K^T, dP = dO V^T, dS to shared memory, dQ += dS K
+//   dK/dV kernel: one CTA per 128-key tile, stepping over 128-query blocks from the diagonal:
+//               S^T = K Q^T and dP^T = V dO^T into TMEM; elementwise warps write P^T and dS^T
+//               back over them as bf16, the tensor-memory A operands of dV += P^T dO and
+//               dK += dS^T Q (accumulating in TMEM)
+//   dQ kernel:  one CTA per 128-query tile, stepping over 128-key blocks up to the diagonal:
+//               S = Q K^T and dP = dO V^T into TMEM; dS as bf16 into a TMEM buffer, the A
+//               operand of dQ += dS K
 // Both are deterministic (no atomics).  Every wait is bounded (see ptx.cuh).
 #include <cmath>
 
