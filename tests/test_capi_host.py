@@ -166,3 +166,22 @@ def test_adamw_rejects_bad_arguments_on_the_host(pkg):
                             None) == 1
     n = C.c_size_t()
     assert L.gpt_adamw_scratch_size(C.byref(n)) == 0 and n.value >= 8 and n.value % 8 == 0
+
+
+def test_bench_clock_sample_parsing():
+    """bench.py's clocks record: median SM clock, max clock, and only the reasons reported Active."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    lines = [
+        "0, 1965, 1965, 300.12, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n",
+        "0, 1500, 1965, 998.50, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "0, 1600, 1965, 990.00, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n",
+        "garbage line\n",
+        "0, [N/A], 1965, 990.00, 0x0, Not Active, Not Active, Not Active, Active\n",
+    ]
+    out = bench.parse_clock_samples(lines)
+    assert out == {"sm_mhz": 1600.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    hot = bench.parse_clock_samples(["0, 1200, 1965, 700, 0x48, Not Active, Active, Active, Not Active\n"])
+    assert hot["reasons"] == ["hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert bench.parse_clock_samples([])["reasons"] == ["no samples"]
