@@ -6,13 +6,9 @@
 //   warps 2..9  epilogue: tcgen05.ld the accumulator rows (one row per thread; two warps per
 //               TMEM lane quadrant, each taking half of the tile's columns), apply the fused
 //               epilogue of the call (bias, residual add, activation, activation gradient,
-//               RoPE + QK-norm, cross-entropy partials or gradient), and write through shared
-//               memory with TMA.  The long-K variant (K >= 8192, the weight gradients) has four
-//               epilogue warps, one per quadrant, and gives the freed shared memory to a
-//               deeper operand ring.
+//               cross-entropy partials or gradient), and write through shared memory with TMA
 // The accumulator is double buffered in tensor memory (2 x BN columns) so the epilogue of one
-// tile overlaps the main loop of the next.  One launch may walk the tiles of up to eight
-// problems of equal K (a layer pair's weight gradients), listed in a problem table.
+// tile overlaps the main loop of the next.
 //
 // PAIR variant (cluster of two CTAs on two SMs): the pair walks 256 x BN tiles with one
 // tcgen05.mma.cta_group::2 (M = 256) per K step, issued by the even CTA.  Each CTA stages its
@@ -23,8 +19,7 @@
 // CTA's "tempty" barrier.  Every cross-CTA arrival is waited for before the final cluster
 // barrier, so neither CTA leaves while its peer may still touch its shared memory.
 //
-// Epilogue data path: each epilogue warp owns 32 rows x BN/2 columns (BN with four epilogue
-// warps) and two 4 KB staging buffers.  A chunk of
+// Epilogue data path: each epilogue warp owns 32 rows x BN/2 columns and two 4 KB staging buffers.  A chunk of
 // 32 fp32 or 64 bf16 columns (128-byte rows) goes registers -> swizzled shared memory -> one TMA
 // tile store (or TMA reduce-add for accumulated gradients), so global writes are whole lines.
 // Epilogue inputs (the residual stream, the saved pre-activation) arrive the same way by TMA
