@@ -185,3 +185,18 @@ def test_bench_clock_sample_parsing():
     hot = bench.parse_clock_samples(["0, 1200, 1965, 700, 0x48, Not Active, Active, Active, Not Active\n"])
     assert hot["reasons"] == ["hw_thermal_slowdown", "sw_thermal_slowdown"]
     assert bench.parse_clock_samples([])["reasons"] == ["no samples"]
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: with the shared library absent, every call raises instead of computing."""
+    import decoder_only_gpt_tcgen05_b200 as g
+    from decoder_only_gpt_tcgen05_b200 import _lib
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "libgpt_b200.so"))
+    with pytest.raises(ImportError, match="missing"):
+        _lib.lib()
+    with pytest.raises(ImportError):
+        g.lr_schedule(10, 100, 1000, 1e-3, 1e-4)
+    n = C.c_int64()
+    with pytest.raises(ImportError):
+        _lib.call("gpt_param_count", C.byref(g.preset("tiny").c()), C.byref(n))
