@@ -541,7 +541,7 @@ def main():
                    "launch": "CUDA graph replay of one captured step" if args.graph else "eager stream launches",
                    "optimizer": ("AdamW step inside every timed step (clip 1.0, decay on 2-D tensors)"
                                  if args.optimizer else "none: forward + backward"),
-                   "l2": "working set (~35 GB of weights and saved activations) far above the 126 MB L2; no flush"},
+                   "l2": "working set (~33 GB of weights, gradients and saved activations) far above the 126 MB L2; no flush"},
         "mfu": {"tflops_per_gpu": tflops, "vs_measured_sustained": tflops / peak_sus,
                 "vs_measured_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
                 "vs_datasheet_2250": tflops / DATASHEET_BF16_TFLOPS,

@@ -200,3 +200,37 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     n = C.c_int64()
     with pytest.raises(ImportError):
         _lib.call("gpt_param_count", C.byref(g.preset("tiny").c()), C.byref(n))
+
+
+def _header_declarations():
+    """{name: number of parameters} of every GPT_API function in include/*.h."""
+    out = {}
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", " ", open(h).read(), flags=re.S)
+        for m in re.finditer(r"GPT_API\s+[\w\s\*]+?\b(gpt_\w+)\s*\(([^)]*)\)\s*;", text):
+            params = m.group(2).strip()
+            out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_headers():
+    """Every ctypes signature in the binding has the header's parameter count; every declared
+    function is either in SIGNATURES or given its own restype/argtypes by the loader."""
+    from decoder_only_gpt_tcgen05_b200 import _lib
+    decl = _header_declarations()
+    assert len(decl) >= 25
+    for name, args in _lib.SIGNATURES.items():
+        assert name in decl, name
+        assert len(args) == decl[name], (name, len(args), decl[name])
+    special = {"gpt_last_error", "gpt_launch_count", "gpt_op_lmhead_ce_scratch_bytes",
+               "gpt_op_lmhead_ce_noalloc_max_scratch_bytes", "gpt_op_adamw_scratch_bytes"}
+    assert set(decl) <= set(_lib.SIGNATURES) | special, set(decl) - set(_lib.SIGNATURES) - special
+    loader = open(os.path.join(ROOT, "decoder_only_gpt_tcgen05_b200", "_lib.py")).read()
+    for name in special:
+        assert f"L.{name}.restype" in loader and f"L.{name}.argtypes" in loader, name
+
+
+def test_d20_workspace_is_the_documented_size(pkg):
+    sz = C.c_size_t()
+    assert pkg.lib().gpt_workspace_size(C.byref(pkg.preset("d20").c()), 16, 2048, C.byref(sz)) == 0
+    assert sz.value / 2**30 == pytest.approx(27.4, abs=0.05)
