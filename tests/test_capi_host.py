@@ -234,3 +234,10 @@ def test_d20_workspace_is_the_documented_size(pkg):
     sz = C.c_size_t()
     assert pkg.lib().gpt_workspace_size(C.byref(pkg.preset("d20").c()), 16, 2048, C.byref(sz)) == 0
     assert sz.value / 2**30 == pytest.approx(27.4, abs=0.05)
+
+
+def test_profile_families_match_the_library(pkg):
+    """bench.py reads per-kernel-family times by position: the Python list of families must have
+    exactly the library's number of profiling kinds (gpt_profile_stop returns that number)."""
+    assert pkg.lib().gpt_profile_stop(0, None, None, None, None) == len(pkg.ops.PROFILE_FAMILIES)
+    assert pkg.ops.PROFILE_FAMILIES[0] == "gemm" and pkg.ops.PROFILE_FAMILIES[-1] == "optim"
