@@ -264,23 +264,23 @@ def causal_attention(q, k, v):
     ([GPT2] CausalSelfAttention, the manual path with the explicit mask).
     q, k, v: [B, H, T, hd].  Returns (o, P)."""
     T, hd = q.shape[-2], q.shape[-1]
-    s = np.einsum("bhid,bhjd->bhij", q, k) / math.sqrt(hd)
+    s = (q @ np.swapaxes(k, -1, -2)) / math.sqrt(hd)
     mask = np.triu(np.ones((T, T), dtype=bool), k=1)
     s = np.where(mask, -np.inf, s)
     s = s - np.max(s, axis=-1, keepdims=True)
     p = np.exp(s)
     p = p / np.sum(p, axis=-1, keepdims=True)
-    return np.einsum("bhij,bhjd->bhid", p, v), p
+    return p @ v, p
 
 
 def causal_attention_bwd(do, q, k, v, p):
     """Reverse of causal_attention given its probabilities p."""
     hd = q.shape[-1]
-    dv = np.einsum("bhij,bhid->bhjd", p, do)
-    dp = np.einsum("bhid,bhjd->bhij", do, v)
+    dv = np.swapaxes(p, -1, -2) @ do
+    dp = do @ np.swapaxes(v, -1, -2)
     ds = p * (dp - np.sum(dp * p, axis=-1, keepdims=True))
-    dq = np.einsum("bhij,bhjd->bhid", ds, k) / math.sqrt(hd)
-    dk = np.einsum("bhij,bhid->bhjd", ds, q) / math.sqrt(hd)
+    dq = (ds @ k) / math.sqrt(hd)
+    dk = (np.swapaxes(ds, -1, -2) @ q) / math.sqrt(hd)
     return dq, dk, dv
 
 
