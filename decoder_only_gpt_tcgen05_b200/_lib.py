@@ -44,6 +44,8 @@ SIGNATURES = {
     "gpt_forward_loss": [_P, _P, _P, _P, _I, _I, _P, C.c_size_t, _P, _P],
     "gpt_backward": [_P, _P, _I, _I, _P, C.c_size_t, _P, _I, _P],
     "gpt_eval_bpb": [_P, _P, _P, _P, _P, _I, _I, _P, C.c_size_t, _P, _P, _P, _P],
+    "gpt_token_losses": [_P, _I, _I, _P, C.c_size_t, _P, _P, _P],
+    "gpt_debug_logits": [_P, _I, _I, _P, C.c_size_t, _P, _P],
     "gpt_sync_status": [_P],
     "gpt_set_wait_timeout_ns": [C.c_uint64],
     "gpt_adamw_scratch_size": [_P],

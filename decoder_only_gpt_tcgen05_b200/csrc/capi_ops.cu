@@ -137,7 +137,7 @@ GPT_API int gpt_op_lmhead_ce_fwd(const void* x, const void* w, const int32_t* ta
   p.ce_part = part;
   p.ce_zy = zy;
   GPTK_TRY(run_gemm(EPI_CE_FWD, 256, Operand{x, D, 0}, Operand{w, D, 0}, p, st));
-  return launch_ce_combine(part, ntn, zy, M, ell, lse, st);
+  return launch_ce_combine(part, ntn, zy, targets, V, M, ell, lse, st);
 }
 
 }  // extern "C"

@@ -370,8 +370,11 @@ int launch_colsum_bf16(const __nv_bfloat16* a, long long lda, int M, int N, floa
 
 // ------------------------------------------------------------------ cross-entropy combine
 
-__global__ void ce_combine_kernel(const float2* __restrict__ part, int ntiles, const float* __restrict__ zy, int M,
-                                  float* __restrict__ ell, float* __restrict__ lse) {
+// A target outside [0, V) has no logit: the row's loss is NaN and the device status word records
+// the bad id (the tile epilogues never match it, so its target-logit slot was not written).
+__global__ void ce_combine_kernel(const float2* __restrict__ part, int ntiles, const float* __restrict__ zy,
+                                  const int* __restrict__ targets, int V, int M, float* __restrict__ ell,
+                                  float* __restrict__ lse, DevCtl ctl) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   for (int m = blockIdx.x * warps + (threadIdx.x >> 5); m < M; m += gridDim.x * warps) {
@@ -388,17 +391,23 @@ __global__ void ce_combine_kernel(const float2* __restrict__ part, int ntiles, c
     if (lane == 0) {
       float l = (mx + log2f(s)) * 0.6931471805599453f;
       lse[m] = l;
-      ell[m] = l - zy[m];
+      const int y = targets[m];
+      if (y < 0 || y >= V) {
+        dev_report(ctl, DEV_ERR_BAD_TOKEN, 1);
+        ell[m] = __int_as_float(0x7fc00000);
+      } else {
+        ell[m] = l - zy[m];
+      }
     }
   }
 }
 
-int launch_ce_combine(const float2* part, int ntiles, const float* zy, int M, float* ell, float* lse,
-                      cudaStream_t st) {
+int launch_ce_combine(const float2* part, int ntiles, const float* zy, const int* targets, int V, int M, float* ell,
+                      float* lse, cudaStream_t st) {
   int grid = cdiv(M, 8);
   if (grid > num_sms() * 16) grid = num_sms() * 16;
-  Prof prof(PK_CE_COMBINE, 0, (double)M * ntiles * 8 + M * 12.0, st);
-  ce_combine_kernel<<<grid, 256, 0, st>>>(part, ntiles, zy, M, ell, lse);
+  Prof prof(PK_CE_COMBINE, 0, (double)M * ntiles * 8 + M * 16.0, st);
+  ce_combine_kernel<<<grid, 256, 0, st>>>(part, ntiles, zy, targets, V, M, ell, lse, device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
@@ -410,7 +419,7 @@ int loss_reduce_blocks() { return kLossBlocks; }
 
 // part_d: [blocks][2] (sum of loss, sum of loss over byte-bearing targets); part_i: [blocks][2] (bytes, count)
 __global__ void loss_partial_kernel(const float* __restrict__ ell, const int* __restrict__ targets,
-                                    const int* __restrict__ tb, int M, double* part_d, long long* part_i) {
+                                    const int* __restrict__ tb, int V, int M, double* part_d, long long* part_i) {
   __shared__ double sd[2][8];
   __shared__ long long si[2][8];
   int per = (M + gridDim.x - 1) / gridDim.x;
@@ -421,7 +430,8 @@ __global__ void loss_partial_kernel(const float* __restrict__ ell, const int* __
     double l = ell[r];
     a += l;
     if (tb) {
-      int bytes = tb[targets[r]];
+      const int y = targets[r];
+      const int bytes = (y >= 0 && y < V) ? tb[y] : 0;  // a bad id was reported by the combine kernel
       if (bytes > 0) {
         b += l;
         nb += bytes;
@@ -467,12 +477,12 @@ __global__ void loss_final_kernel(const double* part_d, const long long* part_i,
   if (bpb) *bpb = NB > 0 ? static_cast<float>(Bs / (0.6931471805599453 * (double)NB)) : NAN;
 }
 
-int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int M, double* part_d,
+int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int V, int M, double* part_d,
                        long long* part_i, float* loss, double* sum_nats, long long* sum_bytes, float* bpb,
                        cudaStream_t st) {
   {
     Prof prof(PK_LOSS, 0, M * 12.0, st);
-    loss_partial_kernel<<<kLossBlocks, 256, 0, st>>>(ell, targets, token_bytes, M, part_d, part_i);
+    loss_partial_kernel<<<kLossBlocks, 256, 0, st>>>(ell, targets, token_bytes, V, M, part_d, part_i);
     GPTK_CUDA(cudaGetLastError());
   }
   {

@@ -36,11 +36,12 @@ int launch_colreduce(const float* part, int R, int N, float* out, int accumulate
 int launch_colsum_f32(const float* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st);
 int launch_colsum_bf16(const __nv_bfloat16* a, long long lda, int M, int N, float* part, int* R, cudaStream_t st);
 int colsum_max_chunks();
-// per-row cross-entropy from the vocab-tile partials: ell = lse - z_y
-int launch_ce_combine(const float2* part, int ntiles, const float* zy, int M, float* ell, float* lse,
-                      cudaStream_t st);
+// per-row cross-entropy from the vocab-tile partials: ell = lse - z_y (NaN, and a device status
+// report, for a target outside [0, V))
+int launch_ce_combine(const float2* part, int ntiles, const float* zy, const int* targets, int V, int M, float* ell,
+                      float* lse, cudaStream_t st);
 // deterministic reduction of per-token losses: loss = sum/M, and bpb sums over targets with bytes > 0
-int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int M, double* part_d,
+int launch_loss_reduce(const float* ell, const int* targets, const int* token_bytes, int V, int M, double* part_d,
                        long long* part_i, float* loss, double* sum_nats, long long* sum_bytes, float* bpb,
                        cudaStream_t st);
 int loss_reduce_blocks();

@@ -369,8 +369,8 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
   }
   float* ell = at<float>(ws, pl.ell);
   float* lse_ce = at<float>(ws, pl.lse_ce);
-  GPTK_TRY(launch_ce_combine(part, pl.ntn, zy, M, ell, lse_ce, st));
-  GPTK_TRY(launch_loss_reduce(ell, tgt_ws, token_bytes, M, at<double>(ws, pl.loss_d), at<long long>(ws, pl.loss_i),
+  GPTK_TRY(launch_ce_combine(part, pl.ntn, zy, tgt_ws, V, M, ell, lse_ce, st));
+  GPTK_TRY(launch_loss_reduce(ell, tgt_ws, token_bytes, V, M, at<double>(ws, pl.loss_d), at<long long>(ws, pl.loss_i),
                               loss ? loss : at<float>(ws, pl.loss_f), sum_nats, sum_bytes, bpb, st));
   return ST_OK;
 }
@@ -718,6 +718,41 @@ GPT_API int gpt_eval_bpb(const gpt_config* cfg, const float* params, const int32
   GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
   return forward_impl(*cfg, L, pl, params, idx, targets, token_bytes, workspace, nullptr, sum_nats,
                       reinterpret_cast<long long*>(sum_bytes), bpb, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_token_losses(const gpt_config* cfg, int32_t B, int32_t T, const void* workspace,
+                             size_t workspace_bytes, float* ell, float* lse, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  Layout L = make_layout(*cfg);
+  Plan pl = make_plan(*cfg, B, T, L.total);
+  GPTK_TRY(check_ws(const_cast<void*>(workspace), workspace_bytes, pl.total));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (ell) GPTK_CUDA(cudaMemcpyAsync(ell, at<float>(const_cast<void*>(workspace), pl.ell), (size_t)pl.M * 4,
+                                     cudaMemcpyDeviceToDevice, st));
+  if (lse) GPTK_CUDA(cudaMemcpyAsync(lse, at<float>(const_cast<void*>(workspace), pl.lse_ce), (size_t)pl.M * 4,
+                                     cudaMemcpyDeviceToDevice, st));
+  return ST_OK;
+}
+
+GPT_API int gpt_debug_logits(const gpt_config* cfg, int32_t B, int32_t T, void* workspace, size_t workspace_bytes,
+                             float* logits, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  if (!logits) return set_error(ST_INVALID_ARG, "null logits");
+  Layout L = make_layout(*cfg);
+  Plan pl = make_plan(*cfg, B, T, L.total);
+  GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
+  // the lm_head product of the fused cross-entropy, on the same operands (the saved final-norm
+  // output and the bf16 weight mirror), with its fp32 tiles stored instead of folded
+  const long long wlm = cfg->tie_embed ? L.wte : L.lm_head;
+  GemmParams p = gp(pl.M, pl.V, pl.D);
+  p.out = logits;
+  p.ldo = pl.V;
+  return gemm(EPI_F32, Operand{at<__nv_bfloat16>(workspace, pl.af), pl.D, 0},
+              Operand{at<__nv_bfloat16>(workspace, pl.wbf) + wlm, pl.D, 0}, p, static_cast<cudaStream_t>(stream), 256);
 }
 
 GPT_API int gpt_sync_status(void* stream) {

@@ -13,11 +13,12 @@
 // library, held until the process exits.  Host code cannot pass the array's
 // name to a kernel (on the host it is only a stand-in symbol), so the first
 // call on each device looks up its device address with cudaGetSymbolAddress,
-// with that device current, and caches it; make that first call before any
-// stream capture.  All calls share the one array and it keeps the last call's
-// contents: the target-logit slots are cleared at the start of every call, and
-// calls that overlap on the GPU (different streams, no ordering between them)
-// race on the array.
+// with that device current, and caches it once the lookup has succeeded; make
+// that first call before any stream capture.  All calls share the one array and
+// it keeps the last call's contents: the target-logit slots are cleared at the
+// start of every call (a row whose target lies outside [0, V) gets a NaN loss
+// and a device status report, never a stale value), and calls that overlap on
+// the GPU (different streams, no ordering between them) race on the array.
 #include <mutex>
 #include <string>
 
@@ -32,23 +33,25 @@ static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 
 static __device__ __align__(256) unsigned char g_ce_scratch[kNoAllocScratchBytes];
 
-static void* g_ce_scratch_addr[64];
-static cudaError_t g_ce_scratch_err[64];
-static std::once_flag g_ce_scratch_once[64];
+static void* g_ce_scratch_addr[64];  // non-null once found on that device
+static std::mutex g_ce_scratch_mu;
 
-// Device address of g_ce_scratch on the current device (looked up once per device).
+// Device address of g_ce_scratch on the current device.  Only a successful lookup is kept: a
+// failed one (an error left pending by an earlier launch, or a first call made while a stream
+// is being captured) is retried by the next call instead of failing every later call.
 static int ce_scratch_address(void** out) {
   int dev = 0;
   GPTK_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return set_error(ST_UNSUPPORTED, "lmhead_ce_noalloc: device index above 63");
-  std::call_once(g_ce_scratch_once[dev], [dev]() {
+  std::lock_guard<std::mutex> lock(g_ce_scratch_mu);
+  if (g_ce_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    g_ce_scratch_err[dev] = cudaGetSymbolAddress(&p, g_ce_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_ce_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return set_error(ST_CUDA, std::string("lmhead_ce_noalloc: cudaGetSymbolAddress failed: ") +
+                                    cudaGetErrorString(e));
     g_ce_scratch_addr[dev] = p;
-  });
-  if (g_ce_scratch_err[dev] != cudaSuccess)
-    return set_error(ST_CUDA, std::string("lmhead_ce_noalloc: cudaGetSymbolAddress failed: ") +
-                                  cudaGetErrorString(g_ce_scratch_err[dev]));
+  }
   *out = g_ce_scratch_addr[dev];
   return ST_OK;
 }
@@ -91,7 +94,7 @@ GPT_API int gpt_op_lmhead_ce_fwd_noalloc(const void* x, const void* w, const int
   p.ce_part = part;
   p.ce_zy = zy;
   GPTK_TRY(run_gemm(EPI_CE_FWD, 256, Operand{x, D, 0}, Operand{w, D, 0}, p, st));
-  return launch_ce_combine(part, (int)ntn, zy, M, ell, lse, st);
+  return launch_ce_combine(part, (int)ntn, zy, targets, V, M, ell, lse, st);
 }
 
 }  // extern "C"

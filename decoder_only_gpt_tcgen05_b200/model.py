@@ -150,6 +150,21 @@ class GPT:
              self.sum_nats.data_ptr(), self.sum_bytes.data_ptr(), self.bpb.data_ptr(), _stream(self.device))
         return self.sum_nats, self.sum_bytes, self.bpb
 
+    def token_losses(self):
+        """(ell, lse): fp32 [B*T] per-token loss and logsumexp of the last forward_loss / eval_bpb."""
+        ell = torch.empty(self.B * self.T, dtype=torch.float32, device=self.device)
+        lse = torch.empty_like(ell)
+        call("gpt_token_losses", C.byref(self._c), self.B, self.T, self.workspace.data_ptr(), self.ws_bytes,
+             ell.data_ptr(), lse.data_ptr(), _stream(self.device))
+        return ell, lse
+
+    def debug_logits(self) -> torch.Tensor:
+        """fp32 [B*T, V] logits of the last forward (recomputed by the lm_head GEMM; small batches only)."""
+        z = torch.empty((self.B * self.T, self.cfg.vocab_size), dtype=torch.float32, device=self.device)
+        call("gpt_debug_logits", C.byref(self._c), self.B, self.T, self.workspace.data_ptr(), self.ws_bytes,
+             z.data_ptr(), _stream(self.device))
+        return z
+
     def _check_tokens(self, idx, targets):
         for t in (idx, targets):
             assert t.dtype == torch.int32 and t.is_contiguous() and t.numel() == self.B * self.T, \

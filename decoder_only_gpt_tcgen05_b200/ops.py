@@ -78,10 +78,24 @@ def attention_bwd(fwd: dict, dout: torch.Tensor, B: int, T: int, H: int, hd: int
     return dqkv
 
 
+def _check_lmhead(x, w, targets, ell=None, lse=None):
+    assert x.dim() == 2 and w.dim() == 2 and x.shape[1] == w.shape[1], "x [M, D] and w [V, D]"
+    for t in (x, w):
+        assert t.dtype == torch.bfloat16 and t.is_contiguous() and t.device == x.device, "x, w: contiguous bf16"
+    assert targets.dtype == torch.int32 and targets.is_contiguous() and targets.device == x.device, \
+        "targets: contiguous int32 on the device of x"
+    assert targets.numel() >= x.shape[0], "one target per row of x"
+    for t in (ell, lse):
+        if t is not None:
+            assert t.dtype == torch.float32 and t.is_contiguous() and t.device == x.device and \
+                t.numel() >= x.shape[0], "ell, lse: contiguous fp32 with at least M elements"
+
+
 def lmhead_ce_fwd(x: torch.Tensor, w: torch.Tensor, targets: torch.Tensor):
     """Per-row (loss, logsumexp) of logits x w^T without storing them.
     x bf16 [M, D], w bf16 [V, D], targets int32 [M]."""
     from ._lib import lib
+    _check_lmhead(x, w, targets)
     M, D = x.shape
     V = w.shape[0]
     ell = torch.empty(M, dtype=torch.float32, device=x.device)
@@ -97,6 +111,7 @@ def lmhead_ce_fwd_noalloc(x: torch.Tensor, w: torch.Tensor, targets: torch.Tenso
     """lmhead_ce_fwd without caller scratch: the library keeps its scratch in a
     fixed device array, so only the outputs are passed (pre-allocate them to
     make the call itself allocation-free)."""
+    _check_lmhead(x, w, targets, ell, lse)
     M, D = x.shape
     V = w.shape[0]
     ell = torch.empty(M, dtype=torch.float32, device=x.device) if ell is None else ell

@@ -104,7 +104,8 @@ GPT_API int gpt_init_weights(const gpt_config* cfg, uint64_t seed, float* params
  * The logits are never written to memory: the lm_head product streams vocab
  * tiles through an online logsumexp.  The activations the backward needs
  * stay in `workspace` (copies of idx and targets included).  T <= block_size
- * when pos == 0.  An id outside [0, V) is reported by gpt_sync_status. */
+ * when pos == 0.  An input id or a target outside [0, V) is reported by
+ * gpt_sync_status (a bad target also makes that token's loss NaN). */
 GPT_API int gpt_forward_loss(const gpt_config* cfg, const float* params, const int32_t* idx, const int32_t* targets,
                              int32_t B, int32_t T, void* workspace, size_t workspace_bytes, float* loss,
                              void* stream);
@@ -173,6 +174,26 @@ GPT_API int gpt_adamw_step(const gpt_config* cfg, float* params, const float* gr
  * 0 <= warmup_iters <= lr_decay_iters and it >= 0. */
 GPT_API int gpt_lr_schedule(int64_t it, int64_t warmup_iters, int64_t lr_decay_iters, double learning_rate,
                             double min_lr, double* lr_out);
+
+/* Per-token results of the last gpt_forward_loss or gpt_eval_bpb on this
+ * workspace (same cfg, B and T): ell fp32 [B*T], the loss logsumexp(z) - z[y]
+ * of each target (the next-token cross-entropy of the "nanoGPT" wiki page,
+ * model.py walkthrough, before its mean), and lse fp32 [B*T], the logsumexp
+ * of its logits row, in token order.  Device-to-device copies out of the workspace, enqueued on
+ * `stream`; either output may be NULL. */
+GPT_API int gpt_token_losses(const gpt_config* cfg, int32_t B, int32_t T, const void* workspace,
+                             size_t workspace_bytes, float* ell, float* lse, void* stream);
+
+/* Debug view of the logits of the last forward on this workspace (the
+ * lm_head output of the "nanoGPT" wiki page, model.py walkthrough), fp32
+ * [B*T, V] row-major, written to the caller's buffer (B*T*V*4 bytes; meant
+ * for small batches).  The training and evaluation calls never form this
+ * matrix: their lm_head product folds each vocab tile into the cross-entropy
+ * in registers.  This call runs the same product (the same kernel on the same
+ * operands: the saved final-norm output and the bf16 weight copy) and stores
+ * its fp32 tiles instead, so tests can compare logits with a reference. */
+GPT_API int gpt_debug_logits(const gpt_config* cfg, int32_t B, int32_t T, void* workspace, size_t workspace_bytes,
+                             float* logits, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait runs out (GPT_ERR_DEVICE_TIMEOUT) or an

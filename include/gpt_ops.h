@@ -80,7 +80,9 @@ GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, cons
  * the tensor cores and folded into a per-row online logsumexp over each
  * 256-wide vocab tile; the M x V logits are never written.
  *   x        bf16 [M, D] (normalised final hidden states), w bf16 [V, D]
- *   targets  int32 [M]; ell, lse out fp32 [M] (loss and logsumexp per row)
+ *   targets  int32 [M]; ell, lse out fp32 [M] (loss and logsumexp per row); a
+ *            target outside [0, V) gives its row a NaN loss and is reported
+ *            by gpt_sync_status (GPT_ERR_INVALID_ARG)
  *   scratch  caller memory of gpt_op_lmhead_ce_scratch_bytes(M, V) bytes
  *            (per-row partials of each vocab tile), 256-byte aligned
  * D must be a multiple of 8. */
@@ -98,8 +100,9 @@ GPT_API int gpt_op_lmhead_ce_fwd(const void* x, const void* w, const int32_t* ta
  * (16 MiB) that every GPU loading the library holds until exit, and it calls
  * no allocator.  It needs gpt_op_lmhead_ce_scratch_bytes(M, V) <= that size
  * (else GPT_ERR_INVALID_ARG, nothing launched).  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress) and caches it;
- * make that first call before any stream capture.  All calls share the one
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it
+ * once the lookup has succeeded (a failed lookup is tried again by the next
+ * call); make that first call before any stream capture.  All calls share the one
  * array, which keeps the last call's contents (the call clears what must
  * start at zero); calls that overlap on the GPU race on it, so order them on
  * one stream or with events.  Arguments as gpt_op_lmhead_ce_fwd. */

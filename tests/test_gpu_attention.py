@@ -32,7 +32,7 @@ def _oracle_attention(qkv, B, T, H, hd, rope, qk_norm, dout, eps=1e-5):
     else:
         qh, kh = q, k
     o, p = O.causal_attention(qh, kh, v)
-    s = np.einsum("bhid,bhjd->bhij", qh, kh) / np.sqrt(hd)
+    s = (qh @ np.swapaxes(kh, -1, -2)) / np.sqrt(hd)
     s = np.where(np.triu(np.ones((T, T), bool), 1), -np.inf, s)
     mx = s.max(-1, keepdims=True)
     lse = (np.log(np.exp(s - mx).sum(-1, keepdims=True)) + mx)[..., 0]
@@ -78,7 +78,7 @@ def test_attention_fwd_bwd_matches_oracle(case):
                                                  dout.double().numpy())
     o = f["o"].double().cpu().numpy()
     rms = np.sqrt(np.mean(o_ref ** 2))
-    assert np.abs(o - o_ref).max() <= 2e-2 * rms * 10, np.abs(o - o_ref).max() / rms
+    assert np.abs(o - o_ref).max() <= 2e-2 * rms, np.abs(o - o_ref).max() / rms
     cos, rel = _cos_rel(o, o_ref)
     assert cos >= 0.9999 and rel <= 1e-2, (cos, rel)
     lse = f["lse"].double().cpu().numpy()

@@ -7,6 +7,8 @@ compute, using properties that hold at any size.
   oracle runs one sequence.
 - Causality: the first P rows of a long sequence's attention equal the length-P
   problem (and with the output gradient zeroed past P, so do the gradients).
+- Heads are independent: every row of one (sequence, head) of the full-size
+  attention launch is checked against the oracle run on that head alone.
 - Rows of the lm_head + cross-entropy are independent: sampled rows are checked
   against fp64 dot products."""
 import dataclasses
@@ -56,23 +58,19 @@ def test_full_size_replicated_batch_matches_one_sequence(name, B, T, bytes_hi):
     assert sb == B * rb
     assert abs(bpb - rbpb) / rbpb <= 2e-3
     assert abs(sn - B * rs) / abs(B * rs) <= 2e-3
-    # sampled rows of the lm_head gradient: dW[v] = sum_m (softmax - onehot)[m, v] af[m] / T
-    c = f["cache"]
-    head = "wte" if cfg.tie_embed else "lm_head"
-    W = O.unflatten(ocfg, p)[head]
-    rows = np.concatenate([np.arange(8), np.random.default_rng(3).choice(cfg.vocab_size, 56, replace=False)])
-    dz = np.exp(c["af"] @ W[rows].T - f["lse"][:, None])
-    for k, v in enumerate(rows):
-        dz[tgt1.reshape(-1) == v, k] -= 1.0
-    ref = dz.T @ c["af"] / T
-    off = O.param_offsets(ocfg)[head][0]
-    got = grads.double().cpu().numpy()[off:off + cfg.vocab_size * cfg.n_embd].reshape(cfg.vocab_size, cfg.n_embd)[rows]
-    if cfg.tie_embed:
-        # the tied table also receives the embedding gradient of the rows that occur as inputs
-        keep = ~np.isin(rows, idx1)
-        got, ref = got[keep], ref[keep]
-    cos, rel = _cos_rel(got, ref)
-    assert cos >= 0.999 and rel <= 3e-2, (cos, rel)
+    # every token's loss and logsumexp: each of the B copies equals the single sequence
+    ell, lse = (t.double().cpu().numpy().reshape(B, T) for t in model.token_losses())
+    z_rms = float(np.sqrt(np.mean(f["cache"]["z"] ** 2)))
+    for got, ref, bar in ((lse, f["lse"], 2e-2), (ell, f["ell"], 4e-2)):
+        assert np.abs(got - ref[None, :]).max() <= bar * z_rms, np.abs(got - ref[None, :]).max() / z_rms
+    assert np.linalg.norm(ell[0] - f["ell"]) <= 2e-3 * np.linalg.norm(f["ell"])
+    # every parameter gradient of every layer against the oracle's backward of the one sequence
+    ref_g = O.backward(ocfg, p, f)
+    got = grads.double().cpu().numpy()
+    for nm, (off, shape) in O.param_offsets(ocfg).items():
+        n = int(np.prod(shape))
+        cos, rel = _cos_rel(got[off:off + n], ref_g[off:off + n])
+        assert cos >= 0.999 and rel <= 3e-2, (nm, cos, rel)
 
 
 def test_attention_sweep_prefix_rows_match_oracle():
@@ -121,3 +119,39 @@ def test_d26_lmhead_ce_full_size_sampled_rows():
     assert np.allclose(ell.cpu().numpy()[rows], ref_ell, rtol=2e-3, atol=2e-3)
     assert np.allclose(lse.cpu().numpy()[rows], ref_lse, rtol=1e-4, atol=1e-3)
     assert math.isfinite(float(ell.sum().item()))
+
+
+@pytest.mark.parametrize("T", [2048, 8192])
+def test_attention_every_row_of_one_head_matches_oracle(T):
+    """The attention sweep's launch at T (B = 32768 / T, 10 heads of 128): all T rows of the
+    first and the last (sequence, head) against the oracle run on that head alone, forward
+    (o, logsumexp) and backward (dq, dk, dv through QK-norm and RoPE)."""
+    from test_gpu_attention import _oracle_attention
+    g = _pkg()
+    H, hd = 10, 128
+    B = 32768 // T
+    qkv = torch.from_numpy(synth.normal((B * T, 3 * H * hd), 3)).bfloat16()
+    dout = torch.from_numpy(synth.normal((B * T, H * hd), 4)).bfloat16()
+    f = g.ops.attention_fwd(qkv.to(DEV), B, T, H, hd)
+    dq = g.ops.attention_bwd(f, dout.to(DEV), B, T, H, hd)
+    torch.cuda.synchronize()
+    o_all = f["o"].double().cpu().numpy()
+    lse_all = f["lse"].double().cpu().numpy()
+    dq_all = dq.double().cpu().numpy()
+    qkv_np = qkv.double().numpy()
+    dout_np = dout.double().numpy()
+    for b, h in ((0, 0), (B - 1, H - 1)):
+        rows = slice(b * T, (b + 1) * T)
+        cols = [slice(i * H * hd + h * hd, i * H * hd + (h + 1) * hd) for i in range(3)]
+        qkv1 = np.concatenate([qkv_np[rows, c] for c in cols], axis=1)
+        o_ref, lse_ref, dqkv_ref = _oracle_attention(qkv1, 1, T, 1, hd, True, True,
+                                                     dout_np[rows, h * hd:(h + 1) * hd])
+        o = o_all[rows, h * hd:(h + 1) * hd]
+        rms = np.sqrt(np.mean(o_ref ** 2))
+        assert np.abs(o - o_ref).max() <= 2e-2 * rms, (T, b, h, np.abs(o - o_ref).max() / rms)
+        cos, rel = _cos_rel(o, o_ref)
+        assert cos >= 0.9999 and rel <= 1e-2, (T, b, h, cos, rel)
+        assert np.abs(lse_all[b, h] - lse_ref[0, 0]).max() < 2e-2
+        for i, nm in enumerate("qkv"):
+            cos, rel = _cos_rel(dq_all[rows, cols[i]], dqkv_ref[:, i * hd:(i + 1) * hd])
+            assert cos >= 0.999 and rel <= 3e-2, (T, b, h, nm, cos, rel)

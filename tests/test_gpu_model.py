@@ -2,8 +2,14 @@
 
 Same seeded tokens and the same parameters on both sides (the GPU-initialised
 buffer is copied to the oracle).  Bar: token and byte counts bit-exact; loss
-and bpb within 2e-3 relative; every parameter gradient at cosine >= 0.999 and
-relative L2 <= 3e-2."""
+and bpb within 2e-3 relative; logits within 2e-2 max-abs relative to their RMS;
+every parameter gradient at cosine >= 0.999 and relative L2 <= 3e-2.
+
+Per token, the loss and the logsumexp are compared element by element.  Both
+are 1-Lipschitz in the max-norm of the logits row (the loss moves with the
+logsumexp and the target logit), so the logits bar gives 2e-2 RMS for every
+logsumexp and 4e-2 RMS for every loss; the loss bar, applied to the vector of
+per-token losses, gives a relative L2 of 2e-3."""
 import dataclasses
 import math
 
@@ -73,14 +79,22 @@ def test_forward_backward_bpb_match_oracle(name, params):
     tgt_d = torch.from_numpy(tgt).to(DEV)
     tb_d = torch.from_numpy(tb).to(DEV)
     loss = model.forward_loss(idx_d, tgt_d).item()
+    ell_d, lse_d = model.token_losses()
+    logits = model.debug_logits().double().cpu().numpy()
     grads = model.backward().double().cpu().numpy()
     sum_nats, sum_bytes, bpb = (t.item() for t in model.eval_bpb(idx_d, tgt_d, tb_d))
     g.model.sync_status()
     p = model.params.double().cpu().numpy()
-    f = O.forward(ocfg, p, idx, tgt)
+    f = O.forward(ocfg, p, idx, tgt, return_logits=True)
     ref_g = O.backward(ocfg, p, f)
     rs, rb, rn, rbpb = O.bits_per_byte(f["ell"], tgt, tb)
     assert abs(loss - f["loss"]) / f["loss"] <= 2e-3, (loss, f["loss"])
+    z_rms = float(np.sqrt(np.mean(f["logits"] ** 2)))
+    assert np.abs(logits - f["logits"]).max() <= 2e-2 * z_rms, np.abs(logits - f["logits"]).max() / z_rms
+    ell, lse = ell_d.double().cpu().numpy(), lse_d.double().cpu().numpy()
+    assert np.abs(lse - f["lse"]).max() <= 2e-2 * z_rms, np.abs(lse - f["lse"]).max() / z_rms
+    assert np.abs(ell - f["ell"]).max() <= 4e-2 * z_rms, np.abs(ell - f["ell"]).max() / z_rms
+    assert np.linalg.norm(ell - f["ell"]) <= 2e-3 * np.linalg.norm(f["ell"])
     assert sum_bytes == rb
     assert abs(sum_nats - rs) / abs(rs) <= 2e-3
     assert abs(bpb - rbpb) / rbpb <= 2e-3
@@ -129,3 +143,22 @@ def test_uniform_logits_loss_is_ln_v():
     model.params[off:off + cfg.vocab_size * cfg.n_embd] = 0
     loss = model.forward_loss(torch.from_numpy(idx).to(DEV), torch.from_numpy(tgt).to(DEV)).item()
     assert abs(loss - math.log(cfg.vocab_size)) <= 1e-5 * math.log(cfg.vocab_size)
+
+
+def test_target_out_of_range_is_reported_and_its_loss_is_nan():
+    g, cfg, ocfg, model, idx, tgt, tb = _setup("d20_ragged", "init")
+    bad = tgt.copy()
+    bad[0, 5] = cfg.vocab_size
+    bad[1, 7] = -1
+    model.forward_loss(torch.from_numpy(idx).to(DEV), torch.from_numpy(bad).to(DEV))
+    ell, _ = model.token_losses()
+    with pytest.raises(g.GptError) as e:
+        g.model.sync_status()
+    assert e.value.code == 1
+    ell = ell.cpu().numpy().reshape(bad.shape)
+    assert np.isnan(ell[0, 5]) and np.isnan(ell[1, 7])
+    assert np.isfinite(np.delete(ell.reshape(-1), [5, bad.shape[1] + 7])).all()
+    # the status word was cleared: a valid batch goes through again
+    model.forward_loss(torch.from_numpy(idx).to(DEV), torch.from_numpy(tgt).to(DEV))
+    g.model.sync_status()
+    assert math.isfinite(model.loss.item())
