@@ -55,6 +55,14 @@ class Config:
     scale_resid_init: int = 0     # residual out-projections init std 0.02/sqrt(2*n_layer)
     rope_base: float = 10000.0
     norm_eps: float = 1e-5
+    # sliding-window layers ([CHAT] gpt.py: _compute_window_sizes() expands a pattern such as
+    # "SSSL" into per-layer (left, right) windows): layer l is a short-window layer when bit
+    # (l mod window_period) of window_pattern is set and window_short > 0; its query i then
+    # sees the keys i - window_short .. i (right window 0: causal).  Other layers see every
+    # earlier key.
+    window_short: int = 0
+    window_pattern: int = 0
+    window_period: int = 1
 
     @property
     def head_dim(self) -> int:
@@ -259,13 +267,30 @@ def relu2_grad(u):
     return 2.0 * np.maximum(u, 0.0)
 
 
-def causal_attention(q, k, v):
+def pattern_bits(pattern: str) -> int:
+    """The window_pattern bits of a pattern string such as "SSSL" (bit i set for an 'S')."""
+    return sum(1 << i for i, ch in enumerate(pattern) if ch == "S")
+
+
+def layer_window(cfg: Config, layer: int):
+    """Left window of a layer's attention (keys i - w .. i visible from query i), or None for
+    the full causal prefix ([CHAT] gpt.py, _compute_window_sizes: pattern letter
+    window_pattern[layer mod period], 'S' short, 'L' long)."""
+    if cfg.window_short > 0 and (cfg.window_pattern >> (layer % cfg.window_period)) & 1:
+        return int(cfg.window_short)
+    return None
+
+
+def causal_attention(q, k, v, window=None):
     """softmax(q k^T / sqrt(hd) + mask) v with S[i, j] = -inf for j > i
-    ([GPT2] CausalSelfAttention, the manual path with the explicit mask).
+    ([GPT2] CausalSelfAttention, the manual path with the explicit mask), and also for
+    j < i - window when a left window is given ([CHAT] gpt.py, per-layer windows).
     q, k, v: [B, H, T, hd].  Returns (o, P)."""
     T, hd = q.shape[-2], q.shape[-1]
     s = (q @ np.swapaxes(k, -1, -2)) / math.sqrt(hd)
     mask = np.triu(np.ones((T, T), dtype=bool), k=1)
+    if window is not None:
+        mask |= np.tril(np.ones((T, T), dtype=bool), k=-(window + 1))
     s = np.where(mask, -np.inf, s)
     s = s - np.max(s, axis=-1, keepdims=True)
     p = np.exp(s)
@@ -367,7 +392,7 @@ def forward(cfg: Config, params, idx, targets, keep_cache=True, return_logits=Fa
             q, rq = rmsnorm(q_rot, cfg.norm_eps)
             k, rk = rmsnorm(k_rot, cfg.norm_eps)
             c["qn"] = (q, rq, k, rk)
-        o, pa = causal_attention(q, k, v)
+        o, pa = causal_attention(q, k, v, layer_window(cfg, l))
         o2 = o.transpose(0, 2, 1, 3).reshape(M, D)
         c.update(a1=a1, q=q, k=k, v=v, P=pa, o=o2)
         x = x + _linear(o2, pr[P + "w_o"], pr.get(P + "b_o") if bias else None)

@@ -31,7 +31,7 @@ import math
 
 import numpy as np
 
-from .gpt_oracle import param_shapes
+from .gpt_oracle import param_offsets, param_shapes
 
 
 def decay_mask(cfg) -> np.ndarray:
@@ -81,3 +81,77 @@ def lr_schedule(it: int, warmup_iters: int, lr_decay_iters: int, learning_rate: 
     decay_ratio = (it - warmup_iters) / (lr_decay_iters - warmup_iters)
     coeff = 0.5 * (1.0 + math.cos(math.pi * decay_ratio))
     return min_lr + coeff * (learning_rate - min_lr)
+
+
+# ------------------------------------------------------------------ Muon + AdamW
+#
+# Source: "Train your own ChatGPT", read the source optim.py -- Muon + AdamW: the transformer's
+# 2-D weight matrices go to Muon, an optimizer that orthogonalizes each update (making all its
+# singular values equal); embeddings, the lm_head and the per-layer scalars go to AdamW.
+#
+# Readings where the page is silent (the published Muon of its authors, K. Jordan et al.,
+# "Muon: An optimizer for hidden layers in neural networks", 2024):
+#   - momentum as an exponential average, buf <- mu buf + (1 - mu) g, with the Nesterov form
+#     u = (1 - mu) g + mu buf (mu = 0.95);
+#   - the orthogonalization is five steps of the quintic Newton-Schulz iteration
+#     X <- a X + (b A + c A^2) X, A = X X^T, (a, b, c) = (3.4445, -4.7750, 2.0315), started from
+#     X = u / (||u||_F + 1e-7) on the wide orientation (the matrix is transposed first when it
+#     has more rows than columns, and back afterwards); it maps every singular value s of X to
+#     phi^5(s), phi(s) = a s + b s^3 + c s^5, which lies in [0.68, 1.21] for s >= 3e-3;
+#   - the update is scaled by sqrt(max(1, rows / cols)) and applied as p <- p - lr * update,
+#     with no weight decay on the Muon matrices;
+#   - AdamW as above on every other tensor (no clipping: the page names none for this loop).
+
+NS_COEFFS = (3.4445, -4.7750, 2.0315)
+MUON_TENSORS = ("w_qkv", "w_o", "w_up", "w_down")
+
+
+def is_muon_tensor(name: str) -> bool:
+    return name.split(".")[-1] in MUON_TENSORS
+
+
+def newton_schulz5(G, steps: int = 5, eps: float = 1e-7) -> np.ndarray:
+    """The quintic Newton-Schulz orthogonalization of a 2-D matrix, in the published order."""
+    X = np.asarray(G, dtype=np.float64)
+    wide = X.shape[0] <= X.shape[1]
+    if not wide:
+        X = X.T
+    X = X / (np.linalg.norm(X) + eps)
+    a, b, c = NS_COEFFS
+    for _ in range(steps):
+        A = X @ X.T
+        B = b * A + c * (A @ A)
+        X = a * X + B @ X
+    return X if wide else X.T
+
+
+def muon_update(g, buf, momentum: float = 0.95, nesterov: bool = True):
+    """(update, new momentum buffer) of one Muon step on one matrix."""
+    g = np.asarray(g, dtype=np.float64)
+    buf = momentum * np.asarray(buf, dtype=np.float64) + (1.0 - momentum) * g
+    u = (1.0 - momentum) * g + momentum * buf if nesterov else buf
+    rows, cols = g.shape
+    return newton_schulz5(u) * math.sqrt(max(1.0, rows / cols)), buf
+
+
+def muon_adamw_step(cfg, p, g, mom, v, t: int, muon_lr: float, muon_momentum: float, nesterov: bool,
+                    adam_lr: float, beta1: float, beta2: float, eps: float, weight_decay: float):
+    """One step of the split optimizer over the flat parameter buffer: Muon on the block
+    matrices (mom holds their momentum), AdamW on every other tensor (mom holds its first
+    moment, v its second; weight decay on the 2-D ones).  Returns new (p, mom, v)."""
+    p = np.array(p, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    mom = np.array(mom, dtype=np.float64)
+    v = np.array(v, dtype=np.float64)
+    for name, (off, shape) in param_offsets(cfg).items():
+        n = int(np.prod(shape))
+        sl = slice(off, off + n)
+        if is_muon_tensor(name):
+            upd, buf = muon_update(g[sl].reshape(shape), mom[sl].reshape(shape), muon_momentum, nesterov)
+            p[sl] -= muon_lr * upd.reshape(-1)
+            mom[sl] = buf.reshape(-1)
+        else:
+            mask = np.full(n, len(shape) == 2)
+            p[sl], mom[sl], v[sl], _ = adamw_step(p[sl], g[sl], mom[sl], v[sl], t, adam_lr, beta1, beta2, eps,
+                                                  weight_decay, mask)
+    return p, mom, v

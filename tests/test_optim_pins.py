@@ -107,3 +107,96 @@ def test_lr_schedule_closed_forms():
     seq = [f(it) for it in range(2000, 600_001, 997)]
     assert all(a >= b for a, b in zip(seq, seq[1:]))
     assert OPT.lr_schedule(5, 0, 0, 1e-3, 1e-4) == 1e-4 and OPT.lr_schedule(0, 0, 0, 1e-3, 1e-4) == 1e-3
+
+
+# ------------------------------------------------------------ Muon
+
+def _spectrum_matrix(rows, cols, svals, seed):
+    """A matrix with the given singular values and random orthogonal factors."""
+    rng = np.random.default_rng(seed)
+    k = min(rows, cols)
+    U, _ = np.linalg.qr(rng.standard_normal((rows, k)))
+    V, _ = np.linalg.qr(rng.standard_normal((cols, k)))
+    return (U * np.asarray(svals)) @ V.T
+
+
+@pytest.mark.parametrize("shape", [(24, 40), (40, 24), (32, 32)])
+def test_newton_schulz_acts_on_singular_values(shape):
+    """Five quintic steps map X = G / ||G||_F to U phi^5(S / ||G||_F) V^T, phi(s) = a s + b s^3 + c s^5:
+    the same result reached through the SVD and the scalar polynomial instead of matrix products
+    (a transposed operand, a wrong coefficient or a dropped normalization differs)."""
+    G = synth.normal(shape, 61).astype(np.float64)
+    U, S, Vt = np.linalg.svd(G, full_matrices=False)
+    s = S / (np.linalg.norm(G) + 1e-7)
+    a, b, c = OPT.NS_COEFFS
+    for _ in range(5):
+        s = a * s + b * s ** 3 + c * s ** 5
+    assert np.allclose(OPT.newton_schulz5(G), (U * s) @ Vt, rtol=1e-10, atol=1e-12)
+
+
+def test_newton_schulz_equalizes_singular_values():
+    """The page's description: the update's singular values become (nearly) equal.  For inputs
+    whose normalized singular values span [3e-3, 1] the five steps land them in [0.68, 1.21]."""
+    for shape, seed in (((64, 96), 62), ((96, 64), 63)):
+        k = min(shape)
+        sv = np.geomspace(1.0, 3e-3 * np.sqrt(k), k)       # ||G||_F ~ sqrt(sum s^2)
+        G = _spectrum_matrix(*shape, sv, seed)
+        out = np.linalg.svd(OPT.newton_schulz5(G), compute_uv=False)
+        assert out.min() >= 0.68 and out.max() <= 1.21, (out.min(), out.max())
+        # the spread of the input (hundreds) collapses to under 2
+        assert out.max() / out.min() < 1.8
+
+
+def test_newton_schulz_invariances():
+    G = synth.normal((20, 36), 64).astype(np.float64)
+    X = OPT.newton_schulz5(G)
+    assert np.allclose(OPT.newton_schulz5(7.5 * G), X, rtol=1e-6, atol=1e-9)     # scale (up to eps)
+    assert np.allclose(OPT.newton_schulz5(G.T), X.T, rtol=1e-12, atol=1e-14)    # orientation
+    rng = np.random.default_rng(65)
+    Q1, _ = np.linalg.qr(rng.standard_normal((20, 20)))
+    Q2, _ = np.linalg.qr(rng.standard_normal((36, 36)))
+    assert np.allclose(OPT.newton_schulz5(Q1 @ G @ Q2), Q1 @ X @ Q2, rtol=1e-9, atol=1e-11)
+
+
+def test_muon_momentum_closed_form():
+    """A constant gradient g: the average after t steps is (1 - mu^t) g and the update is the
+    orthogonalized g scaled by sqrt(max(1, rows/cols)) (the normalization removes the scale, up
+    to the 1e-7 guard, which the steep start of phi^5 amplifies to ~1e-5).  Two different
+    gradients g1, g2: the Nesterov input of step 2 points along (1 + mu) g2 + mu^2 g1, the plain
+    average along g2 + mu g1."""
+    g = synth.normal((12, 8), 66).astype(np.float64)
+    buf = np.zeros_like(g)
+    mu = 0.95
+    for t in range(1, 6):
+        upd, buf = OPT.muon_update(g, buf, mu, True)
+        assert np.allclose(buf, (1 - mu ** t) * g, rtol=1e-13)
+        assert np.allclose(upd, OPT.newton_schulz5(g) * np.sqrt(12 / 8), rtol=1e-4, atol=1e-6)
+    g1, g2 = (synth.normal((10, 30), s).astype(np.float64) for s in (69, 70))
+    for nesterov, direction in ((True, (1 + mu) * g2 + mu ** 2 * g1), (False, g2 + mu * g1)):
+        _, b1 = OPT.muon_update(g1, np.zeros_like(g1), mu, nesterov)
+        upd, _ = OPT.muon_update(g2, b1, mu, nesterov)
+        assert np.allclose(upd, OPT.newton_schulz5(direction), rtol=1e-4, atol=1e-6)
+
+
+def test_muon_adamw_step_routes_tensors():
+    """Block matrices move by -lr * (orthogonalized update); every other tensor takes the AdamW
+    step of its own slice."""
+    cfg = O.Config(n_layer=2, n_embd=16, n_head=2, block_size=8, vocab_size=11, norm=O.NORM_LN, linear_bias=1,
+                   tie_embed=0)
+    n = O.param_count(cfg)
+    p, g = (synth.normal(n, s).astype(np.float64) for s in (67, 68))
+    mom, v = np.zeros(n), np.zeros(n)
+    p2, mom2, v2 = OPT.muon_adamw_step(cfg, p, g, mom, v, 1, 0.02, 0.95, True, 1e-3, 0.9, 0.95, 1e-8, 0.1)
+    seen = set()
+    for name, (off, shape) in O.param_offsets(cfg).items():
+        sl = slice(off, off + int(np.prod(shape)))
+        if OPT.is_muon_tensor(name):
+            seen.add(name.split(".")[-1])
+            upd, _ = OPT.muon_update(g[sl].reshape(shape), np.zeros(shape))
+            assert np.allclose(p2[sl], p[sl] - 0.02 * upd.reshape(-1), rtol=1e-13)
+            assert np.all(v2[sl] == 0)
+        else:
+            ref = OPT.adamw_step(p[sl], g[sl], mom[sl], v[sl], 1, 1e-3, 0.9, 0.95, 1e-8, 0.1,
+                                 np.full(sl.stop - sl.start, len(shape) == 2))
+            assert np.allclose(p2[sl], ref[0], rtol=1e-15) and np.allclose(v2[sl], ref[2], rtol=1e-15)
+    assert seen == set(OPT.MUON_TENSORS)

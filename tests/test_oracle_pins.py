@@ -35,6 +35,9 @@ SMALL_CONFIGS = {
                     pos=O.POS_LEARNED, scale_resid_init=1, vocab_size=19),
     # nanochat block shape at toy size: RoPE, QK-norm, ReLU^2, untied, RMSNorm
     "d20ish": _cfg(norm=O.NORM_RMS, pos=O.POS_ROPE, qk_norm=1, act=O.ACT_RELU2, tie_embed=0),
+    # the same with sliding-window layers in the "SSSL" pattern (short window of 3 keys back)
+    "d20ish_sssl": _cfg(n_layer=4, norm=O.NORM_RMS, pos=O.POS_ROPE, qk_norm=1, act=O.ACT_RELU2, tie_embed=0,
+                        window_short=3, window_pattern=O.pattern_bits("SSSL"), window_period=4),
 }
 
 
@@ -196,6 +199,64 @@ def test_attention_backward_matches_library_autograd():
     F.scaled_dot_product_attention(tq, tk, tv, is_causal=True).backward(torch.from_numpy(do))
     for a, b in ((dq, tq), (dk, tk), (dv, tv)):
         assert np.allclose(a, b.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def _brute_force_window_attention(q, k, v, w):
+    """Row by row: softmax over the keys j with i - w <= j <= i only, then the weighted sum."""
+    B, H, T, hd = q.shape
+    o = np.zeros_like(q)
+    for b in range(B):
+        for h in range(H):
+            for i in range(T):
+                js = [j for j in range(T) if j <= i and (w is None or j >= i - w)]
+                sc = np.array([q[b, h, i] @ k[b, h, j] for j in js]) / np.sqrt(hd)
+                e = np.exp(sc - sc.max())
+                a = e / e.sum()
+                o[b, h, i] = sum(a[n] * v[b, h, j] for n, j in enumerate(js))
+    return o
+
+
+@pytest.mark.parametrize("w", [0, 1, 3, 7, None])
+def test_window_attention_matches_brute_force(w):
+    q, k, v = (synth.normal((1, 2, 11, 4), s).astype(np.float64) for s in (21, 22, 23))
+    o, p = O.causal_attention(q, k, v, w)
+    assert np.allclose(o, _brute_force_window_attention(q, k, v, w), rtol=1e-12, atol=1e-12)
+    i, j = np.indices((11, 11))
+    outside = (j > i) if w is None else ((j > i) | (j < i - w))
+    assert np.all(p[:, :, outside] == 0.0) and np.allclose(p.sum(-1), 1.0)
+
+
+def test_window_special_cases():
+    q, k, v = (synth.normal((2, 2, 13, 8), s).astype(np.float64) for s in (24, 25, 26))
+    full, _ = O.causal_attention(q, k, v)
+    for w in (12, 13, 100):   # a window reaching back to key 0 from every query is the full causal mask
+        assert np.array_equal(O.causal_attention(q, k, v, w)[0], full)
+    assert np.array_equal(O.causal_attention(q, k, v, 0)[0], v)   # each query sees only itself
+
+
+def test_window_pattern_expands_per_layer():
+    cfg = O.Config(n_layer=9, n_embd=16, n_head=2, block_size=16, vocab_size=10, window_short=5,
+                   window_pattern=O.pattern_bits("SSSL"), window_period=4)
+    assert [O.layer_window(cfg, l) for l in range(9)] == [5, 5, 5, None, 5, 5, 5, None, 5]
+    off = O.Config(**{**cfg.__dict__, "window_short": 0})
+    assert all(O.layer_window(off, l) is None for l in range(9))
+
+
+def test_window_layer_sees_only_its_band():
+    """One short-window layer of width w: the logits at position i depend on tokens i - w .. i
+    only, so changing token t0 leaves every position outside [t0, t0 + w] bitwise unchanged."""
+    w = 3
+    cfg = _cfg(n_layer=1, norm=O.NORM_RMS, pos=O.POS_ROPE, qk_norm=1, act=O.ACT_RELU2, tie_embed=0,
+               window_short=w, window_pattern=1, window_period=1)
+    p = _random_params(cfg, 27)
+    idx, tg = synth.next_token_batch(1, 14, cfg.vocab_size, dist="uniform", seed=28)
+    t0 = 5
+    idx2 = idx.copy()
+    idx2[0, t0] = (idx2[0, t0] + 7) % cfg.vocab_size
+    z1 = O.forward(cfg, p, idx, tg, return_logits=True)["logits"]
+    z2 = O.forward(cfg, p, idx2, tg, return_logits=True)["logits"]
+    changed = np.any(z1 != z2, axis=1)
+    assert changed[t0:t0 + w + 1].all() and not changed[:t0].any() and not changed[t0 + w + 1:].any()
 
 
 def test_uniform_attention_closed_form():
