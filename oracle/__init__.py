@@ -7,3 +7,4 @@ from .gpt_oracle import *  # noqa: F401,F403
 from .gpt_oracle import Config  # noqa: F401
 from .presets import PRESETS, preset  # noqa: F401
 from . import optim_oracle as optim  # noqa: F401,E402
+from . import fp8_oracle as fp8  # noqa: F401,E402
