@@ -63,6 +63,9 @@ class Config:
     window_short: int = 0
     window_pattern: int = 0
     window_period: int = 1
+    # [CHAT] fp8.py: the forward's block projections on e4m3 operands, every activation and
+    # weight cast with its own dynamic scale (the lm_head and the backward stay unquantized)
+    fp8: int = 0
 
     @property
     def head_dim(self) -> int:
@@ -352,8 +355,12 @@ def _norm_bwd(cfg, dy, cache, pr, grads, name):
     return dx
 
 
-def _linear(x, w, b):
-    y = x @ w.T
+def _linear(x, w, b, fp8=False):
+    if fp8:
+        from .fp8_oracle import scaled_matmul
+        y = scaled_matmul(x, w, "e4m3", "e4m3")
+    else:
+        y = x @ w.T
     return y + b if b is not None else y
 
 
@@ -382,7 +389,8 @@ def forward(cfg: Config, params, idx, targets, keep_cache=True, return_logits=Fa
         P = f"h{l}."
         c = {}
         a1, c["n1"] = _norm(cfg, x, pr, P + "ln1")
-        qkv = _linear(a1, pr[P + "w_qkv"], pr.get(P + "b_qkv") if bias else None)
+        q8 = bool(cfg.fp8)
+        qkv = _linear(a1, pr[P + "w_qkv"], pr.get(P + "b_qkv") if bias else None, q8)
         q, k, v = (qkv[:, i * D:(i + 1) * D].reshape(B, T, H, hd).transpose(0, 2, 1, 3)
                    for i in range(3))
         if phi is not None:
@@ -395,12 +403,12 @@ def forward(cfg: Config, params, idx, targets, keep_cache=True, return_logits=Fa
         o, pa = causal_attention(q, k, v, layer_window(cfg, l))
         o2 = o.transpose(0, 2, 1, 3).reshape(M, D)
         c.update(a1=a1, q=q, k=k, v=v, P=pa, o=o2)
-        x = x + _linear(o2, pr[P + "w_o"], pr.get(P + "b_o") if bias else None)
+        x = x + _linear(o2, pr[P + "w_o"], pr.get(P + "b_o") if bias else None, q8)
         a2, c["n2"] = _norm(cfg, x, pr, P + "ln2")
-        u = _linear(a2, pr[P + "w_up"], pr.get(P + "b_up") if bias else None)
+        u = _linear(a2, pr[P + "w_up"], pr.get(P + "b_up") if bias else None, q8)
         h = relu2(u) if cfg.act == ACT_RELU2 else gelu(u)
         c.update(a2=a2, u=u, h=h)
-        x = x + _linear(h, pr[P + "w_down"], pr.get(P + "b_down") if bias else None)
+        x = x + _linear(h, pr[P + "w_down"], pr.get(P + "b_down") if bias else None, q8)
         layers.append(c)
     af, nf = _norm(cfg, x, pr, "lnf")
     w_lm = pr["wte"] if cfg.tie_embed else pr["lm_head"]

@@ -74,3 +74,23 @@ def test_kernel_precision_cast():
     assert amax == np.float32(11.0) and s == np.float32(448.0) / np.float32(11.0)
     assert q[4] == 448.0 and q[3] == 0.0
     assert np.array_equal(q, F.quantize((x * s).astype(np.float32), "e4m3"))
+
+
+def test_fp8_model_forward_casts_the_four_projections():
+    """With fp8 = 1 the oracle's forward runs its four block projections through the scaled product:
+    the loss moves by the casts' noise only (well under 1 % here).  Causality no longer holds
+    bitwise: a per-tensor scale is the maximum over every token, so a future token that changes
+    the maximum changes how earlier tokens are cast (a property of the method, kept by the GPU)."""
+    import synth
+    cfg = O.Config(n_layer=2, n_embd=32, n_head=2, block_size=16, vocab_size=29, pos=O.POS_ROPE, qk_norm=1,
+                   act=O.ACT_RELU2, tie_embed=0, fp8=1)
+    p = synth.normal(O.param_count(cfg), 5, std=0.2).astype(np.float64)
+    idx, tg = synth.next_token_batch(2, 12, cfg.vocab_size, dist="uniform", seed=6)
+    f8 = O.forward(cfg, p, idx, tg, return_logits=True)
+    hi = O.forward(O.Config(**{**cfg.__dict__, "fp8": 0}), p, idx, tg, keep_cache=False)
+    assert f8["loss"] != hi["loss"] and abs(f8["loss"] - hi["loss"]) < 1e-2 * hi["loss"]
+    idx2 = idx.copy()
+    idx2[:, 8:] = (idx2[:, 8:] + 3) % cfg.vocab_size
+    z2 = O.forward(cfg, p, idx2, tg, return_logits=True)["logits"].reshape(2, 12, -1)
+    z1 = f8["logits"].reshape(2, 12, -1)[:, :8]
+    assert np.abs(z2[:, :8] - z1).max() < 0.2 * np.abs(z1).max()     # changed only by the casts
