@@ -171,10 +171,11 @@ def oracle_step_seconds(preset_name: str, T: int, seed: int = 1) -> float:
     return time.perf_counter() - t0
 
 
-def cpu_baseline(preset_name: str, budget_s: float = 12.0):
+def cpu_baseline(preset_name: str, budget_s: float = 30.0):
     """Oracle fwd+bwd tokens/s on a bounded sample: one sequence whose length
-    is grown (powers of two from 128, at most the workload's T) until one step
-    takes about `budget_s` seconds."""
+    is grown (powers of two from 128, at most the workload's T) while the next
+    length's step is expected within `budget_s` seconds (d20: T = 2048 on a
+    16-core host)."""
     _, _, T_full, _ = WORKLOADS[preset_name]
     T = 128
     t = oracle_step_seconds(preset_name, T)
@@ -327,8 +328,15 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B (sequences per GPU), e.g. for profiling")
     ap.add_argument("--no-eval", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--optimizer", action="store_true",
-                    help="add nanoGPT's AdamW step (clip_grad_norm_ at 1.0, decay on 2-D tensors) to every step")
+    ap.add_argument("--optimizer", nargs="?", const="adamw", default=None, choices=["adamw", "muon", "zero2"],
+                    help="add an optimizer step to every timed step: adamw (nanoGPT's, clip_grad_norm_ at 1.0, "
+                         "decay on 2-D tensors), muon (Muon on the block matrices + AdamW), zero2 (AdamW on "
+                         "each rank's slice after a reduce-scatter, then an all-gather of the weights)")
+    ap.add_argument("--grad-sync", choices=["overlap", "blocking"], default="overlap",
+                    help="with N > 1: average the gradient bucket by bucket while the backward runs (overlap), "
+                         "or in one all-reduce after it (blocking)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="the forward's block projections on e4m3 operands with dynamic per-tensor scales")
     ap.add_argument("--graph", action="store_true",
                     help="time replays of one step captured in a CUDA graph (one GPU)")
     args = ap.parse_args()
@@ -365,7 +373,9 @@ def main():
     if args.batch:
         B = args.batch
         desc += f" [batch overridden: B={B}]"
-    cfg = g.preset(preset_name)
+    cfg = g.preset(preset_name, fp8=1 if args.fp8 else 0)
+    if args.fp8:
+        desc += " [fp8 e4m3 forward projections]"
     model = g.GPT(cfg, B, T, device=dev, seed=0)
     idx, tgt = synth.next_token_batch(B, T, cfg.vocab_size, seed=1 + rank)
     tb = synth.byte_table(cfg.vocab_size, 1, 16 if preset_name != "gpt2" else 12, seed=2)
@@ -374,13 +384,28 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     from decoder_only_gpt_tcgen05_b200 import dist as gdist
-    opt = g.AdamW(model, lr=6e-4, betas=(0.9, 0.95), weight_decay=0.1, grad_clip=1.0) if args.optimizer else None
+    if args.optimizer == "zero2" and world == 1:
+        ap.error("--optimizer zero2 shards the optimizer over ranks: it needs N > 1")
+    sync = None
+    if world > 1 and (args.grad_sync == "overlap" or args.optimizer == "zero2"):
+        sync = gdist.OverlappedGradSync(model, "reduce_scatter" if args.optimizer == "zero2" else "allreduce")
+    if args.optimizer == "adamw":
+        opt = g.AdamW(model, lr=6e-4, betas=(0.9, 0.95), weight_decay=0.1, grad_clip=1.0)
+    elif args.optimizer == "muon":
+        opt = g.MuonAdamW(model, lr=0.02, momentum=0.95, adam_lr=3e-4, betas=(0.9, 0.95), weight_decay=0.0)
+    elif args.optimizer == "zero2":
+        opt = gdist.ShardedAdamW(sync, lr=6e-4, betas=(0.9, 0.95), weight_decay=0.1)
+    else:
+        opt = None
 
     def step():
         model.forward_loss(idx_d, tgt_d)
-        model.backward()
-        if world > 1:
-            gdist.allreduce_grads_(model.grads)
+        if sync is not None:
+            sync.backward()
+        else:
+            model.backward()
+            if world > 1:
+                gdist.allreduce_grads_(model.grads)
         if opt is not None:
             opt.step()
 
@@ -497,9 +522,18 @@ def main():
     if dms <= 0:
         roof = None
     elif dfl > 0:
-        ach = dfl / (dms / 1000.0) / 1e12
+        ach_exec = dfl / (dms / 1000.0) / 1e12
+        if dom == "gemm":
+            # algorithmic: the linear layers' 6 N tokens of the step (without the lm_head logits the
+            # backward recomputes, and without the Muon products of an optimizer step)
+            alg = 6.0 * matmul_params(cfg) * B * T * nprof
+            fam_ms = dms - prof.get("gemm_muon", (0.0,))[0]
+            ach = alg / (fam_ms / 1000.0) / 1e12
+        else:
+            ach = ach_exec
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peak_sus, "unit": "TFLOP/s",
-                "frac": ach / peak_sus, "traffic": None, "launches_per_step": dcnt // nprof,
+                "frac": ach / peak_sus, "achieved_executed": ach_exec, "frac_executed": ach_exec / peak_sus,
+                "traffic": None, "launches_per_step": dcnt // nprof,
                 "share_of_step": dms / total_prof_ms, "peak_source": f"{peak_src} bf16 sustained"}
     else:
         ach = dby / (dms / 1000.0) / 1e9
@@ -511,10 +545,13 @@ def main():
         try:
             import hashlib
             t = json.load(open(traffic_file)).get(dom)
-            # counters taken on one workload and batch describe that launch mix only
+            # counters taken on one workload and batch describe that launch mix only, and only while
+            # every source file that shapes those launches is unchanged
             if t and t.get("workload") == args.workload and t.get("batch") == B:
-                src = open(os.path.join(ROOT, t["source"]), "rb").read()
-                if hashlib.sha256(src).hexdigest() == t["source_sha256"]:
+                h = hashlib.sha256()
+                for f in t["sources"]:
+                    h.update(open(os.path.join(ROOT, f), "rb").read())
+                if h.hexdigest() == t["sources_sha256"]:
                     roof["traffic"] = t["bytes_per_launch"]
         except Exception:
             pass
@@ -535,12 +572,19 @@ def main():
     line = {
         "metric": metric_name(preset_name), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16+e4m3" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": desc, "B": B, "T": T, "tokens_per_step": tokens,
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "launch": "CUDA graph replay of one captured step" if args.graph else "eager stream launches",
-                   "optimizer": ("AdamW step inside every timed step (clip 1.0, decay on 2-D tensors)"
-                                 if args.optimizer else "none: forward + backward"),
+                   "optimizer": {None: "none: forward + backward",
+                                 "adamw": "AdamW step inside every timed step (clip 1.0, decay on 2-D tensors)",
+                                 "muon": "Muon (5 Newton-Schulz steps, bf16 tensor cores) on the block matrices "
+                                         "+ AdamW on the rest, inside every timed step",
+                                 "zero2": "reduce-scatter + AdamW on each rank's slice + all-gather of the "
+                                          "weights, inside every timed step"}[args.optimizer],
+                   "grad_sync": (None if world == 1 else
+                                 "bucketed on a second stream while the backward runs" if sync is not None
+                                 else "one NCCL all-reduce after the backward"),
                    "l2": "working set (~33 GB of weights, gradients and saved activations) far above the 126 MB L2; no flush"},
         "mfu": {"tflops_per_gpu": tflops, "vs_measured_sustained": tflops / peak_sus,
                 "vs_measured_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),

@@ -10,4 +10,4 @@ from . import ops  # noqa: F401
 from . import model  # noqa: F401
 from .model import GPT, GPTConfig, PRESETS, preset  # noqa: F401
 from . import optim  # noqa: F401
-from .optim import AdamW, lr_schedule  # noqa: F401
+from .optim import AdamW, MuonAdamW, lr_schedule  # noqa: F401

@@ -29,8 +29,8 @@ _F = C.c_float
 # name -> argument types (restype is int for all but gpt_last_error)
 SIGNATURES = {
     "gpt_op_gemm": [_I, _I, _P, _LL, _I, _P, _LL, _I, _I, _I, _I, _P, _LL, _P, _I, _P],
-    "gpt_op_attention_fwd": [_P, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P],
-    "gpt_op_attention_bwd": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P],
+    "gpt_op_attention_fwd": [_P, _I, _I, _I, _I, _I, _I, _I, _F, _F, _P, _P, _P, _P, _P, _P, _P],
+    "gpt_op_attention_bwd": [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P],
     "gpt_op_lmhead_ce_fwd": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P],
     "gpt_op_lmhead_ce_fwd_noalloc": [_P, _P, _P, _I, _I, _I, _P, _P, _P],
     "gpt_op_wait_probe": [C.c_ulonglong, _P],
@@ -52,7 +52,20 @@ SIGNATURES = {
     "gpt_adamw_step": [_P, _P, _P, _P, _P, _LL, _P, _P, _P, _P],
     "gpt_lr_schedule": [_LL, _LL, _LL, C.c_double, C.c_double, _P],
     "gpt_op_adamw": [_P, _P, _P, _P, _LL, _P, _P, _I, _LL, _P, _P, _P, _P],
+    "gpt_op_fp8_quantize": [_P, _I, _LL, _I, _P, _P, _P, _P],
+    "gpt_op_gemm_fp8": [_I, _I, _P, _LL, _I, _P, _LL, _I, _I, _I, _I, _P, _P, _P, _LL, _P, _I, _P],
+    "gpt_muon_scratch_size": [_P, _P],
+    "gpt_grad_buckets": [_P, C.c_int32, _P, _P, _P],
+    "gpt_backward_bucketed": [_P, _P, _I, _I, _P, C.c_size_t, _P, _I, _P, _I, _P],
+    "gpt_muon_step": [_P, _P, _P, _P, _P, _LL, _P, _P, _P],
 }
+
+
+class MuonParams(C.Structure):
+    """gpt_muon of include/gpt.h."""
+    _fields_ = [("lr", C.c_float), ("momentum", C.c_float), ("nesterov", C.c_int32), ("ns_steps", C.c_int32),
+                ("adam_lr", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float), ("eps", C.c_float),
+                ("weight_decay", C.c_float)]
 
 
 class AdamWParams(C.Structure):

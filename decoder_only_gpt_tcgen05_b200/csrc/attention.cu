@@ -80,15 +80,21 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_pairs = gridDim.x;
-  const int pr = n_pairs - 1 - blockIdx.x;  // heaviest first
-  const int bh = blockIdx.y;
+  const int n_pairs = gridDim.y;
+  const int pr = n_pairs - 1 - blockIdx.y;  // heaviest first
+  const int bh = blockIdx.x;
   const int b = bh / s.H, h = bh % s.H;
   const int q0 = pr * 256;
-  // KV tiles each query tile needs (0 when the tile lies past the end of the sequence)
-  const int n_a = 2 * pr + 1;
-  const int n_b = (q0 + 128 < s.T) ? 2 * pr + 2 : 0;
-  const int n_kv = n_b > 0 ? n_b : n_a;
+  // KV blocks of each query tile t: [lo_t, 2 pr + t] (the diagonal block last; the lower end is 0,
+  // or the block of the tile's first query minus the left window).  The ring streams blocks
+  // jlo .. jlo + n_kv - 1, jlo = lo_A; tile t takes ring blocks f[t] .. f[t] + c[t] - 1.
+  // c[1] = 0 when tile B lies past the end of the sequence.
+  const int lo_a = s.win >= 0 ? max(0, (q0 - s.win) / 128) : 0;
+  const int lo_b = s.win >= 0 ? max(0, (q0 + 128 - s.win) / 128) : 0;
+  const int jlo = lo_a;
+  const int c_t[2] = {2 * pr + 1 - lo_a, (q0 + 128 < s.T) ? 2 * pr + 2 - lo_b : 0};
+  const int f_t[2] = {0, lo_b - lo_a};
+  const int n_kv = c_t[1] > 0 ? f_t[1] + c_t[1] : c_t[0];
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
@@ -135,7 +141,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_expect_tx(&kv_full[slot], L::TILE);
       const int col = (seq & 1) ? colv : colk;
       for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::KV + slot * L::TILE + c * 16384, &tm_qkv, &kv_full[slot], col + 64 * c, (seq >> 1) * 128, b);
+        tma_load_3d(sm + L::KV + slot * L::TILE + c * 16384, &tm_qkv, &kv_full[slot], col + 64 * c,
+                    (jlo + (seq >> 1)) * 128, b);
       issued = seq;
     }
     if (!ok) {
@@ -150,7 +157,6 @@ __global__ void __launch_bounds__(320, 1)
     constexpr uint32_t idesc_o = idesc_bf16(128, HD, 0, 1);
     bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 23);
     bool issued = false;
-    const int n_t[2] = {n_a, n_b};
     auto kv_wait = [&](int seq) -> bool {
       return mbar_wait(&kv_full[seq % 3], (seq / 3) & 1, ctl, abort_flag, 24);
     };
@@ -193,13 +199,15 @@ __global__ void __launch_bounds__(320, 1)
         aa[kk] = sdesc_add(dP, (kk >> 2) * 16384 + (kk & 3) * 32);
         bb[kk] = sdesc_add(dV, kk * 2048);
       }
-      umma8_ss(dd, aa, bb, idesc_o, j == 0 ? 0xfeu : 0xffu);
+      umma8_ss(dd, aa, bb, idesc_o, j == f_t[t] ? 0xfeu : 0xffu);
       umma_commit(&o_done[t]);
     };
+    // ring block j (0-based from jlo): tile t computes S for it when f[t] <= j < f[t] + c[t]
+    auto takes = [&](int t, int j) { return c_t[t] > 0 && j >= f_t[t] && j < f_t[t] + c_t[t]; };
     if (ok && kv_wait(0)) {
       tc_fence_after();
       for (int t = 0; t < 2; ++t)
-        if (n_t[t] > 0) issue_s(t, 0);
+        if (takes(t, 0)) issue_s(t, 0);
       umma_commit(&kv_empty[0]);
       issued = true;
     } else {
@@ -207,11 +215,15 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int j = 0; j < n_kv && ok; ++j) {
       for (int t = 0; t < 2 && ok; ++t) {
-        if (j >= n_t[t]) continue;
-        if (!mbar_wait(&p_full[t], j & 1, ctl, abort_flag, 26) || !kv_wait(2 * j + 1)) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(t, j);
-        if (j + 1 < n_t[t]) {
+        if (takes(t, j)) {
+          if (!mbar_wait(&p_full[t], (j - f_t[t]) & 1, ctl, abort_flag, 26) || !kv_wait(2 * j + 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, j);
+        }
+        if (takes(t, j + 1)) {
           if (!kv_wait(2 * j + 2)) { ok = false; break; }
           tc_fence_after();
           issue_s(t, j + 1);
@@ -232,7 +244,8 @@ __global__ void __launch_bounds__(320, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int qi = q0 + 128 * t + r;
-    const int n = t == 0 ? n_a : n_b;
+    const int n = c_t[t];
+    const int jfirst = jlo + f_t[t];  // the tile's first KV block
     const int diag = 2 * pr + t;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tbase + 128 * t + lane_off;
@@ -240,13 +253,17 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t sP = smem_u32(sm + L::P + t * 32768);
     float m = -INFINITY, l = 0.f;
     bool ok = n > 0;
-    for (int j = 0; j < n; ++j) {
-      if (!mbar_wait(&s_full[t], j & 1, ctl, abort_flag, 29)) { ok = false; break; }
+    for (int i = 0; i < n; ++i) {
+      if (!mbar_wait(&s_full[t], i & 1, ctl, abort_flag, 29)) { ok = false; break; }
       tc_fence_after();
       // The row is handled as two halves of 64 scores (two TMEM loads in flight per half):
       // ten warps leave at most 168 registers per thread, too few to hold all 128 scores.
+      const int j = jfirst + i;
       const int kbase = j * 128;
-      const bool dg = (j == diag);
+      // masked: the diagonal block (causal), or a block reaching below the window of the tile's
+      // last query (keys before qi - win do not exist for query qi)
+      const bool dg = (j == diag) || (s.win >= 0 && kbase < q0 + 128 * t + 127 - s.win);
+      const int kmin = s.win >= 0 ? qi - s.win : 0;
       uint32_t raw[64];
       float* sv = reinterpret_cast<float*>(raw);
       float mx8[8];
@@ -259,28 +276,28 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         tmem_fence_regs<64>(raw);
         if (dg) {
-          // diagonal tile: keys after the query (or past the sequence) do not exist
+          // keys after the query, past the sequence or before the window do not exist
 #pragma unroll
           for (int e = 0; e < 64; ++e) {
             const int key = kbase + hf * 64 + e;
-            if (key > qi || key >= s.T) sv[e] = -INFINITY;
+            if (key > qi || key >= s.T || key < kmin) sv[e] = -INFINITY;
           }
         }
 #pragma unroll
-        for (int e = 0; e < 64; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], sv[e]);
+        for (int e = 0; e < 64; e += 2) mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], sv[e], sv[e + 1]);
       }
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      mx *= scale_log2;
+      mx *= scale_log2;  // -inf when every key of the block lies outside this row's window
       const float m_new = fmaxf(m, mx);
       float alpha = 1.f;
       if (m_new > m + 8.f) {
         alpha = ex2_approx(m - m_new);
         m = m_new;
       }
-      if (j > 0) {
+      if (i > 0) {
         // O and P_t are still in use by the previous P V product of this tile
-        if (!mbar_wait(&o_done[t], (j - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
+        if (!mbar_wait(&o_done[t], (i - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
@@ -295,9 +312,12 @@ __global__ void __launch_bounds__(320, 1)
       }
       // P = exp2(s * scale - m) -> shared memory (K-major, 128-byte swizzle; masked scores are
       // -inf and give 0).  The second half is still in registers; the first is read again.
-      float rs8[8];
+      float2 rs2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+      for (int k = 0; k < 4; ++k) rs2[k] = make_float2(0.f, 0.f);
+      // a row with no visible key yet (m = -inf) takes 0 as its offset: its scores are all -inf
+      const float m_off = m == -INFINITY ? 0.f : m;
+      const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_off, -m_off);
 #pragma unroll
       for (int it = 0; it < 2; ++it) {
         const int hf = 1 - it;
@@ -310,25 +330,26 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
               const int key = kbase + e;
-              if (key > qi || key >= s.T) sv[e] = -INFINITY;
+              if (key > qi || key >= s.T || key < kmin) sv[e] = -INFINITY;
             }
           }
         }
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
-          float pv[8];
+          float2 pv[4];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            pv[k] = ex2_approx(fmaf(sv[8 * g + k], scale_log2, -m));
-            rs8[k] += pv[k];
+          for (int k = 0; k < 4; ++k) {
+            const float2 x = ffma2(make_float2(sv[8 * g + 2 * k], sv[8 * g + 2 * k + 1]), sc2, nm2);
+            pv[k] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            rs2[k] = fadd2(rs2[k], pv[k]);
           }
           // 16-byte unit (hf*8 + g): chunk hf (keys 64*hf ..), unit g within the 128-byte row
           st_shared_v4(sP + hf * 16384 + sw128_off(r, g),
-                       make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]), pack_bf16x2(pv[4], pv[5]),
-                                  pack_bf16x2(pv[6], pv[7])));
+                       make_uint4(pack_bf16x2(pv[0].x, pv[0].y), pack_bf16x2(pv[1].x, pv[1].y),
+                                  pack_bf16x2(pv[2].x, pv[2].y), pack_bf16x2(pv[3].x, pv[3].y)));
         }
       }
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      const float rs = ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) + ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
       l = l * alpha + rs;
       fence_async_smem();
       tc_fence_before();
@@ -422,11 +443,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* stats = reinterpret_cast<float*>(sm + L::STATS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;
+  const int kt = blockIdx.x;  // the tiles of one head run side by side (they share Q and dO in L2)
   const int bh = blockIdx.y;
   const int b = bh / s.H, h = bh % s.H;
   const int k0 = kt * 128;
-  const int n_it = (s.T + 127) / 128 - kt;  // query blocks from the diagonal one on
+  // query blocks from the diagonal one on, up to the last query whose window still reaches this
+  // tile's last key
+  int n_it = (s.T + 127) / 128 - kt;
+  if (s.win >= 0) n_it = min(n_it, (k0 + 127 + s.win) / 128 - kt + 1);
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
@@ -590,7 +614,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!mbar_wait(&stats_bar[st], (it >> 1) & 1, ctl, abort_flag, 50)) { ok = false; break; }
       if (!mbar_wait(s_full, it & 1, ctl, abort_flag, 47)) { ok = false; break; }
       tc_fence_after();
-      const bool masked = (it == 0) || (qb + 128 > s.T);
+      // the diagonal block, the ragged end, or a block whose last query's window misses the
+      // tile's first key
+      const bool masked = (it == 0) || (qb + 128 > s.T) || (s.win >= 0 && qb + 127 - s.win > k0);
       for (int hh = 0; hh < 2; ++hh) {
         const int c = 4 * hh + w;  // queries qb + 16c .. qb + 16c + 15
         uint32_t rs[16], rd[16];
@@ -614,7 +640,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
               const int e = 4 * g + k;
               const int q = qb + 16 * c + e;
               float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
-              if (q < key || q >= s.T) pv = 0.f;
+              if (q < key || q >= s.T || (s.win >= 0 && q - s.win > key)) pv = 0.f;
               p[k] = pv;
               ds[k] = pv * (__uint_as_float(rd[e]) - dl[k]);
             }
@@ -722,11 +748,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = gridDim.x;
-  const int qt = n_qt - 1 - blockIdx.x;  // heaviest tiles first
+  const int qt = n_qt - 1 - blockIdx.x;  // heaviest tiles of each head first
   const int bh = blockIdx.y;
   const int b = bh / s.H, h = bh % s.H;
   const int q0 = qt * 128;
-  const int n_kv = qt + 1;  // 128-key blocks 0 .. qt (the last one is the diagonal block)
+  // 128-key blocks j0 .. qt (the last one is the diagonal block; j0 > 0 when the first query's
+  // window starts past key 0); the rings count blocks from j0
+  const int j0 = s.win >= 0 ? max(0, (q0 - s.win) / 128) : 0;
+  const int n_kv = qt + 1 - j0;
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
@@ -782,13 +811,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!mbar_wait(&k_empty[ks], ((j / KS) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
       mbar_expect_tx(&k_full[ks], L::TILE);
       for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::K0 + ks * L::TILE + c * 16384, &tm_kv128, &k_full[ks], colk + 64 * c, j * 128, b);
+        tma_load_3d(sm + L::K0 + ks * L::TILE + c * 16384, &tm_kv128, &k_full[ks], colk + 64 * c, (j0 + j) * 128, b);
       issued_k = j;
       const int vs = j % VS;
       if (!mbar_wait(&v_empty[vs], ((j / VS) & 1) ^ 1u, ctl, abort_flag, 61)) { ok = false; break; }
       mbar_expect_tx(&v_full[vs], L::TILE);
       for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::V0 + vs * L::TILE + c * 16384, &tm_kv128, &v_full[vs], colv + 64 * c, j * 128, b);
+        tma_load_3d(sm + L::V0 + vs * L::TILE + c * 16384, &tm_kv128, &v_full[vs], colv + 64 * c, (j0 + j) * 128, b);
       issued_v = j;
     }
     if (!ok) {
@@ -893,10 +922,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) mbar_arrive(s_free);
       const int bb = j & 1;
       if (!mbar_wait(&ds_empty[bb], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 69)) { ok = false; break; }
-      const int kb = j * 128 + 32 * cg;
+      const int kb = (j0 + j) * 128 + 32 * cg;
       uint32_t dw[16];
-      if ((kb + 31 > q0) || (kb + 32 > s.T) || !row_ok) {
-        // diagonal block, ragged end or rows past T: causal / range mask
+      if ((kb + 31 > q0) || (kb + 32 > s.T) || !row_ok || (s.win >= 0 && kb < q0 + 127 - s.win)) {
+        // diagonal block, ragged end, rows past T or the window's lower edge: mask
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           float d2[2];
@@ -905,7 +934,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int e = 2 * e2 + k;
             const int key = kb + e;
             float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -lse2));
-            if (!row_ok || key > qi || key >= s.T) pv = 0.f;
+            if (!row_ok || key > qi || key >= s.T || (s.win >= 0 && key < qi - s.win)) pv = 0.f;
             d2[k] = pv * (__uint_as_float(rd[e]) - dl);
           }
           dw[e2] = pack_bf16x2(d2[0], d2[1]);
@@ -967,25 +996,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ====================================================================== launchers
 
+double attn_pairs(int T, int win) {
+  const double t = T;
+  if (win < 0 || win >= T - 1) return t * (t + 1) / 2;
+  const double w = win;
+  return w * (w + 1) / 2 + (t - w) * (w + 1);  // rows i < win see i + 1 keys, the rest win + 1
+}
+
 template <int HD>
-static int attn_fwd_t(const __nv_bfloat16* qkv, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
-                      cudaStream_t st) {
+static int attn_fwd_launch(const CUtensorMap& tm, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
+                           float scale_log2, cudaStream_t st) {
   using L = FwdSmem<HD>;
-  CUtensorMap tm;
-  GPTK_TRY(make_tmap_3d(&tm, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
   GPTK_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
-  const float scale_log2 = kLog2e / sqrtf((float)s.hd);
-  dim3 grid((s.T + 255) / 256, s.B * s.H);
-  const double causal = (double)s.B * s.H * ((double)s.T * (s.T + 1) / 2);
+  // (b, h) fastest, so the heaviest causal pairs of every head start first
+  dim3 grid(s.B * s.H, (s.T + 255) / 256);
+  const double causal = (double)s.B * s.H * attn_pairs(s.T, s.win);
   Prof prof(PK_ATTN_FWD, 4.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 4, st);
   attn_fwd_kernel<HD><<<grid, 320, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
 
+template <int HD>
+static int attn_fwd_t(const __nv_bfloat16* qkv, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
+                      cudaStream_t st) {
+  CUtensorMap tm;
+  GPTK_TRY(make_tmap_3d(&tm, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
+  return attn_fwd_launch<HD>(tm, s, o, ldo, lse, kLog2e / sqrtf((float)s.hd), st);
+}
+
 int launch_attn_fwd(const __nv_bfloat16* qkv_pad, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
                     cudaStream_t st) {
   if (s.B < 1 || s.T < 1 || s.H < 1) return set_error(ST_INVALID_ARG, "attention: empty shape");
+  if (s.win < -1) return set_error(ST_INVALID_ARG, "attention: window must be >= 0 (or -1 for none)");
   if (s.B * s.H > 65535) return set_error(ST_UNSUPPORTED, "attention: B*H above 65535");
   if (s.hdp == 64) return attn_fwd_t<64>(qkv_pad, s, o, ldo, lse, st);
   if (s.hdp == 128) return attn_fwd_t<128>(qkv_pad, s, o, ldo, lse, st);
@@ -1003,7 +1046,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
   const float scale = 1.f / sqrtf((float)s.hd);
   const float scale_log2 = kLog2e * scale;
   const DevCtl ctl = device_ctl();
-  const double causal = (double)s.B * s.H * ((double)s.T * (s.T + 1) / 2);
+  const double causal = (double)s.B * s.H * attn_pairs(s.T, s.win);
   {
     using L = DkvSmem<HD>;
     static_assert(L::BYTES <= 232448, "dK/dV shared memory above the per-block limit");
@@ -1030,6 +1073,7 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
 int launch_attn_bwd(const __nv_bfloat16* qkv_pad, const __nv_bfloat16* do_pad, const float* lse,
                     const float* delta, const AttnShape& s, __nv_bfloat16* dqkv_pad, cudaStream_t st) {
   if (s.B < 1 || s.T < 1 || s.H < 1) return set_error(ST_INVALID_ARG, "attention: empty shape");
+  if (s.win < -1) return set_error(ST_INVALID_ARG, "attention: window must be >= 0 (or -1 for none)");
   if (s.B * s.H > 65535) return set_error(ST_UNSUPPORTED, "attention: B*H above 65535");
   if (s.hdp == 64) return attn_bwd_t<64>(qkv_pad, do_pad, lse, delta, s, dqkv_pad, st);
   if (s.hdp == 128) return attn_bwd_t<128>(qkv_pad, do_pad, lse, delta, s, dqkv_pad, st);

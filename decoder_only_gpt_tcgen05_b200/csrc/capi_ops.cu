@@ -71,11 +71,12 @@ static int check_attn_shape(int B, int T, int H, int hd) {
   return ST_OK;
 }
 
-GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, int rope, int qk_norm, float rope_base,
-                                 float eps, void* qkv_norm, float* rstd_q, float* rstd_k, float* rope_cs, void* o,
-                                 float* lse, void* stream) {
+GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, int rope, int qk_norm, int window,
+                                 float rope_base, float eps, void* qkv_norm, float* rstd_q, float* rstd_k,
+                                 float* rope_cs, void* o, float* lse, void* stream) {
   set_error(ST_OK, "");
   GPTK_TRY(check_attn_shape(B, T, H, hd));
+  if (window < -1) return set_error(ST_INVALID_ARG, "attention: window must be >= 0, or -1 for none");
   if (!qkv || !qkv_norm || !o || !lse) return set_error(ST_INVALID_ARG, "attention: null pointer");
   if (rope && !rope_cs) return set_error(ST_INVALID_ARG, "attention: rope needs rope_cs");
   if (qk_norm && (!rstd_q || !rstd_k)) return set_error(ST_INVALID_ARG, "attention: qk_norm needs rstd_q, rstd_k");
@@ -85,16 +86,17 @@ GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, i
   if (rope) GPTK_TRY(launch_rope_table(cs, T, hd / 2, rope_base, st));
   GPTK_TRY(launch_qk_fwd(static_cast<const __nv_bfloat16*>(qkv), cs, M, T, H, hd, hd, rope, qk_norm, eps,
                          static_cast<__nv_bfloat16*>(qkv_norm), rstd_q, rstd_k, st));
-  AttnShape s{B, T, H, hd, hd, 3LL * H * hd};
+  AttnShape s{B, T, H, hd, hd, 3LL * H * hd, window};
   return launch_attn_fwd(static_cast<const __nv_bfloat16*>(qkv_norm), s, static_cast<__nv_bfloat16*>(o),
                          (long long)H * hd, lse, st);
 }
 
 GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, const float* rstd_k, const float* rope_cs,
                                  const void* o, const float* lse, const void* dout, int B, int T, int H, int hd,
-                                 int rope, int qk_norm, float* delta, void* dqkv, void* stream) {
+                                 int rope, int qk_norm, int window, float* delta, void* dqkv, void* stream) {
   set_error(ST_OK, "");
   GPTK_TRY(check_attn_shape(B, T, H, hd));
+  if (window < -1) return set_error(ST_INVALID_ARG, "attention: window must be >= 0, or -1 for none");
   if (!qkv_norm || !o || !lse || !dout || !delta || !dqkv) return set_error(ST_INVALID_ARG, "attention: null pointer");
   if (rope && !rope_cs) return set_error(ST_INVALID_ARG, "attention: rope needs rope_cs");
   if (qk_norm && (!rstd_q || !rstd_k)) return set_error(ST_INVALID_ARG, "attention: qk_norm needs rstd_q, rstd_k");
@@ -104,7 +106,7 @@ GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, cons
   const __nv_bfloat16* dO = static_cast<const __nv_bfloat16*>(dout);
   __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(dqkv);
   GPTK_TRY(launch_attn_delta(static_cast<const __nv_bfloat16*>(o), dO, B, T, H, hd, hd, delta, st));
-  AttnShape s{B, T, H, hd, hd, 3LL * H * hd};
+  AttnShape s{B, T, H, hd, hd, 3LL * H * hd, window};
   GPTK_TRY(launch_attn_bwd(qn, dO, lse, delta, s, dq, st));
   // gradient w.r.t. the normalised q, k, v -> through QK-norm and RoPE, in place
   return launch_qk_bwd(dq, qn, rstd_q, rstd_k, reinterpret_cast<const float2*>(rope_cs), M, T, H, hd, hd, rope,

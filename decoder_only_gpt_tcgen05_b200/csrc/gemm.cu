@@ -83,7 +83,10 @@ int make_tmap_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t ou
   cuuint64_t strides[1] = {ld * (uint64_t)esize};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  CUresult r = fn(map, esize == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  const CUtensorMapDataType dt = esize == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : esize == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                              : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(ST_CUDA, "cuTensorMapEncodeTiled (2d) failed: " + std::to_string((int)r));
@@ -109,10 +112,10 @@ int make_tmap_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, u
 
 // ------------------------------------------------------------ GEMM launcher
 
-template <int BN, int EPI, bool LONGK, bool PAIR>
+template <int BN, int EPI, bool LONGK, bool PAIR, bool F8 = false>
 static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
   using C = GemmCfg<BN, LONGK, PAIR>;
-  auto kern = gemm_kernel<BN, EPI, LONGK, PAIR>;
+  auto kern = gemm_kernel<BN, EPI, LONGK, PAIR, F8>;
   static bool attr_set[64] = {false};
   static int max_pairs[64] = {0};
   int dev = 0;
@@ -144,14 +147,14 @@ static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t
   if (grid > tiles) grid = tiles;
   double flops = 0, bytes = 0;
   for (int q = 0; q < p.n_prob; ++q) {
-    const double M = p.pM[q], N = p.pN[q], K = p.K;
+    const double M = p.pM[q], N = p.pN[q], K = p.pK[q] > 0 ? p.pK[q] : p.K;
     double out_bytes = M * N * 2;
     if (EPI == EPI_F32 || EPI == EPI_RESID) out_bytes = M * N * 4 * (1 + (p.accumulate || EPI == EPI_RESID));
     if (EPI == EPI_UP) out_bytes = M * N * (p.out ? 4 : 2);
     if (EPI == EPI_ACTBWD) out_bytes = M * N * 4;
     if (EPI == EPI_CE_FWD) out_bytes = M * p.tiles_n * 8;
     flops += 2.0 * M * N * K;
-    bytes += (M * K + N * K) * 2 + out_bytes;
+    bytes += (M * K + N * K) * (F8 ? 1 : 2) + out_bytes;
   }
   Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, flops, bytes, st);
   if (PAIR) {
@@ -195,7 +198,26 @@ static int dispatch_epi(int epi, const GemmMaps& maps, const GemmParams& p, cuda
   return set_error(ST_INVALID_ARG, "unknown GEMM epilogue");
 }
 
+template <int BN, bool PAIR>
+static int dispatch_epi_f8(int epi, const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
+  switch (epi) {
+    case EPI_BF16: return launch_gemm_t<BN, EPI_BF16, false, PAIR, true>(maps, p, st);
+    case EPI_F32: return launch_gemm_t<BN, EPI_F32, false, PAIR, true>(maps, p, st);
+    case EPI_RESID: return launch_gemm_t<BN, EPI_RESID, false, PAIR, true>(maps, p, st);
+    case EPI_QKV:
+      if (BN != 256 || !p.tma_out || p.qk_D % 256 != 0)
+        return set_error(ST_UNSUPPORTED, "fused RoPE/QK-norm epilogue needs 256-column tiles over whole heads");
+      return launch_gemm_t<BN, EPI_QKV, false, PAIR, true>(maps, p, st);
+    case EPI_UP: return launch_gemm_t<BN, EPI_UP, false, PAIR, true>(maps, p, st);
+  }
+  return set_error(ST_INVALID_ARG, "GEMM: this epilogue has no 8-bit operand variant");
+}
+
 static int dispatch(int epi, int bn, bool pair, const GemmMaps& maps, const GemmParams& p, cudaStream_t st) {
+  if (p.f8_inv_a) {
+    if (pair) return dispatch_epi_f8<256, true>(epi, maps, p, st);
+    return bn == 256 ? dispatch_epi_f8<256, false>(epi, maps, p, st) : dispatch_epi_f8<128, false>(epi, maps, p, st);
+  }
   if (pair) return dispatch_epi<256, true>(epi, maps, p, st);
   return bn == 256 ? dispatch_epi<256, false>(epi, maps, p, st) : dispatch_epi<128, false>(epi, maps, p, st);
 }
@@ -216,9 +238,15 @@ static bool aligned16(const void* ptr, long long ld, int esize) {
   return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15) == 0 && ((ld * esize) & 15) == 0;
 }
 
-// b_rows: B rows one CTA stages per K step (the tile's N, or half of it for CTA pairs)
+// b_rows: B rows one CTA stages per K step (the tile's N, or half of it for CTA pairs).  8-bit
+// operands (f8) are K-major only, with 128-element (128-byte) boxes along K.
 static int operand_maps(const Operand& A, const Operand& B, int M, int N, int K, int b_rows, CUtensorMap* ta,
-                        CUtensorMap* tb) {
+                        CUtensorMap* tb, bool f8 = false) {
+  if (f8) {
+    if (A.mn_major || B.mn_major) return set_error(ST_UNSUPPORTED, "GEMM: 8-bit operands must be K-major");
+    GPTK_TRY(make_tmap_2d(ta, A.ptr, K, M, A.ld, 128, 128, 1));
+    return make_tmap_2d(tb, B.ptr, K, N, B.ld, 128, b_rows, 1);
+  }
   if (!A.mn_major) {
     GPTK_TRY(make_tmap_2d(ta, A.ptr, K, M, A.ld, 64, 128));
   } else {
@@ -259,7 +287,10 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   std::memset(&maps, 0, sizeof(maps));
   const bool pair = use_pair(bn, (long long)((p.M + 255) / 256) * ((p.N + 255) / 256));
   const int tile_m = pair ? 256 : 128;
-  GPTK_TRY(operand_maps(A, B, p.M, p.N, p.K, pair ? bn / 2 : bn, &maps.a[0], &maps.b[0]));
+  const bool f8 = p.f8_inv_a != nullptr;
+  if (f8 && (!p.f8_inv_b || p.f8_fmt_a < 0 || p.f8_fmt_a > 1 || p.f8_fmt_b < 0 || p.f8_fmt_b > 1))
+    return set_error(ST_INVALID_ARG, "GEMM: 8-bit operands need both inverse scales and formats 0 (e4m3) / 1 (e5m2)");
+  GPTK_TRY(operand_maps(A, B, p.M, p.N, p.K, pair ? bn / 2 : bn, &maps.a[0], &maps.b[0], f8));
   // output / input tensor maps of the TMA epilogue, where the layout allows one
   p.tma_out = 0;
   const bool f32out = (epi == EPI_F32 || epi == EPI_RESID);
@@ -297,9 +328,12 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
 }
 
 int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
-                   cudaStream_t st) {
+                   cudaStream_t st, int epi, int accumulate) {
   if (n < 1 || n > kMaxProblems) return set_error(ST_INVALID_ARG, "grouped GEMM: 1 to 8 problems");
   if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
+  if (!(epi == EPI_F32 || (epi == EPI_BF16 && !accumulate)))
+    return set_error(ST_INVALID_ARG, "grouped GEMM: fp32 (stored or accumulated) or bf16 (stored) outputs");
+  const int es = epi == EPI_F32 ? 4 : 2;
   GemmMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   GemmParams p;
@@ -307,7 +341,7 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
   p.K = K;
   p.a_mn = a_mn;
   p.b_mn = b_mn;
-  p.accumulate = 1;
+  p.accumulate = accumulate;
   p.hd = p.hdp = 1;
   p.tma_out = 1;
   p.prof_kind = prof_kind;
@@ -319,11 +353,13 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
   int start = 0;
   for (int q = 0; q < n; ++q) {
     const GroupProblem& g = probs[q];
-    if (g.M <= 0 || g.N <= 0 || !aligned16(g.out, g.ldo, 4))
+    if (g.M <= 0 || g.N <= 0 || g.K_ext < 0 || g.K_ext > K || !aligned16(g.out, g.ldo, es))
       return set_error(ST_INVALID_ARG, "grouped GEMM: bad problem");
-    GPTK_TRY(operand_maps(Operand{g.a, g.lda, a_mn}, Operand{g.b, g.ldb, b_mn}, g.M, g.N, K, pair ? bn / 2 : bn, &maps.a[q],
-                          &maps.b[q]));
-    GPTK_TRY(make_tmap_2d(&maps.c[q], g.out, g.N, g.M, g.ldo, 32, 32, 4));
+    const int kq = g.K_ext > 0 ? g.K_ext : K;
+    GPTK_TRY(operand_maps(Operand{g.a, g.lda, a_mn}, Operand{g.b, g.ldb, b_mn}, g.M, g.N, kq, pair ? bn / 2 : bn,
+                          &maps.a[q], &maps.b[q]));
+    p.pK[q] = kq;
+    GPTK_TRY(make_tmap_2d(&maps.c[q], g.out, g.N, g.M, g.ldo, es == 4 ? 32 : 64, 32, es));
     p.pM[q] = g.M;
     p.pN[q] = g.N;
     p.ptiles_m[q] = (g.M + tile_m - 1) / tile_m;
@@ -340,7 +376,7 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
   p.group_m = p.pgroup_m[0];
   p.ctl = device_ctl();
   if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
-  return dispatch(EPI_F32, bn, pair, maps, p, st);
+  return dispatch(epi, bn, pair, maps, p, st);
 }
 
 }  // namespace gptk

@@ -23,7 +23,17 @@
 // 32 fp32 or 64 bf16 columns (128-byte rows) goes registers -> swizzled shared memory -> one TMA
 // tile store (or TMA reduce-add for accumulated gradients), so global writes are whole lines.
 // Epilogue inputs (the residual stream, the saved pre-activation) arrive the same way by TMA
-// load.  Rows and columns past M and N are clipped by the tensor maps.
+// load.  Rows and columns past M and N are clipped by the tensor maps.  The fused epilogues:
+// bias; residual add (EPI_RESID); activation with the pre-activation kept or not (EPI_UP); its
+// gradient (EPI_ACTBWD); RoPE + per-head RMSNorm of q and k on the fp32 accumulator, one 128-wide
+// head per epilogue warp of a 256-column tile (EPI_QKV); the per-tile online logsumexp of the
+// cross-entropy (EPI_CE_FWD) and its gradient softmax - onehot (EPI_CE_BWD).
+//
+// Variants: LONGK (reductions over all tokens, the weight gradients) has four epilogue warps and a
+// deeper ring; a grouped launch runs up to eight products with the same K and operand layouts
+// from one problem table (tile_start / pM / pN ...), their tiles in one persistent schedule; F8
+// takes 8-bit operands (kind::f8f6f4, 128 K elements per stage) and scales every accumulator by
+// the operands' inverse scales.
 //
 // Either operand may be K-major (rows of K contiguous elements: the usual [out,in] weight and
 // [tokens,features] activation layouts) or MN-major (M or N contiguous: what the gradient GEMMs
@@ -88,6 +98,12 @@ struct GemmParams {
   int n_prob;
   int tile_start[9];
   int pM[8], pN[8], ptiles_m[8], ptiles_n[8], pgroup_m[8];
+  int pK[8];                  // host only: K extent of each problem (0 = K), for the FLOP count
+  // 8-bit operands (the F8 kernels): formats (0 = e4m3, 1 = e5m2) and the inverse scales that
+  // multiply every accumulator (device scalars: the product is (a s_a)(b s_b)^T / (s_a s_b))
+  int f8_fmt_a, f8_fmt_b;
+  const float* f8_inv_a;
+  const float* f8_inv_b;
 };
 
 constexpr int kMaxProblems = 8;
@@ -289,10 +305,13 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int tile) {
 
 // --------------------------------------------------------------- the kernel
 
-template <int BN, int EPI, bool LONGK, bool PAIR>
+// F8: 8-bit operands (kind::f8f6f4, both K-major): a stage holds 128 K elements (the same 128
+// bytes per row as 64 bf16 ones), four K = 32 MMAs, and the epilogue scales every accumulator.
+template <int BN, int EPI, bool LONGK, bool PAIR, bool F8 = false>
 __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
     gemm_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using C = GemmCfg<BN, LONGK, PAIR>;
+  constexpr int KE = F8 ? 2 * C::BK : C::BK;  // K elements per stage
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -350,7 +369,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   const int num_tiles = p.tile_start[p.n_prob];
-  const int num_k = (p.K + C::BK - 1) / C::BK;
+  const int num_k = (p.K + KE - 1) / KE;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer
@@ -378,33 +397,33 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           if (rank == 0) mbar_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           if (!p.a_mn) {
-            tma_load_2d_pair(a, tmA, fb, kb * C::BK, arow);
+            tma_load_2d_pair(a, tmA, fb, kb * KE, arow);
           } else {
 #pragma unroll
-            for (int c = 0; c < C::BM / 64; ++c) tma_load_2d_pair(a + c * 8192, tmA, fb, arow + c * 64, kb * C::BK);
+            for (int c = 0; c < C::BM / 64; ++c) tma_load_2d_pair(a + c * 8192, tmA, fb, arow + c * 64, kb * KE);
           }
           if (!p.b_mn) {
-            tma_load_2d_pair(b, tmB, fb, kb * C::BK, brow);
+            tma_load_2d_pair(b, tmB, fb, kb * KE, brow);
           } else {
 #pragma unroll
             for (int c = 0; c < C::B_ROWS / 64; ++c)
-              tma_load_2d_pair(b + c * 8192, tmB, fb, brow + c * 64, kb * C::BK);
+              tma_load_2d_pair(b + c * 8192, tmB, fb, brow + c * 64, kb * KE);
           }
         } else {
           mbar_expect_tx(&full[stage], C::STAGE_BYTES);
           if (!p.a_mn) {
-            tma_load_2d(a, tmA, &full[stage], kb * C::BK, arow);
+            tma_load_2d(a, tmA, &full[stage], kb * KE, arow);
           } else {
 #pragma unroll
             for (int c = 0; c < C::BM / 64; ++c)
-              tma_load_2d(a + c * 8192, tmA, &full[stage], arow + c * 64, kb * C::BK);
+              tma_load_2d(a + c * 8192, tmA, &full[stage], arow + c * 64, kb * KE);
           }
           if (!p.b_mn) {
-            tma_load_2d(b, tmB, &full[stage], kb * C::BK, brow);
+            tma_load_2d(b, tmB, &full[stage], kb * KE, brow);
           } else {
 #pragma unroll
             for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(b + c * 8192, tmB, &full[stage], brow + c * 64, kb * C::BK);
+              tma_load_2d(b + c * 8192, tmB, &full[stage], brow + c * 64, kb * KE);
           }
         }
         pending |= 1u << stage;
@@ -438,7 +457,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------ MMA issuer (the even CTA of a pair)
     constexpr uint32_t IDESC_KK = idesc_bf16(C::TILE_M, BN, 0, 0);
-    const uint32_t idesc = IDESC_KK | (static_cast<uint32_t>(p.a_mn) << 15) | (static_cast<uint32_t>(p.b_mn) << 16);
+    const uint32_t idesc = F8 ? idesc_f8(C::TILE_M, BN, p.f8_fmt_a, p.f8_fmt_b)
+                              : IDESC_KK | (static_cast<uint32_t>(p.a_mn) << 15) | (static_cast<uint32_t>(p.b_mn) << 16);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -472,8 +492,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
           aa[kk] = sdesc_add(da, kk * stepA);
           bb[kk] = sdesc_add(db, kk * stepB);
         }
-        if (PAIR) umma4_ss_pair(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
-        else umma4_ss(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
+        if (F8) {
+          if (PAIR) umma4_f8_pair(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
+          else umma4_f8(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
+        } else {
+          if (PAIR) umma4_ss_pair(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
+          else umma4_ss(d_tmem, aa, bb, idesc, kb == 0 ? 0xeu : 0xfu);
+        }
         if (PAIR) {
           // the stage is free in both CTAs once these MMAs have read it
           const uint32_t eb = smem_u32(&empty[stage]);
@@ -535,6 +560,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
     constexpr int CW = F32OUT ? 32 : 64;
     constexpr bool HAS_IN = (EPI == EPI_RESID || EPI == EPI_ACTBWD);
     constexpr int HALF = BN * 4 / C::EPI_WARPS;  // columns per epilogue warp
+    const float f8_scale = F8 ? __ldg(p.f8_inv_a) * __ldg(p.f8_inv_b) : 1.f;
     for (int tile = tile0; tile < num_tiles; tile += tile_step) {
       const TileInfo ti = tile_info(p, tile);
       const int tm = ti.tm, tn = ti.tn;
@@ -604,7 +630,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
             float v[32];
             tmem_ld32(trow + c_begin + 32 * q4, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+            for (int j = 0; j < 32; ++j) {
+              if (F8) v[j] *= f8_scale;
+              ss = fmaf(v[j], v[j], ss);
+            }
           }
           r = rsqrtf(ss * (1.f / 128.f) + p.qk_eps);
           if (row_ok) (part ? p.rstd_k : p.rstd_q)[(long long)row * p.qk_H + hh] = r;
@@ -617,6 +646,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
           float x1[32], x2[32];
           tmem_ld32(trow + c_begin + 32 * rr, x1);
           tmem_ld32(trow + c_begin + 64 + 32 * rr, x2);
+          if (F8) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              x1[j] *= f8_scale;
+              x2[j] *= f8_scale;
+            }
+          }
 #pragma unroll
           for (int j2 = 0; j2 < 16; ++j2) {
             const float4 e = p.qk_rope ? __ldg(csr + 16 * rr + j2) : make_float4(1.f, 0.f, 1.f, 0.f);
@@ -645,6 +681,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
         for (int c = c_begin; c < c_begin + HALF; c += 32) {
           float v[32];
           tmem_ld32(trow + c, v);
+          if (F8) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= f8_scale;
+          }
           epi_chunk_generic<EPI>(p, v, row, n0 + c, row_ok);
         }
       } else {
@@ -666,6 +706,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
           float v[CW];
           tmem_ld32(trow + c, *reinterpret_cast<float(*)[32]>(&v[0]));
           if (CW == 64) tmem_ld32(trow + c + 32, *reinterpret_cast<float(*)[32]>(&v[32 % CW]));
+          if (F8) {
+#pragma unroll
+            for (int j = 0; j < CW; ++j) v[j] *= f8_scale;
+          }
           if (EPI != EPI_ACTBWD && EPI != EPI_CE_BWD) {
             add_bias32(v, p.bias, col0, pN);
             if (CW == 64) add_bias32(v + (32 % CW), p.bias, col0 + 32, pN);

@@ -72,7 +72,8 @@ enum ProfKind : int {
   // GEMM roles (the model tags each GEMM call; untagged calls count as PK_GEMM)
   PK_GEMM_QKV, PK_GEMM_O, PK_GEMM_UP, PK_GEMM_DOWN, PK_GEMM_LM_FWD, PK_GEMM_LM_BWD, PK_GEMM_DGRAD,
   PK_GEMM_WGRAD,
-  PK_OPTIM,  // gradient norm and AdamW update
+  PK_OPTIM,  // optimizer elementwise steps (gradient norm, AdamW update, Muon momentum and updates)
+  PK_GEMM_MUON,  // the Newton-Schulz products of the Muon step
   PK_COUNT
 };
 class Prof {
@@ -88,19 +89,25 @@ struct GemmParams;
 // C[M,N] = A[M,K] B[N,K]^T with the fused epilogue `epi`; bn = 128 or 256.
 int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p, cudaStream_t st);
 
-// One product of a grouped launch: out[M,N] += A B^T in fp32 (accumulating).
+// One product of a grouped launch: out[M,N] (+)= A B^T (fp32, or bf16 when stored).  K_ext, when
+// > 0, is the K extent this problem's operands really have (at most the launch's K): its
+// tensor maps end there and the rest of the launch's K loop reads zeros, so one launch can
+// hold the pieces of a split reduction whose last piece is shorter.
 struct GroupProblem {
   const void* a;
   long long lda;
   const void* b;
   long long ldb;
   int M, N;
-  float* out;
+  void* out;
   long long ldo;
+  int K_ext;
 };
-// Up to 4 accumulating fp32 products with the same K and operand layouts in one persistent
-// launch (their tiles share one schedule, so small products do not leave SMs idle).
+// Up to 8 products with the same K and operand layouts in one persistent launch (their tiles
+// share one schedule, so small products do not leave SMs idle): fp32 outputs accumulated
+// (epi EPI_F32, accumulate 1, the default) or stored (accumulate 0), or bf16 outputs stored
+// (epi EPI_BF16).
 int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
-                   cudaStream_t st);
+                   cudaStream_t st, int epi = 1, int accumulate = 1);
 
 }  // namespace gptk

@@ -286,6 +286,99 @@ int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b
   });
 }
 
+// RMSNorm backward from the saved bf16 output y = x r (the next GEMM's A operand, kept for the
+// weight gradients) instead of x: dx = r (dy - y mean(dy y)); dres (+)= dx in fp32 and a bf16 copy.
+// dy is bf16 (DYB) or fp32.  One warp per row, 8 elements per lane and step (16-byte loads of the
+// bf16 rows); 14 bytes per element with a bf16 dy and accumulation (18 for the x-based kernel).
+__device__ __forceinline__ void bf16x8(uint4 u, float* v) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+  }
+}
+
+template <int NV8, bool DYB>
+__global__ void rms_bwd_kernel(const void* __restrict__ dy_, const __nv_bfloat16* __restrict__ y,
+                               const float* __restrict__ rstd, int M, int D, float* __restrict__ dres,
+                               int dres_init, __nv_bfloat16* __restrict__ dres_bf) {
+  const int warps = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int D8 = D / 8;
+  for (int m = blockIdx.x * warps + w; m < M; m += gridDim.x * warps) {
+    const long long base = (long long)m * D;
+    const float r = rstd[m];
+    float yv[NV8][8], gv[NV8][8];
+    float s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV8; ++i) {
+      const int c = i * 32 + lane;
+      if (c < D8) {
+        bf16x8(reinterpret_cast<const uint4*>(y + base)[c], yv[i]);
+        if (DYB) {
+          bf16x8(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dy_) + base)[c], gv[i]);
+        } else {
+          const float4* g4 = reinterpret_cast<const float4*>(static_cast<const float*>(dy_) + base) + 2 * c;
+          const float4 a = g4[0], b = g4[1];
+          gv[i][0] = a.x; gv[i][1] = a.y; gv[i][2] = a.z; gv[i][3] = a.w;
+          gv[i][4] = b.x; gv[i][5] = b.y; gv[i][6] = b.z; gv[i][7] = b.w;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) s2 = fmaf(gv[i][k], yv[i][k], s2);
+      }
+    }
+    const float m2 = warp_sum(s2) / D;
+#pragma unroll
+    for (int i = 0; i < NV8; ++i) {
+      const int c = i * 32 + lane;
+      if (c < D8) {
+        float o[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[k] = r * (gv[i][k] - yv[i][k] * m2);
+        float4* dr = reinterpret_cast<float4*>(dres + base) + 2 * c;
+        if (!dres_init) {
+          const float4 a = dr[0], b = dr[1];
+          o[0] += a.x; o[1] += a.y; o[2] += a.z; o[3] += a.w; o[4] += b.x; o[5] += b.y; o[6] += b.z; o[7] += b.w;
+        }
+        dr[0] = make_float4(o[0], o[1], o[2], o[3]);
+        dr[1] = make_float4(o[4], o[5], o[6], o[7]);
+        reinterpret_cast<uint4*>(dres_bf + base)[c] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
+                                                                 pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+      }
+    }
+  }
+}
+
+int launch_rms_bwd(const void* dy, int dy_bf16, const __nv_bfloat16* y, const float* rstd, int M, int D,
+                   float* dres, int dres_init, __nv_bfloat16* dres_bf, cudaStream_t st) {
+  if (D % 8) return set_error(ST_UNSUPPORTED, "rms_bwd: n_embd must be a multiple of 8");
+  const int nv8 = (D + 255) / 256;
+  auto run = [&](auto nvc) -> int {
+    constexpr int NV8 = decltype(nvc)::value;
+    int grid = cdiv(M, 8);
+    if (grid > num_sms() * 16) grid = num_sms() * 16;
+    Prof prof(PK_NORM_BWD, 0, (double)M * D * ((dy_bf16 ? 2 : 4) + 2 + 4 + 2 + (dres_init ? 0 : 4)) + M * 4.0, st);
+    if (dy_bf16) rms_bwd_kernel<NV8, true><<<grid, 256, 0, st>>>(dy, y, rstd, M, D, dres, dres_init, dres_bf);
+    else rms_bwd_kernel<NV8, false><<<grid, 256, 0, st>>>(dy, y, rstd, M, D, dres, dres_init, dres_bf);
+    GPTK_CUDA(cudaGetLastError());
+    return (int)ST_OK;
+  };
+  switch (nv8) {
+    case 1: return run(std::integral_constant<int, 1>());
+    case 2: return run(std::integral_constant<int, 2>());
+    case 3: return run(std::integral_constant<int, 3>());
+    case 4: return run(std::integral_constant<int, 4>());
+    case 5: return run(std::integral_constant<int, 5>());
+    case 6: return run(std::integral_constant<int, 6>());
+    case 7: case 8: return run(std::integral_constant<int, 8>());
+    case 9: case 10: case 11: case 12: return run(std::integral_constant<int, 12>());
+    case 13: case 14: case 15: case 16: return run(std::integral_constant<int, 16>());
+  }
+  return set_error(ST_UNSUPPORTED, "rms_bwd: n_embd above 4096");
+}
+
 static const int kNormBwdBlocks = 296;
 
 int launch_norm_bwd(const float* dy, const float* x, const float* mean, const float* rstd, const float* g, int ln,
@@ -907,6 +1000,31 @@ int launch_init_normal(float* params, long long off, long long n, unsigned long 
   if (grid > num_sms() * 16) grid = num_sms() * 16;
   Prof prof(PK_MISC, 0, n * 4.0, st);
   init_normal_kernel<<<grid, 256, 0, st>>>(params, off, n, seed, stdv);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+__global__ void sum_parts_kernel(const float* __restrict__ parts, int n_parts, size_t stride, size_t n4,
+                                 float* __restrict__ out) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    float4 a = reinterpret_cast<const float4*>(parts)[i];
+    for (int p = 1; p < n_parts; ++p) {
+      const float4 b = reinterpret_cast<const float4*>(parts + (size_t)p * stride)[i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    reinterpret_cast<float4*>(out)[i] = a;
+  }
+}
+
+int launch_sum_parts(const float* parts, int n_parts, size_t stride, size_t n, float* out, cudaStream_t st) {
+  if (n % 4 || stride % 4) return set_error(ST_INVALID_ARG, "sum_parts: sizes must be multiples of 4");
+  int grid = (int)cdiv((long long)(n / 4), 256);
+  if (grid > num_sms() * 8) grid = num_sms() * 8;
+  Prof prof(PK_MISC, 0, (double)n * 4 * (n_parts + 1), st);
+  sum_parts_kernel<<<grid, 256, 0, st>>>(parts, n_parts, stride, n / 4, out);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }

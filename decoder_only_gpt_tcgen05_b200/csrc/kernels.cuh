@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <vector>
 
 #include "ptx.cuh"
 
@@ -30,6 +31,12 @@ int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b
 int launch_norm_bwd(const float* dy, const float* x, const float* mean, const float* rstd, const float* g, int ln,
                     int M, int D, float* dres, int dres_init, __nv_bfloat16* dres_bf, float* dg_part,
                     float* db_part, int* nblk_out, cudaStream_t st);
+// RMSNorm backward from the saved bf16 output y (= x rstd): dres (+)= rstd (dy - y mean(dy y)),
+// with a bf16 copy; dy bf16 (dy_bf16 != 0) or fp32
+int launch_rms_bwd(const void* dy, int dy_bf16, const __nv_bfloat16* y, const float* rstd, int M, int D,
+                   float* dres, int dres_init, __nv_bfloat16* dres_bf, cudaStream_t st);
+// out[i] = sum over p < n_parts of parts[p * stride + i], i < n, added in part order
+int launch_sum_parts(const float* parts, int n_parts, size_t stride, size_t n, float* out, cudaStream_t st);
 // out[c] (+)= sum_r part[r][c]  (fixed order)
 int launch_colreduce(const float* part, int R, int N, float* out, int accumulate, cudaStream_t st);
 // column sums of an [M, N] matrix into per-chunk partials (returns the number of chunks)
@@ -78,11 +85,26 @@ int launch_adamw(float* params, const float* grads, float* m, float* v, long lon
                  const unsigned char* run_decay, int n_runs, long long step, const gpt_adamw& h, void* scratch,
                  double* grad_norm, cudaStream_t st);
 
+// ---- Muon step of the block matrices (muon.cu): matrix q is params[offs[q] ...] with shape
+// [rows[q], cols[q]]; mom holds the momentum at the same offsets
+size_t muon_scratch_bytes(const std::vector<long long>& offs, const std::vector<int>& rows,
+                          const std::vector<int>& cols);
+int launch_muon(float* params, const float* grads, float* mom, const std::vector<long long>& offs,
+                const std::vector<int>& rows, const std::vector<int>& cols, const gpt_muon& h, void* scratch,
+                cudaStream_t st);
+
+// ---- 8-bit casts (fp8.cu): amax = max |x|, s = FP8_MAX / amax, out = cast(x s), inv_scale = 1 / s
+int launch_fp8_quantize(const void* x, int x_fp32, long long n, int fmt, void* out, float* amax, float* inv_scale,
+                        cudaStream_t st);
+
 // ---- attention (attention.cu)
 struct AttnShape {
   int B, T, H, hd, hdp;
   long long ld_qkv;  // pitch (elements) between tokens in the padded q|k|v buffer: 3*H*hdp
+  int win;           // left window: query i sees keys i - win .. i (-1: every key up to i)
 };
+// (query, key) pairs a causal attention of T tokens with left window win (-1: none) scores
+double attn_pairs(int T, int win);
 int launch_attn_fwd(const __nv_bfloat16* qkv_pad, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
                     cudaStream_t st);
 int launch_attn_bwd(const __nv_bfloat16* qkv_pad, const __nv_bfloat16* do_pad, const float* lse,

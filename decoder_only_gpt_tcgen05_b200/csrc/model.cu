@@ -9,8 +9,8 @@
 // per row over each vocab tile, so the logits never reach memory.
 //
 // Backward: cross-entropy gradient tiles (recomputed logits, softmax - onehot, bf16
-// dlogits for a block of rows: all of them when they fit in 4 GiB) feed the lm_head
-// data- and weight-gradient GEMMs; each layer then runs
+// dlogits for a block of rows, at most 512 MiB of them) feed the lm_head data- and
+// weight-gradient GEMMs; each layer then runs
 // its GEMM gradients (MN-major operands, no transposes), the activation gradient in
 // the data-gradient epilogue, the flash-attention backward, the QK-norm/RoPE
 // reverse, the norm backward with the residual add, and finally the deterministic
@@ -47,6 +47,7 @@ struct Layout {
   std::vector<ParamInfo> list;
   long long wte = -1, wpe = -1, lnf_g = -1, lnf_b = -1, lm_head = -1;
   std::vector<LayerOff> layer;
+  std::vector<long long> layer_begin, layer_end;  // element range of each layer's tensors
   long long total = 0;
 };
 
@@ -65,6 +66,7 @@ static Layout make_layout(const gpt_config& c) {
   if (c.pos == 0) L.wpe = add_param(L, "wpe", c.block_size, D);
   for (int l = 0; l < c.n_layer; ++l) {
     LayerOff o;
+    L.layer_begin.push_back(L.total);
     const std::string p = "h" + std::to_string(l) + ".";
     if (ln) {
       o.ln1_g = add_param(L, p + "ln1_g", D, 1);
@@ -83,6 +85,7 @@ static Layout make_layout(const gpt_config& c) {
     o.w_down = add_param(L, p + "w_down", D, F);
     if (bias) o.b_down = add_param(L, p + "b_down", D, 1);
     L.layer.push_back(o);
+    L.layer_end.push_back(L.total);
   }
   if (ln) {
     L.lnf_g = add_param(L, "lnf_g", D, 1);
@@ -90,6 +93,23 @@ static Layout make_layout(const gpt_config& c) {
   }
   if (!c.tie_embed) L.lm_head = add_param(L, "lm_head", V, D);
   return L;
+}
+
+// Gradient buckets in the order the backward completes them: the final norm and an untied
+// lm_head (after the lm_head backward), then the layers in pairs from the top (the weight
+// gradients of an odd layer are launched together with those of the even layer below it), then
+// the embeddings (and a tied lm_head, whose table they share).  Each is one contiguous range.
+struct Bucket {
+  long long begin, end;
+};
+static std::vector<Bucket> grad_buckets(const gpt_config& c, const Layout& L) {
+  std::vector<Bucket> b;
+  const long long head = L.lnf_g >= 0 ? L.lnf_g : (c.tie_embed ? L.total : L.lm_head);
+  b.push_back(Bucket{head, L.total});  // may be empty (tied, no LayerNorm)
+  for (int l = c.n_layer - 1; l >= 0; --l)
+    if (!((l & 1) && l > 0)) b.push_back(Bucket{L.layer_begin[l], L.layer_end[(l + 1 < c.n_layer && (l + 1) & 1) ? l + 1 : l]});
+  b.push_back(Bucket{0, L.layer_begin[0]});
+  return b;
 }
 
 static int validate(const gpt_config* c) {
@@ -107,7 +127,17 @@ static int validate(const gpt_config* c) {
   if (hd % 2 || hd > 128) return set_error(ST_UNSUPPORTED, "config: head dim must be even and at most 128");
   if ((c->pos == 1 || c->qk_norm) && hd != 64 && hd != 128)
     return set_error(ST_UNSUPPORTED, "config: RoPE / QK-norm need a head dim of 64 or 128");
+  if (c->window_short < 0 || c->window_period < 1 || c->window_period > 32)
+    return set_error(ST_INVALID_ARG, "config: window_short must be >= 0 and window_period in 1..32");
+  if (c->fp8 != 0 && c->fp8 != 1) return set_error(ST_INVALID_ARG, "config: fp8 must be 0 or 1");
   return ST_OK;
+}
+
+// left window of layer l's attention (-1: every earlier key), from the layer pattern
+static int layer_window(const gpt_config& c, int l) {
+  if (c.window_short > 0 && ((static_cast<unsigned>(c.window_pattern) >> (l % c.window_period)) & 1u))
+    return c.window_short;
+  return -1;
 }
 
 // ------------------------------------------------------------------ workspace plan
@@ -116,11 +146,13 @@ static inline size_t al(size_t x) { return (x + 255) & ~size_t(255); }
 
 struct Plan {
   int B, T, M, D, H, hd, hdp, F, L, V, Vp, ntn, Mc;
+  int nsplit, ks;  // vocabulary pieces of the lm_head logits-gradient product and their K
   long long P;
   // byte offsets into the workspace
   size_t wbf, rope_cs, idx, tgt, xs, a1, st1, qkv, rq, rk, o, lse, a2, st2, u, h, af, stf;
   size_t ce_part, zy, ell, lse_ce, loss_d, loss_i, loss_f;
-  size_t dlog, da, dres, dres_bf, du, do_pad, delta, dqkv_pad, dqkv, part_a, part_b, embed;
+  size_t f8w, f8a, f8s;  // 8-bit block weights, one 8-bit activation, (amax, 1/scale) pairs
+  size_t dlog, da_parts, da, dres, dres_bf, du, do_pad, delta, dqkv_pad, dqkv, part_a, part_b, embed;
   size_t total;
   long long partN;
 };
@@ -139,14 +171,15 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   p.V = c.vocab_size;
   p.Vp = (c.vocab_size + 7) / 8 * 8;
   p.ntn = (c.vocab_size + 255) / 256;
-  // lm_head backward row chunk: every row at once when their bf16 dlogits fit in 4 GiB (then the
-  // three lm_head products fill their waves: with 4096-row chunks the logits-gradient product
-  // d af = dlogits W_lm had 80 tiles of 256 x 256 for 74 CTA pairs), else the largest multiple
-  // of 4096 rows that fits
+  // lm_head backward row block: the bf16 dlogits of one block of rows stay within 512 MiB (8192
+  // rows at V = 32768), so the whole M x V gradient is never held.  The logits-gradient product
+  // d af = dlogits W_lm of a block is split along the vocabulary into pieces that run as one
+  // grouped launch (a 256-row-tile product over 1280 columns alone would leave most SM pairs
+  // idle in its last wave).
   {
-    const long long cap = (4LL << 30) / ((long long)p.Vp * 2);
-    long long mc = cap / 4096 * 4096;
-    if (mc < 4096) mc = 4096;
+    const long long cap = (512LL << 20) / ((long long)p.Vp * 2);
+    long long mc = cap / 256 * 256;
+    if (mc < 256) mc = 256;
     // GPT_LM_CHUNK_ROWS=<n> forces n-row blocks (tests of the blocked path on small batches)
     static const long long forced = []() {
       const char* e = std::getenv("GPT_LM_CHUNK_ROWS");
@@ -154,6 +187,12 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
     }();
     if (forced > 0) mc = forced;
     p.Mc = (int)(mc < p.M ? mc : p.M);
+    // vocabulary pieces of d af = dlogits W_lm: about one block's rows of K each, at most 8
+    int ns = (p.V + p.Mc - 1) / p.Mc;
+    if (ns > kMaxProblems) ns = kMaxProblems;
+    if (ns < 1) ns = 1;
+    p.ks = ((p.V + ns - 1) / ns + 63) / 64 * 64;
+    p.nsplit = (p.V + p.ks - 1) / p.ks;
   }
   p.P = P;
   const size_t M = p.M, D = p.D, F = p.F, L = p.L, H = p.H, hdp = p.hdp;
@@ -188,6 +227,13 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   p.loss_d = take(loss_reduce_blocks() * 2 * 8);
   p.loss_i = take(loss_reduce_blocks() * 2 * 8);
   p.loss_f = take(64);
+  if (c.fp8) {
+    p.f8w = take((size_t)L * 12 * D * D);               // w_qkv, w_o, w_up, w_down of every layer
+    p.f8a = take(M * (F > D ? F : D));
+    p.f8s = take((size_t)(4 * L + 4) * 2 * 4);
+  } else {
+    p.f8w = p.f8a = p.f8s = 0;
+  }
   p.dlog = take((size_t)p.Mc * p.Vp * 2);
   p.da = take(M * D * 4);
   p.dres = take(M * D * 4);
@@ -195,6 +241,12 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   // layers' weight gradients is launched together
   p.dres_bf = take(4 * M * D * 2);  // [slot][sublayer]
   p.du = take(2 * M * F * 2);
+  // the lm_head backward's per-piece d af buffers: in du, which is idle until the first layer's
+  // backward, when it is large enough
+  {
+    const size_t need = p.nsplit > 1 ? (size_t)p.nsplit * p.Mc * p.D * 4 : 256;
+    p.da_parts = need <= 2 * M * F * 2 ? p.du : take(need);
+  }
   p.do_pad = take(M * H * hdp * 2);
   p.delta = take(M * H * 4);
   p.dqkv_pad = take((p.hdp == p.hd ? 2 : 1) * M * 3 * H * hdp * 2);  // [slot] when it is dqkv itself
@@ -261,6 +313,36 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
   GPTK_TRY(launch_cast_bf16(params, wbf, pl.P, st));
   if (c.pos == 1) GPTK_TRY(launch_rope_table(cs, T, hd / 2, (double)c.rope_base, st));
 
+  // 8-bit forward projections: every block weight cast once per forward, each with its own scale;
+  // the activation operand of each projection is cast just before its product
+  uint8_t* f8w = c.fp8 ? at<uint8_t>(ws, pl.f8w) : nullptr;
+  uint8_t* f8a = c.fp8 ? at<uint8_t>(ws, pl.f8a) : nullptr;
+  float* f8s = c.fp8 ? at<float>(ws, pl.f8s) : nullptr;  // [slot][amax, 1/scale]
+  const size_t DD = (size_t)D * D;
+  auto f8w_of = [&](int l, int which) {  // which: 0 qkv, 1 o, 2 up, 3 down
+    const size_t off[4] = {0, 3 * DD, 4 * DD, 8 * DD};
+    return f8w + (size_t)l * 12 * DD + off[which];
+  };
+  if (c.fp8) {
+    for (int l = 0; l < pl.L; ++l) {
+      const LayerOff& o = Lo.layer[l];
+      const long long offs[4] = {o.w_qkv, o.w_o, o.w_up, o.w_down};
+      const size_t sizes[4] = {3 * DD, DD, 4 * DD, 4 * DD};
+      for (int w = 0; w < 4; ++w)
+        GPTK_TRY(launch_fp8_quantize(params + offs[w], 1, (long long)sizes[w], 0, f8w_of(l, w),
+                                     f8s + 2 * (4 * l + w), f8s + 2 * (4 * l + w) + 1, st));
+    }
+  }
+  // the 8-bit operands of one projection: the activation act [M, K] cast into f8a (slot 4L + k)
+  auto f8_setup = [&](GemmParams& p, const __nv_bfloat16* act, long long n, int l, int which, int k) -> int {
+    float* sa = f8s + 2 * (4 * pl.L + k);
+    GPTK_TRY(launch_fp8_quantize(act, 0, n, 0, f8a, sa, sa + 1, st));
+    p.f8_fmt_a = p.f8_fmt_b = 0;
+    p.f8_inv_a = sa + 1;
+    p.f8_inv_b = f8s + 2 * (4 * l + which) + 1;
+    return ST_OK;
+  };
+
   float* xs = at<float>(ws, pl.xs);
   const size_t MD = (size_t)M * D;
   GPTK_TRY(launch_embed_fwd(idx_ws, params + Lo.wte, Lo.wpe >= 0 ? params + Lo.wpe : nullptr, xs, M, T, D, V, st));
@@ -297,6 +379,12 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
       p.ldo = 3LL * D;
       p.bias = o.b_qkv >= 0 ? params + o.b_qkv : nullptr;
       p.prof_kind = PK_GEMM_QKV;
+      Operand qa{a1, D, 0}, qb{wbf + o.w_qkv, D, 0};
+      if (c.fp8) {
+        GPTK_TRY(f8_setup(p, a1, (long long)MD, l, 0, 0));
+        qa = Operand{f8a, D, 0};
+        qb = Operand{f8w_of(l, 0), D, 0};
+      }
       if (fused) {
         p.rope_cs = cs;
         p.rope_T = T;
@@ -307,15 +395,15 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
         p.qk_eps = c.norm_eps;
         p.rstd_q = rq;
         p.rstd_k = rk;
-        GPTK_TRY(gemm(EPI_QKV, Operand{a1, D, 0}, Operand{wbf + o.w_qkv, D, 0}, p, st, 256));
+        GPTK_TRY(gemm(EPI_QKV, qa, qb, p, st, 256));
       } else {
-        GPTK_TRY(gemm(EPI_BF16, Operand{a1, D, 0}, Operand{wbf + o.w_qkv, D, 0}, p, st));
+        GPTK_TRY(gemm(EPI_BF16, qa, qb, p, st));
         if (padded) GPTK_CUDA(cudaMemsetAsync(qkv, 0, (size_t)M * 3 * H * hdp * 2, st));
         if (padded || c.pos == 1 || c.qk_norm)
           GPTK_TRY(launch_qk_fwd(raw, cs, M, T, H, hd, hdp, c.pos == 1, c.qk_norm, c.norm_eps, qkv, rq, rk, st));
       }
     }
-    AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp};
+    AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp, layer_window(c, l)};
     GPTK_TRY(launch_attn_fwd(qkv, as, ob, D, lse, st));
     {
       GemmParams p = gp(M, D, D);
@@ -325,7 +413,12 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
       p.ldr = D;
       p.bias = o.b_o >= 0 ? params + o.b_o : nullptr;
       p.prof_kind = PK_GEMM_O;
-      GPTK_TRY(gemm(EPI_RESID, Operand{ob, D, 0}, Operand{wbf + o.w_o, D, 0}, p, st));
+      if (c.fp8) {
+        GPTK_TRY(f8_setup(p, ob, (long long)MD, l, 1, 1));
+        GPTK_TRY(gemm(EPI_RESID, Operand{f8a, D, 0}, Operand{f8w_of(l, 1), D, 0}, p, st));
+      } else {
+        GPTK_TRY(gemm(EPI_RESID, Operand{ob, D, 0}, Operand{wbf + o.w_o, D, 0}, p, st));
+      }
     }
     // MLP sublayer
     GPTK_TRY(launch_norm_fwd(x_mid, M, D, ln ? params + o.ln2_g : nullptr, o.ln2_b >= 0 ? params + o.ln2_b : nullptr,
@@ -338,7 +431,12 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
       p.act = c.act;
       p.bias = o.b_up >= 0 ? params + o.b_up : nullptr;
       p.prof_kind = PK_GEMM_UP;
-      GPTK_TRY(gemm(EPI_UP, Operand{a2, D, 0}, Operand{wbf + o.w_up, D, 0}, p, st));
+      if (c.fp8) {
+        GPTK_TRY(f8_setup(p, a2, (long long)MD, l, 2, 2));
+        GPTK_TRY(gemm(EPI_UP, Operand{f8a, D, 0}, Operand{f8w_of(l, 2), D, 0}, p, st));
+      } else {
+        GPTK_TRY(gemm(EPI_UP, Operand{a2, D, 0}, Operand{wbf + o.w_up, D, 0}, p, st));
+      }
     }
     {
       GemmParams p = gp(M, D, F);
@@ -348,7 +446,12 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
       p.ldr = D;
       p.bias = o.b_down >= 0 ? params + o.b_down : nullptr;
       p.prof_kind = PK_GEMM_DOWN;
-      GPTK_TRY(gemm(EPI_RESID, Operand{h, F, 0}, Operand{wbf + o.w_down, F, 0}, p, st));
+      if (c.fp8) {
+        GPTK_TRY(f8_setup(p, h, (long long)M * F, l, 3, 3));
+        GPTK_TRY(gemm(EPI_RESID, Operand{f8a, F, 0}, Operand{f8w_of(l, 3), F, 0}, p, st));
+      } else {
+        GPTK_TRY(gemm(EPI_RESID, Operand{h, F, 0}, Operand{wbf + o.w_down, F, 0}, p, st));
+      }
     }
   }
   // final norm + lm_head + cross-entropy
@@ -389,14 +492,19 @@ static int bias_grad_bf16(const __nv_bfloat16* a, int M, int N, float* part, flo
   return launch_colreduce(part, R, N, dst, 1, st);
 }
 
-static int norm_backward(const gpt_config& c, const Plan& pl, const float* dy, const float* x, const float* stats,
-                         const float* params, long long g_off, long long b_off, float* grads, float* dres,
-                         int dres_init, __nv_bfloat16* dres_bf, float* pa, float* pb, cudaStream_t st) {
+// dy: fp32, or bf16 when dy_bf16 (RMSNorm only); y: the saved bf16 output of the forward norm
+static int norm_backward(const gpt_config& c, const Plan& pl, const void* dy, int dy_bf16, const float* x,
+                         const __nv_bfloat16* y, const float* stats, const float* params, long long g_off,
+                         long long b_off, float* grads, float* dres, int dres_init, __nv_bfloat16* dres_bf, float* pa,
+                         float* pb, cudaStream_t st) {
   const int ln = c.norm == 1;
   const int M = pl.M, D = pl.D;
+  // RMSNorm (no gain): the backward needs only the bf16 output and rstd, not the fp32 input
+  if (!ln) return launch_rms_bwd(dy, dy_bf16, y, stats + M, M, D, dres, dres_init, dres_bf, st);
+  if (dy_bf16) return set_error(ST_INVALID_ARG, "LayerNorm backward takes an fp32 dy");
   int nblk = 0;
-  GPTK_TRY(launch_norm_bwd(dy, x, stats, stats + M, ln ? params + g_off : nullptr, ln, M, D, dres, dres_init, dres_bf,
-                           pa, pb, &nblk, st));
+  GPTK_TRY(launch_norm_bwd(static_cast<const float*>(dy), x, stats, stats + M, params + g_off, ln, M, D, dres,
+                           dres_init, dres_bf, pa, pb, &nblk, st));
   if (ln) {
     GPTK_TRY(launch_colreduce(pa, nblk, D, grads + g_off, 1, st));
     if (b_off >= 0) GPTK_TRY(launch_colreduce(pb, nblk, D, grads + b_off, 1, st));
@@ -405,9 +513,16 @@ static int norm_backward(const gpt_config& c, const Plan& pl, const float* dy, c
 }
 
 static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, const float* params, void* ws,
-                         float* grads, int accumulate, cudaStream_t st) {
+                         float* grads, int accumulate, cudaStream_t st, void* const* events = nullptr) {
+  int bucket = 0;  // next gradient bucket to complete (events[bucket] is recorded when it is final)
+  auto done = [&]() -> int {
+    if (events) GPTK_CUDA(cudaEventRecord(static_cast<cudaEvent_t>(events[bucket]), st));
+    ++bucket;
+    return ST_OK;
+  };
   const int M = pl.M, D = pl.D, H = pl.H, hd = pl.hd, hdp = pl.hdp, F = pl.F, T = pl.T, B = pl.B, V = pl.V;
   const size_t MD = (size_t)M * D;
+  const int rms = c.norm == 0;  // RMSNorm: the norm backward reads bf16 data gradients
   __nv_bfloat16* wbf = at<__nv_bfloat16>(ws, pl.wbf);
   const float2* cs = at<float2>(ws, pl.rope_cs);
   const int* idx_ws = at<int>(ws, pl.idx);
@@ -441,9 +556,11 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
 
   if (!accumulate) GPTK_CUDA(cudaMemsetAsync(grads, 0, (size_t)pl.P * 4, st));
 
-  // ---- lm_head + cross-entropy backward, one block of pl.Mc rows at a time (one block for every
-  //      row when the bf16 dlogits fit in 4 GiB)
+  // ---- lm_head + cross-entropy backward, one block of pl.Mc rows at a time: the block's bf16
+  //      dlogits (recomputed logits, softmax - onehot) feed the weight gradient and the
+  //      logits-gradient product, then the next block reuses the buffer
   const long long wlm = c.tie_embed ? Lo.wte : Lo.lm_head;
+  const int nsplit = pl.nsplit, ks = pl.ks;
   for (int r0 = 0; r0 < M; r0 += pl.Mc) {
     const int mc = (M - r0) < pl.Mc ? (M - r0) : pl.Mc;
     {
@@ -464,16 +581,31 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       p.prof_kind = PK_GEMM_WGRAD;
       GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 1}, Operand{af + (size_t)r0 * D, D, 1}, p, st));
     }
-    {  // d af = dlogits W_lm
+    if (nsplit == 1) {  // d af = dlogits W_lm
       GemmParams p = gp(mc, D, V);
       p.out = da + (size_t)r0 * D;
       p.ldo = D;
       p.prof_kind = PK_GEMM_LM_BWD;
       GPTK_TRY(gemm(EPI_F32, Operand{dlog, pl.Vp, 0}, Operand{wbf + wlm, D, 1}, p, st));
+    } else {
+      // d af = sum over vocabulary pieces j of dlogits[:, piece j] W_lm[piece j, :]: each piece to
+      // its own fp32 buffer (stored, not accumulated, so no two tiles add into the same element),
+      // then one pass adds them in piece order: deterministic
+      float* parts = at<float>(ws, pl.da_parts);
+      GroupProblem pieces[kMaxProblems];
+      for (int j = 0; j < nsplit; ++j) {
+        const int k0 = j * ks;
+        const int kext = (V - k0) < ks ? (V - k0) : ks;
+        pieces[j] = GroupProblem{dlog + k0, pl.Vp, wbf + wlm + (size_t)k0 * D, D, mc, D,
+                                 parts + (size_t)j * pl.Mc * D, D, kext};
+      }
+      GPTK_TRY(run_gemm_group(nsplit, pieces, ks, 0, 1, 256, PK_GEMM_LM_BWD, st, EPI_F32, 0));
+      GPTK_TRY(launch_sum_parts(parts, nsplit, (size_t)pl.Mc * D, (size_t)mc * D, da + (size_t)r0 * D, st));
     }
   }
-  GPTK_TRY(norm_backward(c, pl, da, xs + (size_t)(2 * pl.L) * MD, stf, params, Lo.lnf_g, Lo.lnf_b, grads, dres, 1,
+  GPTK_TRY(norm_backward(c, pl, da, 0, xs + (size_t)(2 * pl.L) * MD, af, stf, params, Lo.lnf_g, Lo.lnf_b, grads, dres, 1,
                          dres_bf_mlp_of(pl.L - 1), pa, pb, st));
+  GPTK_TRY(done());  // final norm (+ untied lm_head)
 
   for (int l = pl.L - 1; l >= 0; --l) {
     const LayerOff& o = Lo.layer[l];
@@ -508,15 +640,16 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       GPTK_TRY(gemm(EPI_ACTBWD, Operand{dres_bf_mlp, D, 0}, Operand{wbf + o.w_down, F, 1}, p, st));
     }
     if (o.b_down >= 0) GPTK_TRY(bias_grad_f32(dres, M, D, pa, grads + o.b_down, st));
-    {  // da = du W_up
+    {  // da = du W_up (bf16 for RMSNorm, whose backward reads a bf16 dy)
       GemmParams p = gp(M, D, F);
       p.out = da;
       p.ldo = D;
       p.prof_kind = PK_GEMM_DGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{du, F, 0}, Operand{wbf + o.w_up, D, 1}, p, st));
+      GPTK_TRY(gemm(rms ? EPI_BF16 : EPI_F32, Operand{du, F, 0}, Operand{wbf + o.w_up, D, 1}, p, st));
     }
     if (o.b_up >= 0) GPTK_TRY(bias_grad_bf16(du, M, F, pa, grads + o.b_up, st));
-    GPTK_TRY(norm_backward(c, pl, da, x_mid, st2, params, o.ln2_g, o.ln2_b, grads, dres, 0, dres_bf_att, pa, pb, st));
+    GPTK_TRY(norm_backward(c, pl, da, rms, x_mid, a2, st2, params, o.ln2_g, o.ln2_b, grads, dres, 0, dres_bf_att, pa,
+                           pb, st));
 
     // ---- attention: x_mid = x_in + attn(N(x_in)) W_o^T + b_o
     if (hdp != hd) GPTK_CUDA(cudaMemsetAsync(do_pad, 0, (size_t)M * H * hdp * 2, st));
@@ -531,15 +664,15 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
     }
     if (o.b_o >= 0) GPTK_TRY(bias_grad_f32(dres, M, D, pa, grads + o.b_o, st));
     GPTK_TRY(launch_attn_delta(ob, do_pad, B, T, H, hd, hdp, delta, st));
-    AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp};
+    AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp, layer_window(c, l)};
     GPTK_TRY(launch_attn_bwd(qkv, do_pad, lse, delta, as, dqkv_pad, st));
     GPTK_TRY(launch_qk_bwd(dqkv_pad, qkv, rq, rk, cs, M, T, H, hd, hdp, c.pos == 1, c.qk_norm, dqkv, st));
-    {  // da = dqkv W_qkv
+    {  // da = dqkv W_qkv (bf16 for RMSNorm)
       GemmParams p = gp(M, D, 3 * D);
       p.out = da;
       p.ldo = D;
       p.prof_kind = PK_GEMM_DGRAD;
-      GPTK_TRY(gemm(EPI_F32, Operand{dqkv, 3LL * D, 0}, Operand{wbf + o.w_qkv, D, 1}, p, st));
+      GPTK_TRY(gemm(rms ? EPI_BF16 : EPI_F32, Operand{dqkv, 3LL * D, 0}, Operand{wbf + o.w_qkv, D, 1}, p, st));
     }
     if (o.b_qkv >= 0) GPTK_TRY(bias_grad_bf16(dqkv, M, 3 * D, pa, grads + o.b_qkv, st));
     {  // the layer's four weight gradients W += dY^T X over all tokens, launched together with the
@@ -562,13 +695,14 @@ static int backward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, 
       }
     }
     // the residual gradient of the layer below goes to that layer's slot
-    GPTK_TRY(norm_backward(c, pl, da, x_in, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0,
+    GPTK_TRY(norm_backward(c, pl, da, rms, x_in, a1, st1, params, o.ln1_g, o.ln1_b, grads, dres, 0,
                            l > 0 ? dres_bf_mlp_of(l - 1) : dres_bf_mlp_of(0), pa, pb, st));
+    if (!((l & 1) && l > 0)) GPTK_TRY(done());  // this layer (and the odd one above it)
   }
   // ---- embeddings
   GPTK_TRY(launch_embed_bwd(idx_ws, dres, M, D, V, grads + Lo.wte, at<void>(ws, pl.embed), st));
   if (Lo.wpe >= 0) GPTK_TRY(launch_pos_bwd(dres, B, T, D, grads + Lo.wpe, 1, st));
-  return ST_OK;
+  return done();  // embeddings
 }
 
 // ------------------------------------------------------------------ init
@@ -654,6 +788,83 @@ GPT_API int gpt_adamw_step(const gpt_config* cfg, float* params, const float* gr
                       grad_norm, static_cast<cudaStream_t>(stream));
 }
 
+// The Muon matrices of a layout (block Linear weights) and the runs of every other tensor
+static void muon_split(const Layout& L, std::vector<long long>& offs, std::vector<int>& rows,
+                       std::vector<int>& cols, std::vector<std::vector<const ParamInfo*>>& adam_ranges) {
+  std::vector<const ParamInfo*> cur;
+  for (const ParamInfo& p : L.list) {
+    const std::string base = p.name.substr(p.name.find('.') == std::string::npos ? 0 : p.name.find('.') + 1);
+    const bool muon = base == "w_qkv" || base == "w_o" || base == "w_up" || base == "w_down";
+    if (muon) {
+      offs.push_back(p.off);
+      rows.push_back((int)p.rows);
+      cols.push_back((int)p.cols);
+      if (!cur.empty()) adam_ranges.push_back(cur);
+      cur.clear();
+    } else {
+      cur.push_back(&p);
+    }
+  }
+  if (!cur.empty()) adam_ranges.push_back(cur);
+}
+
+GPT_API int gpt_muon_scratch_size(const gpt_config* cfg, size_t* bytes) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!bytes) return set_error(ST_INVALID_ARG, "null output");
+  Layout L = make_layout(*cfg);
+  std::vector<long long> offs;
+  std::vector<int> rows, cols;
+  std::vector<std::vector<const ParamInfo*>> ranges;
+  muon_split(L, offs, rows, cols, ranges);
+  *bytes = muon_scratch_bytes(offs, rows, cols);
+  return ST_OK;
+}
+
+GPT_API int gpt_muon_step(const gpt_config* cfg, float* params, const float* grads, float* mom, float* v,
+                          int64_t step, const gpt_muon* h, void* scratch, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!h) return set_error(ST_INVALID_ARG, "gpt_muon_step: null hyperparameters");
+  if (!params || !grads || !mom || !v || !scratch) return set_error(ST_INVALID_ARG, "gpt_muon_step: null pointer");
+  if (reinterpret_cast<uintptr_t>(scratch) & 255) return set_error(ST_INVALID_ARG, "gpt_muon_step: scratch alignment");
+  for (const void* q : {(const void*)params, (const void*)grads, (const void*)mom, (const void*)v})
+    if (reinterpret_cast<uintptr_t>(q) & 15) return set_error(ST_INVALID_ARG, "gpt_muon_step: 16-byte alignment");
+  if (step < 1) return set_error(ST_INVALID_ARG, "gpt_muon_step: step must be >= 1");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Layout L = make_layout(*cfg);
+  std::vector<long long> offs;
+  std::vector<int> rows, cols;
+  std::vector<std::vector<const ParamInfo*>> ranges;
+  muon_split(L, offs, rows, cols, ranges);
+  // AdamW on every other tensor, one launch pair per contiguous range (decay on 2-D tensors);
+  // the AdamW scratch is the start of the Muon scratch
+  gpt_adamw ah;
+  ah.lr = h->adam_lr;
+  ah.beta1 = h->beta1;
+  ah.beta2 = h->beta2;
+  ah.eps = h->eps;
+  ah.weight_decay = h->weight_decay;
+  ah.grad_scale = 1.f;
+  ah.grad_clip = 0.f;
+  for (const auto& rg : ranges) {
+    const long long r0 = rg.front()->off;
+    const long long n = rg.back()->off + rg.back()->rows * rg.back()->cols - r0;
+    std::vector<long long> start;
+    std::vector<unsigned char> decay;
+    for (const ParamInfo* p : rg) {
+      const unsigned char d = p->cols > 1 ? 1 : 0;
+      if (decay.empty() || decay.back() != d) {
+        start.push_back(p->off - r0);
+        decay.push_back(d);
+      }
+    }
+    GPTK_TRY(launch_adamw(params + r0, grads + r0, mom + r0, v + r0, n, start.data(), decay.data(), (int)start.size(),
+                          step, ah, scratch, nullptr, st));
+  }
+  return launch_muon(params, grads, mom, offs, rows, cols, *h, scratch, st);
+}
+
 GPT_API int gpt_workspace_size(const gpt_config* cfg, int32_t B, int32_t T, size_t* bytes) {
   set_error(ST_OK, "");
   GPTK_TRY(validate(cfg));
@@ -704,6 +915,40 @@ GPT_API int gpt_backward(const gpt_config* cfg, const float* params, int32_t B, 
   Plan pl = make_plan(*cfg, B, T, L.total);
   GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
   return backward_impl(*cfg, L, pl, params, workspace, grads, accumulate, static_cast<cudaStream_t>(stream));
+}
+
+GPT_API int gpt_grad_buckets(const gpt_config* cfg, int32_t max_buckets, int32_t* n_out, int64_t* begin,
+                             int64_t* end) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  if (!n_out) return set_error(ST_INVALID_ARG, "null output");
+  const std::vector<Bucket> b = grad_buckets(*cfg, make_layout(*cfg));
+  *n_out = (int32_t)b.size();
+  if (max_buckets < (int32_t)b.size() && (begin || end))
+    return set_error(ST_INVALID_ARG, "gpt_grad_buckets: room for " + std::to_string(max_buckets) + " buckets, " +
+                                         std::to_string(b.size()) + " needed");
+  for (size_t k = 0; k < b.size(); ++k) {
+    if (begin) begin[k] = b[k].begin;
+    if (end) end[k] = b[k].end;
+  }
+  return ST_OK;
+}
+
+GPT_API int gpt_backward_bucketed(const gpt_config* cfg, const float* params, int32_t B, int32_t T, void* workspace,
+                                  size_t workspace_bytes, float* grads, int32_t accumulate, void* const* events,
+                                  int32_t n_events, void* stream) {
+  set_error(ST_OK, "");
+  GPTK_TRY(validate(cfg));
+  GPTK_TRY(check_batch(cfg, B, T));
+  if (!params || !grads || !events) return set_error(ST_INVALID_ARG, "null pointer");
+  Layout L = make_layout(*cfg);
+  if (n_events != (int32_t)grad_buckets(*cfg, L).size())
+    return set_error(ST_INVALID_ARG, "gpt_backward_bucketed: one event per gradient bucket (gpt_grad_buckets)");
+  for (int32_t k = 0; k < n_events; ++k)
+    if (!events[k]) return set_error(ST_INVALID_ARG, "gpt_backward_bucketed: null event");
+  Plan pl = make_plan(*cfg, B, T, L.total);
+  GPTK_TRY(check_ws(workspace, workspace_bytes, pl.total));
+  return backward_impl(*cfg, L, pl, params, workspace, grads, accumulate, static_cast<cudaStream_t>(stream), events);
 }
 
 GPT_API int gpt_eval_bpb(const gpt_config* cfg, const float* params, const int32_t* idx, const int32_t* targets,

@@ -313,6 +313,43 @@ __device__ __forceinline__ void umma8_ts(const uint32_t (&d)[8], const uint32_t 
       : "memory");
 }
 
+// Four MMAs of kind::f8f6f4 (8-bit A and B, fp32 accumulate, K = 32 each), back to back; the
+// pair form is the cta_group::2 MMA of a CTA pair.  The formats are in the instruction descriptor.
+__device__ __forceinline__ void umma4_f8(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4], uint32_t idesc,
+                                         uint32_t acc_mask) {
+  asm volatile(
+      "{\n\t.reg .pred p<4>;\n\t.reg .b32 t<4>;\n\t"
+      "and.b32 t0, %10, 1;\n\tsetp.ne.b32 p0, t0, 0;\n\t"
+      "and.b32 t1, %10, 2;\n\tsetp.ne.b32 p1, t1, 0;\n\t"
+      "and.b32 t2, %10, 4;\n\tsetp.ne.b32 p2, t2, 0;\n\t"
+      "and.b32 t3, %10, 8;\n\tsetp.ne.b32 p3, t3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %5, %9, p0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %6, %9, p1;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %3, %7, %9, p2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %8, %9, p3;\n\t"
+      "}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc),
+      "r"(acc_mask)
+      : "memory");
+}
+__device__ __forceinline__ void umma4_f8_pair(uint32_t d, const uint64_t (&a)[4], const uint64_t (&b)[4],
+                                              uint32_t idesc, uint32_t acc_mask) {
+  asm volatile(
+      "{\n\t.reg .pred p<4>;\n\t.reg .b32 t<4>;\n\t"
+      "and.b32 t0, %10, 1;\n\tsetp.ne.b32 p0, t0, 0;\n\t"
+      "and.b32 t1, %10, 2;\n\tsetp.ne.b32 p1, t1, 0;\n\t"
+      "and.b32 t2, %10, 4;\n\tsetp.ne.b32 p2, t2, 0;\n\t"
+      "and.b32 t3, %10, 8;\n\tsetp.ne.b32 p3, t3, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %5, %9, p0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %2, %6, %9, p1;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %3, %7, %9, p2;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %4, %8, %9, p3;\n\t"
+      "}"
+      ::"r"(d), "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "r"(idesc),
+      "r"(acc_mask)
+      : "memory");
+}
+
 // Arrive once on the mbarrier at `bar_cluster` (either CTA of the pair) when every pair MMA
 // issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar_cluster) {
@@ -342,6 +379,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn) << 15) |
          (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator, A and B in the 8-bit formats fa, fb
+// (0 = e4m3, 1 = e5m2), both K-major.
+__host__ __device__ constexpr uint32_t idesc_f8(int M, int N, int fa, int fb) {
+  return (1u << 4) | (static_cast<uint32_t>(fa) << 7) | (static_cast<uint32_t>(fb) << 10) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// fp32 pair -> two 8-bit floats (round to nearest even, saturating at the largest finite value);
+// the first value in the low byte
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint16_t cvt_e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand.
@@ -460,6 +517,34 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100 f32x2 instructions: one instruction for two lanes' worth of work).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 pa, pb, pc;\n\tmov.b64 pa, {%1, %2};\n\tmov.b64 pb, {%3, %4};\n\tmov.b64 pc, {%5, %6};\n\t"
+      "fma.rn.f32x2 %0, pa, pb, pc;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 pa, pb;\n\tmov.b64 pa, {%1, %2};\n\tmov.b64 pb, {%3, %4};\n\t"
+      "add.rn.f32x2 %0, pa, pb;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Hardware square root (sqrt.approx: +0 maps to +0; its error of a few ulp is far below bf16

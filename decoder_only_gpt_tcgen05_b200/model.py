@@ -21,7 +21,8 @@ ACT_GELU, ACT_RELU2 = 0, 1
 class _CConfig(C.Structure):
     _fields_ = [(n, C.c_int32) for n in ("n_layer", "n_embd", "n_head", "block_size", "vocab_size", "norm", "pos",
                                          "act", "tie_embed", "qk_norm", "linear_bias", "scale_resid_init")] + \
-               [("rope_base", C.c_float), ("norm_eps", C.c_float)]
+               [("rope_base", C.c_float), ("norm_eps", C.c_float)] + \
+               [(n, C.c_int32) for n in ("window_short", "window_pattern", "window_period", "fp8")]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -40,6 +41,10 @@ class GPTConfig:
     scale_resid_init: int = 0
     rope_base: float = 10000.0
     norm_eps: float = 1e-5
+    window_short: int = 0     # > 0: left window of the short-window ('S') layers
+    window_pattern: int = 0   # bit (l mod window_period) set: layer l is a short-window layer
+    window_period: int = 1
+    fp8: int = 0              # 1: the forward's block projections on e4m3 operands
 
     def c(self) -> _CConfig:
         return _CConfig(**dataclasses.asdict(self))
@@ -57,6 +62,11 @@ PRESETS = {
     "d26": GPTConfig(n_layer=26, n_embd=1664, n_head=13, block_size=2048, vocab_size=32768, norm=NORM_RMS,
                      pos=POS_ROPE, act=ACT_RELU2, tie_embed=0, qk_norm=1),
 }
+
+
+def pattern_bits(pattern: str) -> int:
+    """window_pattern of a layer pattern string such as "SSSL" (bit i set for an 'S')."""
+    return sum(1 << i for i, ch in enumerate(pattern) if ch == "S")
 
 
 def preset(name: str, **over) -> GPTConfig:

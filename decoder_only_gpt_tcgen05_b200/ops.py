@@ -31,13 +31,43 @@ def gemm(a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, *, a_mn: bool = Fa
     return out
 
 
+FP8_E4M3, FP8_E5M2 = 0, 1
+
+
+def fp8_quantize(x: torch.Tensor, fmt: int = FP8_E4M3, out: torch.Tensor | None = None):
+    """(q uint8 same shape as x, amax fp32 [1], inv_scale fp32 [1]): x cast to 8-bit floats with the
+    per-tensor scale FP8_MAX / max|x|.  x: contiguous bf16 or fp32."""
+    assert x.is_contiguous() and x.dtype in (torch.bfloat16, torch.float32)
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device) if out is None else out
+    assert q.dtype == torch.uint8 and q.is_contiguous() and q.numel() == x.numel()
+    amax = torch.empty(1, dtype=torch.float32, device=x.device)
+    inv = torch.empty(1, dtype=torch.float32, device=x.device)
+    call("gpt_op_fp8_quantize", x.data_ptr(), int(x.dtype == torch.float32), x.numel(), fmt, q.data_ptr(),
+         amax.data_ptr(), inv.data_ptr(), _stream(x))
+    return q, amax, inv
+
+
+def gemm_fp8(a: torch.Tensor, fmt_a: int, inv_a: torch.Tensor, b: torch.Tensor, fmt_b: int, inv_b: torch.Tensor,
+             out: torch.Tensor, *, bias: torch.Tensor | None = None, accumulate: bool = False, bn: int = 256):
+    """out[M,N] = (A B^T) inv_a inv_b for 8-bit (uint8-stored) A [M,K], B [N,K], both K-major."""
+    assert a.dtype == torch.uint8 and b.dtype == torch.uint8 and a.shape[1] == b.shape[1]
+    M, K = a.shape
+    N = b.shape[0]
+    epi = GEMM_OUT_F32 if out.dtype == torch.float32 else GEMM_OUT_BF16
+    call("gpt_op_gemm_fp8", epi, bn, a.data_ptr(), a.stride(0), fmt_a, b.data_ptr(), b.stride(0), fmt_b, M, N, K,
+         inv_a.data_ptr(), inv_b.data_ptr(), out.data_ptr(), out.stride(0),
+         bias.data_ptr() if bias is not None else None, int(accumulate), _stream(out))
+    return out
+
+
 def _ptr(t):
     return t.data_ptr() if t is not None else None
 
 
 def attention_fwd(qkv: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: bool = True, qk_norm: bool = True,
-                  rope_base: float = 10000.0, eps: float = 1e-5, out: dict | None = None):
-    """RoPE + QK-norm + causal attention.  qkv: bf16 [B*T, 3*H*hd] (raw).
+                  window: int = -1, rope_base: float = 10000.0, eps: float = 1e-5, out: dict | None = None):
+    """RoPE + QK-norm + causal attention.  qkv: bf16 [B*T, 3*H*hd] (raw).  window >= 0 limits
+    query i to keys i - window .. i (-1: every earlier key).
     Returns a dict with qkv_norm, rstd_q, rstd_k, rope_cs, o, lse; ``out``, a
     dict returned by an earlier call with the same sizes, is written again
     instead of allocating."""
@@ -54,14 +84,14 @@ def attention_fwd(qkv: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: b
     assert r["qkv_norm"].numel() >= M * 3 * H * hd and r["o"].numel() >= M * H * hd and r["lse"].numel() >= M * H
     assert not rope or r["rope_cs"].numel() >= T * hd
     assert not qk_norm or (r["rstd_q"].numel() >= M * H and r["rstd_k"].numel() >= M * H)
-    call("gpt_op_attention_fwd", qkv.data_ptr(), B, T, H, hd, int(rope), int(qk_norm), rope_base, eps,
+    call("gpt_op_attention_fwd", qkv.data_ptr(), B, T, H, hd, int(rope), int(qk_norm), int(window), rope_base, eps,
          r["qkv_norm"].data_ptr(), _ptr(r["rstd_q"]), _ptr(r["rstd_k"]), _ptr(r["rope_cs"]), r["o"].data_ptr(),
          r["lse"].data_ptr(), _stream(qkv))
     return r
 
 
 def attention_bwd(fwd: dict, dout: torch.Tensor, B: int, T: int, H: int, hd: int, *, rope: bool = True,
-                  qk_norm: bool = True, delta: torch.Tensor | None = None,
+                  qk_norm: bool = True, window: int = -1, delta: torch.Tensor | None = None,
                   dqkv: torch.Tensor | None = None) -> torch.Tensor:
     """dL/dqkv (bf16 [B*T, 3*H*hd]) from dout = dL/do (bf16 [B*T, H*hd]).
     ``delta`` (fp32 [B, H, T] scratch) and ``dqkv`` may be passed in to avoid
@@ -74,7 +104,7 @@ def attention_bwd(fwd: dict, dout: torch.Tensor, B: int, T: int, H: int, hd: int
     assert delta.numel() >= B * H * T and dqkv.numel() >= B * T * 3 * H * hd
     call("gpt_op_attention_bwd", fwd["qkv_norm"].data_ptr(), _ptr(fwd["rstd_q"]), _ptr(fwd["rstd_k"]),
          _ptr(fwd["rope_cs"]), fwd["o"].data_ptr(), fwd["lse"].data_ptr(), dout.data_ptr(), B, T, H, hd, int(rope),
-         int(qk_norm), delta.data_ptr(), dqkv.data_ptr(), _stream(dout))
+         int(qk_norm), int(window), delta.data_ptr(), dqkv.data_ptr(), _stream(dout))
     return dqkv
 
 
@@ -124,7 +154,7 @@ def lmhead_ce_fwd_noalloc(x: torch.Tensor, w: torch.Tensor, targets: torch.Tenso
 PROFILE_FAMILIES = ["gemm", "attn_fwd", "attn_bwd_dkv", "attn_bwd_dq", "norm_fwd", "norm_bwd", "embed_fwd",
                     "embed_bwd", "cast", "ce_combine", "loss", "qk", "delta", "colsum", "misc",
                     "gemm_qkv", "gemm_o", "gemm_up", "gemm_down", "gemm_lm_fwd", "gemm_lm_bwd", "gemm_dgrad",
-                    "gemm_wgrad", "optim"]
+                    "gemm_wgrad", "optim", "gemm_muon"]
 GEMM_FAMILIES = [f for f in PROFILE_FAMILIES if f.startswith("gemm")]
 
 

@@ -11,7 +11,7 @@ import ctypes as C
 
 import torch
 
-from ._lib import AdamWParams, call
+from ._lib import AdamWParams, MuonParams, call
 
 
 def lr_schedule(it: int, warmup_iters: int, lr_decay_iters: int, learning_rate: float, min_lr: float) -> float:
@@ -45,3 +45,27 @@ class AdamW:
              self.v.data_ptr(), self.step_count, C.byref(h), self.scratch.data_ptr(), self.grad_norm.data_ptr(),
              torch.cuda.current_stream(mdl.device).cuda_stream)
         return self.grad_norm
+
+
+class MuonAdamW:
+    """nanochat's split optimizer ("Train your own ChatGPT", read the source optim.py): Muon on the
+    block matrices, AdamW on everything else (include/gpt.h: gpt_muon_step).  Owns the momentum /
+    first-moment buffer, the second-moment buffer, the scratch and the step count."""
+
+    def __init__(self, model, lr: float = 0.02, momentum: float = 0.95, nesterov: bool = True, ns_steps: int = 5,
+                 adam_lr: float = 3e-4, betas=(0.9, 0.95), eps: float = 1e-8, weight_decay: float = 0.0):
+        self.model = model
+        self.h = MuonParams(lr, momentum, int(nesterov), ns_steps, adam_lr, betas[0], betas[1], eps, weight_decay)
+        self.mom = torch.zeros_like(model.params)
+        self.v = torch.zeros_like(model.params)
+        n = C.c_size_t()
+        call("gpt_muon_scratch_size", C.byref(model._c), C.byref(n))
+        self.scratch = torch.empty(n.value, dtype=torch.uint8, device=model.device)
+        self.step_count = 0
+
+    def step(self) -> None:
+        self.step_count += 1
+        mdl = self.model
+        call("gpt_muon_step", C.byref(mdl._c), mdl.params.data_ptr(), mdl.grads.data_ptr(), self.mom.data_ptr(),
+             self.v.data_ptr(), self.step_count, C.byref(self.h), self.scratch.data_ptr(),
+             torch.cuda.current_stream(mdl.device).cuda_stream)

@@ -65,6 +65,21 @@ typedef struct gpt_config {
   int32_t scale_resid_init; /* 1: init std of attn/MLP output projections 0.02/sqrt(2 n_layer) */
   float rope_base;          /* RoPE base (10000)                                        */
   float norm_eps;           /* epsilon of every norm (1e-5)                             */
+  /* Sliding-window layers ("Train your own ChatGPT", read the source gpt.py:
+   * _compute_window_sizes() expands a pattern such as "SSSL" into per-layer
+   * (left, right) windows).  Layer l is a short-window layer when
+   * window_short > 0 and bit (l mod window_period) of window_pattern is set
+   * ("SSSL" = 0x7 with period 4); its query i then sees only the keys
+   * i - window_short .. i.  Every other layer sees all earlier keys.
+   * window_short = 0 turns windows off; window_period is 1..32. */
+  int32_t window_short;
+  int32_t window_pattern;
+  int32_t window_period;
+  /* 1: the forward's block projections (q|k|v, attention output, MLP up and
+   * down) run on 8-bit e4m3 operands, each activation and weight cast with
+   * its own dynamic scale FP8_MAX / max|tensor| ("Train your own ChatGPT",
+   * read the source fp8.py); the lm_head and the backward stay bf16.  0: bf16. */
+  int32_t fp8;
 } gpt_config;
 
 /* Parameters: ONE flat fp32 buffer, tensors back to back in this order:
@@ -117,6 +132,27 @@ GPT_API int gpt_forward_loss(const gpt_config* cfg, const float* params, const i
  * Deterministic: the same inputs give bitwise the same gradients. */
 GPT_API int gpt_backward(const gpt_config* cfg, const float* params, int32_t B, int32_t T, void* workspace,
                          size_t workspace_bytes, float* grads, int32_t accumulate, void* stream);
+
+/* Gradient buckets for data-parallel training ("nanoGPT" wiki page, DDP:
+ * gradients averaged over ranks; "Train your own ChatGPT", read the source
+ * optim.py: DistMuonAdamW launches every gradient reduce_scatter at once so
+ * that communication overlaps compute).  Bucket k is the flat range
+ * [begin[k], end[k]) of the gradient buffer; buckets are listed in the order
+ * the backward completes them (final norm and an untied lm_head; the layers
+ * in pairs from the top; the embeddings last), they do not overlap and
+ * together cover every parameter.  *n_out is the count; begin and end (host
+ * arrays of max_buckets entries) may be NULL to query only the count. */
+GPT_API int gpt_grad_buckets(const gpt_config* cfg, int32_t max_buckets, int32_t* n_out, int64_t* begin,
+                             int64_t* end);
+
+/* gpt_backward that also records events[k] (a cudaEvent_t passed as void*,
+ * created by the caller) on `stream` as soon as bucket k of gpt_grad_buckets
+ * holds its final gradient, so that the caller can start reducing it on
+ * another stream while the backward goes on.  n_events must equal the bucket
+ * count.  The first bucket may be empty; its event is recorded all the same. */
+GPT_API int gpt_backward_bucketed(const gpt_config* cfg, const float* params, int32_t B, int32_t T, void* workspace,
+                                  size_t workspace_bytes, float* grads, int32_t accumulate, void* const* events,
+                                  int32_t n_events, void* stream);
 
 /* Bits per byte of one batch ("Train your own ChatGPT", read the source
  * loss_eval.py): sum_nats = sum of the per-token loss over targets whose
@@ -194,6 +230,44 @@ GPT_API int gpt_token_losses(const gpt_config* cfg, int32_t B, int32_t T, const 
  * its fp32 tiles instead, so tests can compare logits with a reference. */
 GPT_API int gpt_debug_logits(const gpt_config* cfg, int32_t B, int32_t T, void* workspace, size_t workspace_bytes,
                              float* logits, void* stream);
+
+/* Hyperparameters of the split optimizer step ("Train your own ChatGPT", read
+ * the source optim.py -- Muon + AdamW: the transformer's 2-D weight matrices go
+ * to Muon, which orthogonalizes each update, making all its singular values
+ * equal; embeddings, the lm_head and the other tensors go to AdamW). */
+typedef struct gpt_muon {
+  float lr;            /* Muon learning rate, >= 0                                             */
+  float momentum;      /* mu in [0, 1): buf <- mu buf + (1 - mu) g                             */
+  int32_t nesterov;    /* 1: orthogonalize (1 - mu) g + mu buf; 0: buf                         */
+  int32_t ns_steps;    /* Newton-Schulz steps, 1..32 (5)                                       */
+  float adam_lr;       /* AdamW on every other tensor: learning rate                           */
+  float beta1, beta2, eps;
+  float weight_decay;  /* AdamW decay, on the 2-D tensors among them (embeddings, lm_head)     */
+} gpt_muon;
+
+/* Bytes of device scratch (256-byte aligned) that gpt_muon_step needs. */
+GPT_API int gpt_muon_scratch_size(const gpt_config* cfg, size_t* bytes);
+
+/* One step of the split optimizer on the flat parameter buffer.  Every block
+ * matrix (w_qkv, w_o, w_up, w_down of every layer) takes a Muon step, read as
+ * its authors published it (K. Jordan et al., 2024): momentum
+ * buf <- mu buf + (1 - mu) g; u = (1 - mu) g + mu buf (Nesterov) or buf;
+ * X = u / (||u||_F + 1e-7) on the wide orientation; ns_steps of the quintic
+ * Newton-Schulz iteration X <- a X + (b A + c A^2) X, A = X X^T,
+ * (a, b, c) = (3.4445, -4.7750, 2.0315), in bf16 on the tensor cores;
+ * p <- p - lr sqrt(max(1, rows / cols)) X.  Every other tensor takes
+ * gpt_adamw_step's AdamW (no clipping, grad_scale 1) with adam_lr.
+ *   params  fp32 [gpt_param_count], updated in place
+ *   grads   fp32 [gpt_param_count], read only
+ *   mom     fp32 [gpt_param_count]: the Muon momentum of the block matrices and
+ *           the AdamW first moment of the rest (zero before step 1), updated
+ *   v       fp32 [gpt_param_count]: the AdamW second moment (unused entries of
+ *           the block matrices stay untouched), updated
+ *   step    1-based step number (AdamW bias correction)
+ *   scratch gpt_muon_scratch_size bytes
+ * All buffers are distinct and 16-byte aligned. */
+GPT_API int gpt_muon_step(const gpt_config* cfg, float* params, const float* grads, float* mom, float* v,
+                          int64_t step, const gpt_muon* h, void* scratch, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait runs out (GPT_ERR_DEVICE_TIMEOUT) or an

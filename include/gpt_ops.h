@@ -45,11 +45,40 @@ GPT_API int gpt_op_gemm(int epilogue, int bn, const void* a, long long lda, int 
                         long long ldb, int b_mn, int M, int N, int K, void* out, long long ldo,
                         const float* bias, int accumulate, void* stream);
 
+/* 8-bit cast with a dynamic per-tensor scale ("Train your own ChatGPT", read
+ * the source fp8.py: each tensor is rescaled before the cast, scale =
+ * FP8_MAX / max(|tensor|); e4m3 for activations and weights, e5m2 for
+ * gradients):
+ *   amax = max |x|;  s = FP8_MAX / amax (1 when amax == 0);  out = cast(x s)
+ *   inv_scale = 1 / s
+ * with FP8_MAX = 448 (fmt 0, e4m3) or 57344 (fmt 1, e5m2) and a cast that
+ * rounds to nearest (ties to even) and saturates at FP8_MAX.
+ *   x          n values, bf16 (x_fp32 == 0) or fp32 (x_fp32 != 0)
+ *   out        n bytes (8-bit floats); amax, inv_scale: fp32 [1], device
+ * n >= 1. */
+GPT_API int gpt_op_fp8_quantize(const void* x, int x_fp32, long long n, int fmt, void* out, float* amax,
+                                float* inv_scale, void* stream);
+
+/* The product of two 8-bit tensors with their inverse scales folded back in
+ * (same page: the matmul runs on the 8-bit values, as torch._scaled_mm does):
+ *   out[M,N] = (A[M,K] B[N,K]^T) * inv_a * inv_b   (+ bias, or += with accumulate)
+ * on the tensor cores (tcgen05 kind::f8f6f4, fp32 accumulation).  A and B are
+ * K-major 8-bit floats of formats fmt_a, fmt_b (0 e4m3, 1 e5m2; the two may
+ * differ) with row pitches lda, ldb in elements, multiples of 16; inv_a and
+ * inv_b are device fp32 scalars (gpt_op_fp8_quantize's inv_scale).  The
+ * epilogue, bias, accumulate, bn and out are as for gpt_op_gemm. */
+GPT_API int gpt_op_gemm_fp8(int epilogue, int bn, const void* a, long long lda, int fmt_a, const void* b,
+                            long long ldb, int fmt_b, int M, int N, int K, const float* inv_a, const float* inv_b,
+                            void* out, long long ldo, const float* bias, int accumulate, void* stream);
+
 /* Causal self-attention of one layer with RoPE and QK-norm, forward
  * ("nanoGPT" wiki page, CausalSelfAttention: q, k, v split from one fused
  * projection, reshaped to (B, n_head, T, head_dim), causal mask;
- * "nanochat-d20-chat" card, Architecture: RoPE + QK-norm).
+ * "nanochat-d20-chat" card, Architecture: RoPE + QK-norm; "Train your own
+ * ChatGPT", read the source gpt.py: per-layer (left, right) windows).
  *
+ *   window   -1: query i sees keys 0 .. i; >= 0: only keys i - window .. i
+ *            (a sliding-window layer; the right window is 0, causal)
  *   qkv      in  bf16 [B*T, 3*H*hd]  raw q|k|v rows (token-major; head h of q
  *                 at columns h*hd .. h*hd+hd-1, k after all q heads, v after k)
  *   qkv_norm out bf16 [B*T, 3*H*hd]  q, k after RoPE (if rope) and per-head
@@ -61,17 +90,18 @@ GPT_API int gpt_op_gemm(int epilogue, int bn, const void* a, long long lda, int 
  *   o        out bf16 [B*T, H*hd]    softmax(q k^T / sqrt(hd) + mask) v
  *   lse      out fp32 [B, H, T]      natural-log logsumexp of each score row
  * hd must be 64 or 128.  RoPE rotates the pairs (i, i + hd/2). */
-GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, int rope, int qk_norm,
+GPT_API int gpt_op_attention_fwd(const void* qkv, int B, int T, int H, int hd, int rope, int qk_norm, int window,
                                  float rope_base, float eps, void* qkv_norm, float* rstd_q, float* rstd_k,
                                  float* rope_cs, void* o, float* lse, void* stream);
 
 /* Backward of gpt_op_attention_fwd: given dout = dL/do (bf16 [B*T, H*hd]) and
  * the forward's outputs, writes dqkv = dL/dqkv (bf16 [B*T, 3*H*hd], the
- * gradient w.r.t. the RAW projection output, through QK-norm and RoPE).
- * delta is caller scratch, fp32 [B, H, T].  Deterministic. */
+ * gradient w.r.t. the RAW projection output, through QK-norm and RoPE), with
+ * the forward's window.  delta is caller scratch, fp32 [B, H, T].
+ * Deterministic. */
 GPT_API int gpt_op_attention_bwd(const void* qkv_norm, const float* rstd_q, const float* rstd_k,
                                  const float* rope_cs, const void* o, const float* lse, const void* dout, int B,
-                                 int T, int H, int hd, int rope, int qk_norm, float* delta, void* dqkv,
+                                 int T, int H, int hd, int rope, int qk_norm, int window, float* delta, void* dqkv,
                                  void* stream);
 
 /* Fused lm_head + cross-entropy, forward ("nanoGPT" wiki page, model.py
@@ -130,7 +160,8 @@ GPT_API int gpt_op_wait_probe(unsigned long long timeout_ns, void* stream);
  *   attn_bwd_dkv, attn_bwd_dq, norm_fwd, norm_bwd, embed_fwd, embed_bwd,
  *   cast, ce_combine, loss, qk, delta, colsum, misc, then the model's GEMMs by
  *   role: gemm_qkv, gemm_o, gemm_up, gemm_down, gemm_lm_fwd, gemm_lm_bwd,
- *   gemm_dgrad, gemm_wgrad (op-level GEMMs count as gemm). */
+ *   gemm_dgrad, gemm_wgrad (op-level GEMMs count as gemm), then optim (the
+ *   optimizers' elementwise steps) and gemm_muon (the Muon step's products). */
 GPT_API unsigned long long gpt_launch_count(void);
 GPT_API int gpt_profile_start(void);
 GPT_API int gpt_profile_stop(int max_kinds, double* ms, long long* count, double* flops, double* bytes);

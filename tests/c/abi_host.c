@@ -20,9 +20,9 @@ static int fails = 0;
 
 int main(void) {
   /* nanochat d20: RMSNorm, RoPE, ReLU^2, untied, QK-norm, no biases */
-  const gpt_config d20 = {20, 1280, 10, 2048, 32768, 0, 1, 1, 0, 1, 0, 0, 10000.f, 1e-5f};
+  const gpt_config d20 = {20, 1280, 10, 2048, 32768, 0, 1, 1, 0, 1, 0, 0, 10000.f, 1e-5f, 0, 0, 1, 0};
   /* GPT-2 124M: LayerNorm + biases, learned positions, GELU, tied, scaled residual init */
-  const gpt_config gpt2 = {12, 768, 12, 1024, 50304, 1, 0, 0, 1, 0, 1, 1, 10000.f, 1e-5f};
+  const gpt_config gpt2 = {12, 768, 12, 1024, 50304, 1, 0, 0, 1, 0, 1, 1, 10000.f, 1e-5f, 0, 0, 1, 0};
   int64_t n = 0, off = -1, rows = 0, cols = 0;
   int32_t nt = 0;
   char name[32];

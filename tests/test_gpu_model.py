@@ -37,6 +37,9 @@ CASES = {
     "gpt2_ragged": (("gpt2", dict(n_layer=1, n_embd=64, n_head=1, vocab_size=300, block_size=256)), 3, 200, (1, 12)),
     "d20_small": (("d20", dict(n_layer=2, n_embd=256, n_head=2, vocab_size=2048, block_size=512)), 2, 256, (1, 16)),
     "d20_ragged": (("d20", dict(n_layer=1, n_embd=128, n_head=1, vocab_size=777, block_size=512)), 2, 300, (1, 16)),
+    # sliding-window layers in the "SSSL" pattern: layers 0-2 see 100 keys back, layer 3 all
+    "d20_sssl": (("d20", dict(n_layer=4, n_embd=256, n_head=2, vocab_size=2048, block_size=512, window_short=100,
+                              window_pattern=0b0111, window_period=4)), 2, 300, (1, 16)),
 }
 
 
