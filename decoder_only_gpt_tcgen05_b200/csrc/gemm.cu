@@ -327,11 +327,29 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   return dispatch(epi, bn, pair, maps, p, st);
 }
 
+static int run_gemm_group_impl(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
+                               cudaStream_t st, int epi, int accumulate, const void* c, long long ldc,
+                               long long c_rows, const int* c_row, float alpha, float beta);
+
 int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
                    cudaStream_t st, int epi, int accumulate) {
+  return run_gemm_group_impl(n, probs, K, a_mn, b_mn, bn, prof_kind, st, epi, accumulate, nullptr, 0, 0, nullptr, 0.f,
+                             0.f);
+}
+
+int run_gemm_group_axpby(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int prof_kind, const void* c,
+                         long long ldc, long long c_rows, const int* c_row, float alpha, float beta, cudaStream_t st) {
+  if (!c || !c_row) return set_error(ST_INVALID_ARG, "grouped GEMM: linear epilogue without its addend");
+  return run_gemm_group_impl(n, probs, K, a_mn, b_mn, 256, prof_kind, st, EPI_ACTBWD, 0, c, ldc, c_rows, c_row,
+                             alpha, beta);
+}
+
+static int run_gemm_group_impl(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
+                               cudaStream_t st, int epi, int accumulate, const void* c, long long ldc,
+                               long long c_rows, const int* c_row, float alpha, float beta) {
   if (n < 1 || n > kMaxProblems) return set_error(ST_INVALID_ARG, "grouped GEMM: 1 to 8 problems");
   if (bn != 128 && bn != 256) return set_error(ST_INVALID_ARG, "GEMM tile N must be 128 or 256");
-  if (!(epi == EPI_F32 || (epi == EPI_BF16 && !accumulate)))
+  if (!(epi == EPI_F32 || ((epi == EPI_BF16 || epi == EPI_ACTBWD) && !accumulate)))
     return set_error(ST_INVALID_ARG, "grouped GEMM: fp32 (stored or accumulated) or bf16 (stored) outputs");
   const int es = epi == EPI_F32 ? 4 : 2;
   GemmMaps maps;
@@ -369,6 +387,14 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
     start += p.ptiles_m[q] * p.ptiles_n[q];
   }
   p.tile_start[n] = start;
+  if (epi == EPI_ACTBWD) {  // the linear epilogue's addend: one stacked bf16 matrix, a row block per problem
+    if (!aligned16(c, ldc, 2)) return set_error(ST_INVALID_ARG, "grouped GEMM: addend alignment");
+    GPTK_TRY(make_tmap_2d(&maps.r, c, probs[0].N, c_rows, ldc, 64, 32, 2));
+    for (int q = 0; q < n; ++q) p.prow[q] = c_row[q];
+    p.act = 3;
+    p.ax_alpha = alpha;
+    p.ax_beta = beta;
+  }
   p.M = p.pM[0];
   p.N = p.pN[0];
   p.tiles_m = p.ptiles_m[0];

@@ -51,7 +51,8 @@ enum EpiKind : int {
   EPI_RESID = 2,    // out fp32 = resid + acc (+ bias)
   EPI_QKV = 3,      // out bf16 = acc, with RoPE + per-head RMSNorm applied to the q and k heads
   EPI_UP = 4,       // u = acc (+ bias) -> h = act(u) bf16 (out2), and u bf16 (out) unless out is null
-  EPI_ACTBWD = 5,   // out bf16 = acc * act'(u); aux is u, or h = relu(u)^2 when act is ReLU^2
+  EPI_ACTBWD = 5,   // out bf16 = acc * act'(u); aux is u, or h = relu(u)^2 when act is ReLU^2;
+                    // act 3: out bf16 = ax_alpha acc + ax_beta aux (a linear combination)
   EPI_CE_FWD = 6,   // per-row (max, sum exp) partials over this tile's vocab columns + target logit
   EPI_CE_BWD = 7,   // out bf16 = (softmax - onehot) * scale
 };
@@ -73,7 +74,9 @@ struct GemmParams {
   void* out2;                 // EPI_UP: h
   const __nv_bfloat16* aux;   // EPI_ACTBWD: u
   long long ld_aux;
-  int act;                    // 0 GELU(erf), 1 ReLU^2
+  int act;                    // 0 GELU(erf), 1 ReLU^2 (EPI_ACTBWD: 2 ReLU^2 from h, 3 linear)
+  float ax_alpha, ax_beta;    // EPI_ACTBWD with act 3
+  int prow[8];                // grouped launches: the epilogue input's first row for each problem
   // head-padded output layout (generic BF16 path): column c maps to (c / hd) * hdp + c % hd
   int hd, hdp;
   // cross-entropy
@@ -579,7 +582,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
         const int b = chunk_ctr & 1;
         bulk_wait_read<1>();
         mbar_expect_tx(&ibar[b], 4096);
-        tma_load_2d(stg_ptr + b * 4096, tmR, &ibar[b], n0 + c_begin, row0);
+        tma_load_2d(stg_ptr + b * 4096, tmR, &ibar[b], n0 + c_begin, row0 + p.prow[ti.prob]);
       }
       if (!mbar_wait(&tfull[acc], acc_phase, p.ctl, abort_flag, 5)) break;
       tc_fence_after();
@@ -725,6 +728,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
               unstage_f32(buf, lane, in);
 #pragma unroll
               for (int j = 0; j < CW; ++j) v[j] += in[j];
+            } else if (p.act == 3) {  // EPI_ACTBWD, linear: alpha acc + beta aux
+              unstage_bf16(buf, lane, in);
+#pragma unroll
+              for (int j = 0; j < CW; ++j) v[j] = fmaf(p.ax_beta, in[j], p.ax_alpha * v[j]);
             } else if (p.act == 2) {  // EPI_ACTBWD, ReLU^2 from h: 2 relu(u) = 2 sqrt(h)
               unstage_bf16(buf, lane, in);
 #pragma unroll
@@ -784,7 +791,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
             if (HAS_IN && c + CW < c_begin + HALF && col0 + CW < pN) {
               bulk_wait_read<1>();
               mbar_expect_tx(&ibar[b ^ 1], 4096);
-              tma_load_2d(stg_ptr + (b ^ 1) * 4096, tmR, &ibar[b ^ 1], col0 + CW, row0);
+              tma_load_2d(stg_ptr + (b ^ 1) * 4096, tmR, &ibar[b ^ 1], col0 + CW, row0 + p.prow[ti.prob]);
             }
           }
           ++chunk_ctr;

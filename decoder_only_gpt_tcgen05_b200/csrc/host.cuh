@@ -109,5 +109,10 @@ struct GroupProblem {
 // (epi EPI_BF16).
 int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int bn, int prof_kind,
                    cudaStream_t st, int epi = 1, int accumulate = 1);
+// Grouped bf16 products with a linear epilogue: out_q = alpha (A_q B_q^T) + beta C_q, where the
+// C_q are the row blocks of one stacked bf16 matrix c (problem q's rows start at c_row[q], pitch
+// ldc); used where every product has its own addend of its own output's shape.
+int run_gemm_group_axpby(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int prof_kind, const void* c,
+                         long long ldc, long long c_rows, const int* c_row, float alpha, float beta, cudaStream_t st);
 
 }  // namespace gptk

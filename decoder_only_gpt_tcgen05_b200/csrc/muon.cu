@@ -14,9 +14,9 @@
 // Launch sequence per chunk of same-shape matrices:
 //   muon_momentum_kernel   buf update and the Nesterov input's squared norm (fp64 partials)
 //   muon_prep_kernel       X = U / ||U|| in bf16, transposed through shared memory when needed
-//   ns_steps x { grouped GEMM A = X X^T (bf16), grouped GEMM A2 = A A (fp32),
-//                muon_combine_kernel M = b A + c A2 (bf16), grouped GEMM Y = M X (fp32),
-//                muon_axpy_kernel X = a X + Y (bf16, in place) }
+//   ns_steps x { grouped GEMM A = X X^T (bf16),
+//                grouped GEMM M = c (A A) + b A (bf16; the linear combination in the epilogue),
+//                grouped GEMM X' = (M X) + a X (bf16, into the other X buffer) }
 //   muon_update_kernel     W -= lr scale X, transposed back through shared memory when needed
 #include <cmath>
 #include <string>
@@ -126,29 +126,6 @@ __global__ void __launch_bounds__(256) muon_prep_kernel(const float* __restrict_
   }
 }
 
-// M = b A + c A2 over n elements (bf16 A, fp32 A2 -> bf16 M), 2 per thread step
-__global__ void muon_combine_kernel(const __nv_bfloat16* __restrict__ A, const float* __restrict__ A2,
-                                    __nv_bfloat16* __restrict__ M, long long n) {
-  for (long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x); i < n;
-       i += 2LL * gridDim.x * blockDim.x) {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(A + i);
-    const float2 a2 = *reinterpret_cast<const float2*>(A2 + i);
-    *reinterpret_cast<__nv_bfloat162*>(M + i) = __floats2bfloat162_rn(fmaf(kNsC, a2.x, kNsB * __low2float(a)),
-                                                                       fmaf(kNsC, a2.y, kNsB * __high2float(a)));
-  }
-}
-
-// X = a X + Y over n elements (bf16 X in place, fp32 Y), 2 per thread step
-__global__ void muon_axpy_kernel(__nv_bfloat16* __restrict__ X, const float* __restrict__ Y, long long n) {
-  for (long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x); i < n;
-       i += 2LL * gridDim.x * blockDim.x) {
-    const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(X + i);
-    const float2 y = *reinterpret_cast<const float2*>(Y + i);
-    *reinterpret_cast<__nv_bfloat162*>(X + i) =
-        __floats2bfloat162_rn(fmaf(kNsA, __low2float(x), y.x), fmaf(kNsA, __high2float(x), y.y));
-  }
-}
-
 // W[r][c] -= step * X'[r][c] with X' = X (rows <= cols) or X^T (X is [cols, rows]); tiles of 32 x 32
 __global__ void __launch_bounds__(256) muon_update_kernel(float* __restrict__ params, MatList ml, int rows, int cols,
                                                           const __nv_bfloat16* __restrict__ X, float step) {
@@ -182,7 +159,7 @@ struct MuonGroup {
 };
 
 struct MuonScratch {
-  size_t adam, part, x, y, a, a2, m, total;
+  size_t adam, part, x0, x1, a, m, total;
 };
 
 MuonScratch muon_scratch_plan(const std::vector<MuonGroup>& groups) {
@@ -200,14 +177,12 @@ MuonScratch muon_scratch_plan(const std::vector<MuonGroup>& groups) {
   off += al(adamw_scratch_bytes());
   s.part = off;
   off += al((size_t)kChunk * kParts * 8);
-  s.x = off;
+  s.x0 = off;
   off += al((size_t)kChunk * mn * 2);
-  s.y = off;
-  off += al((size_t)kChunk * mn * 4);
+  s.x1 = off;
+  off += al((size_t)kChunk * mn * 2);
   s.a = off;
   off += al((size_t)kChunk * mm * 2);
-  s.a2 = off;
-  off += al((size_t)kChunk * mm * 4);
   s.m = off;
   off += al((size_t)kChunk * mm * 2);
   s.total = off;
@@ -223,11 +198,10 @@ int muon_chunk(float* params, const float* grads, float* mom, const MuonGroup& g
   for (int q = 0; q < nq; ++q) ml.off[q] = grp.offs[first + q];
   char* base = static_cast<char*>(scratch);
   double* part = reinterpret_cast<double*>(base + sp.part);
-  __nv_bfloat16* X = reinterpret_cast<__nv_bfloat16*>(base + sp.x);
-  float* Y = reinterpret_cast<float*>(base + sp.y);
+  __nv_bfloat16* Xb[2] = {reinterpret_cast<__nv_bfloat16*>(base + sp.x0), reinterpret_cast<__nv_bfloat16*>(base + sp.x1)};
   __nv_bfloat16* A = reinterpret_cast<__nv_bfloat16*>(base + sp.a);
-  float* A2 = reinterpret_cast<float*>(base + sp.a2);
   __nv_bfloat16* M = reinterpret_cast<__nv_bfloat16*>(base + sp.m);
+  __nv_bfloat16* X = Xb[0];
   const int nest = h.nesterov ? 1 : 0;
   {
     Prof prof(PK_OPTIM, 0, (double)nq * elems * 12, st);
@@ -240,34 +214,25 @@ int muon_chunk(float* params, const float* grads, float* mom, const MuonGroup& g
     muon_prep_kernel<<<dim3(tiles, nq), 256, 0, st>>>(grads, mom, ml, rows, cols, h.momentum, nest, part, X);
     GPTK_CUDA(cudaGetLastError());
   }
-  GroupProblem gA[kChunk], gA2[kChunk], gY[kChunk];
-  for (int q = 0; q < nq; ++q) {
-    __nv_bfloat16* Xq = X + (size_t)q * m * n;
-    __nv_bfloat16* Aq = A + (size_t)q * m * m;
-    float* A2q = A2 + (size_t)q * m * m;
-    __nv_bfloat16* Mq = M + (size_t)q * m * m;
-    float* Yq = Y + (size_t)q * m * n;
-    gA[q] = GroupProblem{Xq, n, Xq, n, m, m, Aq, m, 0};     // A = X X^T
-    gA2[q] = GroupProblem{Aq, m, Aq, m, m, m, A2q, m, 0};   // A A (A is symmetric: A^T = A)
-    gY[q] = GroupProblem{Mq, m, Xq, n, m, n, Yq, n, 0};     // M X (X read MN-major)
-  }
-  const long long nmm = (long long)nq * m * m, nmn = (long long)nq * m * n;
-  const int ew_grid = num_sms() * 8;
+  int rows_of[kChunk];  // first row of matrix q in the stacked A and X buffers
+  for (int q = 0; q < nq; ++q) rows_of[q] = q * m;
   for (int it = 0; it < h.ns_steps; ++it) {
+    __nv_bfloat16* Xc = Xb[it & 1];
+    __nv_bfloat16* Xn = Xb[(it + 1) & 1];
+    GroupProblem gA[kChunk], gM[kChunk], gX[kChunk];
+    for (int q = 0; q < nq; ++q) {
+      __nv_bfloat16* Xq = Xc + (size_t)q * m * n;
+      __nv_bfloat16* Aq = A + (size_t)q * m * m;
+      __nv_bfloat16* Mq = M + (size_t)q * m * m;
+      gA[q] = GroupProblem{Xq, n, Xq, n, m, m, Aq, m, 0};                   // A = X X^T
+      gM[q] = GroupProblem{Aq, m, Aq, m, m, m, Mq, m, 0};                   // A A (A is symmetric: A^T = A)
+      gX[q] = GroupProblem{Mq, m, Xq, n, m, n, Xn + (size_t)q * m * n, n, 0};  // M X (X read MN-major)
+    }
     GPTK_TRY(run_gemm_group(nq, gA, n, 0, 0, 256, PK_GEMM_MUON, st, EPI_BF16, 0));
-    GPTK_TRY(run_gemm_group(nq, gA2, m, 0, 0, 256, PK_GEMM_MUON, st, EPI_F32, 0));
-    {
-      Prof prof(PK_OPTIM, 0, (double)nmm * 8, st);
-      muon_combine_kernel<<<ew_grid, 256, 0, st>>>(A, A2, M, nmm);
-      GPTK_CUDA(cudaGetLastError());
-    }
-    GPTK_TRY(run_gemm_group(nq, gY, m, 0, 1, 256, PK_GEMM_MUON, st, EPI_F32, 0));
-    {
-      Prof prof(PK_OPTIM, 0, (double)nmn * 8, st);
-      muon_axpy_kernel<<<ew_grid, 256, 0, st>>>(X, Y, nmn);
-      GPTK_CUDA(cudaGetLastError());
-    }
+    GPTK_TRY(run_gemm_group_axpby(nq, gM, m, 0, 0, PK_GEMM_MUON, A, m, (long long)nq * m, rows_of, kNsC, kNsB, st));
+    GPTK_TRY(run_gemm_group_axpby(nq, gX, m, 0, 1, PK_GEMM_MUON, Xc, n, (long long)nq * m, rows_of, 1.f, kNsA, st));
   }
+  X = Xb[h.ns_steps & 1];
   const float step = (float)(h.lr * std::sqrt(rows > cols ? (double)rows / cols : 1.0));
   {
     Prof prof(PK_OPTIM, 0, (double)nq * elems * 10, st);

@@ -5,11 +5,13 @@ The op has two stages, checked one at a time on their own inputs, and the backwa
     the oracle's fp64 rotation and norm of the same raw q|k|v: within 2^-8 of each element (the
     bf16 rounding of the stored value, 2^-9, with room for the fp32 arithmetic before it);
   - attention proper, on exactly those bf16 q, k, v: outputs at cosine >= 0.9999 and relative L2
-    <= 1e-2, and element by element within 2e-2 of their RMS plus 2^-8 of the element itself.
+    <= 1e-2, and element by element within 2e-2 of their RMS plus 2^-8 (|o| + sum_j p_j |v_j|).
     The second term is the bf16 arithmetic the kernel must do: the stored output is bf16 (up to
-    2^-9 of the element) and so are the probabilities that weight v (another 2^-9); for the
-    largest outputs (several times the RMS) those two alone exceed a bar of 2e-2 RMS.  The
-    logsumexp within 2e-3.
+    2^-9 |o|) and so are the probabilities that weight v, which moves each term p_j v_j by up to
+    2^-9 of itself and the row's sum by up to 2^-9 sum_j p_j |v_j| (the factor 2 leaves room for
+    the fp32 sums).  Where a row averages few keys of opposite signs (the first rows of a
+    sequence), sum_j p_j |v_j| is many times |o|, and at T = 8192 those rows' errors are several
+    times 2e-2 of an RMS that the long rows' averaging makes small.  The logsumexp within 2e-3.
     (Against the raw-input oracle instead, the bf16 rounding of the normalised q and k moves the
     scores by up to 2^-8 |q||k| / sqrt(hd), 0.04 with QK-norm at hd = 128, and the outputs by up to
     ~0.1 of their RMS at T = 8192: an input error, not one of the attention kernel.)
@@ -77,16 +79,23 @@ def check_stages(f, qkv_raw, B, T, H, hd, rope, qk_norm, window, what="", rows=N
     assert np.all(np.abs(qn - ref_n)[rows] <= 2.0 ** -8 * np.abs(ref_n)[rows] + 1e-6), (what, "qk stage")
     o_ref, lse_ref, _ = _oracle_attention(qn[:B * T], B, T, H, hd, False, False, np.zeros((B * T, H * hd)),
                                           window=window)
-    assert_output_close(f["o"].double().cpu().numpy()[rows], o_ref[rows], what)
+    # sum_j p_j |v_j|: the same attention applied to |v|
+    qn_abs = qn[:B * T].copy()
+    qn_abs[:, 2 * H * hd:] = np.abs(qn_abs[:, 2 * H * hd:])
+    o_abs = _oracle_attention(qn_abs, B, T, H, hd, False, False, np.zeros((B * T, H * hd)), window=window)[0]
+    assert_output_close(f["o"].double().cpu().numpy()[rows], o_ref[rows], what, o_abs=o_abs[rows])
     lse = f["lse"].double().cpu().numpy()
     t_rows = np.arange(T)[rows if isinstance(rows, slice) else slice(None)]
     assert np.abs(lse[..., t_rows] - lse_ref[..., t_rows]).max() < 2e-3, (what, "lse")
 
 
-def assert_output_close(o, o_ref, what=""):
-    """max over elements of |o - o_ref| - 2^-8 |o_ref| <= 2e-2 RMS(o_ref), plus cosine and relative L2."""
+def assert_output_close(o, o_ref, what="", o_abs=None):
+    """max over elements of |o - o_ref| - 2^-8 (|o_ref| + o_abs) <= 2e-2 RMS(o_ref), plus cosine and
+    relative L2 (o_abs: sum_j p_j |v_j| per element, or |o_ref| when not given)."""
     rms = np.sqrt(np.mean(o_ref ** 2))
-    excess = (np.abs(o - o_ref) - 2.0 ** -8 * np.abs(o_ref)).max()
+    if o_abs is None:
+        o_abs = np.abs(o_ref)
+    excess = (np.abs(o - o_ref) - 2.0 ** -8 * (np.abs(o_ref) + o_abs)).max()
     assert excess <= 2e-2 * rms, (what, excess / rms, np.abs(o - o_ref).max() / rms)
     cos, rel = _cos_rel(o, o_ref)
     assert cos >= 0.9999 and rel <= 1e-2, (what, cos, rel)
