@@ -8,11 +8,8 @@ every parameter gradient at cosine >= 0.999 and relative L2 <= 3e-2.
 The logits bar is the target's 2e-2 max-abs relative to their RMS, or twice the
 deviation that bf16 operands alone cause, whichever is larger: the tensor cores
 take bf16 operands, and on the d20-shaped models rounding just those operands in
-the fp64 oracle already moves the largest logit by 2-4 % of the RMS (see
-bf16_floor.py).  The RMS of the deviation is held to twice that floor's RMS, or
-to one bf16 step (2^-8) of the logits' RMS where the floor is smaller: on the
-one-layer toy model the operands' rounding alone moves the logits by 0.07 % RMS,
-less than the rounding of the stored intermediates it leaves out.
+the fp64 oracle already moves the largest logit by 2.5-4.8 % of the RMS (see
+bf16_floor.py).  The RMS of the deviation is held to twice that floor's RMS too.
 
 Per token, the loss and the logsumexp are compared element by element.  Both
 are 1-Lipschitz in the max-norm of the logits row (the loss moves with the
@@ -107,7 +104,7 @@ def test_forward_backward_bpb_match_oracle(name, params):
     bar = max(2e-2 * z_rms, 2.0 * f_max)
     dz = logits - f["logits"]
     assert np.abs(dz).max() <= bar, (np.abs(dz).max() / z_rms, f_max / z_rms)
-    assert np.sqrt(np.mean(dz ** 2)) <= max(2.0 * f_rms, 2.0 ** -8 * z_rms), (np.sqrt(np.mean(dz ** 2)) / z_rms, f_rms / z_rms)
+    assert np.sqrt(np.mean(dz ** 2)) <= max(2.0 * f_rms, 1e-3 * z_rms), (np.sqrt(np.mean(dz ** 2)) / z_rms, f_rms / z_rms)
     ell, lse = ell_d.double().cpu().numpy(), lse_d.double().cpu().numpy()
     assert np.abs(lse - f["lse"]).max() <= bar, np.abs(lse - f["lse"]).max() / z_rms
     assert np.abs(ell - f["ell"]).max() <= 2 * bar, np.abs(ell - f["ell"]).max() / z_rms
