@@ -34,6 +34,7 @@ SIGNATURES = {
     "gpt_op_lmhead_ce_fwd": [_P, _P, _P, _I, _I, _I, _P, _P, _P, _P],
     "gpt_op_lmhead_ce_fwd_noalloc": [_P, _P, _P, _I, _I, _I, _P, _P, _P],
     "gpt_op_wait_probe": [C.c_ulonglong, _P],
+    "gpt_op_exp2": [_P, C.c_longlong, C.c_int, _P, _P],
     "gpt_profile_start": [],
     "gpt_profile_stop": [_I, _P, _P, _P, _P],
     "gpt_param_count": [_P, _P],

@@ -9,14 +9,16 @@
 // under 128-byte swizzle, so rows past the end of a sequence arrive as zeros.
 //
 // Forward (one CTA per pair of 128-query tiles of one (b, h); heaviest causal pairs first):
-//   warp 0      TMA: the two Q tiles once, then K_j and V_j through a 3-slot ring
-//   warp 1      one thread alternates between the two tiles: S_j = Q K_j^T into that tile's
-//               TMEM scores, then O += P_{j-1} V_{j-1} (P from shared memory, O in TMEM), so
-//               the tensor core works on one tile while the other tile's softmax runs
+//   warp 0      TMA: the two Q tiles once, then K_j and V_j through a ring of 5 (hd 128) or 8
+//               (hd 64) slots, so that the loads run two blocks ahead of the products
+//   warp 1      one thread alternates between the two tiles: O += P_j V_j (P from tensor memory,
+//               V from shared memory), then S_{j+1} = Q K_{j+1}^T into that tile's TMEM scores,
+//               so the tensor core works on one tile while the other tile's softmax runs
 //   warps 2..9  two softmax warpgroups, one per query tile, one query row per thread: row max
-//               and sum in registers, P = exp2(...) written to shared memory in the MMA operand
-//               layout; O is rescaled in TMEM only when the running max grows by more than 2^8
-//               (otherwise the stale max stays exact because O and l use the same one)
+//               and sum in registers, P = exp2(...) as bf16 into the upper half of the tile's
+//               score columns (already read), where it is the A operand of the PV product; O is
+//               rescaled in TMEM only when the running max grows by more than 2^8 (otherwise the
+//               stale max stays exact because O and l use the same one)
 // Backward: delta = rowsum(dO * O) (kernels.cu), then
 //   dK/dV kernel: one CTA per 128-key tile, stepping over 128-query blocks from the diagonal:
 //               S^T = K Q^T and dP^T = V dO^T into TMEM; elementwise warps write P^T and dS^T
@@ -35,48 +37,55 @@ namespace gptk {
 
 static constexpr float kLog2e = 1.4426950408889634f;
 
-// Row r, columns [c0, c0 + 8) of a K-major, 128-byte-swizzled bf16 tile whose rows are 128 bytes:
-// byte offset of the 16-byte unit holding them.
-__device__ __forceinline__ uint32_t sw128_off(int r, int unit) { return r * 128 + ((unit ^ (r & 7)) << 4); }
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
 // ====================================================================== forward
 // One CTA per (b, h, pair of 128-query tiles A = 2p, B = 2p+1): two softmax warpgroups, one
 // per query tile, and one MMA thread that alternates between them, so that the tensor core
 // computes one tile's S or PV while the other tile's softmax runs.  K and V tiles stream
-// through a 3-slot ring shared by both query tiles (K_0, V_0, K_1, V_1, ...).
-// TMEM: S_A [0,128), S_B [128,256), O_A [256,256+HD), O_B [384,384+HD).
+// through one ring shared by both query tiles (K_0, V_0, K_1, V_1, ...).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,256+HD), O_B [384,384+HD).  P_t (bf16, two keys
+// per column) goes over columns [0, 64) of S_t once the softmax holds the scores in registers;
+// the next S_t product is issued only after the PV product that reads P_t has completed.
+// Warpgroup 0 (TMA warp, MMA warp, two idle warps) gives registers to the two softmax
+// warpgroups, so that each softmax thread holds its row's 128 scores at once.
 
 template <int HD>
 struct FwdSmem {
-  static constexpr int TILE = HD * 256;  // 128 rows x HD bf16
-  static constexpr int Q0 = 0;           // Q_A, Q_B
-  static constexpr int KV = 2 * TILE;    // 3 ring slots
-  static constexpr int P = 5 * TILE;     // P_A, P_B: 128 x 128 bf16 each
-  static constexpr int BAR = P + 2 * 32768;
+  static constexpr int TILE = HD * 256;         // 128 rows x HD bf16
+  static constexpr int NS = HD == 128 ? 5 : 8;  // K/V ring slots
+  static constexpr int Q0 = 0;                  // Q_A, Q_B
+  static constexpr int KV = 2 * TILE;           // NS ring slots
+  static constexpr int BAR = KV + NS * TILE;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
 
+constexpr int kFwdThreads = 384;
+constexpr int kFwdRegs = 168;          // per thread at launch: 65536 / 384, rounded down to 8
+constexpr int kFwdRegsProducer = 80;   // warpgroup 0 after setmaxnreg.dec
+constexpr int kFwdRegsSoftmax = 208;  // warpgroups 1, 2 after setmaxnreg.inc
+static_assert(128 * kFwdRegsProducer + 256 * kFwdRegsSoftmax <= kFwdThreads * kFwdRegs,
+              "the register split must fit the registers the block is launched with");
+// 16-key groups of a block whose exponentials go to the FMA pipe (exp2_poly2), the others to
+// ex2.approx: 3 of 8, which balances the MUFU unit (8 cycles per warp instruction) against the
+// issue slots of the polynomial
+constexpr uint32_t kPolyGroups = 0x52u;
+
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnShape s, __nv_bfloat16* __restrict__ o,
                     long long ldo, float* __restrict__ lse_out, float scale_log2, DevCtl ctl) {
   using L = FwdSmem<HD>;
+  constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [3]
-  uint64_t* kv_empty = bars + 4;  // [3]
-  uint64_t* s_full = bars + 7;    // [2] (A, B)
-  uint64_t* p_full = bars + 9;    // [2]
-  uint64_t* o_done = bars + 11;   // [2]
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* kv_full = bars + 1;         // [NS]
+  uint64_t* kv_empty = kv_full + NS;    // [NS]
+  uint64_t* s_full = kv_empty + NS;     // [2] (A, B)
+  uint64_t* p_full = s_full + 2;        // [2]
+  uint64_t* o_done = s_full + 4;        // [2]
+  uint64_t* drain = s_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -99,7 +108,7 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < NS; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
@@ -126,6 +135,8 @@ __global__ void __launch_bounds__(320, 1)
   const int colk = s.H * s.hdp + h * s.hdp;
   const int colv = 2 * s.H * s.hdp + h * s.hdp;
 
+  if (warp < 4) {
+    setmaxnreg_dec<kFwdRegsProducer>();
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------- TMA producer
     bool ok = true;
@@ -135,8 +146,8 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_3d(sm + L::Q0 + t * L::TILE + c * 16384, &tm_qkv, q_full, colq + 64 * c, q0 + 128 * t, b);
     int issued = -1;
     for (int seq = 0; seq < 2 * n_kv && ok; ++seq) {
-      const int slot = seq % 3;
-      const uint32_t ph = (seq / 3) & 1;
+      const int slot = seq % NS;
+      const uint32_t ph = (seq / NS) & 1;
       if (!mbar_wait(&kv_empty[slot], ph ^ 1u, ctl, abort_flag, 20)) { ok = false; break; }
       mbar_expect_tx(&kv_full[slot], L::TILE);
       const int col = (seq & 1) ? colv : colk;
@@ -148,8 +159,8 @@ __global__ void __launch_bounds__(320, 1)
     if (!ok) {
       volatile int never = 0;
       mbar_wait(q_full, 0, ctl, &never, 22);
-      for (int seq = (issued > 1 ? issued - 2 : 0); seq <= issued && issued >= 0; ++seq)
-        mbar_wait(&kv_full[seq % 3], (seq / 3) & 1, ctl, &never, 22);
+      for (int seq = (issued >= NS ? issued - NS + 1 : 0); seq <= issued && issued >= 0; ++seq)
+        mbar_wait(&kv_full[seq % NS], (seq / NS) & 1, ctl, &never, 22);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------- MMA issuer
@@ -158,16 +169,15 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 23);
     bool issued = false;
     auto kv_wait = [&](int seq) -> bool {
-      return mbar_wait(&kv_full[seq % 3], (seq / 3) & 1, ctl, abort_flag, 24);
+      return mbar_wait(&kv_full[seq % NS], (seq / NS) & 1, ctl, abort_flag, 24);
     };
-    // operand descriptors computed once; the MMAs of a product go out back to back (umma8_ss)
+    // operand descriptors computed once; the MMAs of a product go out back to back (umma8_*)
     const uint64_t dQ0 = sdesc_sw128(smem_u32(sm + L::Q0), 16, 1024);
     const uint64_t dKV0 = sdesc_sw128(smem_u32(sm + L::KV), 16, 1024);     // K-major (K for S)
     const uint64_t dKVm0 = sdesc_sw128(smem_u32(sm + L::KV), 16384, 1024);  // MN-major (V for PV)
-    const uint64_t dP0 = sdesc_sw128(smem_u32(sm + L::P), 16, 1024);
     auto issue_s = [&](int t, int j) {
       const uint64_t dQ = sdesc_add(dQ0, t * L::TILE);
-      const uint64_t dK = sdesc_add(dKV0, ((2 * j) % 3) * L::TILE);
+      const uint64_t dK = sdesc_add(dKV0, ((2 * j) % NS) * L::TILE);
       if (HD == 128) {
         uint32_t dd[8];
         uint64_t aa[8], bb[8];
@@ -189,17 +199,16 @@ __global__ void __launch_bounds__(320, 1)
       umma_commit(&s_full[t]);
     };
     auto issue_pv = [&](int t, int j) {
-      const uint64_t dP = sdesc_add(dP0, t * 32768);
-      const uint64_t dV = sdesc_add(dKVm0, ((2 * j + 1) % 3) * L::TILE);
-      uint32_t dd[8];
-      uint64_t aa[8], bb[8];
+      const uint64_t dV = sdesc_add(dKVm0, ((2 * j + 1) % NS) * L::TILE);
+      uint32_t dd[8], aa[8];
+      uint64_t bb[8];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
+      for (int kk = 0; kk < 8; ++kk) {  // keys 16 kk .. 16 kk + 15
         dd[kk] = tbase + 256 + 128 * t;
-        aa[kk] = sdesc_add(dP, (kk >> 2) * 16384 + (kk & 3) * 32);
+        aa[kk] = tbase + 128 * t + 8 * kk;
         bb[kk] = sdesc_add(dV, kk * 2048);
       }
-      umma8_ss(dd, aa, bb, idesc_o, j == f_t[t] ? 0xfeu : 0xffu);
+      umma8_ts(dd, aa, bb, idesc_o, j == f_t[t] ? 0xfeu : 0xffu);
       umma_commit(&o_done[t]);
     };
     // ring block j (0-based from jlo): tile t computes S for it when f[t] <= j < f[t] + c[t]
@@ -225,22 +234,26 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (takes(t, j + 1)) {
           if (!kv_wait(2 * j + 2)) { ok = false; break; }
+          // S_{j+1} overwrites the columns that hold P_j: the PV product must have read them
+          if (takes(t, j) && !mbar_wait(&o_done[t], (j - f_t[t]) & 1, ctl, abort_flag, 25)) { ok = false; break; }
           tc_fence_after();
           issue_s(t, j + 1);
         }
       }
       if (!ok) break;
-      umma_commit(&kv_empty[(2 * j + 1) % 3]);                   // V_j
-      if (j + 1 < n_kv) umma_commit(&kv_empty[(2 * j + 2) % 3]);  // K_{j+1}
+      umma_commit(&kv_empty[(2 * j + 1) % NS]);                   // V_j
+      if (j + 1 < n_kv) umma_commit(&kv_empty[(2 * j + 2) % NS]);  // K_{j+1}
     }
     if (!ok && issued) {
       volatile int never = 0;
       umma_commit(drain);
       mbar_wait(drain, 0, ctl, &never, 28);
     }
-  } else if (warp >= 2) {
-    // ---------------------------------------------- softmax: warpgroup t handles query tile t
-    const int t = (warp - 2) >> 2;
+  }
+  } else {
+    setmaxnreg_inc<kFwdRegsSoftmax>();
+    // ---------------------------------------------- softmax: warpgroup 1 + t handles query tile t
+    const int t = (warp - 4) >> 2;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const int qi = q0 + 128 * t + r;
@@ -250,42 +263,36 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tS = tbase + 128 * t + lane_off;
     const uint32_t tO = tbase + 256 + 128 * t + lane_off;
-    const uint32_t sP = smem_u32(sm + L::P + t * 32768);
     float m = -INFINITY, l = 0.f;
     bool ok = n > 0;
     for (int i = 0; i < n; ++i) {
       if (!mbar_wait(&s_full[t], i & 1, ctl, abort_flag, 29)) { ok = false; break; }
       tc_fence_after();
-      // The row is handled as two halves of 64 scores (two TMEM loads in flight per half):
-      // ten warps leave at most 168 registers per thread, too few to hold all 128 scores.
       const int j = jfirst + i;
       const int kbase = j * 128;
       // masked: the diagonal block (causal), or a block reaching below the window of the tile's
       // last query (keys before qi - win do not exist for query qi)
       const bool dg = (j == diag) || (s.win >= 0 && kbase < q0 + 128 * t + 127 - s.win);
       const int kmin = s.win >= 0 ? qi - s.win : 0;
-      uint32_t raw[64];
+      uint32_t raw[128];
       float* sv = reinterpret_cast<float*>(raw);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32_nowait(tS + 32 * c, raw + 32 * c);
+      tmem_wait_ld();
+      tmem_fence_regs<128>(raw);
+      if (dg) {
+        // keys after the query, past the sequence or before the window do not exist
+#pragma unroll
+        for (int e = 0; e < 128; ++e) {
+          const int key = kbase + e;
+          if (key > qi || key >= s.T || key < kmin) sv[e] = -INFINITY;
+        }
+      }
       float mx8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        tmem_ld32_nowait(tS + hf * 64, raw);
-        tmem_ld32_nowait(tS + hf * 64 + 32, raw + 32);
-        tmem_wait_ld();
-        tmem_fence_regs<64>(raw);
-        if (dg) {
-          // keys after the query, past the sequence or before the window do not exist
-#pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const int key = kbase + hf * 64 + e;
-            if (key > qi || key >= s.T || key < kmin) sv[e] = -INFINITY;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], sv[e], sv[e + 1]);
-      }
+      for (int e = 0; e < 128; e += 2) mx8[(e >> 1) & 7] = fmax3(mx8[(e >> 1) & 7], sv[e], sv[e + 1]);
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= scale_log2;  // -inf when every key of the block lies outside this row's window
@@ -296,7 +303,7 @@ __global__ void __launch_bounds__(320, 1)
         m = m_new;
       }
       if (i > 0) {
-        // O and P_t are still in use by the previous P V product of this tile
+        // O is still in use by the previous P V product of this tile
         if (!mbar_wait(&o_done[t], (i - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -310,48 +317,30 @@ __global__ void __launch_bounds__(320, 1)
           }
         }
       }
-      // P = exp2(s * scale - m) -> shared memory (K-major, 128-byte swizzle; masked scores are
-      // -inf and give 0).  The second half is still in registers; the first is read again.
+      // P = exp2(s * scale - m) as bf16 over score columns [0, 64) (masked scores are -inf and
+      // give 0, or at most 2^-126 on the polynomial path); a row with no visible key yet
+      // (m = -inf) takes 0 as its offset: its scores are all -inf
+      const float m_off = m == -INFINITY ? 0.f : m;
+      const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_off, -m_off);
       float2 rs2[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) rs2[k] = make_float2(0.f, 0.f);
-      // a row with no visible key yet (m = -inf) takes 0 as its offset: its scores are all -inf
-      const float m_off = m == -INFINITY ? 0.f : m;
-      const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_off, -m_off);
 #pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int hf = 1 - it;
-        if (it == 1) {
-          tmem_ld32_nowait(tS, raw);
-          tmem_ld32_nowait(tS + 32, raw + 32);
-          tmem_wait_ld();
-          tmem_fence_regs<64>(raw);
-          if (dg) {
+      for (int g = 0; g < 8; ++g) {
+        uint32_t pw[8];  // keys 16 g .. 16 g + 15, two per word
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-              const int key = kbase + e;
-              if (key > qi || key >= s.T || key < kmin) sv[e] = -INFINITY;
-            }
-          }
+        for (int k = 0; k < 8; ++k) {
+          const int e = 16 * g + 2 * k;
+          const float2 x = ffma2(make_float2(sv[e], sv[e + 1]), sc2, nm2);
+          const float2 pv = ((kPolyGroups >> g) & 1u) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          rs2[k & 3] = fadd2(rs2[k & 3], pv);
+          pw[k] = pack_bf16x2(pv.x, pv.y);
         }
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          float2 pv[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 x = ffma2(make_float2(sv[8 * g + 2 * k], sv[8 * g + 2 * k + 1]), sc2, nm2);
-            pv[k] = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            rs2[k] = fadd2(rs2[k], pv[k]);
-          }
-          // 16-byte unit (hf*8 + g): chunk hf (keys 64*hf ..), unit g within the 128-byte row
-          st_shared_v4(sP + hf * 16384 + sw128_off(r, g),
-                       make_uint4(pack_bf16x2(pv[0].x, pv[0].y), pack_bf16x2(pv[1].x, pv[1].y),
-                                  pack_bf16x2(pv[2].x, pv[2].y), pack_bf16x2(pv[3].x, pv[3].y)));
-        }
+        tmem_st8(tS + 8 * g, pw);
       }
       const float rs = ((rs2[0].x + rs2[0].y) + (rs2[1].x + rs2[1].y)) + ((rs2[2].x + rs2[2].y) + (rs2[3].x + rs2[3].y));
       l = l * alpha + rs;
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
@@ -1008,11 +997,19 @@ static int attn_fwd_launch(const CUtensorMap& tm, const AttnShape& s, __nv_bfloa
                            float scale_log2, cudaStream_t st) {
   using L = FwdSmem<HD>;
   GPTK_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
+  // setmaxnreg.inc waits until the registers it asks for are free in the block's own allocation:
+  // launch only with the allocation the split was made for
+  static const int regs = [] {
+    cudaFuncAttributes fa;
+    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<HD>) == cudaSuccess ? fa.numRegs : 0;
+  }();
+  if (regs * kFwdThreads < 128 * kFwdRegsProducer + 256 * kFwdRegsSoftmax)
+    return set_error(ST_CUDA, "attention forward: built with fewer registers per thread than its warpgroup split");
   // (b, h) fastest, so the heaviest causal pairs of every head start first
   dim3 grid(s.B * s.H, (s.T + 255) / 256);
   const double causal = (double)s.B * s.H * attn_pairs(s.T, s.win);
   Prof prof(PK_ATTN_FWD, 4.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 4, st);
-  attn_fwd_kernel<HD><<<grid, 320, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
+  attn_fwd_kernel<HD><<<grid, kFwdThreads, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }

@@ -1,4 +1,5 @@
 // C ABI of the op-level entry points (include/gpt_ops.h).
+#include <algorithm>
 #include <string>
 
 #include "gemm.cuh"
@@ -22,6 +23,14 @@ __global__ void wait_probe_kernel(DevCtl ctl) {
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait(&bar, 0, ctl, &abort_flag, 99);
 }
+
+// The attention forward's two exponentials, element pairs (x[2i], x[2i+1]) -> out
+__global__ void exp2_pair_kernel(const float* __restrict__ x, long long n_pairs, int poly, float* __restrict__ out) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_pairs; i += (long long)gridDim.x * blockDim.x) {
+    const float2 v = reinterpret_cast<const float2*>(x)[i];
+    reinterpret_cast<float2*>(out)[i] = poly ? exp2_poly2(v) : make_float2(ex2_approx(v.x), ex2_approx(v.y));
+  }
+}
 }  // namespace gptk
 
 extern "C" {
@@ -35,6 +44,20 @@ GPT_API int gpt_op_wait_probe(unsigned long long timeout_ns, void* stream) {
   ctl.timeout_ns = timeout_ns;
   Prof prof(PK_MISC, 0, 0, static_cast<cudaStream_t>(stream));
   wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ctl);
+  GPTK_CUDA(cudaGetLastError());
+  return ST_OK;
+}
+
+GPT_API int gpt_op_exp2(const float* x, long long n, int poly, float* out, void* stream) {
+  set_error(ST_OK, "");
+  if (n < 0 || (n & 1)) return set_error(ST_INVALID_ARG, "exp2: n must be even and >= 0");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 7)
+    return set_error(ST_INVALID_ARG, "exp2: x and out must be 8-byte aligned");
+  if (n == 0) return ST_OK;
+  Prof prof(PK_MISC, 0, 8.0 * n, static_cast<cudaStream_t>(stream));
+  const long long pairs = n / 2;
+  const int grid = static_cast<int>(std::min<long long>((pairs + 255) / 256, 4096));
+  exp2_pair_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, pairs, poly, out);
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }

@@ -547,6 +547,39 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// 2^x for two values at once on the FMA and integer pipes instead of the MUFU unit, so that a
+// kernel bound by the MUFU's 16 results per clock can move part of its exponentials elsewhere.
+// Range reduction x = n + f with n = rint(x), taken exactly from the low mantissa bits of
+// x + 1.5 * 2^23 (f in [-1/2, 1/2]); 2^f from a degree-4 polynomial, the Remez minimax fit of 2^f
+// on [-1/2, 1/2] in relative error computed for this library (2.6e-6 exactly, 2.7e-6 with these
+// fp32 coefficients and Horner steps); n added to the exponent field.  Within that error for
+// -125 <= x <= 127; x is clamped below at -126, so x < -125 (-inf included) gives a value in
+// [0, 2^-125] instead of 2^x.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.f;  // 1.5 * 2^23
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 j = fadd2(x, make_float2(kShift, kShift));
+  const float2 n = fadd2(j, make_float2(-kShift, -kShift));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);  // x - n, exact
+  float2 q = ffma2(make_float2(0.009570102207362652f, 0.009570102207362652f), f,
+                   make_float2(0.05591785907745361f, 0.05591785907745361f));
+  q = ffma2(q, f, make_float2(0.240247443318367f, 0.240247443318367f));
+  q = ffma2(q, f, make_float2(0.6931217908859253f, 0.6931217908859253f));
+  q = ffma2(q, f, make_float2(0.9999992847442627f, 0.9999992847442627f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23)));
+}
+
+// Register budget of a warpgroup (all 128 threads execute it): give back / take registers.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Hardware square root (sqrt.approx: +0 maps to +0; its error of a few ulp is far below bf16
 // rounding).  The IEEE sqrtf leaves its fast path for zero inputs, which ReLU^2 makes common.
 __device__ __forceinline__ float sqrt_approx(float x) {

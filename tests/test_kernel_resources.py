@@ -23,7 +23,7 @@ CSRC = os.path.join(ROOT, "decoder_only_gpt_tcgen05_b200", "csrc")
 # threads per block of each kernel's largest launch (the __launch_bounds__ where it has one)
 BLOCK_THREADS = [
     (r"gemm_kernel", 320),               # TMA warp, MMA warp, 8 epilogue warps (long-K: 4)
-    (r"attn_fwd_kernel", 320),           # TMA warp, MMA warp, two softmax warpgroups
+    (r"attn_fwd_kernel", 384),           # TMA, MMA and two idle warps; two softmax warpgroups
     (r"attn_bwd_(dkv|dq)_kernel", 576),  # TMA warp, MMA warp, 16 elementwise warps
     (r"offsets_kernel", 1024),
     (r".*", 256),                        # every other kernel: blocks of at most 256 threads
