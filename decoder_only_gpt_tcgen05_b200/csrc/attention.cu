@@ -28,6 +28,7 @@
 //               S = Q K^T and dP = dO V^T into TMEM; dS as bf16 into a TMEM buffer, the A
 //               operand of dQ += dS K
 // Both are deterministic (no atomics).  Every wait is bounded (see ptx.cuh).
+#include <algorithm>
 #include <cmath>
 
 #include "host.cuh"
@@ -36,6 +37,7 @@
 namespace gptk {
 
 static constexpr float kLog2e = 1.4426950408889634f;
+
 
 // ====================================================================== forward
 // One CTA per (b, h, pair of 128-query tiles A = 2p, B = 2p+1): two softmax warpgroups, one
@@ -380,8 +382,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
 }
 
+// The w-th item of CTA c in a grid of G CTAs: round r deals items r G .. r G + G - 1, to the
+// CTAs in order on even rounds and in reverse on odd ones, so that every CTA gets a similar mix
+// of the heavy and light items of a list sorted heaviest first.
+__device__ __forceinline__ int zigzag_item(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+
 // ====================================================================== backward: dK, dV
-// One CTA per 128-key tile, stepping over 128-query blocks from the diagonal block on.
+// Persistent: one CTA per SM walks a list of (b, h, 128-key tile) items, heaviest tiles first,
+// dealt to the CTAs in zigzag order; for each item it steps over 128-query blocks from the
+// diagonal block on.
 //   S^T = K Q^T and dP^T = V dO^T go into TMEM (M = 128 keys, N = 128 queries, full-rate MMAs).
 //   Sixteen elementwise warps turn them into P^T = exp2(S^T scale - lse) and
 //   dS^T = P^T (dP^T - delta) and write both back as bf16 over the fp32 columns each warp has
@@ -390,6 +399,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 //   The block's queries go in two halves: the dV/dK products of the first half run while the
 //   elementwise warps work on the second.
 // TMEM: S^T/P^T [0,128), dP^T/dS^T [128,256), dV [256, 256+HD), dK [384, 384+HD).
+// Across items nothing waits for a whole CTA to drain: the next item's K and V load as soon as
+// the last S^T / dP^T products of the current one have read theirs, the query-block ring runs on
+// without a break, and the next item's first S^T / dP^T products run while the elementwise
+// warps write the current item's dK and dV out of TMEM.
 // The per-query statistics (lse in log2 units, delta) of each block are staged in shared
 // memory by the elementwise warps, loaded from global memory one block ahead.
 
@@ -407,6 +420,14 @@ struct DkvSmem {
   static constexpr int BAR = STATS + 2048;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
+
+// The query blocks of key tile kt: from the diagonal block on, up to the last query whose window
+// still reaches the tile's last key.
+__device__ __forceinline__ int dkv_blocks(const AttnShape& s, int kt) {
+  int n = (s.T + 127) / 128 - kt;
+  if (s.win >= 0) n = min(n, (kt * 128 + 127 + s.win) / 128 - kt + 1);
+  return n;
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -427,23 +448,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* stats_bar = bars + 9;  // [2]
   uint64_t* acc_full = bars + 11;
   uint64_t* drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* kv_empty = bars + 13;
+  uint64_t* acc_empty = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* stats = reinterpret_cast<float*>(sm + L::STATS);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kt = blockIdx.x;  // the tiles of one head run side by side (they share Q and dO in L2)
-  const int bh = blockIdx.y;
-  const int b = bh / s.H, h = bh % s.H;
-  const int k0 = kt * 128;
-  // query blocks from the diagonal one on, up to the last query whose window still reaches this
-  // tile's last key
-  int n_it = (s.T + 127) / 128 - kt;
-  if (s.win >= 0) n_it = min(n_it, (k0 + 127 + s.win) / 128 - kt + 1);
+  const int n_kt = (s.T + 127) / 128;
+  const int BH = s.B * s.H;
+  const int n_items = n_kt * BH;  // item w: key tile w / BH (heaviest first), head w % BH
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
@@ -453,6 +472,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(s_full, 1);
     mbar_init(d_done, 1);
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kBwdEw);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -470,43 +490,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tdV = tbase + 256;
   const uint32_t tdK = tbase + 384;
 
-  const int colq = h * s.hdp;
-  const int colk = s.H * s.hdp + h * s.hdp;
-  const int colv = 2 * s.H * s.hdp + h * s.hdp;
-  const int cold = h * s.hdp;
-
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer
     bool ok = true;
-    mbar_expect_tx(kv_full, 2 * L::TILE);
-    for (int c = 0; c < NCH; ++c) {
-      tma_load_3d(sm + L::K + c * 16384, &tm_kv128, kv_full, colk + 64 * c, k0, b);
-      tma_load_3d(sm + L::V + c * 16384, &tm_kv128, kv_full, colv + 64 * c, k0, b);
-    }
-    int issued = -1;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int st = it & 1;
-      if (!mbar_wait(&q_empty[st], ((it >> 1) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
-      const int qb = (kt + it) * 128;
-      mbar_expect_tx(&q_full[st], 2 * L::TILE);
+    int g = 0;                    // query blocks loaded, over all items
+    int kv_issued = -1, issued_g = -1;
+    for (int r = 0; ok; ++r) {
+      const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+      if (w >= n_items) break;
+      const int kt = w / BH, bh = w % BH;
+      const int b = bh / s.H, h = bh % s.H;
+      const int colk = s.H * s.hdp + h * s.hdp, colv = 2 * s.H * s.hdp + h * s.hdp;
+      const int colq = h * s.hdp, cold = h * s.hdp;
+      // K and V of the previous item are read by its S^T / dP^T products until kv_empty
+      if (r > 0 && !mbar_wait(kv_empty, (r - 1) & 1, ctl, abort_flag, 40)) { ok = false; break; }
+      mbar_expect_tx(kv_full, 2 * L::TILE);
       for (int c = 0; c < NCH; ++c) {
-        tma_load_3d(sm + L::Q0 + st * L::TILE + c * 16384, &tm_q128, &q_full[st], colq + 64 * c, qb, b);
-        tma_load_3d(sm + L::DO0 + st * L::TILE + c * 16384, &tm_do128, &q_full[st], cold + 64 * c, qb, b);
+        tma_load_3d(sm + L::K + c * 16384, &tm_kv128, kv_full, colk + 64 * c, kt * 128, b);
+        tma_load_3d(sm + L::V + c * 16384, &tm_kv128, kv_full, colv + 64 * c, kt * 128, b);
       }
-      issued = it;
+      kv_issued = r;
+      const int n_it = dkv_blocks(s, kt);
+      for (int it = 0; it < n_it; ++it, ++g) {
+        const int st = g & 1;
+        if (!mbar_wait(&q_empty[st], ((g >> 1) & 1) ^ 1u, ctl, abort_flag, 40)) { ok = false; break; }
+        const int qb = (kt + it) * 128;
+        mbar_expect_tx(&q_full[st], 2 * L::TILE);
+        for (int c = 0; c < NCH; ++c) {
+          tma_load_3d(sm + L::Q0 + st * L::TILE + c * 16384, &tm_q128, &q_full[st], colq + 64 * c, qb, b);
+          tma_load_3d(sm + L::DO0 + st * L::TILE + c * 16384, &tm_do128, &q_full[st], cold + 64 * c, qb, b);
+        }
+        issued_g = g;
+      }
     }
     if (!ok) {
       // wait (bounded) for the copies still in flight before the CTA goes away
       volatile int never = 0;
-      mbar_wait(kv_full, 0, ctl, &never, 41);
-      for (int it = (issued >= 2 ? issued - 1 : 0); it <= issued && issued >= 0; ++it)
-        mbar_wait(&q_full[it & 1], (it >> 1) & 1, ctl, &never, 41);
+      if (kv_issued >= 0) mbar_wait(kv_full, kv_issued & 1, ctl, &never, 41);
+      for (int gg = (issued_g >= 1 ? issued_g - 1 : 0); gg <= issued_g && issued_g >= 0; ++gg)
+        mbar_wait(&q_full[gg & 1], (gg >> 1) & 1, ctl, &never, 41);
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t idesc_d = idesc_bf16(128, HD, 0, 1);
-    bool ok = mbar_wait(kv_full, 0, ctl, abort_flag, 42);
+    bool ok = true;
     bool issued = false;
     // operand descriptors, computed once: K-major K, V, Q, dO; MN-major Q, dO for dK, dV
     const uint64_t dK = sdesc_sw128(smem_u32(sm + L::K), 16, 1024);
@@ -519,57 +547,67 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       dQm[i] = sdesc_sw128(smem_u32(sm + L::Q0 + i * L::TILE), 16384, 1024);
       dDm[i] = sdesc_sw128(smem_u32(sm + L::DO0 + i * L::TILE), 16384, 1024);
     }
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int st = it & 1;
-      if (!mbar_wait(&q_full[st], (it >> 1) & 1, ctl, abort_flag, 43)) { ok = false; break; }
-      // the S^T / dP^T columns still hold the previous block's P^T / dS^T until its products finish
-      if (it > 0 && !mbar_wait(d_done, (it - 1) & 1, ctl, abort_flag, 44)) { ok = false; break; }
-      tc_fence_after();
-      const uint64_t dQ = st ? dQk[1] : dQk[0], dD = st ? dDk[1] : dDk[0];
-      const uint64_t dQn = st ? dQm[1] : dQm[0], dDn = st ? dDm[1] : dDm[0];
-      // S^T and dP^T, interleaved, in groups of four K steps issued back to back
-#pragma unroll
-      for (int g = 0; g < HD / 64; ++g) {
-        uint32_t dd[8];
-        uint64_t aa[8], bb[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t off = g * 16384 + i * 32;
-          dd[2 * i] = tS;
-          dd[2 * i + 1] = tdP;
-          aa[2 * i] = sdesc_add(dK, off);
-          aa[2 * i + 1] = sdesc_add(dV, off);
-          bb[2 * i] = sdesc_add(dQ, off);
-          bb[2 * i + 1] = sdesc_add(dD, off);
-        }
-        umma8_ss(dd, aa, bb, idesc_s, g == 0 ? 0xfcu : 0xffu);
-      }
-      umma_commit(s_full);
-      issued = true;
-      for (int hh = 0; hh < 2 && ok; ++hh) {
-        if (!mbar_wait(&h_full[hh], it & 1, ctl, abort_flag, 45)) { ok = false; break; }
+    int g = 0;
+    for (int r = 0; ok; ++r) {
+      const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+      if (w >= n_items) break;
+      const int n_it = dkv_blocks(s, w / BH);
+      if (!mbar_wait(kv_full, r & 1, ctl, abort_flag, 42)) { ok = false; break; }
+      for (int it = 0; it < n_it && ok; ++it, ++g) {
+        const int st = g & 1;
+        if (!mbar_wait(&q_full[st], (g >> 1) & 1, ctl, abort_flag, 43)) { ok = false; break; }
+        // the S^T / dP^T columns still hold the previous block's P^T / dS^T until its products finish
+        if (g > 0 && !mbar_wait(d_done, (g - 1) & 1, ctl, abort_flag, 44)) { ok = false; break; }
         tc_fence_after();
-        uint32_t dd[8], aa[8];
-        uint64_t bb[8];
+        const uint64_t dQ = st ? dQk[1] : dQk[0], dD = st ? dDk[1] : dDk[0];
+        const uint64_t dQn = st ? dQm[1] : dQm[0], dDn = st ? dDm[1] : dDm[0];
+        // S^T and dP^T, interleaved, in groups of four K steps issued back to back
 #pragma unroll
-        for (int kq = 0; kq < 4; ++kq) {
-          const int kk = 4 * hh + kq;  // 16 queries
-          dd[2 * kq] = tdV;
-          dd[2 * kq + 1] = tdK;
-          aa[2 * kq] = tS + 16 * kk;
-          aa[2 * kq + 1] = tdP + 16 * kk;
-          bb[2 * kq] = sdesc_add(dDn, kk * 2048);
-          bb[2 * kq + 1] = sdesc_add(dQn, kk * 2048);
+        for (int gq = 0; gq < HD / 64; ++gq) {
+          uint32_t dd[8];
+          uint64_t aa[8], bb[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t off = gq * 16384 + i * 32;
+            dd[2 * i] = tS;
+            dd[2 * i + 1] = tdP;
+            aa[2 * i] = sdesc_add(dK, off);
+            aa[2 * i + 1] = sdesc_add(dV, off);
+            bb[2 * i] = sdesc_add(dQ, off);
+            bb[2 * i + 1] = sdesc_add(dD, off);
+          }
+          umma8_ss(dd, aa, bb, idesc_s, gq == 0 ? 0xfcu : 0xffu);
         }
-        umma8_ts(dd, aa, bb, idesc_d, (hh == 0 && it == 0) ? 0xfcu : 0xffu);
+        umma_commit(s_full);
+        if (it == n_it - 1) umma_commit(kv_empty);  // the item's K and V are no longer read
+        issued = true;
+        // dV and dK of the previous item are in TMEM until the elementwise warps have read them
+        if (it == 0 && r > 0 && !mbar_wait(acc_empty, (r - 1) & 1, ctl, abort_flag, 48)) { ok = false; break; }
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+          if (!mbar_wait(&h_full[hh], g & 1, ctl, abort_flag, 45)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t dd[8], aa[8];
+          uint64_t bb[8];
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            const int kk = 4 * hh + kq;  // 16 queries
+            dd[2 * kq] = tdV;
+            dd[2 * kq + 1] = tdK;
+            aa[2 * kq] = tS + 16 * kk;
+            aa[2 * kq + 1] = tdP + 16 * kk;
+            bb[2 * kq] = sdesc_add(dDn, kk * 2048);
+            bb[2 * kq + 1] = sdesc_add(dQn, kk * 2048);
+          }
+          umma8_ts(dd, aa, bb, idesc_d, (hh == 0 && it == 0) ? 0xfcu : 0xffu);
+        }
+        if (!ok) break;
+        umma_commit(d_done);
+        umma_commit(&q_empty[st]);
       }
       if (!ok) break;
-      umma_commit(d_done);
-      umma_commit(&q_empty[st]);
-    }
-    if (ok) {
       umma_commit(acc_full);
-    } else if (issued) {
+    }
+    if (!ok && issued) {
       volatile int never = 0;
       umma_commit(drain);
       mbar_wait(drain, 0, ctl, &never, 46);
@@ -578,91 +616,117 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------ elementwise warps
     const int ew = warp - 2;         // 0..15
     const int quad = warp & 3;       // TMEM lane quadrant: keys 32 quad .. 32 quad + 31
-    const int w = ew >> 2;           // 16-query group within each half
-    const int r = quad * 32 + lane;  // key row within the tile
-    const int key = k0 + r;
+    const int wq = ew >> 2;          // 16-query group within each half
+    const int r_key = quad * 32 + lane;  // key row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const float* lse_bh = lse + (long long)bh * s.T;
-    const float* del_bh = delta + (long long)bh * s.T;
     // statistics staging: this warp owns 8 queries of each block (lanes 0-7 lse, 8-15 delta)
     const int qq = 8 * ew + (lane & 7);
-    auto stat_of = [&](int qb) -> float {
+    auto stat_of = [&](int bh, int qb) -> float {
       const int q = qb + qq;
       if (lane >= 16 || q >= s.T) return 0.f;
-      return lane < 8 ? __ldg(lse_bh + q) * kLog2e : __ldg(del_bh + q);
+      return lane < 8 ? __ldg(lse + (long long)bh * s.T + q) * kLog2e : __ldg(delta + (long long)bh * s.T + q);
     };
-    float v_next = stat_of(k0);
-    bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
-      const int st = it & 1;
-      const int qb = (kt + it) * 128;
-      if (lane < 16) stats[st * 256 + (lane < 8 ? 0 : 128) + qq] = v_next;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&stats_bar[st]);
-      if (it + 1 < n_it) v_next = stat_of(qb + 128);  // one block ahead
-      if (!mbar_wait(&stats_bar[st], (it >> 1) & 1, ctl, abort_flag, 50)) { ok = false; break; }
-      if (!mbar_wait(s_full, it & 1, ctl, abort_flag, 47)) { ok = false; break; }
-      tc_fence_after();
-      // the diagonal block, the ragged end, or a block whose last query's window misses the
-      // tile's first key
-      const bool masked = (it == 0) || (qb + 128 > s.T) || (s.win >= 0 && qb + 127 - s.win > k0);
-      for (int hh = 0; hh < 2; ++hh) {
-        const int c = 4 * hh + w;  // queries qb + 16c .. qb + 16c + 15
-        uint32_t rs[16], rd[16];
-        tmem_ld16_nowait(tS + lane_off + 16 * c, rs);
-        tmem_ld16_nowait(tdP + lane_off + 16 * c, rd);
-        tmem_wait_ld();
-        tmem_fence_regs<16>(rs);
-        tmem_fence_regs<16>(rd);
-        const float* stl = stats + st * 256 + 16 * c;
-        uint32_t pw[8], dw[8];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float4 l4 = *reinterpret_cast<const float4*>(stl + 4 * g);
-          const float4 d4 = *reinterpret_cast<const float4*>(stl + 128 + 4 * g);
-          const float l2[4] = {l4.x, l4.y, l4.z, l4.w};
-          const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
-          float p[4], ds[4];
-          if (masked) {  // the diagonal block or the ragged end: causal / range mask
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 4 * g + k;
-              const int q = qb + 16 * c + e;
-              float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
-              if (q < key || q >= s.T || (s.win >= 0 && q - s.win > key)) pv = 0.f;
-              p[k] = pv;
-              ds[k] = pv * (__uint_as_float(rd[e]) - dl[k]);
-            }
-          } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = 4 * g + k;
-              p[k] = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
-              ds[k] = p[k] * (__uint_as_float(rd[e]) - dl[k]);
-            }
-          }
-          pw[2 * g] = pack_bf16x2(p[0], p[1]);
-          pw[2 * g + 1] = pack_bf16x2(p[2], p[3]);
-          dw[2 * g] = pack_bf16x2(ds[0], ds[1]);
-          dw[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
-        }
-        // bf16 P^T and dS^T over the first 8 of the 16 columns this warp has just read
-        tmem_st8(tS + lane_off + 16 * c, pw);
-        tmem_st8(tdP + lane_off + 16 * c, dw);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&h_full[hh]);
+    // the block after (item r, block it): the next block of the item, else the next item's first
+    auto next_block = [&](int r, int it, int n_it, int& bh_n, int& qb_n) -> bool {
+      if (it + 1 < n_it) {
+        const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+        bh_n = w % BH;
+        qb_n = (w / BH + it + 1) * 128;
+        return true;
       }
+      const int w = zigzag_item(r + 1, blockIdx.x, gridDim.x);
+      if (w >= n_items) return false;
+      bh_n = w % BH;
+      qb_n = (w / BH) * 128;
+      return true;
+    };
+    bool ok = true;
+    int g = 0;
+    float v_next = 0.f;
+    {
+      const int w0 = zigzag_item(0, blockIdx.x, gridDim.x);
+      if (w0 < n_items) v_next = stat_of(w0 % BH, (w0 / BH) * 128);
     }
-    // epilogue: the four warps of a quadrant split dK (times the softmax scale) and dV
-    if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 49)) {
+    for (int r = 0; ok; ++r) {
+      const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+      if (w >= n_items) break;
+      const int kt = w / BH, bh = w % BH;
+      const int b = bh / s.H, h = bh % s.H;
+      const int k0 = kt * 128;
+      const int key = k0 + r_key;
+      const int n_it = dkv_blocks(s, kt);
+      for (int it = 0; it < n_it; ++it, ++g) {
+        const int st = g & 1;
+        const int qb = (kt + it) * 128;
+        if (lane < 16) stats[st * 256 + (lane < 8 ? 0 : 128) + qq] = v_next;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&stats_bar[st]);
+        int bh_n, qb_n;
+        if (next_block(r, it, n_it, bh_n, qb_n)) v_next = stat_of(bh_n, qb_n);  // one block ahead
+        if (!mbar_wait(&stats_bar[st], (g >> 1) & 1, ctl, abort_flag, 50)) { ok = false; break; }
+        if (!mbar_wait(s_full, g & 1, ctl, abort_flag, 47)) { ok = false; break; }
+        tc_fence_after();
+        // the diagonal block, the ragged end, or a block whose last query's window misses the
+        // tile's first key
+        const bool masked = (it == 0) || (qb + 128 > s.T) || (s.win >= 0 && qb + 127 - s.win > k0);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int c = 4 * hh + wq;  // queries qb + 16c .. qb + 16c + 15
+          uint32_t rs[16], rd[16];
+          tmem_ld16_nowait(tS + lane_off + 16 * c, rs);
+          tmem_ld16_nowait(tdP + lane_off + 16 * c, rd);
+          tmem_wait_ld();
+          tmem_fence_regs<16>(rs);
+          tmem_fence_regs<16>(rd);
+          const float* stl = stats + st * 256 + 16 * c;
+          uint32_t pw[8], dw[8];
+#pragma unroll
+          for (int gg = 0; gg < 4; ++gg) {
+            const float4 l4 = *reinterpret_cast<const float4*>(stl + 4 * gg);
+            const float4 d4 = *reinterpret_cast<const float4*>(stl + 128 + 4 * gg);
+            const float l2[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float dl[4] = {d4.x, d4.y, d4.z, d4.w};
+            float p[4], ds[4];
+            if (masked) {  // the diagonal block or the ragged end: causal / range mask
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int e = 4 * gg + k;
+                const int q = qb + 16 * c + e;
+                float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
+                if (q < key || q >= s.T || (s.win >= 0 && q - s.win > key)) pv = 0.f;
+                p[k] = pv;
+                ds[k] = pv * (__uint_as_float(rd[e]) - dl[k]);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int e = 4 * gg + k;
+                p[k] = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -l2[k]));
+                ds[k] = p[k] * (__uint_as_float(rd[e]) - dl[k]);
+              }
+            }
+            pw[2 * gg] = pack_bf16x2(p[0], p[1]);
+            pw[2 * gg + 1] = pack_bf16x2(p[2], p[3]);
+            dw[2 * gg] = pack_bf16x2(ds[0], ds[1]);
+            dw[2 * gg + 1] = pack_bf16x2(ds[2], ds[3]);
+          }
+          // bf16 P^T and dS^T over the first 8 of the 16 columns this warp has just read
+          tmem_st8(tS + lane_off + 16 * c, pw);
+          tmem_st8(tdP + lane_off + 16 * c, dw);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&h_full[hh]);
+        }
+      }
+      if (!ok) break;
+      // epilogue: the four warps of a quadrant split dK (times the softmax scale) and dV
+      if (!mbar_wait(acc_full, r & 1, ctl, abort_flag, 49)) { ok = false; break; }
       tc_fence_after();
       constexpr int CPW = HD / 2;  // columns per warp
       const bool row_ok = key < s.T;
       const long long m = (long long)b * s.T + key;
-      const int which = w >> 1;  // 0: dK, 1: dV
-      const int cbase = (w & 1) * CPW;
+      const int which = wq >> 1;  // 0: dK, 1: dV
+      const int cbase = (wq & 1) * CPW;
       __nv_bfloat16* dst = dqkv + m * s.ld_qkv + (long long)(1 + which) * s.H * s.hdp + (long long)h * s.hdp;
       const uint32_t tsrc = (which == 0 ? tdK : tdV) + lane_off;
       const float f = which == 0 ? scale : 1.f;
@@ -672,13 +736,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32(tsrc + c, a);
         if (row_ok) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            reinterpret_cast<uint4*>(dst + c)[g] =
-                make_uint4(pack_bf16x2(a[8 * g] * f, a[8 * g + 1] * f), pack_bf16x2(a[8 * g + 2] * f, a[8 * g + 3] * f),
-                           pack_bf16x2(a[8 * g + 4] * f, a[8 * g + 5] * f),
-                           pack_bf16x2(a[8 * g + 6] * f, a[8 * g + 7] * f));
+          for (int gg = 0; gg < 4; ++gg)
+            reinterpret_cast<uint4*>(dst + c)[gg] =
+                make_uint4(pack_bf16x2(a[8 * gg] * f, a[8 * gg + 1] * f), pack_bf16x2(a[8 * gg + 2] * f, a[8 * gg + 3] * f),
+                           pack_bf16x2(a[8 * gg + 4] * f, a[8 * gg + 5] * f),
+                           pack_bf16x2(a[8 * gg + 6] * f, a[8 * gg + 7] * f));
         }
       }
+      // dK and dV have been read: the next item's products may overwrite them
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
 
@@ -690,13 +758,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ====================================================================== backward: dQ
-// One CTA per 128-query tile, stepping over 128-key blocks up to the diagonal one:
+// Persistent like the dK/dV kernel: one CTA per SM walks (b, h, 128-query tile) items, heaviest
+// tiles first, dealt in zigzag order; for each item it steps over 128-key blocks up to the
+// diagonal one:
 //   S = Q K^T and dP = dO V^T into TMEM (N = 128, full rate); sixteen elementwise warps write
 //   dS = P (dP - delta) as bf16 into one of two TMEM buffers, from which dQ += dS K takes its
 //   A operand.  S and dP are free again as soon as the elementwise warps have loaded them, so
 //   the next block's S / dP products run while this block's dS is computed.
 // TMEM: S [0,128), dP [128,256), dQ [256, 256+HD), dS [2] at 384 and 448.
-// Shared memory: Q, dO, a 3-deep K ring (K is read by S and by dQ) and a 2-deep V ring.
+// Shared memory: Q, dO, a 3-deep K ring (K is read by S and by dQ) and a 2-deep V ring; the
+// rings run on across items, and the next item's Q and dO load once the current item's last
+// S / dP products have read theirs.
 
 template <int HD>
 struct DqSmem {
@@ -709,6 +781,12 @@ struct DqSmem {
   static constexpr int BAR = V0 + VS * TILE;
   static constexpr int BYTES = BAR + 256 + 1024;
 };
+
+// The key blocks of query tile qt: j0 .. qt (the last one is the diagonal block; j0 > 0 when the
+// first query's window starts past key 0).
+__device__ __forceinline__ int dq_first_block(const AttnShape& s, int qt) {
+  return s.win >= 0 ? max(0, (qt * 128 - s.win) / 128) : 0;
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -732,23 +810,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ds_empty = s_full + 4;         // [2]
   uint64_t* acc_full = s_full + 6;
   uint64_t* drain = s_full + 7;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 8);
+  uint64_t* q_empty = s_full + 8;
+  uint64_t* acc_empty = s_full + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = gridDim.x;
-  const int qt = n_qt - 1 - blockIdx.x;  // heaviest tiles of each head first
-  const int bh = blockIdx.y;
-  const int b = bh / s.H, h = bh % s.H;
-  const int q0 = qt * 128;
-  // 128-key blocks j0 .. qt (the last one is the diagonal block; j0 > 0 when the first query's
-  // window starts past key 0); the rings count blocks from j0
-  const int j0 = s.win >= 0 ? max(0, (q0 - s.win) / 128) : 0;
-  const int n_kv = qt + 1 - j0;
+  const int n_qt = (s.T + 127) / 128;
+  const int BH = s.B * s.H;
+  const int n_items = n_qt * BH;  // item w: query tile n_qt - 1 - w / BH (heaviest first), head w % BH
   constexpr int NCH = HD / 64;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < KS; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -764,6 +839,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&ds_empty[i], 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kBwdEw);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -781,37 +857,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tdQ = tbase + 256;
   const uint32_t tdS = tbase + 384;  // [2] x 64 columns
 
-  const int colq = h * s.hdp;
-  const int colk = s.H * s.hdp + h * s.hdp;
-  const int colv = 2 * s.H * s.hdp + h * s.hdp;
-  const int cold = h * s.hdp;
-
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer
     bool ok = true;
-    mbar_expect_tx(q_full, 2 * L::TILE);
-    for (int c = 0; c < NCH; ++c) {
-      tma_load_3d(sm + L::Q + c * 16384, &tm_q128, q_full, colq + 64 * c, q0, b);
-      tma_load_3d(sm + L::DO + c * 16384, &tm_do128, q_full, cold + 64 * c, q0, b);
-    }
-    int issued_k = -1, issued_v = -1;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      const int ks = j % KS;
-      if (!mbar_wait(&k_empty[ks], ((j / KS) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
-      mbar_expect_tx(&k_full[ks], L::TILE);
-      for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::K0 + ks * L::TILE + c * 16384, &tm_kv128, &k_full[ks], colk + 64 * c, (j0 + j) * 128, b);
-      issued_k = j;
-      const int vs = j % VS;
-      if (!mbar_wait(&v_empty[vs], ((j / VS) & 1) ^ 1u, ctl, abort_flag, 61)) { ok = false; break; }
-      mbar_expect_tx(&v_full[vs], L::TILE);
-      for (int c = 0; c < NCH; ++c)
-        tma_load_3d(sm + L::V0 + vs * L::TILE + c * 16384, &tm_kv128, &v_full[vs], colv + 64 * c, (j0 + j) * 128, b);
-      issued_v = j;
+    int gj = 0;  // key blocks loaded, over all items
+    int q_issued = -1, issued_k = -1, issued_v = -1;
+    for (int r = 0; ok; ++r) {
+      const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+      if (w >= n_items) break;
+      const int qt = n_qt - 1 - w / BH, bh = w % BH;
+      const int b = bh / s.H, h = bh % s.H;
+      const int colq = h * s.hdp, cold = h * s.hdp;
+      const int colk = s.H * s.hdp + h * s.hdp, colv = 2 * s.H * s.hdp + h * s.hdp;
+      const int j0 = dq_first_block(s, qt);
+      const int n_kv = qt + 1 - j0;
+      // Q and dO of the previous item are read by its S / dP products until q_empty
+      if (r > 0 && !mbar_wait(q_empty, (r - 1) & 1, ctl, abort_flag, 60)) { ok = false; break; }
+      mbar_expect_tx(q_full, 2 * L::TILE);
+      for (int c = 0; c < NCH; ++c) {
+        tma_load_3d(sm + L::Q + c * 16384, &tm_q128, q_full, colq + 64 * c, qt * 128, b);
+        tma_load_3d(sm + L::DO + c * 16384, &tm_do128, q_full, cold + 64 * c, qt * 128, b);
+      }
+      q_issued = r;
+      for (int j = 0; j < n_kv && ok; ++j, ++gj) {
+        const int ks = gj % KS;
+        if (!mbar_wait(&k_empty[ks], ((gj / KS) & 1) ^ 1u, ctl, abort_flag, 60)) { ok = false; break; }
+        mbar_expect_tx(&k_full[ks], L::TILE);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_3d(sm + L::K0 + ks * L::TILE + c * 16384, &tm_kv128, &k_full[ks], colk + 64 * c, (j0 + j) * 128, b);
+        issued_k = gj;
+        const int vs = gj % VS;
+        if (!mbar_wait(&v_empty[vs], ((gj / VS) & 1) ^ 1u, ctl, abort_flag, 61)) { ok = false; break; }
+        mbar_expect_tx(&v_full[vs], L::TILE);
+        for (int c = 0; c < NCH; ++c)
+          tma_load_3d(sm + L::V0 + vs * L::TILE + c * 16384, &tm_kv128, &v_full[vs], colv + 64 * c, (j0 + j) * 128, b);
+        issued_v = gj;
+      }
     }
     if (!ok) {
       volatile int never = 0;
-      mbar_wait(q_full, 0, ctl, &never, 62);
+      if (q_issued >= 0) mbar_wait(q_full, q_issued & 1, ctl, &never, 62);
       for (int j = (issued_k >= KS ? issued_k - KS + 1 : 0); j <= issued_k && issued_k >= 0; ++j)
         mbar_wait(&k_full[j % KS], (j / KS) & 1, ctl, &never, 62);
       for (int j = (issued_v >= VS ? issued_v - VS + 1 : 0); j <= issued_v && issued_v >= 0; ++j)
@@ -821,30 +906,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_s = idesc_bf16(128, 128, 0, 0);
     constexpr uint32_t idesc_d = idesc_bf16(128, HD, 0, 1);
-    bool ok = mbar_wait(q_full, 0, ctl, abort_flag, 63);
+    bool ok = true;
     bool issued = false;
     const uint64_t dQ = sdesc_sw128(smem_u32(sm + L::Q), 16, 1024);
     const uint64_t dD = sdesc_sw128(smem_u32(sm + L::DO), 16, 1024);
     const uint64_t dK0 = sdesc_sw128(smem_u32(sm + L::K0), 16, 1024);       // K-major, stage 0
     const uint64_t dKm0 = sdesc_sw128(smem_u32(sm + L::K0), 16384, 1024);   // MN-major, stage 0
     const uint64_t dV0 = sdesc_sw128(smem_u32(sm + L::V0), 16, 1024);
-    for (int j = 0; j <= n_kv && ok; ++j) {
-      if (j < n_kv) {
-        const int ks = j % KS, vs = j % VS;
-        if (!mbar_wait(&k_full[ks], (j / KS) & 1, ctl, abort_flag, 64)) { ok = false; break; }
-        if (!mbar_wait(&v_full[vs], (j / VS) & 1, ctl, abort_flag, 64)) { ok = false; break; }
+    // The block sequence over all items: S / dP of global block gj go out one step ahead of the
+    // dQ product of block gj - 1, so that the next block's scores overlap this block's dS.
+    int gj = 0;        // next block whose S / dP to issue
+    int r_s = 0;       // item of block gj, and its block index within the item
+    int j_s = 0;
+    int n_s = -1;      // blocks of item r_s (-1: not yet looked up)
+    int r_d = 0, j_d = 0, n_d = -1;  // the same for the next dQ product
+    auto item_blocks = [&](int r) -> int {
+      const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+      if (w >= n_items) return -1;
+      const int qt = n_qt - 1 - w / BH;
+      return qt + 1 - dq_first_block(s, qt);
+    };
+    n_s = item_blocks(0);
+    n_d = n_s;
+    int gd = 0;  // next block whose dQ product to issue
+    while (ok && (n_s > 0 || n_d > 0)) {
+      if (n_s > 0) {
+        const int ks = gj % KS, vs = gj % VS;
+        if (j_s == 0 && !mbar_wait(q_full, r_s & 1, ctl, abort_flag, 63)) { ok = false; break; }
+        if (!mbar_wait(&k_full[ks], (gj / KS) & 1, ctl, abort_flag, 64)) { ok = false; break; }
+        if (!mbar_wait(&v_full[vs], (gj / VS) & 1, ctl, abort_flag, 64)) { ok = false; break; }
         // S / dP are free once the elementwise warps have loaded the previous block's
-        if (j > 0 && !mbar_wait(s_free, (j - 1) & 1, ctl, abort_flag, 65)) { ok = false; break; }
+        if (gj > 0 && !mbar_wait(s_free, (gj - 1) & 1, ctl, abort_flag, 65)) { ok = false; break; }
         tc_fence_after();
         const uint64_t dK = sdesc_add(dK0, ks * L::TILE);
         const uint64_t dV = sdesc_add(dV0, vs * L::TILE);
 #pragma unroll
-        for (int g = 0; g < HD / 64; ++g) {
+        for (int gq = 0; gq < HD / 64; ++gq) {
           uint32_t dd[8];
           uint64_t aa[8], bb[8];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const uint32_t off = g * 16384 + i * 32;
+            const uint32_t off = gq * 16384 + i * 32;
             dd[2 * i] = tS;
             dd[2 * i + 1] = tdP;
             aa[2 * i] = sdesc_add(dQ, off);
@@ -852,18 +954,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bb[2 * i] = sdesc_add(dK, off);
             bb[2 * i + 1] = sdesc_add(dV, off);
           }
-          umma8_ss(dd, aa, bb, idesc_s, g == 0 ? 0xfcu : 0xffu);
+          umma8_ss(dd, aa, bb, idesc_s, gq == 0 ? 0xfcu : 0xffu);
         }
         umma_commit(s_full);
         umma_commit(&v_empty[vs]);
+        if (j_s == n_s - 1) umma_commit(q_empty);  // the item's Q and dO are no longer read
         issued = true;
+        ++gj;
+        if (++j_s == n_s) {
+          ++r_s;
+          j_s = 0;
+          n_s = item_blocks(r_s);
+        }
       }
-      if (j >= 1) {
-        const int jj = j - 1;
-        const int bb = jj & 1;
-        if (!mbar_wait(&ds_full[bb], (jj >> 1) & 1, ctl, abort_flag, 66)) { ok = false; break; }
+      if (gd < gj - 1 || (n_s <= 0 && gd < gj)) {
+        // dQ += dS K of block gd, issued after the S / dP products of block gd + 1 (if any)
+        const int bb = gd & 1;
+        if (!mbar_wait(&ds_full[bb], (gd >> 1) & 1, ctl, abort_flag, 66)) { ok = false; break; }
+        // the item's first dQ product overwrites the previous item's dQ: read out by then
+        if (j_d == 0 && r_d > 0 && !mbar_wait(acc_empty, (r_d - 1) & 1, ctl, abort_flag, 68)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t dKm = sdesc_add(dKm0, (jj % KS) * L::TILE);
+        const uint64_t dKm = sdesc_add(dKm0, (gd % KS) * L::TILE);
         const uint32_t tA = tdS + 64 * bb;
         uint32_t dd[8], aa[8];
         uint64_t bd[8];
@@ -873,15 +984,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           aa[kk] = tA + 8 * kk;
           bd[kk] = sdesc_add(dKm, kk * 2048);
         }
-        umma8_ts(dd, aa, bd, idesc_d, jj == 0 ? 0xfeu : 0xffu);
+        umma8_ts(dd, aa, bd, idesc_d, j_d == 0 ? 0xfeu : 0xffu);
         umma_commit(&ds_empty[bb]);
-        umma_commit(&k_empty[jj % KS]);
+        umma_commit(&k_empty[gd % KS]);
         issued = true;
+        ++gd;
+        if (++j_d == n_d) {
+          umma_commit(acc_full);
+          ++r_d;
+          j_d = 0;
+          n_d = item_blocks(r_d);
+        }
       }
     }
-    if (ok) {
-      umma_commit(acc_full);
-    } else if (issued) {
+    if (!ok && issued) {
       volatile int never = 0;
       umma_commit(drain);
       mbar_wait(drain, 0, ctl, &never, 67);
@@ -891,58 +1007,68 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int ew = warp - 2;
     const int quad = warp & 3;  // TMEM lane quadrant: queries 32 quad .. 32 quad + 31
     const int cg = ew >> 2;     // key columns 32 cg .. 32 cg + 31 of each block
-    const int qi = q0 + quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const bool row_ok = qi < s.T;
-    const float lse2 = row_ok ? lse[(long long)bh * s.T + qi] * kLog2e : 0.f;
-    const float dl = row_ok ? delta[(long long)bh * s.T + qi] : 0.f;
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(s_full, j & 1, ctl, abort_flag, 68)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t rs[32], rd[32];
-      tmem_ld32_nowait(tS + lane_off + 32 * cg, rs);
-      tmem_ld32_nowait(tdP + lane_off + 32 * cg, rd);
-      tmem_wait_ld();
-      tmem_fence_regs<32>(rs);
-      tmem_fence_regs<32>(rd);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      const int bb = j & 1;
-      if (!mbar_wait(&ds_empty[bb], ((j >> 1) & 1) ^ 1u, ctl, abort_flag, 69)) { ok = false; break; }
-      const int kb = (j0 + j) * 128 + 32 * cg;
-      uint32_t dw[16];
-      if ((kb + 31 > q0) || (kb + 32 > s.T) || !row_ok || (s.win >= 0 && kb < q0 + 127 - s.win)) {
-        // diagonal block, ragged end, rows past T or the window's lower edge: mask
+    int gj = 0;
+    for (int r = 0; ok; ++r) {
+      const int w = zigzag_item(r, blockIdx.x, gridDim.x);
+      if (w >= n_items) break;
+      const int qt = n_qt - 1 - w / BH, bh = w % BH;
+      const int b = bh / s.H, h = bh % s.H;
+      const int q0 = qt * 128;
+      const int j0 = dq_first_block(s, qt);
+      const int n_kv = qt + 1 - j0;
+      const int qi = q0 + quad * 32 + lane;
+      const bool row_ok = qi < s.T;
+      const float lse2 = row_ok ? lse[(long long)bh * s.T + qi] * kLog2e : 0.f;
+      const float dl = row_ok ? delta[(long long)bh * s.T + qi] : 0.f;
+      for (int j = 0; j < n_kv; ++j, ++gj) {
+        if (!mbar_wait(s_full, gj & 1, ctl, abort_flag, 68)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t rs[32], rd[32];
+        tmem_ld32_nowait(tS + lane_off + 32 * cg, rs);
+        tmem_ld32_nowait(tdP + lane_off + 32 * cg, rd);
+        tmem_wait_ld();
+        tmem_fence_regs<32>(rs);
+        tmem_fence_regs<32>(rd);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        const int bb = gj & 1;
+        if (!mbar_wait(&ds_empty[bb], ((gj >> 1) & 1) ^ 1u, ctl, abort_flag, 69)) { ok = false; break; }
+        const int kb = (j0 + j) * 128 + 32 * cg;
+        uint32_t dw[16];
+        if ((kb + 31 > q0) || (kb + 32 > s.T) || !row_ok || (s.win >= 0 && kb < q0 + 127 - s.win)) {
+          // diagonal block, ragged end, rows past T or the window's lower edge: mask
 #pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          float d2[2];
+          for (int e2 = 0; e2 < 16; ++e2) {
+            float d2[2];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int e = 2 * e2 + k;
-            const int key = kb + e;
-            float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -lse2));
-            if (!row_ok || key > qi || key >= s.T || (s.win >= 0 && key < qi - s.win)) pv = 0.f;
-            d2[k] = pv * (__uint_as_float(rd[e]) - dl);
+            for (int k = 0; k < 2; ++k) {
+              const int e = 2 * e2 + k;
+              const int key = kb + e;
+              float pv = ex2_approx(fmaf(__uint_as_float(rs[e]), scale_log2, -lse2));
+              if (!row_ok || key > qi || key >= s.T || (s.win >= 0 && key < qi - s.win)) pv = 0.f;
+              d2[k] = pv * (__uint_as_float(rd[e]) - dl);
+            }
+            dw[e2] = pack_bf16x2(d2[0], d2[1]);
           }
-          dw[e2] = pack_bf16x2(d2[0], d2[1]);
-        }
-      } else {
+        } else {
 #pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(rs[2 * e2]), scale_log2, -lse2));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(rs[2 * e2 + 1]), scale_log2, -lse2));
-          dw[e2] = pack_bf16x2(p0 * (__uint_as_float(rd[2 * e2]) - dl), p1 * (__uint_as_float(rd[2 * e2 + 1]) - dl));
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(rs[2 * e2]), scale_log2, -lse2));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(rs[2 * e2 + 1]), scale_log2, -lse2));
+            dw[e2] = pack_bf16x2(p0 * (__uint_as_float(rd[2 * e2]) - dl), p1 * (__uint_as_float(rd[2 * e2 + 1]) - dl));
+          }
         }
+        tmem_st16(tdS + 64 * bb + lane_off + 16 * cg, dw);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_full[bb]);
       }
-      tmem_st16(tdS + 64 * bb + lane_off + 16 * cg, dw);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ds_full[bb]);
-    }
-    if (ok && mbar_wait(acc_full, 0, ctl, abort_flag, 70)) {
+      if (!ok) break;
+      if (!mbar_wait(acc_full, r & 1, ctl, abort_flag, 70)) { ok = false; break; }
       tc_fence_after();
       // the four warps of a quadrant split dQ's columns
       constexpr int CPW = HD / 4;
@@ -973,6 +1099,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 pack_bf16x2(__uint_as_float(a[8 * g + 6]) * scale, __uint_as_float(a[8 * g + 7]) * scale));
         }
       }
+      // dQ has been read: the next item's products may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
     }
   }
 
@@ -1048,7 +1178,9 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     using L = DkvSmem<HD>;
     static_assert(L::BYTES <= 232448, "dK/dV shared memory above the per-block limit");
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dkv_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
-    dim3 grid((s.T + 127) / 128, s.B * s.H);
+    // persistent: one CTA per SM over the (key tile, head) items
+    const long long items = (long long)((s.T + 127) / 128) * s.B * s.H;
+    dim3 grid((unsigned)std::min<long long>(items, num_sms()));
     Prof prof(PK_ATTN_BWD_DKV, 8.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 6, st);
     attn_bwd_dkv_kernel<HD><<<grid, kBwdThreads, L::BYTES, st>>>(qkv128, qkv128, do128, s, lse, delta, dqkv, scale_log2,
                                                                  scale, ctl);
@@ -1058,7 +1190,8 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     using L = DqSmem<HD>;
     static_assert(L::BYTES <= 232448, "dQ shared memory above the per-block limit");
     GPTK_CUDA(cudaFuncSetAttribute(attn_bwd_dq_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
-    dim3 grid((s.T + 127) / 128, s.B * s.H);
+    const long long items = (long long)((s.T + 127) / 128) * s.B * s.H;
+    dim3 grid((unsigned)std::min<long long>(items, num_sms()));
     Prof prof(PK_ATTN_BWD_DQ, 6.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 5, st);
     attn_bwd_dq_kernel<HD><<<grid, kBwdThreads, L::BYTES, st>>>(qkv128, do128, qkv128, s, lse, delta, dqkv, scale_log2,
                                                                 scale, ctl);
