@@ -92,7 +92,18 @@ __global__ void col_scan_kernel(int* __restrict__ cnt, int G, int V, int* __rest
   const int v = blockIdx.x * blockDim.x + threadIdx.x;
   if (v >= V) return;
   int run = 0;
-  for (int g = 0; g < G; ++g) {
+  int g = 0;
+  for (; g + 8 <= G; g += 8) {  // eight independent loads in flight, then the running sum
+    int c[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) c[u] = cnt[(long long)(g + u) * V + v];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      cnt[(long long)(g + u) * V + v] = run;
+      run += c[u];
+    }
+  }
+  for (; g < G; ++g) {
     const long long i = (long long)g * V + v;
     const int c = cnt[i];
     cnt[i] = run;
@@ -101,8 +112,8 @@ __global__ void col_scan_kernel(int* __restrict__ cnt, int G, int V, int* __rest
   total[v] = run;
 }
 
-// single block, 1024 threads: exclusive scan of total[0..V)
-__global__ void offsets_kernel(const int* __restrict__ total, int V, int* __restrict__ offs) {
+// single block, 1024 threads: exclusive scan of total[0..V), straight from global memory (any V)
+__global__ void offsets_global_kernel(const int* __restrict__ total, int V, int* __restrict__ offs) {
   __shared__ int part[1024];
   const int t = threadIdx.x;
   const int per = (V + 1023) / 1024;
@@ -111,7 +122,6 @@ __global__ void offsets_kernel(const int* __restrict__ total, int V, int* __rest
   for (int v = v0; v < v1; ++v) s += total[v];
   part[t] = s;
   __syncthreads();
-  // Hillis-Steele inclusive scan over the 1024 partial sums
   for (int o = 1; o < 1024; o <<= 1) {
     int x = t >= o ? part[t - o] : 0;
     __syncthreads();
@@ -123,6 +133,39 @@ __global__ void offsets_kernel(const int* __restrict__ total, int V, int* __rest
     offs[v] = run;
     run += total[v];
   }
+}
+
+// The same with total staged in shared memory by coalesced loads first (V up to kOffsSmemV), so that
+// each thread's stretch is read from shared memory.
+constexpr int kOffsSmemV = 53248;  // 208 KB
+
+__global__ void offsets_kernel(const int* __restrict__ total, int V, int* __restrict__ offs) {
+  __shared__ int part[1024];
+  extern __shared__ int tot_s[];
+  const int t = threadIdx.x;
+  for (int v = t; v < V; v += 1024) tot_s[v] = total[v];
+  __syncthreads();
+  const int per = (V + 1023) / 1024;
+  const int v0 = t * per, v1 = min(V, v0 + per);
+  int s = 0;
+  for (int v = v0; v < v1; ++v) s += tot_s[v];
+  part[t] = s;
+  __syncthreads();
+  // Hillis-Steele inclusive scan over the 1024 partial sums
+  for (int o = 1; o < 1024; o <<= 1) {
+    int x = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += x;
+    __syncthreads();
+  }
+  int run = t > 0 ? part[t - 1] : 0;
+  for (int v = v0; v < v1; ++v) {
+    const int c = tot_s[v];
+    tot_s[v] = run;
+    run += c;
+  }
+  __syncthreads();
+  for (int v = t; v < V; v += 1024) offs[v] = tot_s[v];
 }
 
 __global__ void scatter_kernel(const int* __restrict__ idx, int M, int V, const int* __restrict__ cnt,
@@ -137,7 +180,11 @@ __global__ void scatter_kernel(const int* __restrict__ idx, int M, int V, const 
 
 __device__ __forceinline__ int clamp_id(int id, int V) { return (id < 0 || id >= V) ? 0 : id; }
 
-// One block per chunk of 256 sorted positions; threads stride over float4 columns.
+// One block per (chunk of 256 sorted positions, 128 float4 columns): each thread owns one float4
+// column and walks the chunk's segments; the rows of a segment are loaded eight at a time (the
+// loads are independent) and added in ascending token order.
+constexpr int kSegCols = 128;
+
 __global__ void segsum_chunk_kernel(const int* __restrict__ idx, const float* __restrict__ dx, int M, int D, int V,
                                     const int* __restrict__ total, const int* __restrict__ offs,
                                     const int* __restrict__ sorted, float* __restrict__ dwte,
@@ -145,29 +192,40 @@ __global__ void segsum_chunk_kernel(const int* __restrict__ idx, const float* __
   const int c = blockIdx.x;
   const int p0 = c * kChunk, p1 = min(M, p0 + kChunk);
   const int D4 = D / 4;
-  for (int col = threadIdx.x; col < D4; col += blockDim.x) {
-    int pos = p0;
-    while (pos < p1) {
-      const int id = clamp_id(idx[sorted[pos]], V);
-      const int bstart = offs[id], bend = bstart + total[id];
-      const int send = min(bend, p1);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int q = pos; q < send; ++q) {
-        const float4 x = reinterpret_cast<const float4*>(dx + (long long)sorted[q] * D)[col];
-        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+  const int col = blockIdx.y * kSegCols + threadIdx.x;
+  if (col >= D4) return;
+  const float4* dx4 = reinterpret_cast<const float4*>(dx) + col;
+  int pos = p0;
+  while (pos < p1) {
+    const int id = clamp_id(idx[sorted[pos]], V);
+    const int bstart = offs[id], bend = bstart + total[id];
+    const int send = min(bend, p1);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int q = pos;
+    for (; q + 8 <= send; q += 8) {
+      float4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(dx4 + (long long)sorted[q + u] * D4);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc.x += x[u].x; acc.y += x[u].y; acc.z += x[u].z; acc.w += x[u].w;
       }
-      if (bstart < p0) {
-        reinterpret_cast<float4*>(head + (long long)c * D)[col] = acc;
-      } else if (bend > p1) {
-        reinterpret_cast<float4*>(tail + (long long)c * D)[col] = acc;
-      } else {
-        float4* w = reinterpret_cast<float4*>(dwte + (long long)id * D) + col;
-        float4 cur = *w;
-        cur.x += acc.x; cur.y += acc.y; cur.z += acc.z; cur.w += acc.w;
-        *w = cur;
-      }
-      pos = send;
     }
+    for (; q < send; ++q) {
+      const float4 x = __ldg(dx4 + (long long)sorted[q] * D4);
+      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    }
+    if (bstart < p0) {
+      reinterpret_cast<float4*>(head + (long long)c * D)[col] = acc;
+    } else if (bend > p1) {
+      reinterpret_cast<float4*>(tail + (long long)c * D)[col] = acc;
+    } else {
+      float4* w = reinterpret_cast<float4*>(dwte + (long long)id * D) + col;
+      float4 cur = *w;
+      cur.x += acc.x; cur.y += acc.y; cur.z += acc.z; cur.w += acc.w;
+      *w = cur;
+    }
+    pos = send;
   }
 }
 
@@ -213,7 +271,12 @@ int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float
   }
   {
     Prof prof(PK_EMBED_BWD, 0, V * 8.0, st);
-    offsets_kernel<<<1, 1024, 0, st>>>(s.total, V, s.offs);
+    if (V <= kOffsSmemV) {
+      GPTK_CUDA(cudaFuncSetAttribute(offsets_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kOffsSmemV * 4));
+      offsets_kernel<<<1, 1024, (size_t)V * sizeof(int), st>>>(s.total, V, s.offs);
+    } else {
+      offsets_global_kernel<<<1, 1024, 0, st>>>(s.total, V, s.offs);
+    }
     GPTK_CUDA(cudaGetLastError());
   }
   {
@@ -224,7 +287,10 @@ int launch_embed_bwd(const int* idx, const float* dx, int M, int D, int V, float
   const int threads = D / 4 < 256 ? ((D / 4 + 31) / 32) * 32 : 256;
   {
     Prof prof(PK_EMBED_BWD, 0, (double)M * D * 4 + M * 8.0, st);
-    segsum_chunk_kernel<<<G, threads, 0, st>>>(idx, dx, M, D, V, s.total, s.offs, s.sorted, dwte, s.head, s.tail);
+    const dim3 grid(G, (D / 4 + kSegCols - 1) / kSegCols);
+    const int seg_threads = D / 4 < kSegCols ? ((D / 4 + 31) / 32) * 32 : kSegCols;
+    segsum_chunk_kernel<<<grid, seg_threads, 0, st>>>(idx, dx, M, D, V, s.total, s.offs, s.sorted, dwte, s.head,
+                                                      s.tail);
     GPTK_CUDA(cudaGetLastError());
   }
   {
