@@ -310,12 +310,23 @@ __global__ void rms_bwd_kernel(const void* __restrict__ dy_, const __nv_bfloat16
   for (int m = blockIdx.x * warps + w; m < M; m += gridDim.x * warps) {
     const long long base = (long long)m * D;
     const float r = rstd[m];
-    float yv[NV8][8], gv[NV8][8];
+    float yv[NV8][8], gv[NV8][8], dv[NV8][8];
     float s2 = 0.f;
 #pragma unroll
     for (int i = 0; i < NV8; ++i) {
       const int c = i * 32 + lane;
       if (c < D8) {
+        // the residual gradient is loaded with the row's other inputs, ahead of the reduction
+        // (rows up to 1536 wide; wider rows load it afterwards, to stay within the registers)
+        if (!dres_init && NV8 <= 6) {
+          const float4* dr = reinterpret_cast<const float4*>(dres + base) + 2 * c;
+          const float4 a = dr[0], b = dr[1];
+          dv[i][0] = a.x; dv[i][1] = a.y; dv[i][2] = a.z; dv[i][3] = a.w;
+          dv[i][4] = b.x; dv[i][5] = b.y; dv[i][6] = b.z; dv[i][7] = b.w;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) dv[i][k] = 0.f;
+        }
         bf16x8(reinterpret_cast<const uint4*>(y + base)[c], yv[i]);
         if (DYB) {
           bf16x8(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(dy_) + base)[c], gv[i]);
@@ -336,9 +347,9 @@ __global__ void rms_bwd_kernel(const void* __restrict__ dy_, const __nv_bfloat16
       if (c < D8) {
         float o[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) o[k] = r * (gv[i][k] - yv[i][k] * m2);
+        for (int k = 0; k < 8; ++k) o[k] = r * (gv[i][k] - yv[i][k] * m2) + dv[i][k];
         float4* dr = reinterpret_cast<float4*>(dres + base) + 2 * c;
-        if (!dres_init) {
+        if (!dres_init && NV8 > 6) {
           const float4 a = dr[0], b = dr[1];
           o[0] += a.x; o[1] += a.y; o[2] += a.z; o[3] += a.w; o[4] += b.x; o[5] += b.y; o[6] += b.z; o[7] += b.w;
         }
@@ -357,11 +368,11 @@ int launch_rms_bwd(const void* dy, int dy_bf16, const __nv_bfloat16* y, const fl
   const int nv8 = (D + 255) / 256;
   auto run = [&](auto nvc) -> int {
     constexpr int NV8 = decltype(nvc)::value;
-    int grid = cdiv(M, 8);
-    if (grid > num_sms() * 16) grid = num_sms() * 16;
+    int grid = cdiv(M, 4);
+    if (grid > num_sms() * 32) grid = num_sms() * 32;
     Prof prof(PK_NORM_BWD, 0, (double)M * D * ((dy_bf16 ? 2 : 4) + 2 + 4 + 2 + (dres_init ? 0 : 4)) + M * 4.0, st);
-    if (dy_bf16) rms_bwd_kernel<NV8, true><<<grid, 256, 0, st>>>(dy, y, rstd, M, D, dres, dres_init, dres_bf);
-    else rms_bwd_kernel<NV8, false><<<grid, 256, 0, st>>>(dy, y, rstd, M, D, dres, dres_init, dres_bf);
+    if (dy_bf16) rms_bwd_kernel<NV8, true><<<grid, 128, 0, st>>>(dy, y, rstd, M, D, dres, dres_init, dres_bf);
+    else rms_bwd_kernel<NV8, false><<<grid, 128, 0, st>>>(dy, y, rstd, M, D, dres, dres_init, dres_bf);
     GPTK_CUDA(cudaGetLastError());
     return (int)ST_OK;
   };

@@ -25,7 +25,8 @@ BLOCK_THREADS = [
     (r"gemm_kernel", 320),               # TMA warp, MMA warp, 8 epilogue warps (long-K: 4)
     (r"attn_fwd_kernel", 384),           # TMA, MMA and two idle warps; two softmax warpgroups
     (r"attn_bwd_(dkv|dq)_kernel", 576),  # TMA warp, MMA warp, 16 elementwise warps
-    (r"offsets_kernel", 1024),
+    (r"offsets_(global_)?kernel", 1024),
+    (r"rms_bwd_kernel", 128),
     (r".*", 256),                        # every other kernel: blocks of at most 256 threads
 ]
 
