@@ -893,12 +893,13 @@ int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, c
 
 // ------------------------------------------------------------------ attention delta
 
-// delta[b, h, t] = sum_d o[m, h hd + d] * dO[m, h hdp + d]: hd / 8 lanes per (token, head) item,
-// 16-byte loads, a segmented shuffle reduction; 32 / (hd / 8) items per warp and pass.
+// delta[b, h, t] = sum_d o[m, h hd + d] * dO[m, h hdp + d]: hd / 32 lanes per (token, head) item,
+// each lane 32 elements of o and of dO in four 16-byte loads each (all eight issued first), a
+// segmented shuffle reduction; 32 / (hd / 32) items per warp and pass.
 template <int HD>
 __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dpad, int B,
                                   int T, int H, int hdp, float* __restrict__ delta) {
-  constexpr int LPI = HD / 8;  // lanes per item
+  constexpr int LPI = HD / 32;  // lanes per item
   constexpr int IPW = 32 / LPI;
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -911,13 +912,22 @@ __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __n
     if (w < total) {
       const long long m = w / H;
       const int h = (int)(w - m * H);
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + m * H * HD + (long long)h * HD) + l8);
-      const uint4 d = __ldg(reinterpret_cast<const uint4*>(dpad + m * H * hdp + (long long)h * hdp) + l8);
-      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, dv[4] = {d.x, d.y, d.z, d.w};
+      const uint4* ap = reinterpret_cast<const uint4*>(o + m * H * HD + (long long)h * HD) + 4 * l8;
+      const uint4* dp = reinterpret_cast<const uint4*>(dpad + m * H * hdp + (long long)h * hdp) + 4 * l8;
+      uint4 a[4], d[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        s = fmaf(__uint_as_float(av[k] << 16), __uint_as_float(dv[k] << 16), s);
-        s = fmaf(__uint_as_float(av[k] & 0xffff0000u), __uint_as_float(dv[k] & 0xffff0000u), s);
+      for (int u = 0; u < 4; ++u) {
+        a[u] = __ldg(ap + u);
+        d[u] = __ldg(dp + u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t av[4] = {a[u].x, a[u].y, a[u].z, a[u].w}, dv[4] = {d[u].x, d[u].y, d[u].z, d[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          s = fmaf(__uint_as_float(av[k] << 16), __uint_as_float(dv[k] << 16), s);
+          s = fmaf(__uint_as_float(av[k] & 0xffff0000u), __uint_as_float(dv[k] & 0xffff0000u), s);
+        }
       }
     }
 #pragma unroll
@@ -964,7 +974,7 @@ int launch_attn_delta(const __nv_bfloat16* o, const __nv_bfloat16* do_pad, int B
     return ST_OK;
   }
   const long long items = (long long)B * T * H;
-  const int ipb = 8 * (hd == 128 ? 2 : 4);  // items per 256-thread block and pass
+  const int ipb = 8 * (hd == 128 ? 8 : 16);  // items per 256-thread block and pass
   long long grid = (items + ipb - 1) / ipb;
   if (grid > (long long)num_sms() * 16) grid = num_sms() * 16;
   Prof prof(PK_DELTA, 0, (double)B * T * H * (hd * 2 + hdp * 2 + 4), st);
