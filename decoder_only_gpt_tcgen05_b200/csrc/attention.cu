@@ -304,10 +304,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         alpha = ex2_approx(m - m_new);
         m = m_new;
       }
+      // O is free here: the MMA thread issued this block's S product only after the tile's
+      // previous P V product had completed, and s_full (a commit of every product issued before)
+      // has been observed
       if (i > 0) {
-        // O is still in use by the previous P V product of this tile
-        if (!mbar_wait(&o_done[t], (i - 1) & 1, ctl, abort_flag, 30)) { ok = false; break; }
-        tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
           for (int c = 0; c < HD / 32; ++c) {
