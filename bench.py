@@ -7,9 +7,12 @@
 
 A step is one gpt_forward_loss + gpt_backward over one batch of B=16
 sequences of T=2048 tokens per GPU (synthetic Zipf(1.1) tokens, random-init
-d20 weights).  With N > 1 every rank processes its own batch (weak scaling)
-and the gradients are summed over ranks with an NCCL all-reduce inside the
-step, as data-parallel training does.  Rank 0 prints one JSON line.
+d20 weights), plus an optimizer step with --optimizer.  With N > 1 every rank
+processes its own batch (weak scaling) and the gradients are averaged over
+ranks inside the step, bucket by bucket on a communication stream while the
+backward goes on (--grad-sync overlap, the default; --grad-sync blocking: one
+all-reduce after the backward; --optimizer zero2: reduce-scatter, sharded
+AdamW, all-gather of the weights).  Rank 0 prints one JSON line.
 
 --impl reference times the oracle (plain fp64 CPU model) on a bounded sample
 of the same workload on the host cores: the deliberately slow baseline.
