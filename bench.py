@@ -317,14 +317,74 @@ def run_attn_sweep(args):
     print(json.dumps(line), flush=True)
 
 
+def run_lmhead(args):
+    """The fused lm_head + cross-entropy forward alone at the d26 shape: 32768 tokens x width
+    1664 x vocabulary 32768 (gpt_op_lmhead_ce_fwd: per-row loss and logsumexp, logits never
+    stored).  Inputs: x N(0, 1) (seed 5) and W N(0, 0.02^2) (seed 6) in bf16, Zipf(1.1) targets
+    (seed 1).  Timed with CUDA events over `steps` back-to-back calls; x and W (232 MB) are above
+    the 126 MB L2."""
+    import torch
+    import decoder_only_gpt_tcgen05_b200 as g
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])   # one kernel timed alone: burst peak
+    M, D, V = 32768, 1664, 32768
+    x = torch.from_numpy(synth.normal((M, D), 5)).to(dev).to(torch.bfloat16)
+    w = torch.from_numpy(synth.normal((V, D), 6, std=0.02)).to(dev).to(torch.bfloat16)
+    _, tgt = synth.next_token_batch(16, 2048, V, seed=1)
+    tgt = torch.from_numpy(tgt.reshape(-1)).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        g.ops.lmhead_ce_fwd(x, w, tgt)
+    torch.cuda.synchronize(dev)
+    n0 = g.ops.launch_count()
+    with ClockSampler(0) as clk:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            g.ops.lmhead_ce_fwd(x, w, tgt)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / args.steps
+    g.model.sync_status(dev)
+    launches = (g.ops.launch_count() - n0) / args.steps
+    g.ops.profile_start()
+    for _ in range(args.steps):
+        g.ops.lmhead_ce_fwd(x, w, tgt)
+    torch.cuda.synchronize(dev)
+    prof = g.ops.profile_stop()
+    flops = 2.0 * M * D * V
+    gemm_ms = prof["gemm"][0] / args.steps
+    ach = flops / gemm_ms / 1e9 if gemm_ms > 0 else None
+    line = {
+        "metric": "d26 fused lm_head + cross-entropy forward TFLOP/s, 32768 tokens x 32768 vocab",
+        "value": flops / ms / 1e9, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "lm_head + CE forward: M=32768, D=1664, V=32768 (d26 shape)",
+                   "l2": "x 109 MB + W 109 MB, above the 126 MB L2; no flush"},
+        "roofline": {"kernel": "gemm (cross-entropy epilogue)", "bound": "tensor", "achieved": ach, "peak": peak,
+                     "unit": "TFLOP/s", "frac": ach / peak if ach else None, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "logits_bytes_not_written": 2 * M * V,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS) + ["attn_sweep"], default="d20",
-                    help="attn_sweep: the attention kernels alone over T = 512..8192 at 32768 tokens")
+    ap.add_argument("--workload", choices=list(WORKLOADS) + ["attn_sweep", "lmhead_d26"], default="d20",
+                    help="attn_sweep: the attention kernels alone over T = 512..8192 at 32768 tokens; "
+                         "lmhead_d26: the fused lm_head + cross-entropy forward alone at the d26 shape")
     ap.add_argument("--profile-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="also print the per-kernel-family table to stderr")
@@ -353,6 +413,11 @@ def main():
         if args.impl != "ours" or world != 1:
             ap.error("attn_sweep times this library's attention kernels on one GPU")
         run_attn_sweep(args)
+        return
+    if args.workload == "lmhead_d26":
+        if args.impl != "ours" or world != 1:
+            ap.error("lmhead_d26 times this library's fused lm_head + cross-entropy on one GPU")
+        run_lmhead(args)
         return
     if args.impl == "reference":
         run_reference(args, rank, world)
