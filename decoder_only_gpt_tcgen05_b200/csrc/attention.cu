@@ -14,17 +14,20 @@
 //   warp 1      one thread alternates between the two tiles: O += P_j V_j (P from tensor memory,
 //               V from shared memory), then S_{j+1} = Q K_{j+1}^T into that tile's TMEM scores,
 //               so the tensor core works on one tile while the other tile's softmax runs
-//   warps 2..9  two softmax warpgroups, one per query tile, one query row per thread: row max
-//               and sum in registers, P = exp2(...) as bf16 into the upper half of the tile's
-//               score columns (already read), where it is the A operand of the PV product; O is
-//               rescaled in TMEM only when the running max grows by more than 2^8 (otherwise the
-//               stale max stays exact because O and l use the same one)
-// Backward: delta = rowsum(dO * O) (kernels.cu), then
-//   dK/dV kernel: one CTA per 128-key tile, stepping over 128-query blocks from the diagonal:
+//   warps 2, 3  idle (they give their registers to the softmax warpgroups with setmaxnreg)
+//   warps 4..11 two softmax warpgroups, one per query tile, one query row per thread holding its
+//               128 scores: row max and sum in registers, P = exp2(...) (3/8 of them on the FMA
+//               pipe) as bf16 over the first 64 score columns (already read), where it is the A
+//               operand of the PV product; O is rescaled in TMEM only when the running max grows
+//               by more than 2^8 (otherwise the stale max stays exact because O and l use the
+//               same one)
+// Backward: delta = rowsum(dO * O) (kernels.cu), then two persistent kernels (one CTA per SM,
+// walking (tile, head) items heaviest first):
+//   dK/dV kernel: per 128-key tile, stepping over 128-query blocks from the diagonal:
 //               S^T = K Q^T and dP^T = V dO^T into TMEM; elementwise warps write P^T and dS^T
 //               back over them as bf16, the tensor-memory A operands of dV += P^T dO and
 //               dK += dS^T Q (accumulating in TMEM)
-//   dQ kernel:  one CTA per 128-query tile, stepping over 128-key blocks up to the diagonal:
+//   dQ kernel:  per 128-query tile, stepping over 128-key blocks up to the diagonal:
 //               S = Q K^T and dP = dO V^T into TMEM; dS as bf16 into a TMEM buffer, the A
 //               operand of dQ += dS K
 // Both are deterministic (no atomics).  Every wait is bounded (see ptx.cuh).
