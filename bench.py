@@ -376,15 +376,83 @@ def run_lmhead(args):
     print(json.dumps(line), flush=True)
 
 
+def run_gemm_shapes(args):
+    """The GEMM kernel alone, bf16 (kind::f16) against 8-bit e4m3 (kind::f8f6f4), on the d20
+    projection shapes at 32768 tokens (QKV, out-projection, MLP up, MLP down) and a square 8192^3.
+    Inputs N(0, 1) (seeds 7, 8), outputs bf16; each product timed with CUDA events over `steps`
+    back-to-back calls.  TFLOP/s on 2 M N K; the 8-bit figures against the bf16 burst peak times
+    the nominal fp8 / bf16 ratio of 2."""
+    import torch
+    import decoder_only_gpt_tcgen05_b200 as g
+    import synth
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    stream = torch.cuda.current_stream(dev)
+    shapes = [("qkv", 32768, 3840, 1280), ("out_proj", 32768, 1280, 1280), ("mlp_up", 32768, 5120, 1280),
+              ("mlp_down", 32768, 1280, 5120), ("square", 8192, 8192, 8192)]
+
+    def timed(fn, k):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / k
+
+    rows = []
+    n0 = g.ops.launch_count()
+    n_calls = 0
+    with ClockSampler(0) as clk:
+        for name, M, N, K in shapes:
+            A = torch.from_numpy(synth.normal((M, K), 7)).to(dev).to(torch.bfloat16)
+            Bw = torch.from_numpy(synth.normal((N, K), 8, std=0.05)).to(dev).to(torch.bfloat16)
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            qa, _, ia = g.ops.fp8_quantize(A, g.ops.FP8_E4M3)
+            qb, _, ib = g.ops.fp8_quantize(Bw, g.ops.FP8_E4M3)
+            ms16 = timed(lambda: g.ops.gemm(A, Bw, out), args.steps)
+            ms8 = timed(lambda: g.ops.gemm_fp8(qa, 0, ia, qb, 0, ib, out), args.steps)
+            n_calls += 2 * (args.warmup + args.steps)
+            fl = 2.0 * M * N * K
+            rows.append({"name": name, "M": M, "N": N, "K": K, "bf16_ms": ms16, "fp8_ms": ms8,
+                         "bf16_tflops": fl / ms16 / 1e9, "fp8_tflops": fl / ms8 / 1e9,
+                         "bf16_frac": fl / ms16 / 1e9 / peak, "fp8_frac": fl / ms8 / 1e9 / (2 * peak)})
+            del A, Bw, out, qa, qb
+        g.model.sync_status(dev)
+    head = next(r for r in rows if r["name"] == "mlp_up")
+    line = {
+        "metric": "GEMM TFLOP/s, bf16 and e4m3 operands, d20 projection shapes at 32768 tokens (MLP up headline)",
+        "value": head["bf16_tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["bf16_ms"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "gemm shapes: " + ", ".join(f"{r['name']} {r['M']}x{r['N']}x{r['K']}" for r in rows),
+                   "l2": "operands and outputs of the d20 shapes above the 126 MB L2; no flush"},
+        "roofline": {"kernel": "gemm (bf16, MLP up)", "bound": "tensor", "achieved": head["bf16_tflops"],
+                     "peak": peak, "unit": "TFLOP/s", "frac": head["bf16_frac"], "traffic": None,
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "shapes": rows,
+        "gpu_launches": (g.ops.launch_count() - n0) / max(1, n_calls),
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS) + ["attn_sweep", "lmhead_d26"], default="d20",
+    ap.add_argument("--workload", choices=list(WORKLOADS) + ["attn_sweep", "lmhead_d26", "gemm"], default="d20",
                     help="attn_sweep: the attention kernels alone over T = 512..8192 at 32768 tokens; "
-                         "lmhead_d26: the fused lm_head + cross-entropy forward alone at the d26 shape")
+                         "lmhead_d26: the fused lm_head + cross-entropy forward alone at the d26 shape; "
+                         "gemm: the GEMM kernel alone, bf16 and e4m3, on the d20 projection shapes")
     ap.add_argument("--profile-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="also print the per-kernel-family table to stderr")
@@ -413,6 +481,11 @@ def main():
         if args.impl != "ours" or world != 1:
             ap.error("attn_sweep times this library's attention kernels on one GPU")
         run_attn_sweep(args)
+        return
+    if args.workload == "gemm":
+        if args.impl != "ours" or world != 1:
+            ap.error("gemm times this library's GEMM kernel on one GPU")
+        run_gemm_shapes(args)
         return
     if args.workload == "lmhead_d26":
         if args.impl != "ours" or world != 1:
