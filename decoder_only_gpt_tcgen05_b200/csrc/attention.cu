@@ -77,7 +77,8 @@ constexpr uint32_t kPolyGroups = 0x52u;
 template <int HD>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnShape s, __nv_bfloat16* __restrict__ o,
-                    long long ldo, float* __restrict__ lse_out, float scale_log2, DevCtl ctl) {
+                    long long ldo, float* __restrict__ lse_out, float scale_log2, unsigned int* __restrict__ amax_bits,
+                    DevCtl ctl) {
   using L = FwdSmem<HD>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -355,12 +356,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float inv_l = 1.f / l;
       const bool row_ok = qi < s.T;
       __nv_bfloat16* orow = o + ((long long)b * s.T + qi) * ldo + (long long)h * s.hd;
+      float am = 0.f;  // max |o| of the row (for an 8-bit cast of o)
 #pragma unroll 1
       for (int c = 0; c < HD / 32; ++c) {
         float ov[32];
         tmem_ld32(tO + c * 32, ov);
 #pragma unroll
         for (int e = 0; e < 32; ++e) ov[e] *= inv_l;
+        if (amax_bits && row_ok) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e < s.hd) am = fmaxf(am, fabsf(ov[e]));
+        }
         if (row_ok) {
           if (s.hd == HD) {
             uint4* d = reinterpret_cast<uint4*>(orow + c * 32);
@@ -375,6 +382,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       if (row_ok) lse_out[(long long)bh * s.T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+      if (amax_bits) {
+        // one atomic per warp; o is stored in bf16 and the rounding is monotonic
+#pragma unroll
+        for (int sh = 16; sh > 0; sh >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, sh));
+        if (lane == 0) atomicMax(amax_bits, __float_as_uint(__bfloat162float(__float2bfloat16_rn(am))));
+      }
     }
   }
 
@@ -1127,7 +1140,7 @@ double attn_pairs(int T, int win) {
 
 template <int HD>
 static int attn_fwd_launch(const CUtensorMap& tm, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
-                           float scale_log2, cudaStream_t st) {
+                           float scale_log2, float* amax, cudaStream_t st) {
   using L = FwdSmem<HD>;
   GPTK_CUDA(cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES));
   // setmaxnreg.inc waits until the registers it asks for are free in the block's own allocation:
@@ -1142,26 +1155,27 @@ static int attn_fwd_launch(const CUtensorMap& tm, const AttnShape& s, __nv_bfloa
   dim3 grid(s.B * s.H, (s.T + 255) / 256);
   const double causal = (double)s.B * s.H * attn_pairs(s.T, s.win);
   Prof prof(PK_ATTN_FWD, 4.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 4, st);
-  attn_fwd_kernel<HD><<<grid, kFwdThreads, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2, device_ctl());
+  attn_fwd_kernel<HD><<<grid, kFwdThreads, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2,
+                                                            reinterpret_cast<unsigned int*>(amax), device_ctl());
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
 
 template <int HD>
 static int attn_fwd_t(const __nv_bfloat16* qkv, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
-                      cudaStream_t st) {
+                      float* amax, cudaStream_t st) {
   CUtensorMap tm;
   GPTK_TRY(make_tmap_3d(&tm, qkv, 3ull * s.H * s.hdp, s.T, s.B, s.ld_qkv, (uint64_t)s.T * s.ld_qkv, 64, 128, 1));
-  return attn_fwd_launch<HD>(tm, s, o, ldo, lse, kLog2e / sqrtf((float)s.hd), st);
+  return attn_fwd_launch<HD>(tm, s, o, ldo, lse, kLog2e / sqrtf((float)s.hd), amax, st);
 }
 
 int launch_attn_fwd(const __nv_bfloat16* qkv_pad, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
-                    cudaStream_t st) {
+                    cudaStream_t st, float* amax) {
   if (s.B < 1 || s.T < 1 || s.H < 1) return set_error(ST_INVALID_ARG, "attention: empty shape");
   if (s.win < -1) return set_error(ST_INVALID_ARG, "attention: window must be >= 0 (or -1 for none)");
   if (s.B * s.H > 65535) return set_error(ST_UNSUPPORTED, "attention: B*H above 65535");
-  if (s.hdp == 64) return attn_fwd_t<64>(qkv_pad, s, o, ldo, lse, st);
-  if (s.hdp == 128) return attn_fwd_t<128>(qkv_pad, s, o, ldo, lse, st);
+  if (s.hdp == 64) return attn_fwd_t<64>(qkv_pad, s, o, ldo, lse, amax, st);
+  if (s.hdp == 128) return attn_fwd_t<128>(qkv_pad, s, o, ldo, lse, amax, st);
   return set_error(ST_UNSUPPORTED, "attention: padded head dim must be 64 or 128");
 }
 

@@ -4,7 +4,9 @@
 //
 // Two HBM-bound launches per tensor: the absolute maximum (a float atomicMax on the bit pattern of
 // |x|, exact and order-independent), then the cast of x * s with round-to-nearest-even and
-// saturation (cvt.rn.satfinite), which also writes 1 / s for the product's epilogue.
+// saturation (cvt.rn.satfinite), which also writes 1 / s for the product's epilogue.  Where the
+// producer of x already folded max |x| into the same kind of slot (the model's FP8 forward: the
+// norms, the attention output, the MLP-up epilogue), the cast runs alone (launch_fp8_cast).
 #include <string>
 
 #include "gemm.cuh"
@@ -86,22 +88,15 @@ __global__ void quantize_kernel(const T* __restrict__ x, long long n, const floa
 
 }  // namespace
 
-int launch_fp8_quantize(const void* x, int x_fp32, long long n, int fmt, void* out, float* amax, float* inv_scale,
-                        cudaStream_t st) {
-  if (n < 1) return set_error(ST_INVALID_ARG, "fp8_quantize: n must be >= 1");
-  if (fmt != 0 && fmt != 1) return set_error(ST_INVALID_ARG, "fp8_quantize: format must be 0 (e4m3) or 1 (e5m2)");
-  if (!x || !out || !amax || !inv_scale) return set_error(ST_INVALID_ARG, "fp8_quantize: null pointer");
-  GPTK_CUDA(cudaMemsetAsync(amax, 0, sizeof(float), st));
+int launch_fp8_cast(const void* x, int x_fp32, long long n, int fmt, void* out, const float* amax, float* inv_scale,
+                    cudaStream_t st) {
+  if (n < 1) return set_error(ST_INVALID_ARG, "fp8_cast: n must be >= 1");
+  if (fmt != 0 && fmt != 1) return set_error(ST_INVALID_ARG, "fp8_cast: format must be 0 (e4m3) or 1 (e5m2)");
+  if (!x || !out || !amax || !inv_scale) return set_error(ST_INVALID_ARG, "fp8_cast: null pointer");
   if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(out) & 7))
-    return set_error(ST_INVALID_ARG, "fp8_quantize: x must be 16-byte and out 8-byte aligned");
+    return set_error(ST_INVALID_ARG, "fp8_cast: x must be 16-byte and out 8-byte aligned");
   long long g = ((n + 7) / 8 + 255) / 256;
   int grid = (int)(g < num_sms() * 8 ? g : num_sms() * 8);
-  {
-    Prof prof(PK_MISC, 0, (double)n * (x_fp32 ? 4 : 2), st);
-    if (x_fp32) amax_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), n, reinterpret_cast<unsigned int*>(amax));
-    else amax_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n, reinterpret_cast<unsigned int*>(amax));
-    GPTK_CUDA(cudaGetLastError());
-  }
   Prof prof(PK_MISC, 0, (double)n * ((x_fp32 ? 4 : 2) + 1), st);
   uint8_t* o = static_cast<uint8_t*>(out);
   if (x_fp32) {
@@ -115,6 +110,25 @@ int launch_fp8_quantize(const void* x, int x_fp32, long long n, int fmt, void* o
   }
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
+}
+
+int launch_fp8_quantize(const void* x, int x_fp32, long long n, int fmt, void* out, float* amax, float* inv_scale,
+                        cudaStream_t st) {
+  if (n < 1) return set_error(ST_INVALID_ARG, "fp8_quantize: n must be >= 1");
+  if (fmt != 0 && fmt != 1) return set_error(ST_INVALID_ARG, "fp8_quantize: format must be 0 (e4m3) or 1 (e5m2)");
+  if (!x || !out || !amax || !inv_scale) return set_error(ST_INVALID_ARG, "fp8_quantize: null pointer");
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(out) & 7))
+    return set_error(ST_INVALID_ARG, "fp8_quantize: x must be 16-byte and out 8-byte aligned");
+  GPTK_CUDA(cudaMemsetAsync(amax, 0, sizeof(float), st));
+  long long g = ((n + 7) / 8 + 255) / 256;
+  int grid = (int)(g < num_sms() * 8 ? g : num_sms() * 8);
+  {
+    Prof prof(PK_MISC, 0, (double)n * (x_fp32 ? 4 : 2), st);
+    if (x_fp32) amax_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), n, reinterpret_cast<unsigned int*>(amax));
+    else amax_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), n, reinterpret_cast<unsigned int*>(amax));
+    GPTK_CUDA(cudaGetLastError());
+  }
+  return launch_fp8_cast(x, x_fp32, n, fmt, out, amax, inv_scale, st);
 }
 
 }  // namespace gptk

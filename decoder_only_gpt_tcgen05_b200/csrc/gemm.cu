@@ -309,6 +309,8 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
     if (epi == EPI_ACTBWD) GPTK_TRY(make_tmap_2d(&maps.r, p.aux, p.N, p.M, p.ld_aux, 64, 32, 2));
     p.tma_out = 1;
   }
+  if (p.amax_h != nullptr && (epi != EPI_UP || !p.tma_out))
+    return set_error(ST_UNSUPPORTED, "GEMM: max |h| is folded only by the MLP-up epilogue's TMA path");
   p.a_mn = A.mn_major;
   p.b_mn = B.mn_major;
   p.tiles_m = (p.M + tile_m - 1) / tile_m;

@@ -107,6 +107,9 @@ struct GemmParams {
   int f8_fmt_a, f8_fmt_b;
   const float* f8_inv_a;
   const float* f8_inv_b;
+  // EPI_UP: when set, max |h| over the stored (bf16) h is folded into *amax_h (a float bit
+  // pattern; the caller zeroes it first) for an 8-bit cast of h that then needs no pass of its own
+  unsigned int* amax_h;
 };
 
 constexpr int kMaxProblems = 8;
@@ -564,6 +567,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
     constexpr bool HAS_IN = (EPI == EPI_RESID || EPI == EPI_ACTBWD);
     constexpr int HALF = BN * 4 / C::EPI_WARPS;  // columns per epilogue warp
     const float f8_scale = F8 ? __ldg(p.f8_inv_a) * __ldg(p.f8_inv_b) : 1.f;
+    float amax_h = 0.f;  // EPI_UP: max |h| of this thread's outputs over all its tiles
     for (int tile = tile0; tile < num_tiles; tile += tile_step) {
       const TileInfo ti = tile_info(p, tile);
       const int tm = ti.tm, tn = ti.tn;
@@ -769,6 +773,11 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
 #pragma unroll
               for (int j = 0; j < CW; ++j) v[j] = act_fwd(v[j], 0);
             }
+            if (p.amax_h != nullptr && row_ok) {
+#pragma unroll
+              for (int j = 0; j < CW; ++j)
+                if (col0 + j < pN) amax_h = fmaxf(amax_h, fabsf(v[j]));
+            }
             stage_bf16(buf, lane, v);
           } else if (F32OUT) {
             stage_f32(buf, lane, v);
@@ -810,6 +819,12 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
       if (!ok) break;
     }
     if (lane == 0) bulk_wait_all();
+    if (EPI == EPI_UP && p.amax_h != nullptr) {
+      // one atomic per epilogue warp; h is stored in bf16 and the rounding is monotonic
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax_h = fmaxf(amax_h, __shfl_xor_sync(0xffffffffu, amax_h, o));
+      if (lane == 0) atomicMax(p.amax_h, __float_as_uint(__bfloat162float(__float2bfloat16_rn(amax_h))));
+    }
   }
 
   __syncthreads();

@@ -114,13 +114,32 @@ int launch_embed_fwd(const int* idx, const float* wte, const float* wpe, float* 
 // ------------------------------------------------------------------ norms
 // One warp per row.  A row of D <= 128*NV floats lives in registers (NV float4 per lane).
 
+// max over the block of each thread's am, rounded to bf16 (the values were stored as bf16, and the
+// rounding is monotonic), into *amax_bits as a float bit pattern (non-negative floats order like
+// their bits, so atomicMax is exact and order-independent)
+__device__ __forceinline__ void block_amax(float am, unsigned int* amax_bits) {
+  __shared__ float red[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = am;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.f;
+    for (int i = 0; i < nw; ++i) m = fmaxf(m, red[i]);
+    atomicMax(amax_bits, __float_as_uint(__bfloat162float(__float2bfloat16_rn(m))));
+  }
+}
+
 template <int NV, bool LN>
 __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const float* __restrict__ g,
                                 const float* __restrict__ b, float eps, __nv_bfloat16* __restrict__ y,
-                                long long ldy, float* __restrict__ mean_out, float* __restrict__ rstd_out) {
+                                long long ldy, float* __restrict__ mean_out, float* __restrict__ rstd_out,
+                                unsigned int* __restrict__ amax_bits) {
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int D4 = D / 4;
+  float am = 0.f;  // max |y| of this thread's elements (for an 8-bit cast of y)
   for (int m = blockIdx.x * warps + (threadIdx.x >> 5); m < M; m += gridDim.x * warps) {
     const float4* xr = reinterpret_cast<const float4*>(x + (long long)m * D);
     float4 v[NV];
@@ -162,9 +181,11 @@ __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const
           }
         }
         yr[c] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+        am = fmaxf(am, fmaxf(fmaxf(fabsf(o.x), fabsf(o.y)), fmaxf(fabsf(o.z), fabsf(o.w))));
       }
     }
   }
+  if (amax_bits) block_amax(am, amax_bits);
 }
 
 template <int NV, bool LN>
@@ -271,16 +292,17 @@ static int norm_dispatch(int D, F&& f) {
 }
 
 int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b, int ln, float eps,
-                    __nv_bfloat16* y, long long ldy, float* mean, float* rstd, cudaStream_t st) {
+                    __nv_bfloat16* y, long long ldy, float* mean, float* rstd, cudaStream_t st, float* amax) {
   return norm_dispatch(D, [&](auto nv) {
     constexpr int NV = decltype(nv)::value;
     int grid = cdiv(M, 8);
     if (grid > num_sms() * 16) grid = num_sms() * 16;
     Prof prof(PK_NORM_FWD, 0, (double)M * D * 6 + M * 8.0, st);
+    unsigned int* ab = reinterpret_cast<unsigned int*>(amax);
     if (ln)
-      norm_fwd_kernel<NV, true><<<grid, 256, 0, st>>>(x, M, D, g, b, eps, y, ldy, mean, rstd);
+      norm_fwd_kernel<NV, true><<<grid, 256, 0, st>>>(x, M, D, g, b, eps, y, ldy, mean, rstd, ab);
     else
-      norm_fwd_kernel<NV, false><<<grid, 256, 0, st>>>(x, M, D, g, b, eps, y, ldy, mean, rstd);
+      norm_fwd_kernel<NV, false><<<grid, 256, 0, st>>>(x, M, D, g, b, eps, y, ldy, mean, rstd, ab);
     GPTK_CUDA(cudaGetLastError());
     return (int)ST_OK;
   });

@@ -24,8 +24,11 @@ int launch_rope_table(float2* cs, int T, int half, double base, cudaStream_t st)
 int launch_embed_fwd(const int* idx, const float* wte, const float* wpe, float* x, int M, int T, int D, int V,
                      cudaStream_t st);
 // y = norm(x) as bf16 [M, ldy]; saves mean (LayerNorm only) and rstd per row
+// amax (optional): max |y| over the output, as a float, atomically folded into *amax (which the
+// caller zeroes first), for an 8-bit cast of y that then needs no pass of its own
 int launch_norm_fwd(const float* x, int M, int D, const float* g, const float* b, int ln, float eps,
-                    __nv_bfloat16* y, long long ldy, float* mean, float* rstd, cudaStream_t st);
+                    __nv_bfloat16* y, long long ldy, float* mean, float* rstd, cudaStream_t st,
+                    float* amax = nullptr);
 // dres (+)= norm'(x)^T dy ; also writes a bf16 copy of the result; LayerNorm gain/bias
 // gradients go to per-block partials (dg_part, db_part: [nblk][D]) for launch_colreduce
 int launch_norm_bwd(const float* dy, const float* x, const float* mean, const float* rstd, const float* g, int ln,
@@ -96,6 +99,9 @@ int launch_muon(float* params, const float* grads, float* mom, const std::vector
 // ---- 8-bit casts (fp8.cu): amax = max |x|, s = FP8_MAX / amax, out = cast(x s), inv_scale = 1 / s
 int launch_fp8_quantize(const void* x, int x_fp32, long long n, int fmt, void* out, float* amax, float* inv_scale,
                         cudaStream_t st);
+// the cast alone, with *amax already computed (max |x| as a float, e.g. by the producer of x)
+int launch_fp8_cast(const void* x, int x_fp32, long long n, int fmt, void* out, const float* amax, float* inv_scale,
+                    cudaStream_t st);
 
 // ---- attention (attention.cu)
 struct AttnShape {
@@ -105,8 +111,9 @@ struct AttnShape {
 };
 // (query, key) pairs a causal attention of T tokens with left window win (-1: none) scores
 double attn_pairs(int T, int win);
+// amax (optional): max |o| folded into *amax as for launch_norm_fwd
 int launch_attn_fwd(const __nv_bfloat16* qkv_pad, const AttnShape& s, __nv_bfloat16* o, long long ldo, float* lse,
-                    cudaStream_t st);
+                    cudaStream_t st, float* amax = nullptr);
 int launch_attn_bwd(const __nv_bfloat16* qkv_pad, const __nv_bfloat16* do_pad, const float* lse,
                     const float* delta, const AttnShape& s, __nv_bfloat16* dqkv_pad, cudaStream_t st);
 

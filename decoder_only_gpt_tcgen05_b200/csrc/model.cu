@@ -230,7 +230,7 @@ static Plan make_plan(const gpt_config& c, int B, int T, long long P) {
   if (c.fp8) {
     p.f8w = take((size_t)L * 12 * D * D);               // w_qkv, w_o, w_up, w_down of every layer
     p.f8a = take(M * (F > D ? F : D));
-    p.f8s = take((size_t)(4 * L + 4) * 2 * 4);
+    p.f8s = take((size_t)(8 * L) * 2 * 4);                // (amax, 1/scale): 4L weights, 4L activations
   } else {
     p.f8w = p.f8a = p.f8s = 0;
   }
@@ -314,7 +314,9 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
   if (c.pos == 1) GPTK_TRY(launch_rope_table(cs, T, hd / 2, (double)c.rope_base, st));
 
   // 8-bit forward projections: every block weight cast once per forward, each with its own scale;
-  // the activation operand of each projection is cast just before its product
+  // the activation operand of each projection is cast just before its product, from the max |x|
+  // that its producer (the norm, the attention output, the MLP-up epilogue) folded into the
+  // activation's slot (slots 4L + 4l + k, zeroed once per forward)
   uint8_t* f8w = c.fp8 ? at<uint8_t>(ws, pl.f8w) : nullptr;
   uint8_t* f8a = c.fp8 ? at<uint8_t>(ws, pl.f8a) : nullptr;
   float* f8s = c.fp8 ? at<float>(ws, pl.f8s) : nullptr;  // [slot][amax, 1/scale]
@@ -323,7 +325,16 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
     const size_t off[4] = {0, 3 * DD, 4 * DD, 8 * DD};
     return f8w + (size_t)l * 12 * DD + off[which];
   };
+  // GPT_FP8_AMAX_PASS=1 (tests): the activations' max |x| from a pass of its own instead of their
+  // producers, which must give the same scales bit for bit
+  static const bool amax_pass = [] {
+    const char* e = std::getenv("GPT_FP8_AMAX_PASS");
+    return e != nullptr && std::atoi(e) == 1;
+  }();
+  auto act_slot = [&](int l, int k) -> float* { return c.fp8 ? f8s + 2 * (4 * pl.L + 4 * l + k) : nullptr; };
+  auto fold_slot = [&](int l, int k) -> float* { return amax_pass ? nullptr : act_slot(l, k); };
   if (c.fp8) {
+    GPTK_CUDA(cudaMemsetAsync(f8s + 2 * 4 * pl.L, 0, (size_t)4 * pl.L * 2 * sizeof(float), st));
     for (int l = 0; l < pl.L; ++l) {
       const LayerOff& o = Lo.layer[l];
       const long long offs[4] = {o.w_qkv, o.w_o, o.w_up, o.w_down};
@@ -333,10 +344,12 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
                                      f8s + 2 * (4 * l + w), f8s + 2 * (4 * l + w) + 1, st));
     }
   }
-  // the 8-bit operands of one projection: the activation act [M, K] cast into f8a (slot 4L + k)
+  // the 8-bit operands of one projection: the activation act [M, K] cast into f8a with the scale
+  // from its slot's max |act|
   auto f8_setup = [&](GemmParams& p, const __nv_bfloat16* act, long long n, int l, int which, int k) -> int {
-    float* sa = f8s + 2 * (4 * pl.L + k);
-    GPTK_TRY(launch_fp8_quantize(act, 0, n, 0, f8a, sa, sa + 1, st));
+    float* sa = act_slot(l, k);
+    if (amax_pass) GPTK_TRY(launch_fp8_quantize(act, 0, n, 0, f8a, sa, sa + 1, st));
+    else GPTK_TRY(launch_fp8_cast(act, 0, n, 0, f8a, sa, sa + 1, st));
     p.f8_fmt_a = p.f8_fmt_b = 0;
     p.f8_inv_a = sa + 1;
     p.f8_inv_b = f8s + 2 * (4 * l + which) + 1;
@@ -366,7 +379,7 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
 
     // attention sublayer
     GPTK_TRY(launch_norm_fwd(x_in, M, D, ln ? params + o.ln1_g : nullptr, o.ln1_b >= 0 ? params + o.ln1_b : nullptr, ln,
-                             c.norm_eps, a1, D, st1, st1 + M, st));
+                             c.norm_eps, a1, D, st1, st1 + M, st, fold_slot(l, 0)));
     {
       // q|k|v = a1 W_qkv^T (+ b): straight into the attention layout when it is unpadded.
       // With 128-wide heads and no bias, RoPE and QK-norm run in the GEMM epilogue on the fp32
@@ -404,7 +417,7 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
       }
     }
     AttnShape as{B, T, H, hd, hdp, 3LL * H * hdp, layer_window(c, l)};
-    GPTK_TRY(launch_attn_fwd(qkv, as, ob, D, lse, st));
+    GPTK_TRY(launch_attn_fwd(qkv, as, ob, D, lse, st, fold_slot(l, 1)));
     {
       GemmParams p = gp(M, D, D);
       p.out = x_mid;
@@ -422,7 +435,7 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
     }
     // MLP sublayer
     GPTK_TRY(launch_norm_fwd(x_mid, M, D, ln ? params + o.ln2_g : nullptr, o.ln2_b >= 0 ? params + o.ln2_b : nullptr,
-                             ln, c.norm_eps, a2, D, st2, st2 + M, st));
+                             ln, c.norm_eps, a2, D, st2, st2 + M, st, fold_slot(l, 2)));
     {
       GemmParams p = gp(M, F, D);
       p.out = c.act == 1 ? nullptr : u;  // ReLU^2 keeps only h: the backward uses 2 relu(u) = 2 sqrt(h)
@@ -433,6 +446,7 @@ static int forward_impl(const gpt_config& c, const Layout& Lo, const Plan& pl, c
       p.prof_kind = PK_GEMM_UP;
       if (c.fp8) {
         GPTK_TRY(f8_setup(p, a2, (long long)MD, l, 2, 2));
+        p.amax_h = reinterpret_cast<unsigned int*>(fold_slot(l, 3));
         GPTK_TRY(gemm(EPI_UP, Operand{f8a, D, 0}, Operand{f8w_of(l, 2), D, 0}, p, st));
       } else {
         GPTK_TRY(gemm(EPI_UP, Operand{a2, D, 0}, Operand{wbf + o.w_up, D, 0}, p, st));

@@ -139,3 +139,46 @@ def test_model_with_fp8_projections_matches_fp8_oracle(name):
         cos = float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
         rel = float(np.linalg.norm(a - b) / np.linalg.norm(b))
         assert cos >= 0.995 and rel <= 0.1, (nm, cos, rel)
+
+
+_FOLD_SCRIPT = r"""
+import sys, hashlib, numpy as np, torch
+sys.path.insert(0, {root!r})
+import synth
+import decoder_only_gpt_tcgen05_b200 as g
+dev = torch.device("cuda:0")
+cfg = g.preset({base!r}, **{over!r})
+model = g.GPT(cfg, {B}, {T}, device=dev, seed=0)
+idx, tgt = synth.next_token_batch({B}, {T}, cfg.vocab_size, seed=1)
+loss = model.forward_loss(torch.from_numpy(idx).to(dev), torch.from_numpy(tgt).to(dev))
+ell, lse = model.token_losses()
+grads = model.backward()
+torch.cuda.synchronize()
+g.model.sync_status(dev)
+h = hashlib.sha256()
+for t in (loss.reshape(1), ell, lse, grads):
+    h.update(t.detach().float().cpu().numpy().tobytes())
+print("DIGEST", h.hexdigest())
+"""
+
+
+@pytest.mark.parametrize("name", list(MODEL_CASES))
+def test_fp8_scales_folded_into_producers_equal_a_separate_pass(name):
+    """The FP8 forward takes each activation's max |x| from its producer (the norm, the attention
+    output, the MLP-up epilogue) instead of a pass of its own.  Both are the exact maximum of the
+    same stored bf16 tensor, so the scales, the 8-bit codes and everything after them must agree
+    bit for bit: the loss, the per-token losses and logsumexps, and the gradients of a run with
+    GPT_FP8_AMAX_PASS=1 (a separate pass) against a default run."""
+    import os
+    import subprocess
+    import sys
+    base, over, B, T = MODEL_CASES[name]
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = _FOLD_SCRIPT.format(root=root, base=base, over=over, B=B, T=T)
+    digests = []
+    for env_val in ("0", "1"):
+        env = dict(os.environ, GPT_FP8_AMAX_PASS=env_val)
+        r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode == 0, r.stderr[-3000:]
+        digests.append([ln for ln in r.stdout.splitlines() if ln.startswith("DIGEST")][-1])
+    assert digests[0] == digests[1], digests
