@@ -75,7 +75,20 @@ __global__ void quantize_kernel(const T* __restrict__ x, long long n, const floa
   auto cvt = [](float lo, float hi) -> uint32_t { return FMT == 0 ? cvt_e4m3x2(lo, hi) : cvt_e5m2x2(lo, hi); };
   const long long n8 = n / 8;
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x, nth = (long long)gridDim.x * blockDim.x;
-  for (long long i = tid; i < n8; i += nth) {
+  long long i = tid;
+  for (; i + nth < n8; i += 2 * nth) {  // two vectors in flight per thread
+    float v[2][8];
+    load8<T>(x + 8 * i, v[0]);
+    load8<T>(x + 8 * (i + nth), v[1]);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      uint2 q;
+      q.x = cvt(v[u][0] * s, v[u][1] * s) | (cvt(v[u][2] * s, v[u][3] * s) << 16);
+      q.y = cvt(v[u][4] * s, v[u][5] * s) | (cvt(v[u][6] * s, v[u][7] * s) << 16);
+      reinterpret_cast<uint2*>(out)[i + u * nth] = q;
+    }
+  }
+  for (; i < n8; i += nth) {
     float v[8];
     load8<T>(x + 8 * i, v);
     uint2 q;
