@@ -13,11 +13,12 @@
 //
 // Launch sequence per chunk of same-shape matrices:
 //   muon_momentum_kernel   buf update and the Nesterov input's squared norm (fp64 partials)
-//   muon_prep_kernel       X = U / ||U|| in bf16, transposed through shared memory when needed
+//   muon_prep_*_kernel     X = U / ||U|| in bf16 (transposed through shared memory when rows > cols)
 //   ns_steps x { grouped GEMM A = X X^T (bf16),
 //                grouped GEMM M = c (A A) + b A (bf16; the linear combination in the epilogue),
 //                grouped GEMM X' = (M X) + a X (bf16, into the other X buffer) }
-//   muon_update_kernel     W -= lr scale X, transposed back through shared memory when needed
+//   muon_update_*_kernel   W -= lr scale X (transposed back through shared memory when rows > cols)
+#include <algorithm>
 #include <cmath>
 #include <string>
 #include <vector>
@@ -31,7 +32,7 @@ namespace gptk {
 
 namespace {
 
-constexpr int kParts = 64;              // fixed partition of each matrix's squared-norm sum
+constexpr int kParts = 256;             // fixed partition of each matrix's squared-norm sum
 constexpr int kChunk = kMaxProblems;    // matrices per grouped launch
 constexpr float kNsA = 3.4445f, kNsB = -4.7750f, kNsC = 2.0315f;
 
@@ -84,72 +85,138 @@ __global__ void __launch_bounds__(256) muon_momentum_kernel(const float* __restr
   }
 }
 
-// X[q] [m, n] bf16 = U / (||U||_F + 1e-7) with U [rows, cols] of matrix q; X = U^T when
-// rows > cols.  32 x 32 tiles through shared memory (blockIdx.x: tile, blockIdx.y: matrix).
-__global__ void __launch_bounds__(256) muon_prep_kernel(const float* __restrict__ g, const float* __restrict__ mom,
-                                                        MatList ml, int rows, int cols, float mu, int nesterov,
-                                                        const double* __restrict__ part,
-                                                        __nv_bfloat16* __restrict__ X) {
-  __shared__ float tile[32][33];
-  __shared__ float s_inv;
-  if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int k = 0; k < kParts; ++k) t += part[blockIdx.y * kParts + k];  // one fixed order
-    s_inv = (float)(1.0 / (sqrt(t) + 1e-7));
-  }
-  const long long base = ml.off[blockIdx.y];
-  const int tiles_c = (cols + 31) / 32;
-  const int r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32 per pass
+// 1 / (||U||_F + 1e-7) of matrix q from its kParts partial sums, added in one fixed order (lane k
+// sums parts 8 k .. 8 k + 7, then a fixed butterfly); called by a whole warp
+__device__ __forceinline__ float muon_inv_norm(const double* __restrict__ part, int q) {
+  static_assert(kParts == 256, "one warp, eight parts per lane");
+  const int lane = threadIdx.x & 31;
+  double t = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) t += part[q * kParts + 8 * lane + k];
+  t = warp_sum_dd(t);
+  return (float)(1.0 / (sqrt(t) + 1e-7));
+}
+
+// The Nesterov input (or buf) of four consecutive elements
+__device__ __forceinline__ float4 muon_u4(const float* __restrict__ g, const float* __restrict__ mom, long long i,
+                                          float mu, int nesterov) {
+  const float4 b = *reinterpret_cast<const float4*>(mom + i);
+  if (!nesterov) return b;
+  const float4 gv = *reinterpret_cast<const float4*>(g + i);
   const float omm = 1.f - mu;
+  return make_float4(fmaf(omm, gv.x, mu * b.x), fmaf(omm, gv.y, mu * b.y), fmaf(omm, gv.z, mu * b.z),
+                     fmaf(omm, gv.w, mu * b.w));
+}
+
+// X[q] = U / (||U||_F + 1e-7) in bf16 for rows <= cols (X has U's layout): four elements per
+// thread, blockIdx.y the matrix of the chunk
+__global__ void __launch_bounds__(256) muon_prep_flat_kernel(const float* __restrict__ g, const float* __restrict__ mom,
+                                                             MatList ml, long long n, float mu, int nesterov,
+                                                             const double* __restrict__ part,
+                                                             __nv_bfloat16* __restrict__ X) {
+  __shared__ float s_inv;
+  if (threadIdx.x < 32) {
+    const float v = muon_inv_norm(part, blockIdx.y);
+    if (threadIdx.x == 0) s_inv = v;
+  }
   __syncthreads();
   const float inv = s_inv;
-  const bool tr = rows > cols;
-  __nv_bfloat16* Xq = X + (long long)blockIdx.y * rows * cols;
-  for (int rr = ty; rr < 32; rr += 8) {
-    const int r = r0 + rr, c = c0 + tx;
-    float u = 0.f;
-    if (r < rows && c < cols) {
-      const long long i = base + (long long)r * cols + c;
-      const float b = mom[i];
-      u = nesterov ? fmaf(omm, g[i], mu * b) : b;
-    }
-    if (tr) tile[rr][tx] = u * inv;
-    else if (r < rows && c < cols) Xq[(long long)r * cols + c] = __float2bfloat16_rn(u * inv);
-  }
-  if (!tr) return;
-  __syncthreads();
-  // X[c][r] = U[r][c]: X is [cols, rows]
-  for (int cc = ty; cc < 32; cc += 8) {
-    const int c = c0 + cc, r = r0 + tx;
-    if (r < rows && c < cols) Xq[(long long)c * rows + r] = __float2bfloat16_rn(tile[tx][cc]);
+  const long long base = ml.off[blockIdx.y];
+  __nv_bfloat16* Xq = X + (long long)blockIdx.y * n;
+  for (long long i = 4LL * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 4LL * gridDim.x * blockDim.x) {
+    const float4 u = muon_u4(g, mom, base + i, mu, nesterov);
+    *reinterpret_cast<uint2*>(Xq + i) = make_uint2(pack_bf16x2(u.x * inv, u.y * inv), pack_bf16x2(u.z * inv, u.w * inv));
   }
 }
 
-// W[r][c] -= step * X'[r][c] with X' = X (rows <= cols) or X^T (X is [cols, rows]); tiles of 32 x 32
-__global__ void __launch_bounds__(256) muon_update_kernel(float* __restrict__ params, MatList ml, int rows, int cols,
-                                                          const __nv_bfloat16* __restrict__ X, float step) {
+// X[q] [cols, rows] = U^T / (||U||_F + 1e-7) in bf16 for rows > cols: 32 x 32 tiles through
+// shared memory (blockIdx.x: tile, blockIdx.y: matrix).  U is read as float4 along a row, X
+// written four rows at a time along a column; both shared-memory passes are free of bank
+// conflicts (row pitch 33).  Sides are multiples of 16, so a vector is in or out as a whole.
+__global__ void __launch_bounds__(256) muon_prep_tr_kernel(const float* __restrict__ g, const float* __restrict__ mom,
+                                                           MatList ml, int rows, int cols, float mu, int nesterov,
+                                                           const double* __restrict__ part,
+                                                           __nv_bfloat16* __restrict__ X) {
   __shared__ float tile[32][33];
+  __shared__ float s_inv;
+  if (threadIdx.x < 32) {
+    const float v = muon_inv_norm(part, blockIdx.y);
+    if (threadIdx.x == 0) s_inv = v;
+  }
   const long long base = ml.off[blockIdx.y];
   const int tiles_c = (cols + 31) / 32;
   const int r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  const __nv_bfloat16* Xq = X + (long long)blockIdx.y * rows * cols;
-  const bool tr = rows > cols;
-  if (tr) {
-    // read X[c][r] along r (contiguous), then update W[r][c] along c
-    for (int cc = ty; cc < 32; cc += 8) {
-      const int c = c0 + cc, r = r0 + tx;
-      tile[tx][cc] = (r < rows && c < cols) ? __bfloat162float(Xq[(long long)c * rows + r]) : 0.f;
-    }
-    __syncthreads();
+  __syncthreads();
+  const float inv = s_inv;
+  {
+    const int rr = threadIdx.x >> 3, cc = 4 * (threadIdx.x & 7);
+    const int r = r0 + rr, c = c0 + cc;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < rows && c < cols) u = muon_u4(g, mom, base + (long long)r * cols + c, mu, nesterov);
+    tile[rr][cc] = u.x * inv;
+    tile[rr][cc + 1] = u.y * inv;
+    tile[rr][cc + 2] = u.z * inv;
+    tile[rr][cc + 3] = u.w * inv;
   }
-  for (int rr = ty; rr < 32; rr += 8) {
-    const int r = r0 + rr, c = c0 + tx;
-    if (r < rows && c < cols) {
-      const float x = tr ? tile[rr][tx] : __bfloat162float(Xq[(long long)r * cols + c]);
-      params[base + (long long)r * cols + c] -= step * x;
-    }
+  __syncthreads();
+  const int oc = threadIdx.x >> 3, orr = 4 * (threadIdx.x & 7);  // X row (a column of U), four rows of U
+  const int c = c0 + oc, r = r0 + orr;
+  if (c < cols && r < rows) {
+    __nv_bfloat16* Xq = X + (long long)blockIdx.y * rows * cols;
+    *reinterpret_cast<uint2*>(Xq + (long long)c * rows + r) =
+        make_uint2(pack_bf16x2(tile[orr][oc], tile[orr + 1][oc]), pack_bf16x2(tile[orr + 2][oc], tile[orr + 3][oc]));
+  }
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// W -= step * X for rows <= cols (X has W's layout): four elements per thread
+__global__ void __launch_bounds__(256) muon_update_flat_kernel(float* __restrict__ params, MatList ml, long long n,
+                                                               const __nv_bfloat16* __restrict__ X, float step) {
+  const long long base = ml.off[blockIdx.y];
+  const __nv_bfloat16* Xq = X + (long long)blockIdx.y * n;
+  for (long long i = 4LL * (blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 4LL * gridDim.x * blockDim.x) {
+    const uint2 xv = *reinterpret_cast<const uint2*>(Xq + i);
+    float4 w = *reinterpret_cast<const float4*>(params + base + i);
+    w.x -= step * bf16lo(xv.x);
+    w.y -= step * bf16hi(xv.x);
+    w.z -= step * bf16lo(xv.y);
+    w.w -= step * bf16hi(xv.y);
+    *reinterpret_cast<float4*>(params + base + i) = w;
+  }
+}
+
+// W[r][c] -= step * X[c][r] for rows > cols (X is [cols, rows]): 32 x 32 tiles through shared
+// memory, X read four rows at a time along its rows, W updated as float4 along its rows
+__global__ void __launch_bounds__(256) muon_update_tr_kernel(float* __restrict__ params, MatList ml, int rows, int cols,
+                                                             const __nv_bfloat16* __restrict__ X, float step) {
+  __shared__ float tile[32][33];  // tile[c][r]
+  const long long base = ml.off[blockIdx.y];
+  const int tiles_c = (cols + 31) / 32;
+  const int r0 = (blockIdx.x / tiles_c) * 32, c0 = (blockIdx.x % tiles_c) * 32;
+  const __nv_bfloat16* Xq = X + (long long)blockIdx.y * rows * cols;
+  {
+    const int oc = threadIdx.x >> 3, orr = 4 * (threadIdx.x & 7);
+    const int c = c0 + oc, r = r0 + orr;
+    uint2 xv = make_uint2(0u, 0u);
+    if (c < cols && r < rows) xv = *reinterpret_cast<const uint2*>(Xq + (long long)c * rows + r);
+    tile[oc][orr] = bf16lo(xv.x);
+    tile[oc][orr + 1] = bf16hi(xv.x);
+    tile[oc][orr + 2] = bf16lo(xv.y);
+    tile[oc][orr + 3] = bf16hi(xv.y);
+  }
+  __syncthreads();
+  const int rr = threadIdx.x >> 3, cc = 4 * (threadIdx.x & 7);
+  const int r = r0 + rr, c = c0 + cc;
+  if (r < rows && c < cols) {
+    float4* wp = reinterpret_cast<float4*>(params + base + (long long)r * cols + c);
+    float4 w = *wp;
+    w.x -= step * tile[cc][rr];
+    w.y -= step * tile[cc + 1][rr];
+    w.z -= step * tile[cc + 2][rr];
+    w.w -= step * tile[cc + 3][rr];
+    *wp = w;
   }
 }
 
@@ -209,9 +276,13 @@ int muon_chunk(float* params, const float* grads, float* mom, const MuonGroup& g
     GPTK_CUDA(cudaGetLastError());
   }
   const int tiles = ((rows + 31) / 32) * ((cols + 31) / 32);
+  const unsigned flat_blocks = (unsigned)std::min<long long>((elems + 1023) / 1024, 2048);
   {
     Prof prof(PK_OPTIM, 0, (double)nq * elems * 10, st);
-    muon_prep_kernel<<<dim3(tiles, nq), 256, 0, st>>>(grads, mom, ml, rows, cols, h.momentum, nest, part, X);
+    if (rows > cols)
+      muon_prep_tr_kernel<<<dim3(tiles, nq), 256, 0, st>>>(grads, mom, ml, rows, cols, h.momentum, nest, part, X);
+    else
+      muon_prep_flat_kernel<<<dim3(flat_blocks, nq), 256, 0, st>>>(grads, mom, ml, elems, h.momentum, nest, part, X);
     GPTK_CUDA(cudaGetLastError());
   }
   int rows_of[kChunk];  // first row of matrix q in the stacked A and X buffers
@@ -236,7 +307,10 @@ int muon_chunk(float* params, const float* grads, float* mom, const MuonGroup& g
   const float step = (float)(h.lr * std::sqrt(rows > cols ? (double)rows / cols : 1.0));
   {
     Prof prof(PK_OPTIM, 0, (double)nq * elems * 10, st);
-    muon_update_kernel<<<dim3(tiles, nq), 256, 0, st>>>(params, ml, rows, cols, X, step);
+    if (rows > cols)
+      muon_update_tr_kernel<<<dim3(tiles, nq), 256, 0, st>>>(params, ml, rows, cols, X, step);
+    else
+      muon_update_flat_kernel<<<dim3(flat_blocks, nq), 256, 0, st>>>(params, ml, elems, X, step);
     GPTK_CUDA(cudaGetLastError());
   }
   return ST_OK;
