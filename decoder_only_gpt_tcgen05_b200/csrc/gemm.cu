@@ -1,5 +1,6 @@
 // Host launcher of the tcgen05 GEMM family and the tensor-map / status helpers.
 #include <cstdlib>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -153,7 +154,7 @@ static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t
     if (EPI == EPI_UP) out_bytes = M * N * (p.out ? 4 : 2);
     if (EPI == EPI_ACTBWD) out_bytes = M * N * 4;
     if (EPI == EPI_CE_FWD) out_bytes = M * p.tiles_n * 8;
-    flops += 2.0 * M * N * K;
+    flops += 2.0 * (p.pelems[q] > 0 ? p.pelems[q] : M * N) * K;
     bytes += (M * K + N * K) * (F8 ? 1 : 2) + out_bytes;
   }
   Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, flops, bytes, st);
@@ -324,6 +325,8 @@ int run_gemm(int epi, int bn, const Operand& A, const Operand& B, GemmParams& p,
   p.ptiles_m[0] = p.tiles_m;
   p.ptiles_n[0] = p.tiles_n;
   p.pgroup_m[0] = p.group_m;
+  p.tile_rows = tile_m;
+  p.tile_cols = bn;
   p.ctl = device_ctl();
   if (p.ctl.status == nullptr) return set_error(ST_CUDA, "device status word unavailable");
   return dispatch(epi, bn, pair, maps, p, st);
@@ -386,8 +389,25 @@ static int run_gemm_group_impl(int n, const GroupProblem* probs, int K, int a_mn
     p.ptiles_n[q] = (g.N + bn - 1) / bn;
     p.pgroup_m[q] = band_height(p.ptiles_m[q], K, tile_m);
     p.tile_start[q] = start;
-    start += p.ptiles_m[q] * p.ptiles_n[q];
+    if (g.upper) {
+      if (g.M != g.N) return set_error(ST_INVALID_ARG, "grouped GEMM: an upper-triangle product must be square");
+      // m-tile tm meets the upper triangle from n-tile tm * tile_m / bn on (tile_info's walk)
+      p.ptri[q] = 1;
+      double elems = 0;
+      for (int tm = 0; tm < p.ptiles_m[q]; ++tm) {
+        const int rows = std::min(tile_m, g.M - tm * tile_m);
+        for (int tn = tm * tile_m / bn; tn < p.ptiles_n[q]; ++tn) {
+          elems += (double)rows * std::min(bn, g.N - tn * bn);
+          ++start;
+        }
+      }
+      p.pelems[q] = elems;
+    } else {
+      start += p.ptiles_m[q] * p.ptiles_n[q];
+    }
   }
+  p.tile_rows = tile_m;
+  p.tile_cols = bn;
   p.tile_start[n] = start;
   if (epi == EPI_ACTBWD) {  // the linear epilogue's addend: one stacked bf16 matrix, a row block per problem
     if (!aligned16(c, ldc, 2)) return set_error(ST_INVALID_ARG, "grouped GEMM: addend alignment");

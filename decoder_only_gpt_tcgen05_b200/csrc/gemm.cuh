@@ -31,7 +31,8 @@
 //
 // Variants: LONGK (reductions over all tokens, the weight gradients) has four epilogue warps and a
 // deeper ring; a grouped launch runs up to eight products with the same K and operand layouts
-// from one problem table (tile_start / pM / pN ...), their tiles in one persistent schedule; F8
+// from one problem table (tile_start / pM / pN ...), their tiles in one persistent schedule (a
+// symmetric product, ptri, takes only the tiles that meet its upper triangle); F8
 // takes 8-bit operands (kind::f8f6f4, 128 K elements per stage) and scales every accumulator by
 // the operands' inverse scales.
 //
@@ -102,6 +103,9 @@ struct GemmParams {
   int tile_start[9];
   int pM[8], pN[8], ptiles_m[8], ptiles_n[8], pgroup_m[8];
   int pK[8];                  // host only: K extent of each problem (0 = K), for the FLOP count
+  int ptri[8];                // 1: problem q computes only the tiles meeting its upper triangle
+  int tile_rows, tile_cols;   // the launch's output tile (rows: 256 for CTA pairs, else 128)
+  double pelems[8];           // host only: output elements problem q computes (0 = M N)
   // 8-bit operands (the F8 kernels): formats (0 = e4m3, 1 = e5m2) and the inverse scales that
   // multiply every accumulator (device scalars: the product is (a s_a)(b s_b)^T / (s_a s_b))
   int f8_fmt_a, f8_fmt_b;
@@ -299,6 +303,20 @@ __device__ __forceinline__ TileInfo tile_info(const GemmParams& p, int tile) {
   t.M = p.pM[q];
   t.N = p.pN[q];
   const int local = tile - p.tile_start[q];
+  if (p.ptri[q]) {
+    // upper-triangle problems: m-tile tm takes the n-tiles from the one holding column
+    // tm * tile_rows (its first row) on, in row order
+    int tm = 0, rest = local;
+    for (;;) {
+      const int cnt = p.ptiles_n[q] - tm * p.tile_rows / p.tile_cols;
+      if (rest < cnt || tm + 1 >= p.ptiles_m[q]) break;
+      rest -= cnt;
+      ++tm;
+    }
+    t.tm = tm;
+    t.tn = tm * p.tile_rows / p.tile_cols + rest;
+    return t;
+  }
   const int per_band = p.pgroup_m[q] * p.ptiles_n[q];
   const int band = local / per_band;
   const int first = band * p.pgroup_m[q];

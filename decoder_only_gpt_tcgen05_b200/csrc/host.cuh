@@ -102,6 +102,9 @@ struct GroupProblem {
   void* out;
   long long ldo;
   int K_ext;
+  // 1: the product is symmetric (M == N, e.g. X X^T); only the tiles that meet the upper
+  // triangle (row <= column) are computed, the rest of out is left as it is
+  int upper;
 };
 // Up to 8 products with the same K and operand layouts in one persistent launch (their tiles
 // share one schedule, so small products do not leave SMs idle): fp32 outputs accumulated

@@ -14,8 +14,9 @@
 // Launch sequence per chunk of same-shape matrices:
 //   muon_momentum_kernel   buf update and the Nesterov input's squared norm (fp64 partials)
 //   muon_prep_*_kernel     X = U / ||U|| in bf16 (transposed through shared memory when rows > cols)
-//   ns_steps x { grouped GEMM A = X X^T (bf16),
-//                grouped GEMM M = c (A A) + b A (bf16; the linear combination in the epilogue),
+//   ns_steps x { grouped GEMM A = X X^T (bf16; upper-triangle tiles only), muon_mirror_kernel,
+//                grouped GEMM M = c (A A) + b A (bf16; the linear combination in the epilogue;
+//                upper-triangle tiles only), muon_mirror_kernel,
 //                grouped GEMM X' = (M X) + a X (bf16, into the other X buffer) }
 //   muon_update_*_kernel   W -= lr scale X (transposed back through shared memory when rows > cols)
 #include <algorithm>
@@ -220,6 +221,62 @@ __global__ void __launch_bounds__(256) muon_update_tr_kernel(float* __restrict__
   }
 }
 
+// The strictly lower triangle of each symmetric m x m bf16 matrix of a stack of nq from its upper
+// triangle (the grouped products A = X X^T and A A compute only the tiles that meet the upper
+// one).  The blocks (bi, bj), bj <= bi, of 64 x 64 elements are dealt to the CTAs in turn; each goes
+// through shared memory as fp32 (row pitch 65), read and written as 16-byte vectors.
+constexpr int kMirrorCtas = 16;  // CTAs per SM at most (eight are resident: 16.6 KB of shared memory each)
+__global__ void __launch_bounds__(256) muon_mirror_kernel(__nv_bfloat16* __restrict__ A, int m, int nq) {
+  __shared__ float tile[64][65];
+  const int nb = (m + 63) / 64;
+  const int per = nb * (nb + 1) / 2;  // lower blocks of one matrix, the diagonal ones included
+  const int rr = threadIdx.x >> 3, cc = 8 * (threadIdx.x & 7);  // 32 rows x 64 columns per pass
+  for (int w = blockIdx.x; w < per * nq; w += gridDim.x) {
+    const int q = w / per;
+    int bi = 0, rest = w - q * per;
+    while (rest > bi) {  // block row bi holds bi + 1 blocks
+      rest -= bi + 1;
+      ++bi;
+    }
+    const int bj = rest;
+    __nv_bfloat16* Aq = A + (long long)q * m * m;
+    // the upper block (bj, bi): rows bj*64 + rr (+32), columns bi*64 + cc .. cc + 7
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = bj * 64 + rr + 32 * h, c = bi * 64 + cc;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < m && c < m) v = *reinterpret_cast<const uint4*>(Aq + (long long)r * m + c);
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        tile[rr + 32 * h][cc + 2 * k] = __uint_as_float(wv[k] << 16);
+        tile[rr + 32 * h][cc + 2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
+      }
+    }
+    __syncthreads();
+    // rows bi*64 + rr (+32), columns bj*64 + cc .. cc + 7 of the lower block: A[r][c] = A[c][r]
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int orow = rr + 32 * h;
+      const int r = bi * 64 + orow, c = bj * 64 + cc;
+      if (r < m && c < m) {
+        __nv_bfloat16* d = Aq + (long long)r * m + c;
+        if (bi > bj) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) wv[k] = pack_bf16x2(tile[cc + 2 * k][orow], tile[cc + 2 * k + 1][orow]);
+          *reinterpret_cast<uint4*>(d) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            if (c + k < r) d[k] = __float2bfloat16_rn(tile[cc + k][orow]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
 struct MuonGroup {
   int rows, cols;
   std::vector<long long> offs;
@@ -295,12 +352,26 @@ int muon_chunk(float* params, const float* grads, float* mom, const MuonGroup& g
       __nv_bfloat16* Xq = Xc + (size_t)q * m * n;
       __nv_bfloat16* Aq = A + (size_t)q * m * m;
       __nv_bfloat16* Mq = M + (size_t)q * m * m;
-      gA[q] = GroupProblem{Xq, n, Xq, n, m, m, Aq, m, 0};                   // A = X X^T
-      gM[q] = GroupProblem{Aq, m, Aq, m, m, m, Mq, m, 0};                   // A A (A is symmetric: A^T = A)
+      // A = X X^T and A A are symmetric: only their upper-triangle tiles are computed, and the
+      // lower triangle is copied from the upper one
+      gA[q] = GroupProblem{Xq, n, Xq, n, m, m, Aq, m, 0, 1};                   // A = X X^T
+      gM[q] = GroupProblem{Aq, m, Aq, m, m, m, Mq, m, 0, 1};                   // A A (A^T = A)
       gX[q] = GroupProblem{Mq, m, Xq, n, m, n, Xn + (size_t)q * m * n, n, 0};  // M X (X read MN-major)
     }
+    const int mirror_blocks = ((m + 63) / 64) * ((m + 63) / 64 + 1) / 2 * nq;
+    const int mirror_grid = std::min(mirror_blocks, num_sms() * kMirrorCtas);  // every block resident at once
     GPTK_TRY(run_gemm_group(nq, gA, n, 0, 0, 256, PK_GEMM_MUON, st, EPI_BF16, 0));
+    {
+      Prof prof(PK_OPTIM, 0, (double)nq * m * m * 2, st);
+      muon_mirror_kernel<<<mirror_grid, 256, 0, st>>>(A, m, nq);
+      GPTK_CUDA(cudaGetLastError());
+    }
     GPTK_TRY(run_gemm_group_axpby(nq, gM, m, 0, 0, PK_GEMM_MUON, A, m, (long long)nq * m, rows_of, kNsC, kNsB, st));
+    {
+      Prof prof(PK_OPTIM, 0, (double)nq * m * m * 2, st);
+      muon_mirror_kernel<<<mirror_grid, 256, 0, st>>>(M, m, nq);
+      GPTK_CUDA(cudaGetLastError());
+    }
     GPTK_TRY(run_gemm_group_axpby(nq, gX, m, 0, 1, PK_GEMM_MUON, Xc, n, (long long)nq * m, rows_of, 1.f, kNsA, st));
   }
   X = Xb[h.ns_steps & 1];
