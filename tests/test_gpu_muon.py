@@ -30,6 +30,9 @@ CASES = {
     "d20_small": ("d20", dict(n_layer=3, n_embd=256, n_head=2, vocab_size=2048, block_size=512)),
     # more same-shape matrices than one grouped launch takes (8 per chunk)
     "d20_deep": ("d20", dict(n_layer=10, n_embd=128, n_head=1, vocab_size=512, block_size=512)),
+    # 512-wide matrices: the symmetric products X X^T and A A skip the tiles below their diagonal
+    # (128 x 256 tiles: 6 of 8 computed) and the lower triangles are copied from the upper ones
+    "d20_wide": ("d20", dict(n_layer=1, n_embd=512, n_head=4, vocab_size=1024, block_size=256)),
 }
 
 
@@ -89,3 +92,17 @@ def test_muon_step_matches_oracle(name, nesterov):
         rp = p.copy()
         rm = mom.copy()
         rv = v.copy()
+
+
+def test_muon_upper_triangle_tiles_in_cta_pairs():
+    """The d20_wide case again with 256 x 256 CTA-pair tiles forced (GPT_GEMM_PAIR=1, read once per
+    process, hence a child process): 3 of the 4 tiles of each symmetric product are computed."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, GPT_GEMM_PAIR="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", "-m", "gpu",
+                        f"{__file__}::test_muon_step_matches_oracle[d20_wide-True]"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert "1 passed" in r.stdout, r.stdout[-2000:]
