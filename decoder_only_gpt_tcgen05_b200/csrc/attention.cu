@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_pairs = gridDim.y;
   const int pr = n_pairs - 1 - blockIdx.y;  // heaviest first
@@ -136,6 +137,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  pdl_wait();  // q, k, v (and dO, lse, delta) come from the kernels before this one
 
   const int colq = h * s.hdp;
   const int colk = s.H * s.hdp + h * s.hdp;
@@ -470,6 +472,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* stats = reinterpret_cast<float*>(sm + L::STATS);
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_kt = (s.T + 127) / 128;
   const int BH = s.B * s.H;
@@ -501,6 +504,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  pdl_wait();  // q, k, v (and dO, lse, delta) come from the kernels before this one
   const uint32_t tS = tbase;
   const uint32_t tdP = tbase + 128;
   const uint32_t tdV = tbase + 256;
@@ -831,6 +835,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_qt = (s.T + 127) / 128;
   const int BH = s.B * s.H;
@@ -868,6 +873,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  pdl_wait();  // q, k, v (and dO, lse, delta) come from the kernels before this one
   const uint32_t tS = tbase;
   const uint32_t tdP = tbase + 128;
   const uint32_t tdQ = tbase + 256;
@@ -1155,8 +1161,8 @@ static int attn_fwd_launch(const CUtensorMap& tm, const AttnShape& s, __nv_bfloa
   dim3 grid(s.B * s.H, (s.T + 255) / 256);
   const double causal = (double)s.B * s.H * attn_pairs(s.T, s.win);
   Prof prof(PK_ATTN_FWD, 4.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 4, st);
-  attn_fwd_kernel<HD><<<grid, kFwdThreads, L::BYTES, st>>>(tm, s, o, ldo, lse, scale_log2,
-                                                            reinterpret_cast<unsigned int*>(amax), device_ctl());
+  GPTK_CUDA(launch_pdl(attn_fwd_kernel<HD>, grid, dim3(kFwdThreads), L::BYTES, st, tm, s, o, ldo, lse, scale_log2,
+                       reinterpret_cast<unsigned int*>(amax), device_ctl()));
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;
 }
@@ -1199,8 +1205,8 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     const long long items = (long long)((s.T + 127) / 128) * s.B * s.H;
     dim3 grid((unsigned)std::min<long long>(items, num_sms()));
     Prof prof(PK_ATTN_BWD_DKV, 8.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 6, st);
-    attn_bwd_dkv_kernel<HD><<<grid, kBwdThreads, L::BYTES, st>>>(qkv128, qkv128, do128, s, lse, delta, dqkv, scale_log2,
-                                                                 scale, ctl);
+    GPTK_CUDA(launch_pdl(attn_bwd_dkv_kernel<HD>, grid, dim3(kBwdThreads), L::BYTES, st, qkv128, qkv128, do128, s, lse,
+                         delta, dqkv, scale_log2, scale, ctl));
     GPTK_CUDA(cudaGetLastError());
   }
   {
@@ -1210,8 +1216,8 @@ static int attn_bwd_t(const __nv_bfloat16* qkv, const __nv_bfloat16* dop, const 
     const long long items = (long long)((s.T + 127) / 128) * s.B * s.H;
     dim3 grid((unsigned)std::min<long long>(items, num_sms()));
     Prof prof(PK_ATTN_BWD_DQ, 6.0 * s.hd * causal, (double)s.B * s.T * s.H * s.hd * 2 * 5, st);
-    attn_bwd_dq_kernel<HD><<<grid, kBwdThreads, L::BYTES, st>>>(qkv128, do128, qkv128, s, lse, delta, dqkv, scale_log2,
-                                                                scale, ctl);
+    GPTK_CUDA(launch_pdl(attn_bwd_dq_kernel<HD>, grid, dim3(kBwdThreads), L::BYTES, st, qkv128, do128, qkv128, s, lse,
+                         delta, dqkv, scale_log2, scale, ctl));
     GPTK_CUDA(cudaGetLastError());
   }
   return ST_OK;

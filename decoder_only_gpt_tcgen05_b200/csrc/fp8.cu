@@ -68,6 +68,7 @@ __global__ void amax_kernel(const T* __restrict__ x, long long n, unsigned int* 
 template <typename T, int FMT>
 __global__ void quantize_kernel(const T* __restrict__ x, long long n, const float* __restrict__ amax,
                                 uint8_t* __restrict__ out, float* __restrict__ inv_scale) {
+  pdl_trigger();
   const float fmax = FMT == 0 ? kMaxE4m3 : kMaxE5m2;
   const float a = *amax;
   const float s = a > 0.f ? fmax / a : 1.f;

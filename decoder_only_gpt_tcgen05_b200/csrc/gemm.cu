@@ -160,20 +160,22 @@ static int launch_gemm_t(const GemmMaps& maps, const GemmParams& p, cudaStream_t
   Prof prof(p.prof_kind > 0 ? p.prof_kind : PK_GEMM, flops, bytes, st);
   if (PAIR) {
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(2 * grid, 1, 1);
     cfg.blockDim = dim3(C::THREADS, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     GPTK_CUDA(cudaLaunchKernelEx(&cfg, kern, maps, p));
   } else {
-    kern<<<grid, C::THREADS, C::SMEM, st>>>(maps, p);
+    GPTK_CUDA(launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, maps, p));
   }
   GPTK_CUDA(cudaGetLastError());
   return ST_OK;

@@ -351,6 +351,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::STAGES + 5 + 2 * C::EPI_WARPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   // CTA pairs: rank within the pair, and the pair's place in the persistent tile walk
@@ -391,6 +392,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, LONGK, PAIR>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the operands and epilogue inputs come from the kernels before this one
 
   const int num_tiles = p.tile_start[p.n_prob];
   const int num_k = (p.K + KE - 1) / KE;

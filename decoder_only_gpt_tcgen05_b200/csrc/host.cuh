@@ -7,6 +7,7 @@
 
 #include <cstdint>
 #include <string>
+#include <utility>
 
 #include "ptx.cuh"
 
@@ -117,5 +118,23 @@ int run_gemm_group(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, 
 // ldc); used where every product has its own addend of its own output's shape.
 int run_gemm_group_axpby(int n, const GroupProblem* probs, int K, int a_mn, int b_mn, int prof_kind, const void* c,
                          long long ldc, long long c_rows, const int* c_row, float alpha, float beta, cudaStream_t st);
+
+// Launch with programmatic stream serialization: the kernel may be scheduled while the previous
+// kernel on the stream finishes (it must run pdl_wait() before touching global memory).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace gptk

@@ -37,6 +37,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // ------------------------------------------------------------------ cast
 
 __global__ void cast_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst, long long n4) {
+  pdl_trigger();
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     float4 v = src[i];
     dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
@@ -136,6 +137,7 @@ __global__ void norm_fwd_kernel(const float* __restrict__ x, int M, int D, const
                                 const float* __restrict__ b, float eps, __nv_bfloat16* __restrict__ y,
                                 long long ldy, float* __restrict__ mean_out, float* __restrict__ rstd_out,
                                 unsigned int* __restrict__ amax_bits) {
+  pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int D4 = D / 4;
@@ -194,6 +196,7 @@ __global__ void norm_bwd_kernel(const float* __restrict__ dy, const float* __res
                                 const float* __restrict__ g, int M, int D, float* __restrict__ dres, int dres_init,
                                 __nv_bfloat16* __restrict__ dres_bf, float* __restrict__ dg_part,
                                 float* __restrict__ db_part) {
+  pdl_trigger();
   extern __shared__ float red[];  // [warps][2][D] (LayerNorm only)
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5;
@@ -325,6 +328,7 @@ template <int NV8, bool DYB>
 __global__ void rms_bwd_kernel(const void* __restrict__ dy_, const __nv_bfloat16* __restrict__ y,
                                const float* __restrict__ rstd, int M, int D, float* __restrict__ dres,
                                int dres_init, __nv_bfloat16* __restrict__ dres_bf) {
+  pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int w = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -661,6 +665,7 @@ template <int PPL>
 __global__ void qk_fwd_kernel(const __nv_bfloat16* __restrict__ src, const float2* __restrict__ cs, int M, int T,
                               int H, int hd, int hdp, int rope, int qk_norm, float eps, __nv_bfloat16* dst,
                               float* __restrict__ rq, float* __restrict__ rk, int in_place) {
+  pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int half = hd / 2;
@@ -708,6 +713,7 @@ __global__ void qk_bwd_kernel(const __nv_bfloat16* dpad, const __nv_bfloat16* __
                               const float* __restrict__ rq, const float* __restrict__ rk,
                               const float2* __restrict__ cs, int M, int T, int H, int hd, int hdp, int rope,
                               int qk_norm, __nv_bfloat16* dqkv) {
+  pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int half = hd / 2;
@@ -794,6 +800,7 @@ template <int HD>
 __global__ void qk_bwd_vec_kernel(__nv_bfloat16* __restrict__ dqkv, const __nv_bfloat16* __restrict__ qpad,
                                   const float* __restrict__ rq, const float* __restrict__ rk,
                                   const float2* __restrict__ cs, int M, int T, int H, int rope, int qk_norm) {
+  pdl_trigger();
   constexpr int HALF = HD / 2;
   constexpr int LPI = HD / 8;
   constexpr int IPW = 32 / LPI;
@@ -921,6 +928,7 @@ int launch_qk_bwd(const __nv_bfloat16* dqkv_pad, const __nv_bfloat16* qkv_pad, c
 template <int HD>
 __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dpad, int B,
                                   int T, int H, int hdp, float* __restrict__ delta) {
+  pdl_trigger();
   constexpr int LPI = HD / 32;  // lanes per item
   constexpr int IPW = 32 / LPI;
   const int warps = blockDim.x >> 5;
@@ -966,6 +974,7 @@ __global__ void attn_delta_kernel(const __nv_bfloat16* __restrict__ o, const __n
 // any even head dim: one warp per (token, head)
 __global__ void attn_delta_generic_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dpad,
                                           int B, int T, int H, int hd, int hdp, float* __restrict__ delta) {
+  pdl_trigger();
   const int warps = blockDim.x >> 5;
   const int lane = threadIdx.x & 31;
   const int total = B * T * H;
@@ -1049,6 +1058,7 @@ int launch_init_normal(float* params, long long off, long long n, unsigned long 
 
 __global__ void sum_parts_kernel(const float* __restrict__ parts, int n_parts, size_t stride, size_t n4,
                                  float* __restrict__ out) {
+  pdl_trigger();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
     float4 a = reinterpret_cast<const float4*>(parts)[i];
     for (int p = 1; p < n_parts; ++p) {

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(256) muon_prep_flat_kernel(const float* __rest
                                                              MatList ml, long long n, float mu, int nesterov,
                                                              const double* __restrict__ part,
                                                              __nv_bfloat16* __restrict__ X) {
+  pdl_trigger();
   __shared__ float s_inv;
   if (threadIdx.x < 32) {
     const float v = muon_inv_norm(part, blockIdx.y);
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(256) muon_prep_tr_kernel(const float* __restri
                                                            MatList ml, int rows, int cols, float mu, int nesterov,
                                                            const double* __restrict__ part,
                                                            __nv_bfloat16* __restrict__ X) {
+  pdl_trigger();
   __shared__ float tile[32][33];
   __shared__ float s_inv;
   if (threadIdx.x < 32) {
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(256) muon_update_tr_kernel(float* __restrict__
 // through shared memory as fp32 (row pitch 65), read and written as 16-byte vectors.
 constexpr int kMirrorCtas = 16;  // CTAs per SM at most (eight are resident: 16.6 KB of shared memory each)
 __global__ void __launch_bounds__(256) muon_mirror_kernel(__nv_bfloat16* __restrict__ A, int m, int nq) {
+  pdl_trigger();
   __shared__ float tile[64][65];
   const int nb = (m + 63) / 64;
   const int per = nb * (nb + 1) / 2;  // lower blocks of one matrix, the diagonal ones included

@@ -39,6 +39,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+//
+// A kernel launched with programmatic stream serialization (launch_pdl) may start while the
+// kernel before it on the stream is still finishing: its prologue (barrier set-up, TMEM
+// allocation, tensor-map prefetch) overlaps the other kernel's last CTAs.  pdl_wait() blocks until
+// that kernel has completed and its memory is visible; every thread runs it before its first
+// global load or store.  pdl_trigger() lets the next kernel be scheduled as soon as every CTA of
+// this one has started (it changes nothing for a kernel launched the usual way).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
