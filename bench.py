@@ -710,6 +710,8 @@ def main():
             print(f"{k:14s} {v['ms_per_step']:9.3f} ms  x{v['launches_per_step']:5d}  "
                   f"{(v['tflops'] or 0):8.1f} TF/s  {(v['gbs'] or 0):8.1f} GB/s", file=sys.stderr)
 
+    # fp32 weights and gradients, and the step's workspace (their bf16 copy, the saved activations)
+    working_set_gb = (model.params.numel() * 8 + model.ws_bytes) / 1e9
     line = {
         "metric": metric_name(preset_name), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -726,7 +728,8 @@ def main():
                    "grad_sync": (None if world == 1 else
                                  "bucketed on a second stream while the backward runs" if sync is not None
                                  else "one NCCL all-reduce after the backward"),
-                   "l2": "working set (~33 GB of weights, gradients and saved activations) far above the 126 MB L2; no flush"},
+                   "l2": f"working set ({working_set_gb:.1f} GB of weights, gradients and workspace) far above the "
+                         "126 MB L2; no flush"},
         "mfu": {"tflops_per_gpu": tflops, "vs_measured_sustained": tflops / peak_sus,
                 "vs_measured_burst": tflops / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]),
                 "vs_datasheet_2250": tflops / DATASHEET_BF16_TFLOPS,
