@@ -16,9 +16,9 @@
 //               so the tensor core works on one tile while the other tile's softmax runs
 //   warps 2, 3  idle (they give their registers to the softmax warpgroups with setmaxnreg)
 //   warps 4..11 two softmax warpgroups, one per query tile, one query row per thread holding its
-//               128 scores: row max and sum in registers, P = exp2(...) (3/8 of them on the FMA
-//               pipe) as bf16 over the first 64 score columns (already read), where it is the A
-//               operand of the PV product; O is rescaled in TMEM only when the running max grows
+//               128 scores: row max and sum in registers, P = exp2(...) (ex2.approx) as bf16
+//               over the first 64 score columns (already read), where it is the A operand of the
+//               PV product; O is rescaled in TMEM only when the running max grows
 //               by more than 2^8 (otherwise the stale max stays exact because O and l use the
 //               same one)
 // Backward: delta = rowsum(dO * O) (kernels.cu), then two persistent kernels (one CTA per SM,
@@ -69,10 +69,6 @@ constexpr int kFwdRegsProducer = 80;   // warpgroup 0 after setmaxnreg.dec
 constexpr int kFwdRegsSoftmax = 208;  // warpgroups 1, 2 after setmaxnreg.inc
 static_assert(128 * kFwdRegsProducer + 256 * kFwdRegsSoftmax <= kFwdThreads * kFwdRegs,
               "the register split must fit the registers the block is launched with");
-// 16-key groups of a block whose exponentials go to the FMA pipe (exp2_poly2), the others to
-// ex2.approx: 3 of 8, which balances the MUFU unit (8 cycles per warp instruction) against the
-// issue slots of the polynomial
-constexpr uint32_t kPolyGroups = 0x52u;
 
 template <int HD>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -326,8 +322,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       // P = exp2(s * scale - m) as bf16 over score columns [0, 64) (masked scores are -inf and
-      // give 0, or at most 2^-126 on the polynomial path); a row with no visible key yet
-      // (m = -inf) takes 0 as its offset: its scores are all -inf
+      // give 0); a row with no visible key yet (m = -inf) takes 0 as its offset: its scores are
+      // all -inf
       const float m_off = m == -INFINITY ? 0.f : m;
       const float2 sc2 = make_float2(scale_log2, scale_log2), nm2 = make_float2(-m_off, -m_off);
       float2 rs2[4];
@@ -340,7 +336,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int k = 0; k < 8; ++k) {
           const int e = 16 * g + 2 * k;
           const float2 x = ffma2(make_float2(sv[e], sv[e + 1]), sc2, nm2);
-          const float2 pv = ((kPolyGroups >> g) & 1u) ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          const float2 pv = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           rs2[k & 3] = fadd2(rs2[k & 3], pv);
           pw[k] = pack_bf16x2(pv.x, pv.y);
         }

@@ -148,10 +148,11 @@ GPT_API int gpt_op_lmhead_ce_fwd_noalloc(const void* x, const void* w, const int
  * usable.  Nothing faults, traps or hangs. */
 GPT_API int gpt_op_wait_probe(unsigned long long timeout_ns, void* stream);
 
-/* The two exponentials of the attention forward's softmax, for testing them
- * against their error bounds (no counterpart on the pages): out[i] = 2^x[i]
- * for the n (even) fp32 values at x, with poly = 0 the MUFU approximation
- * (ex2.approx.ftz) and poly = 1 the FMA-pipe polynomial (range reduction to
+/* The attention softmax's exponential and an FMA-pipe alternative to it, for
+ * testing them against their error bounds (no counterpart on the pages):
+ * out[i] = 2^x[i] for the n (even) fp32 values at x, with poly = 0 the MUFU
+ * approximation the attention kernels use (ex2.approx.ftz) and poly = 1 the
+ * FMA-pipe polynomial (range reduction to
  * [-1/2, 1/2], degree-4 minimax polynomial, relative error below 3e-6 for
  * -125 <= x <= 127; x below -125, -inf included, gives a value in
  * [0, 2^-125]).  x and out: device, 8-byte aligned, fp32.  Invalid n or
